@@ -1,0 +1,300 @@
+"""CPU fp64 oracle for the Mixtral top-2-of-8 sparse-MoE SwiGLU feed-forward layer.
+
+TEST INFRASTRUCTURE ONLY.  Nothing in the product path imports, calls or links this
+module; only ``tests/``, ``__graft_entry__.smoke()`` and the ``cpu_baseline`` /
+``--impl reference`` legs of ``bench.py`` may use it.  It shares no code, table or
+helper with the CUDA library; the two meet only through the seeded input generator.
+
+What it computes (sources, cited as page title + section/equation):
+
+* Router logits ``l = x . W_g`` over ``E`` experts, shape ``[T, E]``
+  -- crackai "Mixtral of Experts", section "Top-2 Routing in Detail" (gate_logits);
+  notion notes "Mixtral of Experts", section "Sparse gating", eq. G(x).
+* Gate ``G(x) = Softmax(TopK(x . W_g))`` where every logit outside the top k is set
+  to -inf before the softmax, so only k experts get non-zero weight
+  -- notion notes, "Sparse gating", eq. G(x) and the sentence under it.
+* The same weights written the other way round: softmax over all E, keep the top
+  two, divide by their sum -- ml-canon "52 Mixtral", section "PyTorch Mixtral's MoE
+  FFN (top-2 of 8)".  Both forms are computed here and must agree.
+* K = 2 and the expert function is SwiGLU -- notion notes, "Implementation";
+  atlas "Mixtral", "Design overview" (SwiGLU, inner dimension 14336).  The SwiGLU
+  form ``E_e(x) = W2[e] (silu(W1[e] x) * (W3[e] x))`` with ``silu(z) = z sigma(z)``
+  is the plain reading of "SwiGLU architecture" (gate branch W1, linear branch W3,
+  no biases: the pages show none).
+* Output ``y = sum_i G(x)_i E_i(x)`` -- notion notes, "Architectural details" and
+  "Implementation", eq. y; crackai, "Top-2 Routing in Detail"
+  (y = w_1 Expert_{i1}(x) + w_2 Expert_{i2}(x)).
+* Grouping tokens by expert and scattering results back -- ml-canon "52 Mixtral",
+  "Questions worth asking" (gather and scatter); notion notes, "Expert Parallelism"
+  (output returned to the original token location).
+
+Readings where the pages are silent (each is also listed in the design notes):
+
+* Ties in the top-2 choice go to the lower expert index; experts are ordered by
+  (logit descending, index ascending) and slot 0 holds the larger logit.
+* Selection is made on the fp64 logits (exact products of the bf16/fp32 inputs,
+  summed in fp64), never on rounded softmax values.
+* ``w1 = 1 / (1 + exp(l2 - l1))`` in fp64, rounded once to float32;
+  ``w2 = 1 - w1`` evaluated in float32 so that the pair sums to exactly 1.
+* No capacity limit and no token dropping: every token reaches exactly 2 experts.
+* The permutation is a stable counting sort by expert of the flattened
+  (token, slot) index ``f = t*k + j``: within one expert's group rows are in
+  ascending token order.
+* Inputs are taken as exact values (bf16/fp32 promoted to fp64); nothing is rounded
+  in between.
+
+Every public function here is pinned by tests in ``tests/test_oracle_pins.py``
+against closed forms, brute force on tiny inputs and the pages' printed numbers.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+__all__ = [
+    "router_logits",
+    "top2_select",
+    "gate_weights",
+    "gate_weights_f32",
+    "gate_dense_topk_softmax",
+    "gate_dense_softmax_topk_renorm",
+    "permutation",
+    "gather_rows",
+    "silu",
+    "expert_swiglu",
+    "expert_ffn_grouped",
+    "combine",
+    "moe_layer",
+    "moe_layer_dense",
+    "mixtral_param_counts",
+]
+
+
+def _f64(a) -> np.ndarray:
+    return np.asarray(a, dtype=np.float64)
+
+
+def router_logits(x, Wg) -> np.ndarray:
+    """``l[t, e] = sum_i x[t, i] * W_g[i, e]`` in fp64.
+
+    crackai "Mixtral of Experts", "Top-2 Routing in Detail": gate_logits = x . W_gate,
+    shape [tokens, 8]; notion notes, "Sparse gating", eq. G(x) (x . W_g).
+    """
+    return _f64(x) @ _f64(Wg)
+
+
+def top2_select(logits, k: int = 2) -> np.ndarray:
+    """Indices of the k largest logits per token, ordered (logit desc, index asc).
+
+    notion notes, "Sparse gating" (TopK keeps the top-k values); K = 2 per
+    "Implementation".  Ties are broken toward the lower expert index (reading: the
+    pages are silent).  A stable ascending sort of ``-logits`` yields exactly that
+    order.  Returns int32 ``[T, k]``.
+    """
+    l = _f64(logits)
+    order = np.argsort(-l, axis=1, kind="stable")
+    return order[:, :k].astype(np.int32)
+
+
+def gate_weights(logits, idx) -> np.ndarray:
+    """fp64 weights of the two kept experts: softmax restricted to the top two.
+
+    For k = 2 the restricted softmax is ``w1 = 1/(1 + exp(l2 - l1))`` and
+    ``w2 = 1/(1 + exp(l1 - l2))`` (the softmax of two numbers); notion notes,
+    "Sparse gating", eq. G(x).
+    """
+    l = _f64(logits)
+    l1 = np.take_along_axis(l, idx[:, :1].astype(np.int64), axis=1)[:, 0]
+    l2 = np.take_along_axis(l, idx[:, 1:2].astype(np.int64), axis=1)[:, 0]
+    w1 = 1.0 / (1.0 + np.exp(l2 - l1))
+    w2 = 1.0 / (1.0 + np.exp(l1 - l2))
+    return np.stack([w1, w2], axis=1)
+
+
+def gate_weights_f32(logits, idx) -> np.ndarray:
+    """The float32 weights as the layer stores them (reading of the silent rounding).
+
+    ``w1`` is the fp64 value rounded once to float32, and ``w2 = 1 - w1`` is
+    evaluated in float32 so that ``w1 + w2 == 1`` exactly in float32.
+    """
+    w = gate_weights(logits, idx)
+    w1 = w[:, 0].astype(np.float32)
+    w2 = (np.float32(1.0) - w1).astype(np.float32)
+    return np.stack([w1, w2], axis=1)
+
+
+def gate_dense_topk_softmax(logits, k: int = 2) -> np.ndarray:
+    """Dense ``G(x) = Softmax(TopK(l))``: logits outside the top k set to -inf.
+
+    notion notes, "Sparse gating", eq. G(x): "all other values ... are set to -inf,
+    leading to 0 weights".  Returns fp64 ``[T, E]``.
+    """
+    l = _f64(logits)
+    idx = top2_select(l, k)
+    masked = np.full_like(l, -np.inf)
+    rows = np.arange(l.shape[0])[:, None]
+    masked[rows, idx] = l[rows, idx]
+    m = masked.max(axis=1, keepdims=True)
+    e = np.exp(masked - m)  # exp(-inf) == 0
+    return e / e.sum(axis=1, keepdims=True)
+
+
+def gate_dense_softmax_topk_renorm(logits, k: int = 2) -> np.ndarray:
+    """Dense gate from softmax over all E, then top k, then renormalise.
+
+    ml-canon "52 Mixtral", "PyTorch Mixtral's MoE FFN (top-2 of 8)": softmax over the
+    experts, keep the top two, divide by their sum.  The kept set is chosen on the
+    logits (softmax is monotone) with the same tie rule.  Returns fp64 ``[T, E]``.
+    """
+    l = _f64(logits)
+    m = l.max(axis=1, keepdims=True)
+    p = np.exp(l - m)
+    p = p / p.sum(axis=1, keepdims=True)
+    idx = top2_select(l, k)
+    rows = np.arange(l.shape[0])[:, None]
+    kept = p[rows, idx]
+    kept = kept / kept.sum(axis=1, keepdims=True)
+    G = np.zeros_like(l)
+    G[rows, idx] = kept
+    return G
+
+
+def permutation(idx, E: int):
+    """Group the flattened (token, slot) pairs by expert (stable counting sort).
+
+    ml-canon "52 Mixtral", "Questions worth asking" (gather tokens by expert and
+    scatter them back); notion notes, "Expert Parallelism" (results returned to the
+    original token location).  Row order inside a group is ascending in the
+    flattened index ``f = t*k + j`` (reading: the pages are silent).
+
+    Returns ``offsets[E+1]`` (group e owns rows offsets[e]:offsets[e+1]),
+    ``perm_token[P]`` (source token of each row) and ``inv_perm[T, k]`` (row that
+    holds pair (t, j)), all int32.
+    """
+    idx = np.asarray(idx)
+    T, k = idx.shape
+    flat = idx.reshape(-1).astype(np.int64)
+    counts = np.bincount(flat, minlength=E)
+    offsets = np.zeros(E + 1, dtype=np.int64)
+    offsets[1:] = np.cumsum(counts)
+    perm = np.argsort(flat, kind="stable")
+    perm_token = perm // k
+    inv = np.empty(T * k, dtype=np.int64)
+    inv[perm] = np.arange(T * k)
+    return (offsets.astype(np.int32), perm_token.astype(np.int32),
+            inv.reshape(T, k).astype(np.int32))
+
+
+def gather_rows(x, perm_token) -> np.ndarray:
+    """``x_perm[r] = x[perm_token[r]]`` (pure data movement; dtype preserved)."""
+    return np.asarray(x)[np.asarray(perm_token, dtype=np.int64)]
+
+
+def silu(z) -> np.ndarray:
+    """``silu(z) = z * sigma(z) = z / (1 + exp(-z))`` in fp64."""
+    z = _f64(z)
+    with np.errstate(over="ignore"):
+        return z / (1.0 + np.exp(-z))
+
+
+def expert_swiglu(xr, W1e, W3e, W2e) -> np.ndarray:
+    """One expert's SwiGLU FFN on rows ``xr[n, d]``: ``(silu(xr W1e^T) * (xr W3e^T)) W2e^T``.
+
+    Shapes: ``W1e, W3e`` are ``[h, d]``, ``W2e`` is ``[d, h]`` (the stacked layouts
+    W1/W3 ``[E, h, d]`` and W2 ``[E, d, h]``).  notion notes, "Implementation"
+    (SwiGLU expert function); atlas "Mixtral", "Design overview" (inner dim 14336).
+    """
+    xr = _f64(xr)
+    a = xr @ _f64(W1e).T
+    b = xr @ _f64(W3e).T
+    return (silu(a) * b) @ _f64(W2e).T
+
+
+def expert_ffn_grouped(x_perm, offsets, W1, W3, W2) -> np.ndarray:
+    """Run every expert group through its own SwiGLU FFN; returns fp64 ``Y[P, d]``.
+
+    An empty group contributes nothing (no rows).
+    """
+    x_perm = _f64(x_perm)
+    P = x_perm.shape[0]
+    d = np.asarray(W2).shape[1]
+    Y = np.zeros((P, d), dtype=np.float64)
+    E = len(offsets) - 1
+    for e in range(E):
+        lo, hi = int(offsets[e]), int(offsets[e + 1])
+        if hi > lo:
+            Y[lo:hi] = expert_swiglu(x_perm[lo:hi], W1[e], W3[e], W2[e])
+    return Y
+
+
+def combine(Y, inv_perm, w) -> np.ndarray:
+    """``y[t] = sum_j w[t, j] * Y[inv_perm[t, j]]`` in fp64.
+
+    crackai "Mixtral of Experts", "Top-2 Routing in Detail":
+    y = w_1 Expert_{i1}(x) + w_2 Expert_{i2}(x); notion notes, eq. y.
+    """
+    Y = _f64(Y)
+    w = _f64(w)
+    inv = np.asarray(inv_perm, dtype=np.int64)
+    y = np.zeros((inv.shape[0], Y.shape[1]), dtype=np.float64)
+    for j in range(inv.shape[1]):
+        y += w[:, j:j + 1] * Y[inv[:, j]]
+    return y
+
+
+def moe_layer(x, Wg, W1, W3, W2, k: int = 2) -> dict:
+    """The routed layer (oracle O1): route, group by expert, SwiGLU per group, combine.
+
+    Returns a dict with every intermediate: ``logits`` (fp64), ``idx`` (int32
+    ``[T, k]``), ``w`` (fp64), ``w_f32`` (float32 as stored by the layer),
+    ``offsets``, ``perm_token``, ``inv_perm`` (int32), ``Y`` (fp64 ``[P, d]``) and
+    ``y`` (fp64 ``[T, d]``).  ``y`` uses the fp64 gate (the definition).
+    """
+    E = np.asarray(Wg).shape[1]
+    logits = router_logits(x, Wg)
+    idx = top2_select(logits, k)
+    w = gate_weights(logits, idx)
+    offsets, perm_token, inv_perm = permutation(idx, E)
+    x_perm = gather_rows(_f64(x), perm_token)
+    Y = expert_ffn_grouped(x_perm, offsets, W1, W3, W2)
+    y = combine(Y, inv_perm, w)
+    return dict(logits=logits, idx=idx, w=w, w_f32=gate_weights_f32(logits, idx),
+                offsets=offsets, perm_token=perm_token, inv_perm=inv_perm, Y=Y, y=y)
+
+
+def moe_layer_dense(x, Wg, W1, W3, W2, k: int = 2) -> np.ndarray:
+    """Brute-force layer (oracle O2): every expert on every token, weighted by dense G.
+
+    ``y = sum_{e=0}^{E-1} G(x)_e E_e(x)`` with ``G`` the -inf-masked softmax, exactly
+    as notion notes, "Implementation", eq. y is written (experts with G = 0 are still
+    evaluated and multiplied by zero).  No grouping or permutation.
+    """
+    x = _f64(x)
+    G = gate_dense_topk_softmax(router_logits(x, Wg), k)
+    y = np.zeros((x.shape[0], np.asarray(W2).shape[1]), dtype=np.float64)
+    for e in range(G.shape[1]):
+        y += G[:, e:e + 1] * expert_swiglu(x, W1[e], W3[e], W2[e])
+    return y
+
+
+def mixtral_param_counts(d: int = 32 * 128, h: int = 14336, E: int = 8, k: int = 2,
+                         layers: int = 32, vocab: int = 32000, n_heads: int = 32,
+                         n_kv_heads: int = 8, head_dim: int = 128) -> dict:
+    """Closed-form parameter counts of the whole model from the pages' dimensions.
+
+    atlas "Mixtral", "Design overview": 32 layers, 8 experts per layer, SwiGLU
+    inner dim 14336, 32 query / 8 KV heads of dim 128; vocab 32000 ("Notable
+    omissions").  The model dim is the heads x head_dim product (the pages never
+    print it directly).  Attention is grouped-query (q and o are d x d; k and v
+    are d x (kv_heads * head_dim)); embeddings are untied (input + output); each
+    layer has two RMSNorm weight vectors and there is a final norm.  Returns total
+    and active (k of E experts) counts.
+    """
+    expert = 3 * d * h
+    router = d * E
+    attn = 2 * d * (n_heads * head_dim) + 2 * d * (n_kv_heads * head_dim)
+    norms = 2 * d
+    per_layer_shared = attn + router + norms
+    embed = 2 * vocab * d
+    total = layers * (E * expert + per_layer_shared) + embed + d
+    active = layers * (k * expert + per_layer_shared) + embed + d
+    return dict(total=total, active=active, expert_per_layer=E * expert)
