@@ -1,0 +1,142 @@
+/*
+ * moe.h -- C ABI of libmoe: the Mixtral top-2-of-8 sparse-MoE SwiGLU feed-forward
+ * layer on one NVIDIA B200 (sm_100a).
+ *
+ * The layer (notion notes "Mixtral of Experts", "Sparse gating" eq. G(x) and
+ * "Implementation" eq. y; crackai "Mixtral of Experts", "Top-2 Routing in Detail"):
+ *     l      = x . W_g                              router logits, [T, E]
+ *     G(x)   = Softmax(TopK(l)), K = 2              logits outside the top 2 -> -inf
+ *     E_e(x) = W2[e] (silu(W1[e] x) * (W3[e] x))    SwiGLU expert (atlas "Mixtral",
+ *                                                   "Design overview": inner dim h)
+ *     y      = sum_e G(x)_e E_e(x) = w1 E_{i1}(x) + w2 E_{i2}(x)
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Ownership: the caller owns every buffer.  The library never allocates, frees
+ *   or synchronises on these calls; all scratch lives in the caller's workspace.
+ *   All entry points are stateless and may be called from several host threads.
+ * - Pointers are DEVICE pointers (cudaMalloc or equivalent) unless stated
+ *   otherwise, 16-byte aligned, tensors dense and row-major.  Outputs must not
+ *   alias inputs.
+ * - Execution: work is queued on `stream` and runs asynchronously.  Argument
+ *   errors are returned before anything is queued.  A failed launch returns
+ *   MOE_ERR_CUDA.  Errors found on the device (a pipeline wait that ran out of
+ *   time) are recorded in the workspace status word; read it with
+ *   moe_device_status().
+ * - dtype: MOE_BF16 (bfloat16 activations and weights, fp32 accumulation on tensor
+ *   cores) or MOE_F32 (fp32 everywhere, CUDA cores, no TF32).
+ * - Supported shapes: k == 2; 2 <= E <= 32; d and h multiples of 8; T >= 0
+ *   (T == 0 is a no-op returning MOE_OK).  Inputs must be finite.
+ * - Routing: experts are ranked by (logit descending, index ascending), so ties go
+ *   to the lower index; logits are accumulated in fp64 from the exact products of
+ *   the inputs.  Slot 0 holds the larger logit.  w1 = 1/(1+exp(l_i2-l_i1)) is
+ *   computed in fp64 and rounded once to float; w2 = 1 - w1 in float.
+ * - Grouping: the (token, slot) pairs are stably sorted by expert over the
+ *   flattened index f = t*k + j; group e owns rows offsets[e] .. offsets[e+1]-1 in
+ *   ascending token order.
+ */
+#ifndef MOE_H_
+#define MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1, /* null/misaligned pointer, negative or inconsistent size */
+    MOE_ERR_UNSUPPORTED = 2, /* k != 2, E outside [2, 32], d or h not a multiple of 8 */
+    MOE_ERR_WORKSPACE = 3,   /* ws_bytes smaller than moe_workspace_bytes() */
+    MOE_ERR_CUDA = 4,        /* a CUDA call or kernel launch failed */
+    MOE_ERR_TIMEOUT = 5      /* a device-side pipeline wait gave up (moe_device_status) */
+} moe_status;
+
+/* Device status flags, OR-ed into the workspace status word. */
+#define MOE_DEV_FLAG_TIMEOUT 0x1u
+
+/* Bytes of workspace that moe_layer_forward needs for this shape (a 1 KiB-aligned
+ * layout of routing results, permutation, gathered rows x_perm, the SwiGLU
+ * activations H and the fp32 expert outputs).  It also covers moe_permute and
+ * moe_expert_ffn.  Returns 0 for unsupported arguments. */
+size_t moe_workspace_bytes(int T, int d, int h, int E, int k, moe_dtype dt);
+
+/* Router + top-2 + softmax of the two kept logits.
+ * crackai "Mixtral of Experts", "Top-2 Routing in Detail" (gate_logits = x . W_gate);
+ * notion notes, "Sparse gating" eq. G(x).
+ *   x        [T, d]  dt          tokens
+ *   Wg       [d, E]  dt          router weights
+ *   topk_idx [T, k]  int32 out   chosen experts, slot 0 = larger logit
+ *   topk_w   [T, k]  float out   their gate weights (sum exactly 1 in float) */
+moe_status moe_route(const void *x, const void *Wg, int T, int d, int E, int k,
+                     moe_dtype dt, int32_t *topk_idx, float *topk_w,
+                     cudaStream_t stream);
+
+/* Group token rows by expert: histogram, exclusive scan, stable ranks, row gather.
+ * ml-canon "52 Mixtral", "Questions worth asking" (gather and scatter tokens);
+ * notion notes, "Expert Parallelism" (outputs returned to the token's location).
+ *   topk_idx   [T, k]     int32 in
+ *   x          [T, d]     dt in
+ *   offsets    [E + 1]    int32 out   group e = rows offsets[e] .. offsets[e+1]-1
+ *   perm_token [T*k]      int32 out   source token of each grouped row
+ *   inv_perm   [T, k]     int32 out   grouped row holding pair (t, j)
+ *   x_perm     [T*k, d]   dt out      x_perm[r] = x[perm_token[r]]
+ *   ws, ws_bytes                       workspace (>= moe_workspace_bytes)
+ * topk_idx entries must lie in [0, E) and differ within a token. */
+moe_status moe_permute(const int32_t *topk_idx, const void *x, int T, int d, int E,
+                       int k, moe_dtype dt, int32_t *offsets, int32_t *perm_token,
+                       int32_t *inv_perm, void *x_perm, void *ws, size_t ws_bytes,
+                       cudaStream_t stream);
+
+/* Per-expert SwiGLU FFN over the grouped rows (notion notes, "Implementation":
+ * SwiGLU expert function; atlas "Mixtral", "Design overview").
+ *   x_perm  [rows, d]   dt in        rows grouped by expert
+ *   offsets [E + 1]     int32 in     device copy; offsets[E] must equal rows
+ *   W1, W3  [E, h, d]   dt in        gate and up projections (d contiguous)
+ *   W2      [E, d, h]   dt in        down projection (h contiguous)
+ *   y_perm  [rows, d]   float out    Y_r = W2[e](silu(W1[e] x_r) * W3[e] x_r)
+ *   ws, ws_bytes                      workspace (holds H [rows, h])
+ * bf16 runs on tcgen05 tensor cores (fp32 accumulation in tensor memory; H is
+ * rounded once to bf16); f32 runs on CUDA cores in fp32. */
+moe_status moe_expert_ffn(const void *x_perm, const int32_t *offsets, const void *W1,
+                          const void *W3, const void *W2, int rows, int d, int h,
+                          int E, moe_dtype dt, float *y_perm, void *ws,
+                          size_t ws_bytes, cudaStream_t stream);
+
+/* Weighted un-permute: y[t] = w[t,0] Y[inv[t,0]] + w[t,1] Y[inv[t,1]] in fp32,
+ * rounded once to dt.  crackai "Mixtral of Experts", "Top-2 Routing in Detail"
+ * (y = w_1 Expert_{i1}(x) + w_2 Expert_{i2}(x)); notion notes, eq. y.
+ *   y_perm   [T*k, d] float in;  inv_perm [T, k] int32 in;  topk_w [T, k] float in
+ *   y        [T, d]   dt out */
+moe_status moe_combine(const float *y_perm, const int32_t *inv_perm,
+                       const float *topk_w, int T, int d, int k, moe_dtype dt, void *y,
+                       cudaStream_t stream);
+
+/* The whole layer: route -> permute -> expert FFN -> combine, queued on `stream`
+ * with no host synchronisation (group sizes stay on the device).
+ *   x [T, d], Wg [d, E], W1/W3 [E, h, d], W2 [E, d, h] in dt;  y [T, d] out in dt. */
+moe_status moe_layer_forward(const void *x, const void *Wg, const void *W1,
+                             const void *W3, const void *W2, int T, int d, int h,
+                             int E, int k, moe_dtype dt, void *y, void *ws,
+                             size_t ws_bytes, cudaStream_t stream);
+
+/* Synchronise `stream`, read the workspace status word into *flags (host
+ * pointer; MOE_DEV_FLAG_* bits), then clear it.  Returns MOE_ERR_TIMEOUT if the
+ * timeout flag was set, MOE_OK otherwise.  Diagnostic call: it synchronises. */
+moe_status moe_device_status(void *ws, size_t ws_bytes, uint32_t *flags,
+                             cudaStream_t stream);
+
+/* Static description of a status code. */
+const char *moe_status_string(moe_status st);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_H_ */

@@ -212,11 +212,12 @@ def expert_swiglu(xr, W1e, W3e, W2e) -> np.ndarray:
 def expert_ffn_grouped(x_perm, offsets, W1, W3, W2) -> np.ndarray:
     """Run every expert group through its own SwiGLU FFN; returns fp64 ``Y[P, d]``.
 
-    An empty group contributes nothing (no rows).
+    An empty group contributes nothing (no rows).  ``W1``/``W3``/``W2`` only need
+    to support ``[e]`` indexing, so large stacks can be handed over one expert at a
+    time.
     """
     x_perm = _f64(x_perm)
-    P = x_perm.shape[0]
-    d = np.asarray(W2).shape[1]
+    P, d = x_perm.shape
     Y = np.zeros((P, d), dtype=np.float64)
     E = len(offsets) - 1
     for e in range(E):
@@ -249,8 +250,8 @@ def moe_layer(x, Wg, W1, W3, W2, k: int = 2) -> dict:
     ``offsets``, ``perm_token``, ``inv_perm`` (int32), ``Y`` (fp64 ``[P, d]``) and
     ``y`` (fp64 ``[T, d]``).  ``y`` uses the fp64 gate (the definition).
     """
-    E = np.asarray(Wg).shape[1]
     logits = router_logits(x, Wg)
+    E = logits.shape[1]
     idx = top2_select(logits, k)
     w = gate_weights(logits, idx)
     offsets, perm_token, inv_perm = permutation(idx, E)
@@ -270,7 +271,7 @@ def moe_layer_dense(x, Wg, W1, W3, W2, k: int = 2) -> np.ndarray:
     """
     x = _f64(x)
     G = gate_dense_topk_softmax(router_logits(x, Wg), k)
-    y = np.zeros((x.shape[0], np.asarray(W2).shape[1]), dtype=np.float64)
+    y = np.zeros(x.shape, dtype=np.float64)
     for e in range(G.shape[1]):
         y += G[:, e:e + 1] * expert_swiglu(x, W1[e], W3[e], W2[e])
     return y

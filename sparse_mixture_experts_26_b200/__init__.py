@@ -1,0 +1,183 @@
+"""Mixtral top-2-of-8 sparse-MoE SwiGLU layer on NVIDIA B200 (sm_100a).
+
+A thin ctypes binding over ``libmoe.so`` (C ABI declared in ``include/moe.h``).
+Every step of the layer runs in the library's CUDA kernels; this module only
+checks tensor properties, passes device pointers and the current CUDA stream, and
+turns status codes into exceptions.  There is no CPU fallback: importing the
+package fails if the library has not been built.
+
+Entry points (same names as the C ABI):
+    moe_route, moe_permute, moe_expert_ffn, moe_combine, moe_layer_forward,
+    moe_workspace_bytes, moe_device_status, moe_status_string
+plus the conveniences ``alloc_workspace`` and ``layer_forward``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "LIB_PATH", "MoeError", "moe_workspace_bytes", "moe_route", "moe_permute",
+    "moe_expert_ffn", "moe_combine", "moe_layer_forward", "moe_device_status",
+    "moe_status_string", "alloc_workspace", "layer_forward", "EXPORTED_SYMBOLS",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe.so")
+
+MOE_F32, MOE_BF16 = 0, 1
+_STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
+                 3: "MOE_ERR_WORKSPACE", 4: "MOE_ERR_CUDA", 5: "MOE_ERR_TIMEOUT"}
+EXPORTED_SYMBOLS = ("moe_workspace_bytes", "moe_route", "moe_permute", "moe_expert_ffn",
+                    "moe_combine", "moe_layer_forward", "moe_device_status",
+                    "moe_status_string")
+
+
+class MoeError(RuntimeError):
+    def __init__(self, fn: str, code: int, msg: str):
+        super().__init__(f"{fn} -> {_STATUS_NAMES.get(code, code)}: {msg}")
+        self.code = code
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing; build it with "
+            "`python -m sparse_mixture_experts_26_b200.build` (nvcc, sm_100a)")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i32, sz, u32p = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_void_p
+    sigs = {
+        "moe_workspace_bytes": (sz, [i32, i32, i32, i32, i32, i32]),
+        "moe_route": (i32, [vp, vp, i32, i32, i32, i32, i32, vp, vp, vp]),
+        "moe_permute": (i32, [vp, vp, i32, i32, i32, i32, i32, vp, vp, vp, vp, vp, sz, vp]),
+        "moe_expert_ffn": (i32, [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, vp, vp, sz, vp]),
+        "moe_combine": (i32, [vp, vp, vp, i32, i32, i32, i32, vp, vp]),
+        "moe_layer_forward": (i32, [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, vp,
+                                    sz, vp]),
+        "moe_device_status": (i32, [vp, sz, u32p, vp]),
+        "moe_status_string": (ctypes.c_char_p, [i32]),
+    }
+    for name, (res, args) in sigs.items():
+        f = getattr(lib, name)
+        f.restype = res
+        f.argtypes = args
+    return lib
+
+
+_lib = _load()
+
+
+def moe_status_string(code: int) -> str:
+    return _lib.moe_status_string(int(code)).decode()
+
+
+def _check(fn: str, code: int) -> None:
+    if code != 0:
+        raise MoeError(fn, code, moe_status_string(code))
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return MOE_BF16
+    if t.dtype == torch.float32:
+        return MOE_F32
+    raise TypeError(f"unsupported dtype {t.dtype} (bf16 or fp32)")
+
+
+def _dev(*ts: torch.Tensor) -> None:
+    for t in ts:
+        if not t.is_cuda:
+            raise ValueError("all tensors must be CUDA tensors")
+        if not t.is_contiguous():
+            raise ValueError("all tensors must be contiguous")
+
+
+def _ptr(t: torch.Tensor | None) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def moe_workspace_bytes(T: int, d: int, h: int, E: int = 8, k: int = 2,
+                        dtype: torch.dtype = torch.bfloat16) -> int:
+    dt = MOE_BF16 if dtype == torch.bfloat16 else MOE_F32
+    return int(_lib.moe_workspace_bytes(T, d, h, E, k, dt))
+
+
+def alloc_workspace(T: int, d: int, h: int, E: int = 8, k: int = 2,
+                    dtype: torch.dtype = torch.bfloat16, device="cuda") -> torch.Tensor:
+    """A zeroed workspace of ``moe_workspace_bytes`` bytes (the status word starts at 0)."""
+    n = moe_workspace_bytes(T, d, h, E, k, dtype)
+    if n == 0:
+        raise MoeError("moe_workspace_bytes", 2, "unsupported shape")
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def moe_route(x, Wg, topk_idx, topk_w, k: int = 2, stream=None) -> None:
+    _dev(x, Wg, topk_idx, topk_w)
+    T, d = x.shape
+    E = Wg.shape[1]
+    _check("moe_route", _lib.moe_route(_ptr(x), _ptr(Wg), T, d, E, k, _dt(x), _ptr(topk_idx),
+                                       _ptr(topk_w), _stream(stream)))
+
+
+def moe_permute(topk_idx, x, offsets, perm_token, inv_perm, x_perm, ws, E: int, k: int = 2,
+                stream=None) -> None:
+    _dev(topk_idx, x, offsets, perm_token, inv_perm, x_perm, ws)
+    T, d = x.shape
+    _check("moe_permute", _lib.moe_permute(
+        _ptr(topk_idx), _ptr(x), T, d, E, k, _dt(x), _ptr(offsets), _ptr(perm_token),
+        _ptr(inv_perm), _ptr(x_perm), _ptr(ws), ws.numel() * ws.element_size(),
+        _stream(stream)))
+
+
+def moe_expert_ffn(x_perm, offsets, W1, W3, W2, y_perm, ws, stream=None) -> None:
+    _dev(x_perm, offsets, W1, W3, W2, y_perm, ws)
+    rows, d = x_perm.shape
+    E, h, _ = W1.shape
+    _check("moe_expert_ffn", _lib.moe_expert_ffn(
+        _ptr(x_perm), _ptr(offsets), _ptr(W1), _ptr(W3), _ptr(W2), rows, d, h, E, _dt(x_perm),
+        _ptr(y_perm), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def moe_combine(y_perm, inv_perm, topk_w, y, k: int = 2, stream=None) -> None:
+    _dev(y_perm, inv_perm, topk_w, y)
+    T, d = y.shape
+    _check("moe_combine", _lib.moe_combine(_ptr(y_perm), _ptr(inv_perm), _ptr(topk_w), T, d, k,
+                                           _dt(y), _ptr(y), _stream(stream)))
+
+
+def moe_layer_forward(x, Wg, W1, W3, W2, y, ws, k: int = 2, stream=None) -> None:
+    _dev(x, Wg, W1, W3, W2, y, ws)
+    T, d = x.shape
+    E, h, _ = W1.shape
+    _check("moe_layer_forward", _lib.moe_layer_forward(
+        _ptr(x), _ptr(Wg), _ptr(W1), _ptr(W3), _ptr(W2), T, d, h, E, k, _dt(x), _ptr(y),
+        _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def moe_device_status(ws, stream=None) -> int:
+    """Synchronise, return and clear the workspace's device status flags."""
+    flags = ctypes.c_uint32(0)
+    code = _lib.moe_device_status(_ptr(ws), ws.numel() * ws.element_size(),
+                                  ctypes.addressof(flags), _stream(stream))
+    if code not in (0, 5):
+        _check("moe_device_status", code)
+    return int(flags.value)
+
+
+def layer_forward(x, Wg, W1, W3, W2, ws=None, out=None, stream=None) -> torch.Tensor:
+    """Run the whole layer, allocating the workspace and output with torch if not given."""
+    T, d = x.shape
+    E, h, _ = W1.shape
+    if ws is None:
+        ws = alloc_workspace(T, d, h, E, 2, x.dtype, x.device)
+    if out is None:
+        out = torch.empty_like(x)
+    moe_layer_forward(x, Wg, W1, W3, W2, out, ws, stream=stream)
+    return out

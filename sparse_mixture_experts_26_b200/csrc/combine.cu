@@ -1,0 +1,75 @@
+// combine.cu -- weighted un-permute of the expert outputs.
+//
+// crackai "Mixtral of Experts", "Top-2 Routing in Detail":
+// y = w_1 Expert_{i1}(x) + w_2 Expert_{i2}(x); notion notes "Mixtral of Experts",
+// "Implementation", eq. y.  Each output element is w0*Y[r0] + w1*Y[r1] evaluated in
+// fp32 (slot 0 first, one fused multiply-add for slot 1) and rounded once to the
+// output dtype.  Pure streaming: reads 2 fp32 rows, writes 1 row per token.
+#include <cuda_bf16.h>
+
+#include "moe_internal.h"
+
+namespace moe {
+namespace {
+
+constexpr int kCombineThreads = 256;
+
+__device__ __forceinline__ void store4(float* y, size_t i, float4 v) {
+    reinterpret_cast<float4*>(y)[i] = v;
+}
+__device__ __forceinline__ void store4(__nv_bfloat16* y, size_t i, float4 v) {
+    __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y);
+    __nv_bfloat162 hi = __floats2bfloat162_rn(v.z, v.w);
+    uint2 u;
+    u.x = *reinterpret_cast<uint32_t*>(&lo);
+    u.y = *reinterpret_cast<uint32_t*>(&hi);
+    reinterpret_cast<uint2*>(y)[i] = u;
+}
+
+template <typename Tout>
+__global__ void __launch_bounds__(kCombineThreads)
+    combine_kernel(const float4* __restrict__ Y, const int32_t* __restrict__ inv,
+                   const float* __restrict__ w, int T, int d4, Tout* __restrict__ y) {
+    const size_t n = static_cast<size_t>(T) * d4;
+    const unsigned P = 2u * static_cast<unsigned>(T);
+    for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
+         i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+        const size_t t = i / d4;
+        const size_t c = i - t * d4;
+        const unsigned r0 = static_cast<unsigned>(inv[2 * t]);
+        const unsigned r1 = static_cast<unsigned>(inv[2 * t + 1]);
+        const float w0 = w[2 * t], w1 = w[2 * t + 1];
+        // inv_perm entries outside [0, 2T) would come from an invalid permutation;
+        // they contribute nothing instead of reading out of bounds.
+        const float4 a = r0 < P ? Y[static_cast<size_t>(r0) * d4 + c] : make_float4(0, 0, 0, 0);
+        const float4 b = r1 < P ? Y[static_cast<size_t>(r1) * d4 + c] : make_float4(0, 0, 0, 0);
+        float4 o;
+        o.x = fmaf(w1, b.x, w0 * a.x);
+        o.y = fmaf(w1, b.y, w0 * a.y);
+        o.z = fmaf(w1, b.z, w0 * a.z);
+        o.w = fmaf(w1, b.w, w0 * a.w);
+        store4(y, i, o);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_combine(const float* Y, const int32_t* inv_perm, const float* w, int T,
+                           int d, moe_dtype dt, void* y, cudaStream_t s) {
+    const int d4 = d / 4;
+    const size_t n = static_cast<size_t>(T) * d4;
+    size_t blocks = (n + kCombineThreads - 1) / kCombineThreads;
+    const size_t cap = static_cast<size_t>(device_sm_count()) * 8;
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    if (dt == MOE_BF16)
+        combine_kernel<__nv_bfloat16><<<static_cast<unsigned>(blocks), kCombineThreads, 0, s>>>(
+            reinterpret_cast<const float4*>(Y), inv_perm, w, T, d4,
+            static_cast<__nv_bfloat16*>(y));
+    else
+        combine_kernel<float><<<static_cast<unsigned>(blocks), kCombineThreads, 0, s>>>(
+            reinterpret_cast<const float4*>(Y), inv_perm, w, T, d4, static_cast<float*>(y));
+    return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,437 @@
+// grouped_gemm_sm100.cu -- the per-expert SwiGLU FFN on 5th-generation tensor cores.
+//
+// notion notes "Mixtral of Experts", "Implementation": the expert function is the
+// SwiGLU FFN; atlas "Mixtral", "Design overview": inner dimension 14336.  notion
+// notes, "Architectural details" mention that single-GPU MoE runs with specialised
+// sparse-matmul kernels (Megablocks); this is a grouped GEMM instead: every expert's
+// rows are contiguous after the permutation, so each expert is one dense GEMM over
+// its own rows, and all experts run in one persistent launch.
+//
+//   GEMM1 (+SwiGLU):  H[r, n] = silu(x_r . W1[e, n]) * (x_r . W3[e, n])   bf16 out
+//   GEMM2:            Y[r, c] = H_r . W2[e, c]                            fp32 out
+//
+// Both are "TN" products with both operands K-major, the native tcgen05 layout:
+//   A = grouped activations [rows, K], B = the expert's weight rows [N, K].
+//
+// Design (one CTA per SM, persistent, 6 warps):
+//   warp 0      TMA producer: 128x64 A tile + 256x64 B tile per stage (48 KiB),
+//               kStages-deep ring of shared-memory stages guarded by mbarriers.
+//   warp 1      allocates 512 TMEM columns; one thread issues tcgen05.mma
+//               (M=128, N=256, K=16; four per 64-wide K block) into one of two
+//               128x256 fp32 accumulators, and commits stage/accumulator barriers.
+//   warps 2-5   epilogue: tcgen05.ld the accumulator (one row per thread), apply
+//               silu(a)*b (GEMM1) or nothing (GEMM2), store to global, release
+//               the accumulator.  The other accumulator is being filled meanwhile.
+// For GEMM1 the B tile stacks 128 rows of W1 over the same 128 rows of W3, so
+// accumulator columns [0,128) hold a and [128,256) hold b for the same outputs.
+//
+// Tiles never mix experts' weights: a tile is (expert, 128-row block of that
+// expert's rows, output-column block).  A row block may run past the expert's last
+// row into the next expert (or past the end, where TMA fills zeros); those rows
+// are computed but not stored.  Group sizes are read on the device, so the host
+// never waits for the routing.  Every wait is bounded (see sm100_ptx.cuh).
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include <cstdio>
+#include <mutex>
+
+#include "moe_internal.h"
+#include "sm100_ptx.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kBM = 128;        // rows per tile (TMEM lanes)
+constexpr int kBK = 64;         // K per stage: one 128-byte swizzle atom of bf16
+constexpr int kMmaN = 256;      // accumulator columns per tile
+constexpr int kStages = 4;
+constexpr int kABytes = kBM * kBK * 2;      // 16 KiB
+constexpr int kBBytes = kMmaN * kBK * 2;    // 32 KiB
+constexpr int kStageBytes = kABytes + kBBytes;
+constexpr int kThreads = 192;
+constexpr int kEpiThreads = 128;
+constexpr uint32_t kTmemCols = 2 * kMmaN;   // two accumulators: all 512 columns
+constexpr uint32_t kIdesc = idesc_bf16_f32(kBM, kMmaN);
+constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 1024 /*bookkeeping*/;
+
+enum Epilogue { kEpiSwiGLU = 0, kEpiStoreF32 = 1 };
+
+struct GemmArgs {
+    const int32_t* offsets;  // [E+1] group row offsets (device)
+    int E;
+    int rows;           // grouped rows (T*k)
+    int K;              // reduction length
+    int N;              // output columns
+    int b_rows;         // rows of one expert in the flattened weight view [E*b_rows, K]
+    int n_tiles;        // output-column tiles per row block
+    void* out;          // H (bf16) or Y (fp32), row-major [rows, N]
+    uint32_t* status;   // workspace status word
+};
+
+struct Bookkeeping {
+    uint64_t full[kStages];
+    uint64_t empty[kStages];
+    uint64_t tmem_full[2];
+    uint64_t tmem_empty[2];
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort_flag;
+    int off[kMaxExperts + 1];        // sanitised group offsets
+    int tile_start[kMaxExperts + 1]; // prefix sum of tiles per group
+};
+static_assert(sizeof(Bookkeeping) <= 1024, "bookkeeping must fit its reserve");
+
+struct TileCoord {
+    int e, row0, row_end, nt;
+};
+
+__device__ __forceinline__ TileCoord decode_tile(const Bookkeeping& bk, int E, int tile) {
+    int g = 0;
+    while (g + 1 < E && tile >= bk.tile_start[g + 1]) ++g;
+    const int local = tile - bk.tile_start[g];
+    const int m_tiles = (bk.off[g + 1] - bk.off[g] + kBM - 1) / kBM;
+    TileCoord c;
+    c.e = g;
+    c.row0 = bk.off[g] + (local % m_tiles) * kBM;  // row blocks inner: weight tile reuse
+    c.nt = local / m_tiles;
+    c.row_end = bk.off[g + 1];
+    return c;
+}
+
+__device__ __forceinline__ float bits_f32(uint32_t u) { return __uint_as_float(u); }
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ float silu_mul(float a, float b) {
+    return a / (1.0f + __expf(-a)) * b;
+}
+
+// Bounded wait used only while tearing down after an abort.
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
+    const unsigned long long t0 = global_timer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (global_timer_ns() - t0 > kDrainTimeoutNs) break;
+    }
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(kThreads, 1)
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
+                        const __grid_constant__ CUtensorMap tmB0,
+                        const __grid_constant__ CUtensorMap tmB1, const GemmArgs args) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint8_t* sA = smem;
+    uint8_t* sB = smem + kStages * kABytes;
+    Bookkeeping& bk = *reinterpret_cast<Bookkeeping*>(smem + kStages * kStageBytes);
+    volatile int* abort_flag = &bk.abort_flag;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int E = args.E;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&bk.full[s], 1);
+            mbar_init(&bk.empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&bk.tmem_full[a], 1);
+            mbar_init(&bk.tmem_empty[a], kEpiThreads);
+        }
+        mbar_init(&bk.drain, 1);
+        bk.abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB0);
+        if (EPI == kEpiSwiGLU) tma_prefetch_desc(&tmB1);
+    }
+    if (warp == 1) tmem_alloc(&bk.tmem_base, kTmemCols);
+
+    // The routing results come from the previous launch on the stream.
+    pdl_wait();
+    if (threadIdx.x == 0) {
+        // Offsets are clamped to [0, rows] and made monotone so that nothing below
+        // can address rows outside the buffers, whatever the device array holds.
+        int prev = 0;
+        for (int g = 0; g <= E; ++g) {
+            int v = args.offsets[g];
+            v = v < prev ? prev : (v > args.rows ? args.rows : v);
+            bk.off[g] = v;
+            prev = v;
+        }
+        bk.off[E] = args.rows > prev ? prev : args.rows;
+        bk.tile_start[0] = 0;
+        for (int g = 0; g < E; ++g)
+            bk.tile_start[g + 1] =
+                bk.tile_start[g] + (bk.off[g + 1] - bk.off[g] + kBM - 1) / kBM * args.n_tiles;
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    const uint32_t tmem_base = bk.tmem_base;
+    const int total_tiles = bk.tile_start[E];
+    const int num_kb = (args.K + kBK - 1) / kBK;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t pending = 0, pending_phase = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
+                const TileCoord c = decode_tile(bk, E, tile);
+                const int brow = c.e * args.b_rows + c.nt * (EPI == kEpiSwiGLU ? 128 : 256);
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    if (!mbar_wait_bounded(&bk.empty[stage], phase ^ 1u, abort_flag,
+                                           args.status)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&bk.full[stage], kStageBytes);
+                    const int kc = kb * kBK;
+                    uint8_t* a_dst = sA + stage * kABytes;
+                    uint8_t* b_dst = sB + stage * kBBytes;
+                    tma_load_2d(&tmA, &bk.full[stage], a_dst, kc, c.row0);
+                    if (EPI == kEpiSwiGLU) {
+                        tma_load_2d(&tmB0, &bk.full[stage], b_dst, kc, brow);
+                        tma_load_2d(&tmB1, &bk.full[stage], b_dst + kBBytes / 2, kc, brow);
+                    } else {
+                        tma_load_2d(&tmB0, &bk.full[stage], b_dst, kc, brow);
+                        tma_load_2d(&tmB0, &bk.full[stage], b_dst + kBBytes / 2, kc, brow + 128);
+                    }
+                    pending |= 1u << stage;
+                    pending_phase = (pending_phase & ~(1u << stage)) | (phase << stage);
+                    if (++stage == kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (!ok) {
+                // Let copies already in flight land before the block can exit.
+                for (int s = 0; s < kStages; ++s)
+                    if (pending & (1u << s)) drain_wait(&bk.full[s], (pending_phase >> s) & 1u);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            bool ok = true, issued = false;
+            for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
+                if (!mbar_wait_bounded(&bk.tmem_empty[acc], acc_phase ^ 1u, abort_flag,
+                                       args.status)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kMmaN);
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    if (!mbar_wait_bounded(&bk.full[stage], phase, abort_flag, args.status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t ad = sw128_kmajor_desc(smem_u32(sA + stage * kABytes));
+                    const uint64_t bd = sw128_kmajor_desc(smem_u32(sB + stage * kBBytes));
+#pragma unroll
+                    for (int k = 0; k < kBK / 16; ++k)
+                        umma_bf16(d_tmem, ad + 2 * k, bd + 2 * k, kIdesc, (kb | k) != 0);
+                    umma_commit(&bk.empty[stage]);
+                    issued = true;
+                    if (++stage == kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                umma_commit(&bk.tmem_full[acc]);
+                acc ^= 1;
+                if (acc == 0) acc_phase ^= 1u;
+            }
+            if (!ok && issued) {
+                // Wait for the MMAs still reading shared memory / writing TMEM.
+                umma_commit(&bk.drain);
+                drain_wait(&bk.drain, 0);
+            }
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int q = warp & 3;  // TMEM lane quarter this warp may access
+        const int row_in_tile = q * 32 + lane;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
+            const TileCoord c = decode_tile(bk, E, tile);
+            if (!mbar_wait_bounded(&bk.tmem_full[acc], acc_phase, abort_flag, args.status))
+                break;
+            tc_fence_after();
+            const uint32_t tbase =
+                tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * kMmaN);
+            const int row = c.row0 + row_in_tile;
+            const bool valid = row < c.row_end;
+            if (EPI == kEpiSwiGLU) {
+                __nv_bfloat16* out =
+                    static_cast<__nv_bfloat16*>(args.out) + static_cast<size_t>(row) * args.N;
+                const int col0 = c.nt * 128;
+#pragma unroll 1
+                for (int ch = 0; ch < 4; ++ch) {
+                    uint32_t a[32], b[32];
+                    tmem_ld_32cols(tbase + ch * 32, a);
+                    tmem_ld_32cols(tbase + 128 + ch * 32, b);
+                    tmem_ld_wait();
+                    uint32_t p[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        p[i] = pack_bf16x2(silu_mul(bits_f32(a[2 * i]), bits_f32(b[2 * i])),
+                                           silu_mul(bits_f32(a[2 * i + 1]), bits_f32(b[2 * i + 1])));
+                    if (valid) {
+#pragma unroll
+                        for (int v = 0; v < 4; ++v) {
+                            const int col = col0 + ch * 32 + v * 8;
+                            if (col < args.N)
+                                *reinterpret_cast<uint4*>(out + col) =
+                                    make_uint4(p[4 * v], p[4 * v + 1], p[4 * v + 2], p[4 * v + 3]);
+                        }
+                    }
+                }
+            } else {
+                float* out = static_cast<float*>(args.out) + static_cast<size_t>(row) * args.N;
+                const int col0 = c.nt * 256;
+#pragma unroll 1
+                for (int ch = 0; ch < 8; ++ch) {
+                    uint32_t v[32];
+                    tmem_ld_32cols(tbase + ch * 32, v);
+                    tmem_ld_wait();
+                    if (valid) {
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            const int col = col0 + ch * 32 + j * 4;
+                            if (col < args.N)
+                                *reinterpret_cast<float4*>(out + col) =
+                                    make_float4(bits_f32(v[4 * j]), bits_f32(v[4 * j + 1]),
+                                                bits_f32(v[4 * j + 2]), bits_f32(v[4 * j + 3]));
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&bk.tmem_empty[acc]);
+            acc ^= 1;
+            if (acc == 0) acc_phase ^= 1u;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, kTmemCols);
+    }
+}
+
+// ---------------------------------------------------------------- host side
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// Row-major bf16 matrix [rows, cols] viewed as a 2-D tensor; box = 64 columns (one
+// 128-byte swizzle span) x box_rows rows, 128-byte swizzle, zero fill out of bounds.
+bool encode_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                    uint32_t box_rows) {
+    EncodeTiledFn enc = get_encode_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols * 2};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(kBK), box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+           CUDA_SUCCESS;
+}
+
+template <int EPI>
+cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
+                        const GemmArgs& args, int grid, cudaStream_t s, bool pdl) {
+    auto kern = grouped_gemm_kernel<EPI>;
+    static int configured[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && !configured[dev]) {
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+        configured[dev] = 1;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kern, a, b0, b1, args);
+}
+
+}  // namespace
+
+cudaError_t launch_ffn_bf16(const void* x_perm, const int32_t* offsets, const void* W1,
+                            const void* W3, const void* W2, int rows, int d, int h, int E,
+                            void* H, float* Y, uint32_t* status, cudaStream_t s) {
+    CUtensorMap mx, mw1, mw3, mh, mw2;
+    if (!encode_bf16_2d(&mx, x_perm, rows, d, kBM) ||
+        !encode_bf16_2d(&mw1, W1, static_cast<uint64_t>(E) * h, d, 128) ||
+        !encode_bf16_2d(&mw3, W3, static_cast<uint64_t>(E) * h, d, 128) ||
+        !encode_bf16_2d(&mh, H, rows, h, kBM) ||
+        !encode_bf16_2d(&mw2, W2, static_cast<uint64_t>(E) * d, h, 128))
+        return cudaErrorInvalidValue;
+
+    const int sms = device_sm_count();
+    // Upper bound on row blocks: sum_e ceil(n_e / 128) <= (rows + 127 E) / 128.
+    const long long row_blocks = (static_cast<long long>(rows) + 127LL * E) / kBM;
+
+    GemmArgs g1{offsets, E, rows, d, h, h, (h + 127) / 128, H, status};
+    long long tiles1 = row_blocks * g1.n_tiles;
+    int grid1 = static_cast<int>(tiles1 < sms ? (tiles1 < 1 ? 1 : tiles1) : sms);
+    cudaError_t err = launch_gemm<kEpiSwiGLU>(mx, mw1, mw3, g1, grid1, s, false);
+    if (err != cudaSuccess) return err;
+
+    GemmArgs g2{offsets, E, rows, h, d, d, (d + 255) / 256, Y, status};
+    long long tiles2 = row_blocks * g2.n_tiles;
+    int grid2 = static_cast<int>(tiles2 < sms ? (tiles2 < 1 ? 1 : tiles2) : sms);
+    return launch_gemm<kEpiStoreF32>(mh, mw2, mw2, g2, grid2, s, false);
+}
+
+}  // namespace moe

@@ -1,0 +1,220 @@
+// moe_api.cu -- the extern "C" entry points of libmoe (declared in include/moe.h).
+//
+// Each entry point validates its arguments on the host, then queues its kernels on
+// the caller's stream.  Nothing here allocates, frees or synchronises (except the
+// diagnostic moe_device_status and the opt-in MOE_DEBUG_SYNC=1 mode, which
+// synchronises after every launch and reports device-side flags).
+#include <cuda_runtime.h>
+
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include "moe_internal.h"
+
+namespace moe {
+
+int device_sm_count() {
+    static int cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (dev >= 0 && dev < 64 && cache[dev] > 0) return cache[dev];
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+        n = 148;
+    if (dev >= 0 && dev < 64) cache[dev] = n;
+    return n;
+}
+
+bool debug_sync_enabled() {
+    static int v = -1;
+    if (v < 0) {
+        const char* e = std::getenv("MOE_DEBUG_SYNC");
+        v = (e && e[0] == '1') ? 1 : 0;
+    }
+    return v == 1;
+}
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+moe_status check_shape(int T, int d, int h, int E, int k, moe_dtype dt, bool need_h) {
+    if (T < 0 || d <= 0 || (need_h && h <= 0) || E <= 0 || k <= 0) return MOE_ERR_INVALID_ARG;
+    if (dt != MOE_F32 && dt != MOE_BF16) return MOE_ERR_INVALID_ARG;
+    if (k != 2 || E < 2 || E > kMaxExperts) return MOE_ERR_UNSUPPORTED;
+    if (d % 8 != 0 || (need_h && h % 8 != 0)) return MOE_ERR_UNSUPPORTED;
+    // 32-bit row indices and element offsets inside one grouped buffer.
+    const long long P = 2LL * T;
+    if (P * d >= (1LL << 40) || (need_h && P * h >= (1LL << 40)) || T > (1 << 29))
+        return MOE_ERR_UNSUPPORTED;
+    return MOE_OK;
+}
+
+bool ptrs_ok(std::initializer_list<const void*> ps) {
+    for (const void* p : ps)
+        if (p == nullptr || !aligned16(p)) return false;
+    return true;
+}
+
+moe_status finish(cudaError_t err, cudaStream_t s, uint32_t* status) {
+    if (err != cudaSuccess) return MOE_ERR_CUDA;
+    if (debug_sync_enabled()) {
+        if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+        if (status) {
+            uint32_t flags = 0;
+            if (cudaMemcpy(&flags, status, 4, cudaMemcpyDeviceToHost) != cudaSuccess)
+                return MOE_ERR_CUDA;
+            if (flags & MOE_DEV_FLAG_TIMEOUT) return MOE_ERR_TIMEOUT;
+        }
+    }
+    return MOE_OK;
+}
+
+template <typename T>
+T* at(void* ws, size_t off) {
+    return reinterpret_cast<T*>(static_cast<char*>(ws) + off);
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+size_t moe_workspace_bytes(int T, int d, int h, int E, int k, moe_dtype dt) {
+    if (check_shape(T, d, h, E, k, dt, true) != MOE_OK) return 0;
+    return ws_layout(T, d, h, E, k, dt).total;
+}
+
+const char* moe_status_string(moe_status st) {
+    switch (st) {
+        case MOE_OK: return "ok";
+        case MOE_ERR_INVALID_ARG: return "invalid argument (null/misaligned pointer or bad size)";
+        case MOE_ERR_UNSUPPORTED: return "unsupported shape (need k == 2, 2 <= E <= 32, d and h multiples of 8)";
+        case MOE_ERR_WORKSPACE: return "workspace too small";
+        case MOE_ERR_CUDA: return "CUDA error";
+        case MOE_ERR_TIMEOUT: return "device pipeline wait timed out";
+    }
+    return "unknown status";
+}
+
+moe_status moe_route(const void* x, const void* Wg, int T, int d, int E, int k, moe_dtype dt,
+                     int32_t* topk_idx, float* topk_w, cudaStream_t stream) {
+    moe_status st = check_shape(T, d, 8, E, k, dt, false);
+    if (st != MOE_OK) return st;
+    if (T == 0) return MOE_OK;
+    if (!ptrs_ok({x, Wg, topk_idx, topk_w})) return MOE_ERR_INVALID_ARG;
+    return finish(launch_route(x, Wg, T, d, E, dt, topk_idx, topk_w, stream), stream, nullptr);
+}
+
+moe_status moe_permute(const int32_t* topk_idx, const void* x, int T, int d, int E, int k,
+                       moe_dtype dt, int32_t* offsets, int32_t* perm_token, int32_t* inv_perm,
+                       void* x_perm, void* ws, size_t ws_bytes, cudaStream_t stream) {
+    moe_status st = check_shape(T, d, 8, E, k, dt, false);
+    if (st != MOE_OK) return st;
+    if (!ptrs_ok({offsets, ws})) return MOE_ERR_INVALID_ARG;
+    const WsLayout L = ws_layout(T, d, 8, E, k, dt);
+    if (ws_bytes < L.permute_need) return MOE_ERR_WORKSPACE;
+    if (T == 0) {
+        // Empty batch: every group is empty.
+        if (cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (E + 1), stream) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        return MOE_OK;
+    }
+    if (!ptrs_ok({topk_idx, x, perm_token, inv_perm, x_perm})) return MOE_ERR_INVALID_ARG;
+    uint32_t* status = at<uint32_t>(ws, L.status);
+    return finish(launch_permute(topk_idx, x, T, d, E, dt, offsets, perm_token, inv_perm, x_perm,
+                                 at<int32_t>(ws, L.blk_counts), at<int32_t>(ws, L.blk_base),
+                                 status, stream),
+                  stream, status);
+}
+
+moe_status moe_expert_ffn(const void* x_perm, const int32_t* offsets, const void* W1,
+                          const void* W3, const void* W2, int rows, int d, int h, int E,
+                          moe_dtype dt, float* y_perm, void* ws, size_t ws_bytes,
+                          cudaStream_t stream) {
+    if (rows < 0 || rows % 2 != 0) return MOE_ERR_INVALID_ARG;
+    const int T = rows / 2;
+    moe_status st = check_shape(T, d, h, E, 2, dt, true);
+    if (st != MOE_OK) return st;
+    if (rows == 0) return MOE_OK;
+    if (!ptrs_ok({x_perm, offsets, W1, W3, W2, y_perm, ws})) return MOE_ERR_INVALID_ARG;
+    const WsLayout L = ws_layout(T, d, h, E, 2, dt);
+    if (ws_bytes < L.ffn_need) return MOE_ERR_WORKSPACE;
+    uint32_t* status = at<uint32_t>(ws, L.status);
+    cudaError_t err;
+    if (dt == MOE_BF16) {
+        err = launch_ffn_bf16(x_perm, offsets, W1, W3, W2, rows, d, h, E, at<void>(ws, L.H), y_perm,
+                              status, stream);
+        if (err == cudaErrorInvalidValue) return MOE_ERR_INVALID_ARG;  // tensor map refused
+    } else {
+        err = launch_ffn_f32(static_cast<const float*>(x_perm), offsets,
+                             static_cast<const float*>(W1), static_cast<const float*>(W3),
+                             static_cast<const float*>(W2), rows, d, h, E, at<float>(ws, L.H),
+                             y_perm, stream);
+    }
+    return finish(err, stream, status);
+}
+
+moe_status moe_combine(const float* y_perm, const int32_t* inv_perm, const float* topk_w, int T,
+                       int d, int k, moe_dtype dt, void* y, cudaStream_t stream) {
+    moe_status st = check_shape(T, d, 8, 2, k, dt, false);
+    if (st != MOE_OK) return st;
+    if (T == 0) return MOE_OK;
+    if (!ptrs_ok({y_perm, inv_perm, topk_w, y})) return MOE_ERR_INVALID_ARG;
+    return finish(launch_combine(y_perm, inv_perm, topk_w, T, d, dt, y, stream), stream, nullptr);
+}
+
+moe_status moe_layer_forward(const void* x, const void* Wg, const void* W1, const void* W3,
+                             const void* W2, int T, int d, int h, int E, int k, moe_dtype dt,
+                             void* y, void* ws, size_t ws_bytes, cudaStream_t stream) {
+    moe_status st = check_shape(T, d, h, E, k, dt, true);
+    if (st != MOE_OK) return st;
+    if (T == 0) return MOE_OK;
+    if (!ptrs_ok({x, Wg, W1, W3, W2, y, ws})) return MOE_ERR_INVALID_ARG;
+    const WsLayout L = ws_layout(T, d, h, E, k, dt);
+    if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+    uint32_t* status = at<uint32_t>(ws, L.status);
+    int32_t* idx = at<int32_t>(ws, L.topk_idx);
+    float* w = at<float>(ws, L.topk_w);
+    int32_t* offsets = at<int32_t>(ws, L.offsets);
+    int32_t* perm_token = at<int32_t>(ws, L.perm_token);
+    int32_t* inv_perm = at<int32_t>(ws, L.inv_perm);
+    void* x_perm = at<void>(ws, L.x_perm);
+    float* Y = at<float>(ws, L.Y);
+    const int P = 2 * T;
+
+    cudaError_t err = launch_route(x, Wg, T, d, E, dt, idx, w, stream);
+    if ((st = finish(err, stream, status)) != MOE_OK) return st;
+    err = launch_permute(idx, x, T, d, E, dt, offsets, perm_token, inv_perm, x_perm,
+                         at<int32_t>(ws, L.blk_counts), at<int32_t>(ws, L.blk_base), status,
+                         stream);
+    if ((st = finish(err, stream, status)) != MOE_OK) return st;
+    if (dt == MOE_BF16) {
+        err = launch_ffn_bf16(x_perm, offsets, W1, W3, W2, P, d, h, E, at<void>(ws, L.H), Y, status,
+                              stream);
+        if (err == cudaErrorInvalidValue) return MOE_ERR_INVALID_ARG;
+    } else {
+        err = launch_ffn_f32(static_cast<const float*>(x_perm), offsets,
+                             static_cast<const float*>(W1), static_cast<const float*>(W3),
+                             static_cast<const float*>(W2), P, d, h, E, at<float>(ws, L.H), Y,
+                             stream);
+    }
+    if ((st = finish(err, stream, status)) != MOE_OK) return st;
+    err = launch_combine(Y, inv_perm, w, T, d, dt, y, stream);
+    return finish(err, stream, status);
+}
+
+moe_status moe_device_status(void* ws, size_t ws_bytes, uint32_t* flags, cudaStream_t stream) {
+    if (!ws || !flags || ws_bytes < 256) return MOE_ERR_INVALID_ARG;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return MOE_ERR_CUDA;
+    uint32_t v = 0;
+    if (cudaMemcpy(&v, ws, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaMemset(ws, 0, 4) != cudaSuccess) return MOE_ERR_CUDA;
+    *flags = v;
+    return (v & MOE_DEV_FLAG_TIMEOUT) ? MOE_ERR_TIMEOUT : MOE_OK;
+}
+
+}  // extern "C"

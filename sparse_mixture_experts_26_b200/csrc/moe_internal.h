@@ -1,0 +1,80 @@
+// moe_internal.h -- host-side pieces shared by the libmoe translation units:
+// the workspace layout and the launchers of each kernel family.
+#pragma once
+
+#include <cuda_runtime_api.h>
+
+#include <cstddef>
+#include <cstdint>
+
+#include "../../include/moe.h"
+
+namespace moe {
+
+constexpr int kMaxExperts = 32;
+// Tokens handled by one block of the permutation count / rank kernels.
+constexpr int kPermChunk = 2048;
+
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+inline size_t dtype_bytes(moe_dtype dt) { return dt == MOE_BF16 ? 2 : 4; }
+
+// Byte offsets of every workspace region (1 KiB aligned).  The status word sits at
+// offset 0 so that every entry point sharing a workspace reports into one place.
+struct WsLayout {
+    size_t status, topk_idx, topk_w, offsets, blk_counts, blk_base, perm_token, inv_perm,
+        x_perm, H, Y, total;
+    // Bytes needed by moe_permute (status + count/base scratch) and by moe_expert_ffn
+    // (status + H); moe_layer_forward needs `total`.
+    size_t permute_need, ffn_need;
+};
+
+inline int perm_blocks(int T) { return (T + kPermChunk - 1) / kPermChunk; }
+
+inline WsLayout ws_layout(int T, int d, int h, int E, int k, moe_dtype dt) {
+    WsLayout L{};
+    const size_t P = static_cast<size_t>(T) * k;
+    const size_t nb = static_cast<size_t>(perm_blocks(T));
+    size_t o = 0;
+    auto take = [&](size_t bytes) {
+        size_t at = o;
+        o = align_up(o + bytes, 1024);
+        return at;
+    };
+    L.status = take(256);
+    L.blk_counts = take(nb * E * 4);
+    L.blk_base = take(nb * E * 4);
+    L.permute_need = o;
+    L.H = take(P * h * (dt == MOE_BF16 ? 2 : 4));
+    L.ffn_need = o;
+    L.topk_idx = take(P * 4);
+    L.topk_w = take(P * 4);
+    L.offsets = take((E + 1) * 4);
+    L.perm_token = take(P * 4);
+    L.inv_perm = take(P * 4);
+    L.x_perm = take(P * d * dtype_bytes(dt));
+    L.Y = take(P * d * 4);
+    L.total = o;
+    return L;
+}
+
+int device_sm_count();
+bool debug_sync_enabled();
+
+// ---- launchers (each returns cudaGetLastError() of its launch) ----
+cudaError_t launch_route(const void* x, const void* Wg, int T, int d, int E, moe_dtype dt,
+                         int32_t* idx, float* w, cudaStream_t s);
+cudaError_t launch_permute(const int32_t* idx, const void* x, int T, int d, int E, moe_dtype dt,
+                           int32_t* offsets, int32_t* perm_token, int32_t* inv_perm,
+                           void* x_perm, int32_t* blk_counts, int32_t* blk_base,
+                           uint32_t* status, cudaStream_t s);
+cudaError_t launch_ffn_f32(const float* x_perm, const int32_t* offsets, const float* W1,
+                           const float* W3, const float* W2, int rows, int d, int h, int E,
+                           float* H, float* Y, cudaStream_t s);
+// Returns cudaErrorInvalidValue if a tensor map cannot be encoded.
+cudaError_t launch_ffn_bf16(const void* x_perm, const int32_t* offsets, const void* W1,
+                            const void* W3, const void* W2, int rows, int d, int h, int E,
+                            void* H, float* Y, uint32_t* status, cudaStream_t s);
+cudaError_t launch_combine(const float* Y, const int32_t* inv_perm, const float* w, int T,
+                           int d, moe_dtype dt, void* y, cudaStream_t s);
+
+}  // namespace moe

@@ -1,0 +1,119 @@
+"""Host-side checks of the C ABI: the library loads, exports every symbol that
+include/moe.h declares, sizes its workspace, and rejects bad arguments before it
+touches the GPU (so these run without one)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe.h")
+
+OK, INVALID, UNSUPPORTED, WORKSPACE = 0, 1, 2, 3
+F32, BF16 = 0, 1
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from sparse_mixture_experts_26_b200.build import LIB, build
+    if not os.path.exists(LIB):
+        build()
+    L = ctypes.CDLL(LIB)
+    vp, i32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    L.moe_workspace_bytes.restype = sz
+    L.moe_workspace_bytes.argtypes = [i32] * 6
+    L.moe_route.argtypes = [vp, vp, i32, i32, i32, i32, i32, vp, vp, vp]
+    L.moe_permute.argtypes = [vp, vp, i32, i32, i32, i32, i32, vp, vp, vp, vp, vp, sz, vp]
+    L.moe_expert_ffn.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, vp, vp, sz, vp]
+    L.moe_combine.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp, vp]
+    L.moe_layer_forward.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, vp,
+                                    sz, vp]
+    L.moe_status_string.restype = ctypes.c_char_p
+    L.moe_status_string.argtypes = [i32]
+    return L
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("moe_route", "moe_permute", "moe_expert_ffn", "moe_combine",
+                     "moe_layer_forward", "moe_workspace_bytes", "moe_status_string"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_binding_exports_the_same_names():
+    import sparse_mixture_experts_26_b200 as m
+    for name in declared_functions():
+        assert callable(getattr(m, name)), name
+    assert set(m.EXPORTED_SYMBOLS) == set(declared_functions())
+
+
+def test_workspace_sizes(lib):
+    d, h = 4096, 14336
+    n16 = lib.moe_workspace_bytes(16, d, h, 8, 2, BF16)
+    n4k = lib.moe_workspace_bytes(4096, d, h, 8, 2, BF16)
+    assert 0 < n16 < n4k
+    P = 2 * 4096
+    # must hold at least x_perm (bf16), H (bf16) and the fp32 expert outputs
+    assert n4k >= P * d * 2 + P * h * 2 + P * d * 4
+    assert n4k % 1024 == 0
+    assert lib.moe_workspace_bytes(16, d, h, 8, 3, BF16) == 0      # k != 2
+    assert lib.moe_workspace_bytes(16, 4095, h, 8, 2, BF16) == 0   # d % 8
+    assert lib.moe_workspace_bytes(16, d, h, 33, 2, BF16) == 0     # E > 32
+    assert lib.moe_workspace_bytes(-1, d, h, 8, 2, BF16) == 0
+
+
+FAKE = 1 << 20  # 16-byte aligned, never dereferenced: validation fails first
+
+
+def test_route_validation(lib):
+    p = FAKE
+    assert lib.moe_route(None, p, 4, 64, 8, 2, BF16, p, p, None) == INVALID
+    assert lib.moe_route(p + 2, p, 4, 64, 8, 2, BF16, p, p, None) == INVALID  # misaligned
+    assert lib.moe_route(p, p, 4, 64, 8, 3, BF16, p, p, None) == UNSUPPORTED
+    assert lib.moe_route(p, p, 4, 60, 8, 2, BF16, p, p, None) == UNSUPPORTED
+    assert lib.moe_route(p, p, 4, 64, 1, 2, BF16, p, p, None) == UNSUPPORTED
+    assert lib.moe_route(p, p, -1, 64, 8, 2, BF16, p, p, None) == INVALID
+    assert lib.moe_route(p, p, 4, 64, 8, 2, 7, p, p, None) == INVALID
+    assert lib.moe_route(None, None, 0, 64, 8, 2, BF16, None, None, None) == OK  # T=0 no-op
+
+
+def test_layer_validation(lib):
+    p = FAKE
+    need = lib.moe_workspace_bytes(8, 64, 128, 8, 2, BF16)
+    assert lib.moe_layer_forward(p, p, p, p, p, 8, 64, 128, 8, 2, BF16, p, p, need - 1,
+                                 None) == WORKSPACE
+    assert lib.moe_layer_forward(p, p, p, p, None, 8, 64, 128, 8, 2, BF16, p, p, need,
+                                 None) == INVALID
+    assert lib.moe_layer_forward(p, p, p, p, p, 8, 64, 100, 8, 2, BF16, p, p, need,
+                                 None) == UNSUPPORTED
+    assert lib.moe_layer_forward(p, p, p, p, p, 0, 64, 128, 8, 2, BF16, p, p, 0, None) == OK
+
+
+def test_ffn_permute_combine_validation(lib):
+    p = FAKE
+    assert lib.moe_expert_ffn(p, p, p, p, p, 7, 64, 128, 8, BF16, p, p, 1 << 30,
+                              None) == INVALID  # odd row count
+    assert lib.moe_expert_ffn(p, p, p, p, p, 8, 64, 128, 8, BF16, p, p, 16, None) == WORKSPACE
+    assert lib.moe_permute(p, p, 8, 64, 8, 2, BF16, p, p, p, p, p, 0, None) == WORKSPACE
+    assert lib.moe_permute(p, p, 8, 64, 8, 2, BF16, None, p, p, p, p, 1 << 20,
+                           None) == INVALID
+    assert lib.moe_combine(p, p, p, 8, 64, 3, BF16, p, None) == UNSUPPORTED
+    assert lib.moe_combine(p, None, p, 8, 64, 2, BF16, p, None) == INVALID
+
+
+def test_status_strings(lib):
+    for code in range(6):
+        assert lib.moe_status_string(code)
+    assert b"unknown" in lib.moe_status_string(99)
