@@ -1,0 +1,438 @@
+#!/usr/bin/env python
+"""Benchmark of the Mixtral top-2 sparse-MoE layer on B200 through libmoe's C ABI.
+
+One step = one moe_layer_forward over one batch of the workload (router, grouping,
+expert SwiGLU FFN on tensor cores, combine).  Default workload: the decode batch of
+the Mixtral-8x7B layer (T=16, d=4096, h=14336, E=8, k=2, bf16), which streams every
+touched expert's weights from HBM; ``--workload prefill`` etc. select the others.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...     # the CPU oracle, timed on host cores
+
+Under torchrun (N > 1) every rank runs its own batch with replicated weights (tokens
+are independent, so the work shards with no collective in the data path); the step
+time is the max over ranks and ``value`` counts the tokens of all ranks.
+
+Printed: one JSON line (rank 0).  The expert weights (2.8 GB) are larger than L2 and
+are streamed every step, so no L2 flush is inserted between steps.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer tokens/s and % of roofline (bf16 TC peak prefill; HBM GB/s decode)"
+UNIT = "tokens/s"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+PROFILES = os.path.join(ROOT, "profiles")
+GEMM_SOURCE = os.path.join(ROOT, "sparse_mixture_experts_26_b200", "csrc",
+                           "grouped_gemm_sm100.cu")
+
+
+# ------------------------------------------------------------------ ranks
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def init_dist(backend: str):
+    import datetime
+
+    import torch.distributed as dist
+    rank, world, _ = dist_env()
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return rank, world
+
+
+def barrier(world: int, device=None):
+    if world > 1:
+        import torch.distributed as dist
+        if device is not None and dist.get_backend() == "nccl":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """Max of a per-rank float over all ranks (the slowest rank sets the step time)."""
+    if world == 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64,
+                     device=device if device is not None else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ peaks / profiles
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+def source_digest(path: str) -> str:
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def ncu_traffic(kernel_tag: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on the
+    current kernel source (``source_sha256_16`` line matches); else None."""
+    p = os.path.join(PROFILES, f"{kernel_tag}_{workload}.md")
+    if not os.path.exists(p):
+        return None
+    text = open(p).read()
+    m = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    h = re.search(r"source_sha256_16:\s*([0-9a-f]+)", text)
+    if not m or not h or h.group(1) != source_digest(GEMM_SOURCE):
+        return None
+    return float(m.group(1))
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while the GPU works."""
+
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
+        "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
+        "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
+    }
+
+    def __init__(self, device_index: int, period_s: float = 0.01):
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+            phys = device_index
+            if vis:
+                ids = [v.strip() for v in vis.split(",") if v.strip()]
+                if device_index < len(ids) and ids[device_index].isdigit():
+                    phys = int(ids[device_index])
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(phys)
+            self._nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._nv = None
+        self.period = period_s
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM)
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                self.samples.append(mhz)
+                for name, bit in self.REASONS.items():
+                    if r & bit and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self._nv is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._t is not None:
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------ oracle timing
+def oracle_tokens_per_s(inp_cpu, sample_tokens, budget_s: float):
+    """Time the CPU oracle (as it stands) on ``sample_tokens`` tokens of the workload,
+    repeating until ``budget_s`` seconds; returns (tokens/s, threads, repeats)."""
+    from oracle import moe_oracle as O
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max((p.get("num_threads", 1) for p in threadpool_info()
+                       if p.get("user_api") == "blas"), default=1)
+    except Exception:
+        threads = os.cpu_count() or 1
+    x = inp_cpu["x"][:sample_tokens]
+    t0 = time.perf_counter()
+    reps = 0
+    while True:
+        O.moe_layer(x, inp_cpu["Wg"], inp_cpu["W1"], inp_cpu["W3"], inp_cpu["W2"])
+        reps += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return reps * sample_tokens / dt, int(threads), reps, dt
+
+
+def cpu_copy(inp):
+    """Exact host copies of the inputs as float32 numpy arrays (bf16 widens exactly)."""
+    return {k: v.float().cpu().numpy() for k, v in inp.items()}
+
+
+# ------------------------------------------------------------------ workload config
+def workload_config(wl, extra=None):
+    cfg = {
+        "workload": f"{wl.name}: Mixtral-8x7B MoE layer, T={wl.T} d={wl.d} h={wl.h} "
+                    f"E={wl.E} top-{wl.k}, {wl.dtype}" if wl.d == 4096 else wl.note,
+        "T": wl.T, "d": wl.d, "h": wl.h, "E": wl.E, "k": wl.k, "seed": wl.seed,
+        "routing": wl.kind,
+        "l2": "no flush: inputs larger than L2 (2.8 GB of expert weights streamed per step)",
+    }
+    if extra:
+        cfg.update(extra)
+    return cfg
+
+
+def algorithmic_bytes_gemm1(wl, touched: int) -> int:
+    """W1 and W3 of every touched expert, the gathered rows read, H written."""
+    P = wl.T * wl.k
+    return touched * 2 * wl.h * wl.d * 2 + P * wl.d * 2 + P * wl.h * 2
+
+
+def algorithmic_flops_gemm1(wl) -> int:
+    return 2 * wl.T * wl.k * wl.d * 2 * wl.h
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args):
+    import numpy as np
+    import torch
+
+    import sparse_mixture_experts_26_b200 as moe
+    from workloads import WORKLOADS, make_inputs
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    init_dist("nccl")
+    wl = WORKLOADS[args.workload]
+    # each rank draws its own batch; weights are the same on every rank
+    inp = make_inputs(wl, device)
+    if world > 1 and rank > 0:
+        g = torch.Generator(device=device)
+        g.manual_seed(wl.seed * 1000 + rank)
+        inp["x"] = torch.randn(inp["x"].shape, generator=g, device=device).to(inp["x"].dtype)
+    x, Wg, W1, W3, W2 = (inp[k] for k in ("x", "Wg", "W1", "W3", "W2"))
+    T, d, h, E = wl.T, wl.d, wl.h, wl.E
+    ws = moe.alloc_workspace(T, d, h, E, wl.k, x.dtype, device)
+    y = torch.empty_like(x)
+    stream = torch.cuda.current_stream(device)
+
+    K, W = args.steps, args.warmup
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
+    for row in evs:  # create the underlying CUDA events before handing them over
+        for e in row:
+            e.record(stream)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    with ClockSampler(local) as clocks:
+        for _ in range(W):
+            moe.moe_layer_forward(x, Wg, W1, W3, W2, y, ws)
+        torch.cuda.synchronize()
+        barrier(world, device)
+        torch.cuda.synchronize()
+        start.record(stream)
+        for i in range(K):
+            moe.moe_layer_forward_events(x, Wg, W1, W3, W2, y, ws,
+                                         [e.cuda_event for e in evs[i]])
+        end.record(stream)
+        torch.cuda.synchronize()
+        barrier(world, device)
+    ms_local = start.elapsed_time(end) / K
+    flags = moe.moe_device_status(ws)
+    if flags:
+        raise RuntimeError(f"device status flags {flags:#x} after the timed region")
+    ms = max_over_ranks(ms_local, world, device)
+    value = world * T / (ms * 1e-3)
+
+    # per-stage averages (same timed region, same stream)
+    def stage(a, b):
+        return sum(evs[i][a].elapsed_time(evs[i][b]) for i in range(K)) / K
+    t_gemm1 = stage(1, 2)
+    t_gemm2 = stage(2, 3)
+    stages_ms = {"route+permute": stage(0, 1), "gemm1_swiglu": t_gemm1, "gemm2": t_gemm2,
+                 "combine": stage(3, 4)}
+
+    # routing statistics of this batch (for the algorithmic byte count)
+    idx = torch.empty(T, 2, dtype=torch.int32, device=device)
+    wts = torch.empty(T, 2, dtype=torch.float32, device=device)
+    moe.moe_route(x, Wg, idx, wts)
+    counts = torch.bincount(idx.flatten().long(), minlength=E).cpu().numpy()
+    touched = int((counts > 0).sum())
+
+    peaks, peak_src = load_peaks()
+    if wl.T <= 256:  # weight streaming: HBM-bound
+        bound, unit = "hbm", "GB/s"
+        ach = algorithmic_bytes_gemm1(wl, touched) / (t_gemm1 * 1e-3) / 1e9
+        peak = float(peaks["hbm_gbs"])
+        tag = "gemm1_swiglu"
+    else:
+        bound, unit = "tensor", "TFLOP/s"
+        ach = algorithmic_flops_gemm1(wl) / (t_gemm1 * 1e-3) / 1e12
+        peak = float(peaks["bf16_tflops"])
+        tag = "gemm1_swiglu"
+    traffic = ncu_traffic(tag, wl.name)
+    roofline = {"bound": bound, "achieved": round(ach, 1), "peak": peak, "unit": unit,
+                "frac": round(ach / peak, 4), "traffic": traffic,
+                "kernel": "grouped_gemm_kernel<SwiGLU> (GEMM1 + silu*gate epilogue)",
+                "peak_source": f"{peak_src} ({'burst' if bound == 'tensor' else 'copy'})"}
+    layer_bytes = touched * 3 * h * d * 2 + T * d * 2 * 2
+    layer = {"ms": round(ms, 4), "tflops": round(wl.active_flops() / (ms * 1e-3) / 1e12, 1),
+             "hbm_gbs": round(layer_bytes / (ms * 1e-3) / 1e9, 1),
+             "experts_touched": touched,
+             "stage_ms": {k: round(v, 4) for k, v in stages_ms.items()}}
+
+    # end to end: pinned host x -> device, layer, y -> pinned host, every step
+    x_host = x.cpu().pin_memory()
+    y_host = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+    x_dev = torch.empty_like(x)
+    for _ in range(2):
+        x_dev.copy_(x_host, non_blocking=True)
+        moe.moe_layer_forward(x_dev, Wg, W1, W3, W2, y, ws)
+        y_host.copy_(y, non_blocking=True)
+    torch.cuda.synchronize()
+    barrier(world, device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(K):
+        x_dev.copy_(x_host, non_blocking=True)
+        moe.moe_layer_forward(x_dev, Wg, W1, W3, W2, y, ws)
+        y_host.copy_(y, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world, device)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / K, world, device)
+    e2e = {"value": round(world * T / (e2e_ms * 1e-3), 1), "unit": UNIT,
+           "h2d_bytes_per_step": x.numel() * x.element_size(),
+           "d2h_bytes_per_step": y.numel() * y.element_size()}
+
+    cpu_baseline = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        inp_cpu = cpu_copy(inp)
+        n = min(T, args.cpu_sample_tokens)
+        tps, threads, reps, dt = oracle_tokens_per_s(inp_cpu, n, args.cpu_budget_s)
+        cpu_baseline = {"value": round(tps, 3), "unit": UNIT, "cores": threads,
+                        "kind": "oracle",
+                        "sample": f"fp64 numpy oracle on the first {n} tokens of the batch, "
+                                  f"{reps} repeat(s) in {dt:.1f} s"}
+
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    if rank != 0:
+        return None
+    return {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+        "steps": K, "warmup": W, "ms_per_step": round(ms, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype,
+        "data": "synthetic (seeded normal draws of the Mixtral-8x7B layer shapes; "
+                "random-init weights)",
+        "config": workload_config(wl, {"parallelism": f"replicas x{world} (tokens sharded, "
+                                                      "weights replicated)"}),
+        "roofline": roofline, "layer": layer, "cpu_baseline": cpu_baseline, "e2e": e2e,
+        "gpu_launches": moe.LAUNCHES_PER_LAYER * K,
+        "clocks": clocks.summary(),
+    }
+
+
+# ------------------------------------------------------------------ reference arm
+def run_reference(args):
+    """The CPU oracle as it stands, on host cores, on a bounded sample per step."""
+    import torch
+
+    from workloads import WORKLOADS, make_inputs
+
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return None
+    wl = WORKLOADS[args.workload]
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    inp_cpu = cpu_copy(make_inputs(wl, dev))
+    n = min(wl.T, args.cpu_sample_tokens)
+    from oracle import moe_oracle as O
+    x = inp_cpu["x"][:n]
+    for _ in range(args.warmup):
+        O.moe_layer(x, inp_cpu["Wg"], inp_cpu["W1"], inp_cpu["W3"], inp_cpu["W2"])
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        O.moe_layer(x, inp_cpu["Wg"], inp_cpu["W1"], inp_cpu["W3"], inp_cpu["W2"])
+    dt = time.perf_counter() - t0
+    ms = dt / args.steps * 1e3
+    value = n / (ms * 1e-3)
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max((p.get("num_threads", 1) for p in threadpool_info()
+                       if p.get("user_api") == "blas"), default=1)
+    except Exception:
+        threads = os.cpu_count() or 1
+    sample = f"fp64 numpy oracle on the first {n} of the batch's {wl.T} tokens per step"
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(wl),
+        "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": int(threads),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=None)
+    ap.add_argument("--warmup", type=int, default=None)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="decode",
+                    choices=["decode", "prefill", "skew", "long", "tiny_f32"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-sample-tokens", type=int, default=16)
+    ap.add_argument("--cpu-budget-s", type=float, default=10.0)
+    args = ap.parse_args(argv)
+    ref = args.impl == "reference"
+    if args.steps is None:
+        args.steps = 3 if ref else (200 if args.workload == "decode" else 20)
+    if args.warmup is None:
+        args.warmup = 1 if ref else 10
+    if not ref and args.warmup < 3:
+        args.warmup = 3
+    out = run_reference(args) if ref else run_ours(args)
+    if out is not None:
+        print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()

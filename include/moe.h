@@ -126,6 +126,18 @@ moe_status moe_layer_forward(const void *x, const void *Wg, const void *W1,
                              int E, int k, moe_dtype dt, void *y, void *ws,
                              size_t ws_bytes, cudaStream_t stream);
 
+/* moe_layer_forward that also records up to five caller-created events on `stream`
+ * between its stages, for timing them without a profiler:
+ *   events[0] before the router, events[1] after the permutation (before the
+ *   expert FFN), events[2] after the first FFN kernel (GEMM1 + SwiGLU), events[3]
+ *   after the second (GEMM2), events[4] after the combine.
+ * n_events may be 0..5; events beyond n_events are not recorded. */
+moe_status moe_layer_forward_events(const void *x, const void *Wg, const void *W1,
+                                    const void *W3, const void *W2, int T, int d, int h,
+                                    int E, int k, moe_dtype dt, void *y, void *ws,
+                                    size_t ws_bytes, cudaEvent_t *events, int n_events,
+                                    cudaStream_t stream);
+
 /* Synchronise `stream`, read the workspace status word into *flags (host
  * pointer; MOE_DEV_FLAG_* bits), then clear it.  Returns MOE_ERR_TIMEOUT if the
  * timeout flag was set, MOE_OK otherwise.  Diagnostic call: it synchronises. */

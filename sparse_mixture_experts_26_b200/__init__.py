@@ -21,7 +21,8 @@ import torch
 __all__ = [
     "LIB_PATH", "MoeError", "moe_workspace_bytes", "moe_route", "moe_permute",
     "moe_expert_ffn", "moe_combine", "moe_layer_forward", "moe_device_status",
-    "moe_status_string", "alloc_workspace", "layer_forward", "EXPORTED_SYMBOLS",
+    "moe_status_string", "moe_layer_forward_events", "alloc_workspace", "layer_forward",
+    "EXPORTED_SYMBOLS", "LAUNCHES_PER_LAYER",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe.so")
@@ -30,8 +31,11 @@ MOE_F32, MOE_BF16 = 0, 1
 _STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
                  3: "MOE_ERR_WORKSPACE", 4: "MOE_ERR_CUDA", 5: "MOE_ERR_TIMEOUT"}
 EXPORTED_SYMBOLS = ("moe_workspace_bytes", "moe_route", "moe_permute", "moe_expert_ffn",
-                    "moe_combine", "moe_layer_forward", "moe_device_status",
-                    "moe_status_string")
+                    "moe_combine", "moe_layer_forward", "moe_layer_forward_events",
+                    "moe_device_status", "moe_status_string")
+# Kernels one moe_layer_forward queues: router 1, permutation 4 (count, scan, rank,
+# gather), expert FFN 2 (GEMM1 + SwiGLU, GEMM2), combine 1.
+LAUNCHES_PER_LAYER = 8
 
 
 class MoeError(RuntimeError):
@@ -55,6 +59,8 @@ def _load() -> ctypes.CDLL:
         "moe_combine": (i32, [vp, vp, vp, i32, i32, i32, i32, vp, vp]),
         "moe_layer_forward": (i32, [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, vp,
                                     sz, vp]),
+        "moe_layer_forward_events": (i32, [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
+                                           vp, vp, sz, vp, i32, vp]),
         "moe_device_status": (i32, [vp, sz, u32p, vp]),
         "moe_status_string": (ctypes.c_char_p, [i32]),
     }
@@ -159,6 +165,19 @@ def moe_layer_forward(x, Wg, W1, W3, W2, y, ws, k: int = 2, stream=None) -> None
     _check("moe_layer_forward", _lib.moe_layer_forward(
         _ptr(x), _ptr(Wg), _ptr(W1), _ptr(W3), _ptr(W2), T, d, h, E, k, _dt(x), _ptr(y),
         _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def moe_layer_forward_events(x, Wg, W1, W3, W2, y, ws, events, k: int = 2,
+                             stream=None) -> None:
+    """``moe_layer_forward`` recording ``events`` (created, up to 5 handles) between stages."""
+    _dev(x, Wg, W1, W3, W2, y, ws)
+    T, d = x.shape
+    E, h, _ = W1.shape
+    handles = (ctypes.c_void_p * max(1, len(events)))(*[int(e) for e in events])
+    _check("moe_layer_forward_events", _lib.moe_layer_forward_events(
+        _ptr(x), _ptr(Wg), _ptr(W1), _ptr(W3), _ptr(W2), T, d, h, E, k, _dt(x), _ptr(y),
+        _ptr(ws), ws.numel() * ws.element_size(), ctypes.addressof(handles), len(events),
+        _stream(stream)))
 
 
 def moe_device_status(ws, stream=None) -> int:

@@ -84,7 +84,7 @@ __global__ void __launch_bounds__(kFfnThreads)
 
 cudaError_t launch_ffn_f32(const float* x_perm, const int32_t* offsets, const float* W1,
                            const float* W3, const float* W2, int rows, int d, int h, int E,
-                           float* H, float* Y, cudaStream_t s) {
+                           float* H, float* Y, cudaStream_t s, cudaEvent_t between) {
     const int warps = kFfnThreads / 32;
     const size_t cap = static_cast<size_t>(device_sm_count()) * 16;
     size_t b1 = (static_cast<size_t>(rows) * h + warps - 1) / warps;
@@ -93,6 +93,10 @@ cudaError_t launch_ffn_f32(const float* x_perm, const int32_t* offsets, const fl
     b2 = b2 > cap ? cap : (b2 < 1 ? 1 : b2);
     ffn1_f32_kernel<<<static_cast<unsigned>(b1), kFfnThreads, 0, s>>>(x_perm, offsets, W1, W3,
                                                                        rows, d, h, E, H);
+    if (between) {
+        cudaError_t err = cudaEventRecord(between, s);
+        if (err != cudaSuccess) return err;
+    }
     ffn2_f32_kernel<<<static_cast<unsigned>(b2), kFfnThreads, 0, s>>>(H, offsets, W2, rows, d,
                                                                        h, E, Y);
     return cudaGetLastError();

@@ -409,7 +409,8 @@ cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b0, const CUten
 
 cudaError_t launch_ffn_bf16(const void* x_perm, const int32_t* offsets, const void* W1,
                             const void* W3, const void* W2, int rows, int d, int h, int E,
-                            void* H, float* Y, uint32_t* status, cudaStream_t s) {
+                            void* H, float* Y, uint32_t* status, cudaStream_t s,
+                            cudaEvent_t between) {
     CUtensorMap mx, mw1, mw3, mh, mw2;
     if (!encode_bf16_2d(&mx, x_perm, rows, d, kBM) ||
         !encode_bf16_2d(&mw1, W1, static_cast<uint64_t>(E) * h, d, 128) ||
@@ -427,6 +428,7 @@ cudaError_t launch_ffn_bf16(const void* x_perm, const int32_t* offsets, const vo
     int grid1 = static_cast<int>(tiles1 < sms ? (tiles1 < 1 ? 1 : tiles1) : sms);
     cudaError_t err = launch_gemm<kEpiSwiGLU>(mx, mw1, mw3, g1, grid1, s, false);
     if (err != cudaSuccess) return err;
+    if (between && (err = cudaEventRecord(between, s)) != cudaSuccess) return err;
 
     GemmArgs g2{offsets, E, rows, h, d, d, (d + 255) / 256, Y, status};
     long long tiles2 = row_blocks * g2.n_tiles;

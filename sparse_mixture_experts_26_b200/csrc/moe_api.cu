@@ -167,11 +167,19 @@ moe_status moe_combine(const float* y_perm, const int32_t* inv_perm, const float
     return finish(launch_combine(y_perm, inv_perm, topk_w, T, d, dt, y, stream), stream, nullptr);
 }
 
-moe_status moe_layer_forward(const void* x, const void* Wg, const void* W1, const void* W3,
-                             const void* W2, int T, int d, int h, int E, int k, moe_dtype dt,
-                             void* y, void* ws, size_t ws_bytes, cudaStream_t stream) {
+}  // extern "C"
+
+namespace moe {
+namespace {
+
+// The layer, with optional events recorded between its stages (profiling).
+moe_status layer_forward_impl(const void* x, const void* Wg, const void* W1, const void* W3,
+                              const void* W2, int T, int d, int h, int E, int k, moe_dtype dt,
+                              void* y, void* ws, size_t ws_bytes, cudaEvent_t* ev, int n_ev,
+                              cudaStream_t stream) {
     moe_status st = check_shape(T, d, h, E, k, dt, true);
     if (st != MOE_OK) return st;
+    if (n_ev < 0 || (n_ev > 0 && ev == nullptr)) return MOE_ERR_INVALID_ARG;
     if (T == 0) return MOE_OK;
     if (!ptrs_ok({x, Wg, W1, W3, W2, y, ws})) return MOE_ERR_INVALID_ARG;
     const WsLayout L = ws_layout(T, d, h, E, k, dt);
@@ -185,26 +193,54 @@ moe_status moe_layer_forward(const void* x, const void* Wg, const void* W1, cons
     void* x_perm = at<void>(ws, L.x_perm);
     float* Y = at<float>(ws, L.Y);
     const int P = 2 * T;
+    auto mark = [&](int i) -> bool {
+        return i >= n_ev || cudaEventRecord(ev[i], stream) == cudaSuccess;
+    };
 
+    if (!mark(0)) return MOE_ERR_CUDA;
     cudaError_t err = launch_route(x, Wg, T, d, E, dt, idx, w, stream);
     if ((st = finish(err, stream, status)) != MOE_OK) return st;
     err = launch_permute(idx, x, T, d, E, dt, offsets, perm_token, inv_perm, x_perm,
                          at<int32_t>(ws, L.blk_counts), at<int32_t>(ws, L.blk_base), status,
                          stream);
     if ((st = finish(err, stream, status)) != MOE_OK) return st;
+    if (!mark(1)) return MOE_ERR_CUDA;
     if (dt == MOE_BF16) {
         err = launch_ffn_bf16(x_perm, offsets, W1, W3, W2, P, d, h, E, at<void>(ws, L.H), Y, status,
-                              stream);
+                              stream, n_ev > 2 ? ev[2] : nullptr);
         if (err == cudaErrorInvalidValue) return MOE_ERR_INVALID_ARG;
     } else {
         err = launch_ffn_f32(static_cast<const float*>(x_perm), offsets,
                              static_cast<const float*>(W1), static_cast<const float*>(W3),
                              static_cast<const float*>(W2), P, d, h, E, at<float>(ws, L.H), Y,
-                             stream);
+                             stream, n_ev > 2 ? ev[2] : nullptr);
     }
     if ((st = finish(err, stream, status)) != MOE_OK) return st;
+    if (!mark(3)) return MOE_ERR_CUDA;
     err = launch_combine(Y, inv_perm, w, T, d, dt, y, stream);
-    return finish(err, stream, status);
+    if ((st = finish(err, stream, status)) != MOE_OK) return st;
+    if (!mark(4)) return MOE_ERR_CUDA;
+    return MOE_OK;
+}
+
+}  // namespace
+}  // namespace moe
+
+extern "C" {
+
+moe_status moe_layer_forward(const void* x, const void* Wg, const void* W1, const void* W3,
+                             const void* W2, int T, int d, int h, int E, int k, moe_dtype dt,
+                             void* y, void* ws, size_t ws_bytes, cudaStream_t stream) {
+    return layer_forward_impl(x, Wg, W1, W3, W2, T, d, h, E, k, dt, y, ws, ws_bytes, nullptr, 0,
+                              stream);
+}
+
+moe_status moe_layer_forward_events(const void* x, const void* Wg, const void* W1,
+                                    const void* W3, const void* W2, int T, int d, int h, int E,
+                                    int k, moe_dtype dt, void* y, void* ws, size_t ws_bytes,
+                                    cudaEvent_t* events, int n_events, cudaStream_t stream) {
+    return layer_forward_impl(x, Wg, W1, W3, W2, T, d, h, E, k, dt, y, ws, ws_bytes, events,
+                              n_events, stream);
 }
 
 moe_status moe_device_status(void* ws, size_t ws_bytes, uint32_t* flags, cudaStream_t stream) {

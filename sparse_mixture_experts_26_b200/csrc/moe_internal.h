@@ -13,7 +13,7 @@ namespace moe {
 
 constexpr int kMaxExperts = 32;
 // Tokens handled by one block of the permutation count / rank kernels.
-constexpr int kPermChunk = 2048;
+constexpr int kPermChunk = 256;
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 inline size_t dtype_bytes(moe_dtype dt) { return dt == MOE_BF16 ? 2 : 4; }
@@ -69,11 +69,14 @@ cudaError_t launch_permute(const int32_t* idx, const void* x, int T, int d, int 
                            uint32_t* status, cudaStream_t s);
 cudaError_t launch_ffn_f32(const float* x_perm, const int32_t* offsets, const float* W1,
                            const float* W3, const float* W2, int rows, int d, int h, int E,
-                           float* H, float* Y, cudaStream_t s);
+                           float* H, float* Y, cudaStream_t s, cudaEvent_t between = nullptr);
 // Returns cudaErrorInvalidValue if a tensor map cannot be encoded.
 cudaError_t launch_ffn_bf16(const void* x_perm, const int32_t* offsets, const void* W1,
                             const void* W3, const void* W2, int rows, int d, int h, int E,
-                            void* H, float* Y, uint32_t* status, cudaStream_t s);
+                            void* H, float* Y, uint32_t* status, cudaStream_t s,
+                            cudaEvent_t between = nullptr);
+// `between` (optional) is recorded on `s` after the first FFN kernel (GEMM1 + SwiGLU)
+// and before the second (GEMM2).
 cudaError_t launch_combine(const float* Y, const int32_t* inv_perm, const float* w, int T,
                            int d, moe_dtype dt, void* y, cudaStream_t s);
 

@@ -3,12 +3,15 @@
 // crackai "Mixtral of Experts", "Top-2 Routing in Detail": gate_logits = x . W_gate;
 // notion notes "Mixtral of Experts", "Sparse gating", eq. G(x) = Softmax(TopK(x . W_g)).
 //
-// One warp per token.  Each lane reads 16-byte vectors of the token's row and
-// accumulates all E logits in fp64: a bf16 x bf16 (or fp32 x fp32) product is exact
-// in fp64, so the logits carry only the rounding of the fp64 sum and the top-2
-// choice does not depend on the reduction order except at ties closer than ~1e-16
-// relative.  W_g (d x E) is staged in shared memory once per block when it fits.
-// The kernel is bound by reading x once (2*d bytes per token).
+// A block takes kTokPerBlock tokens; its 8 warps split the model dimension d in
+// interleaved 32-element chunks, so lanes read consecutive W_g rows (conflict-free,
+// coalesced) and each converted weight row is reused for all tokens of the block.
+// Every logit is accumulated in fp64: a bf16 x bf16 (or fp32 x fp32) product is
+// exact in fp64, so the logits carry only the rounding of the fp64 sums and the
+// top-2 choice does not depend on the summation order except at ties closer than
+// ~1e-16 relative.  Warp partials are combined by a shuffle tree and then across
+// warps in a fixed order, so the result is deterministic.  The kernel reads x once
+// (2*d bytes per token); W_g (d*E elements) comes from L2 once per block.
 #include <cuda_bf16.h>
 
 #include <cfloat>
@@ -30,102 +33,113 @@ __device__ __forceinline__ double to_f64<__nv_bfloat16>(__nv_bfloat16 v) {
 }
 
 constexpr int kRouteThreads = 256;
+constexpr int kRouteWarps = kRouteThreads / 32;
+// Tokens per block: 4 for E <= 8 (32 fp64 accumulators per lane), 1 for E <= 32.
+template <int MAXE>
+constexpr int tok_per_block() { return MAXE <= 8 ? 4 : 1; }
 
-template <typename Tin, int MAXE, bool WG_IN_SMEM>
+// Load W_g row i (E entries) as fp64.
+template <typename Tin, int MAXE>
+__device__ __forceinline__ void load_wrow(const Tin* __restrict__ Wg, int i, int E,
+                                          double (&wv)[MAXE]) {
+    const Tin* row = Wg + static_cast<size_t>(i) * E;
+    if (MAXE == 8 && sizeof(Tin) == 2) {
+        if (E == 8) {
+            const uint4 u = __ldg(reinterpret_cast<const uint4*>(row));
+            const uint32_t q[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                wv[2 * j] = static_cast<double>(__uint_as_float(q[j] << 16));
+                wv[2 * j + 1] = static_cast<double>(__uint_as_float(q[j] & 0xffff0000u));
+            }
+            return;
+        }
+    }
+#pragma unroll
+    for (int e = 0; e < MAXE; ++e) wv[e] = e < E ? to_f64(row[e]) : 0.0;
+}
+
+template <typename Tin, int MAXE>
 __global__ void __launch_bounds__(kRouteThreads)
     route_kernel(const Tin* __restrict__ x, const Tin* __restrict__ Wg, int T, int d, int E,
                  int32_t* __restrict__ idx, float* __restrict__ w) {
-    extern __shared__ __align__(16) unsigned char route_smem[];
-    const Tin* wg = Wg;
-    if (WG_IN_SMEM) {
-        Tin* s = reinterpret_cast<Tin*>(route_smem);
-        const int n = d * E;
-        // 16-byte copies (d*E*sizeof(Tin) is a multiple of 16 since d % 8 == 0 and
-        // sizeof(Tin) * 8 >= 16).
-        const int nvec = n * static_cast<int>(sizeof(Tin)) / 16;
-        for (int i = threadIdx.x; i < nvec; i += blockDim.x)
-            reinterpret_cast<uint4*>(s)[i] = reinterpret_cast<const uint4*>(Wg)[i];
-        __syncthreads();
-        wg = s;
-    }
-    constexpr int V = 16 / sizeof(Tin);  // elements per 16-byte vector
-    const int lane = threadIdx.x & 31;
-    const int warps_per_block = blockDim.x >> 5;
-    const int gwarp = blockIdx.x * warps_per_block + (threadIdx.x >> 5);
-    const int nwarps = gridDim.x * warps_per_block;
+    constexpr int kTokPerBlock = tok_per_block<MAXE>();
+    __shared__ double part[kRouteWarps][kTokPerBlock][MAXE];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int t0 = blockIdx.x * kTokPerBlock;
+    const int ntok = min(kTokPerBlock, T - t0);
 
-    for (int t = gwarp; t < T; t += nwarps) {
-        double acc[MAXE];
+    double acc[kTokPerBlock][MAXE];
 #pragma unroll
-        for (int e = 0; e < MAXE; ++e) acc[e] = 0.0;
-        const Tin* xt = x + static_cast<size_t>(t) * d;
-        for (int i0 = lane * V; i0 < d; i0 += 32 * V) {
-            Tin xv[V];
-            *reinterpret_cast<uint4*>(xv) = *reinterpret_cast<const uint4*>(xt + i0);
+    for (int tb = 0; tb < kTokPerBlock; ++tb)
 #pragma unroll
-            for (int v = 0; v < V; ++v) {
-                const double xd = to_f64(xv[v]);
-                const Tin* row = wg + static_cast<size_t>(i0 + v) * E;
+        for (int e = 0; e < MAXE; ++e) acc[tb][e] = 0.0;
+
+    for (int i = warp * 32 + lane; i < d; i += kRouteThreads) {
+        double wv[MAXE];
+        load_wrow<Tin, MAXE>(Wg, i, E, wv);
 #pragma unroll
-                for (int e = 0; e < MAXE; ++e)
-                    if (e < E) acc[e] = fma(xd, to_f64(row[e]), acc[e]);
+        for (int tb = 0; tb < kTokPerBlock; ++tb) {
+            if (tb < ntok) {
+                const double xv = to_f64(x[static_cast<size_t>(t0 + tb) * d + i]);
+#pragma unroll
+                for (int e = 0; e < MAXE; ++e) acc[tb][e] = fma(xv, wv[e], acc[tb][e]);
             }
         }
+    }
+#pragma unroll
+    for (int tb = 0; tb < kTokPerBlock; ++tb)
 #pragma unroll
         for (int e = 0; e < MAXE; ++e) {
-            if (e < E) {
-                double s = acc[e];
+            double s = acc[tb][e];
 #pragma unroll
-                for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-                acc[e] = s;
+            for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+            if (lane == 0) part[warp][tb][e] = s;
+        }
+    __syncthreads();
+    if (threadIdx.x < ntok) {
+        const int tb = threadIdx.x;
+        double l[MAXE];
+#pragma unroll
+        for (int e = 0; e < MAXE; ++e) {
+            double s = 0.0;
+#pragma unroll
+            for (int wi = 0; wi < kRouteWarps; ++wi) s += part[wi][tb][e];
+            l[e] = s;
+        }
+        // (logit desc, index asc): strict comparisons keep the first maximum.
+        double b1 = l[0];
+        int i1 = 0;
+#pragma unroll
+        for (int e = 1; e < MAXE; ++e)
+            if (e < E && l[e] > b1) {
+                b1 = l[e];
+                i1 = e;
             }
-        }
-        if (lane == 0) {
-            // (logit desc, index asc): strict comparisons keep the first maximum.
-            double b1 = acc[0];
-            int i1 = 0;
+        double b2 = -DBL_MAX;
+        int i2 = -1;
 #pragma unroll
-            for (int e = 1; e < MAXE; ++e)
-                if (e < E && acc[e] > b1) {
-                    b1 = acc[e];
-                    i1 = e;
-                }
-            double b2 = -DBL_MAX;
-            int i2 = -1;
-#pragma unroll
-            for (int e = 0; e < MAXE; ++e)
-                if (e < E && e != i1 && (i2 < 0 || acc[e] > b2)) {
-                    b2 = acc[e];
-                    i2 = e;
-                }
-            const float w1 = static_cast<float>(1.0 / (1.0 + exp(b2 - b1)));
-            idx[2 * t] = i1;
-            idx[2 * t + 1] = i2;
-            w[2 * t] = w1;
-            w[2 * t + 1] = 1.0f - w1;  // exact (Sterbenz): the pair sums to 1 in float
-        }
+        for (int e = 0; e < MAXE; ++e)
+            if (e < E && e != i1 && (i2 < 0 || l[e] > b2)) {
+                b2 = l[e];
+                i2 = e;
+            }
+        const float w1 = static_cast<float>(1.0 / (1.0 + exp(b2 - b1)));
+        const int t = t0 + tb;
+        idx[2 * t] = i1;
+        idx[2 * t + 1] = i2;
+        w[2 * t] = w1;
+        w[2 * t + 1] = 1.0f - w1;  // exact (Sterbenz): the pair sums to 1 in float
     }
 }
 
 template <typename Tin, int MAXE>
 cudaError_t launch_route_t(const void* x, const void* Wg, int T, int d, int E, int32_t* idx,
                            float* w, cudaStream_t s) {
-    const size_t wg_bytes = static_cast<size_t>(d) * E * sizeof(Tin);
-    const int warps = kRouteThreads / 32;
-    int blocks = (T + warps - 1) / warps;
-    const int cap = device_sm_count() * 4;
-    if (blocks > cap) blocks = cap;
-    if (wg_bytes <= 64 * 1024) {
-        auto k = route_kernel<Tin, MAXE, true>;
-        if (wg_bytes > 48 * 1024)
-            cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(wg_bytes));
-        k<<<blocks, kRouteThreads, wg_bytes, s>>>(static_cast<const Tin*>(x),
-                                                   static_cast<const Tin*>(Wg), T, d, E, idx, w);
-    } else {
-        route_kernel<Tin, MAXE, false><<<blocks, kRouteThreads, 0, s>>>(
-            static_cast<const Tin*>(x), static_cast<const Tin*>(Wg), T, d, E, idx, w);
-    }
+    constexpr int tb = tok_per_block<MAXE>();
+    const int blocks = (T + tb - 1) / tb;
+    route_kernel<Tin, MAXE><<<blocks, kRouteThreads, 0, s>>>(
+        static_cast<const Tin*>(x), static_cast<const Tin*>(Wg), T, d, E, idx, w);
     return cudaGetLastError();
 }
 
