@@ -48,7 +48,7 @@ def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(
             f"{LIB_PATH} is missing; build it with "
-            "`python -m sparse_mixture_experts_26_b200.build` (nvcc, sm_100a)")
+            "`python sparse_mixture_experts_26_b200/build.py` (nvcc, sm_100a)")
     lib = ctypes.CDLL(LIB_PATH)
     vp, i32, sz, u32p = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_void_p
     sigs = {

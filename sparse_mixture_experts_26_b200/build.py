@@ -1,8 +1,10 @@
 """Build ``libmoe.so`` in-tree with nvcc for sm_100a.
 
-``python -m sparse_mixture_experts_26_b200.build`` (or ``build()``) compiles every
+``python sparse_mixture_experts_26_b200/build.py`` (or ``build()``) compiles every
 ``csrc/*.cu`` to an object under ``_build/`` and links the shared library next to
 this file, where the binding loads it.  nvcc cross-compiles, so no GPU is needed.
+Run it as a script (or load it by path): importing it as ``<package>.build`` would
+first import the package, which loads the very library this builds.
 """
 from __future__ import annotations
 

@@ -16,10 +16,12 @@ F32, BF16 = 0, 1
 
 @pytest.fixture(scope="module")
 def lib():
-    from sparse_mixture_experts_26_b200.build import LIB, build
-    if not os.path.exists(LIB):
-        build()
-    L = ctypes.CDLL(LIB)
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "_moe_build", os.path.join(ROOT, "sparse_mixture_experts_26_b200", "build.py"))
+    b = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(b)
+    L = ctypes.CDLL(b.build())
     vp, i32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
     L.moe_workspace_bytes.restype = sz
     L.moe_workspace_bytes.argtypes = [i32] * 6
@@ -52,7 +54,7 @@ def test_library_exports_every_declared_symbol(lib):
         assert hasattr(lib, name), name
 
 
-def test_binding_exports_the_same_names():
+def test_binding_exports_the_same_names(lib):
     import sparse_mixture_experts_26_b200 as m
     for name in declared_functions():
         assert callable(getattr(m, name)), name
