@@ -118,6 +118,30 @@ moe_status moe_combine(const float *y_perm, const int32_t *inv_perm,
                        const float *topk_w, int T, int d, int k, moe_dtype dt, void *y,
                        cudaStream_t stream);
 
+/* moe_expert_ffn for callers that cannot allocate device memory -- for example an
+ * op inside an inference engine that owns all device allocations and gives its
+ * ops no allocator, or a serving loop that must not allocate once it is running.
+ * It takes no workspace: its scratch (the SwiGLU activations H [rows, h] and a
+ * status word) lives in a library-owned __device__ array of
+ * MOE_STATIC_SCRATCH_BYTES bytes that every GPU loading the library keeps until
+ * the process exits.  No counterpart in the paper: it exists only for such callers.
+ *   Arguments, layouts and results are those of moe_expert_ffn, minus ws/ws_bytes.
+ *   Limit: rows * h * sizeof(dt) <= MOE_STATIC_SCRATCH_BYTES - 256, else
+ *   MOE_ERR_WORKSPACE is returned and nothing is queued (8 MiB: 292 grouped rows
+ *   of a bf16 Mixtral expert with h = 14336, i.e. up to 146 tokens).
+ *   The first call on a device, with that device current, looks up the array's
+ *   device address (cudaGetSymbolAddress) and caches it; make that first call
+ *   before any stream capture on the device.
+ *   All calls share the one array, which keeps the previous call's contents; each
+ *   call clears the status word itself.  Calls whose work overlaps on the GPU
+ *   (other streams, other threads) race on the array: serialise them.
+ *   Allocates nothing: no cudaMalloc, cudaFree or allocating library call. */
+#define MOE_STATIC_SCRATCH_BYTES ((size_t)8 << 20)
+moe_status moe_expert_ffn_static(const void *x_perm, const int32_t *offsets,
+                                 const void *W1, const void *W3, const void *W2, int rows,
+                                 int d, int h, int E, moe_dtype dt, float *y_perm,
+                                 cudaStream_t stream);
+
 /* The whole layer: route -> permute -> expert FFN -> combine, queued on `stream`
  * with no host synchronisation (group sizes stay on the device).
  *   x [T, d], Wg [d, E], W1/W3 [E, h, d], W2 [E, d, h] in dt;  y [T, d] out in dt. */

@@ -22,7 +22,7 @@ __all__ = [
     "LIB_PATH", "MoeError", "moe_workspace_bytes", "moe_route", "moe_permute",
     "moe_expert_ffn", "moe_combine", "moe_layer_forward", "moe_device_status",
     "moe_status_string", "moe_layer_forward_events", "alloc_workspace", "layer_forward",
-    "EXPORTED_SYMBOLS", "LAUNCHES_PER_LAYER",
+    "EXPORTED_SYMBOLS", "LAUNCHES_PER_LAYER", "moe_expert_ffn_static",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe.so")
@@ -32,7 +32,7 @@ _STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED"
                  3: "MOE_ERR_WORKSPACE", 4: "MOE_ERR_CUDA", 5: "MOE_ERR_TIMEOUT"}
 EXPORTED_SYMBOLS = ("moe_workspace_bytes", "moe_route", "moe_permute", "moe_expert_ffn",
                     "moe_combine", "moe_layer_forward", "moe_layer_forward_events",
-                    "moe_device_status", "moe_status_string")
+                    "moe_device_status", "moe_status_string", "moe_expert_ffn_static")
 # Kernels one moe_layer_forward queues: router 1, permutation 4 (count, scan, rank,
 # gather), expert FFN 2 (GEMM1 + SwiGLU, GEMM2), combine 1.
 LAUNCHES_PER_LAYER = 8
@@ -63,6 +63,7 @@ def _load() -> ctypes.CDLL:
                                            vp, vp, sz, vp, i32, vp]),
         "moe_device_status": (i32, [vp, sz, u32p, vp]),
         "moe_status_string": (ctypes.c_char_p, [i32]),
+        "moe_expert_ffn_static": (i32, [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, vp, vp]),
     }
     for name, (res, args) in sigs.items():
         f = getattr(lib, name)
@@ -188,6 +189,18 @@ def moe_device_status(ws, stream=None) -> int:
     if code not in (0, 5):
         _check("moe_device_status", code)
     return int(flags.value)
+
+
+def moe_expert_ffn_static(x_perm, offsets, W1, W3, W2, y_perm, stream=None) -> None:
+    """``moe_expert_ffn`` without a workspace, for callers that cannot allocate device
+    memory: the scratch is a fixed 8 MiB array inside the library (see include/moe.h
+    for the size limit, the first-call set-up and why overlapping calls race)."""
+    _dev(x_perm, offsets, W1, W3, W2, y_perm)
+    rows, d = x_perm.shape
+    E, h, _ = W1.shape
+    _check("moe_expert_ffn_static", _lib.moe_expert_ffn_static(
+        _ptr(x_perm), _ptr(offsets), _ptr(W1), _ptr(W3), _ptr(W2), rows, d, h, E, _dt(x_perm),
+        _ptr(y_perm), _stream(stream)))
 
 
 def layer_forward(x, Wg, W1, W3, W2, ws=None, out=None, stream=None) -> torch.Tensor:
