@@ -36,8 +36,15 @@ METRIC = "MoE-layer tokens/s and % of roofline (bf16 TC peak prefill; HBM GB/s d
 UNIT = "tokens/s"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 PROFILES = os.path.join(ROOT, "profiles")
-GEMM_SOURCE = os.path.join(ROOT, "sparse_mixture_experts_26_b200", "csrc",
-                           "grouped_gemm_sm100.cu")
+CSRC = os.path.join(ROOT, "sparse_mixture_experts_26_b200", "csrc")
+# Dominant kernel of each regime and the file that holds it.
+DOMINANT = {
+    "decode": ("decode_gemm_kernel<SwiGLU> (gate/up GEMM + silu*gate, weight streaming)",
+               "decode_gemm_swiglu", os.path.join(CSRC, "decode_gemm_sm100.cu")),
+    "grouped": ("grouped_gemm_kernel<SwiGLU> (GEMM1 + silu*gate epilogue)",
+                "grouped_gemm_swiglu", os.path.join(CSRC, "grouped_gemm_sm100.cu")),
+}
+DECODE_MAX_TOKENS = 64  # the library switches to the weight-streaming kernels here
 
 
 # ------------------------------------------------------------------ ranks
@@ -94,16 +101,16 @@ def source_digest(path: str) -> str:
         return hashlib.sha256(f.read()).hexdigest()[:16]
 
 
-def ncu_traffic(kernel_tag: str, workload: str):
+def ncu_traffic(kernel_tag: str, workload: str, source: str):
     """DRAM bytes per launch from a committed ncu summary, if it was taken on the
-    current kernel source (``source_sha256_16`` line matches); else None."""
+    current kernel source (its ``source_sha256_16`` line matches); else None."""
     p = os.path.join(PROFILES, f"{kernel_tag}_{workload}.md")
     if not os.path.exists(p):
         return None
     text = open(p).read()
     m = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
     h = re.search(r"source_sha256_16:\s*([0-9a-f]+)", text)
-    if not m or not h or h.group(1) != source_digest(GEMM_SOURCE):
+    if not m or not h or h.group(1) != source_digest(source):
         return None
     return float(m.group(1))
 
@@ -292,20 +299,19 @@ def run_ours(args):
     touched = int((counts > 0).sum())
 
     peaks, peak_src = load_peaks()
-    if wl.T <= 256:  # weight streaming: HBM-bound
+    regime = "decode" if wl.T <= DECODE_MAX_TOKENS else "grouped"
+    kname, tag, ksrc = DOMINANT[regime]
+    if regime == "decode":  # weight streaming: HBM-bound
         bound, unit = "hbm", "GB/s"
         ach = algorithmic_bytes_gemm1(wl, touched) / (t_gemm1 * 1e-3) / 1e9
         peak = float(peaks["hbm_gbs"])
-        tag = "gemm1_swiglu"
     else:
         bound, unit = "tensor", "TFLOP/s"
         ach = algorithmic_flops_gemm1(wl) / (t_gemm1 * 1e-3) / 1e12
         peak = float(peaks["bf16_tflops"])
-        tag = "gemm1_swiglu"
-    traffic = ncu_traffic(tag, wl.name)
+    traffic = ncu_traffic(tag, wl.name, ksrc)
     roofline = {"bound": bound, "achieved": round(ach, 1), "peak": peak, "unit": unit,
-                "frac": round(ach / peak, 4), "traffic": traffic,
-                "kernel": "grouped_gemm_kernel<SwiGLU> (GEMM1 + silu*gate epilogue)",
+                "frac": round(ach / peak, 4), "traffic": traffic, "kernel": kname,
                 "peak_source": f"{peak_src} ({'burst' if bound == 'tensor' else 'copy'})"}
     layer_bytes = touched * 3 * h * d * 2 + T * d * 2 * 2
     layer = {"ms": round(ms, 4), "tflops": round(wl.active_flops() / (ms * 1e-3) / 1e12, 1),

@@ -4,7 +4,9 @@
 // y = w_1 Expert_{i1}(x) + w_2 Expert_{i2}(x); notion notes "Mixtral of Experts",
 // "Implementation", eq. y.  Each output element is w0*Y[r0] + w1*Y[r1] evaluated in
 // fp32 (slot 0 first, one fused multiply-add for slot 1) and rounded once to the
-// output dtype.  Pure streaming: reads 2 fp32 rows, writes 1 row per token.
+// output dtype.  Pure streaming: reads 2 fp32 rows, writes 1 row per token.  When
+// the expert outputs arrive as split-K partial sums, each row is first summed over
+// the partials in a fixed order, so the result does not depend on scheduling.
 #include <cuda_bf16.h>
 
 #include "moe_internal.h"
@@ -26,10 +28,25 @@ __device__ __forceinline__ void store4(__nv_bfloat16* y, size_t i, float4 v) {
     reinterpret_cast<uint2*>(y)[i] = u;
 }
 
+// Row r of the in-order sum of nsplit arrays split_stride4 float4s apart.
+__device__ __forceinline__ float4 split_sum(const float4* __restrict__ Y, int nsplit,
+                                           size_t split_stride4, size_t at) {
+    float4 a = Y[at];
+    for (int i = 1; i < nsplit; ++i) {
+        const float4 b = Y[static_cast<size_t>(i) * split_stride4 + at];
+        a.x += b.x;
+        a.y += b.y;
+        a.z += b.z;
+        a.w += b.w;
+    }
+    return a;
+}
+
 template <typename Tout>
 __global__ void __launch_bounds__(kCombineThreads)
-    combine_kernel(const float4* __restrict__ Y, const int32_t* __restrict__ inv,
-                   const float* __restrict__ w, int T, int d4, Tout* __restrict__ y) {
+    combine_kernel(const float4* __restrict__ Y, int nsplit, size_t split_stride4,
+                   const int32_t* __restrict__ inv, const float* __restrict__ w, int T, int d4,
+                   Tout* __restrict__ y) {
     const size_t n = static_cast<size_t>(T) * d4;
     const unsigned P = 2u * static_cast<unsigned>(T);
     for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
@@ -41,8 +58,10 @@ __global__ void __launch_bounds__(kCombineThreads)
         const float w0 = w[2 * t], w1 = w[2 * t + 1];
         // inv_perm entries outside [0, 2T) would come from an invalid permutation;
         // they contribute nothing instead of reading out of bounds.
-        const float4 a = r0 < P ? Y[static_cast<size_t>(r0) * d4 + c] : make_float4(0, 0, 0, 0);
-        const float4 b = r1 < P ? Y[static_cast<size_t>(r1) * d4 + c] : make_float4(0, 0, 0, 0);
+        const float4 a = r0 < P ? split_sum(Y, nsplit, split_stride4, static_cast<size_t>(r0) * d4 + c)
+                                : make_float4(0, 0, 0, 0);
+        const float4 b = r1 < P ? split_sum(Y, nsplit, split_stride4, static_cast<size_t>(r1) * d4 + c)
+                                : make_float4(0, 0, 0, 0);
         float4 o;
         o.x = fmaf(w1, b.x, w0 * a.x);
         o.y = fmaf(w1, b.y, w0 * a.y);
@@ -52,23 +71,45 @@ __global__ void __launch_bounds__(kCombineThreads)
     }
 }
 
-}  // namespace
+__global__ void __launch_bounds__(kCombineThreads)
+    sum_splits_kernel(const float4* __restrict__ parts, int nsplit, size_t n4,
+                      float4* __restrict__ Y) {
+    for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n4;
+         i += static_cast<size_t>(gridDim.x) * blockDim.x)
+        Y[i] = split_sum(parts, nsplit, n4, i);
+}
 
-cudaError_t launch_combine(const float* Y, const int32_t* inv_perm, const float* w, int T,
-                           int d, moe_dtype dt, void* y, cudaStream_t s) {
-    const int d4 = d / 4;
-    const size_t n = static_cast<size_t>(T) * d4;
+unsigned grid_for(size_t n) {
     size_t blocks = (n + kCombineThreads - 1) / kCombineThreads;
     const size_t cap = static_cast<size_t>(device_sm_count()) * 8;
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
+    return static_cast<unsigned>(blocks);
+}
+
+}  // namespace
+
+cudaError_t launch_sum_splits(const float* parts, int nsplit, size_t n, float* Y,
+                              cudaStream_t s) {
+    const size_t n4 = n / 4;
+    sum_splits_kernel<<<grid_for(n4), kCombineThreads, 0, s>>>(
+        reinterpret_cast<const float4*>(parts), nsplit, n4, reinterpret_cast<float4*>(Y));
+    return cudaGetLastError();
+}
+
+cudaError_t launch_combine(const float* Y, int nsplit, size_t split_stride,
+                           const int32_t* inv_perm, const float* w, int T, int d, moe_dtype dt,
+                           void* y, cudaStream_t s) {
+    const int d4 = d / 4;
+    const unsigned blocks = grid_for(static_cast<size_t>(T) * d4);
     if (dt == MOE_BF16)
-        combine_kernel<__nv_bfloat16><<<static_cast<unsigned>(blocks), kCombineThreads, 0, s>>>(
-            reinterpret_cast<const float4*>(Y), inv_perm, w, T, d4,
+        combine_kernel<__nv_bfloat16><<<blocks, kCombineThreads, 0, s>>>(
+            reinterpret_cast<const float4*>(Y), nsplit, split_stride / 4, inv_perm, w, T, d4,
             static_cast<__nv_bfloat16*>(y));
     else
-        combine_kernel<float><<<static_cast<unsigned>(blocks), kCombineThreads, 0, s>>>(
-            reinterpret_cast<const float4*>(Y), inv_perm, w, T, d4, static_cast<float*>(y));
+        combine_kernel<float><<<blocks, kCombineThreads, 0, s>>>(
+            reinterpret_cast<const float4*>(Y), nsplit, split_stride / 4, inv_perm, w, T, d4,
+            static_cast<float*>(y));
     return cudaGetLastError();
 }
 

@@ -345,13 +345,39 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
+template <int EPI>
+cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
+                        const GemmArgs& args, int grid, cudaStream_t s, bool pdl) {
+    auto kern = grouped_gemm_kernel<EPI>;
+    static int configured[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && !configured[dev]) {
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+        configured[dev] = 1;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kern, a, b0, b1, args);
+}
+
+}  // namespace
+
 // ---------------------------------------------------------------- host side
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
                                    const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
-EncodeTiledFn get_encode_fn() {
+static EncodeTiledFn get_encode_fn() {
     static EncodeTiledFn fn = nullptr;
     static std::once_flag once;
     std::call_once(once, [] {
@@ -381,36 +407,33 @@ bool encode_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t 
            CUDA_SUCCESS;
 }
 
-template <int EPI>
-cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
-                        const GemmArgs& args, int grid, cudaStream_t s, bool pdl) {
-    auto kern = grouped_gemm_kernel<EPI>;
-    static int configured[64] = {0};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 64 && !configured[dev]) {
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-        configured[dev] = 1;
-    }
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = kSmemBytes;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = pdl ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, kern, a, b0, b1, args);
-}
-
-}  // namespace
 
 cudaError_t launch_ffn_bf16(const void* x_perm, const int32_t* offsets, const void* W1,
                             const void* W3, const void* W2, int rows, int d, int h, int E,
-                            void* H, float* Y, uint32_t* status, cudaStream_t s,
+                            void* H, float* Y, float* partials, int partial_cap, bool reduce,
+                            FfnOut* out, uint32_t* status, cudaStream_t s,
                             cudaEvent_t between) {
+    if (rows <= kDecodeMaxRows) {
+        // Largest split of the down projection's K blocks (at most partial_cap) that
+        // leaves no K range empty.
+        const int num_kb = (h + 63) / 64;
+        int ksplit = partials ? (partial_cap < kDecodeSplitK ? partial_cap : kDecodeSplitK) : 1;
+        while (ksplit > 1 && ((num_kb + ksplit - 1) / ksplit) * (ksplit - 1) >= num_kb) --ksplit;
+        if (ksplit < 1) ksplit = 1;
+        float* dst = ksplit > 1 ? partials : Y;
+        cudaError_t err = launch_ffn_bf16_decode(x_perm, offsets, W1, W3, W2, rows, d, h, E, H,
+                                                 dst, ksplit, status, s, between);
+        if (err != cudaSuccess) return err;
+        if (ksplit > 1 && reduce) {
+            err = launch_sum_splits(partials, ksplit, static_cast<size_t>(rows) * d, Y, s);
+            if (err != cudaSuccess) return err;
+            ksplit = 1;
+            dst = Y;
+        }
+        if (out) *out = FfnOut{dst, ksplit};
+        return cudaSuccess;
+    }
+    if (out) *out = FfnOut{Y, 1};
     CUtensorMap mx, mw1, mw3, mh, mw2;
     if (!encode_bf16_2d(&mx, x_perm, rows, d, kBM) ||
         !encode_bf16_2d(&mw1, W1, static_cast<uint64_t>(E) * h, d, 128) ||

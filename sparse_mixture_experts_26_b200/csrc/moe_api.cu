@@ -147,6 +147,7 @@ moe_status moe_expert_ffn(const void* x_perm, const int32_t* offsets, const void
     cudaError_t err;
     if (dt == MOE_BF16) {
         err = launch_ffn_bf16(x_perm, offsets, W1, W3, W2, rows, d, h, E, at<void>(ws, L.H), y_perm,
+                              at<float>(ws, L.Ypart), kDecodeSplitK, /*reduce=*/true, nullptr,
                               status, stream);
         if (err == cudaErrorInvalidValue) return MOE_ERR_INVALID_ARG;  // tensor map refused
     } else {
@@ -164,7 +165,8 @@ moe_status moe_combine(const float* y_perm, const int32_t* inv_perm, const float
     if (st != MOE_OK) return st;
     if (T == 0) return MOE_OK;
     if (!ptrs_ok({y_perm, inv_perm, topk_w, y})) return MOE_ERR_INVALID_ARG;
-    return finish(launch_combine(y_perm, inv_perm, topk_w, T, d, dt, y, stream), stream, nullptr);
+    return finish(launch_combine(y_perm, 1, 0, inv_perm, topk_w, T, d, dt, y, stream), stream,
+                  nullptr);
 }
 
 }  // extern "C"
@@ -205,9 +207,11 @@ moe_status layer_forward_impl(const void* x, const void* Wg, const void* W1, con
                          stream);
     if ((st = finish(err, stream, status)) != MOE_OK) return st;
     if (!mark(1)) return MOE_ERR_CUDA;
+    FfnOut fo{Y, 1};
     if (dt == MOE_BF16) {
-        err = launch_ffn_bf16(x_perm, offsets, W1, W3, W2, P, d, h, E, at<void>(ws, L.H), Y, status,
-                              stream, n_ev > 2 ? ev[2] : nullptr);
+        err = launch_ffn_bf16(x_perm, offsets, W1, W3, W2, P, d, h, E, at<void>(ws, L.H), Y,
+                              at<float>(ws, L.Ypart), kDecodeSplitK, /*reduce=*/false, &fo,
+                              status, stream, n_ev > 2 ? ev[2] : nullptr);
         if (err == cudaErrorInvalidValue) return MOE_ERR_INVALID_ARG;
     } else {
         err = launch_ffn_f32(static_cast<const float*>(x_perm), offsets,
@@ -217,7 +221,8 @@ moe_status layer_forward_impl(const void* x, const void* Wg, const void* W1, con
     }
     if ((st = finish(err, stream, status)) != MOE_OK) return st;
     if (!mark(3)) return MOE_ERR_CUDA;
-    err = launch_combine(Y, inv_perm, w, T, d, dt, y, stream);
+    err = launch_combine(fo.Y, fo.nsplit, static_cast<size_t>(P) * d, inv_perm, w, T, d, dt, y,
+                         stream);
     if ((st = finish(err, stream, status)) != MOE_OK) return st;
     if (!mark(4)) return MOE_ERR_CUDA;
     return MOE_OK;

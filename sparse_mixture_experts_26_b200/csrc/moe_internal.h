@@ -15,6 +15,11 @@ constexpr int kMaxExperts = 32;
 // Tokens handled by one block of the permutation count / rank kernels.
 constexpr int kPermChunk = 256;
 
+// Grouped rows at or below which the weight-streaming (swap-AB) expert FFN is used,
+// and how many K ranges its down projection is split into at most.
+constexpr int kDecodeMaxRows = 128;
+constexpr int kDecodeSplitK = 4;
+
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 inline size_t dtype_bytes(moe_dtype dt) { return dt == MOE_BF16 ? 2 : 4; }
 
@@ -22,7 +27,7 @@ inline size_t dtype_bytes(moe_dtype dt) { return dt == MOE_BF16 ? 2 : 4; }
 // offset 0 so that every entry point sharing a workspace reports into one place.
 struct WsLayout {
     size_t status, topk_idx, topk_w, offsets, blk_counts, blk_base, perm_token, inv_perm,
-        x_perm, H, Y, total;
+        x_perm, H, Ypart, Y, total;
     // Bytes needed by moe_permute (status + count/base scratch) and by moe_expert_ffn
     // (status + H); moe_layer_forward needs `total`.
     size_t permute_need, ffn_need;
@@ -45,6 +50,8 @@ inline WsLayout ws_layout(int T, int d, int h, int E, int k, moe_dtype dt) {
     L.blk_base = take(nb * E * 4);
     L.permute_need = o;
     L.H = take(P * h * (dt == MOE_BF16 ? 2 : 4));
+    // fp32 partial sums of the split-K down projection (small batches, bf16 only)
+    L.Ypart = take(dt == MOE_BF16 && P <= kDecodeMaxRows ? kDecodeSplitK * P * d * 4 : 0);
     L.ffn_need = o;
     L.topk_idx = take(P * 4);
     L.topk_w = take(P * 4);
@@ -70,14 +77,35 @@ cudaError_t launch_permute(const int32_t* idx, const void* x, int T, int d, int 
 cudaError_t launch_ffn_f32(const float* x_perm, const int32_t* offsets, const float* W1,
                            const float* W3, const float* W2, int rows, int d, int h, int E,
                            float* H, float* Y, cudaStream_t s, cudaEvent_t between = nullptr);
-// Returns cudaErrorInvalidValue if a tensor map cannot be encoded.
+// bf16 expert FFN.  The result is the sum of `out->nsplit` fp32 arrays [rows, d]
+// starting at `out->Y`, `rows * d` floats apart: Y itself (nsplit = 1), or -- when
+// the small-batch kernels run and `partials` has room for `partial_cap` of them --
+// the split-K partial sums in `partials`.  With reduce = true the partials are
+// summed (in order) into Y before returning, so Y always holds the result.
+// `between` (optional) is recorded on `s` after the first FFN kernel (GEMM1 +
+// SwiGLU) and before the second.  Returns cudaErrorInvalidValue if a tensor map
+// cannot be encoded.
+struct FfnOut {
+    const float* Y;
+    int nsplit;
+};
 cudaError_t launch_ffn_bf16(const void* x_perm, const int32_t* offsets, const void* W1,
                             const void* W3, const void* W2, int rows, int d, int h, int E,
-                            void* H, float* Y, uint32_t* status, cudaStream_t s,
+                            void* H, float* Y, float* partials, int partial_cap, bool reduce,
+                            FfnOut* out, uint32_t* status, cudaStream_t s,
                             cudaEvent_t between = nullptr);
-// `between` (optional) is recorded on `s` after the first FFN kernel (GEMM1 + SwiGLU)
-// and before the second (GEMM2).
-cudaError_t launch_combine(const float* Y, const int32_t* inv_perm, const float* w, int T,
-                           int d, moe_dtype dt, void* y, cudaStream_t s);
+// Small-batch expert FFN; the down projection writes `ksplit` partial arrays.
+cudaError_t launch_ffn_bf16_decode(const void* x_perm, const int32_t* offsets, const void* W1,
+                                   const void* W3, const void* W2, int rows, int d, int h, int E,
+                                   void* H, float* Yout, int ksplit, uint32_t* status,
+                                   cudaStream_t s, cudaEvent_t between);
+// y[t] = w0 * S(inv[t,0]) + w1 * S(inv[t,1]) with S(r) the in-order sum of the
+// nsplit arrays Y + i * split_stride at row r.
+cudaError_t launch_combine(const float* Y, int nsplit, size_t split_stride,
+                           const int32_t* inv_perm, const float* w, int T, int d, moe_dtype dt,
+                           void* y, cudaStream_t s);
+// Y[i] = sum over j < nsplit of parts[j * n + i] (in order), for i < n.
+cudaError_t launch_sum_splits(const float* parts, int nsplit, size_t n, float* Y,
+                              cudaStream_t s);
 
 }  // namespace moe

@@ -77,8 +77,8 @@ extern "C" moe_status moe_expert_ffn_static(const void* x_perm, const int32_t* o
 
     cudaError_t err;
     if (dt == MOE_BF16) {
-        err = launch_ffn_bf16(x_perm, offsets, W1, W3, W2, rows, d, h, E, H, y_perm, status,
-                              stream);
+        err = launch_ffn_bf16(x_perm, offsets, W1, W3, W2, rows, d, h, E, H, y_perm, nullptr, 0,
+                              /*reduce=*/true, nullptr, status, stream);
         if (err == cudaErrorInvalidValue) return MOE_ERR_INVALID_ARG;
     } else {
         err = launch_ffn_f32(static_cast<const float*>(x_perm), offsets,

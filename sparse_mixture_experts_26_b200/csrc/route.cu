@@ -3,7 +3,7 @@
 // crackai "Mixtral of Experts", "Top-2 Routing in Detail": gate_logits = x . W_gate;
 // notion notes "Mixtral of Experts", "Sparse gating", eq. G(x) = Softmax(TopK(x . W_g)).
 //
-// A block takes kTokPerBlock tokens; its 8 warps split the model dimension d in
+// A block takes TB tokens; its 8 warps split the model dimension d in
 // interleaved 32-element chunks, so lanes read consecutive W_g rows (conflict-free,
 // coalesced) and each converted weight row is reused for all tokens of the block.
 // Every logit is accumulated in fp64: a bf16 x bf16 (or fp32 x fp32) product is
@@ -34,61 +34,86 @@ __device__ __forceinline__ double to_f64<__nv_bfloat16>(__nv_bfloat16 v) {
 
 constexpr int kRouteThreads = 256;
 constexpr int kRouteWarps = kRouteThreads / 32;
-// Tokens per block: 4 for E <= 8 (32 fp64 accumulators per lane), 1 for E <= 32.
-template <int MAXE>
-constexpr int tok_per_block() { return MAXE <= 8 ? 4 : 1; }
+// Loads of kUnroll loop iterations are issued before any of them is used, so each
+// warp keeps several memory requests in flight instead of waiting on one at a time.
+constexpr int kUnroll = 4;
 
-// Load W_g row i (E entries) as fp64.
+__device__ __forceinline__ void widen_bf16x8(const uint4& u, double (&wv)[8]) {
+    const uint32_t q[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        wv[2 * j] = static_cast<double>(__uint_as_float(q[j] << 16));
+        wv[2 * j + 1] = static_cast<double>(__uint_as_float(q[j] & 0xffff0000u));
+    }
+}
+
+// W_g row i (E entries) as fp64, generic E.
 template <typename Tin, int MAXE>
 __device__ __forceinline__ void load_wrow(const Tin* __restrict__ Wg, int i, int E,
                                           double (&wv)[MAXE]) {
     const Tin* row = Wg + static_cast<size_t>(i) * E;
-    if (MAXE == 8 && sizeof(Tin) == 2) {
-        if (E == 8) {
-            const uint4 u = __ldg(reinterpret_cast<const uint4*>(row));
-            const uint32_t q[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                wv[2 * j] = static_cast<double>(__uint_as_float(q[j] << 16));
-                wv[2 * j + 1] = static_cast<double>(__uint_as_float(q[j] & 0xffff0000u));
-            }
-            return;
-        }
-    }
 #pragma unroll
     for (int e = 0; e < MAXE; ++e) wv[e] = e < E ? to_f64(row[e]) : 0.0;
 }
 
-template <typename Tin, int MAXE>
+// TB tokens per block; 8 warps split d in interleaved 32-element chunks.
+template <typename Tin, int MAXE, int TB>
 __global__ void __launch_bounds__(kRouteThreads)
     route_kernel(const Tin* __restrict__ x, const Tin* __restrict__ Wg, int T, int d, int E,
                  int32_t* __restrict__ idx, float* __restrict__ w) {
-    constexpr int kTokPerBlock = tok_per_block<MAXE>();
-    __shared__ double part[kRouteWarps][kTokPerBlock][MAXE];
+    __shared__ double part[kRouteWarps][TB][MAXE];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int t0 = blockIdx.x * kTokPerBlock;
-    const int ntok = min(kTokPerBlock, T - t0);
+    const int t0 = blockIdx.x * TB;
+    const int ntok = min(TB, T - t0);
 
-    double acc[kTokPerBlock][MAXE];
+    double acc[TB][MAXE];
 #pragma unroll
-    for (int tb = 0; tb < kTokPerBlock; ++tb)
+    for (int tb = 0; tb < TB; ++tb)
 #pragma unroll
         for (int e = 0; e < MAXE; ++e) acc[tb][e] = 0.0;
 
-    for (int i = warp * 32 + lane; i < d; i += kRouteThreads) {
-        double wv[MAXE];
-        load_wrow<Tin, MAXE>(Wg, i, E, wv);
+    // Fast path: bf16 with exactly 8 experts (one 16-byte W_g row per element).
+    constexpr bool kRow16 = (sizeof(Tin) == 2 && MAXE == 8);
+    const bool row16 = kRow16 && E == 8;
+    for (int i0 = warp * 32 + lane; i0 < d; i0 += kRouteThreads * kUnroll) {
+        uint4 wq[kUnroll];
+        Tin xv[kUnroll][TB];
 #pragma unroll
-        for (int tb = 0; tb < kTokPerBlock; ++tb) {
-            if (tb < ntok) {
-                const double xv = to_f64(x[static_cast<size_t>(t0 + tb) * d + i]);
+        for (int u = 0; u < kUnroll; ++u) {
+            const int i = i0 + u * kRouteThreads;
+            if (i < d) {
+                if (row16) wq[u] = __ldg(reinterpret_cast<const uint4*>(Wg) + i);
 #pragma unroll
-                for (int e = 0; e < MAXE; ++e) acc[tb][e] = fma(xv, wv[e], acc[tb][e]);
+                for (int tb = 0; tb < TB; ++tb)
+                    if (tb < ntok) xv[u][tb] = x[static_cast<size_t>(t0 + tb) * d + i];
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int i = i0 + u * kRouteThreads;
+            if (i < d) {
+                double wv[MAXE];
+                if constexpr (kRow16) {
+                    if (row16)
+                        widen_bf16x8(wq[u], reinterpret_cast<double(&)[8]>(wv));
+                    else
+                        load_wrow<Tin, MAXE>(Wg, i, E, wv);
+                } else {
+                    load_wrow<Tin, MAXE>(Wg, i, E, wv);
+                }
+#pragma unroll
+                for (int tb = 0; tb < TB; ++tb) {
+                    if (tb < ntok) {
+                        const double xd = to_f64(xv[u][tb]);
+#pragma unroll
+                        for (int e = 0; e < MAXE; ++e) acc[tb][e] = fma(xd, wv[e], acc[tb][e]);
+                    }
+                }
             }
         }
     }
 #pragma unroll
-    for (int tb = 0; tb < kTokPerBlock; ++tb)
+    for (int tb = 0; tb < TB; ++tb)
 #pragma unroll
         for (int e = 0; e < MAXE; ++e) {
             double s = acc[tb][e];
@@ -133,14 +158,23 @@ __global__ void __launch_bounds__(kRouteThreads)
     }
 }
 
+template <typename Tin, int MAXE, int TB>
+cudaError_t launch_route_tb(const void* x, const void* Wg, int T, int d, int E, int32_t* idx,
+                            float* w, cudaStream_t s) {
+    const int blocks = (T + TB - 1) / TB;
+    route_kernel<Tin, MAXE, TB><<<blocks, kRouteThreads, 0, s>>>(
+        static_cast<const Tin*>(x), static_cast<const Tin*>(Wg), T, d, E, idx, w);
+    return cudaGetLastError();
+}
+
+// Small batches: one token per block, so the work spreads over T SMs.  Large
+// batches: 4 tokens per block (each widened W_g row serves 4 tokens).  E > 8: one
+// token per block to bound the fp64 accumulators per thread.
 template <typename Tin, int MAXE>
 cudaError_t launch_route_t(const void* x, const void* Wg, int T, int d, int E, int32_t* idx,
                            float* w, cudaStream_t s) {
-    constexpr int tb = tok_per_block<MAXE>();
-    const int blocks = (T + tb - 1) / tb;
-    route_kernel<Tin, MAXE><<<blocks, kRouteThreads, 0, s>>>(
-        static_cast<const Tin*>(x), static_cast<const Tin*>(Wg), T, d, E, idx, w);
-    return cudaGetLastError();
+    if (MAXE > 8 || T <= 4 * 148) return launch_route_tb<Tin, MAXE, 1>(x, Wg, T, d, E, idx, w, s);
+    return launch_route_tb<Tin, MAXE, (MAXE > 8 ? 1 : 4)>(x, Wg, T, d, E, idx, w, s);
 }
 
 }  // namespace

@@ -101,8 +101,12 @@ def check_routing_and_permutation(g, x_cpu, Wg_cpu, E):
 
 
 SMALL = [  # (T, d, h, kind): ragged row blocks, K tails, N tails, empty groups
+    # T <= 64 runs the weight-streaming kernels (token tiles of 16, 32 or 64)
     (1, 64, 128, "plain"), (2, 64, 128, "plain"), (3, 128, 256, "plain"),
-    (17, 128, 256, "plain"), (129, 256, 512, "plain"), (300, 136, 200, "plain"),
+    (5, 136, 200, "plain"), (16, 256, 384, "skew"), (17, 128, 256, "plain"),
+    (33, 128, 256, "plain"), (64, 256, 512, "plain"),
+    # T > 64 runs the grouped GEMM (128-row blocks)
+    (65, 128, 256, "plain"), (129, 256, 512, "plain"), (300, 136, 200, "plain"),
     (1000, 512, 1024, "plain"), (700, 256, 384, "skew"), (513, 128, 256, "long"),
 ]
 
@@ -160,15 +164,16 @@ def test_empty_batch_is_a_noop():
     torch.cuda.synchronize()
 
 
-def test_exact_invariants_on_gpu():
+@pytest.mark.parametrize("T", [16, 257])  # weight-streaming and grouped-GEMM kernels
+def test_exact_invariants_on_gpu(T):
     """Bit-exact properties that need no oracle: W2 x 2 doubles y; permuting tokens
     permutes y; relabelling experts consistently leaves y unchanged."""
-    wl = small("inv", T=257, d=256, h=384, seed=77)
+    wl = small("inv", T=T, d=256, h=384, seed=77)
     inp = make_inputs(wl, "cuda")
     y = layer_y(inp)
     s = dict(inp, W2=inp["W2"] * 2)
     assert torch.equal(layer_y(s), y * 2)
-    p = torch.randperm(257, generator=torch.Generator().manual_seed(0)).cuda()
+    p = torch.randperm(T, generator=torch.Generator().manual_seed(0)).cuda()
     s = dict(inp, x=inp["x"][p].contiguous())
     assert torch.equal(layer_y(s), y[p])
     q = torch.tensor([3, 7, 0, 5, 1, 6, 2, 4], device="cuda")
