@@ -63,7 +63,8 @@ typedef enum {
 
 /* Bytes of workspace that moe_layer_forward needs for this shape (a 1 KiB-aligned
  * layout of routing results, permutation, gathered rows x_perm, the SwiGLU
- * activations H and the fp32 expert outputs).  It also covers moe_permute and
+ * activations H, the fp32 expert outputs and, for batches of at most 64 tokens, the
+ * fp32 partial sums of the split-K down projection).  It also covers moe_permute and
  * moe_expert_ffn.  Returns 0 for unsupported arguments. */
 size_t moe_workspace_bytes(int T, int d, int h, int E, int k, moe_dtype dt);
 
