@@ -367,7 +367,7 @@ def run_ours(args):
         "config": workload_config(wl, {"parallelism": f"replicas x{world} (tokens sharded, "
                                                       "weights replicated)"}),
         "roofline": roofline, "layer": layer, "cpu_baseline": cpu_baseline, "e2e": e2e,
-        "gpu_launches": moe.LAUNCHES_PER_LAYER * K,
+        "gpu_launches": moe.launches_per_layer(T) * K,
         "clocks": clocks.summary(),
     }
 

@@ -22,7 +22,7 @@ __all__ = [
     "LIB_PATH", "MoeError", "moe_workspace_bytes", "moe_route", "moe_permute",
     "moe_expert_ffn", "moe_combine", "moe_layer_forward", "moe_device_status",
     "moe_status_string", "moe_layer_forward_events", "alloc_workspace", "layer_forward",
-    "EXPORTED_SYMBOLS", "LAUNCHES_PER_LAYER", "moe_expert_ffn_static",
+    "EXPORTED_SYMBOLS", "launches_per_layer", "moe_expert_ffn_static",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe.so")
@@ -33,9 +33,10 @@ _STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED"
 EXPORTED_SYMBOLS = ("moe_workspace_bytes", "moe_route", "moe_permute", "moe_expert_ffn",
                     "moe_combine", "moe_layer_forward", "moe_layer_forward_events",
                     "moe_device_status", "moe_status_string", "moe_expert_ffn_static")
-# Kernels one moe_layer_forward queues: router 1, permutation 4 (count, scan, rank,
-# gather), expert FFN 2 (GEMM1 + SwiGLU, GEMM2), combine 1.
-LAUNCHES_PER_LAYER = 8
+def launches_per_layer(T: int) -> int:
+    """Kernels one moe_layer_forward queues: router 1, permutation 1 (T <= 512) or 4
+    (count, scan, rank, gather), expert FFN 2 (gate/up + SwiGLU, down), combine 1."""
+    return 1 + (1 if T <= 512 else 4) + 2 + 1
 
 
 class MoeError(RuntimeError):

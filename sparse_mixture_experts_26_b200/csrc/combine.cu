@@ -10,6 +10,7 @@
 #include <cuda_bf16.h>
 
 #include "moe_internal.h"
+#include "sm100_ptx.cuh"
 
 namespace moe {
 namespace {
@@ -47,6 +48,8 @@ __global__ void __launch_bounds__(kCombineThreads)
     combine_kernel(const float4* __restrict__ Y, int nsplit, size_t split_stride4,
                    const int32_t* __restrict__ inv, const float* __restrict__ w, int T, int d4,
                    Tout* __restrict__ y) {
+    pdl_wait();
+    pdl_launch_dependents();
     const size_t n = static_cast<size_t>(T) * d4;
     const unsigned P = 2u * static_cast<unsigned>(T);
     for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
@@ -74,6 +77,8 @@ __global__ void __launch_bounds__(kCombineThreads)
 __global__ void __launch_bounds__(kCombineThreads)
     sum_splits_kernel(const float4* __restrict__ parts, int nsplit, size_t n4,
                       float4* __restrict__ Y) {
+    pdl_wait();
+    pdl_launch_dependents();
     for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n4;
          i += static_cast<size_t>(gridDim.x) * blockDim.x)
         Y[i] = split_sum(parts, nsplit, n4, i);
@@ -92,9 +97,9 @@ unsigned grid_for(size_t n) {
 cudaError_t launch_sum_splits(const float* parts, int nsplit, size_t n, float* Y,
                               cudaStream_t s) {
     const size_t n4 = n / 4;
-    sum_splits_kernel<<<grid_for(n4), kCombineThreads, 0, s>>>(
-        reinterpret_cast<const float4*>(parts), nsplit, n4, reinterpret_cast<float4*>(Y));
-    return cudaGetLastError();
+    return launch_k(sum_splits_kernel, grid_for(n4), kCombineThreads, 0, s,
+                    reinterpret_cast<const float4*>(parts), nsplit, n4,
+                    reinterpret_cast<float4*>(Y));
 }
 
 cudaError_t launch_combine(const float* Y, int nsplit, size_t split_stride,
@@ -103,14 +108,12 @@ cudaError_t launch_combine(const float* Y, int nsplit, size_t split_stride,
     const int d4 = d / 4;
     const unsigned blocks = grid_for(static_cast<size_t>(T) * d4);
     if (dt == MOE_BF16)
-        combine_kernel<__nv_bfloat16><<<blocks, kCombineThreads, 0, s>>>(
-            reinterpret_cast<const float4*>(Y), nsplit, split_stride / 4, inv_perm, w, T, d4,
-            static_cast<__nv_bfloat16*>(y));
-    else
-        combine_kernel<float><<<blocks, kCombineThreads, 0, s>>>(
-            reinterpret_cast<const float4*>(Y), nsplit, split_stride / 4, inv_perm, w, T, d4,
-            static_cast<float*>(y));
-    return cudaGetLastError();
+        return launch_k(combine_kernel<__nv_bfloat16>, blocks, kCombineThreads, 0, s,
+                        reinterpret_cast<const float4*>(Y), nsplit, split_stride / 4, inv_perm,
+                        w, T, d4, static_cast<__nv_bfloat16*>(y));
+    return launch_k(combine_kernel<float>, blocks, kCombineThreads, 0, s,
+                    reinterpret_cast<const float4*>(Y), nsplit, split_stride / 4, inv_perm, w, T,
+                    d4, static_cast<float*>(y));
 }
 
 }  // namespace moe

@@ -190,6 +190,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 1) tmem_alloc(&bk.tmem_base, kTmemCols);
 
     pdl_wait();
+    pdl_launch_dependents();
     if (threadIdx.x == 0) {
         int prev = 0;
         for (int g = 0; g <= E; ++g) {
@@ -381,8 +382,7 @@ cudaError_t launch_decode(const CUtensorMap& w0, const CUtensorMap& w1, const CU
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
         configured[dev] = 1;
     }
-    kern<<<grid, kThreads, C::kSmem, s>>>(w0, w1, x, args);
-    return cudaGetLastError();
+    return launch_k(kern, grid, kThreads, C::kSmem, s, w0, w1, x, args);
 }
 
 template <int NT>

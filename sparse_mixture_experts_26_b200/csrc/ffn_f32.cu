@@ -8,6 +8,7 @@
 //   pass 2: Y[r, c] = H[r] . W2[e, c]
 // where e is the group that owns grouped row r.
 #include "moe_internal.h"
+#include "sm100_ptx.cuh"
 
 namespace moe {
 namespace {
@@ -30,6 +31,8 @@ __global__ void __launch_bounds__(kFfnThreads)
     ffn1_f32_kernel(const float* __restrict__ xp, const int32_t* __restrict__ offsets,
                     const float* __restrict__ W1, const float* __restrict__ W3, int rows, int d,
                     int h, int E, float* __restrict__ H) {
+    pdl_wait();
+    pdl_launch_dependents();
     __shared__ int s_off[kMaxExperts + 1];
     if (threadIdx.x <= E) s_off[threadIdx.x] = offsets[threadIdx.x];
     __syncthreads();
@@ -60,6 +63,8 @@ __global__ void __launch_bounds__(kFfnThreads)
     ffn2_f32_kernel(const float* __restrict__ H, const int32_t* __restrict__ offsets,
                     const float* __restrict__ W2, int rows, int d, int h, int E,
                     float* __restrict__ Y) {
+    pdl_wait();
+    pdl_launch_dependents();
     __shared__ int s_off[kMaxExperts + 1];
     if (threadIdx.x <= E) s_off[threadIdx.x] = offsets[threadIdx.x];
     __syncthreads();
@@ -91,15 +96,12 @@ cudaError_t launch_ffn_f32(const float* x_perm, const int32_t* offsets, const fl
     size_t b2 = (static_cast<size_t>(rows) * d + warps - 1) / warps;
     b1 = b1 > cap ? cap : (b1 < 1 ? 1 : b1);
     b2 = b2 > cap ? cap : (b2 < 1 ? 1 : b2);
-    ffn1_f32_kernel<<<static_cast<unsigned>(b1), kFfnThreads, 0, s>>>(x_perm, offsets, W1, W3,
-                                                                       rows, d, h, E, H);
-    if (between) {
-        cudaError_t err = cudaEventRecord(between, s);
-        if (err != cudaSuccess) return err;
-    }
-    ffn2_f32_kernel<<<static_cast<unsigned>(b2), kFfnThreads, 0, s>>>(H, offsets, W2, rows, d,
-                                                                       h, E, Y);
-    return cudaGetLastError();
+    cudaError_t err = launch_k(ffn1_f32_kernel, static_cast<unsigned>(b1), kFfnThreads, 0, s,
+                               x_perm, offsets, W1, W3, rows, d, h, E, H);
+    if (err != cudaSuccess) return err;
+    if (between && (err = cudaEventRecord(between, s)) != cudaSuccess) return err;
+    return launch_k(ffn2_f32_kernel, static_cast<unsigned>(b2), kFfnThreads, 0, s, H, offsets,
+                    W2, rows, d, h, E, Y);
 }
 
 }  // namespace moe

@@ -157,6 +157,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // The routing results come from the previous launch on the stream.
     pdl_wait();
+    pdl_launch_dependents();
     if (threadIdx.x == 0) {
         // Offsets are clamped to [0, rows] and made monotone so that nothing below
         // can address rows outside the buffers, whatever the device array holds.
@@ -347,7 +348,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <int EPI>
 cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
-                        const GemmArgs& args, int grid, cudaStream_t s, bool pdl) {
+                        const GemmArgs& args, int grid, cudaStream_t s) {
     auto kern = grouped_gemm_kernel<EPI>;
     static int configured[64] = {0};
     int dev = 0;
@@ -356,17 +357,7 @@ cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b0, const CUten
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
         configured[dev] = 1;
     }
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = kSmemBytes;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = pdl ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, kern, a, b0, b1, args);
+    return launch_k(kern, grid, kThreads, kSmemBytes, s, a, b0, b1, args);
 }
 
 }  // namespace
@@ -449,14 +440,14 @@ cudaError_t launch_ffn_bf16(const void* x_perm, const int32_t* offsets, const vo
     GemmArgs g1{offsets, E, rows, d, h, h, (h + 127) / 128, H, status};
     long long tiles1 = row_blocks * g1.n_tiles;
     int grid1 = static_cast<int>(tiles1 < sms ? (tiles1 < 1 ? 1 : tiles1) : sms);
-    cudaError_t err = launch_gemm<kEpiSwiGLU>(mx, mw1, mw3, g1, grid1, s, false);
+    cudaError_t err = launch_gemm<kEpiSwiGLU>(mx, mw1, mw3, g1, grid1, s);
     if (err != cudaSuccess) return err;
     if (between && (err = cudaEventRecord(between, s)) != cudaSuccess) return err;
 
     GemmArgs g2{offsets, E, rows, h, d, d, (d + 255) / 256, Y, status};
     long long tiles2 = row_blocks * g2.n_tiles;
     int grid2 = static_cast<int>(tiles2 < sms ? (tiles2 < 1 ? 1 : tiles2) : sms);
-    return launch_gemm<kEpiStoreF32>(mh, mw2, mw2, g2, grid2, s, false);
+    return launch_gemm<kEpiStoreF32>(mh, mw2, mw2, g2, grid2, s);
 }
 
 }  // namespace moe

@@ -26,6 +26,24 @@ int device_sm_count() {
     return n;
 }
 
+namespace {
+thread_local bool t_pdl_scope = false;
+bool pdl_allowed() {
+    static int v = -1;
+    if (v < 0) {
+        const char* e = std::getenv("MOE_NO_PDL");
+        v = (e && e[0] == '1') ? 0 : 1;
+    }
+    return v == 1;
+}
+// Small batches: every kernel is short, so overlapping launches pays off.
+bool small_batch(int T) { return T <= 64; }
+}  // namespace
+
+bool pdl_enabled() { return t_pdl_scope && pdl_allowed(); }
+PdlScope::PdlScope(bool on) : prev(t_pdl_scope) { t_pdl_scope = on; }
+PdlScope::~PdlScope() { t_pdl_scope = prev; }
+
 bool debug_sync_enabled() {
     static int v = -1;
     if (v < 0) {
@@ -106,6 +124,7 @@ moe_status moe_route(const void* x, const void* Wg, int T, int d, int E, int k, 
     if (st != MOE_OK) return st;
     if (T == 0) return MOE_OK;
     if (!ptrs_ok({x, Wg, topk_idx, topk_w})) return MOE_ERR_INVALID_ARG;
+    PdlScope pdl(small_batch(T));
     return finish(launch_route(x, Wg, T, d, E, dt, topk_idx, topk_w, stream), stream, nullptr);
 }
 
@@ -125,6 +144,7 @@ moe_status moe_permute(const int32_t* topk_idx, const void* x, int T, int d, int
     }
     if (!ptrs_ok({topk_idx, x, perm_token, inv_perm, x_perm})) return MOE_ERR_INVALID_ARG;
     uint32_t* status = at<uint32_t>(ws, L.status);
+    PdlScope pdl(small_batch(T));
     return finish(launch_permute(topk_idx, x, T, d, E, dt, offsets, perm_token, inv_perm, x_perm,
                                  at<int32_t>(ws, L.blk_counts), at<int32_t>(ws, L.blk_base),
                                  status, stream),
@@ -144,6 +164,7 @@ moe_status moe_expert_ffn(const void* x_perm, const int32_t* offsets, const void
     const WsLayout L = ws_layout(T, d, h, E, 2, dt);
     if (ws_bytes < L.ffn_need) return MOE_ERR_WORKSPACE;
     uint32_t* status = at<uint32_t>(ws, L.status);
+    PdlScope pdl(small_batch(T));
     cudaError_t err;
     if (dt == MOE_BF16) {
         err = launch_ffn_bf16(x_perm, offsets, W1, W3, W2, rows, d, h, E, at<void>(ws, L.H), y_perm,
@@ -165,6 +186,7 @@ moe_status moe_combine(const float* y_perm, const int32_t* inv_perm, const float
     if (st != MOE_OK) return st;
     if (T == 0) return MOE_OK;
     if (!ptrs_ok({y_perm, inv_perm, topk_w, y})) return MOE_ERR_INVALID_ARG;
+    PdlScope pdl(small_batch(T));
     return finish(launch_combine(y_perm, 1, 0, inv_perm, topk_w, T, d, dt, y, stream), stream,
                   nullptr);
 }
@@ -195,6 +217,7 @@ moe_status layer_forward_impl(const void* x, const void* Wg, const void* W1, con
     void* x_perm = at<void>(ws, L.x_perm);
     float* Y = at<float>(ws, L.Y);
     const int P = 2 * T;
+    PdlScope pdl(small_batch(T));
     auto mark = [&](int i) -> bool {
         return i >= n_ev || cudaEventRecord(ev[i], stream) == cudaSuccess;
     };

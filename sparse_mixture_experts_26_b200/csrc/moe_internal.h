@@ -2,10 +2,11 @@
 // the workspace layout and the launchers of each kernel family.
 #pragma once
 
-#include <cuda_runtime_api.h>
+#include <cuda_runtime.h>
 
 #include <cstddef>
 #include <cstdint>
+#include <utility>
 
 #include "../../include/moe.h"
 
@@ -66,6 +67,36 @@ inline WsLayout ws_layout(int T, int d, int h, int E, int k, moe_dtype dt) {
 
 int device_sm_count();
 bool debug_sync_enabled();
+// Programmatic dependent launch: used for the launches made inside a PdlScope(true)
+// (the entry points open one for small batches, where launch gaps matter and every
+// kernel is short), never when MOE_NO_PDL=1.  Measured: on T=16 it saves ~2% of the
+// layer; on T=4096 early-resident dependents cost ~3%, so large batches do not use it.
+bool pdl_enabled();
+struct PdlScope {
+    explicit PdlScope(bool on);
+    ~PdlScope();
+    bool prev;
+};
+
+// Launch `kern` on `s` with programmatic stream serialisation: the kernel may be
+// scheduled while the previous kernel on the stream is finishing, and every libmoe
+// kernel calls griddepcontrol.wait before it reads anything a previous kernel wrote.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                     Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl_enabled() ? 1 : 0;
+    cudaError_t err = cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+    return err != cudaSuccess ? err : cudaGetLastError();
+}
 
 // ---- launchers (each returns cudaGetLastError() of its launch) ----
 cudaError_t launch_route(const void* x, const void* Wg, int T, int d, int E, moe_dtype dt,

@@ -17,6 +17,7 @@
 #include <cfloat>
 
 #include "moe_internal.h"
+#include "sm100_ptx.cuh"
 
 namespace moe {
 namespace {
@@ -62,6 +63,8 @@ __global__ void __launch_bounds__(kRouteThreads)
     route_kernel(const Tin* __restrict__ x, const Tin* __restrict__ Wg, int T, int d, int E,
                  int32_t* __restrict__ idx, float* __restrict__ w) {
     __shared__ double part[kRouteWarps][TB][MAXE];
+    pdl_wait();
+    pdl_launch_dependents();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int t0 = blockIdx.x * TB;
     const int ntok = min(TB, T - t0);
@@ -162,19 +165,149 @@ template <typename Tin, int MAXE, int TB>
 cudaError_t launch_route_tb(const void* x, const void* Wg, int T, int d, int E, int32_t* idx,
                             float* w, cudaStream_t s) {
     const int blocks = (T + TB - 1) / TB;
-    route_kernel<Tin, MAXE, TB><<<blocks, kRouteThreads, 0, s>>>(
-        static_cast<const Tin*>(x), static_cast<const Tin*>(Wg), T, d, E, idx, w);
-    return cudaGetLastError();
+    return launch_k(route_kernel<Tin, MAXE, TB>, blocks, kRouteThreads, 0, s,
+                    static_cast<const Tin*>(x), static_cast<const Tin*>(Wg), T, d, E, idx, w);
 }
 
-// Small batches: one token per block, so the work spreads over T SMs.  Large
-// batches: 4 tokens per block (each widened W_g row serves 4 tokens).  E > 8: one
-// token per block to bound the fp64 accumulators per thread.
+// Large bf16 batches, E <= 8, d % 32 == 0: fp64 tensor-core MMA.
+// mma.sync m8n8k4 .f64 computes D[8x8] += A[8x4] B[4x8] in fp64, so a warp turns 8
+// tokens x 8 experts x 4 elements of the dot products into one instruction; every
+// widened x value feeds 8 FMAs and every widened W_g value 8 tokens.  Lane (g, q)
+// (g = lane/4, q = lane%4) supplies x[token g][8q + s] and W_g[8q + s][expert g] at
+// step s of a 32-element K block (the K order inside the block is permuted
+// consistently in A and B, which leaves the dot product unchanged), loading each as
+// one 16-byte vector.  W_g is staged once per persistent block, transposed to
+// [expert][d] in shared memory (64 KiB at d = 4096).  A block is 8 warps = 2 groups
+// of 8 tokens x 4 K quarters; the quarters' partial logits are added in a fixed
+// order, so results are deterministic.
+constexpr int kMmaGroupsPerBlock = 2;
+constexpr int kMmaKSplit = kRouteWarps / kMmaGroupsPerBlock;  // 4
+
+__device__ __forceinline__ void dmma_8x8x4(double& d0, double& d1, double a, double b) {
+    asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0,%1}, {%2}, {%3}, {%0,%1};"
+                 : "+d"(d0), "+d"(d1)
+                 : "d"(a), "d"(b));
+}
+
+__device__ __forceinline__ double bf16_lo(uint32_t u) { return __uint_as_float(u << 16); }
+__device__ __forceinline__ double bf16_hi(uint32_t u) { return __uint_as_float(u & 0xffff0000u); }
+
+__global__ void __launch_bounds__(kRouteThreads)
+    route_dmma_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ Wg,
+                      int T, int d, int E, int32_t* __restrict__ idx, float* __restrict__ w) {
+    extern __shared__ __align__(16) unsigned char route_smem[];
+    __nv_bfloat16* wgT = reinterpret_cast<__nv_bfloat16*>(route_smem);  // [8][d]
+    __shared__ double part[kRouteWarps][32][2];
+    pdl_wait();
+    pdl_launch_dependents();
+    for (int r = threadIdx.x; r < d; r += blockDim.x) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+            wgT[e * d + r] = e < E ? Wg[static_cast<size_t>(r) * E + e] : __float2bfloat16(0.f);
+    }
+    __syncthreads();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 2, q = lane & 3;
+    const int grp_in_block = warp / kMmaKSplit, ks = warp % kMmaKSplit;
+    const int kq = d / kMmaKSplit;                 // multiple of 8 (d % 32 == 0)
+    const int k_begin = ks * kq, k_end = k_begin + kq;
+    const int ngroups = (T + 7) / 8;
+    const uint4* wrow = reinterpret_cast<const uint4*>(wgT + g * d);
+    for (int grp0 = blockIdx.x * kMmaGroupsPerBlock; grp0 < ngroups;
+         grp0 += gridDim.x * kMmaGroupsPerBlock) {
+        const int grp = grp0 + grp_in_block;
+        const int t = grp * 8 + g;
+        const bool valid = grp < ngroups && t < T;
+        const uint4* xrow = reinterpret_cast<const uint4*>(x + static_cast<size_t>(valid ? t : 0) * d);
+        double c0 = 0.0, c1 = 0.0;
+        for (int k0 = k_begin; k0 < k_end; k0 += 32 * kUnroll) {
+            uint4 xv[kUnroll], wv[kUnroll];
+#pragma unroll
+            for (int u = 0; u < kUnroll; ++u) {
+                const int kk = k0 + u * 32 + 8 * q;
+                const bool in = kk < k_end;
+                xv[u] = (valid && in) ? __ldg(xrow + kk / 8) : make_uint4(0, 0, 0, 0);
+                wv[u] = in ? wrow[kk / 8] : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int u = 0; u < kUnroll; ++u) {
+                const uint32_t xa[4] = {xv[u].x, xv[u].y, xv[u].z, xv[u].w};
+                const uint32_t wa[4] = {wv[u].x, wv[u].y, wv[u].z, wv[u].w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    dmma_8x8x4(c0, c1, bf16_lo(xa[j]), bf16_lo(wa[j]));
+                    dmma_8x8x4(c0, c1, bf16_hi(xa[j]), bf16_hi(wa[j]));
+                }
+            }
+        }
+        // lane (g, q) holds logits of token g for experts 2q and 2q+1 (partial over ks)
+        part[warp][lane][0] = c0;
+        part[warp][lane][1] = c1;
+        __syncthreads();
+        if (ks == 0) {  // warp-uniform: all 32 lanes take part in the shuffles
+            double v0 = 0.0, v1 = 0.0;
+#pragma unroll
+            for (int s2 = 0; s2 < kMmaKSplit; ++s2) {
+                v0 += part[warp + s2][lane][0];
+                v1 += part[warp + s2][lane][1];
+            }
+            double l[8];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                l[2 * j] = __shfl_sync(0xffffffffu, v0, (lane & ~3) + j, 32);
+                l[2 * j + 1] = __shfl_sync(0xffffffffu, v1, (lane & ~3) + j, 32);
+            }
+            if (q == 0 && valid) {
+                double b1 = l[0];
+                int i1 = 0;
+#pragma unroll
+                for (int e = 1; e < 8; ++e)
+                    if (e < E && l[e] > b1) {
+                        b1 = l[e];
+                        i1 = e;
+                    }
+                double b2 = -DBL_MAX;
+                int i2 = -1;
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    if (e < E && e != i1 && (i2 < 0 || l[e] > b2)) {
+                        b2 = l[e];
+                        i2 = e;
+                    }
+                const float w1 = static_cast<float>(1.0 / (1.0 + exp(b2 - b1)));
+                idx[2 * t] = i1;
+                idx[2 * t + 1] = i2;
+                w[2 * t] = w1;
+                w[2 * t + 1] = 1.0f - w1;
+            }
+        }
+        __syncthreads();
+    }
+}
+
+// Small batches: one token per block, so the work spreads over T SMs.  Large bf16
+// batches (E <= 8, d % 32 == 0, W_g fits shared memory): the fp64 tensor-core kernel
+// above.  Otherwise: one token per block.
 template <typename Tin, int MAXE>
 cudaError_t launch_route_t(const void* x, const void* Wg, int T, int d, int E, int32_t* idx,
                            float* w, cudaStream_t s) {
-    if (MAXE > 8 || T <= 4 * 148) return launch_route_tb<Tin, MAXE, 1>(x, Wg, T, d, E, idx, w, s);
-    return launch_route_tb<Tin, MAXE, (MAXE > 8 ? 1 : 4)>(x, Wg, T, d, E, idx, w, s);
+    const size_t wgt_bytes = static_cast<size_t>(8) * d * 2;
+    if (sizeof(Tin) == 2 && MAXE == 8 && T > 64 && d % 32 == 0 && wgt_bytes <= 96 * 1024) {
+        auto kern = route_dmma_kernel;
+        static int configured[64] = {0};
+        int dev = 0;
+        cudaGetDevice(&dev);
+        if (dev < 64 && !configured[dev]) {
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 96 * 1024);
+            configured[dev] = 1;
+        }
+        const int blocks_needed = ((T + 7) / 8 + kMmaGroupsPerBlock - 1) / kMmaGroupsPerBlock;
+        const int cap = 3 * device_sm_count();
+        return launch_k(kern, blocks_needed < cap ? blocks_needed : cap, kRouteThreads, wgt_bytes,
+                        s, static_cast<const __nv_bfloat16*>(x),
+                        static_cast<const __nv_bfloat16*>(Wg), T, d, E, idx, w);
+    }
+    return launch_route_tb<Tin, MAXE, 1>(x, Wg, T, d, E, idx, w, s);
 }
 
 }  // namespace

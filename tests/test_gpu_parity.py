@@ -206,3 +206,24 @@ def test_full_size_workloads(name):
     assert err <= BF16_TOL, err
     assert worst_token(y, ref["y"]) <= TOKEN_TOL
     assert torch.equal(layer_y(inp), g["y"])
+
+
+@pytest.mark.parametrize("T", [40, 700])  # one-launch and four-launch permutation paths
+def test_out_of_range_expert_ids_are_flagged(T):
+    """Expert ids outside [0, E) are skipped by the permutation kernels' bounds checks
+    and reported through the workspace status word (flag 0x2)."""
+    d, E = 64, 8
+    x = torch.randn(T, d, device="cuda").to(torch.bfloat16)
+    idx = torch.randint(0, E, (T, 2), dtype=torch.int32, device="cuda")
+    idx[:, 1] = (idx[:, 0] + 1) % E
+    idx[3, 1] = E + 5
+    idx[T - 1, 0] = -2
+    ws = moe.alloc_workspace(T, d, 64, E, 2, torch.bfloat16)
+    off = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    pt = torch.full((2 * T,), -7, dtype=torch.int32, device="cuda")
+    inv = torch.full((T, 2), -7, dtype=torch.int32, device="cuda")
+    xp = torch.zeros(2 * T, d, dtype=torch.bfloat16, device="cuda")
+    moe.moe_permute(idx, x, off, pt, inv, xp, ws, E)
+    assert moe.moe_device_status(ws) & 0x2
+    assert int(off[-1]) == 2 * T - 2  # the two bad pairs are left out
+    assert int(inv[3, 1]) == -7 and int(inv[T - 1, 0]) == -7
