@@ -1,0 +1,483 @@
+// grouped_gemm_pair_sm100.cu -- the per-expert SwiGLU FFN for large batches on pairs of
+// SMs (tcgen05 cta_group::2).
+//
+// Same computation as grouped_gemm_sm100.cu (notion notes "Mixtral of Experts",
+// "Implementation": SwiGLU expert function; atlas "Mixtral", "Design overview"):
+//   GEMM1 (+SwiGLU):  H[r, n] = silu(x_r . W1[e, n]) * (x_r . W3[e, n])   bf16 out
+//   GEMM2:            Y[r, c] = H_r . W2[e, c]                            fp32 out
+// but each tile is computed by a cluster of two CTAs on two SMs.  One thread of the
+// leader CTA issues tcgen05.mma.cta_group::2 with M = 256 rows (128 from each CTA's
+// shared memory) and N = 256 columns whose B operand is split between the CTAs
+// (128 rows of B each); each CTA's tensor memory receives its 128 rows x 256
+// columns.  Per SM this halves the B bytes staged per K block (32 KiB per stage
+// instead of 48 KiB for the same math), which leaves room for 6 pipeline stages
+// and cuts the L2->SM traffic by a third.
+//
+// GEMM1 splits B as [128 rows of W1 | the same 128 rows of W3]: the leader stages
+// the W1 rows, the peer the W3 rows, so accumulator columns 0..127 hold a = x.W1 and
+// 128..255 hold b = x.W3 for the same outputs (as in the single-SM kernel).
+//
+// An expert's rows are covered by 256-row blocks; a last block with at most 128 rows
+// is issued with M = 128 (64 rows per CTA) so that no more rows are wasted than with
+// 128-row tiles.  In that mode the accumulator uses the "2x2" data-path layout:
+// columns 0..127 of the tile in TMEM lanes 0..63 and columns 128..255 in lanes
+// 64..127, both in the first 128 TMEM columns of the buffer.
+//
+// Synchronisation: both CTAs' TMA loads count their bytes on the leader's "full"
+// barrier; the leader's MMA completions are multicast to both CTAs' "empty" and
+// "tmem_full" barriers; both CTAs' epilogues arrive on the leader's "tmem_empty"
+// barrier.  Every wait is bounded; a CTA that gives up raises the status flag.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "moe_internal.h"
+#include "sm100_ptx.cuh"
+
+namespace moe {
+
+// Defined in grouped_gemm_sm100.cu.
+bool encode_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                    uint32_t box_rows);
+
+namespace {
+
+constexpr int kRowsPerCta = 128;
+constexpr int kPairRows = 2 * kRowsPerCta;   // rows per full pair tile
+constexpr int kBK = 64;
+constexpr int kN = 256;                      // accumulator columns per tile
+constexpr int kStages = 6;
+constexpr int kABytes = kRowsPerCta * kBK * 2;  // 16 KiB
+constexpr int kBBytes = 128 * kBK * 2;          // 16 KiB: this CTA's half of B
+constexpr int kStageBytes = kABytes + kBBytes;
+constexpr int kThreads = 192;
+constexpr int kEpiThreads = 128;
+constexpr uint32_t kTmemCols = 2 * kN;
+constexpr uint32_t kIdescFull = idesc_bf16_f32(2 * kRowsPerCta, kN);
+constexpr uint32_t kIdescHalf = idesc_bf16_f32(kRowsPerCta, kN);
+constexpr int kXferBytes = 32 * 64 * 4;  // one 32-column chunk of b for 64 rows
+constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 1024 /*bookkeeping*/ +
+                           kXferBytes;
+constexpr int kXferBarrier = 1;
+constexpr uint16_t kBothCtas = 0x3;
+
+enum Epilogue { kEpiSwiGLU = 0, kEpiStoreF32 = 1 };
+
+struct PairArgs {
+    const int32_t* offsets;
+    int E;
+    int rows;
+    int K;
+    int N;        // output columns
+    int b_rows;   // rows of one expert in the flattened weight view
+    int n_tiles;  // column tiles per row block
+    void* out;
+    uint32_t* status;
+};
+
+struct PairBook {
+    uint64_t full[kStages];
+    uint64_t empty[kStages];
+    uint64_t tmem_full[2];
+    uint64_t tmem_empty[2];
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort_flag;
+    int off[kMaxExperts + 1];
+    int tile_start[kMaxExperts + 1];
+};
+static_assert(sizeof(PairBook) <= 1024, "bookkeeping reserve");
+
+struct PairTile {
+    int e, row0, row_end, nt;
+    bool half;
+};
+
+__device__ __forceinline__ PairTile decode_pair_tile(const PairBook& bk, int E, int tile) {
+    int g = 0;
+    while (g + 1 < E && tile >= bk.tile_start[g + 1]) ++g;
+    const int local = tile - bk.tile_start[g];
+    const int blocks = (bk.off[g + 1] - bk.off[g] + kPairRows - 1) / kPairRows;
+    PairTile t;
+    t.e = g;
+    t.row0 = bk.off[g] + (local % blocks) * kPairRows;
+    t.nt = local / blocks;
+    t.row_end = bk.off[g + 1];
+    t.half = t.row_end - t.row0 <= kRowsPerCta;
+    return t;
+}
+
+__device__ __forceinline__ float bits_f32(uint32_t u) { return __uint_as_float(u); }
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ float silu_mul(float a, float b) {
+    return a / (1.0f + __expf(-a)) * b;
+}
+
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
+    const unsigned long long t0 = global_timer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (global_timer_ns() - t0 > kDrainTimeoutNs) break;
+    }
+}
+
+__device__ __forceinline__ void short_pause_ns(unsigned long long ns) {
+    const unsigned long long t0 = global_timer_ns();
+    while (global_timer_ns() - t0 < ns) {
+    }
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(kThreads, 1)
+    grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
+                             const __grid_constant__ CUtensorMap tmB0,
+                             const __grid_constant__ CUtensorMap tmB1, const PairArgs args) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint8_t* sA = smem;
+    uint8_t* sB = smem + kStages * kABytes;
+    PairBook& bk = *reinterpret_cast<PairBook*>(smem + kStages * kStageBytes);
+    float* xfer = reinterpret_cast<float*>(smem + kStages * kStageBytes + 1024);
+    volatile int* abort_flag = &bk.abort_flag;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int E = args.E;
+    const uint32_t rank = cluster_ctarank();  // 0 = leader, 1 = peer
+    const bool leader = rank == 0;
+    const int pair = blockIdx.x >> 1;
+    const int npairs = gridDim.x >> 1;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&bk.full[s], 1);
+            mbar_init(&bk.empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&bk.tmem_full[a], 1);
+            mbar_init(&bk.tmem_empty[a], 2 * kEpiThreads);
+        }
+        mbar_init(&bk.drain, 1);
+        bk.abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB0);
+        if (EPI == kEpiSwiGLU) tma_prefetch_desc(&tmB1);
+    }
+    if (warp == 1) tmem_alloc_pair(&bk.tmem_base, kTmemCols);
+
+    pdl_wait();
+    if (threadIdx.x == 0) {
+        int prev = 0;
+        for (int g = 0; g <= E; ++g) {
+            int v = args.offsets[g];
+            v = v < prev ? prev : (v > args.rows ? args.rows : v);
+            bk.off[g] = v;
+            prev = v;
+        }
+        bk.tile_start[0] = 0;
+        for (int g = 0; g < E; ++g)
+            bk.tile_start[g + 1] = bk.tile_start[g] +
+                                   (bk.off[g + 1] - bk.off[g] + kPairRows - 1) / kPairRows *
+                                       args.n_tiles;
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();  // both CTAs' barriers are initialised before either signals the other
+    tc_fence_after();
+
+    const uint32_t tmem_base = bk.tmem_base;
+    const int total = bk.tile_start[E];
+    const int num_kb = (args.K + kBK - 1) / kBK;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t pending = 0, pending_phase = 0;
+            bool ok = true, issued = false;
+            const CUtensorMap* tmB = (EPI == kEpiSwiGLU && !leader) ? &tmB1 : &tmB0;
+            for (int tile = pair; ok && tile < total; tile += npairs) {
+                const PairTile t = decode_pair_tile(bk, E, tile);
+                const int a_row = t.row0 + static_cast<int>(rank) * (t.half ? 64 : kRowsPerCta);
+                const int b_row = t.e * args.b_rows + t.nt * (EPI == kEpiSwiGLU ? 128 : 256) +
+                                  (EPI == kEpiSwiGLU ? 0 : static_cast<int>(rank) * 128);
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    if (!mbar_wait_bounded(&bk.empty[stage], phase ^ 1u, abort_flag,
+                                           args.status)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t full_leader = map_to_cta(smem_u32(&bk.full[stage]), 0);
+                    if (leader) mbar_arrive_expect_tx(&bk.full[stage], 2 * kStageBytes);
+                    const int kc = kb * kBK;
+                    tma_load_2d_pair(&tmA, full_leader, sA + stage * kABytes, kc, a_row);
+                    tma_load_2d_pair(tmB, full_leader, sB + stage * kBBytes, kc, b_row);
+                    issued = true;
+                    pending |= 1u << stage;
+                    pending_phase = (pending_phase & ~(1u << stage)) | (phase << stage);
+                    if (++stage == kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (!ok && issued) {
+                if (leader) {
+                    for (int s = 0; s < kStages; ++s)
+                        if (pending & (1u << s)) drain_wait(&bk.full[s], (pending_phase >> s) & 1u);
+                } else {
+                    // The peer's copies complete on the leader's barriers; give them
+                    // time to land before this CTA's shared memory can be released.
+                    short_pause_ns(2000000ull);
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer (leader)
+        if (lane == 0 && leader) {
+            int stage = 0, acc = 0;
+            uint32_t phase = 0, acc_phase = 0;
+            bool ok = true, issued = false;
+            for (int tile = pair; ok && tile < total; tile += npairs) {
+                const PairTile t = decode_pair_tile(bk, E, tile);
+                const uint32_t idesc = t.half ? kIdescHalf : kIdescFull;
+                if (!mbar_wait_bounded(&bk.tmem_empty[acc], acc_phase ^ 1u, abort_flag,
+                                       args.status)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kN);
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    if (!mbar_wait_bounded(&bk.full[stage], phase, abort_flag, args.status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t ad = sw128_kmajor_desc(smem_u32(sA + stage * kABytes));
+                    const uint64_t bd = sw128_kmajor_desc(smem_u32(sB + stage * kBBytes));
+#pragma unroll
+                    for (int k = 0; k < kBK / 16; ++k)
+                        umma_bf16_pair(d_tmem, ad + 2 * k, bd + 2 * k, idesc, (kb | k) != 0);
+                    umma_commit_pair(&bk.empty[stage], kBothCtas);
+                    issued = true;
+                    if (++stage == kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                umma_commit_pair(&bk.tmem_full[acc], kBothCtas);
+                acc ^= 1;
+                if (acc == 0) acc_phase ^= 1u;
+            }
+            if (!ok && issued) {
+                umma_commit_pair(&bk.drain, 0x1);
+                drain_wait(&bk.drain, 0);
+            }
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ epilogue (both CTAs)
+        const int q = warp & 3;
+        const uint32_t empty_leader0 = map_to_cta(smem_u32(&bk.tmem_empty[0]), 0);
+        const uint32_t empty_leader1 = map_to_cta(smem_u32(&bk.tmem_empty[1]), 0);
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int tile = pair; tile < total; tile += npairs) {
+            const PairTile t = decode_pair_tile(bk, E, tile);
+            if (!mbar_wait_bounded(&bk.tmem_full[acc], acc_phase, abort_flag, args.status))
+                break;
+            tc_fence_after();
+            const uint32_t tlane = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                                   static_cast<uint32_t>(acc * kN);
+            if (!t.half) {
+                const int row = t.row0 + static_cast<int>(rank) * kRowsPerCta + q * 32 + lane;
+                const bool valid = row < t.row_end;
+                if (EPI == kEpiSwiGLU) {
+                    __nv_bfloat16* out =
+                        static_cast<__nv_bfloat16*>(args.out) + static_cast<size_t>(row) * args.N;
+                    const int col0 = t.nt * 128;
+#pragma unroll 1
+                    for (int ch = 0; ch < 4; ++ch) {
+                        uint32_t a[32], b[32];
+                        tmem_ld_32cols(tlane + ch * 32, a);
+                        tmem_ld_32cols(tlane + 128 + ch * 32, b);
+                        tmem_ld_wait();
+                        uint32_t p[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i)
+                            p[i] = pack_bf16x2(silu_mul(bits_f32(a[2 * i]), bits_f32(b[2 * i])),
+                                               silu_mul(bits_f32(a[2 * i + 1]), bits_f32(b[2 * i + 1])));
+                        if (valid) {
+#pragma unroll
+                            for (int v = 0; v < 4; ++v) {
+                                const int col = col0 + ch * 32 + v * 8;
+                                if (col < args.N)
+                                    *reinterpret_cast<uint4*>(out + col) =
+                                        make_uint4(p[4 * v], p[4 * v + 1], p[4 * v + 2], p[4 * v + 3]);
+                            }
+                        }
+                    }
+                } else {
+                    float* out = static_cast<float*>(args.out) + static_cast<size_t>(row) * args.N;
+                    const int col0 = t.nt * 256;
+#pragma unroll 1
+                    for (int ch = 0; ch < 8; ++ch) {
+                        uint32_t v[32];
+                        tmem_ld_32cols(tlane + ch * 32, v);
+                        tmem_ld_wait();
+                        if (valid) {
+#pragma unroll
+                            for (int j = 0; j < 8; ++j) {
+                                const int col = col0 + ch * 32 + j * 4;
+                                if (col < args.N)
+                                    *reinterpret_cast<float4*>(out + col) =
+                                        make_float4(bits_f32(v[4 * j]), bits_f32(v[4 * j + 1]),
+                                                    bits_f32(v[4 * j + 2]), bits_f32(v[4 * j + 3]));
+                            }
+                        }
+                    }
+                }
+            } else {
+                // 64 rows per CTA; lanes 0..63 hold tile columns 0..127 and lanes 64..127
+                // hold columns 128..255, both in TMEM columns 0..127 of the buffer.
+                const int m = (q & 1) * 32 + lane;
+                const int row = t.row0 + static_cast<int>(rank) * 64 + m;
+                const bool valid = row < t.row_end;
+                const bool upper = q >= 2;  // holds tile columns 128..255
+                if (EPI == kEpiSwiGLU) {
+                    __nv_bfloat16* out =
+                        static_cast<__nv_bfloat16*>(args.out) + static_cast<size_t>(row) * args.N;
+                    const int col0 = t.nt * 128;
+#pragma unroll 1
+                    for (int ch = 0; ch < 4; ++ch) {
+                        uint32_t v[32];
+                        tmem_ld_32cols(tlane + ch * 32, v);
+                        tmem_ld_wait();
+                        if (upper) {  // b for rows m, columns ch*32 .. ch*32+31
+#pragma unroll
+                            for (int j = 0; j < 32; ++j) xfer[j * 64 + m] = bits_f32(v[j]);
+                        }
+                        asm volatile("bar.sync %0, %1;" ::"r"(kXferBarrier), "r"(kEpiThreads)
+                                     : "memory");
+                        if (!upper && valid) {
+                            uint32_t p[16];
+#pragma unroll
+                            for (int i = 0; i < 16; ++i)
+                                p[i] = pack_bf16x2(silu_mul(bits_f32(v[2 * i]), xfer[(2 * i) * 64 + m]),
+                                                   silu_mul(bits_f32(v[2 * i + 1]),
+                                                            xfer[(2 * i + 1) * 64 + m]));
+#pragma unroll
+                            for (int u = 0; u < 4; ++u) {
+                                const int col = col0 + ch * 32 + u * 8;
+                                if (col < args.N)
+                                    *reinterpret_cast<uint4*>(out + col) =
+                                        make_uint4(p[4 * u], p[4 * u + 1], p[4 * u + 2], p[4 * u + 3]);
+                            }
+                        }
+                        asm volatile("bar.sync %0, %1;" ::"r"(kXferBarrier), "r"(kEpiThreads)
+                                     : "memory");
+                    }
+                } else {
+                    float* out = static_cast<float*>(args.out) + static_cast<size_t>(row) * args.N;
+                    const int col0 = t.nt * 256 + (upper ? 128 : 0);
+#pragma unroll 1
+                    for (int ch = 0; ch < 4; ++ch) {
+                        uint32_t v[32];
+                        tmem_ld_32cols(tlane + ch * 32, v);
+                        tmem_ld_wait();
+                        if (valid) {
+#pragma unroll
+                            for (int j = 0; j < 8; ++j) {
+                                const int col = col0 + ch * 32 + j * 4;
+                                if (col < args.N)
+                                    *reinterpret_cast<float4*>(out + col) =
+                                        make_float4(bits_f32(v[4 * j]), bits_f32(v[4 * j + 1]),
+                                                    bits_f32(v[4 * j + 2]), bits_f32(v[4 * j + 3]));
+                            }
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive_cluster(acc == 0 ? empty_leader0 : empty_leader1);
+            acc ^= 1;
+            if (acc == 0) acc_phase ^= 1u;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();  // the leader's MMAs into this CTA's TMEM are done on both sides
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem_base, kTmemCols);
+    }
+}
+
+template <int EPI>
+cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
+                        const PairArgs& args, int npairs, cudaStream_t s) {
+    auto kern = grouped_gemm_pair_kernel<EPI>;
+    static int configured[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && !configured[dev]) {
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+        configured[dev] = 1;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * npairs);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t err = cudaLaunchKernelEx(&cfg, kern, a, b0, b1, args);
+    return err != cudaSuccess ? err : cudaGetLastError();
+}
+
+}  // namespace
+
+// Large-batch expert FFN on CTA pairs (both GEMMs).
+cudaError_t launch_ffn_bf16_pair(const void* x_perm, const int32_t* offsets, const void* W1,
+                                 const void* W3, const void* W2, int rows, int d, int h, int E,
+                                 void* H, float* Y, uint32_t* status, cudaStream_t s,
+                                 cudaEvent_t between) {
+    CUtensorMap mx, mw1, mw3, mh, mw2;
+    if (!encode_bf16_2d(&mx, x_perm, rows, d, kRowsPerCta) ||
+        !encode_bf16_2d(&mw1, W1, static_cast<uint64_t>(E) * h, d, 128) ||
+        !encode_bf16_2d(&mw3, W3, static_cast<uint64_t>(E) * h, d, 128) ||
+        !encode_bf16_2d(&mh, H, rows, h, kRowsPerCta) ||
+        !encode_bf16_2d(&mw2, W2, static_cast<uint64_t>(E) * d, h, 128))
+        return cudaErrorInvalidValue;
+    const int max_pairs = device_sm_count() / 2;
+    const long long blocks = (static_cast<long long>(rows) + (kPairRows - 1LL) * E) / kPairRows;
+    PairArgs g1{offsets, E, rows, d, h, h, (h + 127) / 128, H, status};
+    long long t1 = blocks * g1.n_tiles;
+    cudaError_t err = launch_pair<kEpiSwiGLU>(
+        mx, mw1, mw3, g1, static_cast<int>(t1 < max_pairs ? (t1 < 1 ? 1 : t1) : max_pairs), s);
+    if (err != cudaSuccess) return err;
+    if (between && (err = cudaEventRecord(between, s)) != cudaSuccess) return err;
+    PairArgs g2{offsets, E, rows, h, d, d, (d + 255) / 256, Y, status};
+    long long t2 = blocks * g2.n_tiles;
+    return launch_pair<kEpiStoreF32>(
+        mh, mw2, mw2, g2, static_cast<int>(t2 < max_pairs ? (t2 < 1 ? 1 : t2) : max_pairs), s);
+}
+
+}  // namespace moe

@@ -425,6 +425,9 @@ cudaError_t launch_ffn_bf16(const void* x_perm, const int32_t* offsets, const vo
         return cudaSuccess;
     }
     if (out) *out = FfnOut{Y, 1};
+    if (rows >= kPairMinRows && pair_gemm_enabled())
+        return launch_ffn_bf16_pair(x_perm, offsets, W1, W3, W2, rows, d, h, E, H, Y, status, s,
+                                    between);
     CUtensorMap mx, mw1, mw3, mh, mw2;
     if (!encode_bf16_2d(&mx, x_perm, rows, d, kBM) ||
         !encode_bf16_2d(&mw1, W1, static_cast<uint64_t>(E) * h, d, 128) ||

@@ -41,6 +41,15 @@ bool small_batch(int T) { return T <= 64; }
 }  // namespace
 
 bool pdl_enabled() { return t_pdl_scope && pdl_allowed(); }
+
+bool pair_gemm_enabled() {
+    static int v = -1;
+    if (v < 0) {
+        const char* e = std::getenv("MOE_GEMM_PAIR");
+        v = (e && e[0] == '0') ? 0 : 1;
+    }
+    return v == 1;
+}
 PdlScope::PdlScope(bool on) : prev(t_pdl_scope) { t_pdl_scope = on; }
 PdlScope::~PdlScope() { t_pdl_scope = prev; }
 

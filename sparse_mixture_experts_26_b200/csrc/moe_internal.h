@@ -125,6 +125,14 @@ cudaError_t launch_ffn_bf16(const void* x_perm, const int32_t* offsets, const vo
                             void* H, float* Y, float* partials, int partial_cap, bool reduce,
                             FfnOut* out, uint32_t* status, cudaStream_t s,
                             cudaEvent_t between = nullptr);
+// Large-batch expert FFN on CTA pairs (tcgen05 cta_group::2).
+cudaError_t launch_ffn_bf16_pair(const void* x_perm, const int32_t* offsets, const void* W1,
+                                 const void* W3, const void* W2, int rows, int d, int h, int E,
+                                 void* H, float* Y, uint32_t* status, cudaStream_t s,
+                                 cudaEvent_t between);
+// Grouped rows from which the CTA-pair kernels are used (MOE_GEMM_PAIR=0 disables them).
+constexpr int kPairMinRows = 2048;
+bool pair_gemm_enabled();
 // Small-batch expert FFN; the down projection writes `ksplit` partial arrays.
 cudaError_t launch_ffn_bf16_decode(const void* x_perm, const int32_t* offsets, const void* W1,
                                    const void* W3, const void* W2, int rows, int d, int h, int E,

@@ -108,6 +108,9 @@ SMALL = [  # (T, d, h, kind): ragged row blocks, K tails, N tails, empty groups
     # T > 64 runs the grouped GEMM (128-row blocks)
     (65, 128, 256, "plain"), (129, 256, 512, "plain"), (300, 136, 200, "plain"),
     (1000, 512, 1024, "plain"), (700, 256, 384, "skew"), (513, 128, 256, "long"),
+    # >= 2048 grouped rows run the CTA-pair grouped GEMM (256-row blocks; an expert's
+    # last block of <= 128 rows runs in the pair's 128-row mode)
+    (1100, 256, 384, "plain"), (1500, 136, 200, "skew"), (2500, 128, 256, "long"),
 ]
 
 
