@@ -43,8 +43,11 @@ DOMINANT = {
                "decode_gemm_swiglu", os.path.join(CSRC, "decode_gemm_sm100.cu")),
     "grouped": ("grouped_gemm_kernel<SwiGLU> (GEMM1 + silu*gate epilogue)",
                 "grouped_gemm_swiglu", os.path.join(CSRC, "grouped_gemm_sm100.cu")),
+    "pair": ("grouped_gemm_pair_kernel<SwiGLU> (CTA-pair GEMM1 + silu*gate epilogue)",
+             "grouped_gemm_pair_swiglu", os.path.join(CSRC, "grouped_gemm_pair_sm100.cu")),
 }
-DECODE_MAX_TOKENS = 64  # the library switches to the weight-streaming kernels here
+DECODE_MAX_TOKENS = 64    # the library switches to the weight-streaming kernels here
+PAIR_MIN_TOKENS = 1024    # ... and to the CTA-pair kernels here (2048 grouped rows)
 
 
 # ------------------------------------------------------------------ ranks
@@ -299,7 +302,12 @@ def run_ours(args):
     touched = int((counts > 0).sum())
 
     peaks, peak_src = load_peaks()
-    regime = "decode" if wl.T <= DECODE_MAX_TOKENS else "grouped"
+    if wl.T <= DECODE_MAX_TOKENS:
+        regime = "decode"
+    elif wl.T >= PAIR_MIN_TOKENS and os.environ.get("MOE_GEMM_PAIR", "1") != "0":
+        regime = "pair"
+    else:
+        regime = "grouped"
     kname, tag, ksrc = DOMINANT[regime]
     if regime == "decode":  # weight streaming: HBM-bound
         bound, unit = "hbm", "GB/s"

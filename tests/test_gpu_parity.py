@@ -230,3 +230,18 @@ def test_out_of_range_expert_ids_are_flagged(T):
     assert moe.moe_device_status(ws) & 0x2
     assert int(off[-1]) == 2 * T - 2  # the two bad pairs are left out
     assert int(inv[3, 1]) == -7 and int(inv[T - 1, 0]) == -7
+
+
+@pytest.mark.parametrize("E", [2, 4, 16, 32])
+@pytest.mark.parametrize("T", [40, 300])  # weight-streaming and grouped kernels
+def test_other_expert_counts(E, T):
+    """The layer for E other than 8 (the ABI allows 2..32): routing and permutation
+    bit-exact, output within the bf16 tolerance."""
+    wl = small("e", T=T, d=128, h=256, E=E, seed=E * 1000 + T)
+    inp = make_inputs(wl, "cuda")
+    g = run_steps(inp, E)
+    x_cpu = f64(inp["x"])
+    check_routing_and_permutation(g, x_cpu, f64(inp["Wg"]), E)
+    ref = O.moe_layer(x_cpu, f64(inp["Wg"]), f64(inp["W1"]), f64(inp["W3"]), f64(inp["W2"]))
+    assert rel_fro(f64(g["y"]), ref["y"]) <= BF16_TOL
+    assert torch.equal(layer_y(inp), g["y"])
