@@ -65,7 +65,9 @@ typedef enum {
  * layout of routing results, permutation, gathered rows x_perm, the SwiGLU
  * activations H, the fp32 expert outputs and, for batches of at most 64 tokens, the
  * fp32 partial sums of the split-K down projection).  It also covers moe_permute and
- * moe_expert_ffn.  Returns 0 for unsupported arguments. */
+ * moe_expert_ffn.  Zero the workspace once before its first use: it holds a status
+ * word and dependency counters that every call leaves at zero.  Returns 0 for
+ * unsupported arguments. */
 size_t moe_workspace_bytes(int T, int d, int h, int E, int k, moe_dtype dt);
 
 /* Router + top-2 + softmax of the two kept logits.
@@ -154,8 +156,9 @@ moe_status moe_layer_forward(const void *x, const void *Wg, const void *W1,
 /* moe_layer_forward that also records up to five caller-created events on `stream`
  * between its stages, for timing them without a profiler:
  *   events[0] before the router, events[1] after the permutation (before the
- *   expert FFN), events[2] after the first FFN kernel (GEMM1 + SwiGLU), events[3]
- *   after the second (GEMM2), events[4] after the combine.
+ *   expert FFN), events[2] after the first FFN kernel (GEMM1 + SwiGLU; for batches
+ *   of at most 64 tokens, where one fused kernel runs both GEMMs, after it),
+ *   events[3] after the expert FFN, events[4] after the combine.
  * n_events may be 0..5; events beyond n_events are not recorded. */
 moe_status moe_layer_forward_events(const void *x, const void *Wg, const void *W1,
                                     const void *W3, const void *W2, int T, int d, int h,

@@ -385,6 +385,403 @@ cudaError_t launch_decode(const CUtensorMap& w0, const CUtensorMap& w1, const CU
     return launch_k(kern, grid, kThreads, C::kSmem, s, w0, w1, x, args);
 }
 
+// ---------------------------------------------------------------- fused gate/up + down
+// One persistent cooperative launch runs both GEMMs.  Its unit list is all gate/up
+// tiles (expert, token chunk, 64-row block of W1/W3), then all down units (expert,
+// token chunk, 128-row block of W2, K range), experts in order.  A down unit needs
+// only the H columns of its own K range, i.e. the gate/up tiles with the same expert
+// and h-blocks in that range; each such tile bumps ready[e][ks] after its H stores
+// are visible, and the down unit's producer waits (bounded) for the count before it
+// loads H.  SMs that run out of gate/up tiles start streaming W2 at once, so neither
+// the gate/up tail nor the launch boundary leaves HBM idle.  The readers of a
+// counter also count themselves and the last one resets both counters to zero, so
+// every launch starts from zeroed counters (repeated launches and graph replays).
+struct FusedArgs {
+    const int32_t* offsets;
+    int E;
+    int rows;
+    int d;
+    int h;
+    int n_hb;      // 64-row W1/W3 blocks per expert: ceil(h / 64)
+    int n_db;      // 128-row W2 blocks per expert: ceil(d / 128)
+    int ksplit;    // K ranges of the down projection
+    void* H;       // bf16 [rows, h]
+    float* Ypart;  // ksplit fp32 partials [ksplit][rows][d]
+    uint32_t* ready;    // [E][ksplit]
+    uint32_t* readers;  // [E][ksplit]
+    uint32_t* status;
+};
+
+template <int NACC>
+struct FusedBook {
+    uint64_t full[16];
+    uint64_t empty[16];
+    uint64_t tmem_full[NACC];
+    uint64_t tmem_empty[NACC];
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort_flag;
+    int off[kMaxExperts + 1];
+    int start1[kMaxExperts + 1];  // gate/up tiles before expert g
+    int start2[kMaxExperts + 1];  // down units before expert g
+};
+
+struct FusedUnit {
+    bool down;
+    int e, row0, nvalid, chunks, blk, ks, kb0, kb1;
+};
+
+template <int NACC>
+__device__ __forceinline__ FusedUnit fused_unit(const FusedBook<NACC>& bk, const FusedArgs& a,
+                                                int NTc, int num_kb1, int kps, int num_kb2,
+                                                int u) {
+    FusedUnit f;
+    const int n1 = bk.start1[a.E];
+    int g = 0, local;
+    if (u < n1) {
+        while (g + 1 < a.E && u >= bk.start1[g + 1]) ++g;
+        local = u - bk.start1[g];
+        f.down = false;
+        f.ks = 0;
+        const int chunk = local / a.n_hb;
+        f.blk = local - chunk * a.n_hb;
+        f.row0 = bk.off[g] + chunk * NTc;
+        f.kb0 = 0;
+        f.kb1 = num_kb1;
+    } else {
+        const int v = u - n1;
+        while (g + 1 < a.E && v >= bk.start2[g + 1]) ++g;
+        local = v - bk.start2[g];
+        f.down = true;
+        f.ks = local % a.ksplit;
+        local /= a.ksplit;
+        const int chunk = local / a.n_db;
+        f.blk = local - chunk * a.n_db;
+        f.row0 = bk.off[g] + chunk * NTc;
+        f.kb0 = f.ks * kps;
+        f.kb1 = min(num_kb2, f.kb0 + kps);
+    }
+    f.e = g;
+    f.chunks = (bk.off[g + 1] - bk.off[g] + NTc - 1) / NTc;
+    const int left = bk.off[g + 1] - f.row0;
+    f.nvalid = left < NTc ? left : NTc;
+    return f;
+}
+
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+template <int NT>
+__global__ void __launch_bounds__(kThreads, 1)
+    decode_ffn_fused_kernel(const __grid_constant__ CUtensorMap tmW1,
+                            const __grid_constant__ CUtensorMap tmW3,
+                            const __grid_constant__ CUtensorMap tmX,
+                            const __grid_constant__ CUtensorMap tmW2,
+                            const __grid_constant__ CUtensorMap tmH, const FusedArgs args) {
+    using C = DecodeCfg<kSwiGLU, NT>;  // same stage layout for both GEMMs
+    constexpr int NACC = C::kAcc;
+    constexpr int J1 = kM / 2;         // 64 output columns of H per gate/up tile
+    using Book = FusedBook<NACC>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint8_t* sA = smem;
+    uint8_t* sB = smem + C::kStages * C::kAStage;
+    Book& bk = *reinterpret_cast<Book*>(sB + C::kStages * C::kBStage);
+    float* xfer = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(&bk) + 2048);
+    static_assert(sizeof(Book) <= 2048, "bookkeeping reserve");
+    volatile int* abort_flag = &bk.abort_flag;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int E = args.E;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::kStages; ++s) {
+            mbar_init(&bk.full[s], 1);
+            mbar_init(&bk.empty[s], 1);
+        }
+        for (int a = 0; a < NACC; ++a) {
+            mbar_init(&bk.tmem_full[a], 1);
+            mbar_init(&bk.tmem_empty[a], kEpiThreads);
+        }
+        mbar_init(&bk.drain, 1);
+        bk.abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmW1);
+        tma_prefetch_desc(&tmW3);
+        tma_prefetch_desc(&tmX);
+        tma_prefetch_desc(&tmW2);
+        tma_prefetch_desc(&tmH);
+    }
+    if (warp == 1) tmem_alloc(&bk.tmem_base, kTmemCols);
+
+    pdl_wait();
+    pdl_launch_dependents();
+    if (threadIdx.x == 0) {
+        int prev = 0;
+        for (int g = 0; g <= E; ++g) {
+            int v = args.offsets[g];
+            v = v < prev ? prev : (v > args.rows ? args.rows : v);
+            bk.off[g] = v;
+            prev = v;
+        }
+        bk.start1[0] = 0;
+        bk.start2[0] = 0;
+        for (int g = 0; g < E; ++g) {
+            const int chunks = (bk.off[g + 1] - bk.off[g] + NT - 1) / NT;
+            bk.start1[g + 1] = bk.start1[g] + chunks * args.n_hb;
+            bk.start2[g + 1] = bk.start2[g] + chunks * args.n_db * args.ksplit;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    const uint32_t tmem_base = bk.tmem_base;
+    const int total = bk.start1[E] + bk.start2[E];
+    const int num_kb1 = (args.d + kBK - 1) / kBK;
+    const int num_kb2 = (args.h + kBK - 1) / kBK;
+    const int kps = (num_kb2 + args.ksplit - 1) / args.ksplit;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            const uint64_t evict_first = l2_policy_evict_first();
+            int stage = 0;
+            uint32_t phase = 0, pending = 0, pending_phase = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; ok && u < total; u += gridDim.x) {
+                const FusedUnit f = fused_unit(bk, args, NT, num_kb1, kps, num_kb2, u);
+                if (f.down) {
+                    // wait until every gate/up tile of this K range has published its H
+                    const uint32_t need = static_cast<uint32_t>(f.chunks * (f.kb1 - f.kb0));
+                    const uint32_t* rdy = args.ready + f.e * args.ksplit + f.ks;
+                    if (ld_acquire_gpu(rdy) < need) {
+                        const unsigned long long t0 = global_timer_ns();
+                        while (ld_acquire_gpu(rdy) < need) {
+                            if (*abort_flag) {
+                                ok = false;
+                                break;
+                            }
+                            if (global_timer_ns() - t0 > kWaitTimeoutNs) {
+                                *abort_flag = 1;
+                                if (args.status) atomicOr(args.status, 1u);
+                                ok = false;
+                                break;
+                            }
+                        }
+                        if (!ok) break;
+                    }
+                    fence_proxy_async_global();
+                    // the last reader of this counter resets it for the next launch
+                    uint32_t* rd = args.readers + f.e * args.ksplit + f.ks;
+                    if (atomicAdd(rd, 1u) + 1u == static_cast<uint32_t>(f.chunks * args.n_db)) {
+                        *const_cast<uint32_t*>(rdy) = 0u;
+                        *rd = 0u;
+                    }
+                }
+                const int wrow = f.down ? f.e * args.d + f.blk * kM : f.e * args.h + f.blk * J1;
+                for (int kb = f.kb0; kb < f.kb1; ++kb) {
+                    if (!mbar_wait_bounded(&bk.empty[stage], phase ^ 1u, abort_flag,
+                                           args.status)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&bk.full[stage], C::kStageTx);
+                    const int kc = kb * kBK;
+                    uint8_t* a = sA + stage * C::kAStage;
+                    uint8_t* b = sB + stage * C::kBStage;
+                    if (f.down) {
+                        tma_load_2d_hint(&tmW2, &bk.full[stage], a, kc, wrow, evict_first);
+                        tma_load_2d(&tmH, &bk.full[stage], b, kc, f.row0);
+                    } else {
+                        tma_load_2d_hint(&tmW1, &bk.full[stage], a, kc, wrow, evict_first);
+                        tma_load_2d_hint(&tmW3, &bk.full[stage], a + J1 * 128, kc, wrow,
+                                         evict_first);
+                        tma_load_2d(&tmX, &bk.full[stage], b, kc, f.row0);
+                    }
+                    pending |= 1u << stage;
+                    pending_phase = (pending_phase & ~(1u << stage)) | (phase << stage);
+                    if (++stage == C::kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (!ok) {
+                for (int s2 = 0; s2 < C::kStages; ++s2)
+                    if (pending & (1u << s2)) drain_wait(&bk.full[s2], (pending_phase >> s2) & 1u);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            int stage = 0, acc = 0;
+            uint32_t phase = 0, acc_phase = 0;
+            bool ok = true, issued = false;
+            for (int u = blockIdx.x; ok && u < total; u += gridDim.x) {
+                const FusedUnit f = fused_unit(bk, args, NT, num_kb1, kps, num_kb2, u);
+                if (!mbar_wait_bounded(&bk.tmem_empty[acc], acc_phase ^ 1u, abort_flag,
+                                       args.status)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * NT);
+                for (int kb = f.kb0; kb < f.kb1; ++kb) {
+                    if (!mbar_wait_bounded(&bk.full[stage], phase, abort_flag, args.status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t ad = sw128_kmajor_desc(smem_u32(sA + stage * C::kAStage));
+                    const uint64_t bd = sw128_kmajor_desc(smem_u32(sB + stage * C::kBStage));
+#pragma unroll
+                    for (int k = 0; k < kBK / 16; ++k)
+                        umma_bf16(d_tmem, ad + 2 * k, bd + 2 * k, C::kIdesc,
+                                  (kb > f.kb0 || k > 0) ? 1u : 0u);
+                    umma_commit(&bk.empty[stage]);
+                    issued = true;
+                    if (++stage == C::kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                umma_commit(&bk.tmem_full[acc]);
+                if (++acc == NACC) {
+                    acc = 0;
+                    acc_phase ^= 1u;
+                }
+            }
+            if (!ok && issued) {
+                umma_commit(&bk.drain);
+                drain_wait(&bk.drain, 0);
+            }
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int q = warp & 3;
+        const int r = q * 32 + lane;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int u = blockIdx.x; u < total; u += gridDim.x) {
+            const FusedUnit f = fused_unit(bk, args, NT, num_kb1, kps, num_kb2, u);
+            if (!mbar_wait_bounded(&bk.tmem_full[acc], acc_phase, abort_flag, args.status))
+                break;
+            tc_fence_after();
+            uint32_t v[NT];
+            tmem_ld_cols<NT>(tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                                 static_cast<uint32_t>(acc * NT),
+                             v);
+            tmem_ld_wait();
+            tc_fence_before();
+            mbar_arrive(&bk.tmem_empty[acc]);
+            if (!f.down) {
+#pragma unroll
+                for (int c = 0; c < NT; ++c) xfer[c * kM + r] = __uint_as_float(v[c]);
+                asm volatile("bar.sync %0, %1;" ::"r"(kXferBarrier), "r"(kEpiThreads) : "memory");
+                if (r < J1) {
+                    const int col = f.blk * J1 + r;
+                    if (col < args.h) {
+                        __nv_bfloat16* out = static_cast<__nv_bfloat16*>(args.H);
+#pragma unroll
+                        for (int c = 0; c < NT; ++c) {
+                            if (c < f.nvalid) {
+                                const float a = xfer[c * kM + r];
+                                const float b = xfer[c * kM + J1 + r];
+                                out[static_cast<size_t>(f.row0 + c) * args.h + col] =
+                                    __float2bfloat16_rn(a / (1.0f + __expf(-a)) * b);
+                            }
+                        }
+                    }
+                    __threadfence();  // H stores visible at device scope before the count
+                }
+                asm volatile("bar.sync %0, %1;" ::"r"(kXferBarrier), "r"(kEpiThreads) : "memory");
+                if (r == 0) {
+                    fence_proxy_async_global();
+                    atomicAdd(args.ready + f.e * args.ksplit + f.blk / kps, 1u);
+                }
+            } else {
+                const int col = f.blk * kM + r;
+                if (col < args.d) {
+                    float* out = args.Ypart + static_cast<size_t>(f.ks) * args.rows * args.d;
+#pragma unroll
+                    for (int c = 0; c < NT; ++c)
+                        if (c < f.nvalid)
+                            out[static_cast<size_t>(f.row0 + c) * args.d + col] =
+                                __uint_as_float(v[c]);
+                }
+            }
+            if (++acc == NACC) {
+                acc = 0;
+                acc_phase ^= 1u;
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, kTmemCols);
+    }
+}
+
+template <int NT>
+cudaError_t launch_ffn_fused_nt(const void* x_perm, const int32_t* offsets, const void* W1,
+                                const void* W3, const void* W2, int rows, int d, int h, int E,
+                                void* H, float* Ypart, int ksplit, uint32_t* counters,
+                                uint32_t* status, cudaStream_t s) {
+    CUtensorMap mw1, mw3, mx, mw2, mh;
+    if (!encode_bf16_2d(&mw1, W1, static_cast<uint64_t>(E) * h, d, kM / 2) ||
+        !encode_bf16_2d(&mw3, W3, static_cast<uint64_t>(E) * h, d, kM / 2) ||
+        !encode_bf16_2d(&mx, x_perm, rows, d, NT) ||
+        !encode_bf16_2d(&mw2, W2, static_cast<uint64_t>(E) * d, h, kM) ||
+        !encode_bf16_2d(&mh, H, rows, h, NT))
+        return cudaErrorInvalidValue;
+    using C = DecodeCfg<kSwiGLU, NT>;
+    auto kern = decode_ffn_fused_kernel<NT>;
+    static int configured[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && !configured[dev]) {
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+        configured[dev] = 1;
+    }
+    FusedArgs a{offsets, E, rows, d, h, (h + 63) / 64, (d + kM - 1) / kM, ksplit, H, Ypart,
+                counters, counters + E * ksplit, status};
+    const int sms = device_sm_count();
+    const long long chunks = static_cast<long long>(rows) / NT + E;
+    const long long units = chunks * (a.n_hb + static_cast<long long>(a.n_db) * ksplit);
+    // Every CTA must be resident at once (down units wait for other CTAs' tiles), so
+    // the launch is cooperative: one CTA per SM at most.
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(units < sms ? units : sms));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = C::kSmem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t err = cudaLaunchKernelEx(&cfg, kern, mw1, mw3, mx, mw2, mh, a);
+    return err != cudaSuccess ? err : cudaGetLastError();
+}
+
 template <int NT>
 cudaError_t launch_ffn_decode_nt(const void* x_perm, const int32_t* offsets, const void* W1,
                                  const void* W3, const void* W2, int rows, int d, int h, int E,
@@ -413,6 +810,21 @@ cudaError_t launch_ffn_decode_nt(const void* x_perm, const int32_t* offsets, con
 }
 
 }  // namespace
+
+cudaError_t launch_ffn_bf16_decode_fused(const void* x_perm, const int32_t* offsets,
+                                         const void* W1, const void* W3, const void* W2, int rows,
+                                         int d, int h, int E, void* H, float* Ypart, int ksplit,
+                                         uint32_t* counters, uint32_t* status, cudaStream_t s) {
+    const int T = rows / 2;
+    if (T <= 16)
+        return launch_ffn_fused_nt<16>(x_perm, offsets, W1, W3, W2, rows, d, h, E, H, Ypart,
+                                       ksplit, counters, status, s);
+    if (T <= 32)
+        return launch_ffn_fused_nt<32>(x_perm, offsets, W1, W3, W2, rows, d, h, E, H, Ypart,
+                                       ksplit, counters, status, s);
+    return launch_ffn_fused_nt<64>(x_perm, offsets, W1, W3, W2, rows, d, h, E, H, Ypart, ksplit,
+                                   counters, status, s);
+}
 
 cudaError_t launch_ffn_bf16_decode(const void* x_perm, const int32_t* offsets, const void* W1,
                                    const void* W3, const void* W2, int rows, int d, int h, int E,

@@ -403,7 +403,7 @@ cudaError_t launch_ffn_bf16(const void* x_perm, const int32_t* offsets, const vo
                             const void* W3, const void* W2, int rows, int d, int h, int E,
                             void* H, float* Y, float* partials, int partial_cap, bool reduce,
                             FfnOut* out, uint32_t* status, cudaStream_t s,
-                            cudaEvent_t between) {
+                            cudaEvent_t between, uint32_t* counters) {
     if (rows <= kDecodeMaxRows) {
         // Largest split of the down projection's K blocks (at most partial_cap) that
         // leaves no K range empty.
@@ -412,8 +412,15 @@ cudaError_t launch_ffn_bf16(const void* x_perm, const int32_t* offsets, const vo
         while (ksplit > 1 && ((num_kb + ksplit - 1) / ksplit) * (ksplit - 1) >= num_kb) --ksplit;
         if (ksplit < 1) ksplit = 1;
         float* dst = ksplit > 1 ? partials : Y;
-        cudaError_t err = launch_ffn_bf16_decode(x_perm, offsets, W1, W3, W2, rows, d, h, E, H,
-                                                 dst, ksplit, status, s, between);
+        cudaError_t err;
+        if (counters) {
+            err = launch_ffn_bf16_decode_fused(x_perm, offsets, W1, W3, W2, rows, d, h, E, H, dst,
+                                               ksplit, counters, status, s);
+            if (err == cudaSuccess && between) err = cudaEventRecord(between, s);
+        } else {
+            err = launch_ffn_bf16_decode(x_perm, offsets, W1, W3, W2, rows, d, h, E, H, dst,
+                                         ksplit, status, s, between);
+        }
         if (err != cudaSuccess) return err;
         if (ksplit > 1 && reduce) {
             err = launch_sum_splits(partials, ksplit, static_cast<size_t>(rows) * d, Y, s);

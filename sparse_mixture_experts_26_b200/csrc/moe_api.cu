@@ -178,7 +178,7 @@ moe_status moe_expert_ffn(const void* x_perm, const int32_t* offsets, const void
     if (dt == MOE_BF16) {
         err = launch_ffn_bf16(x_perm, offsets, W1, W3, W2, rows, d, h, E, at<void>(ws, L.H), y_perm,
                               at<float>(ws, L.Ypart), kDecodeSplitK, /*reduce=*/true, nullptr,
-                              status, stream);
+                              status, stream, nullptr, at<uint32_t>(ws, L.sync));
         if (err == cudaErrorInvalidValue) return MOE_ERR_INVALID_ARG;  // tensor map refused
     } else {
         err = launch_ffn_f32(static_cast<const float*>(x_perm), offsets,
@@ -243,7 +243,8 @@ moe_status layer_forward_impl(const void* x, const void* Wg, const void* W1, con
     if (dt == MOE_BF16) {
         err = launch_ffn_bf16(x_perm, offsets, W1, W3, W2, P, d, h, E, at<void>(ws, L.H), Y,
                               at<float>(ws, L.Ypart), kDecodeSplitK, /*reduce=*/false, &fo,
-                              status, stream, n_ev > 2 ? ev[2] : nullptr);
+                              status, stream, n_ev > 2 ? ev[2] : nullptr,
+                              at<uint32_t>(ws, L.sync));
         if (err == cudaErrorInvalidValue) return MOE_ERR_INVALID_ARG;
     } else {
         err = launch_ffn_f32(static_cast<const float*>(x_perm), offsets,

@@ -19,7 +19,7 @@ constexpr int kPermChunk = 256;
 // Grouped rows at or below which the weight-streaming (swap-AB) expert FFN is used,
 // and how many K ranges its down projection is split into at most.
 constexpr int kDecodeMaxRows = 128;
-constexpr int kDecodeSplitK = 4;
+constexpr int kDecodeSplitK = 8;
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 inline size_t dtype_bytes(moe_dtype dt) { return dt == MOE_BF16 ? 2 : 4; }
@@ -27,7 +27,7 @@ inline size_t dtype_bytes(moe_dtype dt) { return dt == MOE_BF16 ? 2 : 4; }
 // Byte offsets of every workspace region (1 KiB aligned).  The status word sits at
 // offset 0 so that every entry point sharing a workspace reports into one place.
 struct WsLayout {
-    size_t status, topk_idx, topk_w, offsets, blk_counts, blk_base, perm_token, inv_perm,
+    size_t status, sync, topk_idx, topk_w, offsets, blk_counts, blk_base, perm_token, inv_perm,
         x_perm, H, Ypart, Y, total;
     // Bytes needed by moe_permute (status + count/base scratch) and by moe_expert_ffn
     // (status + H); moe_layer_forward needs `total`.
@@ -47,6 +47,8 @@ inline WsLayout ws_layout(int T, int d, int h, int E, int k, moe_dtype dt) {
         return at;
     };
     L.status = take(256);
+    // dependency counters of the fused small-batch FFN (zero between calls)
+    L.sync = take(2 * kMaxExperts * kDecodeSplitK * 4);
     L.blk_counts = take(nb * E * 4);
     L.blk_base = take(nb * E * 4);
     L.permute_need = o;
@@ -124,7 +126,9 @@ cudaError_t launch_ffn_bf16(const void* x_perm, const int32_t* offsets, const vo
                             const void* W3, const void* W2, int rows, int d, int h, int E,
                             void* H, float* Y, float* partials, int partial_cap, bool reduce,
                             FfnOut* out, uint32_t* status, cudaStream_t s,
-                            cudaEvent_t between = nullptr);
+                            cudaEvent_t between = nullptr, uint32_t* counters = nullptr);
+// With `counters` (2 * kMaxExperts * kDecodeSplitK zeroed words, left zeroed) small
+// batches run the fused single-launch FFN; `between` is then recorded after it.
 // Large-batch expert FFN on CTA pairs (tcgen05 cta_group::2).
 cudaError_t launch_ffn_bf16_pair(const void* x_perm, const int32_t* offsets, const void* W1,
                                  const void* W3, const void* W2, int rows, int d, int h, int E,
@@ -133,6 +137,12 @@ cudaError_t launch_ffn_bf16_pair(const void* x_perm, const int32_t* offsets, con
 // Grouped rows from which the CTA-pair kernels are used (MOE_GEMM_PAIR=0 disables them).
 constexpr int kPairMinRows = 2048;
 bool pair_gemm_enabled();
+// Small-batch expert FFN as one cooperative launch (gate/up and split-K down units
+// with per-(expert, K range) dependency counters, 2*E*ksplit zeroed words).
+cudaError_t launch_ffn_bf16_decode_fused(const void* x_perm, const int32_t* offsets,
+                                         const void* W1, const void* W3, const void* W2, int rows,
+                                         int d, int h, int E, void* H, float* Ypart, int ksplit,
+                                         uint32_t* counters, uint32_t* status, cudaStream_t s);
 // Small-batch expert FFN; the down projection writes `ksplit` partial arrays.
 cudaError_t launch_ffn_bf16_decode(const void* x_perm, const int32_t* offsets, const void* W1,
                                    const void* W3, const void* W2, int rows, int d, int h, int E,
