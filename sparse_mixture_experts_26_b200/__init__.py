@@ -35,8 +35,9 @@ EXPORTED_SYMBOLS = ("moe_workspace_bytes", "moe_route", "moe_permute", "moe_expe
                     "moe_device_status", "moe_status_string", "moe_expert_ffn_static")
 def launches_per_layer(T: int) -> int:
     """Kernels one moe_layer_forward queues: router 1, permutation 1 (T <= 512) or 4
-    (count, scan, rank, gather), expert FFN 2 (gate/up + SwiGLU, down), combine 1."""
-    return 1 + (1 if T <= 512 else 4) + 2 + 1
+    (count, scan, rank, gather), expert FFN 1 (T <= 64: gate/up and down fused) or 2,
+    combine 1."""
+    return 1 + (1 if T <= 512 else 4) + (1 if T <= 64 else 2) + 1
 
 
 class MoeError(RuntimeError):
