@@ -66,6 +66,8 @@ __all__ = [
     "moe_layer",
     "moe_layer_dense",
     "mixtral_param_counts",
+    "capacity_keep",
+    "capacity_from_factor",
 ]
 
 
@@ -242,8 +244,44 @@ def combine(Y, inv_perm, w) -> np.ndarray:
     return y
 
 
-def moe_layer(x, Wg, W1, W3, W2, k: int = 2) -> dict:
+def capacity_from_factor(factor: float, T: int, k: int, E: int) -> int:
+    """Per-expert capacity for a capacity factor: ceil(factor * T * k / E) rows.
+
+    ml-canon "52 Mixtral", "Questions worth asking": a capacity factor caps the
+    tokens each expert takes (the pages give no formula; this is the usual one:
+    the factor times an even share of the T*k (token, slot) pairs).
+    """
+    import math
+    return int(math.ceil(factor * T * k / E))
+
+
+def capacity_keep(idx, E: int, capacity) -> np.ndarray:
+    """Boolean ``[T, k]``: is pair (t, j) within its expert's capacity?
+
+    Reading (the pages only say "a cap on tokens per expert"): each expert keeps the
+    first ``capacity`` of its pairs in the stable grouping order (ascending token,
+    then slot) and drops the rest.  ``capacity=None`` keeps everything.
+    """
+    idx = np.asarray(idx)
+    keep = np.ones(idx.shape, dtype=bool)
+    if capacity is None:
+        return keep
+    T, k = idx.shape
+    seen = np.zeros(E, dtype=np.int64)
+    for t in range(T):
+        for j in range(k):
+            e = int(idx[t, j])
+            keep[t, j] = seen[e] < capacity
+            seen[e] += 1
+    return keep
+
+
+def moe_layer(x, Wg, W1, W3, W2, k: int = 2, capacity=None) -> dict:
     """The routed layer (oracle O1): route, group by expert, SwiGLU per group, combine.
+
+    With ``capacity`` (opt-in), a pair beyond its expert's capacity is dropped: its
+    expert output is not computed and it contributes nothing to y; the other
+    weights are left as they are (see ``capacity_keep``).
 
     Returns a dict with every intermediate: ``logits`` (fp64), ``idx`` (int32
     ``[T, k]``), ``w`` (fp64), ``w_f32`` (float32 as stored by the layer),
@@ -256,10 +294,21 @@ def moe_layer(x, Wg, W1, W3, W2, k: int = 2) -> dict:
     w = gate_weights(logits, idx)
     offsets, perm_token, inv_perm = permutation(idx, E)
     x_perm = gather_rows(_f64(x), perm_token)
-    Y = expert_ffn_grouped(x_perm, offsets, W1, W3, W2)
-    y = combine(Y, inv_perm, w)
+    keep = capacity_keep(idx, E, capacity)
+    if capacity is not None:
+        # only the first `capacity` rows of each group are run through the expert
+        Y = np.zeros((x_perm.shape[0], x_perm.shape[1]), dtype=np.float64)
+        for e in range(E):
+            lo = int(offsets[e])
+            hi = min(int(offsets[e + 1]), lo + int(capacity))
+            if hi > lo:
+                Y[lo:hi] = expert_swiglu(x_perm[lo:hi], W1[e], W3[e], W2[e])
+    else:
+        Y = expert_ffn_grouped(x_perm, offsets, W1, W3, W2)
+    y = combine(Y, inv_perm, w * keep)
     return dict(logits=logits, idx=idx, w=w, w_f32=gate_weights_f32(logits, idx),
-                offsets=offsets, perm_token=perm_token, inv_perm=inv_perm, Y=Y, y=y)
+                offsets=offsets, perm_token=perm_token, inv_perm=inv_perm, Y=Y, y=y,
+                keep=keep)
 
 
 def moe_layer_dense(x, Wg, W1, W3, W2, k: int = 2) -> np.ndarray:

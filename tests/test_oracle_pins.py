@@ -335,3 +335,51 @@ def test_param_counts_match_the_pages():
             v, dec = g[f"{key}_{src}"]
             assert round(n / 1e9, dec) == v, (key, src, n)
     assert c["total"] == 46_702_792_704 and c["active"] == 12_879_925_248
+
+
+# ---------------------------------------------------------------- capacity (opt-in)
+
+def _capped_by_loops(inp, capacity):
+    """Per token, by loops: keep pair (t, j) iff fewer than `capacity` earlier pairs
+    (in token, then slot order) went to the same expert; sum the kept experts."""
+    l = O.router_logits(inp["x"], inp["Wg"])
+    idx = O.top2_select(l)
+    w = O.gate_weights(l, idx)
+    E = inp["Wg"].shape[1]
+    seen = [0] * E
+    y = np.zeros(inp["x"].shape)
+    for t in range(idx.shape[0]):
+        for j in range(2):
+            e = int(idx[t, j])
+            if seen[e] < capacity:
+                y[t] += w[t, j] * O.expert_swiglu(inp["x"][t:t + 1], inp["W1"][e], inp["W3"][e],
+                                                  inp["W2"][e])[0]
+            seen[e] += 1
+    return y
+
+
+@pytest.mark.parametrize("capacity", [0, 1, 3, 7, 1000])
+def test_capacity_matches_per_token_loops(capacity):
+    inp = _inputs(small("cap", T=29, d=16, h=24, seed=4, kind="skew"))
+    out = O.moe_layer(**inp, capacity=capacity)
+    np.testing.assert_allclose(out["y"], _capped_by_loops(inp, capacity), rtol=1e-12, atol=1e-14)
+
+
+def test_capacity_special_cases():
+    inp = _inputs(small("cap2", T=40, d=16, h=24, seed=6, kind="skew"))
+    full = O.moe_layer(**inp)
+    counts = np.diff(full["offsets"])
+    # a capacity at or above every group's size changes nothing
+    big = O.moe_layer(**inp, capacity=int(counts.max()))
+    np.testing.assert_array_equal(big["y"], full["y"])
+    assert big["keep"].all()
+    # capacity 0 drops everything
+    np.testing.assert_array_equal(O.moe_layer(**inp, capacity=0)["y"], 0.0)
+    # the number of kept pairs per expert is min(count, capacity)
+    for c in (1, 4, 9):
+        keep = O.capacity_keep(full["idx"], 8, c)
+        kept = np.bincount(full["idx"][keep].ravel(), minlength=8)
+        np.testing.assert_array_equal(kept, np.minimum(counts, c))
+    assert O.capacity_from_factor(1.0, 4096, 2, 8) == 1024
+    assert O.capacity_from_factor(1.25, 4096, 2, 8) == 1280
+    assert O.capacity_from_factor(1.25, 10, 2, 8) == 4
