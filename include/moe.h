@@ -153,6 +153,19 @@ moe_status moe_layer_forward(const void *x, const void *Wg, const void *W1,
                              int E, int k, moe_dtype dt, void *y, void *ws,
                              size_t ws_bytes, cudaStream_t stream);
 
+/* The layer with an opt-in per-expert capacity (token dropping).  ml-canon "52
+ * Mixtral", "Questions worth asking": a capacity factor caps the tokens each expert
+ * takes.  Each expert keeps the first `capacity` of its (token, slot) pairs in the
+ * grouping order (ascending token, then slot); a dropped pair's expert output is
+ * not computed and contributes nothing to y, and the other gate weight of that
+ * token is not renormalised.  capacity < 0 means no limit (= moe_layer_forward); a
+ * capacity factor f corresponds to capacity = ceil(f * T * k / E).  Other
+ * arguments as moe_layer_forward. */
+moe_status moe_layer_forward_capacity(const void *x, const void *Wg, const void *W1,
+                                      const void *W3, const void *W2, int T, int d, int h,
+                                      int E, int k, moe_dtype dt, int capacity, void *y,
+                                      void *ws, size_t ws_bytes, cudaStream_t stream);
+
 /* moe_layer_forward that also records up to five caller-created events on `stream`
  * between its stages, for timing them without a profiler:
  *   events[0] before the router, events[1] after the permutation (before the

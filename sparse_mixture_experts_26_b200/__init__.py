@@ -23,6 +23,7 @@ __all__ = [
     "moe_expert_ffn", "moe_combine", "moe_layer_forward", "moe_device_status",
     "moe_status_string", "moe_layer_forward_events", "alloc_workspace", "layer_forward",
     "EXPORTED_SYMBOLS", "launches_per_layer", "moe_expert_ffn_static",
+    "moe_layer_forward_capacity",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe.so")
@@ -32,7 +33,8 @@ _STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED"
                  3: "MOE_ERR_WORKSPACE", 4: "MOE_ERR_CUDA", 5: "MOE_ERR_TIMEOUT"}
 EXPORTED_SYMBOLS = ("moe_workspace_bytes", "moe_route", "moe_permute", "moe_expert_ffn",
                     "moe_combine", "moe_layer_forward", "moe_layer_forward_events",
-                    "moe_device_status", "moe_status_string", "moe_expert_ffn_static")
+                    "moe_device_status", "moe_status_string", "moe_expert_ffn_static",
+                    "moe_layer_forward_capacity")
 def launches_per_layer(T: int) -> int:
     """Kernels one moe_layer_forward queues: router 1, permutation 1 (T <= 512) or 4
     (count, scan, rank, gather), expert FFN 1 (T <= 64: gate/up and down fused) or 2,
@@ -66,6 +68,8 @@ def _load() -> ctypes.CDLL:
         "moe_device_status": (i32, [vp, sz, u32p, vp]),
         "moe_status_string": (ctypes.c_char_p, [i32]),
         "moe_expert_ffn_static": (i32, [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, vp, vp]),
+        "moe_layer_forward_capacity": (i32, [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
+                                             i32, vp, vp, sz, vp]),
     }
     for name, (res, args) in sigs.items():
         f = getattr(lib, name)
@@ -168,6 +172,18 @@ def moe_layer_forward(x, Wg, W1, W3, W2, y, ws, k: int = 2, stream=None) -> None
     _check("moe_layer_forward", _lib.moe_layer_forward(
         _ptr(x), _ptr(Wg), _ptr(W1), _ptr(W3), _ptr(W2), T, d, h, E, k, _dt(x), _ptr(y),
         _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def moe_layer_forward_capacity(x, Wg, W1, W3, W2, y, ws, capacity: int, k: int = 2,
+                               stream=None) -> None:
+    """The layer with each expert keeping at most ``capacity`` (token, slot) pairs, in
+    token order; dropped pairs contribute nothing.  ``capacity < 0``: no limit."""
+    _dev(x, Wg, W1, W3, W2, y, ws)
+    T, d = x.shape
+    E, h, _ = W1.shape
+    _check("moe_layer_forward_capacity", _lib.moe_layer_forward_capacity(
+        _ptr(x), _ptr(Wg), _ptr(W1), _ptr(W3), _ptr(W2), T, d, h, E, k, _dt(x), int(capacity),
+        _ptr(y), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
 
 
 def moe_layer_forward_events(x, Wg, W1, W3, W2, y, ws, events, k: int = 2,

@@ -47,7 +47,8 @@ template <typename Tout>
 __global__ void __launch_bounds__(kCombineThreads)
     combine_kernel(const float4* __restrict__ Y, int nsplit, size_t split_stride4,
                    const int32_t* __restrict__ inv, const float* __restrict__ w, int T, int d4,
-                   Tout* __restrict__ y) {
+                   Tout* __restrict__ y, const int32_t* __restrict__ idx,
+                   const int32_t* __restrict__ offsets, int E, int cap) {
     pdl_wait();
     pdl_launch_dependents();
     const size_t n = static_cast<size_t>(T) * d4;
@@ -58,13 +59,23 @@ __global__ void __launch_bounds__(kCombineThreads)
         const size_t c = i - t * d4;
         const unsigned r0 = static_cast<unsigned>(inv[2 * t]);
         const unsigned r1 = static_cast<unsigned>(inv[2 * t + 1]);
-        const float w0 = w[2 * t], w1 = w[2 * t + 1];
+        float w0 = w[2 * t], w1 = w[2 * t + 1];
+        if (cap != INT_MAX) {
+            // a pair `cap` or more rows into its expert's group was dropped
+            const unsigned e0 = static_cast<unsigned>(idx[2 * t]);
+            const unsigned e1 = static_cast<unsigned>(idx[2 * t + 1]);
+            if (e0 >= static_cast<unsigned>(E) || static_cast<int>(r0) - offsets[e0] >= cap) w0 = 0.f;
+            if (e1 >= static_cast<unsigned>(E) || static_cast<int>(r1) - offsets[e1] >= cap) w1 = 0.f;
+        }
         // inv_perm entries outside [0, 2T) would come from an invalid permutation;
         // they contribute nothing instead of reading out of bounds.
-        const float4 a = r0 < P ? split_sum(Y, nsplit, split_stride4, static_cast<size_t>(r0) * d4 + c)
-                                : make_float4(0, 0, 0, 0);
-        const float4 b = r1 < P ? split_sum(Y, nsplit, split_stride4, static_cast<size_t>(r1) * d4 + c)
-                                : make_float4(0, 0, 0, 0);
+        // dropped pairs (w == 0) are not read: their rows were never written
+        const float4 a = (r0 < P && w0 != 0.f)
+                             ? split_sum(Y, nsplit, split_stride4, static_cast<size_t>(r0) * d4 + c)
+                             : make_float4(0, 0, 0, 0);
+        const float4 b = (r1 < P && w1 != 0.f)
+                             ? split_sum(Y, nsplit, split_stride4, static_cast<size_t>(r1) * d4 + c)
+                             : make_float4(0, 0, 0, 0);
         float4 o;
         o.x = fmaf(w1, b.x, w0 * a.x);
         o.y = fmaf(w1, b.y, w0 * a.y);
@@ -104,16 +115,18 @@ cudaError_t launch_sum_splits(const float* parts, int nsplit, size_t n, float* Y
 
 cudaError_t launch_combine(const float* Y, int nsplit, size_t split_stride,
                            const int32_t* inv_perm, const float* w, int T, int d, moe_dtype dt,
-                           void* y, cudaStream_t s) {
+                           void* y, cudaStream_t s, const int32_t* idx, const int32_t* offsets,
+                           int E, int cap) {
+    if (cap != INT_MAX && (!idx || !offsets)) return cudaErrorInvalidValue;
     const int d4 = d / 4;
     const unsigned blocks = grid_for(static_cast<size_t>(T) * d4);
     if (dt == MOE_BF16)
         return launch_k(combine_kernel<__nv_bfloat16>, blocks, kCombineThreads, 0, s,
                         reinterpret_cast<const float4*>(Y), nsplit, split_stride / 4, inv_perm,
-                        w, T, d4, static_cast<__nv_bfloat16*>(y));
+                        w, T, d4, static_cast<__nv_bfloat16*>(y), idx, offsets, E, cap);
     return launch_k(combine_kernel<float>, blocks, kCombineThreads, 0, s,
                     reinterpret_cast<const float4*>(Y), nsplit, split_stride / 4, inv_perm, w, T,
-                    d4, static_cast<float*>(y));
+                    d4, static_cast<float*>(y), idx, offsets, E, cap);
 }
 
 }  // namespace moe

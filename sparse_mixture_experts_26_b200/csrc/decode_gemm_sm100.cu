@@ -59,6 +59,7 @@ struct DecodeArgs {
     int ksplit;      // K ranges per tile (down GEMM), 1 for gate/up
     void* out;       // H bf16 [rows, N], or ksplit fp32 partials [ksplit][rows][N]
     uint32_t* status;
+    int cap;         // rows kept per group (capacity; INT_MAX = no limit)
 };
 
 template <int MODE, int NT>
@@ -89,6 +90,7 @@ struct DecodeBook {
     uint32_t tmem_base;
     int abort_flag;
     int off[kMaxExperts + 1];
+    int end[kMaxExperts];
     int tile_start[kMaxExperts + 1];
 };
 
@@ -109,7 +111,7 @@ __device__ __forceinline__ Tile decode_tile(const DecodeBook<NACC>& bk, int E, i
     const int chunk = local / nwb;
     t.wb = local - chunk * nwb;
     t.row0 = bk.off[g] + chunk * NTc;
-    const int left = bk.off[g + 1] - t.row0;
+    const int left = bk.end[g] - t.row0;
     t.nvalid = left < NTc ? left : NTc;
     return t;
 }
@@ -201,7 +203,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         bk.tile_start[0] = 0;
         for (int g = 0; g < E; ++g) {
-            const int chunks = (bk.off[g + 1] - bk.off[g] + NT - 1) / NT;
+            const int n = bk.off[g + 1] - bk.off[g];
+            bk.end[g] = bk.off[g] + (n < args.cap ? n : args.cap);
+            const int chunks = (bk.end[g] - bk.off[g] + NT - 1) / NT;
             bk.tile_start[g + 1] = bk.tile_start[g] + chunks * args.n_wblocks * ksplit;
         }
     }
@@ -410,6 +414,7 @@ struct FusedArgs {
     uint32_t* ready;    // [E][ksplit]
     uint32_t* readers;  // [E][ksplit]
     uint32_t* status;
+    int cap;            // rows kept per group (capacity; INT_MAX = no limit)
 };
 
 template <int NACC>
@@ -422,6 +427,7 @@ struct FusedBook {
     uint32_t tmem_base;
     int abort_flag;
     int off[kMaxExperts + 1];
+    int end[kMaxExperts];         // end of the rows kept in group g (capacity)
     int start1[kMaxExperts + 1];  // gate/up tiles before expert g
     int start2[kMaxExperts + 1];  // down units before expert g
 };
@@ -462,8 +468,8 @@ __device__ __forceinline__ FusedUnit fused_unit(const FusedBook<NACC>& bk, const
         f.kb1 = min(num_kb2, f.kb0 + kps);
     }
     f.e = g;
-    f.chunks = (bk.off[g + 1] - bk.off[g] + NTc - 1) / NTc;
-    const int left = bk.off[g + 1] - f.row0;
+    f.chunks = (bk.end[g] - bk.off[g] + NTc - 1) / NTc;
+    const int left = bk.end[g] - f.row0;
     f.nvalid = left < NTc ? left : NTc;
     return f;
 }
@@ -538,7 +544,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         bk.start1[0] = 0;
         bk.start2[0] = 0;
         for (int g = 0; g < E; ++g) {
-            const int chunks = (bk.off[g + 1] - bk.off[g] + NT - 1) / NT;
+            const int n = bk.off[g + 1] - bk.off[g];
+            bk.end[g] = bk.off[g] + (n < args.cap ? n : args.cap);
+            const int chunks = (bk.end[g] - bk.off[g] + NT - 1) / NT;
             bk.start1[g + 1] = bk.start1[g] + chunks * args.n_hb;
             bk.start2[g + 1] = bk.start2[g] + chunks * args.n_db * args.ksplit;
         }
@@ -744,7 +752,7 @@ template <int NT>
 cudaError_t launch_ffn_fused_nt(const void* x_perm, const int32_t* offsets, const void* W1,
                                 const void* W3, const void* W2, int rows, int d, int h, int E,
                                 void* H, float* Ypart, int ksplit, uint32_t* counters,
-                                uint32_t* status, cudaStream_t s) {
+                                uint32_t* status, cudaStream_t s, int cap) {
     CUtensorMap mw1, mw3, mx, mw2, mh;
     if (!encode_bf16_2d(&mw1, W1, static_cast<uint64_t>(E) * h, d, kM / 2) ||
         !encode_bf16_2d(&mw3, W3, static_cast<uint64_t>(E) * h, d, kM / 2) ||
@@ -762,7 +770,7 @@ cudaError_t launch_ffn_fused_nt(const void* x_perm, const int32_t* offsets, cons
         configured[dev] = 1;
     }
     FusedArgs a{offsets, E, rows, d, h, (h + 63) / 64, (d + kM - 1) / kM, ksplit, H, Ypart,
-                counters, counters + E * ksplit, status};
+                counters, counters + E * ksplit, status, cap};
     const int sms = device_sm_count();
     const long long chunks = static_cast<long long>(rows) / NT + E;
     const long long units = chunks * (a.n_hb + static_cast<long long>(a.n_db) * ksplit);
@@ -786,7 +794,7 @@ template <int NT>
 cudaError_t launch_ffn_decode_nt(const void* x_perm, const int32_t* offsets, const void* W1,
                                  const void* W3, const void* W2, int rows, int d, int h, int E,
                                  void* H, float* Yout, int ksplit, uint32_t* status,
-                                 cudaStream_t s, cudaEvent_t between) {
+                                 cudaStream_t s, cudaEvent_t between, int cap) {
     constexpr int J1 = DecodeCfg<kSwiGLU, NT>::kJ, J2 = DecodeCfg<kDown, NT>::kJ;
     CUtensorMap mw1, mw3, mx, mw2, mh;
     if (!encode_bf16_2d(&mw1, W1, static_cast<uint64_t>(E) * h, d, J1) ||
@@ -798,13 +806,13 @@ cudaError_t launch_ffn_decode_nt(const void* x_perm, const int32_t* offsets, con
     const int sms = device_sm_count();
     // Units per launch are at most (rows/NT + E) * weight blocks * K ranges.
     const long long chunks = static_cast<long long>(rows) / NT + E;
-    DecodeArgs a1{offsets, E, rows, d, h, h, (h + J1 - 1) / J1, 1, H, status};
+    DecodeArgs a1{offsets, E, rows, d, h, h, (h + J1 - 1) / J1, 1, H, status, cap};
     const long long t1 = chunks * a1.n_wblocks;
     cudaError_t err = launch_decode<kSwiGLU, NT>(mw1, mw3, mx, a1,
                                                   static_cast<int>(t1 < sms ? t1 : sms), s);
     if (err != cudaSuccess) return err;
     if (between && (err = cudaEventRecord(between, s)) != cudaSuccess) return err;
-    DecodeArgs a2{offsets, E, rows, h, d, d, (d + J2 - 1) / J2, ksplit, Yout, status};
+    DecodeArgs a2{offsets, E, rows, h, d, d, (d + J2 - 1) / J2, ksplit, Yout, status, cap};
     const long long t2 = chunks * a2.n_wblocks * ksplit;
     return launch_decode<kDown, NT>(mw2, mw2, mh, a2, static_cast<int>(t2 < sms ? t2 : sms), s);
 }
@@ -814,31 +822,32 @@ cudaError_t launch_ffn_decode_nt(const void* x_perm, const int32_t* offsets, con
 cudaError_t launch_ffn_bf16_decode_fused(const void* x_perm, const int32_t* offsets,
                                          const void* W1, const void* W3, const void* W2, int rows,
                                          int d, int h, int E, void* H, float* Ypart, int ksplit,
-                                         uint32_t* counters, uint32_t* status, cudaStream_t s) {
+                                         uint32_t* counters, uint32_t* status, cudaStream_t s,
+                                         int cap) {
     const int T = rows / 2;
     if (T <= 16)
         return launch_ffn_fused_nt<16>(x_perm, offsets, W1, W3, W2, rows, d, h, E, H, Ypart,
-                                       ksplit, counters, status, s);
+                                       ksplit, counters, status, s, cap);
     if (T <= 32)
         return launch_ffn_fused_nt<32>(x_perm, offsets, W1, W3, W2, rows, d, h, E, H, Ypart,
-                                       ksplit, counters, status, s);
+                                       ksplit, counters, status, s, cap);
     return launch_ffn_fused_nt<64>(x_perm, offsets, W1, W3, W2, rows, d, h, E, H, Ypart, ksplit,
-                                   counters, status, s);
+                                   counters, status, s, cap);
 }
 
 cudaError_t launch_ffn_bf16_decode(const void* x_perm, const int32_t* offsets, const void* W1,
                                    const void* W3, const void* W2, int rows, int d, int h, int E,
                                    void* H, float* Yout, int ksplit, uint32_t* status,
-                                   cudaStream_t s, cudaEvent_t between) {
+                                   cudaStream_t s, cudaEvent_t between, int cap) {
     const int T = rows / 2;  // a group holds each token at most once
     if (T <= 16)
         return launch_ffn_decode_nt<16>(x_perm, offsets, W1, W3, W2, rows, d, h, E, H, Yout,
-                                        ksplit, status, s, between);
+                                        ksplit, status, s, between, cap);
     if (T <= 32)
         return launch_ffn_decode_nt<32>(x_perm, offsets, W1, W3, W2, rows, d, h, E, H, Yout,
-                                        ksplit, status, s, between);
+                                        ksplit, status, s, between, cap);
     return launch_ffn_decode_nt<64>(x_perm, offsets, W1, W3, W2, rows, d, h, E, H, Yout, ksplit,
-                                    status, s, between);
+                                    status, s, between, cap);
 }
 
 }  // namespace moe

@@ -30,7 +30,7 @@ __device__ __forceinline__ float warp_sum(float v) {
 __global__ void __launch_bounds__(kFfnThreads)
     ffn1_f32_kernel(const float* __restrict__ xp, const int32_t* __restrict__ offsets,
                     const float* __restrict__ W1, const float* __restrict__ W3, int rows, int d,
-                    int h, int E, float* __restrict__ H) {
+                    int h, int E, int cap, float* __restrict__ H) {
     pdl_wait();
     pdl_launch_dependents();
     __shared__ int s_off[kMaxExperts + 1];
@@ -44,6 +44,7 @@ __global__ void __launch_bounds__(kFfnThreads)
         const int r = static_cast<int>(o / h);
         const int j = static_cast<int>(o - static_cast<size_t>(r) * h);
         const int e = group_of(s_off, E, r);
+        if (r - s_off[e] >= cap) continue;  // beyond the expert's capacity (warp-uniform)
         const float* xr = xp + static_cast<size_t>(r) * d;
         const float* w1 = W1 + (static_cast<size_t>(e) * h + j) * d;
         const float* w3 = W3 + (static_cast<size_t>(e) * h + j) * d;
@@ -61,7 +62,7 @@ __global__ void __launch_bounds__(kFfnThreads)
 
 __global__ void __launch_bounds__(kFfnThreads)
     ffn2_f32_kernel(const float* __restrict__ H, const int32_t* __restrict__ offsets,
-                    const float* __restrict__ W2, int rows, int d, int h, int E,
+                    const float* __restrict__ W2, int rows, int d, int h, int E, int cap,
                     float* __restrict__ Y) {
     pdl_wait();
     pdl_launch_dependents();
@@ -76,6 +77,7 @@ __global__ void __launch_bounds__(kFfnThreads)
         const int r = static_cast<int>(o / d);
         const int c = static_cast<int>(o - static_cast<size_t>(r) * d);
         const int e = group_of(s_off, E, r);
+        if (r - s_off[e] >= cap) continue;
         const float* hr = H + static_cast<size_t>(r) * h;
         const float* w2 = W2 + (static_cast<size_t>(e) * d + c) * h;
         float acc = 0.f;
@@ -89,19 +91,19 @@ __global__ void __launch_bounds__(kFfnThreads)
 
 cudaError_t launch_ffn_f32(const float* x_perm, const int32_t* offsets, const float* W1,
                            const float* W3, const float* W2, int rows, int d, int h, int E,
-                           float* H, float* Y, cudaStream_t s, cudaEvent_t between) {
+                           float* H, float* Y, cudaStream_t s, cudaEvent_t between, int cap) {
     const int warps = kFfnThreads / 32;
-    const size_t cap = static_cast<size_t>(device_sm_count()) * 16;
+    const size_t max_blocks = static_cast<size_t>(device_sm_count()) * 16;
     size_t b1 = (static_cast<size_t>(rows) * h + warps - 1) / warps;
     size_t b2 = (static_cast<size_t>(rows) * d + warps - 1) / warps;
-    b1 = b1 > cap ? cap : (b1 < 1 ? 1 : b1);
-    b2 = b2 > cap ? cap : (b2 < 1 ? 1 : b2);
+    b1 = b1 > max_blocks ? max_blocks : (b1 < 1 ? 1 : b1);
+    b2 = b2 > max_blocks ? max_blocks : (b2 < 1 ? 1 : b2);
     cudaError_t err = launch_k(ffn1_f32_kernel, static_cast<unsigned>(b1), kFfnThreads, 0, s,
-                               x_perm, offsets, W1, W3, rows, d, h, E, H);
+                               x_perm, offsets, W1, W3, rows, d, h, E, cap, H);
     if (err != cudaSuccess) return err;
     if (between && (err = cudaEventRecord(between, s)) != cudaSuccess) return err;
     return launch_k(ffn2_f32_kernel, static_cast<unsigned>(b2), kFfnThreads, 0, s, H, offsets,
-                    W2, rows, d, h, E, Y);
+                    W2, rows, d, h, E, cap, Y);
 }
 
 }  // namespace moe

@@ -72,6 +72,7 @@ struct PairArgs {
     int n_tiles;  // column tiles per row block
     void* out;
     uint32_t* status;
+    int cap;      // rows kept per group (capacity; INT_MAX = no limit)
 };
 
 struct PairBook {
@@ -83,6 +84,7 @@ struct PairBook {
     uint32_t tmem_base;
     int abort_flag;
     int off[kMaxExperts + 1];
+    int end[kMaxExperts];
     int tile_start[kMaxExperts + 1];
 };
 static_assert(sizeof(PairBook) <= 1024, "bookkeeping reserve");
@@ -96,12 +98,12 @@ __device__ __forceinline__ PairTile decode_pair_tile(const PairBook& bk, int E, 
     int g = 0;
     while (g + 1 < E && tile >= bk.tile_start[g + 1]) ++g;
     const int local = tile - bk.tile_start[g];
-    const int blocks = (bk.off[g + 1] - bk.off[g] + kPairRows - 1) / kPairRows;
+    const int blocks = (bk.end[g] - bk.off[g] + kPairRows - 1) / kPairRows;
     PairTile t;
     t.e = g;
     t.row0 = bk.off[g] + (local % blocks) * kPairRows;
     t.nt = local / blocks;
-    t.row_end = bk.off[g + 1];
+    t.row_end = bk.end[g];
     t.half = t.row_end - t.row0 <= kRowsPerCta;
     return t;
 }
@@ -182,10 +184,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             prev = v;
         }
         bk.tile_start[0] = 0;
-        for (int g = 0; g < E; ++g)
+        for (int g = 0; g < E; ++g) {
+            const int n = bk.off[g + 1] - bk.off[g];
+            bk.end[g] = bk.off[g] + (n < args.cap ? n : args.cap);
             bk.tile_start[g + 1] = bk.tile_start[g] +
-                                   (bk.off[g + 1] - bk.off[g] + kPairRows - 1) / kPairRows *
+                                   (bk.end[g] - bk.off[g] + kPairRows - 1) / kPairRows *
                                        args.n_tiles;
+        }
     }
     tc_fence_before();
     __syncthreads();
@@ -458,7 +463,7 @@ cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b0, const CUten
 cudaError_t launch_ffn_bf16_pair(const void* x_perm, const int32_t* offsets, const void* W1,
                                  const void* W3, const void* W2, int rows, int d, int h, int E,
                                  void* H, float* Y, uint32_t* status, cudaStream_t s,
-                                 cudaEvent_t between) {
+                                 cudaEvent_t between, int cap) {
     CUtensorMap mx, mw1, mw3, mh, mw2;
     if (!encode_bf16_2d(&mx, x_perm, rows, d, kRowsPerCta) ||
         !encode_bf16_2d(&mw1, W1, static_cast<uint64_t>(E) * h, d, 128) ||
@@ -468,13 +473,13 @@ cudaError_t launch_ffn_bf16_pair(const void* x_perm, const int32_t* offsets, con
         return cudaErrorInvalidValue;
     const int max_pairs = device_sm_count() / 2;
     const long long blocks = (static_cast<long long>(rows) + (kPairRows - 1LL) * E) / kPairRows;
-    PairArgs g1{offsets, E, rows, d, h, h, (h + 127) / 128, H, status};
+    PairArgs g1{offsets, E, rows, d, h, h, (h + 127) / 128, H, status, cap};
     long long t1 = blocks * g1.n_tiles;
     cudaError_t err = launch_pair<kEpiSwiGLU>(
         mx, mw1, mw3, g1, static_cast<int>(t1 < max_pairs ? (t1 < 1 ? 1 : t1) : max_pairs), s);
     if (err != cudaSuccess) return err;
     if (between && (err = cudaEventRecord(between, s)) != cudaSuccess) return err;
-    PairArgs g2{offsets, E, rows, h, d, d, (d + 255) / 256, Y, status};
+    PairArgs g2{offsets, E, rows, h, d, d, (d + 255) / 256, Y, status, cap};
     long long t2 = blocks * g2.n_tiles;
     return launch_pair<kEpiStoreF32>(
         mh, mw2, mw2, g2, static_cast<int>(t2 < max_pairs ? (t2 < 1 ? 1 : t2) : max_pairs), s);

@@ -67,6 +67,7 @@ struct GemmArgs {
     int n_tiles;        // output-column tiles per row block
     void* out;          // H (bf16) or Y (fp32), row-major [rows, N]
     uint32_t* status;   // workspace status word
+    int cap;            // rows kept per group (capacity; INT_MAX = no limit)
 };
 
 struct Bookkeeping {
@@ -78,6 +79,7 @@ struct Bookkeeping {
     uint32_t tmem_base;
     int abort_flag;
     int off[kMaxExperts + 1];        // sanitised group offsets
+    int end[kMaxExperts];            // end of the rows kept in group g (capacity)
     int tile_start[kMaxExperts + 1]; // prefix sum of tiles per group
 };
 static_assert(sizeof(Bookkeeping) <= 1024, "bookkeeping must fit its reserve");
@@ -90,12 +92,12 @@ __device__ __forceinline__ TileCoord decode_tile(const Bookkeeping& bk, int E, i
     int g = 0;
     while (g + 1 < E && tile >= bk.tile_start[g + 1]) ++g;
     const int local = tile - bk.tile_start[g];
-    const int m_tiles = (bk.off[g + 1] - bk.off[g] + kBM - 1) / kBM;
+    const int m_tiles = (bk.end[g] - bk.off[g] + kBM - 1) / kBM;
     TileCoord c;
     c.e = g;
     c.row0 = bk.off[g] + (local % m_tiles) * kBM;  // row blocks inner: weight tile reuse
     c.nt = local / m_tiles;
-    c.row_end = bk.off[g + 1];
+    c.row_end = bk.end[g];
     return c;
 }
 
@@ -168,11 +170,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             bk.off[g] = v;
             prev = v;
         }
-        bk.off[E] = args.rows > prev ? prev : args.rows;
         bk.tile_start[0] = 0;
-        for (int g = 0; g < E; ++g)
+        for (int g = 0; g < E; ++g) {
+            const int n = bk.off[g + 1] - bk.off[g];
+            bk.end[g] = bk.off[g] + (n < args.cap ? n : args.cap);
             bk.tile_start[g + 1] =
-                bk.tile_start[g] + (bk.off[g + 1] - bk.off[g] + kBM - 1) / kBM * args.n_tiles;
+                bk.tile_start[g] + (bk.end[g] - bk.off[g] + kBM - 1) / kBM * args.n_tiles;
+        }
     }
     tc_fence_before();
     __syncthreads();
@@ -403,7 +407,7 @@ cudaError_t launch_ffn_bf16(const void* x_perm, const int32_t* offsets, const vo
                             const void* W3, const void* W2, int rows, int d, int h, int E,
                             void* H, float* Y, float* partials, int partial_cap, bool reduce,
                             FfnOut* out, uint32_t* status, cudaStream_t s,
-                            cudaEvent_t between, uint32_t* counters) {
+                            cudaEvent_t between, uint32_t* counters, int cap) {
     if (rows <= kDecodeMaxRows) {
         // Largest split of the down projection's K blocks (at most partial_cap) that
         // leaves no K range empty.
@@ -413,13 +417,18 @@ cudaError_t launch_ffn_bf16(const void* x_perm, const int32_t* offsets, const vo
         if (ksplit < 1) ksplit = 1;
         float* dst = ksplit > 1 ? partials : Y;
         cudaError_t err;
+        err = cudaErrorNotSupported;
         if (counters) {
             err = launch_ffn_bf16_decode_fused(x_perm, offsets, W1, W3, W2, rows, d, h, E, H, dst,
-                                               ksplit, counters, status, s);
-            if (err == cudaSuccess && between) err = cudaEventRecord(between, s);
-        } else {
+                                               ksplit, counters, status, s, cap);
+            if (err == cudaErrorCooperativeLaunchTooLarge || err == cudaErrorNotSupported)
+                cudaGetLastError();  // clear it: the two-launch path below needs no co-residency
+            else if (err == cudaSuccess && between)
+                err = cudaEventRecord(between, s);
+        }
+        if (err == cudaErrorCooperativeLaunchTooLarge || err == cudaErrorNotSupported) {
             err = launch_ffn_bf16_decode(x_perm, offsets, W1, W3, W2, rows, d, h, E, H, dst,
-                                         ksplit, status, s, between);
+                                         ksplit, status, s, between, cap);
         }
         if (err != cudaSuccess) return err;
         if (ksplit > 1 && reduce) {
@@ -434,7 +443,7 @@ cudaError_t launch_ffn_bf16(const void* x_perm, const int32_t* offsets, const vo
     if (out) *out = FfnOut{Y, 1};
     if (rows >= kPairMinRows && pair_gemm_enabled())
         return launch_ffn_bf16_pair(x_perm, offsets, W1, W3, W2, rows, d, h, E, H, Y, status, s,
-                                    between);
+                                    between, cap);
     CUtensorMap mx, mw1, mw3, mh, mw2;
     if (!encode_bf16_2d(&mx, x_perm, rows, d, kBM) ||
         !encode_bf16_2d(&mw1, W1, static_cast<uint64_t>(E) * h, d, 128) ||
@@ -447,14 +456,14 @@ cudaError_t launch_ffn_bf16(const void* x_perm, const int32_t* offsets, const vo
     // Upper bound on row blocks: sum_e ceil(n_e / 128) <= (rows + 127 E) / 128.
     const long long row_blocks = (static_cast<long long>(rows) + 127LL * E) / kBM;
 
-    GemmArgs g1{offsets, E, rows, d, h, h, (h + 127) / 128, H, status};
+    GemmArgs g1{offsets, E, rows, d, h, h, (h + 127) / 128, H, status, cap};
     long long tiles1 = row_blocks * g1.n_tiles;
     int grid1 = static_cast<int>(tiles1 < sms ? (tiles1 < 1 ? 1 : tiles1) : sms);
     cudaError_t err = launch_gemm<kEpiSwiGLU>(mx, mw1, mw3, g1, grid1, s);
     if (err != cudaSuccess) return err;
     if (between && (err = cudaEventRecord(between, s)) != cudaSuccess) return err;
 
-    GemmArgs g2{offsets, E, rows, h, d, d, (d + 255) / 256, Y, status};
+    GemmArgs g2{offsets, E, rows, h, d, d, (d + 255) / 256, Y, status, cap};
     long long tiles2 = row_blocks * g2.n_tiles;
     int grid2 = static_cast<int>(tiles2 < sms ? (tiles2 < 1 ? 1 : tiles2) : sms);
     return launch_gemm<kEpiStoreF32>(mh, mw2, mw2, g2, grid2, s);

@@ -209,7 +209,7 @@ namespace {
 moe_status layer_forward_impl(const void* x, const void* Wg, const void* W1, const void* W3,
                               const void* W2, int T, int d, int h, int E, int k, moe_dtype dt,
                               void* y, void* ws, size_t ws_bytes, cudaEvent_t* ev, int n_ev,
-                              cudaStream_t stream) {
+                              cudaStream_t stream, int cap) {
     moe_status st = check_shape(T, d, h, E, k, dt, true);
     if (st != MOE_OK) return st;
     if (n_ev < 0 || (n_ev > 0 && ev == nullptr)) return MOE_ERR_INVALID_ARG;
@@ -244,18 +244,18 @@ moe_status layer_forward_impl(const void* x, const void* Wg, const void* W1, con
         err = launch_ffn_bf16(x_perm, offsets, W1, W3, W2, P, d, h, E, at<void>(ws, L.H), Y,
                               at<float>(ws, L.Ypart), kDecodeSplitK, /*reduce=*/false, &fo,
                               status, stream, n_ev > 2 ? ev[2] : nullptr,
-                              at<uint32_t>(ws, L.sync));
+                              at<uint32_t>(ws, L.sync), cap);
         if (err == cudaErrorInvalidValue) return MOE_ERR_INVALID_ARG;
     } else {
         err = launch_ffn_f32(static_cast<const float*>(x_perm), offsets,
                              static_cast<const float*>(W1), static_cast<const float*>(W3),
                              static_cast<const float*>(W2), P, d, h, E, at<float>(ws, L.H), Y,
-                             stream, n_ev > 2 ? ev[2] : nullptr);
+                             stream, n_ev > 2 ? ev[2] : nullptr, cap);
     }
     if ((st = finish(err, stream, status)) != MOE_OK) return st;
     if (!mark(3)) return MOE_ERR_CUDA;
     err = launch_combine(fo.Y, fo.nsplit, static_cast<size_t>(P) * d, inv_perm, w, T, d, dt, y,
-                         stream);
+                         stream, idx, offsets, E, cap);
     if ((st = finish(err, stream, status)) != MOE_OK) return st;
     if (!mark(4)) return MOE_ERR_CUDA;
     return MOE_OK;
@@ -270,7 +270,15 @@ moe_status moe_layer_forward(const void* x, const void* Wg, const void* W1, cons
                              const void* W2, int T, int d, int h, int E, int k, moe_dtype dt,
                              void* y, void* ws, size_t ws_bytes, cudaStream_t stream) {
     return layer_forward_impl(x, Wg, W1, W3, W2, T, d, h, E, k, dt, y, ws, ws_bytes, nullptr, 0,
-                              stream);
+                              stream, INT_MAX);
+}
+
+moe_status moe_layer_forward_capacity(const void* x, const void* Wg, const void* W1,
+                                      const void* W3, const void* W2, int T, int d, int h, int E,
+                                      int k, moe_dtype dt, int capacity, void* y, void* ws,
+                                      size_t ws_bytes, cudaStream_t stream) {
+    return layer_forward_impl(x, Wg, W1, W3, W2, T, d, h, E, k, dt, y, ws, ws_bytes, nullptr, 0,
+                              stream, capacity < 0 ? INT_MAX : capacity);
 }
 
 moe_status moe_layer_forward_events(const void* x, const void* Wg, const void* W1,
@@ -278,7 +286,7 @@ moe_status moe_layer_forward_events(const void* x, const void* Wg, const void* W
                                     int k, moe_dtype dt, void* y, void* ws, size_t ws_bytes,
                                     cudaEvent_t* events, int n_events, cudaStream_t stream) {
     return layer_forward_impl(x, Wg, W1, W3, W2, T, d, h, E, k, dt, y, ws, ws_bytes, events,
-                              n_events, stream);
+                              n_events, stream, INT_MAX);
 }
 
 moe_status moe_device_status(void* ws, size_t ws_bytes, uint32_t* flags, cudaStream_t stream) {

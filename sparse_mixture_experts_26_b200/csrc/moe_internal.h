@@ -4,6 +4,7 @@
 
 #include <cuda_runtime.h>
 
+#include <climits>
 #include <cstddef>
 #include <cstdint>
 #include <utility>
@@ -107,9 +108,12 @@ cudaError_t launch_permute(const int32_t* idx, const void* x, int T, int d, int 
                            int32_t* offsets, int32_t* perm_token, int32_t* inv_perm,
                            void* x_perm, int32_t* blk_counts, int32_t* blk_base,
                            uint32_t* status, cudaStream_t s);
+// `cap` (all FFN launchers): rows kept per expert group -- the first `cap` rows of
+// each group are computed, the rest are neither computed nor written.
 cudaError_t launch_ffn_f32(const float* x_perm, const int32_t* offsets, const float* W1,
                            const float* W3, const float* W2, int rows, int d, int h, int E,
-                           float* H, float* Y, cudaStream_t s, cudaEvent_t between = nullptr);
+                           float* H, float* Y, cudaStream_t s, cudaEvent_t between = nullptr,
+                           int cap = INT_MAX);
 // bf16 expert FFN.  The result is the sum of `out->nsplit` fp32 arrays [rows, d]
 // starting at `out->Y`, `rows * d` floats apart: Y itself (nsplit = 1), or -- when
 // the small-batch kernels run and `partials` has room for `partial_cap` of them --
@@ -126,14 +130,15 @@ cudaError_t launch_ffn_bf16(const void* x_perm, const int32_t* offsets, const vo
                             const void* W3, const void* W2, int rows, int d, int h, int E,
                             void* H, float* Y, float* partials, int partial_cap, bool reduce,
                             FfnOut* out, uint32_t* status, cudaStream_t s,
-                            cudaEvent_t between = nullptr, uint32_t* counters = nullptr);
+                            cudaEvent_t between = nullptr, uint32_t* counters = nullptr,
+                            int cap = INT_MAX);
 // With `counters` (2 * kMaxExperts * kDecodeSplitK zeroed words, left zeroed) small
 // batches run the fused single-launch FFN; `between` is then recorded after it.
 // Large-batch expert FFN on CTA pairs (tcgen05 cta_group::2).
 cudaError_t launch_ffn_bf16_pair(const void* x_perm, const int32_t* offsets, const void* W1,
                                  const void* W3, const void* W2, int rows, int d, int h, int E,
                                  void* H, float* Y, uint32_t* status, cudaStream_t s,
-                                 cudaEvent_t between);
+                                 cudaEvent_t between, int cap);
 // Grouped rows from which the CTA-pair kernels are used (MOE_GEMM_PAIR=0 disables them).
 constexpr int kPairMinRows = 2048;
 bool pair_gemm_enabled();
@@ -142,17 +147,21 @@ bool pair_gemm_enabled();
 cudaError_t launch_ffn_bf16_decode_fused(const void* x_perm, const int32_t* offsets,
                                          const void* W1, const void* W3, const void* W2, int rows,
                                          int d, int h, int E, void* H, float* Ypart, int ksplit,
-                                         uint32_t* counters, uint32_t* status, cudaStream_t s);
+                                         uint32_t* counters, uint32_t* status, cudaStream_t s,
+                                         int cap);
 // Small-batch expert FFN; the down projection writes `ksplit` partial arrays.
 cudaError_t launch_ffn_bf16_decode(const void* x_perm, const int32_t* offsets, const void* W1,
                                    const void* W3, const void* W2, int rows, int d, int h, int E,
                                    void* H, float* Yout, int ksplit, uint32_t* status,
-                                   cudaStream_t s, cudaEvent_t between);
+                                   cudaStream_t s, cudaEvent_t between, int cap);
 // y[t] = w0 * S(inv[t,0]) + w1 * S(inv[t,1]) with S(r) the in-order sum of the
-// nsplit arrays Y + i * split_stride at row r.
+// nsplit arrays Y + i * split_stride at row r.  With cap < INT_MAX (and idx,
+// offsets, E given) a pair whose row lies cap or more rows into its expert's group
+// was dropped and contributes nothing.
 cudaError_t launch_combine(const float* Y, int nsplit, size_t split_stride,
                            const int32_t* inv_perm, const float* w, int T, int d, moe_dtype dt,
-                           void* y, cudaStream_t s);
+                           void* y, cudaStream_t s, const int32_t* idx = nullptr,
+                           const int32_t* offsets = nullptr, int E = 0, int cap = INT_MAX);
 // Y[i] = sum over j < nsplit of parts[j * n + i] (in order), for i < n.
 cudaError_t launch_sum_splits(const float* parts, int nsplit, size_t n, float* Y,
                               cudaStream_t s);

@@ -245,3 +245,75 @@ def test_other_expert_counts(E, T):
     ref = O.moe_layer(x_cpu, f64(inp["Wg"]), f64(inp["W1"]), f64(inp["W3"]), f64(inp["W2"]))
     assert rel_fro(f64(g["y"]), ref["y"]) <= BF16_TOL
     assert torch.equal(layer_y(inp), g["y"])
+
+
+def capped_y(inp, capacity):
+    x = inp["x"]
+    T, d = x.shape
+    E, h, _ = inp["W1"].shape
+    ws = moe.alloc_workspace(T, d, h, E, 2, x.dtype, x.device)
+    y = torch.empty_like(x)
+    moe.moe_layer_forward_capacity(x, inp["Wg"], inp["W1"], inp["W3"], inp["W2"], y, ws,
+                                   capacity)
+    assert moe.moe_device_status(ws) == 0
+    return y
+
+
+@pytest.mark.parametrize("T,d,h,kind,cap,dtype", [
+    (16, 256, 384, "skew", 3, "bf16"),       # fused weight-streaming kernel
+    (40, 128, 256, "skew", 5, "bf16"),
+    (300, 136, 200, "skew", 40, "bf16"),     # single-SM grouped GEMM
+    (1500, 136, 200, "skew", 300, "bf16"),   # CTA-pair grouped GEMM (half tiles too)
+    (1100, 256, 384, "plain", 260, "bf16"),
+    (64, 128, 256, "skew", 10, "f32"),       # fp32 CUDA-core FFN
+])
+def test_capacity_layer(T, d, h, kind, cap, dtype):
+    """Opt-in capacity: each expert keeps its first `cap` pairs in token order."""
+    wl = small("cap", T=T, d=d, h=h, seed=300 + T, kind=kind, dtype=dtype)
+    inp = make_inputs(wl, "cuda")
+    y = f64(capped_y(inp, cap))
+    c = {k: f64(v) for k, v in inp.items()}
+    ref = O.moe_layer(c["x"], c["Wg"], c["W1"], c["W3"], c["W2"], capacity=cap)
+    assert not ref["keep"].all()  # the cap really drops pairs here
+    tol = F32_TOL if dtype == "f32" else BF16_TOL
+    assert rel_fro(y, ref["y"]) <= tol
+    assert worst_token(y, ref["y"]) <= (tol if dtype == "f32" else TOKEN_TOL)
+
+
+@pytest.mark.parametrize("T", [16, 300, 1500])
+def test_capacity_special_cases_on_gpu(T):
+    wl = small("cap0", T=T, d=128, h=256, seed=7, kind="skew")
+    inp = make_inputs(wl, "cuda")
+    y_full = layer_y(inp)
+    assert torch.equal(capped_y(inp, 2 * T), y_full)  # no group exceeds 2T rows
+    assert torch.equal(capped_y(inp, -1), y_full)     # negative: no limit
+    assert (capped_y(inp, 0) == 0).all()
+
+
+def test_capacity_full_size_skewed():
+    """Skewed Mixtral-shaped workload at capacity factor 1.25 (1280 rows per expert):
+    expert 0 (~3500 rows) is cut; sampled tokens against the fp64 oracle."""
+    wl = WORKLOADS["skew"]
+    cap = O.capacity_from_factor(1.25, wl.T, 2, wl.E)
+    inp = make_inputs(wl, "cuda")
+    y = capped_y(inp, cap)
+    x_cpu = inp["x"].float().cpu().numpy()
+    Wg_cpu = inp["Wg"].float().cpu().numpy()
+    idx = O.top2_select(O.router_logits(x_cpu, Wg_cpu))
+    keep = O.capacity_keep(idx, wl.E, cap)
+    assert (~keep).sum() > 1000
+    rng = np.random.default_rng(1)
+    sample = np.unique(np.concatenate([[0, wl.T - 1], rng.choice(wl.T, 64, replace=False)]))
+    # the oracle's capacity decision needs every token's routing; apply it per sample
+    w = O.gate_weights(O.router_logits(x_cpu[sample], Wg_cpu), idx[sample]) * keep[sample]
+    ref = np.zeros((len(sample), wl.d))
+    for j in range(2):
+        for e in range(wl.E):
+            rows = np.nonzero(idx[sample, j] == e)[0]
+            if len(rows):
+                ref[rows] += w[rows, j:j + 1] * O.expert_swiglu(
+                    x_cpu[sample][rows], inp["W1"][e].float().cpu().numpy(),
+                    inp["W3"][e].float().cpu().numpy(), inp["W2"][e].float().cpu().numpy())
+    got = y[torch.as_tensor(sample, device="cuda")].double().cpu().numpy()
+    assert rel_fro(got, ref) <= BF16_TOL
+    assert worst_token(got, ref) <= TOKEN_TOL
