@@ -172,7 +172,7 @@ moe_status moe_layer_forward_capacity(const void *x, const void *Wg, const void 
  *   expert FFN), events[2] after the first FFN kernel (GEMM1 + SwiGLU; for batches
  *   of at most 64 tokens, where one fused kernel runs both GEMMs, after it),
  *   events[3] after the expert FFN, events[4] after the combine.
- * n_events may be 0..5; events beyond n_events are not recorded. */
+ * n_events may be 0..5; events beyond n_events, and null handles, are not recorded. */
 moe_status moe_layer_forward_events(const void *x, const void *Wg, const void *W1,
                                     const void *W3, const void *W2, int T, int d, int h,
                                     int E, int k, moe_dtype dt, void *y, void *ws,

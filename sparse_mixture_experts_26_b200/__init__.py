@@ -188,11 +188,12 @@ def moe_layer_forward_capacity(x, Wg, W1, W3, W2, y, ws, capacity: int, k: int =
 
 def moe_layer_forward_events(x, Wg, W1, W3, W2, y, ws, events, k: int = 2,
                              stream=None) -> None:
-    """``moe_layer_forward`` recording ``events`` (created, up to 5 handles) between stages."""
+    """``moe_layer_forward`` recording ``events`` (up to 5 created handles, or None to skip
+    one) between its stages."""
     _dev(x, Wg, W1, W3, W2, y, ws)
     T, d = x.shape
     E, h, _ = W1.shape
-    handles = (ctypes.c_void_p * max(1, len(events)))(*[int(e) for e in events])
+    handles = (ctypes.c_void_p * max(1, len(events)))(*[int(e) if e else None for e in events])
     _check("moe_layer_forward_events", _lib.moe_layer_forward_events(
         _ptr(x), _ptr(Wg), _ptr(W1), _ptr(W3), _ptr(W2), T, d, h, E, k, _dt(x), _ptr(y),
         _ptr(ws), ws.numel() * ws.element_size(), ctypes.addressof(handles), len(events),

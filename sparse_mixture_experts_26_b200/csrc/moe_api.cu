@@ -227,8 +227,8 @@ moe_status layer_forward_impl(const void* x, const void* Wg, const void* W1, con
     float* Y = at<float>(ws, L.Y);
     const int P = 2 * T;
     PdlScope pdl(small_batch(T));
-    auto mark = [&](int i) -> bool {
-        return i >= n_ev || cudaEventRecord(ev[i], stream) == cudaSuccess;
+    auto mark = [&](int i) -> bool {  // null handles are skipped
+        return i >= n_ev || ev[i] == nullptr || cudaEventRecord(ev[i], stream) == cudaSuccess;
     };
 
     if (!mark(0)) return MOE_ERR_CUDA;
