@@ -185,6 +185,19 @@ moe_status moe_layer_forward_events(const void *x, const void *Wg, const void *W
 moe_status moe_device_status(void *ws, size_t ws_bytes, uint32_t *flags,
                              cudaStream_t stream);
 
+/* Self-test of the device-side failure detection (no counterpart in the paper; it
+ * checks this library's safety mechanism).  Runs, on `stream`, the same bounded
+ * waits the pipelines use -- an mbarrier wait and a device-counter wait -- against
+ * a barrier and a counter that nothing completes, with a limit of `limit_seconds`
+ * (0 < limit <= 10).  Both waits must give up: outcome[0] (barrier) and outcome[1]
+ * (counter) are set to 2 ("gave up") or 1 ("completed", a failure of the test), and
+ * MOE_DEV_FLAG_TIMEOUT is raised in the workspace status word, where
+ * moe_device_status() reports it.  Nothing hangs, traps or faults; the context
+ * stays usable.  Synchronises `stream`.  ws: a workspace of >= 2 KiB (as from
+ * moe_workspace_bytes); outcome: host array of 2. */
+moe_status moe_selftest_wait_timeout(void *ws, size_t ws_bytes, double limit_seconds,
+                                     uint32_t *outcome, cudaStream_t stream);
+
 /* Static description of a status code. */
 const char *moe_status_string(moe_status st);
 

@@ -23,7 +23,7 @@ __all__ = [
     "moe_expert_ffn", "moe_combine", "moe_layer_forward", "moe_device_status",
     "moe_status_string", "moe_layer_forward_events", "alloc_workspace", "layer_forward",
     "EXPORTED_SYMBOLS", "launches_per_layer", "moe_expert_ffn_static",
-    "moe_layer_forward_capacity",
+    "moe_layer_forward_capacity", "moe_selftest_wait_timeout",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe.so")
@@ -34,7 +34,7 @@ _STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED"
 EXPORTED_SYMBOLS = ("moe_workspace_bytes", "moe_route", "moe_permute", "moe_expert_ffn",
                     "moe_combine", "moe_layer_forward", "moe_layer_forward_events",
                     "moe_device_status", "moe_status_string", "moe_expert_ffn_static",
-                    "moe_layer_forward_capacity")
+                    "moe_layer_forward_capacity", "moe_selftest_wait_timeout")
 def launches_per_layer(T: int) -> int:
     """Kernels one moe_layer_forward queues: router 1, permutation 1 (T <= 512) or 4
     (count, scan, rank, gather), expert FFN 1 (T <= 64: gate/up and down fused) or 2,
@@ -70,6 +70,7 @@ def _load() -> ctypes.CDLL:
         "moe_expert_ffn_static": (i32, [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, vp, vp]),
         "moe_layer_forward_capacity": (i32, [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
                                              i32, vp, vp, sz, vp]),
+        "moe_selftest_wait_timeout": (i32, [vp, sz, ctypes.c_double, vp, vp]),
     }
     for name, (res, args) in sigs.items():
         f = getattr(lib, name)
@@ -220,6 +221,16 @@ def moe_expert_ffn_static(x_perm, offsets, W1, W3, W2, y_perm, stream=None) -> N
     _check("moe_expert_ffn_static", _lib.moe_expert_ffn_static(
         _ptr(x_perm), _ptr(offsets), _ptr(W1), _ptr(W3), _ptr(W2), rows, d, h, E, _dt(x_perm),
         _ptr(y_perm), _stream(stream)))
+
+
+def moe_selftest_wait_timeout(ws, limit_seconds: float = 0.05, stream=None):
+    """Run the bounded-wait self-test; returns (barrier outcome, counter outcome), each 2
+    when the wait gave up as it must.  The timeout flag is left in the status word."""
+    out = (ctypes.c_uint32 * 2)()
+    _check("moe_selftest_wait_timeout", _lib.moe_selftest_wait_timeout(
+        _ptr(ws), ws.numel() * ws.element_size(), float(limit_seconds), ctypes.addressof(out),
+        _stream(stream)))
+    return int(out[0]), int(out[1])
 
 
 def layer_forward(x, Wg, W1, W3, W2, ws=None, out=None, stream=None) -> torch.Tensor:

@@ -474,12 +474,6 @@ __device__ __forceinline__ FusedUnit fused_unit(const FusedBook<NACC>& bk, const
     return f;
 }
 
-__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
-    uint32_t v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-
 __device__ __forceinline__ void fence_proxy_async_global() {
     asm volatile("fence.proxy.async.global;" ::: "memory");
 }
@@ -574,21 +568,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     // wait until every gate/up tile of this K range has published its H
                     const uint32_t need = static_cast<uint32_t>(f.chunks * (f.kb1 - f.kb0));
                     const uint32_t* rdy = args.ready + f.e * args.ksplit + f.ks;
-                    if (ld_acquire_gpu(rdy) < need) {
-                        const unsigned long long t0 = global_timer_ns();
-                        while (ld_acquire_gpu(rdy) < need) {
-                            if (*abort_flag) {
-                                ok = false;
-                                break;
-                            }
-                            if (global_timer_ns() - t0 > kWaitTimeoutNs) {
-                                *abort_flag = 1;
-                                if (args.status) atomicOr(args.status, 1u);
-                                ok = false;
-                                break;
-                            }
-                        }
-                        if (!ok) break;
+                    if (!flag_wait_bounded(rdy, need, abort_flag, args.status)) {
+                        ok = false;
+                        break;
                     }
                     fence_proxy_async_global();
                     // the last reader of this counter resets it for the next launch

@@ -289,6 +289,27 @@ moe_status moe_layer_forward_events(const void* x, const void* Wg, const void* W
                               n_events, stream, INT_MAX);
 }
 
+moe_status moe_selftest_wait_timeout(void* ws, size_t ws_bytes, double limit_seconds,
+                                     uint32_t* outcome, cudaStream_t stream) {
+    if (!ws || !outcome || ws_bytes < 2048 || !(limit_seconds > 0.0) || limit_seconds > 10.0)
+        return MOE_ERR_INVALID_ARG;
+    // status word at offset 0; scratch words at offset 1024 (inside the first region
+    // of every workspace layout, which is at least 2 KiB)
+    uint32_t* status = static_cast<uint32_t*>(ws);
+    uint32_t* scratch = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + 1024);
+    const auto ns = static_cast<unsigned long long>(limit_seconds * 1e9);
+    if (launch_selftest_wait(status, scratch, ns, stream) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return MOE_ERR_CUDA;
+    uint32_t got[2] = {0, 0};
+    if (cudaMemcpy(got, scratch + 1, sizeof(got), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    outcome[0] = got[0];
+    outcome[1] = got[1];
+    // the scratch words must be zero again for the layer's own use of this region
+    if (cudaMemset(scratch, 0, 3 * sizeof(uint32_t)) != cudaSuccess) return MOE_ERR_CUDA;
+    return MOE_OK;
+}
+
 moe_status moe_device_status(void* ws, size_t ws_bytes, uint32_t* flags, cudaStream_t stream) {
     if (!ws || !flags || ws_bytes < 256) return MOE_ERR_INVALID_ARG;
     if (cudaStreamSynchronize(stream) != cudaSuccess) return MOE_ERR_CUDA;

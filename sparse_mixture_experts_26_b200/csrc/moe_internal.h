@@ -162,6 +162,9 @@ cudaError_t launch_combine(const float* Y, int nsplit, size_t split_stride,
                            const int32_t* inv_perm, const float* w, int T, int d, moe_dtype dt,
                            void* y, cudaStream_t s, const int32_t* idx = nullptr,
                            const int32_t* offsets = nullptr, int E = 0, int cap = INT_MAX);
+// Bounded-wait self-test (see moe_selftest_wait_timeout).
+cudaError_t launch_selftest_wait(uint32_t* status, uint32_t* scratch, unsigned long long limit_ns,
+                                 cudaStream_t s);
 // Y[i] = sum over j < nsplit of parts[j * n + i] (in order), for i < n.
 cudaError_t launch_sum_splits(const float* parts, int nsplit, size_t n, float* Y,
                               cudaStream_t s);

@@ -79,6 +79,30 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
     }
 }
 
+// Wait until *counter >= need (acquire, device scope).  Returns false (after setting
+// *abort_flag and the status word) once `limit_ns` has passed, or when another role
+// has set *abort_flag.
+__device__ __forceinline__ bool flag_wait_bounded(const uint32_t* counter, uint32_t need,
+                                                  volatile int* abort_flag, uint32_t* status,
+                                                  unsigned long long limit_ns = kWaitTimeoutNs) {
+    auto load = [&]() {
+        uint32_t v;
+        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(counter) : "memory");
+        return v;
+    };
+    if (load() >= need) return true;
+    const unsigned long long t0 = global_timer_ns();
+    while (load() < need) {
+        if (*abort_flag) return false;
+        if (global_timer_ns() - t0 > limit_ns) {
+            *abort_flag = 1;
+            if (status) atomicOr(status, 1u);  // MOE_DEV_FLAG_TIMEOUT
+            return false;
+        }
+    }
+    return true;
+}
+
 // ------------------------------------------------------------------ TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
