@@ -68,6 +68,8 @@ __all__ = [
     "mixtral_param_counts",
     "capacity_keep",
     "capacity_from_factor",
+    "moe_layer_backward",
+    "moe_layer_backward_dense",
 ]
 
 
@@ -324,6 +326,143 @@ def moe_layer_dense(x, Wg, W1, W3, W2, k: int = 2) -> np.ndarray:
     for e in range(G.shape[1]):
         y += G[:, e:e + 1] * expert_swiglu(x, W1[e], W3[e], W2[e])
     return y
+
+
+def _silu_grad(z) -> np.ndarray:
+    """d silu / dz = sigma(z) (1 + z (1 - sigma(z))) in fp64."""
+    z = _f64(z)
+    with np.errstate(over="ignore"):
+        s = 1.0 / (1.0 + np.exp(-z))
+    return s * (1.0 + z * (1.0 - s))
+
+
+def moe_layer_backward(x, Wg, W1, W3, W2, dy, k: int = 2, capacity=None) -> dict:
+    """Gradients of the routed layer (oracle O1) for an upstream gradient ``dy[T, d]``.
+
+    crackai "Mixtral of Experts", "Key Takeaways": routing is learned jointly with the
+    model, so the gradient reaches the router through the gate weights.  Reading (the
+    pages state no backward pass): the exact derivative of ``y`` with the top-2 choice
+    held fixed (it is piecewise constant in the inputs), computed group by group:
+
+    * grouped row ``r`` of token ``t``, slot ``j``: ``dY[r] = w[t, j] dy[t]`` and
+      ``dw[t, j] = <dy[t], Y[r]>``;
+    * per expert, with ``a = x W1^T``, ``b = x W3^T``, ``H = silu(a) b``:
+      ``dW2 = dY^T H``, ``dH = dY W2``, ``da = dH b silu'(a)``, ``db = dH silu(a)``,
+      ``dW1 = da^T x``, ``dW3 = db^T x``, ``dx_perm = da W1 + db W3``;
+    * ``dx[t] = sum_j dx_perm[inv[t, j]]``;
+    * gate: ``w1 = sigma(l_i1 - l_i2)``, ``w2 = 1 - w1``, so the logit gap receives
+      ``(dw1 - dw2) w1 w2``, logit ``i1`` that amount and logit ``i2`` its negative;
+      ``dWg = x^T dlogits`` and ``dx += dlogits Wg^T``.
+
+    A pair dropped by ``capacity`` contributes nothing to ``y`` and so receives and
+    passes on no gradient.  Returns ``dx, dWg, dW1, dW3, dW2`` (fp64, shaped like the
+    inputs), ``dw [T, k]``, ``dlogits [T, E]``, ``dY [P, d]`` (grouped order),
+    ``dH [P, h]`` and the forward dict under ``fwd``.
+    """
+    if k != 2:
+        raise ValueError("the gate derivative is written for k = 2")
+    fwd = moe_layer(x, Wg, W1, W3, W2, k, capacity)
+    x = _f64(x)
+    Wg = _f64(Wg)
+    dy = _f64(dy)
+    T, d = x.shape
+    E = fwd["logits"].shape[1]
+    idx, w, keep = fwd["idx"], fwd["w"], fwd["keep"]
+    offsets, perm_token, inv = fwd["offsets"], fwd["perm_token"], fwd["inv_perm"]
+    inv = np.asarray(inv, dtype=np.int64)
+    P = T * k
+    h = np.asarray(W1[0]).shape[0] if E else 0
+    slot = np.empty(P, dtype=np.int64)
+    for j in range(k):
+        slot[inv[:, j]] = j
+    tok = np.asarray(perm_token, dtype=np.int64)
+    wk = w * keep
+    dY = wk[tok, slot][:, None] * dy[tok]
+    dw = np.zeros((T, k), dtype=np.float64)
+    for j in range(k):
+        dw[:, j] = np.einsum("td,td->t", dy, fwd["Y"][inv[:, j]]) * keep[:, j]
+    x_perm = gather_rows(x, tok)
+    dx_perm = np.zeros((P, d), dtype=np.float64)
+    dH = np.zeros((P, h), dtype=np.float64)
+    dW1 = np.zeros((E, h, d), dtype=np.float64)
+    dW3 = np.zeros((E, h, d), dtype=np.float64)
+    dW2 = np.zeros((E, d, h), dtype=np.float64)
+    for e in range(E):
+        lo = int(offsets[e])
+        hi = int(offsets[e + 1])
+        if capacity is not None:
+            hi = min(hi, lo + int(capacity))
+        if hi <= lo:
+            continue
+        W1e, W3e, W2e = _f64(W1[e]), _f64(W3[e]), _f64(W2[e])
+        xr = x_perm[lo:hi]
+        a = xr @ W1e.T
+        b = xr @ W3e.T
+        He = silu(a) * b
+        g = dY[lo:hi]
+        dW2[e] = g.T @ He
+        dHe = g @ W2e
+        dH[lo:hi] = dHe
+        da = dHe * b * _silu_grad(a)
+        db = dHe * silu(a)
+        dW1[e] = da.T @ xr
+        dW3[e] = db.T @ xr
+        dx_perm[lo:hi] = da @ W1e + db @ W3e
+    dx = np.zeros((T, d), dtype=np.float64)
+    for j in range(k):
+        dx += dx_perm[inv[:, j]]
+    gap = (dw[:, 0] - dw[:, 1]) * w[:, 0] * w[:, 1]
+    dlogits = np.zeros((T, E), dtype=np.float64)
+    rows = np.arange(T)
+    dlogits[rows, idx[:, 0]] += gap
+    dlogits[rows, idx[:, 1]] -= gap
+    dWg = x.T @ dlogits
+    dx += dlogits @ Wg.T
+    return dict(dx=dx, dWg=dWg, dW1=dW1, dW3=dW3, dW2=dW2, dw=dw, dlogits=dlogits, dY=dY,
+                dH=dH, fwd=fwd)
+
+
+def moe_layer_backward_dense(x, Wg, W1, W3, W2, dy, k: int = 2) -> dict:
+    """Brute-force gradients (oracle O2): every expert on every token, dense gate.
+
+    ``y = sum_e G_e E_e(x)`` with ``G`` the -inf-masked softmax of notion notes,
+    "Sparse gating", eq. G(x) (mask held fixed).  ``dG_e = <dy, E_e(x)>``; the softmax
+    Jacobian gives ``dlogits = G * (dG - <G, dG>)`` (zero outside the mask, because G
+    is); each expert's weights get ``G_e`` times its plain SwiGLU gradient.  No
+    grouping, no permutation, and a different route through the gate derivative than
+    ``moe_layer_backward``.
+    """
+    x = _f64(x)
+    Wg = _f64(Wg)
+    dy = _f64(dy)
+    T, d = x.shape
+    G = gate_dense_topk_softmax(router_logits(x, Wg), k)
+    E = G.shape[1]
+    h = np.asarray(W1[0]).shape[0]
+    dx = np.zeros((T, d), dtype=np.float64)
+    dW1 = np.zeros((E, h, d), dtype=np.float64)
+    dW3 = np.zeros((E, h, d), dtype=np.float64)
+    dW2 = np.zeros((E, d, h), dtype=np.float64)
+    dG = np.zeros((T, E), dtype=np.float64)
+    for e in range(E):
+        W1e, W3e, W2e = _f64(W1[e]), _f64(W3[e]), _f64(W2[e])
+        a = x @ W1e.T
+        b = x @ W3e.T
+        He = silu(a) * b
+        Ye = He @ W2e.T
+        dG[:, e] = np.einsum("td,td->t", dy, Ye)
+        g = G[:, e:e + 1] * dy
+        dW2[e] = g.T @ He
+        dHe = g @ W2e
+        da = dHe * b * _silu_grad(a)
+        db = dHe * silu(a)
+        dW1[e] = da.T @ x
+        dW3[e] = db.T @ x
+        dx += da @ W1e + db @ W3e
+    dlogits = G * (dG - np.sum(G * dG, axis=1, keepdims=True))
+    dWg = x.T @ dlogits
+    dx += dlogits @ Wg.T
+    return dict(dx=dx, dWg=dWg, dW1=dW1, dW3=dW3, dW2=dW2, dlogits=dlogits)
 
 
 def mixtral_param_counts(d: int = 32 * 128, h: int = 14336, E: int = 8, k: int = 2,

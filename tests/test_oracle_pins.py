@@ -383,3 +383,104 @@ def test_capacity_special_cases():
     assert O.capacity_from_factor(1.0, 4096, 2, 8) == 1024
     assert O.capacity_from_factor(1.25, 4096, 2, 8) == 1280
     assert O.capacity_from_factor(1.25, 10, 2, 8) == 4
+
+
+# ---------------------------------------------------------------- backward (training)
+
+def _fd_case(seed=1, T=4, d=5, h=3, E=4):
+    rng = np.random.default_rng(seed)
+    return dict(x=rng.normal(size=(T, d)), Wg=rng.normal(size=(d, E)),
+                W1=rng.normal(size=(E, h, d)) / 2, W3=rng.normal(size=(E, h, d)) / 2,
+                W2=rng.normal(size=(E, d, h)) / 2), rng.normal(size=(T, d))
+
+
+def _finite_differences(inp, dy, capacity=None, eps=1e-6):
+    """Central differences of L = sum(dy * y) with respect to every input entry."""
+    names = ("x", "Wg", "W1", "W3", "W2")
+
+    def loss(args):
+        return float((O.moe_layer(*args, capacity=capacity)["y"] * dy).sum())
+
+    out = {}
+    for i, n in enumerate(names):
+        A = inp[n]
+        fd = np.zeros_like(A)
+        for ix in np.ndindex(A.shape):
+            plus = [inp[m].copy() for m in names]
+            minus = [inp[m].copy() for m in names]
+            plus[i][ix] += eps
+            minus[i][ix] -= eps
+            fd[ix] = (loss(plus) - loss(minus)) / (2 * eps)
+        out["d" + n] = fd
+    return out
+
+
+def _fd_agrees(g, fd, tol=1e-7):
+    return all(np.abs(fd[k] - g[k]).max() <= tol * max(np.abs(fd[k]).max(), 1e-12)
+               for k in fd)
+
+
+@pytest.mark.parametrize("capacity", [None, 1])
+def test_backward_matches_finite_differences(capacity):
+    """The top-2 choice is held fixed: random inputs keep every logit gap far above
+    the step, so central differences of the forward oracle pin every gradient."""
+    inp, dy = _fd_case()
+    g = O.moe_layer_backward(**inp, dy=dy, capacity=capacity)
+    fd = _finite_differences(inp, dy, capacity)
+    for k in fd:
+        np.testing.assert_allclose(g[k], fd[k], rtol=0, atol=1e-7 * np.abs(fd[k]).max())
+    if capacity is not None:
+        # dropped pairs pass nothing on
+        assert not g["fwd"]["keep"].all()
+        np.testing.assert_array_equal(g["dw"][~g["fwd"]["keep"]], 0.0)
+
+
+@pytest.mark.parametrize("mistake", ["silu_grad_is_sigmoid", "gate_sign", "no_router_term"])
+def test_backward_planted_mistakes_are_caught(monkeypatch, mistake):
+    inp, dy = _fd_case(seed=2)
+    fd = _finite_differences(inp, dy)
+    if mistake == "silu_grad_is_sigmoid":
+        monkeypatch.setattr(O, "_silu_grad", lambda z: 1.0 / (1.0 + np.exp(-np.asarray(z))))
+        g = O.moe_layer_backward(**inp, dy=dy)
+    else:
+        g = dict(O.moe_layer_backward(**inp, dy=dy))
+        if mistake == "gate_sign":
+            g["dWg"] = -g["dWg"]
+        else:
+            g["dx"] = g["dx"] - g["dlogits"] @ inp["Wg"].T
+    assert not _fd_agrees(g, fd)
+
+
+@pytest.mark.parametrize("T,d,h,kind", [(1, 8, 16, "plain"), (37, 24, 40, "skew"),
+                                        (64, 16, 24, "long")])
+def test_backward_routed_equals_dense(T, d, h, kind):
+    """O1 (per group, sigmoid of the logit gap) against O2 (every expert, softmax
+    Jacobian of the masked dense gate)."""
+    inp = _inputs(small("bw", T=T, d=d, h=h, seed=50 + T, kind=kind))
+    dy = np.random.default_rng(T).normal(size=(T, d))
+    g = O.moe_layer_backward(**inp, dy=dy)
+    gd = O.moe_layer_backward_dense(**inp, dy=dy)
+    for k in ("dx", "dWg", "dW1", "dW3", "dW2", "dlogits"):
+        scale = max(np.abs(gd[k]).max(), 1e-300)
+        assert np.abs(g[k] - gd[k]).max() <= 1e-12 * scale, k
+
+
+def test_backward_invariants():
+    inp = _inputs(small("bwi", T=50, d=16, h=24, seed=9, kind="skew"))
+    rng = np.random.default_rng(3)
+    dy1, dy2 = rng.normal(size=(50, 16)), rng.normal(size=(50, 16))
+    g1 = O.moe_layer_backward(**inp, dy=dy1)
+    g2 = O.moe_layer_backward(**inp, dy=dy2)
+    g12 = O.moe_layer_backward(**inp, dy=dy1 + 2 * dy2)
+    for k in ("dx", "dWg", "dW1", "dW3", "dW2", "dw"):
+        np.testing.assert_allclose(g12[k], g1[k] + 2 * g2[k], rtol=1e-10,
+                                   atol=1e-12 * np.abs(g12[k]).max())
+    # a shift of all logits changes nothing: each token's logit gradients sum to 0,
+    # and only the two chosen experts' logits receive any
+    s = g1["dlogits"].sum(axis=1)
+    assert np.abs(s).max() <= 1e-14 * np.abs(g1["dlogits"]).max()
+    assert (np.count_nonzero(g1["dlogits"], axis=1) <= 2).all()
+    # experts nobody chose get no weight gradient
+    counts = np.bincount(g1["fwd"]["idx"].ravel(), minlength=8)
+    for e in np.flatnonzero(counts == 0):
+        assert not g1["dW1"][e].any() and not g1["dW2"][e].any()
