@@ -198,6 +198,34 @@ moe_status moe_device_status(void *ws, size_t ws_bytes, uint32_t *flags,
 moe_status moe_selftest_wait_timeout(void *ws, size_t ws_bytes, double limit_seconds,
                                      uint32_t *outcome, cudaStream_t stream);
 
+/* Bytes of backward workspace moe_layer_backward needs for these sizes (0 for an
+ * unsupported shape: the backward pass is built for bf16 layers with h % 64 == 0). */
+size_t moe_backward_workspace_bytes(int T, int d, int h, int E, int k, moe_dtype dt);
+
+/* Gradients of the layer, for training.  crackai "Mixtral of Experts", "Key
+ * Takeaways": routing is learned jointly with the model.  The pages print no backward
+ * formulas; this is the exact derivative of moe_layer_forward (or, with capacity >= 0,
+ * moe_layer_forward_capacity) with the top-2 choice held fixed: for an upstream
+ * gradient dy of L with respect to y it returns dL/dx, dL/dWg, dL/dW1, dL/dW3 and
+ * dL/dW2.  The gate weights w1 = sigma(l_i1 - l_i2), w2 = 1 - w1 pass the gradient
+ * to the two chosen logits only; a pair dropped by the capacity passes nothing.
+ *
+ * Arguments: x, Wg, W1, W3, W2 and T, d, h, E, k, dt exactly as given to the forward
+ * call; dy bf16 [T, d].  fwd_ws: the workspace of that forward call, unchanged since
+ * (it holds the routing, the permutation, the gathered rows, H and the expert
+ * outputs).  Outputs (caller-owned, device): dx bf16 [T, d]; dWg, dW1, dW3, dW2 fp32
+ * with the shapes of Wg [d, E], W1/W3 [E, h, d] and W2 [E, d, h] (overwritten, not
+ * accumulated; an expert that received no rows gets zeros).  bwd_ws: device scratch
+ * of moe_backward_workspace_bytes bytes; its status word (offset 0) collects device
+ * flags like the forward's.  Only dt == MOE_BF16 and h % 64 == 0 are supported
+ * (MOE_ERR_UNSUPPORTED otherwise).  Queued on `stream`; argument errors return before
+ * anything is queued. */
+moe_status moe_layer_backward(const void *x, const void *Wg, const void *W1, const void *W3,
+                              const void *W2, const void *dy, int T, int d, int h, int E, int k,
+                              moe_dtype dt, int capacity, void *dx, float *dWg, float *dW1,
+                              float *dW3, float *dW2, const void *fwd_ws, size_t fwd_ws_bytes,
+                              void *bwd_ws, size_t bwd_ws_bytes, cudaStream_t stream);
+
 /* Static description of a status code. */
 const char *moe_status_string(moe_status st);
 

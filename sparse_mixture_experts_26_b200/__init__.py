@@ -23,7 +23,8 @@ __all__ = [
     "moe_expert_ffn", "moe_combine", "moe_layer_forward", "moe_device_status",
     "moe_status_string", "moe_layer_forward_events", "alloc_workspace", "layer_forward",
     "EXPORTED_SYMBOLS", "launches_per_layer", "moe_expert_ffn_static",
-    "moe_layer_forward_capacity", "moe_selftest_wait_timeout",
+    "moe_layer_forward_capacity", "moe_selftest_wait_timeout", "moe_backward_workspace_bytes",
+    "moe_layer_backward", "alloc_backward_workspace", "layer_backward",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe.so")
@@ -34,7 +35,8 @@ _STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED"
 EXPORTED_SYMBOLS = ("moe_workspace_bytes", "moe_route", "moe_permute", "moe_expert_ffn",
                     "moe_combine", "moe_layer_forward", "moe_layer_forward_events",
                     "moe_device_status", "moe_status_string", "moe_expert_ffn_static",
-                    "moe_layer_forward_capacity", "moe_selftest_wait_timeout")
+                    "moe_layer_forward_capacity", "moe_selftest_wait_timeout",
+                    "moe_backward_workspace_bytes", "moe_layer_backward")
 def launches_per_layer(T: int) -> int:
     """Kernels one moe_layer_forward queues: router 1, permutation 1 (T <= 512) or 4
     (count, scan, rank, gather), expert FFN 1 (T <= 64: gate/up and down fused) or 2,
@@ -71,6 +73,9 @@ def _load() -> ctypes.CDLL:
         "moe_layer_forward_capacity": (i32, [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
                                              i32, vp, vp, sz, vp]),
         "moe_selftest_wait_timeout": (i32, [vp, sz, ctypes.c_double, vp, vp]),
+        "moe_backward_workspace_bytes": (sz, [i32, i32, i32, i32, i32, i32]),
+        "moe_layer_backward": (i32, [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32,
+                                     vp, vp, vp, vp, vp, vp, sz, vp, sz, vp]),
     }
     for name, (res, args) in sigs.items():
         f = getattr(lib, name)
@@ -243,3 +248,45 @@ def layer_forward(x, Wg, W1, W3, W2, ws=None, out=None, stream=None) -> torch.Te
         out = torch.empty_like(x)
     moe_layer_forward(x, Wg, W1, W3, W2, out, ws, stream=stream)
     return out
+
+
+def moe_backward_workspace_bytes(T: int, d: int, h: int, E: int = 8, k: int = 2,
+                                 dtype: torch.dtype = torch.bfloat16) -> int:
+    dt = MOE_BF16 if dtype == torch.bfloat16 else MOE_F32
+    return int(_lib.moe_backward_workspace_bytes(T, d, h, E, k, dt))
+
+
+def alloc_backward_workspace(T: int, d: int, h: int, E: int = 8, k: int = 2,
+                             dtype: torch.dtype = torch.bfloat16, device="cuda") -> torch.Tensor:
+    n = moe_backward_workspace_bytes(T, d, h, E, k, dtype)
+    if n == 0:
+        raise MoeError("moe_backward_workspace_bytes", 2, "unsupported shape")
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def moe_layer_backward(x, Wg, W1, W3, W2, dy, dx, dWg, dW1, dW3, dW2, fwd_ws, bwd_ws,
+                       capacity: int = -1, k: int = 2, stream=None) -> None:
+    """Gradients of the layer for upstream gradient ``dy``; ``fwd_ws`` is the workspace
+    of the forward call on the same inputs (``capacity`` as given to it, -1 for none)."""
+    _dev(x, Wg, W1, W3, W2, dy, dx, dWg, dW1, dW3, dW2, fwd_ws, bwd_ws)
+    T, d = x.shape
+    E, h, _ = W1.shape
+    _check("moe_layer_backward", _lib.moe_layer_backward(
+        _ptr(x), _ptr(Wg), _ptr(W1), _ptr(W3), _ptr(W2), _ptr(dy), T, d, h, E, k, _dt(x),
+        int(capacity), _ptr(dx), _ptr(dWg), _ptr(dW1), _ptr(dW3), _ptr(dW2), _ptr(fwd_ws),
+        fwd_ws.numel() * fwd_ws.element_size(), _ptr(bwd_ws),
+        bwd_ws.numel() * bwd_ws.element_size(), _stream(stream)))
+
+
+def layer_backward(x, Wg, W1, W3, W2, dy, fwd_ws, capacity: int = -1, bwd_ws=None):
+    """Allocating convenience wrapper: returns (dx, dWg, dW1, dW3, dW2)."""
+    T, d = x.shape
+    E, h, _ = W1.shape
+    if bwd_ws is None:
+        bwd_ws = alloc_backward_workspace(T, d, h, E, 2, x.dtype, x.device)
+    dx = torch.empty_like(x)
+    f32 = dict(dtype=torch.float32, device=x.device)
+    dWg, dW1 = torch.empty(Wg.shape, **f32), torch.empty(W1.shape, **f32)
+    dW3, dW2 = torch.empty(W3.shape, **f32), torch.empty(W2.shape, **f32)
+    moe_layer_backward(x, Wg, W1, W3, W2, dy, dx, dWg, dW1, dW3, dW2, fwd_ws, bwd_ws, capacity)
+    return dx, dWg, dW1, dW3, dW2

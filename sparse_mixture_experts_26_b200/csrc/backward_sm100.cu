@@ -1,0 +1,893 @@
+// backward_sm100.cu -- gradients of the layer for training.
+//
+// crackai "Mixtral of Experts", "Key Takeaways": routing is learned jointly with the
+// model, so the backward pass reaches the router through the two gate weights.  The
+// pages print no backward formulas; this is the exact derivative of the forward
+// layer with the top-2 choice held fixed (it is piecewise constant in the inputs).
+// For grouped row r = (token t, slot j) of expert e, with a = x W1^T, b = x W3^T:
+//
+//   dY[r]   = w[t,j] dy[t]                       (bf16, prep kernel)
+//   dw[t,j] = <dy[t], Y[r]>                      (prep kernel; Y saved by the forward)
+//   dH      = dY W2_e                            (GEMM, K = d; W2_e read MN-major)
+//   du      = dH * b * silu'(a),  dv = dH * silu(a)
+//                                                (GEMM recomputing a and b, K = d, with
+//                                                 the elementwise step as its epilogue)
+//   dX      = [du dv] [W1_e ; W3_e]              (GEMM, K = 2h; weights read MN-major)
+//   dx[t]   = dX[r(t,0)] + dX[r(t,1)] + dlogits[t] Wg^T
+//   dW2_e   = dY_e^T H_e,  [dW1_e ; dW3_e] = [du dv]_e^T x_e
+//                                                (GEMMs whose reduction runs over the
+//                                                 expert's own rows; both operands
+//                                                 MN-major)
+//   dlogits: the gap l_i1 - l_i2 gets (dw1 - dw2) w1 w2, logit i1 that, i2 minus that;
+//   dWg     = x^T dlogits                        (CUDA cores, fixed-order reduction)
+//
+// The GEMMs use the same engine layout as the forward (persistent, warp-specialised:
+// TMA producer, single-thread tcgen05.mma issuer, four epilogue warps; 128x256 fp32
+// accumulators double-buffered in TMEM).  An operand stored with its M/N dimension
+// contiguous is loaded as 64-column x 64-row boxes with 128-byte swizzle and handed to
+// the tensor core as an MN-major operand (transpose bit in the instruction
+// descriptor), so no weight or activation is ever transposed in memory.  In the
+// weight-gradient GEMMs the reduction runs over an expert's rows, which start and
+// end anywhere: the rows of a last, partial K block that belong to the next expert
+// are zeroed in shared memory before the MMA reads them.  Every wait is bounded.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "moe_internal.h"
+#include "sm100_ptx.cuh"
+
+namespace moe {
+
+// Defined in grouped_gemm_sm100.cu.
+bool encode_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                    uint32_t box_rows);
+
+namespace {
+
+constexpr int kBM = 128;                   // accumulator rows (TMEM lanes)
+constexpr int kBK = 64;                    // K per stage
+constexpr int kN = 256;                    // accumulator columns
+constexpr int kStages = 4;
+constexpr int kABytes = kBM * kBK * 2;     // 16 KiB
+constexpr int kBBytes = kN * kBK * 2;      // 32 KiB
+constexpr int kStageBytes = kABytes + kBBytes;
+constexpr int kThreads = 192;
+constexpr int kEpiThreads = 128;
+constexpr uint32_t kTmemCols = 2 * kN;
+constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 1024 /*bookkeeping*/;
+constexpr int kBox = 64 * 128;             // one 64-column x 64-row box: 8 KiB
+constexpr int kVoteBarrier = 2;
+
+enum RowMode { kModeDH = 0, kModeDUV = 1, kModeDX = 2 };
+enum WMode { kModeW2 = 0, kModeW13 = 1 };
+
+// Shared-memory descriptor of an MN-major operand with 128-byte swizzle: each k is
+// one 128-byte row of 64 consecutive M/N elements; consecutive 64-element groups of
+// M/N are one box (kBox bytes) apart (leading byte offset), 8-row groups of k are
+// 1024 bytes apart (stride byte offset).  Version 1 (bit 46), swizzle mode 2.
+__device__ __forceinline__ uint64_t sw128_mn_desc(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
+    d |= static_cast<uint64_t>(kBox >> 4) << 16;
+    d |= static_cast<uint64_t>(1024u >> 4) << 32;
+    d |= static_cast<uint64_t>(1u) << 46;
+    d |= static_cast<uint64_t>(2u) << 61;
+    return d;
+}
+// Descriptor step for K = 16: MN-major 16 rows of 128 bytes; K-major 32 bytes.
+constexpr uint64_t kMnStep = (16 * 128) >> 4;
+constexpr uint64_t kKStep = 32 >> 4;
+
+// bf16 x bf16 -> f32, M x N; transpose bits 15 (A) / 16 (B) select MN-major operands.
+__host__ __device__ constexpr uint32_t idesc_major(int M, int N, bool a_mn, bool b_mn) {
+    return idesc_bf16_f32(M, N) | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16);
+}
+
+struct Book {
+    uint64_t full[kStages];
+    uint64_t empty[kStages];
+    uint64_t tmem_full[2];
+    uint64_t tmem_empty[2];
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort_flag;
+    int off[kMaxExperts + 1];
+    int end[kMaxExperts];
+    int tile_start[kMaxExperts + 1];
+};
+static_assert(sizeof(Book) <= 1024, "bookkeeping reserve");
+
+__device__ __forceinline__ float bits_f32(uint32_t u) { return __uint_as_float(u); }
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
+    const unsigned long long t0 = global_timer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (global_timer_ns() - t0 > kDrainTimeoutNs) break;
+    }
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Group offsets (clamped, monotone) and kept ends; thread 0 only.
+__device__ __forceinline__ void load_groups(Book& bk, const int32_t* offsets, int E, int rows,
+                                            int cap) {
+    int prev = 0;
+    for (int g = 0; g <= E; ++g) {
+        int v = offsets[g];
+        v = v < prev ? prev : (v > rows ? rows : v);
+        bk.off[g] = v;
+        prev = v;
+    }
+    for (int g = 0; g < E; ++g) {
+        const int n = bk.off[g + 1] - bk.off[g];
+        bk.end[g] = bk.off[g] + (n < cap ? n : cap);
+    }
+}
+
+__device__ __forceinline__ void init_barriers(Book& bk) {
+    for (int s = 0; s < kStages; ++s) {
+        mbar_init(&bk.full[s], 1);
+        mbar_init(&bk.empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+        mbar_init(&bk.tmem_full[a], 1);
+        mbar_init(&bk.tmem_empty[a], kEpiThreads);
+    }
+    mbar_init(&bk.drain, 1);
+    bk.abort_flag = 0;
+    fence_mbar_init();
+}
+
+// ================================================================ row-grouped GEMMs
+// Tiles are (expert, 128-row block of its rows, 256-column block of the output), as in
+// the forward; A is always the grouped activation [rows, K], K-major.
+//   kModeDH : dH[r, :h]   = dY[r] . W2_e          B = W2_e [d, h] rows = k  (MN-major)
+//   kModeDUV: du, dv      from a = x W1_e^T, b = x W3_e^T and dH (epilogue)
+//             B = 128 rows of W1_e over the same 128 rows of W3_e (K-major, as GEMM1)
+//   kModeDX : dX[r, :d]   = [du dv][r] . [W1_e ; W3_e]   B rows = k (MN-major),
+//             k < h from W1, k >= h from W3
+struct RowArgs {
+    const int32_t* offsets;
+    int E;
+    int rows;
+    int K;         // reduction length (d, d, 2h)
+    int N;         // output columns (h, h, d)
+    int n_tiles;
+    int h;
+    int d;
+    void* out;         // dH fp32 [rows, h] | DUV bf16 [rows, 2h] | dX fp32 [rows, d]
+    const float* dH;   // kModeDUV: dH fp32 [rows, h]
+    uint32_t* status;
+    int cap;
+};
+
+template <int MODE>
+__global__ void __launch_bounds__(kThreads, 1)
+    bwd_rows_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
+                    const __grid_constant__ CUtensorMap tmB1, const RowArgs args) {
+    constexpr bool kBmn = MODE != kModeDUV;
+    constexpr uint32_t kIdesc = idesc_major(kBM, kN, false, kBmn);
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint8_t* sA = smem;
+    uint8_t* sB = smem + kStages * kABytes;
+    Book& bk = *reinterpret_cast<Book*>(smem + kStages * kStageBytes);
+    volatile int* abort_flag = &bk.abort_flag;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int E = args.E;
+
+    if (threadIdx.x == 0) init_barriers(bk);
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB0);
+        tma_prefetch_desc(&tmB1);
+    }
+    if (warp == 1) tmem_alloc(&bk.tmem_base, kTmemCols);
+    if (threadIdx.x == 0) {
+        load_groups(bk, args.offsets, E, args.rows, args.cap);
+        bk.tile_start[0] = 0;
+        for (int g = 0; g < E; ++g)
+            bk.tile_start[g + 1] =
+                bk.tile_start[g] + (bk.end[g] - bk.off[g] + kBM - 1) / kBM * args.n_tiles;
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = bk.tmem_base;
+    const int total = bk.tile_start[E];
+    const int num_kb = (args.K + kBK - 1) / kBK;
+
+    auto tile_of = [&](int tile, int& e, int& row0, int& row_end, int& nt) {
+        int g = 0;
+        while (g + 1 < E && tile >= bk.tile_start[g + 1]) ++g;
+        const int local = tile - bk.tile_start[g];
+        const int m_tiles = (bk.end[g] - bk.off[g] + kBM - 1) / kBM;
+        e = g;
+        row0 = bk.off[g] + (local % m_tiles) * kBM;
+        nt = local / m_tiles;
+        row_end = bk.end[g];
+    };
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0, pending = 0, pending_phase = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+                int e, row0, row_end, nt;
+                tile_of(tile, e, row0, row_end, nt);
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    if (!mbar_wait_bounded(&bk.empty[stage], phase ^ 1u, abort_flag,
+                                           args.status)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&bk.full[stage], kStageBytes);
+                    const int kc = kb * kBK;
+                    uint8_t* a = sA + stage * kABytes;
+                    uint8_t* b = sB + stage * kBBytes;
+                    tma_load_2d(&tmA, &bk.full[stage], a, kc, row0);
+                    if (MODE == kModeDUV) {
+                        const int brow = e * args.h + nt * 128;
+                        tma_load_2d(&tmB0, &bk.full[stage], b, kc, brow);
+                        tma_load_2d(&tmB1, &bk.full[stage], b + kBBytes / 2, kc, brow);
+                    } else {
+                        const CUtensorMap* map = &tmB0;
+                        int krow;
+                        if (MODE == kModeDH) {
+                            krow = e * args.d + kc;
+                        } else {
+                            const bool second = kc >= args.h;
+                            map = second ? &tmB1 : &tmB0;
+                            krow = e * args.h + (second ? kc - args.h : kc);
+                        }
+#pragma unroll
+                        for (int i = 0; i < kN / 64; ++i)
+                            tma_load_2d(map, &bk.full[stage], b + i * kBox, nt * kN + 64 * i, krow);
+                    }
+                    pending |= 1u << stage;
+                    pending_phase = (pending_phase & ~(1u << stage)) | (phase << stage);
+                    if (++stage == kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (!ok)
+                for (int s = 0; s < kStages; ++s)
+                    if (pending & (1u << s)) drain_wait(&bk.full[s], (pending_phase >> s) & 1u);
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        if (lane == 0) {
+            int stage = 0, acc = 0;
+            uint32_t phase = 0, acc_phase = 0;
+            bool ok = true, issued = false;
+            for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+                if (!mbar_wait_bounded(&bk.tmem_empty[acc], acc_phase ^ 1u, abort_flag,
+                                       args.status)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kN);
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    if (!mbar_wait_bounded(&bk.full[stage], phase, abort_flag, args.status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t ad = sw128_kmajor_desc(smem_u32(sA + stage * kABytes));
+                    const uint32_t bs = smem_u32(sB + stage * kBBytes);
+                    const uint64_t bd = kBmn ? sw128_mn_desc(bs) : sw128_kmajor_desc(bs);
+#pragma unroll
+                    for (int k = 0; k < kBK / 16; ++k)
+                        umma_bf16(d_tmem, ad + kKStep * k, bd + (kBmn ? kMnStep : kKStep) * k,
+                                  kIdesc, (kb | k) != 0);
+                    umma_commit(&bk.empty[stage]);
+                    issued = true;
+                    if (++stage == kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                umma_commit(&bk.tmem_full[acc]);
+                acc ^= 1;
+                if (acc == 0) acc_phase ^= 1u;
+            }
+            if (!ok && issued) {
+                umma_commit(&bk.drain);
+                drain_wait(&bk.drain, 0);
+            }
+        }
+        __syncwarp();
+    } else {
+        const int q = warp & 3;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+            int e, row0, row_end, nt;
+            tile_of(tile, e, row0, row_end, nt);
+            if (!bar_all(mbar_wait_bounded(&bk.tmem_full[acc], acc_phase, abort_flag,
+                                           args.status),
+                         kVoteBarrier, kEpiThreads))
+                break;
+            tc_fence_after();
+            const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                                   static_cast<uint32_t>(acc * kN);
+            const int row = row0 + q * 32 + lane;
+            const bool valid = row < row_end;
+            if (MODE == kModeDUV) {
+                const int h = args.h;
+                const float* g = args.dH + static_cast<size_t>(row) * h;
+                __nv_bfloat16* du = static_cast<__nv_bfloat16*>(args.out) + static_cast<size_t>(row) * 2 * h;
+                const int col0 = nt * 128;
+#pragma unroll 1
+                for (int ch = 0; ch < 4; ++ch) {
+                    uint32_t a[32], b[32];
+                    tmem_ld_32cols(tbase + ch * 32, a);
+                    tmem_ld_32cols(tbase + 128 + ch * 32, b);
+                    tmem_ld_wait();
+                    const int c0 = col0 + ch * 32;
+                    if (valid && c0 < h) {
+                        // h % 64 == 0, so a 32-column chunk is either whole or absent
+                        float gv[32];
+#pragma unroll
+                        for (int v = 0; v < 8; ++v) {
+                            const float4 t4 = *reinterpret_cast<const float4*>(g + c0 + 4 * v);
+                            gv[4 * v] = t4.x;
+                            gv[4 * v + 1] = t4.y;
+                            gv[4 * v + 2] = t4.z;
+                            gv[4 * v + 3] = t4.w;
+                        }
+                        uint32_t pu[16], pv[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            float ru[2], rv[2];
+#pragma unroll
+                            for (int u = 0; u < 2; ++u) {
+                                const float av = bits_f32(a[2 * i + u]);
+                                const float bv = bits_f32(b[2 * i + u]);
+                                const float s = 1.0f / (1.0f + __expf(-av));
+                                ru[u] = gv[2 * i + u] * bv * (s * (1.0f + av * (1.0f - s)));
+                                rv[u] = gv[2 * i + u] * (av * s);
+                            }
+                            pu[i] = pack_bf16x2(ru[0], ru[1]);
+                            pv[i] = pack_bf16x2(rv[0], rv[1]);
+                        }
+#pragma unroll
+                        for (int v = 0; v < 4; ++v) {
+                            *reinterpret_cast<uint4*>(du + c0 + 8 * v) =
+                                make_uint4(pu[4 * v], pu[4 * v + 1], pu[4 * v + 2], pu[4 * v + 3]);
+                            *reinterpret_cast<uint4*>(du + h + c0 + 8 * v) =
+                                make_uint4(pv[4 * v], pv[4 * v + 1], pv[4 * v + 2], pv[4 * v + 3]);
+                        }
+                    }
+                }
+            } else {
+                float* out = static_cast<float*>(args.out) + static_cast<size_t>(row) * args.N;
+                const int col0 = nt * kN;
+#pragma unroll 1
+                for (int ch = 0; ch < 8; ++ch) {
+                    uint32_t v[32];
+                    tmem_ld_32cols(tbase + ch * 32, v);
+                    tmem_ld_wait();
+                    if (valid) {
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            const int col = col0 + ch * 32 + j * 4;
+                            if (col < args.N)
+                                *reinterpret_cast<float4*>(out + col) =
+                                    make_float4(bits_f32(v[4 * j]), bits_f32(v[4 * j + 1]),
+                                                bits_f32(v[4 * j + 2]), bits_f32(v[4 * j + 3]));
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&bk.tmem_empty[acc]);
+            acc ^= 1;
+            if (acc == 0) acc_phase ^= 1u;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, kTmemCols);
+    }
+}
+
+// ================================================================ weight gradients
+// out[e][m][n] = sum over the rows r of expert e of A[r, m] * B[r, n]: both operands
+// are grouped activations, row-major with m / n contiguous (MN-major).  Tiles are
+// (expert, 256-column block, 128-row block), row blocks inner so that consecutive
+// tiles share B.  An expert with no rows gets a zero tile.
+//   kModeW2 : A = dY [rows, d], B = H [rows, h]         -> dW2 [E, d, h]
+//   kModeW13: A = [du dv] [rows, 2h], B = x [rows, d]   -> dW1 [E, h, d] (m < h),
+//                                                          dW3 [E, h, d] (m >= h)
+struct WArgs {
+    const int32_t* offsets;
+    int E;
+    int rows;
+    int M;
+    int N;
+    int m_tiles;
+    int n_tiles;
+    int split;       // output rows m < split go to out0, the rest to out1
+    float* out0;
+    float* out1;
+    uint32_t* status;
+    int cap;
+};
+
+template <int MODE>
+__global__ void __launch_bounds__(kThreads, 1)
+    bwd_wgrad_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                     const WArgs args) {
+    constexpr uint32_t kIdesc = idesc_major(kBM, kN, true, true);
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint8_t* sA = smem;
+    uint8_t* sB = smem + kStages * kABytes;
+    Book& bk = *reinterpret_cast<Book*>(smem + kStages * kStageBytes);
+    volatile int* abort_flag = &bk.abort_flag;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int E = args.E;
+
+    if (threadIdx.x == 0) init_barriers(bk);
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+    }
+    if (warp == 1) tmem_alloc(&bk.tmem_base, kTmemCols);
+    if (threadIdx.x == 0) load_groups(bk, args.offsets, E, args.rows, args.cap);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = bk.tmem_base;
+    const int per_e = args.m_tiles * args.n_tiles;
+    const int total = E * per_e;
+
+    auto tile_of = [&](int tile, int& e, int& mt, int& nt, int& r0, int& n_rows) {
+        e = tile / per_e;
+        const int local = tile - e * per_e;
+        mt = local % args.m_tiles;
+        nt = local / args.m_tiles;
+        r0 = bk.off[e];
+        n_rows = bk.end[e] - bk.off[e];
+    };
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0, pending = 0, pending_phase = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+                int e, mt, nt, r0, n_rows;
+                tile_of(tile, e, mt, nt, r0, n_rows);
+                const int nkb = (n_rows + kBK - 1) / kBK;
+                for (int kb = 0; kb < nkb; ++kb) {
+                    if (!mbar_wait_bounded(&bk.empty[stage], phase ^ 1u, abort_flag,
+                                           args.status)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&bk.full[stage], kStageBytes);
+                    const int r = r0 + kb * kBK;
+                    uint8_t* a = sA + stage * kABytes;
+                    uint8_t* b = sB + stage * kBBytes;
+#pragma unroll
+                    for (int i = 0; i < kBM / 64; ++i)
+                        tma_load_2d(&tmA, &bk.full[stage], a + i * kBox, mt * kBM + 64 * i, r);
+#pragma unroll
+                    for (int i = 0; i < kN / 64; ++i)
+                        tma_load_2d(&tmB, &bk.full[stage], b + i * kBox, nt * kN + 64 * i, r);
+                    pending |= 1u << stage;
+                    pending_phase = (pending_phase & ~(1u << stage)) | (phase << stage);
+                    if (++stage == kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (!ok)
+                for (int s = 0; s < kStages; ++s)
+                    if (pending & (1u << s)) drain_wait(&bk.full[s], (pending_phase >> s) & 1u);
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // The whole warp runs this loop: lane 0 waits and issues, all lanes zero the
+        // rows of a last partial K block that belong to the next expert.
+        int stage = 0, acc = 0;
+        uint32_t phase = 0, acc_phase = 0;
+        bool ok = true, issued = false;
+        for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+            int e, mt, nt, r0, n_rows;
+            tile_of(tile, e, mt, nt, r0, n_rows);
+            const int nkb = (n_rows + kBK - 1) / kBK;
+            if (nkb == 0) continue;  // zero tile: written by the epilogue alone
+            int got = 1;
+            if (lane == 0)
+                got = mbar_wait_bounded(&bk.tmem_empty[acc], acc_phase ^ 1u, abort_flag,
+                                        args.status);
+            ok = __shfl_sync(0xffffffffu, got, 0) != 0;
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kN);
+            for (int kb = 0; kb < nkb; ++kb) {
+                if (lane == 0) got = mbar_wait_bounded(&bk.full[stage], phase, abort_flag, args.status);
+                ok = __shfl_sync(0xffffffffu, got, 0) != 0;
+                if (!ok) break;
+                const int kv = n_rows - kb * kBK;  // rows of this block inside the group
+                if (kv < kBK) {
+                    // Rows kv..63 belong to the next group (or were dropped by the
+                    // capacity and never written): clear them in every A and B box.
+                    uint8_t* a = sA + stage * kABytes;
+                    uint8_t* b = sB + stage * kBBytes;
+                    const int nz = (kBK - kv) * 8;  // 16-byte chunks per box to clear
+                    constexpr int kBoxes = (kBM + kN) / 64;
+                    for (int i = lane; i < kBoxes * nz; i += 32) {
+                        const int box = i / nz, c = i - box * nz;
+                        uint8_t* base = box < kBM / 64 ? a + box * kBox : b + (box - kBM / 64) * kBox;
+                        *reinterpret_cast<uint4*>(base + kv * 128 + c * 16) =
+                            make_uint4(0u, 0u, 0u, 0u);
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                }
+                if (lane == 0) {
+                    tc_fence_after();
+                    const uint64_t ad = sw128_mn_desc(smem_u32(sA + stage * kABytes));
+                    const uint64_t bd = sw128_mn_desc(smem_u32(sB + stage * kBBytes));
+#pragma unroll
+                    for (int k = 0; k < kBK / 16; ++k)
+                        umma_bf16(d_tmem, ad + kMnStep * k, bd + kMnStep * k, kIdesc,
+                                  (kb | k) != 0);
+                    umma_commit(&bk.empty[stage]);
+                }
+                issued = true;
+                __syncwarp();
+                if (++stage == kStages) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+            if (!ok) break;
+            if (lane == 0) umma_commit(&bk.tmem_full[acc]);
+            __syncwarp();
+            acc ^= 1;
+            if (acc == 0) acc_phase ^= 1u;
+        }
+        if (!ok && issued && lane == 0) {
+            umma_commit(&bk.drain);
+            drain_wait(&bk.drain, 0);
+        }
+        __syncwarp();
+    } else {
+        const int q = warp & 3;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+            int e, mt, nt, r0, n_rows;
+            tile_of(tile, e, mt, nt, r0, n_rows);
+            const int m = mt * kBM + q * 32 + lane;
+            const bool mvalid = m < args.M;
+            float* out = m < args.split
+                             ? args.out0 + (static_cast<size_t>(e) * args.split + m) * args.N
+                             : args.out1 + (static_cast<size_t>(e) * (args.M - args.split) +
+                                            (m - args.split)) * args.N;
+            const int col0 = nt * kN;
+            if (n_rows == 0) {
+                if (mvalid)
+                    for (int col = col0; col < col0 + kN && col < args.N; col += 4)
+                        *reinterpret_cast<float4*>(out + col) = make_float4(0.f, 0.f, 0.f, 0.f);
+                continue;
+            }
+            if (!mbar_wait_bounded(&bk.tmem_full[acc], acc_phase, abort_flag, args.status)) break;
+            tc_fence_after();
+            const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                                   static_cast<uint32_t>(acc * kN);
+#pragma unroll 1
+            for (int ch = 0; ch < 8; ++ch) {
+                uint32_t v[32];
+                tmem_ld_32cols(tbase + ch * 32, v);
+                tmem_ld_wait();
+                if (mvalid) {
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const int col = col0 + ch * 32 + j * 4;
+                        if (col < args.N)
+                            *reinterpret_cast<float4*>(out + col) =
+                                make_float4(bits_f32(v[4 * j]), bits_f32(v[4 * j + 1]),
+                                            bits_f32(v[4 * j + 2]), bits_f32(v[4 * j + 3]));
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&bk.tmem_empty[acc]);
+            acc ^= 1;
+            if (acc == 0) acc_phase ^= 1u;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, kTmemCols);
+    }
+}
+
+// ================================================================ CUDA-core kernels
+constexpr int kPrepThreads = 256;
+
+// Is pair (t, j) kept?  (expert id valid, grouped row in range, within capacity)
+__device__ __forceinline__ bool pair_kept(const int32_t* idx, const int32_t* offsets,
+                                          const int32_t* inv, int f, int E, int P, int cap) {
+    const unsigned e = static_cast<unsigned>(idx[f]);
+    const unsigned r = static_cast<unsigned>(inv[f]);
+    if (e >= static_cast<unsigned>(E) || r >= static_cast<unsigned>(P)) return false;
+    return cap == INT_MAX || static_cast<int>(r) - offsets[e] < cap;
+}
+
+// One block per token: dY rows of its two pairs, dw, and the token's logit gradients.
+// Y is the sum of nsplit fp32 arrays split_stride floats apart (in order).
+__global__ void __launch_bounds__(kPrepThreads)
+    bwd_prep_kernel(const __nv_bfloat16* __restrict__ dy, const int32_t* __restrict__ idx,
+                    const float* __restrict__ w, const int32_t* __restrict__ inv,
+                    const int32_t* __restrict__ offsets, int T, int d, int E, int cap,
+                    const float* __restrict__ Y, int nsplit, size_t split_stride,
+                    __nv_bfloat16* __restrict__ dY, float* __restrict__ dw,
+                    float* __restrict__ dlogits) {
+    __shared__ float red[2][kPrepThreads / 32];
+    const int P = 2 * T;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int t = blockIdx.x; t < T; t += gridDim.x) {
+        const bool keep0 = pair_kept(idx, offsets, inv, 2 * t, E, P, cap);
+        const bool keep1 = pair_kept(idx, offsets, inv, 2 * t + 1, E, P, cap);
+        const int r0 = inv[2 * t], r1 = inv[2 * t + 1];
+        const float w0 = keep0 ? w[2 * t] : 0.f, w1 = keep1 ? w[2 * t + 1] : 0.f;
+        float s0 = 0.f, s1 = 0.f;
+        for (int c = threadIdx.x; c < d; c += blockDim.x) {
+            const float g = __bfloat162float(dy[static_cast<size_t>(t) * d + c]);
+            if (keep0) {
+                float y = Y[static_cast<size_t>(r0) * d + c];
+                for (int s = 1; s < nsplit; ++s) y += Y[s * split_stride + static_cast<size_t>(r0) * d + c];
+                s0 = fmaf(g, y, s0);
+                dY[static_cast<size_t>(r0) * d + c] = __float2bfloat16_rn(w0 * g);
+            }
+            if (keep1) {
+                float y = Y[static_cast<size_t>(r1) * d + c];
+                for (int s = 1; s < nsplit; ++s) y += Y[s * split_stride + static_cast<size_t>(r1) * d + c];
+                s1 = fmaf(g, y, s1);
+                dY[static_cast<size_t>(r1) * d + c] = __float2bfloat16_rn(w1 * g);
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            s0 += __shfl_xor_sync(0xffffffffu, s0, o);
+            s1 += __shfl_xor_sync(0xffffffffu, s1, o);
+        }
+        if (lane == 0) {
+            red[0][warp] = s0;
+            red[1][warp] = s1;
+        }
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            float a = 0.f, b = 0.f;
+            for (int i = 0; i < kPrepThreads / 32; ++i) {
+                a += red[0][i];
+                b += red[1][i];
+            }
+            dw[2 * t] = a;
+            dw[2 * t + 1] = b;
+            // w1 = sigma(l_i1 - l_i2), w2 = 1 - w1 (the stored weights, even if dropped)
+            const float gap = (a - b) * w[2 * t] * w[2 * t + 1];
+            for (int e = 0; e < E; ++e) dlogits[static_cast<size_t>(t) * E + e] = 0.f;
+            const unsigned e0 = static_cast<unsigned>(idx[2 * t]);
+            const unsigned e1 = static_cast<unsigned>(idx[2 * t + 1]);
+            if (e0 < static_cast<unsigned>(E)) dlogits[static_cast<size_t>(t) * E + e0] += gap;
+            if (e1 < static_cast<unsigned>(E)) dlogits[static_cast<size_t>(t) * E + e1] -= gap;
+        }
+        __syncthreads();
+    }
+}
+
+// dx[t, c] = dX[r0, c] + dX[r1, c] (kept pairs) + sum_e dlogits[t, e] Wg[c, e], one rounding.
+__global__ void __launch_bounds__(kPrepThreads)
+    bwd_dx_kernel(const float* __restrict__ dX, const int32_t* __restrict__ idx,
+                  const int32_t* __restrict__ inv, const int32_t* __restrict__ offsets, int T,
+                  int d, int E, int cap, const float* __restrict__ dlogits,
+                  const __nv_bfloat16* __restrict__ Wg, __nv_bfloat16* __restrict__ dx) {
+    const int P = 2 * T;
+    const size_t n = static_cast<size_t>(T) * d;
+    for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
+         i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+        const int t = static_cast<int>(i / d);
+        const int c = static_cast<int>(i - static_cast<size_t>(t) * d);
+        float v = 0.f;
+        if (pair_kept(idx, offsets, inv, 2 * t, E, P, cap))
+            v += dX[static_cast<size_t>(inv[2 * t]) * d + c];
+        if (pair_kept(idx, offsets, inv, 2 * t + 1, E, P, cap))
+            v += dX[static_cast<size_t>(inv[2 * t + 1]) * d + c];
+        const float* dl = dlogits + static_cast<size_t>(t) * E;
+        const __nv_bfloat16* wr = Wg + static_cast<size_t>(c) * E;
+        for (int e = 0; e < E; ++e) v = fmaf(dl[e], __bfloat162float(wr[e]), v);
+        dx[i] = __float2bfloat16_rn(v);
+    }
+}
+
+// dWg = x^T dlogits in two deterministic passes: per chunk of kWgChunk tokens a
+// partial [d, E], then the partials summed in chunk order.
+constexpr int kWgChunk = 256;
+
+__global__ void __launch_bounds__(kPrepThreads)
+    bwd_dwg_partial_kernel(const __nv_bfloat16* __restrict__ x, const float* __restrict__ dlogits,
+                           int T, int d, int E, float* __restrict__ part) {
+    __shared__ float dl[kWgChunk * kMaxExperts];
+    const int chunk = blockIdx.y;
+    const int t0 = chunk * kWgChunk;
+    const int nt = min(kWgChunk, T - t0);
+    for (int i = threadIdx.x; i < nt * E; i += blockDim.x)
+        dl[i] = dlogits[static_cast<size_t>(t0) * E + i];
+    __syncthreads();
+    const int c = blockIdx.x * blockDim.x + threadIdx.x;
+    if (c >= d) return;
+    float acc[kMaxExperts];
+#pragma unroll
+    for (int e = 0; e < kMaxExperts; ++e) acc[e] = 0.f;
+    for (int t = 0; t < nt; ++t) {
+        const float xv = __bfloat162float(x[static_cast<size_t>(t0 + t) * d + c]);
+#pragma unroll
+        for (int e = 0; e < kMaxExperts; ++e)
+            if (e < E) acc[e] = fmaf(xv, dl[t * E + e], acc[e]);
+    }
+    float* out = part + (static_cast<size_t>(chunk) * d + c) * E;
+#pragma unroll
+    for (int e = 0; e < kMaxExperts; ++e)
+        if (e < E) out[e] = acc[e];
+}
+
+__global__ void __launch_bounds__(kPrepThreads)
+    bwd_dwg_reduce_kernel(const float* __restrict__ part, int nchunk, int d, int E,
+                          float* __restrict__ dWg) {
+    const size_t n = static_cast<size_t>(d) * E;
+    for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
+         i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+        float s = part[i];
+        for (int c = 1; c < nchunk; ++c) s += part[static_cast<size_t>(c) * n + i];
+        dWg[i] = s;
+    }
+}
+
+// Opt each GEMM kernel into its dynamic shared memory once per device.  `slot` names
+// the kernel: the instantiations share one function type, so it cannot be the key.
+enum KernelSlot { kSlotDH, kSlotDUV, kSlotDX, kSlotW2, kSlotW13, kSlots };
+template <typename Kern>
+void configure(Kern kern, KernelSlot slot) {
+    static int configured[kSlots][64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && !configured[slot][dev]) {
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+        configured[slot][dev] = 1;
+    }
+}
+
+int grid_for(long long work, int cap) {
+    return static_cast<int>(work < 1 ? 1 : (work < cap ? work : cap));
+}
+
+}  // namespace
+
+size_t bwd_dwg_chunks(int T) { return static_cast<size_t>((T + kWgChunk - 1) / kWgChunk); }
+
+cudaError_t launch_layer_backward(const BwdArgs& a, cudaStream_t s) {
+    const int T = a.T, d = a.d, h = a.h, E = a.E, P = 2 * T;
+    const int sms = device_sm_count();
+    cudaError_t err;
+    // 1. dY, dw, dlogits
+    err = launch_k(bwd_prep_kernel, grid_for(T, 8 * sms), kPrepThreads, 0, s,
+                   static_cast<const __nv_bfloat16*>(a.dy), a.idx, a.w, a.inv, a.offsets, T, d, E,
+                   a.cap, a.Y, a.nsplit, a.split_stride, static_cast<__nv_bfloat16*>(a.dY), a.dw,
+                   a.dlogits);
+    if (err != cudaSuccess) return err;
+
+    CUtensorMap m_dY128, m_W2, m_x, m_W1r, m_W3r, m_duv128, m_W1mn, m_W3mn;
+    if (!encode_bf16_2d(&m_dY128, a.dY, P, d, kBM) ||
+        !encode_bf16_2d(&m_W2, a.W2, static_cast<uint64_t>(E) * d, h, 64) ||
+        !encode_bf16_2d(&m_x, a.x_perm, P, d, kBM) ||
+        !encode_bf16_2d(&m_W1r, a.W1, static_cast<uint64_t>(E) * h, d, 128) ||
+        !encode_bf16_2d(&m_W3r, a.W3, static_cast<uint64_t>(E) * h, d, 128) ||
+        !encode_bf16_2d(&m_duv128, a.DUV, P, 2 * h, kBM) ||
+        !encode_bf16_2d(&m_W1mn, a.W1, static_cast<uint64_t>(E) * h, d, 64) ||
+        !encode_bf16_2d(&m_W3mn, a.W3, static_cast<uint64_t>(E) * h, d, 64))
+        return cudaErrorInvalidValue;
+    const long long row_blocks = (static_cast<long long>(P) + 127LL * E) / kBM;
+
+    // 2. dH = dY W2_e
+    {
+        RowArgs r{a.offsets, E, P, d, h, (h + kN - 1) / kN, h, d, a.dH, nullptr, a.status, a.cap};
+        configure(bwd_rows_kernel<kModeDH>, kSlotDH);
+        err = launch_k(bwd_rows_kernel<kModeDH>, grid_for(row_blocks * r.n_tiles, sms), kThreads,
+                       kSmemBytes, s, m_dY128, m_W2, m_W2, r);
+        if (err != cudaSuccess) return err;
+    }
+    // 3. du, dv (recomputes a and b)
+    {
+        RowArgs r{a.offsets, E, P, d, h, (h + 127) / 128, h, d, a.DUV, a.dH, a.status, a.cap};
+        configure(bwd_rows_kernel<kModeDUV>, kSlotDUV);
+        err = launch_k(bwd_rows_kernel<kModeDUV>, grid_for(row_blocks * r.n_tiles, sms),
+                       kThreads, kSmemBytes, s, m_x, m_W1r, m_W3r, r);
+        if (err != cudaSuccess) return err;
+    }
+    // 4. dX = [du dv] [W1_e ; W3_e]
+    {
+        RowArgs r{a.offsets, E, P, 2 * h, d, (d + kN - 1) / kN, h, d, a.dX, nullptr, a.status,
+                  a.cap};
+        configure(bwd_rows_kernel<kModeDX>, kSlotDX);
+        err = launch_k(bwd_rows_kernel<kModeDX>, grid_for(row_blocks * r.n_tiles, sms), kThreads,
+                       kSmemBytes, s, m_duv128, m_W1mn, m_W3mn, r);
+        if (err != cudaSuccess) return err;
+    }
+    // 5. dx
+    {
+        const long long n = static_cast<long long>(T) * d;
+        err = launch_k(bwd_dx_kernel, grid_for((n + kPrepThreads - 1) / kPrepThreads, 8 * sms),
+                       kPrepThreads, 0, s, static_cast<const float*>(a.dX), a.idx, a.inv,
+                       a.offsets, T, d, E, a.cap, static_cast<const float*>(a.dlogits),
+                       static_cast<const __nv_bfloat16*>(a.Wg), static_cast<__nv_bfloat16*>(a.dx));
+        if (err != cudaSuccess) return err;
+    }
+    // 6. weight gradients
+    CUtensorMap m_dY64, m_H64, m_duv64, m_x64;
+    if (!encode_bf16_2d(&m_dY64, a.dY, P, d, 64) || !encode_bf16_2d(&m_H64, a.H, P, h, 64) ||
+        !encode_bf16_2d(&m_duv64, a.DUV, P, 2 * h, 64) ||
+        !encode_bf16_2d(&m_x64, a.x_perm, P, d, 64))
+        return cudaErrorInvalidValue;
+    {
+        WArgs w{a.offsets, E, P, d, h, (d + kBM - 1) / kBM, (h + kN - 1) / kN, d, a.dW2, a.dW2,
+                a.status, a.cap};
+        configure(bwd_wgrad_kernel<kModeW2>, kSlotW2);
+        err = launch_k(bwd_wgrad_kernel<kModeW2>,
+                       grid_for(static_cast<long long>(E) * w.m_tiles * w.n_tiles, sms), kThreads,
+                       kSmemBytes, s, m_dY64, m_H64, w);
+        if (err != cudaSuccess) return err;
+    }
+    {
+        WArgs w{a.offsets, E, P, 2 * h, d, (2 * h + kBM - 1) / kBM, (d + kN - 1) / kN, h, a.dW1,
+                a.dW3, a.status, a.cap};
+        configure(bwd_wgrad_kernel<kModeW13>, kSlotW13);
+        err = launch_k(bwd_wgrad_kernel<kModeW13>,
+                       grid_for(static_cast<long long>(E) * w.m_tiles * w.n_tiles, sms), kThreads,
+                       kSmemBytes, s, m_duv64, m_x64, w);
+        if (err != cudaSuccess) return err;
+    }
+    // 7. dWg
+    {
+        const int nchunk = static_cast<int>(bwd_dwg_chunks(T));
+        err = launch_k(bwd_dwg_partial_kernel, dim3((d + kPrepThreads - 1) / kPrepThreads, nchunk),
+                       kPrepThreads, 0, s, static_cast<const __nv_bfloat16*>(a.x),
+                       static_cast<const float*>(a.dlogits), T, d, E, a.dwg_part);
+        if (err != cudaSuccess) return err;
+        const long long n = static_cast<long long>(d) * E;
+        err = launch_k(bwd_dwg_reduce_kernel, grid_for((n + kPrepThreads - 1) / kPrepThreads, 4 * sms),
+                       kPrepThreads, 0, s, static_cast<const float*>(a.dwg_part), nchunk, d, E,
+                       a.dWg);
+    }
+    return err;
+}
+
+}  // namespace moe

@@ -45,6 +45,7 @@ constexpr int kThreads = 192;    // TMA warp, MMA warp, 4 epilogue warps
 constexpr int kEpiThreads = 128;
 constexpr uint32_t kTmemCols = 128;
 constexpr int kXferBarrier = 1;  // named barrier id for the epilogue exchange
+constexpr int kVoteBarrier = 2;  // epilogue vote after a bounded wait
 
 enum DecodeMode { kSwiGLU = 0, kDown = 1 };
 
@@ -316,7 +317,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t acc_phase = 0;
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
             const Tile t = decode_tile(bk, E, args.n_wblocks, ksplit, NT, tile);
-            if (!mbar_wait_bounded(&bk.tmem_full[acc], acc_phase, abort_flag, args.status))
+            if (!bar_all(mbar_wait_bounded(&bk.tmem_full[acc], acc_phase, abort_flag, args.status),
+                         kVoteBarrier, kEpiThreads))
                 break;
             tc_fence_after();
             uint32_t v[NT];
@@ -669,7 +671,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t acc_phase = 0;
         for (int u = blockIdx.x; u < total; u += gridDim.x) {
             const FusedUnit f = fused_unit(bk, args, NT, num_kb1, kps, num_kb2, u);
-            if (!mbar_wait_bounded(&bk.tmem_full[acc], acc_phase, abort_flag, args.status))
+            if (!bar_all(mbar_wait_bounded(&bk.tmem_full[acc], acc_phase, abort_flag, args.status),
+                         kVoteBarrier, kEpiThreads))
                 break;
             tc_fence_after();
             uint32_t v[NT];

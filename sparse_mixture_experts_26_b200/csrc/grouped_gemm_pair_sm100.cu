@@ -58,6 +58,7 @@ constexpr int kXferBytes = 32 * 64 * 4;  // one 32-column chunk of b for 64 rows
 constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 1024 /*bookkeeping*/ +
                            kXferBytes;
 constexpr int kXferBarrier = 1;
+constexpr int kVoteBarrier = 2;  // epilogue vote after a bounded wait
 constexpr uint16_t kBothCtas = 0x3;
 
 enum Epilogue { kEpiSwiGLU = 0, kEpiStoreF32 = 1 };
@@ -300,7 +301,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t acc_phase = 0;
         for (int tile = pair; tile < total; tile += npairs) {
             const PairTile t = decode_pair_tile(bk, E, tile);
-            if (!mbar_wait_bounded(&bk.tmem_full[acc], acc_phase, abort_flag, args.status))
+            if (!bar_all(mbar_wait_bounded(&bk.tmem_full[acc], acc_phase, abort_flag, args.status),
+                         kVoteBarrier, kEpiThreads))
                 break;
             tc_fence_after();
             const uint32_t tlane = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +

@@ -409,12 +409,7 @@ cudaError_t launch_ffn_bf16(const void* x_perm, const int32_t* offsets, const vo
                             FfnOut* out, uint32_t* status, cudaStream_t s,
                             cudaEvent_t between, uint32_t* counters, int cap) {
     if (rows <= kDecodeMaxRows) {
-        // Largest split of the down projection's K blocks (at most partial_cap) that
-        // leaves no K range empty.
-        const int num_kb = (h + 63) / 64;
-        int ksplit = partials ? (partial_cap < kDecodeSplitK ? partial_cap : kDecodeSplitK) : 1;
-        while (ksplit > 1 && ((num_kb + ksplit - 1) / ksplit) * (ksplit - 1) >= num_kb) --ksplit;
-        if (ksplit < 1) ksplit = 1;
+        int ksplit = partials ? decode_ksplit(h, partial_cap) : 1;
         float* dst = ksplit > 1 ? partials : Y;
         cudaError_t err;
         err = cudaErrorNotSupported;

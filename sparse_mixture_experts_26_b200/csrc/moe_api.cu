@@ -103,6 +103,32 @@ T* at(void* ws, size_t off) {
     return reinterpret_cast<T*>(static_cast<char*>(ws) + off);
 }
 
+// Backward workspace regions (1 KiB aligned); the status word at offset 0.
+struct BwdLayout {
+    size_t status, dY, dw, dlogits, dH, DUV, dX, dwg_part, total;
+};
+
+BwdLayout bwd_layout(int T, int d, int h, int E) {
+    BwdLayout B{};
+    const size_t P = 2 * static_cast<size_t>(T);
+    size_t o = 0;
+    auto take = [&](size_t bytes) {
+        size_t at_ = o;
+        o = align_up(o + bytes, 1024);
+        return at_;
+    };
+    B.status = take(256);
+    B.dY = take(P * d * 2);
+    B.dw = take(P * 4);
+    B.dlogits = take(static_cast<size_t>(T) * E * 4);
+    B.dH = take(P * h * 4);
+    B.DUV = take(P * 2 * h * 2);
+    B.dX = take(P * d * 4);
+    B.dwg_part = take(bwd_dwg_chunks(T) * d * E * 4);
+    B.total = o;
+    return B;
+}
+
 }  // namespace
 }  // namespace moe
 
@@ -287,6 +313,70 @@ moe_status moe_layer_forward_events(const void* x, const void* Wg, const void* W
                                     cudaEvent_t* events, int n_events, cudaStream_t stream) {
     return layer_forward_impl(x, Wg, W1, W3, W2, T, d, h, E, k, dt, y, ws, ws_bytes, events,
                               n_events, stream, INT_MAX);
+}
+
+size_t moe_backward_workspace_bytes(int T, int d, int h, int E, int k, moe_dtype dt) {
+    if (check_shape(T, d, h, E, k, dt, true) != MOE_OK) return 0;
+    if (dt != MOE_BF16 || h % 64 != 0) return 0;
+    return bwd_layout(T, d, h, E).total;
+}
+
+moe_status moe_layer_backward(const void* x, const void* Wg, const void* W1, const void* W3,
+                              const void* W2, const void* dy, int T, int d, int h, int E, int k,
+                              moe_dtype dt, int capacity, void* dx, float* dWg, float* dW1,
+                              float* dW3, float* dW2, const void* fwd_ws, size_t fwd_ws_bytes,
+                              void* bwd_ws, size_t bwd_ws_bytes, cudaStream_t stream) {
+    moe_status st = check_shape(T, d, h, E, k, dt, true);
+    if (st != MOE_OK) return st;
+    if (dt != MOE_BF16 || h % 64 != 0) return MOE_ERR_UNSUPPORTED;
+    if (T == 0) return MOE_OK;
+    if (!ptrs_ok({x, Wg, W1, W3, W2, dy, dx, dWg, dW1, dW3, dW2, fwd_ws, bwd_ws}))
+        return MOE_ERR_INVALID_ARG;
+    const WsLayout L = ws_layout(T, d, h, E, k, dt);
+    const BwdLayout B = bwd_layout(T, d, h, E);
+    if (fwd_ws_bytes < L.total || bwd_ws_bytes < B.total) return MOE_ERR_WORKSPACE;
+    const int P = 2 * T;
+    // Where the forward left the expert outputs: split-K partials for small batches.
+    const int nsplit = P <= kDecodeMaxRows ? decode_ksplit(h, kDecodeSplitK) : 1;
+    void* fws = const_cast<void*>(fwd_ws);
+    BwdArgs a{};
+    a.T = T;
+    a.d = d;
+    a.h = h;
+    a.E = E;
+    a.cap = capacity < 0 ? INT_MAX : capacity;
+    a.dy = dy;
+    a.idx = at<int32_t>(fws, L.topk_idx);
+    a.w = at<float>(fws, L.topk_w);
+    a.inv = at<int32_t>(fws, L.inv_perm);
+    a.offsets = at<int32_t>(fws, L.offsets);
+    a.Y = nsplit > 1 ? at<float>(fws, L.Ypart) : at<float>(fws, L.Y);
+    a.nsplit = nsplit;
+    a.split_stride = static_cast<size_t>(P) * d;
+    a.x_perm = at<void>(fws, L.x_perm);
+    a.H = at<void>(fws, L.H);
+    a.x = x;
+    a.Wg = Wg;
+    a.W1 = W1;
+    a.W3 = W3;
+    a.W2 = W2;
+    a.dx = dx;
+    a.dWg = dWg;
+    a.dW1 = dW1;
+    a.dW3 = dW3;
+    a.dW2 = dW2;
+    a.dY = at<void>(bwd_ws, B.dY);
+    a.dw = at<float>(bwd_ws, B.dw);
+    a.dlogits = at<float>(bwd_ws, B.dlogits);
+    a.dH = at<float>(bwd_ws, B.dH);
+    a.DUV = at<void>(bwd_ws, B.DUV);
+    a.dX = at<float>(bwd_ws, B.dX);
+    a.dwg_part = at<float>(bwd_ws, B.dwg_part);
+    a.status = at<uint32_t>(bwd_ws, B.status);
+    PdlScope pdl(false);  // the backward kernels do not wait on griddepcontrol
+    cudaError_t err = launch_layer_backward(a, stream);
+    if (err == cudaErrorInvalidValue) return MOE_ERR_INVALID_ARG;  // tensor map refused
+    return finish(err, stream, a.status);
 }
 
 moe_status moe_selftest_wait_timeout(void* ws, size_t ws_bytes, double limit_seconds,

@@ -162,6 +162,44 @@ cudaError_t launch_combine(const float* Y, int nsplit, size_t split_stride,
                            const int32_t* inv_perm, const float* w, int T, int d, moe_dtype dt,
                            void* y, cudaStream_t s, const int32_t* idx = nullptr,
                            const int32_t* offsets = nullptr, int E = 0, int cap = INT_MAX);
+// K ranges of the small-batch down projection: the largest split (at most
+// partial_cap and kDecodeSplitK) that leaves no K range of 64-wide blocks empty.
+inline int decode_ksplit(int h, int partial_cap) {
+    const int num_kb = (h + 63) / 64;
+    int ksplit = partial_cap < kDecodeSplitK ? partial_cap : kDecodeSplitK;
+    while (ksplit > 1 && ((num_kb + ksplit - 1) / ksplit) * (ksplit - 1) >= num_kb) --ksplit;
+    return ksplit < 1 ? 1 : ksplit;
+}
+// Everything the backward pass reads and writes (bf16 layer; see backward_sm100.cu).
+struct BwdArgs {
+    int T, d, h, E, cap;
+    // upstream gradient and the forward's saved state
+    const void* dy;            // bf16 [T, d]
+    const int32_t* idx;        // [T, 2]
+    const float* w;            // [T, 2]
+    const int32_t* inv;        // [T, 2]
+    const int32_t* offsets;    // [E + 1]
+    const float* Y;            // expert outputs: sum of nsplit arrays [2T, d]
+    int nsplit;
+    size_t split_stride;       // floats between those arrays
+    const void* x_perm;        // bf16 [2T, d]
+    const void* H;             // bf16 [2T, h]
+    const void *x, *Wg, *W1, *W3, *W2;
+    // outputs
+    void* dx;                  // bf16 [T, d]
+    float *dWg, *dW1, *dW3, *dW2;
+    // scratch (backward workspace)
+    void* dY;                  // bf16 [2T, d]
+    float* dw;                 // [T, 2]
+    float* dlogits;            // [T, E]
+    float* dH;                 // [2T, h]
+    void* DUV;                 // bf16 [2T, 2h]: du then dv
+    float* dX;                 // [2T, d]
+    float* dwg_part;           // [ceil(T / 256), d, E]
+    uint32_t* status;
+};
+size_t bwd_dwg_chunks(int T);
+cudaError_t launch_layer_backward(const BwdArgs& a, cudaStream_t s);
 // Bounded-wait self-test (see moe_selftest_wait_timeout).
 cudaError_t launch_selftest_wait(uint32_t* status, uint32_t* scratch, unsigned long long limit_ns,
                                  cudaStream_t s);

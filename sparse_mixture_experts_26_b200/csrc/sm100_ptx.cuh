@@ -79,6 +79,23 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
     }
 }
 
+// True on every participating thread iff `v` is true on all `nthreads` threads
+// arriving at named barrier `id`.  Epilogue warps vote with it after a bounded wait,
+// so that all of them leave together when any one gave up (a later named barrier
+// would otherwise wait for threads that have left).
+__device__ __forceinline__ bool bar_all(bool v, uint32_t id, uint32_t nthreads) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "barrier.cta.red.and.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"(static_cast<uint32_t>(v)), "r"(id), "r"(nthreads)
+        : "memory");
+    return r != 0;
+}
+
 // Wait until *counter >= need (acquire, device scope).  Returns false (after setting
 // *abort_flag and the status word) once `limit_ns` has passed, or when another role
 // has set *abort_flag.

@@ -1,0 +1,179 @@
+"""Parity of the backward pass (training gradients) with the fp64 oracle, via the C ABI.
+
+The gradients pass through several bf16 roundings that the oracle does not make:
+the scaled upstream rows w*dy (one rounding each), H saved by the forward, and du,
+dv (one rounding each) feed tensor-core GEMMs with fp32 accumulation.  Each rounding
+is a relative error of at most 2^-9 per element, independent across elements, so
+over the three to four roundings on any path a relative Frobenius error of a few
+1e-3 is expected; the gate is 1e-2 (and 2e-2 for the router gradient, whose logit
+gap (dw1 - dw2) can cancel).  Full-size layers are checked on sampled tokens and
+sampled weight entries that the oracle computes one by one.
+"""
+import numpy as np
+import pytest
+import torch
+
+import sparse_mixture_experts_26_b200 as moe
+from oracle import moe_oracle as O
+from workloads import WORKLOADS, make_inputs, small
+
+pytestmark = pytest.mark.gpu
+
+BWD_TOL = 1e-2
+ROUTER_TOL = 2e-2
+
+
+def f64(t):
+    return t.detach().to(torch.float64).cpu().numpy()
+
+
+def rel_fro(a, b):
+    return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300))
+
+
+def seeded_dy(T, d, seed):
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    return torch.randn(T, d, generator=g).to(torch.bfloat16).cuda()
+
+
+def gpu_grads(inp, dy, capacity=-1):
+    x = inp["x"]
+    T, d = x.shape
+    E, h, _ = inp["W1"].shape
+    ws = moe.alloc_workspace(T, d, h, E, 2, x.dtype, x.device)
+    y = torch.empty_like(x)
+    moe.moe_layer_forward_capacity(x, inp["Wg"], inp["W1"], inp["W3"], inp["W2"], y, ws,
+                                   capacity)
+    out = moe.layer_backward(x, inp["Wg"], inp["W1"], inp["W3"], inp["W2"], dy, ws, capacity)
+    assert moe.moe_device_status(ws) == 0
+    return dict(zip(("dx", "dWg", "dW1", "dW3", "dW2"), out)), ws
+
+
+SHAPES = [  # (T, d, h, kind): decode-path and grouped-path forwards, ragged tiles
+    (1, 64, 128, "plain"), (16, 128, 256, "skew"), (37, 136, 192, "plain"),
+    (64, 256, 384, "plain"), (300, 136, 192, "plain"), (700, 256, 384, "skew"),
+    (1100, 256, 384, "plain"), (2500, 128, 256, "long"),
+]
+
+
+@pytest.mark.parametrize("T,d,h,kind", SHAPES)
+def test_backward_small_shapes(T, d, h, kind):
+    wl = small("bw", T=T, d=d, h=h, seed=500 + T, kind=kind)
+    inp = make_inputs(wl, "cuda")
+    dy = seeded_dy(T, d, 77 + T)
+    g, _ = gpu_grads(inp, dy)
+    c = {k: f64(v) for k, v in inp.items()}
+    ref = O.moe_layer_backward(c["x"], c["Wg"], c["W1"], c["W3"], c["W2"], f64(dy))
+    for k in ("dx", "dW1", "dW3", "dW2"):
+        err = rel_fro(f64(g[k]), ref[k])
+        assert err <= BWD_TOL, (k, err)
+    assert rel_fro(f64(g["dWg"]), ref["dWg"]) <= ROUTER_TOL
+    # experts that received no rows get exact zeros
+    counts = np.bincount(ref["fwd"]["idx"].ravel(), minlength=wl.E)
+    for e in np.flatnonzero(counts == 0):
+        assert not g["dW1"][e].any() and not g["dW3"][e].any() and not g["dW2"][e].any()
+
+
+@pytest.mark.parametrize("T,d,h,cap", [(16, 128, 256, 3), (300, 136, 192, 40),
+                                       (1500, 136, 192, 300)])
+def test_backward_with_capacity(T, d, h, cap):
+    wl = small("bwc", T=T, d=d, h=h, seed=600 + T, kind="skew")
+    inp = make_inputs(wl, "cuda")
+    dy = seeded_dy(T, d, 91 + T)
+    g, _ = gpu_grads(inp, dy, cap)
+    c = {k: f64(v) for k, v in inp.items()}
+    ref = O.moe_layer_backward(c["x"], c["Wg"], c["W1"], c["W3"], c["W2"], f64(dy), capacity=cap)
+    assert not ref["fwd"]["keep"].all()
+    for k in ("dx", "dW1", "dW3", "dW2"):
+        assert rel_fro(f64(g[k]), ref[k]) <= BWD_TOL, k
+    assert rel_fro(f64(g["dWg"]), ref["dWg"]) <= ROUTER_TOL
+
+
+def test_backward_is_deterministic_and_rejects_unsupported():
+    wl = small("bwd", T=300, d=136, h=192, seed=3, kind="plain")
+    inp = make_inputs(wl, "cuda")
+    dy = seeded_dy(300, 136, 5)
+    g1, ws = gpu_grads(inp, dy)
+    out2 = moe.layer_backward(inp["x"], inp["Wg"], inp["W1"], inp["W3"], inp["W2"], dy, ws)
+    for k, v in zip(("dx", "dWg", "dW1", "dW3", "dW2"), out2):
+        assert torch.equal(v, g1[k]), k
+    assert moe.moe_backward_workspace_bytes(16, 128, 200, 8) == 0       # h % 64 != 0
+    assert moe.moe_backward_workspace_bytes(16, 128, 256, 8, 2, torch.float32) == 0
+
+
+# ---------------------------------------------------------------- full size, sampled
+
+def _sampled_reference(inp, dy, tokens, entries):
+    """fp64 oracle values of dx[t] for `tokens` and of single weight-gradient entries
+    (name, e, i, j), computed from the definitions one at a time."""
+    x = f64(inp["x"])
+    Wg = f64(inp["Wg"])
+    dyn = f64(dy)
+    logits = O.router_logits(x, Wg)
+    idx = O.top2_select(logits)
+    w = O.gate_weights(logits, idx)
+    W1, W3, W2 = inp["W1"], inp["W3"], inp["W2"]
+    out = {}
+    for t in tokens:
+        dxt = np.zeros(x.shape[1])
+        dws = []
+        for j in range(2):
+            e = int(idx[t, j])
+            W1e, W3e, W2e = (f64(W[e]) for W in (W1, W3, W2))
+            a = W1e @ x[t]
+            b = W3e @ x[t]
+            Y = W2e @ (O.silu(a) * b)
+            dws.append(float(dyn[t] @ Y))
+            dH = W2e.T @ (w[t, j] * dyn[t])
+            s = 1.0 / (1.0 + np.exp(-a))
+            da = dH * b * s * (1.0 + a * (1.0 - s))
+            db = dH * O.silu(a)
+            dxt += W1e.T @ da + W3e.T @ db
+        gap = (dws[0] - dws[1]) * w[t, 0] * w[t, 1]
+        dxt += gap * (Wg[:, idx[t, 0]] - Wg[:, idx[t, 1]])
+        out[("dx", t)] = dxt
+    for name, e, i, j in entries:
+        sel = np.argwhere(idx == e)  # (token, slot) pairs of expert e
+        ts, js = sel[:, 0], sel[:, 1]
+        xe = x[ts]
+        g = w[ts, js][:, None] * dyn[ts]  # dY rows of expert e
+        W1e, W3e, W2e = (f64(W[e]) for W in (W1, W3, W2))
+        if name == "dW2":  # dW2[e][i, j] = sum_r dY[r, i] H[r, j]
+            a = xe @ W1e[j]
+            b = xe @ W3e[j]
+            out[(name, e, i, j)] = float(g[:, i] @ (O.silu(a) * b))
+        else:  # dW1 / dW3 [e][j, i] = sum_r du|dv[r, j] x[r, i]
+            a = xe @ W1e[j]
+            b = xe @ W3e[j]
+            dH = g @ W2e[:, j]
+            s = 1.0 / (1.0 + np.exp(-a))
+            d_ = dH * b * s * (1.0 + a * (1.0 - s)) if name == "dW1" else dH * O.silu(a)
+            out[(name, e, j, i)] = float(d_ @ xe[:, i])
+    return out
+
+
+@pytest.mark.parametrize("workload", ["decode", "prefill"])
+def test_backward_full_size_sampled(workload):
+    wl = WORKLOADS[workload]
+    inp = make_inputs(wl, "cuda")
+    dy = seeded_dy(wl.T, wl.d, 4242)
+    g, _ = gpu_grads(inp, dy)
+    rng = np.random.default_rng(11)
+    tokens = sorted(set([0, wl.T - 1] + list(rng.integers(0, wl.T, 4))))
+    entries = [(n, int(rng.integers(0, wl.E)), int(rng.integers(0, wl.d)),
+                int(rng.integers(0, wl.h))) for n in ("dW2", "dW1", "dW3") for _ in range(3)]
+    ref = _sampled_reference(inp, dy, tokens, entries)
+    dx = f64(g["dx"])
+    for t in tokens:
+        assert rel_fro(dx[t], ref[("dx", t)]) <= BWD_TOL, t
+    # weight entries: compare against the entry's own scale (sum of |terms| would be
+    # tighter; the norm of the whole gradient row is a stable, generous scale)
+    for key, v in ref.items():
+        if key[0] == "dx":
+            continue
+        name, e, r_, c_ = key
+        got = g[name][e, r_, c_].item()
+        row = f64(g[name][e, r_])
+        scale = np.linalg.norm(row) / np.sqrt(row.size) + 1e-30
+        assert abs(got - v) <= BWD_TOL * max(abs(v), scale), (key, got, v)

@@ -134,6 +134,30 @@ def test_layer_bf16_small_shapes(T, d, h, kind):
     assert torch.equal(layer_y(inp), g["y"])
 
 
+@pytest.mark.parametrize("T,kind", [(1, "plain"), (16, "skew"), (40, "plain"), (64, "skew")])
+def test_small_batch_layer_repeated_calls(T, kind):
+    """The small-batch expert FFN is one cooperative launch whose dependency counters
+    must be zero again after every call: repeated calls on one workspace, interleaved
+    with a smaller batch, each into an output pre-filled with NaN, reproduce the
+    step-wise result bit for bit."""
+    wl = small("rep", T=T, d=256, h=384, seed=900 + T, kind=kind)
+    inp = make_inputs(wl, "cuda")
+    x, Wg, W1, W3, W2 = (inp[k] for k in ("x", "Wg", "W1", "W3", "W2"))
+    Ts = max(1, T // 3)
+    sub = {k: (v[:Ts].contiguous() if k == "x" else v) for k, v in inp.items()}
+    ref = run_steps(inp, wl.E)["y"]
+    ref_sub = run_steps(sub, wl.E)["y"]
+    ws = moe.alloc_workspace(T, 256, 384, wl.E, 2, x.dtype, x.device)
+    for _ in range(3):
+        y = torch.full_like(x, float("nan"))
+        moe.moe_layer_forward(x, Wg, W1, W3, W2, y, ws)
+        assert torch.equal(y, ref)
+        y_sub = torch.full_like(sub["x"], float("nan"))
+        moe.moe_layer_forward(sub["x"], Wg, W1, W3, W2, y_sub, ws)
+        assert torch.equal(y_sub, ref_sub)
+    assert moe.moe_device_status(ws) == 0
+
+
 @pytest.mark.parametrize("T,d,h", [(64, 128, 256), (1, 8, 8), (37, 24, 40), (300, 64, 96)])
 def test_layer_f32(T, d, h):
     wl = WORKLOADS["tiny_f32"] if (T, d, h) == (64, 128, 256) else small(
