@@ -184,9 +184,10 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ oracle timing
-def oracle_tokens_per_s(inp_cpu, sample_tokens, budget_s: float):
+def oracle_tokens_per_s(inp_cpu, sample_tokens, budget_s: float, backward: bool = False):
     """Time the CPU oracle (as it stands) on ``sample_tokens`` tokens of the workload,
-    repeating until ``budget_s`` seconds; returns (tokens/s, threads, repeats)."""
+    repeating until ``budget_s`` seconds; returns (tokens/s, threads, repeats).  With
+    ``backward`` the oracle's gradient pass (which runs its own forward) is timed."""
     from oracle import moe_oracle as O
     try:
         from threadpoolctl import threadpool_info
@@ -195,15 +196,32 @@ def oracle_tokens_per_s(inp_cpu, sample_tokens, budget_s: float):
     except Exception:
         threads = os.cpu_count() or 1
     x = inp_cpu["x"][:sample_tokens]
+    dy = backward_dy_cpu(x.shape)
     t0 = time.perf_counter()
     reps = 0
     while True:
-        O.moe_layer(x, inp_cpu["Wg"], inp_cpu["W1"], inp_cpu["W3"], inp_cpu["W2"])
+        if backward:
+            O.moe_layer_backward(x, inp_cpu["Wg"], inp_cpu["W1"], inp_cpu["W3"], inp_cpu["W2"],
+                                 dy)
+        else:
+            O.moe_layer(x, inp_cpu["Wg"], inp_cpu["W1"], inp_cpu["W3"], inp_cpu["W2"])
         reps += 1
         if time.perf_counter() - t0 >= budget_s:
             break
     dt = time.perf_counter() - t0
     return reps * sample_tokens / dt, int(threads), reps, dt
+
+
+def backward_dy(T: int, d: int, seed: int = 4242):
+    """The seeded upstream gradient dL/dy of the backward benchmark (bf16 values)."""
+    import torch
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    return torch.randn(T, d, generator=g).to(torch.bfloat16)
+
+
+def backward_dy_cpu(shape):
+    return backward_dy(*shape).float().numpy()
 
 
 def cpu_copy(inp):
@@ -423,6 +441,183 @@ def run_ours(args):
     }
 
 
+# ------------------------------------------------------------------ our arm, backward
+BWD_METRIC = "MoE-layer backward tokens/s (dx, dW1, dW3, dW2, dWg) and % of bf16 TC peak"
+BWD_STAGES = ["prep (dY, dw, dlogits)", "dH = dY W2", "du, dv (recompute a, b)",
+              "dX = [du dv][W1; W3]", "dx combine", "dW2", "dW1 + dW3", "dWg"]
+BWD_KERNELS = {  # stage index -> (kernel, profile tag, flops per launch as a function)
+    1: ("bwd_rows_kernel<kModeDH>", "bwd_dh"),
+    2: ("bwd_rows_kernel<kModeDUV>", "bwd_duv"),
+    3: ("bwd_rows_kernel<kModeDX>", "bwd_dx"),
+    5: ("bwd_wgrad_kernel<kModeW2>", "bwd_wgrad_w2"),
+    6: ("bwd_wgrad_kernel<kModeW13>", "bwd_wgrad_w13"),
+}
+
+
+def backward_stage_flops(wl):
+    """Tensor-core flops of each GEMM stage (2*P*d*h units; P = 2T grouped rows)."""
+    u = 2 * (wl.T * wl.k) * wl.d * wl.h
+    return {1: u, 2: 2 * u, 3: 2 * u, 5: u, 6: 2 * u}
+
+
+def run_ours_backward(args):
+    import torch
+
+    import sparse_mixture_experts_26_b200 as moe
+    from workloads import WORKLOADS, make_inputs
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    init_dist("nccl")
+    wl = WORKLOADS[args.workload]
+    if wl.dtype != "bf16":
+        raise SystemExit("the backward pass is built for bf16 layers")
+    inp = make_inputs(wl, device)
+    if world > 1 and rank > 0:
+        g = torch.Generator(device=device)
+        g.manual_seed(wl.seed * 1000 + rank)
+        inp["x"] = torch.randn(inp["x"].shape, generator=g, device=device).to(inp["x"].dtype)
+    x, Wg, W1, W3, W2 = (inp[k] for k in ("x", "Wg", "W1", "W3", "W2"))
+    T, d, h, E = wl.T, wl.d, wl.h, wl.E
+    ws = moe.alloc_workspace(T, d, h, E, wl.k, x.dtype, device)
+    bws = moe.alloc_backward_workspace(T, d, h, E, wl.k, x.dtype, device)
+    y = torch.empty_like(x)
+    moe.moe_layer_forward(x, Wg, W1, W3, W2, y, ws)  # the saved state the backward reads
+    dy = backward_dy(T, d).to(device)
+    dx = torch.empty_like(x)
+    f32 = dict(dtype=torch.float32, device=device)
+    dWg, dW1 = torch.empty(Wg.shape, **f32), torch.empty(W1.shape, **f32)
+    dW3, dW2 = torch.empty(W3.shape, **f32), torch.empty(W2.shape, **f32)
+    stream = torch.cuda.current_stream(device)
+    K, W = args.steps, args.warmup
+    nst = len(BWD_STAGES) + 1
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nst)] for _ in range(K)]
+    for row in evs:
+        for e in row:
+            e.record(stream)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def step(dy_, dx_, ev=None):
+        if ev is None:
+            moe.moe_layer_backward(x, Wg, W1, W3, W2, dy_, dx_, dWg, dW1, dW3, dW2, ws, bws)
+        else:
+            moe.moe_layer_backward_events(x, Wg, W1, W3, W2, dy_, dx_, dWg, dW1, dW3, dW2, ws,
+                                          bws, [e.cuda_event for e in ev])
+
+    with ClockSampler(local) as clocks:
+        for _ in range(W):
+            step(dy, dx)
+        torch.cuda.synchronize()
+        barrier(world, device)
+        torch.cuda.synchronize()
+        start.record(stream)
+        for i in range(K):
+            step(dy, dx, evs[i])
+        end.record(stream)
+        torch.cuda.synchronize()
+        barrier(world, device)
+    ms_local = start.elapsed_time(end) / K
+    flags = moe.moe_device_status(bws)
+    if flags:
+        raise RuntimeError(f"device status flags {flags:#x} after the timed region")
+    ms = max_over_ranks(ms_local, world, device)
+    value = world * T / (ms * 1e-3)
+    st_ms = [sum(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(K)) / K
+             for j in range(nst - 1)]
+    flops = backward_stage_flops(wl)
+    dom = max(BWD_KERNELS, key=lambda j: st_ms[j])
+    kname, tag = BWD_KERNELS[dom]
+    peaks, peak_src = load_peaks()
+    ach = flops[dom] / (st_ms[dom] * 1e-3) / 1e12
+    peak = float(peaks["bf16_tflops"])
+    roofline = {"bound": "tensor", "achieved": round(ach, 1), "peak": peak, "unit": "TFLOP/s",
+                "frac": round(ach / peak, 4),
+                "traffic": ncu_traffic(tag, wl.name, os.path.join(CSRC, "backward_sm100.cu")),
+                "kernel": f"{kname} (stage '{BWD_STAGES[dom]}')",
+                "peak_source": f"{peak_src} (burst)"}
+    total_flops = sum(flops.values())
+    layer = {"ms": round(ms, 4), "tflops": round(total_flops / (ms * 1e-3) / 1e12, 1),
+             "stage_ms": {n: round(v, 4) for n, v in zip(BWD_STAGES, st_ms)},
+             "stage_tflops": {BWD_STAGES[j]: round(flops[j] / (st_ms[j] * 1e-3) / 1e12, 1)
+                              for j in flops}}
+
+    # End to end through the public API with host buffers: dy in from pinned host memory,
+    # dx back to pinned host memory, both on their own streams, double-buffered; the
+    # weight gradients stay on the device for the optimizer.
+    dy_host = dy.cpu().pin_memory()
+    dx_host = [torch.empty(dx.shape, dtype=dx.dtype).pin_memory() for _ in range(2)]
+    dy_dev = [torch.empty_like(dy) for _ in range(2)]
+    dx_dev = [torch.empty_like(dx) for _ in range(2)]
+    s_in, s_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_step = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+    for e in ev_step + ev_out:
+        e.record(stream)
+
+    def e2e_steps(n):
+        for i in range(n):
+            b = i & 1
+            with torch.cuda.stream(s_in):
+                s_in.wait_event(ev_step[b])
+                dy_dev[b].copy_(dy_host, non_blocking=True)
+                ev_in[b].record(s_in)
+            stream.wait_event(ev_in[b])
+            stream.wait_event(ev_out[b])
+            step(dy_dev[b], dx_dev[b])
+            ev_step[b].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_step[b])
+                dx_host[b].copy_(dx_dev[b], non_blocking=True)
+                ev_out[b].record(s_out)
+
+    e2e_steps(2)
+    torch.cuda.synchronize()
+    barrier(world, device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s_in)
+    e2e_steps(K)
+    s_out.wait_stream(stream)
+    e1.record(s_out)
+    torch.cuda.synchronize()
+    barrier(world, device)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / K, world, device)
+    e2e = {"value": round(world * T / (e2e_ms * 1e-3), 1), "unit": UNIT,
+           "h2d_bytes_per_step": dy.numel() * dy.element_size(),
+           "d2h_bytes_per_step": dx.numel() * dx.element_size(),
+           "pipeline": "double-buffered: dy in and dx out on their own streams; weight "
+                       "gradients stay on the device"}
+
+    cpu_baseline = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        n = min(T, args.cpu_sample_tokens_bwd)
+        tps, threads, reps, dt = oracle_tokens_per_s(cpu_copy(inp), n, args.cpu_budget_s,
+                                                     backward=True)
+        cpu_baseline = {"value": round(tps, 3), "unit": UNIT, "cores": threads,
+                        "kind": "oracle",
+                        "sample": f"fp64 numpy oracle backward (with its forward) on the "
+                                  f"first {n} tokens of the batch, {reps} repeat(s) in "
+                                  f"{dt:.1f} s"}
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    if rank != 0:
+        return None
+    return {
+        "metric": BWD_METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+        "steps": K, "warmup": W, "ms_per_step": round(ms, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype,
+        "data": "synthetic (seeded normal draws of the Mixtral-8x7B layer shapes and of dy; "
+                "random-init weights)",
+        "config": workload_config(wl, {"pass": "backward (after one forward that fills the "
+                                               "saved state)",
+                                       "parallelism": f"replicas x{world}"}),
+        "roofline": roofline, "layer": layer, "cpu_baseline": cpu_baseline, "e2e": e2e,
+        "gpu_launches": 9 * K, "clocks": clocks.summary(),
+    }
+
+
 # ------------------------------------------------------------------ reference arm
 def run_reference(args):
     """The CPU oracle as it stands, on host cores, on a bounded sample per step."""
@@ -438,12 +633,23 @@ def run_reference(args):
     inp_cpu = cpu_copy(make_inputs(wl, dev))
     n = min(wl.T, args.cpu_sample_tokens)
     from oracle import moe_oracle as O
+    if args.backward:
+        n = min(wl.T, args.cpu_sample_tokens_bwd)
     x = inp_cpu["x"][:n]
+    dy = backward_dy_cpu(x.shape)
+
+    def one():
+        if args.backward:
+            O.moe_layer_backward(x, inp_cpu["Wg"], inp_cpu["W1"], inp_cpu["W3"], inp_cpu["W2"],
+                                 dy)
+        else:
+            O.moe_layer(x, inp_cpu["Wg"], inp_cpu["W1"], inp_cpu["W3"], inp_cpu["W2"])
+
     for _ in range(args.warmup):
-        O.moe_layer(x, inp_cpu["Wg"], inp_cpu["W1"], inp_cpu["W3"], inp_cpu["W2"])
+        one()
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        O.moe_layer(x, inp_cpu["Wg"], inp_cpu["W1"], inp_cpu["W3"], inp_cpu["W2"])
+        one()
     dt = time.perf_counter() - t0
     ms = dt / args.steps * 1e3
     value = n / (ms * 1e-3)
@@ -453,13 +659,14 @@ def run_reference(args):
                        if p.get("user_api") == "blas"), default=1)
     except Exception:
         threads = os.cpu_count() or 1
-    sample = f"fp64 numpy oracle on the first {n} of the batch's {wl.T} tokens per step"
+    sample = (f"fp64 numpy oracle {'backward (with its forward) ' if args.backward else ''}"
+              f"on the first {n} of the batch's {wl.T} tokens per step")
     return {
-        "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": UNIT,
+        "impl": "reference", "metric": BWD_METRIC if args.backward else METRIC, "value": round(value, 3), "unit": UNIT,
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": workload_config(wl),
+        "config": workload_config(wl, {"pass": "backward"} if args.backward else None),
         "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": int(threads),
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0,
@@ -478,6 +685,9 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-tokens", type=int, default=16)
     ap.add_argument("--cpu-budget-s", type=float, default=10.0)
+    ap.add_argument("--backward", action="store_true",
+                    help="time the layer's backward pass instead of its forward")
+    ap.add_argument("--cpu-sample-tokens-bwd", type=int, default=4)
     args = ap.parse_args(argv)
     ref = args.impl == "reference"
     if args.steps is None:
@@ -486,7 +696,10 @@ def main(argv=None):
         args.warmup = 1 if ref else 10
     if not ref and args.warmup < 3:
         args.warmup = 3
-    out = run_reference(args) if ref else run_ours(args)
+    if ref:
+        out = run_reference(args)
+    else:
+        out = run_ours_backward(args) if args.backward else run_ours(args)
     if out is not None:
         print(json.dumps(out), flush=True)
 

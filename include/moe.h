@@ -226,6 +226,18 @@ moe_status moe_layer_backward(const void *x, const void *Wg, const void *W1, con
                               float *dW3, float *dW2, const void *fwd_ws, size_t fwd_ws_bytes,
                               void *bwd_ws, size_t bwd_ws_bytes, cudaStream_t stream);
 
+/* moe_layer_backward with caller-created events recorded on `stream` before its first
+ * launch and after each stage: [0] start, [1] dY/dw/logit gradients, [2] dH, [3] du/dv,
+ * [4] dX, [5] dx, [6] dW2, [7] dW1/dW3, [8] dWg.  Null handles (or n_events <= i) are
+ * skipped.  For timing the stages (bench.py). */
+moe_status moe_layer_backward_events(const void *x, const void *Wg, const void *W1,
+                                     const void *W3, const void *W2, const void *dy, int T, int d,
+                                     int h, int E, int k, moe_dtype dt, int capacity, void *dx,
+                                     float *dWg, float *dW1, float *dW3, float *dW2,
+                                     const void *fwd_ws, size_t fwd_ws_bytes, void *bwd_ws,
+                                     size_t bwd_ws_bytes, cudaEvent_t *events, int n_events,
+                                     cudaStream_t stream);
+
 /* Static description of a status code. */
 const char *moe_status_string(moe_status st);
 

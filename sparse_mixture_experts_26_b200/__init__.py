@@ -25,6 +25,7 @@ __all__ = [
     "EXPORTED_SYMBOLS", "launches_per_layer", "moe_expert_ffn_static",
     "moe_layer_forward_capacity", "moe_selftest_wait_timeout", "moe_backward_workspace_bytes",
     "moe_layer_backward", "alloc_backward_workspace", "layer_backward",
+    "moe_layer_backward_events",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe.so")
@@ -36,7 +37,8 @@ EXPORTED_SYMBOLS = ("moe_workspace_bytes", "moe_route", "moe_permute", "moe_expe
                     "moe_combine", "moe_layer_forward", "moe_layer_forward_events",
                     "moe_device_status", "moe_status_string", "moe_expert_ffn_static",
                     "moe_layer_forward_capacity", "moe_selftest_wait_timeout",
-                    "moe_backward_workspace_bytes", "moe_layer_backward")
+                    "moe_backward_workspace_bytes", "moe_layer_backward",
+                    "moe_layer_backward_events")
 def launches_per_layer(T: int) -> int:
     """Kernels one moe_layer_forward queues: router 1, permutation 1 (T <= 512) or 4
     (count, scan, rank, gather), expert FFN 1 (T <= 64: gate/up and down fused) or 2,
@@ -76,6 +78,9 @@ def _load() -> ctypes.CDLL:
         "moe_backward_workspace_bytes": (sz, [i32, i32, i32, i32, i32, i32]),
         "moe_layer_backward": (i32, [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32,
                                      vp, vp, vp, vp, vp, vp, sz, vp, sz, vp]),
+        "moe_layer_backward_events": (i32, [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
+                                            i32, vp, vp, vp, vp, vp, vp, sz, vp, sz, vp, i32,
+                                            vp]),
     }
     for name, (res, args) in sigs.items():
         f = getattr(lib, name)
@@ -276,6 +281,22 @@ def moe_layer_backward(x, Wg, W1, W3, W2, dy, dx, dWg, dW1, dW3, dW2, fwd_ws, bw
         int(capacity), _ptr(dx), _ptr(dWg), _ptr(dW1), _ptr(dW3), _ptr(dW2), _ptr(fwd_ws),
         fwd_ws.numel() * fwd_ws.element_size(), _ptr(bwd_ws),
         bwd_ws.numel() * bwd_ws.element_size(), _stream(stream)))
+
+
+def moe_layer_backward_events(x, Wg, W1, W3, W2, dy, dx, dWg, dW1, dW3, dW2, fwd_ws, bwd_ws,
+                              events, capacity: int = -1, k: int = 2, stream=None) -> None:
+    """``moe_layer_backward`` recording ``events`` (up to 9 created handles, or None to
+    skip one) before its first launch and after each stage."""
+    _dev(x, Wg, W1, W3, W2, dy, dx, dWg, dW1, dW3, dW2, fwd_ws, bwd_ws)
+    T, d = x.shape
+    E, h, _ = W1.shape
+    handles = (ctypes.c_void_p * max(1, len(events)))(*[int(e) if e else None for e in events])
+    _check("moe_layer_backward_events", _lib.moe_layer_backward_events(
+        _ptr(x), _ptr(Wg), _ptr(W1), _ptr(W3), _ptr(W2), _ptr(dy), T, d, h, E, k, _dt(x),
+        int(capacity), _ptr(dx), _ptr(dWg), _ptr(dW1), _ptr(dW3), _ptr(dW2), _ptr(fwd_ws),
+        fwd_ws.numel() * fwd_ws.element_size(), _ptr(bwd_ws),
+        bwd_ws.numel() * bwd_ws.element_size(), ctypes.addressof(handles), len(events),
+        _stream(stream)))
 
 
 def layer_backward(x, Wg, W1, W3, W2, dy, fwd_ws, capacity: int = -1, bwd_ws=None):

@@ -41,6 +41,8 @@ namespace moe {
 // Defined in grouped_gemm_sm100.cu.
 bool encode_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
                     uint32_t box_rows);
+bool encode_f32_3d(CUtensorMap* map, const void* base, uint64_t batches, uint64_t rows,
+                   uint64_t cols, uint32_t box_cols, uint32_t box_rows);
 
 namespace {
 
@@ -55,8 +57,15 @@ constexpr int kThreads = 192;
 constexpr int kEpiThreads = 128;
 constexpr uint32_t kTmemCols = 2 * kN;
 constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 1024 /*bookkeeping*/;
+// Weight-gradient epilogue: each epilogue warp stages 32-row x 32-column fp32 chunks
+// (4 KiB) of its own accumulator rows for TMA stores, OUTBUFS buffers per warp.
+constexpr int kStageOutBytes = 32 * 32 * 4;  // 4 KiB
+template <int STAGES, int OUTBUFS>
+constexpr int wgrad_smem_bytes() {
+    return STAGES * kStageBytes + 4 * OUTBUFS * kStageOutBytes + 1024 /*align*/ + 1024 /*book*/;
+}
+constexpr int kVoteBarrier = 2;  // epilogue vote after a bounded wait
 constexpr int kBox = 64 * 128;             // one 64-column x 64-row box: 8 KiB
-constexpr int kVoteBarrier = 2;
 
 enum RowMode { kModeDH = 0, kModeDUV = 1, kModeDX = 2 };
 enum WMode { kModeW2 = 0, kModeW13 = 1 };
@@ -131,8 +140,8 @@ __device__ __forceinline__ void load_groups(Book& bk, const int32_t* offsets, in
     }
 }
 
-__device__ __forceinline__ void init_barriers(Book& bk) {
-    for (int s = 0; s < kStages; ++s) {
+__device__ __forceinline__ void init_barriers(Book& bk, int stages = kStages) {
+    for (int s = 0; s < stages; ++s) {
         mbar_init(&bk.full[s], 1);
         mbar_init(&bk.empty[s], 1);
     }
@@ -413,6 +422,19 @@ __global__ void __launch_bounds__(kThreads, 1)
 // are grouped activations, row-major with m / n contiguous (MN-major).  Tiles are
 // (expert, 256-column block, 128-row block), row blocks inner so that consecutive
 // tiles share B.  An expert with no rows gets a zero tile.
+// The output is written by TMA, each epilogue warp on its own: a 32-column chunk of
+// the warp's 32 accumulator rows goes to one of its staging buffers in the
+// 128-byte-swizzled layout (row r at r * 128 bytes, 16-byte chunk j at position
+// j ^ (r % 8), so the warp's stores hit distinct banks), and lane 0 stores it with a
+// 3-D tensor store ([E, rows, cols]: rows past an expert's last are outside the
+// tensor and not written).  A buffer is reused once its previous store has read it;
+// no block-wide barrier is involved.  A tile that straddles the dW1 / dW3 boundary
+// (h not a multiple of 128) is stored row by row instead.
+// STAGES input stages and the staging buffers share the shared memory: a short
+// reduction (few rows per expert) leaves the kernel bound by its output stores (more
+// buffers); a long one wants deeper input stages.
+// Tiles run column blocks innermost, so the CTAs running at one time write
+// neighbouring parts of the same output rows.
 //   kModeW2 : A = dY [rows, d], B = H [rows, h]         -> dW2 [E, d, h]
 //   kModeW13: A = [du dv] [rows, 2h], B = x [rows, d]   -> dW1 [E, h, d] (m < h),
 //                                                          dW3 [E, h, d] (m >= h)
@@ -431,25 +453,31 @@ struct WArgs {
     int cap;
 };
 
-template <int MODE>
+template <int MODE, int STAGES, int OUTBUFS>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_wgrad_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                     const WArgs args) {
+                     const __grid_constant__ CUtensorMap tmO0,
+                     const __grid_constant__ CUtensorMap tmO1, const WArgs args) {
     constexpr uint32_t kIdesc = idesc_major(kBM, kN, true, true);
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     uint8_t* sA = smem;
-    uint8_t* sB = smem + kStages * kABytes;
-    Book& bk = *reinterpret_cast<Book*>(smem + kStages * kStageBytes);
+    static_assert(STAGES >= 2 && STAGES <= kStages && OUTBUFS >= 2, "pipeline shape");
+    static_assert(wgrad_smem_bytes<STAGES, OUTBUFS>() <= 232448, "shared memory");
+    uint8_t* sB = smem + STAGES * kABytes;
+    uint8_t* sOut = smem + STAGES * kStageBytes;  // staging buffers, 1 KiB aligned
+    Book& bk = *reinterpret_cast<Book*>(sOut + 4 * OUTBUFS * kStageOutBytes);
     volatile int* abort_flag = &bk.abort_flag;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int E = args.E;
 
-    if (threadIdx.x == 0) init_barriers(bk);
+    if (threadIdx.x == 0) init_barriers(bk, STAGES);
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
+        tma_prefetch_desc(&tmO0);
+        tma_prefetch_desc(&tmO1);
     }
     if (warp == 1) tmem_alloc(&bk.tmem_base, kTmemCols);
     if (threadIdx.x == 0) load_groups(bk, args.offsets, E, args.rows, args.cap);
@@ -463,8 +491,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto tile_of = [&](int tile, int& e, int& mt, int& nt, int& r0, int& n_rows) {
         e = tile / per_e;
         const int local = tile - e * per_e;
-        mt = local % args.m_tiles;
-        nt = local / args.m_tiles;
+        nt = local % args.n_tiles;
+        mt = local / args.n_tiles;
         r0 = bk.off[e];
         n_rows = bk.end[e] - bk.off[e];
     };
@@ -496,14 +524,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tma_load_2d(&tmB, &bk.full[stage], b + i * kBox, nt * kN + 64 * i, r);
                     pending |= 1u << stage;
                     pending_phase = (pending_phase & ~(1u << stage)) | (phase << stage);
-                    if (++stage == kStages) {
+                    if (++stage == STAGES) {
                         stage = 0;
                         phase ^= 1u;
                     }
                 }
             }
             if (!ok)
-                for (int s = 0; s < kStages; ++s)
+                for (int s = 0; s < STAGES; ++s)
                     if (pending & (1u << s)) drain_wait(&bk.full[s], (pending_phase >> s) & 1u);
         }
         __syncwarp();
@@ -532,13 +560,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!ok) break;
                 const int kv = n_rows - kb * kBK;  // rows of this block inside the group
                 if (kv < kBK) {
-                    // Rows kv..63 belong to the next group (or were dropped by the
-                    // capacity and never written): clear them in every A and B box.
+                    // Rows kv..63 belong to the next group: clear them in A (its rows
+                    // there may never have been written, e.g. dropped pairs' dY); with a
+                    // capacity, B's dropped rows may hold garbage too, so clear B as well.
                     uint8_t* a = sA + stage * kABytes;
                     uint8_t* b = sB + stage * kBBytes;
                     const int nz = (kBK - kv) * 8;  // 16-byte chunks per box to clear
-                    constexpr int kBoxes = (kBM + kN) / 64;
-                    for (int i = lane; i < kBoxes * nz; i += 32) {
+                    const int boxes = (args.cap != INT_MAX ? kBM + kN : kBM) / 64;
+                    for (int i = lane; i < boxes * nz; i += 32) {
                         const int box = i / nz, c = i - box * nz;
                         uint8_t* base = box < kBM / 64 ? a + box * kBox : b + (box - kBM / 64) * kBox;
                         *reinterpret_cast<uint4*>(base + kv * 128 + c * 16) =
@@ -559,7 +588,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 issued = true;
                 __syncwarp();
-                if (++stage == kStages) {
+                if (++stage == STAGES) {
                     stage = 0;
                     phase ^= 1u;
                 }
@@ -577,12 +606,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
     } else {
         const int q = warp & 3;
-        int acc = 0;
+        const int r = q * 32 + lane;          // accumulator row of this thread
+        uint8_t* wstage = sOut + q * OUTBUFS * kStageOutBytes;  // this warp's buffers
+        int acc = 0, buf = 0;
         uint32_t acc_phase = 0;
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
             int e, mt, nt, r0, n_rows;
             tile_of(tile, e, mt, nt, r0, n_rows);
-            const int m = mt * kBM + q * 32 + lane;
+            const int m0 = mt * kBM;
+            const int m = m0 + r;
             const bool mvalid = m < args.M;
             float* out = m < args.split
                              ? args.out0 + (static_cast<size_t>(e) * args.split + m) * args.N
@@ -595,16 +627,37 @@ __global__ void __launch_bounds__(kThreads, 1)
                         *reinterpret_cast<float4*>(out + col) = make_float4(0.f, 0.f, 0.f, 0.f);
                 continue;
             }
-            if (!mbar_wait_bounded(&bk.tmem_full[acc], acc_phase, abort_flag, args.status)) break;
+            if (!bar_all(mbar_wait_bounded(&bk.tmem_full[acc], acc_phase, abort_flag,
+                                           args.status),
+                         kVoteBarrier, kEpiThreads))
+                break;
             tc_fence_after();
             const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                                    static_cast<uint32_t>(acc * kN);
+            const bool second = m0 >= args.split;
+            const bool straddle = m0 < args.split && m0 + kBM > args.split;
 #pragma unroll 1
             for (int ch = 0; ch < 8; ++ch) {
                 uint32_t v[32];
                 tmem_ld_32cols(tbase + ch * 32, v);
                 tmem_ld_wait();
-                if (mvalid) {
+                if (!straddle) {
+                    uint8_t* st = wstage + buf * kStageOutBytes;
+                    if (lane == 0) bulk_wait_group_read<OUTBUFS - 1>();  // buffer free again
+                    __syncwarp();
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        *reinterpret_cast<uint4*>(st + lane * 128 + ((j ^ (lane & 7)) << 4)) =
+                            make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_3d(second ? &tmO1 : &tmO0, st, col0 + ch * 32,
+                                     (second ? m0 - args.split : m0) + q * 32, e);
+                        bulk_commit_group();
+                    }
+                    if (++buf == OUTBUFS) buf = 0;
+                } else if (mvalid) {
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
                         const int col = col0 + ch * 32 + j * 4;
@@ -620,6 +673,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             acc ^= 1;
             if (acc == 0) acc_phase ^= 1u;
         }
+        if (lane == 0) bulk_wait_group<0>();  // every store complete before the block exits
     }
 
     tc_fence_before();
@@ -705,33 +759,68 @@ __global__ void __launch_bounds__(kPrepThreads)
     }
 }
 
-// dx[t, c] = dX[r0, c] + dX[r1, c] (kept pairs) + sum_e dlogits[t, e] Wg[c, e], one rounding.
+// dx[t, c] = dX[r0, c] + dX[r1, c] (kept pairs) + sum_e dlogits[t, e] Wg[c, e], one
+// rounding.  Four columns per thread (d % 8 == 0), 16-byte loads of dX.
 __global__ void __launch_bounds__(kPrepThreads)
     bwd_dx_kernel(const float* __restrict__ dX, const int32_t* __restrict__ idx,
                   const int32_t* __restrict__ inv, const int32_t* __restrict__ offsets, int T,
                   int d, int E, int cap, const float* __restrict__ dlogits,
                   const __nv_bfloat16* __restrict__ Wg, __nv_bfloat16* __restrict__ dx) {
     const int P = 2 * T;
-    const size_t n = static_cast<size_t>(T) * d;
+    const int d4 = d / 4;
+    const size_t n = static_cast<size_t>(T) * d4;
     for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
          i += static_cast<size_t>(gridDim.x) * blockDim.x) {
-        const int t = static_cast<int>(i / d);
-        const int c = static_cast<int>(i - static_cast<size_t>(t) * d);
-        float v = 0.f;
-        if (pair_kept(idx, offsets, inv, 2 * t, E, P, cap))
-            v += dX[static_cast<size_t>(inv[2 * t]) * d + c];
-        if (pair_kept(idx, offsets, inv, 2 * t + 1, E, P, cap))
-            v += dX[static_cast<size_t>(inv[2 * t + 1]) * d + c];
+        const int t = static_cast<int>(i / d4);
+        const int c = static_cast<int>(i - static_cast<size_t>(t) * d4) * 4;
+        float v[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            if (pair_kept(idx, offsets, inv, 2 * t + j, E, P, cap)) {
+                const float4 a = *reinterpret_cast<const float4*>(
+                    dX + static_cast<size_t>(inv[2 * t + j]) * d + c);
+                v[0] += a.x;
+                v[1] += a.y;
+                v[2] += a.z;
+                v[3] += a.w;
+            }
+        }
         const float* dl = dlogits + static_cast<size_t>(t) * E;
-        const __nv_bfloat16* wr = Wg + static_cast<size_t>(c) * E;
-        for (int e = 0; e < E; ++e) v = fmaf(dl[e], __bfloat162float(wr[e]), v);
-        dx[i] = __float2bfloat16_rn(v);
+        if (E == 8) {
+            // W_g rows of the four columns: one 16-byte load each
+            float g[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) g[e] = dl[e];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const uint4 q = *reinterpret_cast<const uint4*>(Wg + static_cast<size_t>(c + u) * 8);
+                const uint32_t w4[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+                for (int p2 = 0; p2 < 4; ++p2) {
+                    v[u] = fmaf(g[2 * p2], __uint_as_float(w4[p2] << 16), v[u]);
+                    v[u] = fmaf(g[2 * p2 + 1], __uint_as_float(w4[p2] & 0xffff0000u), v[u]);
+                }
+            }
+        } else {
+            for (int e = 0; e < E; ++e) {
+                const float g = dl[e];
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                    v[u] = fmaf(g, __bfloat162float(Wg[static_cast<size_t>(c + u) * E + e]), v[u]);
+            }
+        }
+        __nv_bfloat162 lo = __floats2bfloat162_rn(v[0], v[1]);
+        __nv_bfloat162 hi = __floats2bfloat162_rn(v[2], v[3]);
+        uint2 o;
+        o.x = *reinterpret_cast<uint32_t*>(&lo);
+        o.y = *reinterpret_cast<uint32_t*>(&hi);
+        *reinterpret_cast<uint2*>(dx + static_cast<size_t>(t) * d + c) = o;
     }
 }
 
 // dWg = x^T dlogits in two deterministic passes: per chunk of kWgChunk tokens a
 // partial [d, E], then the partials summed in chunk order.
-constexpr int kWgChunk = 256;
+constexpr int kWgChunk = 64;
 
 __global__ void __launch_bounds__(kPrepThreads)
     bwd_dwg_partial_kernel(const __nv_bfloat16* __restrict__ x, const float* __restrict__ dlogits,
@@ -774,16 +863,37 @@ __global__ void __launch_bounds__(kPrepThreads)
 
 // Opt each GEMM kernel into its dynamic shared memory once per device.  `slot` names
 // the kernel: the instantiations share one function type, so it cannot be the key.
-enum KernelSlot { kSlotDH, kSlotDUV, kSlotDX, kSlotW2, kSlotW13, kSlots };
+enum KernelSlot { kSlotDH, kSlotDUV, kSlotDX, kSlotW2, kSlotW13, kSlotW2s, kSlotW13s, kSlots };
 template <typename Kern>
-void configure(Kern kern, KernelSlot slot) {
+void configure(Kern kern, KernelSlot slot, int smem_bytes) {
     static int configured[kSlots][64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev >= 0 && dev < 64 && !configured[slot][dev]) {
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
         configured[slot][dev] = 1;
     }
+}
+
+// Grouped rows at or below which the weight-gradient GEMMs use the store-bound shape.
+constexpr int kWgradShortRows = 1024;
+constexpr int kWgradLong[2] = {4, 2};   // input stages, staging buffers per epilogue warp
+constexpr int kWgradShort[2] = {2, 8};
+
+template <int MODE>
+cudaError_t launch_wgrad(bool short_k, int grid, cudaStream_t s, const CUtensorMap& A,
+                         const CUtensorMap& B, const CUtensorMap& O0, const CUtensorMap& O1,
+                         const WArgs& w) {
+    if (short_k) {
+        constexpr int st = kWgradShort[0], ob = kWgradShort[1];
+        auto kern = bwd_wgrad_kernel<MODE, st, ob>;
+        configure(kern, MODE == kModeW2 ? kSlotW2s : kSlotW13s, wgrad_smem_bytes<st, ob>());
+        return launch_k(kern, grid, kThreads, wgrad_smem_bytes<st, ob>(), s, A, B, O0, O1, w);
+    }
+    constexpr int st = kWgradLong[0], ob = kWgradLong[1];
+    auto kern = bwd_wgrad_kernel<MODE, st, ob>;
+    configure(kern, MODE == kModeW2 ? kSlotW2 : kSlotW13, wgrad_smem_bytes<st, ob>());
+    return launch_k(kern, grid, kThreads, wgrad_smem_bytes<st, ob>(), s, A, B, O0, O1, w);
 }
 
 int grid_for(long long work, int cap) {
@@ -798,12 +908,16 @@ cudaError_t launch_layer_backward(const BwdArgs& a, cudaStream_t s) {
     const int T = a.T, d = a.d, h = a.h, E = a.E, P = 2 * T;
     const int sms = device_sm_count();
     cudaError_t err;
+    auto mark = [&](int i) -> cudaError_t {  // optional events between the launches
+        return (i < a.n_ev && a.ev[i]) ? cudaEventRecord(a.ev[i], s) : cudaSuccess;
+    };
+    if ((err = mark(0)) != cudaSuccess) return err;
     // 1. dY, dw, dlogits
     err = launch_k(bwd_prep_kernel, grid_for(T, 8 * sms), kPrepThreads, 0, s,
                    static_cast<const __nv_bfloat16*>(a.dy), a.idx, a.w, a.inv, a.offsets, T, d, E,
                    a.cap, a.Y, a.nsplit, a.split_stride, static_cast<__nv_bfloat16*>(a.dY), a.dw,
                    a.dlogits);
-    if (err != cudaSuccess) return err;
+    if (err != cudaSuccess || (err = mark(1)) != cudaSuccess) return err;
 
     CUtensorMap m_dY128, m_W2, m_x, m_W1r, m_W3r, m_duv128, m_W1mn, m_W3mn;
     if (!encode_bf16_2d(&m_dY128, a.dY, P, d, kBM) ||
@@ -820,60 +934,62 @@ cudaError_t launch_layer_backward(const BwdArgs& a, cudaStream_t s) {
     // 2. dH = dY W2_e
     {
         RowArgs r{a.offsets, E, P, d, h, (h + kN - 1) / kN, h, d, a.dH, nullptr, a.status, a.cap};
-        configure(bwd_rows_kernel<kModeDH>, kSlotDH);
+        configure(bwd_rows_kernel<kModeDH>, kSlotDH, kSmemBytes);
         err = launch_k(bwd_rows_kernel<kModeDH>, grid_for(row_blocks * r.n_tiles, sms), kThreads,
                        kSmemBytes, s, m_dY128, m_W2, m_W2, r);
-        if (err != cudaSuccess) return err;
+        if (err != cudaSuccess || (err = mark(2)) != cudaSuccess) return err;
     }
     // 3. du, dv (recomputes a and b)
     {
         RowArgs r{a.offsets, E, P, d, h, (h + 127) / 128, h, d, a.DUV, a.dH, a.status, a.cap};
-        configure(bwd_rows_kernel<kModeDUV>, kSlotDUV);
+        configure(bwd_rows_kernel<kModeDUV>, kSlotDUV, kSmemBytes);
         err = launch_k(bwd_rows_kernel<kModeDUV>, grid_for(row_blocks * r.n_tiles, sms),
                        kThreads, kSmemBytes, s, m_x, m_W1r, m_W3r, r);
-        if (err != cudaSuccess) return err;
+        if (err != cudaSuccess || (err = mark(3)) != cudaSuccess) return err;
     }
     // 4. dX = [du dv] [W1_e ; W3_e]
     {
         RowArgs r{a.offsets, E, P, 2 * h, d, (d + kN - 1) / kN, h, d, a.dX, nullptr, a.status,
                   a.cap};
-        configure(bwd_rows_kernel<kModeDX>, kSlotDX);
+        configure(bwd_rows_kernel<kModeDX>, kSlotDX, kSmemBytes);
         err = launch_k(bwd_rows_kernel<kModeDX>, grid_for(row_blocks * r.n_tiles, sms), kThreads,
                        kSmemBytes, s, m_duv128, m_W1mn, m_W3mn, r);
-        if (err != cudaSuccess) return err;
+        if (err != cudaSuccess || (err = mark(4)) != cudaSuccess) return err;
     }
     // 5. dx
     {
-        const long long n = static_cast<long long>(T) * d;
+        const long long n = static_cast<long long>(T) * (d / 4);
         err = launch_k(bwd_dx_kernel, grid_for((n + kPrepThreads - 1) / kPrepThreads, 8 * sms),
                        kPrepThreads, 0, s, static_cast<const float*>(a.dX), a.idx, a.inv,
                        a.offsets, T, d, E, a.cap, static_cast<const float*>(a.dlogits),
                        static_cast<const __nv_bfloat16*>(a.Wg), static_cast<__nv_bfloat16*>(a.dx));
-        if (err != cudaSuccess) return err;
+        if (err != cudaSuccess || (err = mark(5)) != cudaSuccess) return err;
     }
     // 6. weight gradients
-    CUtensorMap m_dY64, m_H64, m_duv64, m_x64;
+    CUtensorMap m_dY64, m_H64, m_duv64, m_x64, m_dW2, m_dW1, m_dW3;
     if (!encode_bf16_2d(&m_dY64, a.dY, P, d, 64) || !encode_bf16_2d(&m_H64, a.H, P, h, 64) ||
         !encode_bf16_2d(&m_duv64, a.DUV, P, 2 * h, 64) ||
-        !encode_bf16_2d(&m_x64, a.x_perm, P, d, 64))
+        !encode_bf16_2d(&m_x64, a.x_perm, P, d, 64) ||
+        !encode_f32_3d(&m_dW2, a.dW2, E, d, h, 32, 32) ||
+        !encode_f32_3d(&m_dW1, a.dW1, E, h, d, 32, 32) ||
+        !encode_f32_3d(&m_dW3, a.dW3, E, h, d, 32, 32))
         return cudaErrorInvalidValue;
+    // Few rows per expert: the output stores bound the kernel (deep staging); many:
+    // the reduction does (deep input pipeline).
+    const bool short_k = P <= kWgradShortRows;
     {
         WArgs w{a.offsets, E, P, d, h, (d + kBM - 1) / kBM, (h + kN - 1) / kN, d, a.dW2, a.dW2,
                 a.status, a.cap};
-        configure(bwd_wgrad_kernel<kModeW2>, kSlotW2);
-        err = launch_k(bwd_wgrad_kernel<kModeW2>,
-                       grid_for(static_cast<long long>(E) * w.m_tiles * w.n_tiles, sms), kThreads,
-                       kSmemBytes, s, m_dY64, m_H64, w);
-        if (err != cudaSuccess) return err;
+        err = launch_wgrad<kModeW2>(short_k, grid_for(static_cast<long long>(E) * w.m_tiles * w.n_tiles, sms),
+                                    s, m_dY64, m_H64, m_dW2, m_dW2, w);
+        if (err != cudaSuccess || (err = mark(6)) != cudaSuccess) return err;
     }
     {
         WArgs w{a.offsets, E, P, 2 * h, d, (2 * h + kBM - 1) / kBM, (d + kN - 1) / kN, h, a.dW1,
                 a.dW3, a.status, a.cap};
-        configure(bwd_wgrad_kernel<kModeW13>, kSlotW13);
-        err = launch_k(bwd_wgrad_kernel<kModeW13>,
-                       grid_for(static_cast<long long>(E) * w.m_tiles * w.n_tiles, sms), kThreads,
-                       kSmemBytes, s, m_duv64, m_x64, w);
-        if (err != cudaSuccess) return err;
+        err = launch_wgrad<kModeW13>(short_k, grid_for(static_cast<long long>(E) * w.m_tiles * w.n_tiles, sms),
+                                     s, m_duv64, m_x64, m_dW1, m_dW3, w);
+        if (err != cudaSuccess || (err = mark(7)) != cudaSuccess) return err;
     }
     // 7. dWg
     {
@@ -886,8 +1002,9 @@ cudaError_t launch_layer_backward(const BwdArgs& a, cudaStream_t s) {
         err = launch_k(bwd_dwg_reduce_kernel, grid_for((n + kPrepThreads - 1) / kPrepThreads, 4 * sms),
                        kPrepThreads, 0, s, static_cast<const float*>(a.dwg_part), nchunk, d, E,
                        a.dWg);
+        if (err != cudaSuccess) return err;
     }
-    return err;
+    return mark(8);
 }
 
 }  // namespace moe

@@ -386,6 +386,22 @@ static EncodeTiledFn get_encode_fn() {
     return fn;
 }
 
+// fp32 tensor [batches, rows, cols] (row-major, contiguous) viewed as 3-D; box =
+// box_cols x box_rows x 1 with 128-byte swizzle (box_cols * 4 must be 128 at most).
+bool encode_f32_3d(CUtensorMap* map, const void* base, uint64_t batches, uint64_t rows,
+                   uint64_t cols, uint32_t box_cols, uint32_t box_rows) {
+    EncodeTiledFn enc = get_encode_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[3] = {cols, rows, batches};
+    const cuuint64_t strides[2] = {cols * 4, rows * cols * 4};
+    const cuuint32_t box[3] = {box_cols, box_rows, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides,
+               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+           CUDA_SUCCESS;
+}
+
 // Row-major bf16 matrix [rows, cols] viewed as a 2-D tensor; box = 64 columns (one
 // 128-byte swizzle span) x box_rows rows, 128-byte swizzle, zero fill out of bounds.
 bool encode_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,

@@ -321,13 +321,20 @@ size_t moe_backward_workspace_bytes(int T, int d, int h, int E, int k, moe_dtype
     return bwd_layout(T, d, h, E).total;
 }
 
-moe_status moe_layer_backward(const void* x, const void* Wg, const void* W1, const void* W3,
-                              const void* W2, const void* dy, int T, int d, int h, int E, int k,
-                              moe_dtype dt, int capacity, void* dx, float* dWg, float* dW1,
-                              float* dW3, float* dW2, const void* fwd_ws, size_t fwd_ws_bytes,
-                              void* bwd_ws, size_t bwd_ws_bytes, cudaStream_t stream) {
+}  // extern "C"
+
+namespace moe {
+namespace {
+
+moe_status layer_backward_impl(const void* x, const void* Wg, const void* W1, const void* W3,
+                               const void* W2, const void* dy, int T, int d, int h, int E, int k,
+                               moe_dtype dt, int capacity, void* dx, float* dWg, float* dW1,
+                               float* dW3, float* dW2, const void* fwd_ws, size_t fwd_ws_bytes,
+                               void* bwd_ws, size_t bwd_ws_bytes, cudaEvent_t* ev, int n_ev,
+                               cudaStream_t stream) {
     moe_status st = check_shape(T, d, h, E, k, dt, true);
     if (st != MOE_OK) return st;
+    if (n_ev < 0 || (n_ev > 0 && ev == nullptr)) return MOE_ERR_INVALID_ARG;
     if (dt != MOE_BF16 || h % 64 != 0) return MOE_ERR_UNSUPPORTED;
     if (T == 0) return MOE_OK;
     if (!ptrs_ok({x, Wg, W1, W3, W2, dy, dx, dWg, dW1, dW3, dW2, fwd_ws, bwd_ws}))
@@ -373,10 +380,39 @@ moe_status moe_layer_backward(const void* x, const void* Wg, const void* W1, con
     a.dX = at<float>(bwd_ws, B.dX);
     a.dwg_part = at<float>(bwd_ws, B.dwg_part);
     a.status = at<uint32_t>(bwd_ws, B.status);
+    a.ev = ev;
+    a.n_ev = n_ev;
     PdlScope pdl(false);  // the backward kernels do not wait on griddepcontrol
     cudaError_t err = launch_layer_backward(a, stream);
     if (err == cudaErrorInvalidValue) return MOE_ERR_INVALID_ARG;  // tensor map refused
     return finish(err, stream, a.status);
+}
+
+}  // namespace
+}  // namespace moe
+
+extern "C" {
+
+moe_status moe_layer_backward(const void* x, const void* Wg, const void* W1, const void* W3,
+                              const void* W2, const void* dy, int T, int d, int h, int E, int k,
+                              moe_dtype dt, int capacity, void* dx, float* dWg, float* dW1,
+                              float* dW3, float* dW2, const void* fwd_ws, size_t fwd_ws_bytes,
+                              void* bwd_ws, size_t bwd_ws_bytes, cudaStream_t stream) {
+    return layer_backward_impl(x, Wg, W1, W3, W2, dy, T, d, h, E, k, dt, capacity, dx, dWg, dW1,
+                               dW3, dW2, fwd_ws, fwd_ws_bytes, bwd_ws, bwd_ws_bytes, nullptr, 0,
+                               stream);
+}
+
+moe_status moe_layer_backward_events(const void* x, const void* Wg, const void* W1,
+                                     const void* W3, const void* W2, const void* dy, int T, int d,
+                                     int h, int E, int k, moe_dtype dt, int capacity, void* dx,
+                                     float* dWg, float* dW1, float* dW3, float* dW2,
+                                     const void* fwd_ws, size_t fwd_ws_bytes, void* bwd_ws,
+                                     size_t bwd_ws_bytes, cudaEvent_t* events, int n_events,
+                                     cudaStream_t stream) {
+    return layer_backward_impl(x, Wg, W1, W3, W2, dy, T, d, h, E, k, dt, capacity, dx, dWg, dW1,
+                               dW3, dW2, fwd_ws, fwd_ws_bytes, bwd_ws, bwd_ws_bytes, events,
+                               n_events, stream);
 }
 
 moe_status moe_selftest_wait_timeout(void* ws, size_t ws_bytes, double limit_seconds,

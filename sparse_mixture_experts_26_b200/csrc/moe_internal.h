@@ -195,8 +195,12 @@ struct BwdArgs {
     float* dH;                 // [2T, h]
     void* DUV;                 // bf16 [2T, 2h]: du then dv
     float* dX;                 // [2T, d]
-    float* dwg_part;           // [ceil(T / 256), d, E]
+    float* dwg_part;           // [bwd_dwg_chunks(T), d, E]
     uint32_t* status;
+    // optional events recorded before the first launch and after each stage:
+    // prep, dH, du/dv, dX, dx, dW2, dW1/dW3, dWg (null handles skipped)
+    cudaEvent_t* ev;
+    int n_ev;
 };
 size_t bwd_dwg_chunks(int T);
 cudaError_t launch_layer_backward(const BwdArgs& a, cudaStream_t s);
