@@ -236,7 +236,8 @@ def workload_config(wl, extra=None):
                     f"E={wl.E} top-{wl.k}, {wl.dtype}" if wl.d == 4096 else wl.note,
         "T": wl.T, "d": wl.d, "h": wl.h, "E": wl.E, "k": wl.k, "seed": wl.seed,
         "routing": wl.kind,
-        "l2": "no flush: inputs larger than L2 (2.8 GB of expert weights streamed per step)",
+        "l2": f"no flush: inputs larger than L2 ({3 * wl.E * wl.d * wl.h * 2 / 1e9:.1f} GB of "
+              "expert weights streamed per step)",
     }
     if extra:
         cfg.update(extra)
@@ -460,6 +461,16 @@ def backward_stage_flops(wl):
     return {1: u, 2: 2 * u, 3: 2 * u, 5: u, 6: 2 * u}
 
 
+def wgrad_bytes(wl, stage: int) -> int:
+    """Algorithmic bytes of a weight-gradient launch: fp32 outputs written once, the
+    two grouped bf16 operands read once (stage 5: dW2 from dY and H; stage 6: dW1 and
+    dW3 from [du dv] and x)."""
+    P = wl.T * wl.k
+    if stage == 5:
+        return wl.E * wl.d * wl.h * 4 + P * (wl.d + wl.h) * 2
+    return 2 * wl.E * wl.h * wl.d * 4 + P * (2 * wl.h + wl.d) * 2
+
+
 def run_ours_backward(args):
     import torch
 
@@ -529,13 +540,33 @@ def run_ours_backward(args):
     dom = max(BWD_KERNELS, key=lambda j: st_ms[j])
     kname, tag = BWD_KERNELS[dom]
     peaks, peak_src = load_peaks()
-    ach = flops[dom] / (st_ms[dom] * 1e-3) / 1e12
-    peak = float(peaks["bf16_tflops"])
-    roofline = {"bound": "tensor", "achieved": round(ach, 1), "peak": peak, "unit": "TFLOP/s",
-                "frac": round(ach / peak, 4),
-                "traffic": ncu_traffic(tag, wl.name, os.path.join(CSRC, "backward_sm100.cu")),
+    if T <= DECODE_MAX_TOKENS and dom in (5, 6):
+        # a few rows per expert: the weight-gradient GEMMs are bound by writing their
+        # fp32 outputs, so their roofline is HBM bandwidth
+        bound, unit, peak_kind = "hbm", "GB/s", "copy"
+        ach = wgrad_bytes(wl, dom) / (st_ms[dom] * 1e-3) / 1e9
+        peak = float(peaks["hbm_gbs"])
+    else:
+        bound, unit, peak_kind = "tensor", "TFLOP/s", "burst"
+        ach = flops[dom] / (st_ms[dom] * 1e-3) / 1e12
+        peak = float(peaks["bf16_tflops"])
+    src = os.path.join(CSRC, "backward_sm100.cu")
+    traffic, traffic_note = ncu_traffic(tag, wl.name, src), None
+    if traffic is None and wl.name == "prefill" and dom in (5, 6):
+        # The full backward holds ~10 GB, too much for a --set full capture: scale the
+        # half-width capture (same rows per expert) by the kernel's algorithmic bytes.
+        t_half = ncu_traffic(tag, "prefill_half", src)
+        if t_half is not None:
+            half = WORKLOADS["prefill_half"]
+            traffic = round(t_half * wgrad_bytes(wl, dom) / wgrad_bytes(half, dom))
+            traffic_note = ("scaled from the prefill_half capture by algorithmic bytes "
+                            f"({wgrad_bytes(wl, dom) / wgrad_bytes(half, dom):.2f}x)")
+    roofline = {"bound": bound, "achieved": round(ach, 1), "peak": peak, "unit": unit,
+                "frac": round(ach / peak, 4), "traffic": traffic,
                 "kernel": f"{kname} (stage '{BWD_STAGES[dom]}')",
-                "peak_source": f"{peak_src} (burst)"}
+                "peak_source": f"{peak_src} ({peak_kind})"}
+    if traffic_note:
+        roofline["traffic_note"] = traffic_note
     total_flops = sum(flops.values())
     layer = {"ms": round(ms, 4), "tflops": round(total_flops / (ms * 1e-3) / 1e12, 1),
              "stage_ms": {n: round(v, 4) for n, v in zip(BWD_STAGES, st_ms)},
@@ -681,7 +712,7 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=None)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="decode",
-                    choices=["decode", "prefill", "skew", "long", "tiny_f32"])
+                    choices=["decode", "prefill", "skew", "long", "tiny_f32", "prefill_half"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-tokens", type=int, default=16)
     ap.add_argument("--cpu-budget-s", type=float, default=10.0)

@@ -72,6 +72,11 @@ WORKLOADS = {
                      note="Mixtral-8x7B layer, T=4096, skewed routing, bf16"),
     "long": Workload("long", T=32768, d=MIXTRAL_D, h=MIXTRAL_H, seed=4, kind="long",
                      note="Mixtral-8x7B layer, T=32768 (32K context), bf16"),
+    # Half-width layer with the prefill's rows per expert, for profiler captures that
+    # must hold a few GB on the device at most (backward: about 3 GB).
+    "prefill_half": Workload("prefill_half", T=4096, d=MIXTRAL_D // 2, h=MIXTRAL_H // 2,
+                             seed=5, note="half-width layer (d=2048, h=7168), T=4096, "
+                                          "bf16: profiling case"),
 }
 
 SKEW_OFFSETS = (2.0, 1.0, 0.0, 0.0, 0.0, 0.0, -4.0, -4.0)
