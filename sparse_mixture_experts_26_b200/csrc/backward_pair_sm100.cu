@@ -1,0 +1,514 @@
+// backward_pair_sm100.cu -- the weight-gradient GEMMs of the backward pass on pairs of
+// SMs (tcgen05 cta_group::2), for reductions over many rows per expert.
+//
+// Same computation as bwd_wgrad_kernel in backward_sm100.cu (the exact derivative of
+// the layer; crackai "Mixtral of Experts", "Key Takeaways": the router and experts are
+// learned jointly):  out[e][m][n] = sum over the rows r of expert e of A[r, m] B[r, n],
+// with dW2 = dY^T H and [dW1; dW3] = [du dv]^T x.  A tile is 256 output rows (m) x 256
+// output columns (n), computed by a cluster of two CTAs: each CTA stages its own 128
+// columns of A and its own 128 columns of B per 64-row K block (both MN-major boxes),
+// and one thread of the leader issues tcgen05.mma.cta_group::2 (M = 256 from the two
+// A halves, N = 256 from the two B halves); each CTA's TMEM receives its 128 rows.
+// Per SM a stage is 32 KiB instead of 48 KiB for the same math, which leaves room for
+// 6 stages next to the output staging buffers.
+//
+// A reduction starts and ends at arbitrary rows, so the rows of an expert's last,
+// partial K block that belong to the next expert must be zero before the MMA reads
+// them.  Whole K blocks take the plain pair path: both CTAs' TMA loads count their
+// bytes on the leader's "full" barrier.  A partial block's loads complete instead on
+// a barrier of each CTA's own ("landed"); a fix-up warp in each CTA waits there,
+// clears the rows in its own tiles and makes the writes visible to the tensor core
+// (fence.proxy.async); the peer's then arrives on the leader's "fixed" barrier, and
+// the leader's, once both are done, arrives on "full".  (A handshake on every block
+// instead measured 2-4x slower: a cluster-scope arrive per block serialises the
+// pipeline.)  The leader's MMA completions are multicast to both CTAs' "empty" and
+// "tmem_full" barriers; both epilogues arrive on the leader's "tmem_empty".  The
+// epilogue writes with per-warp TMA tensor stores, as the single-SM kernel does.
+// Every wait is bounded.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "moe_internal.h"
+#include "sm100_ptx.cuh"
+
+namespace moe {
+
+bool encode_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                    uint32_t box_rows);
+bool encode_f32_3d(CUtensorMap* map, const void* base, uint64_t batches, uint64_t rows,
+                   uint64_t cols, uint32_t box_cols, uint32_t box_rows);
+
+namespace {
+
+constexpr int kRows = 128;                  // output rows per CTA (TMEM lanes)
+constexpr int kBK = 64;                     // K rows per stage
+constexpr int kN = 256;                     // output columns per tile
+constexpr int kStages = 6;
+constexpr int kBox = 64 * 128;              // one 64-column x 64-row bf16 box: 8 KiB
+constexpr int kABytes = 2 * kBox;           // this CTA's 128 columns of A
+constexpr int kBBytes = 2 * kBox;           // this CTA's 128 columns of B
+constexpr int kStageBytes = kABytes + kBBytes;
+constexpr int kThreads = 224;  // TMA, MMA, 4 epilogue warps, fix-up warp
+constexpr int kEpiThreads = 128;
+constexpr uint32_t kTmemCols = 2 * kN;
+constexpr int kOutBufs = 2;                 // staging buffers per epilogue warp
+constexpr int kStageOutBytes = 32 * 32 * 4; // one 32 x 32 fp32 chunk
+constexpr int kSmemBytes = kStages * kStageBytes + 4 * kOutBufs * kStageOutBytes +
+                           1024 /*align*/ + 1024 /*book*/;
+static_assert(kSmemBytes <= 232448, "shared memory");
+constexpr int kVoteBarrier = 2;
+constexpr uint16_t kBothCtas = 0x3;
+constexpr uint64_t kMnStep = (16 * 128) >> 4;  // descriptor step for K = 16 rows
+
+__device__ __forceinline__ uint64_t sw128_mn_desc(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
+    d |= static_cast<uint64_t>(kBox >> 4) << 16;   // next 64-wide M/N group: one box on
+    d |= static_cast<uint64_t>(1024u >> 4) << 32;  // next 8 rows of K
+    d |= static_cast<uint64_t>(1u) << 46;
+    d |= static_cast<uint64_t>(2u) << 61;
+    return d;
+}
+// M = 256 (two CTAs), N = 256, both operands MN-major.
+constexpr uint32_t kIdesc = idesc_bf16_f32(2 * kRows, kN) | (1u << 15) | (1u << 16);
+
+struct Book {
+    uint64_t landed[kStages];    // partial blocks: this CTA's loads are in shared memory
+    uint64_t fixed[kStages];     // leader, partial blocks: the peer cleared its rows
+    uint64_t full[kStages];      // leader: both CTAs' stages are ready for the MMA
+    uint64_t empty[kStages];     // the MMAs reading a stage are done (multicast)
+    uint64_t tmem_full[2];
+    uint64_t tmem_empty[2];      // leader: both epilogues drained the accumulator
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort_flag;
+    int off[kMaxExperts + 1];
+    int end[kMaxExperts];
+};
+static_assert(sizeof(Book) <= 1024, "bookkeeping reserve");
+
+struct PArgs {
+    const int32_t* offsets;
+    int E;
+    int rows;
+    int M;
+    int N;
+    int m_pairs;     // ceil(M / 256)
+    int n_tiles;     // ceil(N / 256)
+    int split;       // output rows m < split go to out0 (tmO0), the rest to out1 (tmO1)
+    float* out0;
+    float* out1;
+    uint32_t* status;
+    int cap;
+};
+
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
+    const unsigned long long t0 = global_timer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (global_timer_ns() - t0 > kDrainTimeoutNs) break;
+    }
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ float bits_f32(uint32_t u) { return __uint_as_float(u); }
+
+// Bounded wait with cluster-scope acquire: pairs with the peer's cluster-scope release
+// arrive, so the peer's shared-memory writes before it are ordered before what follows.
+__device__ __forceinline__ bool wait_cluster_bounded(uint64_t* bar, uint32_t parity,
+                                                     volatile int* abort_flag, uint32_t* status) {
+    auto try_wait = [&]() {
+        uint32_t done;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(done)
+            : "r"(smem_u32(bar)), "r"(parity)
+            : "memory");
+        return done != 0;
+    };
+    if (try_wait()) return true;
+    const unsigned long long t0 = global_timer_ns();
+    while (!try_wait()) {
+        if (*abort_flag) return false;
+        if (global_timer_ns() - t0 > kWaitTimeoutNs) {
+            *abort_flag = 1;
+            if (status) atomicOr(status, 1u);  // MOE_DEV_FLAG_TIMEOUT
+            return false;
+        }
+    }
+    return true;
+}
+
+__device__ __forceinline__ void short_pause_ns(unsigned long long ns) {
+    const unsigned long long t0 = global_timer_ns();
+    while (global_timer_ns() - t0 < ns) {
+    }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    bwd_wgrad_pair_kernel(const __grid_constant__ CUtensorMap tmA,
+                          const __grid_constant__ CUtensorMap tmB,
+                          const __grid_constant__ CUtensorMap tmO0,
+                          const __grid_constant__ CUtensorMap tmO1, const PArgs args) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint8_t* sA = smem;
+    uint8_t* sB = smem + kStages * kABytes;
+    uint8_t* sOut = smem + kStages * kStageBytes;
+    Book& bk = *reinterpret_cast<Book*>(sOut + 4 * kOutBufs * kStageOutBytes);
+    volatile int* abort_flag = &bk.abort_flag;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int E = args.E;
+    const uint32_t rank = cluster_ctarank();  // 0 = leader, 1 = peer
+    const bool leader = rank == 0;
+    const int pair = blockIdx.x >> 1;
+    const int npairs = gridDim.x >> 1;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&bk.landed[s], 1);
+            mbar_init(&bk.fixed[s], 1);
+            mbar_init(&bk.full[s], 1);
+            mbar_init(&bk.empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&bk.tmem_full[a], 1);
+            mbar_init(&bk.tmem_empty[a], 2 * kEpiThreads);
+        }
+        mbar_init(&bk.drain, 1);
+        bk.abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+        tma_prefetch_desc(&tmO0);
+        tma_prefetch_desc(&tmO1);
+    }
+    if (warp == 1) tmem_alloc_pair(&bk.tmem_base, kTmemCols);
+    if (threadIdx.x == 0) {
+        int prev = 0;
+        for (int g = 0; g <= E; ++g) {
+            int v = args.offsets[g];
+            v = v < prev ? prev : (v > args.rows ? args.rows : v);
+            bk.off[g] = v;
+            prev = v;
+        }
+        for (int g = 0; g < E; ++g) {
+            const int n = bk.off[g + 1] - bk.off[g];
+            bk.end[g] = bk.off[g] + (n < args.cap ? n : args.cap);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();  // both CTAs' barriers are initialised before either signals the other
+    tc_fence_after();
+
+    const uint32_t tmem_base = bk.tmem_base;
+    const int per_e = args.m_pairs * args.n_tiles;
+    const int total = E * per_e;
+
+    auto tile_of = [&](int tile, int& e, int& mp, int& nt, int& r0, int& n_rows) {
+        e = tile / per_e;
+        const int local = tile - e * per_e;
+        nt = local % args.n_tiles;  // column blocks innermost
+        mp = local / args.n_tiles;
+        r0 = bk.off[e];
+        n_rows = bk.end[e] - bk.off[e];
+    };
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer (both)
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0, lpar = 0;     // ring phase; parity of each landed[s]
+            uint32_t pend_full = 0, pend_full_ph = 0, pend_land = 0, pend_land_ph = 0;
+            bool ok = true, issued = false;
+            for (int tile = pair; ok && tile < total; tile += npairs) {
+                int e, mp, nt, r0, n_rows;
+                tile_of(tile, e, mp, nt, r0, n_rows);
+                const int nkb = (n_rows + kBK - 1) / kBK;
+                const int mcol = mp * 2 * kRows + static_cast<int>(rank) * kRows;
+                const int ncol = nt * kN + static_cast<int>(rank) * (kN / 2);
+                for (int kb = 0; kb < nkb; ++kb) {
+                    if (!mbar_wait_bounded(&bk.empty[stage], phase ^ 1u, abort_flag,
+                                           args.status)) {
+                        ok = false;
+                        break;
+                    }
+                    const int r = r0 + kb * kBK;
+                    uint8_t* a = sA + stage * kABytes;
+                    uint8_t* b = sB + stage * kBBytes;
+                    const uint32_t bit = 1u << stage;
+                    if (n_rows - kb * kBK < kBK) {
+                        // partial block: land locally, the fix-up warp takes over
+                        mbar_arrive_expect_tx(&bk.landed[stage], kStageBytes);
+                        tma_load_2d(&tmA, &bk.landed[stage], a, mcol, r);
+                        tma_load_2d(&tmA, &bk.landed[stage], a + kBox, mcol + 64, r);
+                        tma_load_2d(&tmB, &bk.landed[stage], b, ncol, r);
+                        tma_load_2d(&tmB, &bk.landed[stage], b + kBox, ncol + 64, r);
+                        pend_land |= bit;
+                        pend_land_ph = (pend_land_ph & ~bit) | (lpar & bit);
+                        lpar ^= bit;
+                    } else {
+                        const uint32_t full_leader = map_to_cta(smem_u32(&bk.full[stage]), 0);
+                        if (leader) mbar_arrive_expect_tx(&bk.full[stage], 2 * kStageBytes);
+                        tma_load_2d_pair(&tmA, full_leader, a, mcol, r);
+                        tma_load_2d_pair(&tmA, full_leader, a + kBox, mcol + 64, r);
+                        tma_load_2d_pair(&tmB, full_leader, b, ncol, r);
+                        tma_load_2d_pair(&tmB, full_leader, b + kBox, ncol + 64, r);
+                        pend_full |= bit;
+                        pend_full_ph = (pend_full_ph & ~bit) | (phase << stage);
+                    }
+                    issued = true;
+                    if (++stage == kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (!ok && issued) {
+                // let copies in flight land before this CTA's shared memory is released
+                for (int s = 0; s < kStages; ++s)
+                    if (pend_land & (1u << s)) drain_wait(&bk.landed[s], (pend_land_ph >> s) & 1u);
+                if (leader) {
+                    for (int s = 0; s < kStages; ++s)
+                        if (pend_full & (1u << s)) drain_wait(&bk.full[s], (pend_full_ph >> s) & 1u);
+                } else if (pend_full) {
+                    short_pause_ns(2000000ull);  // its pair copies count on the leader's barriers
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer (leader)
+        if (lane == 0 && leader) {
+            int stage = 0, acc = 0;
+            uint32_t phase = 0, acc_phase = 0;
+            bool ok = true, issued = false;
+            for (int tile = pair; ok && tile < total; tile += npairs) {
+                int e, mp, nt, r0, n_rows;
+                tile_of(tile, e, mp, nt, r0, n_rows);
+                const int nkb = (n_rows + kBK - 1) / kBK;
+                if (nkb == 0) continue;  // zero tile: written by the epilogues alone
+                if (!mbar_wait_bounded(&bk.tmem_empty[acc], acc_phase ^ 1u, abort_flag,
+                                       args.status)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kN);
+                for (int kb = 0; kb < nkb; ++kb) {
+                    if (!mbar_wait_bounded(&bk.full[stage], phase, abort_flag, args.status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t ad = sw128_mn_desc(smem_u32(sA + stage * kABytes));
+                    const uint64_t bd = sw128_mn_desc(smem_u32(sB + stage * kBBytes));
+#pragma unroll
+                    for (int k = 0; k < kBK / 16; ++k)
+                        umma_bf16_pair(d_tmem, ad + kMnStep * k, bd + kMnStep * k, kIdesc,
+                                       (kb | k) != 0);
+                    umma_commit_pair(&bk.empty[stage], kBothCtas);
+                    issued = true;
+                    if (++stage == kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                umma_commit_pair(&bk.tmem_full[acc], kBothCtas);
+                acc ^= 1;
+                if (acc == 0) acc_phase ^= 1u;
+            }
+            if (!ok && issued) {
+                umma_commit_pair(&bk.drain, 0x1);
+                drain_wait(&bk.drain, 0);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 6) {
+        // ------------------------------------------- fix-up of partial K blocks (both)
+        int stage = 0;
+        uint32_t lpar = 0, fpar = 0;  // parity of each landed[s] / fixed[s]
+        const uint32_t cap_rows = args.cap != INT_MAX ? 1u : 0u;
+        bool ok = true;
+        for (int tile = pair; ok && tile < total; tile += npairs) {
+            int e, mp, nt, r0, n_rows;
+            tile_of(tile, e, mp, nt, r0, n_rows);
+            const int nkb = (n_rows + kBK - 1) / kBK;
+            for (int kb = 0; kb < nkb; ++kb) {
+                const int kv = n_rows - kb * kBK;  // rows of this block inside the group
+                if (kv < kBK) {
+                    const uint32_t bit = 1u << stage;
+                    int got = 1;
+                    if (lane == 0)
+                        got = mbar_wait_bounded(&bk.landed[stage], (lpar >> stage) & 1u,
+                                                abort_flag, args.status);
+                    lpar ^= bit;
+                    ok = __shfl_sync(0xffffffffu, got, 0) != 0;
+                    if (!ok) break;
+                    // rows kv..63 belong to the next group: clear them in this CTA's A
+                    // boxes (and B boxes when a capacity may have left rows unwritten)
+                    uint8_t* a = sA + stage * kABytes;
+                    uint8_t* b = sB + stage * kBBytes;
+                    const int nz = (kBK - kv) * 8;
+                    const int boxes = cap_rows ? 4 : 2;
+                    for (int i = lane; i < boxes * nz; i += 32) {
+                        const int box = i / nz, c = i - box * nz;
+                        uint8_t* base = box < 2 ? a + box * kBox : b + (box - 2) * kBox;
+                        *reinterpret_cast<uint4*>(base + kv * 128 + c * 16) =
+                            make_uint4(0u, 0u, 0u, 0u);
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        if (!leader) {
+                            mbar_arrive_cluster(map_to_cta(smem_u32(&bk.fixed[stage]), 0));
+                        } else {
+                            got = wait_cluster_bounded(&bk.fixed[stage], (fpar >> stage) & 1u,
+                                                       abort_flag, args.status);
+                            if (got) mbar_arrive(&bk.full[stage]);
+                        }
+                    }
+                    fpar ^= bit;
+                    ok = __shfl_sync(0xffffffffu, got, 0) != 0;
+                    if (!ok) break;
+                }
+                if (++stage == kStages) stage = 0;
+            }
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ epilogue (both)
+        const int q = warp & 3;  // warps 2..5: TMEM lane quarters 2, 3, 0, 1
+        const uint32_t empty_leader0 = map_to_cta(smem_u32(&bk.tmem_empty[0]), 0);
+        const uint32_t empty_leader1 = map_to_cta(smem_u32(&bk.tmem_empty[1]), 0);
+        uint8_t* wstage = sOut + q * kOutBufs * kStageOutBytes;
+        int acc = 0, buf = 0;
+        uint32_t acc_phase = 0;
+        for (int tile = pair; tile < total; tile += npairs) {
+            int e, mp, nt, r0, n_rows;
+            tile_of(tile, e, mp, nt, r0, n_rows);
+            const int m0 = mp * 2 * kRows + static_cast<int>(rank) * kRows;  // this CTA's rows
+            const int m = m0 + q * 32 + lane;
+            const bool mvalid = m < args.M;
+            float* out = m < args.split
+                             ? args.out0 + (static_cast<size_t>(e) * args.split + m) * args.N
+                             : args.out1 + (static_cast<size_t>(e) * (args.M - args.split) +
+                                            (m - args.split)) * args.N;
+            const int col0 = nt * kN;
+            if (n_rows == 0) {
+                if (mvalid)
+                    for (int col = col0; col < col0 + kN && col < args.N; col += 4)
+                        *reinterpret_cast<float4*>(out + col) = make_float4(0.f, 0.f, 0.f, 0.f);
+                continue;
+            }
+            if (!bar_all(mbar_wait_bounded(&bk.tmem_full[acc], acc_phase, abort_flag,
+                                           args.status),
+                         kVoteBarrier, kEpiThreads))
+                break;
+            tc_fence_after();
+            const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                                   static_cast<uint32_t>(acc * kN);
+            // A slice that starts at or past M (the peer's half of a last, partial pair
+            // tile) stores nothing: for dW2 the second output map is the first one again.
+            const bool slice_valid = m0 < args.M;
+            const bool second = m0 >= args.split;
+            const bool straddle = m0 < args.split && m0 + kRows > args.split;
+#pragma unroll 1
+            for (int ch = 0; ch < 8; ++ch) {
+                uint32_t v[32];
+                tmem_ld_32cols(tbase + ch * 32, v);
+                tmem_ld_wait();
+                if (!slice_valid) continue;
+                if (!straddle) {
+                    uint8_t* st = wstage + buf * kStageOutBytes;
+                    if (lane == 0) bulk_wait_group_read<kOutBufs - 1>();
+                    __syncwarp();
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        *reinterpret_cast<uint4*>(st + lane * 128 + ((j ^ (lane & 7)) << 4)) =
+                            make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_3d(second ? &tmO1 : &tmO0, st, col0 + ch * 32,
+                                     (second ? m0 - args.split : m0) + q * 32, e);
+                        bulk_commit_group();
+                    }
+                    if (++buf == kOutBufs) buf = 0;
+                } else if (mvalid) {
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const int col = col0 + ch * 32 + j * 4;
+                        if (col < args.N)
+                            *reinterpret_cast<float4*>(out + col) =
+                                make_float4(bits_f32(v[4 * j]), bits_f32(v[4 * j + 1]),
+                                            bits_f32(v[4 * j + 2]), bits_f32(v[4 * j + 3]));
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive_cluster(acc == 0 ? empty_leader0 : empty_leader1);
+            acc ^= 1;
+            if (acc == 0) acc_phase ^= 1u;
+        }
+        if (lane == 0) bulk_wait_group<0>();  // every store complete before the block exits
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();  // the leader's MMAs into this CTA's TMEM and smem are done
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem_base, kTmemCols);
+    }
+}
+
+}  // namespace
+
+// Weight gradients on CTA pairs: A [rows, M] and B [rows, N] grouped bf16 operands
+// (tensor maps with 64 x 64 boxes), outputs through 3-D fp32 maps with 32 x 32 boxes.
+cudaError_t launch_wgrad_pair(const CUtensorMap& A, const CUtensorMap& B, const CUtensorMap& O0,
+                              const CUtensorMap& O1, const int32_t* offsets, int E, int rows,
+                              int M, int N, int split, float* out0, float* out1, uint32_t* status,
+                              int cap, cudaStream_t s) {
+    static int configured[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && !configured[dev]) {
+        cudaFuncSetAttribute(bwd_wgrad_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kSmemBytes);
+        configured[dev] = 1;
+    }
+    PArgs p{offsets, E, rows, M, N, (M + 2 * kRows - 1) / (2 * kRows), (N + kN - 1) / kN, split,
+            out0, out1, status, cap};
+    const long long tiles = static_cast<long long>(E) * p.m_pairs * p.n_tiles;
+    const int max_pairs = device_sm_count() / 2;
+    const int npairs = static_cast<int>(tiles < max_pairs ? (tiles < 1 ? 1 : tiles) : max_pairs);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * npairs);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t err = cudaLaunchKernelEx(&cfg, bwd_wgrad_pair_kernel, A, B, O0, O1, p);
+    return err != cudaSuccess ? err : cudaGetLastError();
+}
+
+}  // namespace moe

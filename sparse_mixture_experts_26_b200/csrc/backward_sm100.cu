@@ -43,6 +43,11 @@ bool encode_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t 
                     uint32_t box_rows);
 bool encode_f32_3d(CUtensorMap* map, const void* base, uint64_t batches, uint64_t rows,
                    uint64_t cols, uint32_t box_cols, uint32_t box_rows);
+// Defined in backward_pair_sm100.cu.
+cudaError_t launch_wgrad_pair(const CUtensorMap& A, const CUtensorMap& B, const CUtensorMap& O0,
+                              const CUtensorMap& O1, const int32_t* offsets, int E, int rows,
+                              int M, int N, int split, float* out0, float* out1, uint32_t* status,
+                              int cap, cudaStream_t s);
 
 namespace {
 
@@ -974,21 +979,40 @@ cudaError_t launch_layer_backward(const BwdArgs& a, cudaStream_t s) {
         !encode_f32_3d(&m_dW1, a.dW1, E, h, d, 32, 32) ||
         !encode_f32_3d(&m_dW3, a.dW3, E, h, d, 32, 32))
         return cudaErrorInvalidValue;
-    // Few rows per expert: the output stores bound the kernel (deep staging); many:
-    // the reduction does (deep input pipeline).
-    const bool short_k = P <= kWgradShortRows;
-    {
+    // Few rows per expert: the output stores bound the kernel (single-SM kernel with
+    // deep staging); many: the reduction does (CTA pairs, deep input pipeline).
+    if (P <= kWgradShortRows) {
         WArgs w{a.offsets, E, P, d, h, (d + kBM - 1) / kBM, (h + kN - 1) / kN, d, a.dW2, a.dW2,
                 a.status, a.cap};
-        err = launch_wgrad<kModeW2>(short_k, grid_for(static_cast<long long>(E) * w.m_tiles * w.n_tiles, sms),
+        err = launch_wgrad<kModeW2>(true, grid_for(static_cast<long long>(E) * w.m_tiles * w.n_tiles, sms),
                                     s, m_dY64, m_H64, m_dW2, m_dW2, w);
         if (err != cudaSuccess || (err = mark(6)) != cudaSuccess) return err;
-    }
-    {
-        WArgs w{a.offsets, E, P, 2 * h, d, (2 * h + kBM - 1) / kBM, (d + kN - 1) / kN, h, a.dW1,
-                a.dW3, a.status, a.cap};
-        err = launch_wgrad<kModeW13>(short_k, grid_for(static_cast<long long>(E) * w.m_tiles * w.n_tiles, sms),
-                                     s, m_duv64, m_x64, m_dW1, m_dW3, w);
+        WArgs w13{a.offsets, E, P, 2 * h, d, (2 * h + kBM - 1) / kBM, (d + kN - 1) / kN, h,
+                  a.dW1, a.dW3, a.status, a.cap};
+        err = launch_wgrad<kModeW13>(true, grid_for(static_cast<long long>(E) * w13.m_tiles * w13.n_tiles, sms),
+                                     s, m_duv64, m_x64, m_dW1, m_dW3, w13);
+        if (err != cudaSuccess || (err = mark(7)) != cudaSuccess) return err;
+    } else {
+        // A device that cannot co-schedule a CTA pair takes the single-SM kernel.
+        err = launch_wgrad_pair(m_dY64, m_H64, m_dW2, m_dW2, a.offsets, E, P, d, h, d, a.dW2,
+                                a.dW2, a.status, a.cap, s);
+        if (err != cudaSuccess) {
+            cudaGetLastError();
+            WArgs w{a.offsets, E, P, d, h, (d + kBM - 1) / kBM, (h + kN - 1) / kN, d, a.dW2,
+                    a.dW2, a.status, a.cap};
+            err = launch_wgrad<kModeW2>(false, grid_for(static_cast<long long>(E) * w.m_tiles * w.n_tiles, sms),
+                                        s, m_dY64, m_H64, m_dW2, m_dW2, w);
+        }
+        if (err != cudaSuccess || (err = mark(6)) != cudaSuccess) return err;
+        err = launch_wgrad_pair(m_duv64, m_x64, m_dW1, m_dW3, a.offsets, E, P, 2 * h, d, h, a.dW1,
+                                a.dW3, a.status, a.cap, s);
+        if (err != cudaSuccess) {
+            cudaGetLastError();
+            WArgs w{a.offsets, E, P, 2 * h, d, (2 * h + kBM - 1) / kBM, (d + kN - 1) / kN, h,
+                    a.dW1, a.dW3, a.status, a.cap};
+            err = launch_wgrad<kModeW13>(false, grid_for(static_cast<long long>(E) * w.m_tiles * w.n_tiles, sms),
+                                         s, m_duv64, m_x64, m_dW1, m_dW3, w);
+        }
         if (err != cudaSuccess || (err = mark(7)) != cudaSuccess) return err;
     }
     // 7. dWg
