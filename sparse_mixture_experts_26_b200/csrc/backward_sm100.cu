@@ -43,6 +43,11 @@ bool encode_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t 
                     uint32_t box_rows);
 bool encode_f32_3d(CUtensorMap* map, const void* base, uint64_t batches, uint64_t rows,
                    uint64_t cols, uint32_t box_cols, uint32_t box_rows);
+// Defined in grouped_gemm_pair_sm100.cu.
+cudaError_t launch_bwd_rows_pair(int mode, const CUtensorMap& a, const CUtensorMap& b0,
+                                 const CUtensorMap& b1, const int32_t* offsets, int E, int rows,
+                                 int d, int h, void* out, const float* dH, uint32_t* status,
+                                 int cap, cudaStream_t s);
 // Defined in backward_pair_sm100.cu.
 cudaError_t launch_wgrad_pair(const CUtensorMap& A, const CUtensorMap& B, const CUtensorMap& O0,
                               const CUtensorMap& O1, const int32_t* offsets, int E, int rows,
@@ -935,9 +940,15 @@ cudaError_t launch_layer_backward(const BwdArgs& a, cudaStream_t s) {
         !encode_bf16_2d(&m_W3mn, a.W3, static_cast<uint64_t>(E) * h, d, 64))
         return cudaErrorInvalidValue;
     const long long row_blocks = (static_cast<long long>(P) + 127LL * E) / kBM;
+    // Many rows: the CTA-pair forms of the three row GEMMs (the forward's pair engine).
+    const bool pairs = P >= kPairMinRows && pair_gemm_enabled();
 
     // 2. dH = dY W2_e
-    {
+    if (pairs) {
+        err = launch_bwd_rows_pair(0, m_dY128, m_W2, m_W2, a.offsets, E, P, d, h, a.dH, nullptr,
+                                   a.status, a.cap, s);
+        if (err != cudaSuccess || (err = mark(2)) != cudaSuccess) return err;
+    } else {
         RowArgs r{a.offsets, E, P, d, h, (h + kN - 1) / kN, h, d, a.dH, nullptr, a.status, a.cap};
         configure(bwd_rows_kernel<kModeDH>, kSlotDH, kSmemBytes);
         err = launch_k(bwd_rows_kernel<kModeDH>, grid_for(row_blocks * r.n_tiles, sms), kThreads,
@@ -945,7 +956,11 @@ cudaError_t launch_layer_backward(const BwdArgs& a, cudaStream_t s) {
         if (err != cudaSuccess || (err = mark(2)) != cudaSuccess) return err;
     }
     // 3. du, dv (recomputes a and b)
-    {
+    if (pairs) {
+        err = launch_bwd_rows_pair(1, m_x, m_W1r, m_W3r, a.offsets, E, P, d, h, a.DUV, a.dH,
+                                   a.status, a.cap, s);
+        if (err != cudaSuccess || (err = mark(3)) != cudaSuccess) return err;
+    } else {
         RowArgs r{a.offsets, E, P, d, h, (h + 127) / 128, h, d, a.DUV, a.dH, a.status, a.cap};
         configure(bwd_rows_kernel<kModeDUV>, kSlotDUV, kSmemBytes);
         err = launch_k(bwd_rows_kernel<kModeDUV>, grid_for(row_blocks * r.n_tiles, sms),
@@ -953,7 +968,11 @@ cudaError_t launch_layer_backward(const BwdArgs& a, cudaStream_t s) {
         if (err != cudaSuccess || (err = mark(3)) != cudaSuccess) return err;
     }
     // 4. dX = [du dv] [W1_e ; W3_e]
-    {
+    if (pairs) {
+        err = launch_bwd_rows_pair(2, m_duv128, m_W1mn, m_W3mn, a.offsets, E, P, d, h, a.dX,
+                                   nullptr, a.status, a.cap, s);
+        if (err != cudaSuccess || (err = mark(4)) != cudaSuccess) return err;
+    } else {
         RowArgs r{a.offsets, E, P, 2 * h, d, (d + kN - 1) / kN, h, d, a.dX, nullptr, a.status,
                   a.cap};
         configure(bwd_rows_kernel<kModeDX>, kSlotDX, kSmemBytes);

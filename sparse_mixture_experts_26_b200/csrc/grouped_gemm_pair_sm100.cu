@@ -61,7 +61,15 @@ constexpr int kXferBarrier = 1;
 constexpr int kVoteBarrier = 2;  // epilogue vote after a bounded wait
 constexpr uint16_t kBothCtas = 0x3;
 
-enum Epilogue { kEpiSwiGLU = 0, kEpiStoreF32 = 1 };
+// kEpiBwdSwiGLU (backward pass): the accumulator holds a = x.W1 and b = x.W3 as for
+// kEpiSwiGLU; with g = dH of the same outputs the epilogue writes du = g b silu'(a)
+// and dv = g silu(a) (bf16, row stride 2N: du in columns [0, N), dv in [N, 2N)).
+enum Epilogue { kEpiSwiGLU = 0, kEpiStoreF32 = 1, kEpiBwdSwiGLU = 2 };
+// B operand: K-major weight rows (the forward), or MN-major (weights [K, N] read as
+// 64 x 64 boxes; backward dH = dY W2), optionally taken from W1 for k < h and from W3
+// for k >= h (backward dX = [du dv] [W1; W3]).
+enum BOperand { kBKMajor = 0, kBMn = 1, kBMnSplit = 2 };
+constexpr int kBoxMn = 64 * 128;  // one 64 x 64 bf16 box of an MN-major operand
 
 struct PairArgs {
     const int32_t* offsets;
@@ -74,6 +82,8 @@ struct PairArgs {
     void* out;
     uint32_t* status;
     int cap;      // rows kept per group (capacity; INT_MAX = no limit)
+    int h;             // kBMnSplit: the K index where W3 takes over from W1
+    const float* dH;   // kEpiBwdSwiGLU: dH fp32 [rows, N]
 };
 
 struct PairBook {
@@ -120,6 +130,23 @@ __device__ __forceinline__ float silu_mul(float a, float b) {
     return a / (1.0f + __expf(-a)) * b;
 }
 
+// du = g b silu'(a), dv = g silu(a) for one output of the backward SwiGLU step.
+__device__ __forceinline__ void bwd_swiglu(float a, float b, float g, float& du, float& dv) {
+    const float s = 1.0f / (1.0f + __expf(-a));
+    du = g * b * (s * (1.0f + a * (1.0f - s)));
+    dv = g * (a * s);
+}
+
+__device__ __forceinline__ uint64_t sw128_mn_desc_pair(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
+    d |= static_cast<uint64_t>(kBoxMn >> 4) << 16;  // next 64-wide group of N: one box on
+    d |= static_cast<uint64_t>(1024u >> 4) << 32;   // next 8 rows of K
+    d |= static_cast<uint64_t>(1u) << 46;
+    d |= static_cast<uint64_t>(2u) << 61;
+    return d;
+}
+
 __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
     const unsigned long long t0 = global_timer_ns();
     while (!mbar_try_wait(bar, parity)) {
@@ -133,7 +160,7 @@ __device__ __forceinline__ void short_pause_ns(unsigned long long ns) {
     }
 }
 
-template <int EPI>
+template <int EPI, int BOP = kBKMajor>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                              const __grid_constant__ CUtensorMap tmB0,
@@ -171,7 +198,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB0);
-        if (EPI == kEpiSwiGLU) tma_prefetch_desc(&tmB1);
+        if (EPI != kEpiStoreF32 || BOP == kBMnSplit) tma_prefetch_desc(&tmB1);
     }
     if (warp == 1) tmem_alloc_pair(&bk.tmem_base, kTmemCols);
 
@@ -209,12 +236,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t phase = 0;
             uint32_t pending = 0, pending_phase = 0;
             bool ok = true, issued = false;
-            const CUtensorMap* tmB = (EPI == kEpiSwiGLU && !leader) ? &tmB1 : &tmB0;
+            constexpr bool kStacked = EPI != kEpiStoreF32;  // B = [W1 rows | W3 rows]
+            const CUtensorMap* tmB = (kStacked && !leader) ? &tmB1 : &tmB0;
             for (int tile = pair; ok && tile < total; tile += npairs) {
                 const PairTile t = decode_pair_tile(bk, E, tile);
                 const int a_row = t.row0 + static_cast<int>(rank) * (t.half ? 64 : kRowsPerCta);
-                const int b_row = t.e * args.b_rows + t.nt * (EPI == kEpiSwiGLU ? 128 : 256) +
-                                  (EPI == kEpiSwiGLU ? 0 : static_cast<int>(rank) * 128);
+                const int b_row = t.e * args.b_rows + t.nt * (kStacked ? 128 : 256) +
+                                  (kStacked ? 0 : static_cast<int>(rank) * 128);
+                const int b_col = t.nt * 256 + static_cast<int>(rank) * 128;  // MN-major B
                 for (int kb = 0; kb < num_kb; ++kb) {
                     if (!mbar_wait_bounded(&bk.empty[stage], phase ^ 1u, abort_flag,
                                            args.status)) {
@@ -225,7 +254,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (leader) mbar_arrive_expect_tx(&bk.full[stage], 2 * kStageBytes);
                     const int kc = kb * kBK;
                     tma_load_2d_pair(&tmA, full_leader, sA + stage * kABytes, kc, a_row);
-                    tma_load_2d_pair(tmB, full_leader, sB + stage * kBBytes, kc, b_row);
+                    if (BOP == kBKMajor) {
+                        tma_load_2d_pair(tmB, full_leader, sB + stage * kBBytes, kc, b_row);
+                    } else {
+                        const CUtensorMap* mb = &tmB0;
+                        int krow = t.e * args.b_rows + kc;
+                        if (BOP == kBMnSplit) {
+                            const bool second = kc >= args.h;
+                            mb = second ? &tmB1 : &tmB0;
+                            krow = t.e * args.h + (second ? kc - args.h : kc);
+                        }
+                        tma_load_2d_pair(mb, full_leader, sB + stage * kBBytes, b_col, krow);
+                        tma_load_2d_pair(mb, full_leader, sB + stage * kBBytes + kBoxMn,
+                                         b_col + 64, krow);
+                    }
                     issued = true;
                     pending |= 1u << stage;
                     pending_phase = (pending_phase & ~(1u << stage)) | (phase << stage);
@@ -255,7 +297,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             bool ok = true, issued = false;
             for (int tile = pair; ok && tile < total; tile += npairs) {
                 const PairTile t = decode_pair_tile(bk, E, tile);
-                const uint32_t idesc = t.half ? kIdescHalf : kIdescFull;
+                constexpr uint32_t kBT = BOP == kBKMajor ? 0u : (1u << 16);  // B MN-major
+                const uint32_t idesc = (t.half ? kIdescHalf : kIdescFull) | kBT;
                 if (!mbar_wait_bounded(&bk.tmem_empty[acc], acc_phase ^ 1u, abort_flag,
                                        args.status)) {
                     ok = false;
@@ -270,10 +313,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     tc_fence_after();
                     const uint64_t ad = sw128_kmajor_desc(smem_u32(sA + stage * kABytes));
-                    const uint64_t bd = sw128_kmajor_desc(smem_u32(sB + stage * kBBytes));
+                    const uint32_t bs = smem_u32(sB + stage * kBBytes);
+                    const uint64_t bd = BOP == kBKMajor ? sw128_kmajor_desc(bs) : sw128_mn_desc_pair(bs);
+                    constexpr uint64_t kBStep = BOP == kBKMajor ? 2 : (16 * 128) >> 4;
 #pragma unroll
                     for (int k = 0; k < kBK / 16; ++k)
-                        umma_bf16_pair(d_tmem, ad + 2 * k, bd + 2 * k, idesc, (kb | k) != 0);
+                        umma_bf16_pair(d_tmem, ad + 2 * k, bd + kBStep * k, idesc, (kb | k) != 0);
                     umma_commit_pair(&bk.empty[stage], kBothCtas);
                     issued = true;
                     if (++stage == kStages) {
@@ -332,6 +377,49 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 if (col < args.N)
                                     *reinterpret_cast<uint4*>(out + col) =
                                         make_uint4(p[4 * v], p[4 * v + 1], p[4 * v + 2], p[4 * v + 3]);
+                            }
+                        }
+                    }
+                } else if (EPI == kEpiBwdSwiGLU) {
+                    // du, dv for this row's 128 outputs (N = h is a multiple of 64)
+                    const int N = args.N;
+                    __nv_bfloat16* duv =
+                        static_cast<__nv_bfloat16*>(args.out) + static_cast<size_t>(row) * 2 * N;
+                    const float* g = args.dH + static_cast<size_t>(row) * N;
+                    const int col0 = t.nt * 128;
+#pragma unroll 1
+                    for (int ch = 0; ch < 4; ++ch) {
+                        uint32_t a[32], b[32];
+                        tmem_ld_32cols(tlane + ch * 32, a);
+                        tmem_ld_32cols(tlane + 128 + ch * 32, b);
+                        tmem_ld_wait();
+                        const int c0 = col0 + ch * 32;
+                        if (valid && c0 < N) {
+                            float gv[32];
+#pragma unroll
+                            for (int v = 0; v < 8; ++v) {
+                                const float4 t4 = *reinterpret_cast<const float4*>(g + c0 + 4 * v);
+                                gv[4 * v] = t4.x;
+                                gv[4 * v + 1] = t4.y;
+                                gv[4 * v + 2] = t4.z;
+                                gv[4 * v + 3] = t4.w;
+                            }
+                            uint32_t pu[16], pv[16];
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) {
+                                float u0, v0, u1, v1;
+                                bwd_swiglu(bits_f32(a[2 * i]), bits_f32(b[2 * i]), gv[2 * i], u0, v0);
+                                bwd_swiglu(bits_f32(a[2 * i + 1]), bits_f32(b[2 * i + 1]),
+                                           gv[2 * i + 1], u1, v1);
+                                pu[i] = pack_bf16x2(u0, u1);
+                                pv[i] = pack_bf16x2(v0, v1);
+                            }
+#pragma unroll
+                            for (int v = 0; v < 4; ++v) {
+                                *reinterpret_cast<uint4*>(duv + c0 + 8 * v) =
+                                    make_uint4(pu[4 * v], pu[4 * v + 1], pu[4 * v + 2], pu[4 * v + 3]);
+                                *reinterpret_cast<uint4*>(duv + N + c0 + 8 * v) =
+                                    make_uint4(pv[4 * v], pv[4 * v + 1], pv[4 * v + 2], pv[4 * v + 3]);
                             }
                         }
                     }
@@ -395,6 +483,47 @@ __global__ void __launch_bounds__(kThreads, 1)
                         asm volatile("bar.sync %0, %1;" ::"r"(kXferBarrier), "r"(kEpiThreads)
                                      : "memory");
                     }
+                } else if (EPI == kEpiBwdSwiGLU) {
+                    const int N = args.N;
+                    __nv_bfloat16* duv =
+                        static_cast<__nv_bfloat16*>(args.out) + static_cast<size_t>(row) * 2 * N;
+                    const float* g = args.dH + static_cast<size_t>(row) * N;
+                    const int col0 = t.nt * 128;
+#pragma unroll 1
+                    for (int ch = 0; ch < 4; ++ch) {
+                        uint32_t v[32];
+                        tmem_ld_32cols(tlane + ch * 32, v);
+                        tmem_ld_wait();
+                        if (upper) {  // b for rows m, columns ch*32 .. ch*32+31
+#pragma unroll
+                            for (int j = 0; j < 32; ++j) xfer[j * 64 + m] = bits_f32(v[j]);
+                        }
+                        asm volatile("bar.sync %0, %1;" ::"r"(kXferBarrier), "r"(kEpiThreads)
+                                     : "memory");
+                        const int c0 = col0 + ch * 32;
+                        if (!upper && valid && c0 < N) {
+                            uint32_t pu[16], pv[16];
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) {
+                                float u0, v0, u1, v1;
+                                bwd_swiglu(bits_f32(v[2 * i]), xfer[(2 * i) * 64 + m],
+                                           g[c0 + 2 * i], u0, v0);
+                                bwd_swiglu(bits_f32(v[2 * i + 1]), xfer[(2 * i + 1) * 64 + m],
+                                           g[c0 + 2 * i + 1], u1, v1);
+                                pu[i] = pack_bf16x2(u0, u1);
+                                pv[i] = pack_bf16x2(v0, v1);
+                            }
+#pragma unroll
+                            for (int u = 0; u < 4; ++u) {
+                                *reinterpret_cast<uint4*>(duv + c0 + 8 * u) =
+                                    make_uint4(pu[4 * u], pu[4 * u + 1], pu[4 * u + 2], pu[4 * u + 3]);
+                                *reinterpret_cast<uint4*>(duv + N + c0 + 8 * u) =
+                                    make_uint4(pv[4 * u], pv[4 * u + 1], pv[4 * u + 2], pv[4 * u + 3]);
+                            }
+                        }
+                        asm volatile("bar.sync %0, %1;" ::"r"(kXferBarrier), "r"(kEpiThreads)
+                                     : "memory");
+                    }
                 } else {
                     float* out = static_cast<float*>(args.out) + static_cast<size_t>(row) * args.N;
                     const int col0 = t.nt * 256 + (upper ? 128 : 0);
@@ -432,10 +561,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-template <int EPI>
+template <int EPI, int BOP = kBKMajor>
 cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
                         const PairArgs& args, int npairs, cudaStream_t s) {
-    auto kern = grouped_gemm_pair_kernel<EPI>;
+    auto kern = grouped_gemm_pair_kernel<EPI, BOP>;
     static int configured[64] = {0};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -485,6 +614,32 @@ cudaError_t launch_ffn_bf16_pair(const void* x_perm, const int32_t* offsets, con
     long long t2 = blocks * g2.n_tiles;
     return launch_pair<kEpiStoreF32>(
         mh, mw2, mw2, g2, static_cast<int>(t2 < max_pairs ? (t2 < 1 ? 1 : t2) : max_pairs), s);
+}
+
+// Backward row-grouped GEMMs on CTA pairs (the backward pass is described in
+// backward_sm100.cu): mode 0  dH = dY W2_e (B = W2 read MN-major), fp32 [rows, h];
+// mode 1  du, dv from a = x W1_e^T, b = x W3_e^T and dH (B = [W1 | W3] rows, as GEMM1),
+// bf16 [rows, 2h]; mode 2  dX = [du dv] [W1_e; W3_e] (B MN-major, W1 for k < h, then
+// W3), fp32 [rows, d].  A maps have 128-row boxes, MN-major B maps 64 x 64 boxes.
+cudaError_t launch_bwd_rows_pair(int mode, const CUtensorMap& a, const CUtensorMap& b0,
+                                 const CUtensorMap& b1, const int32_t* offsets, int E, int rows,
+                                 int d, int h, void* out, const float* dH, uint32_t* status,
+                                 int cap, cudaStream_t s) {
+    const int max_pairs = device_sm_count() / 2;
+    const long long blocks = (static_cast<long long>(rows) + (kPairRows - 1LL) * E) / kPairRows;
+    auto grid = [&](long long tiles) {
+        return static_cast<int>(tiles < max_pairs ? (tiles < 1 ? 1 : tiles) : max_pairs);
+    };
+    if (mode == 0) {
+        PairArgs g{offsets, E, rows, d, h, d, (h + 255) / 256, out, status, cap, h, nullptr};
+        return launch_pair<kEpiStoreF32, kBMn>(a, b0, b0, g, grid(blocks * g.n_tiles), s);
+    }
+    if (mode == 1) {
+        PairArgs g{offsets, E, rows, d, h, h, (h + 127) / 128, out, status, cap, h, dH};
+        return launch_pair<kEpiBwdSwiGLU, kBKMajor>(a, b0, b1, g, grid(blocks * g.n_tiles), s);
+    }
+    PairArgs g{offsets, E, rows, 2 * h, d, h, (d + 255) / 256, out, status, cap, h, nullptr};
+    return launch_pair<kEpiStoreF32, kBMnSplit>(a, b0, b1, g, grid(blocks * g.n_tiles), s);
 }
 
 }  // namespace moe
