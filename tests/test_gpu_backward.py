@@ -177,3 +177,16 @@ def test_backward_full_size_sampled(workload):
         row = f64(g[name][e, r_])
         scale = np.linalg.norm(row) / np.sqrt(row.size) + 1e-30
         assert abs(got - v) <= BWD_TOL * max(abs(v), scale), (key, got, v)
+
+
+@pytest.mark.parametrize("T,E", [(40, 4), (300, 16), (1200, 2)])
+def test_backward_other_expert_counts(T, E):
+    wl = small("bwe", T=T, d=128, h=192, E=E, seed=E * 100 + T)
+    inp = make_inputs(wl, "cuda")
+    dy = seeded_dy(T, 128, 3 + T)
+    g, _ = gpu_grads(inp, dy)
+    c = {k: f64(v) for k, v in inp.items()}
+    ref = O.moe_layer_backward(c["x"], c["Wg"], c["W1"], c["W3"], c["W2"], f64(dy))
+    for k in ("dx", "dW1", "dW3", "dW2"):
+        assert rel_fro(f64(g[k]), ref[k]) <= BWD_TOL, k
+    assert rel_fro(f64(g["dWg"]), ref["dWg"]) <= ROUTER_TOL
