@@ -446,13 +446,24 @@ def run_ours(args):
 BWD_METRIC = "MoE-layer backward tokens/s (dx, dW1, dW3, dW2, dWg) and % of bf16 TC peak"
 BWD_STAGES = ["prep (dY, dw, dlogits)", "dH = dY W2", "du, dv (recompute a, b)",
               "dX = [du dv][W1; W3]", "dx combine", "dW2", "dW1 + dW3", "dWg"]
-BWD_KERNELS = {  # stage index -> (kernel, profile tag, flops per launch as a function)
-    1: ("bwd_rows_kernel<kModeDH>", "bwd_dh"),
-    2: ("bwd_rows_kernel<kModeDUV>", "bwd_duv"),
-    3: ("bwd_rows_kernel<kModeDX>", "bwd_dx"),
-    5: ("bwd_wgrad_kernel<kModeW2>", "bwd_wgrad_w2"),
-    6: ("bwd_wgrad_kernel<kModeW13>", "bwd_wgrad_w13"),
-}
+BWD_KERNELS = (1, 2, 3, 5, 6)  # the tensor-core stages
+BWD_PAIR_MIN_ROWS = 2048      # row GEMMs on CTA pairs from here (grouped rows)
+BWD_WGRAD_SHORT_ROWS = 1024   # weight gradients on single SMs up to here
+
+
+def backward_kernel(wl, stage: int):
+    """(kernel name, profile tag) of a backward GEMM stage for this workload."""
+    P = wl.T * wl.k
+    if stage in (5, 6):
+        single = P <= BWD_WGRAD_SHORT_ROWS
+        name = ("bwd_wgrad_kernel<%s>" % ("kModeW2" if stage == 5 else "kModeW13") if single
+                else "bwd_wgrad_pair_kernel")
+        return name, "bwd_wgrad_w2" if stage == 5 else "bwd_wgrad_w13"
+    pair = P >= BWD_PAIR_MIN_ROWS
+    names = {1: ("grouped_gemm_pair_kernel<StoreF32, B MN-major>", "bwd_rows_kernel<kModeDH>"),
+             2: ("grouped_gemm_pair_kernel<BwdSwiGLU>", "bwd_rows_kernel<kModeDUV>"),
+             3: ("grouped_gemm_pair_kernel<StoreF32, B MN-major split>", "bwd_rows_kernel<kModeDX>")}
+    return names[stage][0 if pair else 1], {1: "bwd_dh", 2: "bwd_duv", 3: "bwd_dx"}[stage]
 
 
 def backward_stage_flops(wl):
@@ -538,7 +549,7 @@ def run_ours_backward(args):
              for j in range(nst - 1)]
     flops = backward_stage_flops(wl)
     dom = max(BWD_KERNELS, key=lambda j: st_ms[j])
-    kname, tag = BWD_KERNELS[dom]
+    kname, tag = backward_kernel(wl, dom)
     peaks, peak_src = load_peaks()
     if T <= DECODE_MAX_TOKENS and dom in (5, 6):
         # a few rows per expert: the weight-gradient GEMMs are bound by writing their
@@ -550,7 +561,9 @@ def run_ours_backward(args):
         bound, unit, peak_kind = "tensor", "TFLOP/s", "burst"
         ach = flops[dom] / (st_ms[dom] * 1e-3) / 1e12
         peak = float(peaks["bf16_tflops"])
-    src = os.path.join(CSRC, "backward_sm100.cu")
+    src = os.path.join(CSRC, "backward_pair_sm100.cu" if "pair" in kname else "backward_sm100.cu")
+    if dom in (1, 2, 3) and "pair" in kname:
+        src = os.path.join(CSRC, "grouped_gemm_pair_sm100.cu")
     traffic, traffic_note = ncu_traffic(tag, wl.name, src), None
     if traffic is None and wl.name == "prefill" and dom in (5, 6):
         # The full backward holds ~10 GB, too much for a --set full capture: scale the
