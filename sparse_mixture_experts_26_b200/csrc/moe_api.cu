@@ -5,6 +5,7 @@
 // diagnostic moe_device_status and the opt-in MOE_DEBUG_SYNC=1 mode, which
 // synchronises after every launch and reports device-side flags).
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <cstdlib>
 #include <cstring>
@@ -63,6 +64,15 @@ bool debug_sync_enabled() {
 }
 
 namespace {
+
+// NVTX range around the host-side work of one stage (shows up in nsys / ncu timelines;
+// free when no tool is attached).
+struct NvtxRange {
+    explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange&) = delete;
+    NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -257,31 +267,45 @@ moe_status layer_forward_impl(const void* x, const void* Wg, const void* W1, con
         return i >= n_ev || ev[i] == nullptr || cudaEventRecord(ev[i], stream) == cudaSuccess;
     };
 
+    NvtxRange layer_range("moe_layer_forward");
     if (!mark(0)) return MOE_ERR_CUDA;
-    cudaError_t err = launch_route(x, Wg, T, d, E, dt, idx, w, stream);
+    cudaError_t err;
+    {
+        NvtxRange r("route");
+        err = launch_route(x, Wg, T, d, E, dt, idx, w, stream);
+    }
     if ((st = finish(err, stream, status)) != MOE_OK) return st;
-    err = launch_permute(idx, x, T, d, E, dt, offsets, perm_token, inv_perm, x_perm,
-                         at<int32_t>(ws, L.blk_counts), at<int32_t>(ws, L.blk_base), status,
-                         stream);
+    {
+        NvtxRange r("permute");
+        err = launch_permute(idx, x, T, d, E, dt, offsets, perm_token, inv_perm, x_perm,
+                             at<int32_t>(ws, L.blk_counts), at<int32_t>(ws, L.blk_base), status,
+                             stream);
+    }
     if ((st = finish(err, stream, status)) != MOE_OK) return st;
     if (!mark(1)) return MOE_ERR_CUDA;
     FfnOut fo{Y, 1};
-    if (dt == MOE_BF16) {
-        err = launch_ffn_bf16(x_perm, offsets, W1, W3, W2, P, d, h, E, at<void>(ws, L.H), Y,
-                              at<float>(ws, L.Ypart), kDecodeSplitK, /*reduce=*/false, &fo,
-                              status, stream, n_ev > 2 ? ev[2] : nullptr,
-                              at<uint32_t>(ws, L.sync), cap);
-        if (err == cudaErrorInvalidValue) return MOE_ERR_INVALID_ARG;
-    } else {
-        err = launch_ffn_f32(static_cast<const float*>(x_perm), offsets,
-                             static_cast<const float*>(W1), static_cast<const float*>(W3),
-                             static_cast<const float*>(W2), P, d, h, E, at<float>(ws, L.H), Y,
-                             stream, n_ev > 2 ? ev[2] : nullptr, cap);
+    {
+        NvtxRange r("expert_ffn");
+        if (dt == MOE_BF16) {
+            err = launch_ffn_bf16(x_perm, offsets, W1, W3, W2, P, d, h, E, at<void>(ws, L.H), Y,
+                                  at<float>(ws, L.Ypart), kDecodeSplitK, /*reduce=*/false, &fo,
+                                  status, stream, n_ev > 2 ? ev[2] : nullptr,
+                                  at<uint32_t>(ws, L.sync), cap);
+            if (err == cudaErrorInvalidValue) return MOE_ERR_INVALID_ARG;
+        } else {
+            err = launch_ffn_f32(static_cast<const float*>(x_perm), offsets,
+                                 static_cast<const float*>(W1), static_cast<const float*>(W3),
+                                 static_cast<const float*>(W2), P, d, h, E, at<float>(ws, L.H),
+                                 Y, stream, n_ev > 2 ? ev[2] : nullptr, cap);
+        }
     }
     if ((st = finish(err, stream, status)) != MOE_OK) return st;
     if (!mark(3)) return MOE_ERR_CUDA;
-    err = launch_combine(fo.Y, fo.nsplit, static_cast<size_t>(P) * d, inv_perm, w, T, d, dt, y,
-                         stream, idx, offsets, E, cap);
+    {
+        NvtxRange r("combine");
+        err = launch_combine(fo.Y, fo.nsplit, static_cast<size_t>(P) * d, inv_perm, w, T, d, dt,
+                             y, stream, idx, offsets, E, cap);
+    }
     if ((st = finish(err, stream, status)) != MOE_OK) return st;
     if (!mark(4)) return MOE_ERR_CUDA;
     return MOE_OK;
@@ -383,6 +407,7 @@ moe_status layer_backward_impl(const void* x, const void* Wg, const void* W1, co
     a.ev = ev;
     a.n_ev = n_ev;
     PdlScope pdl(false);  // the backward kernels do not wait on griddepcontrol
+    NvtxRange range("moe_layer_backward");
     cudaError_t err = launch_layer_backward(a, stream);
     if (err == cudaErrorInvalidValue) return MOE_ERR_INVALID_ARG;  // tensor map refused
     return finish(err, stream, a.status);
