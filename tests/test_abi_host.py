@@ -119,3 +119,49 @@ def test_status_strings(lib):
     for code in range(6):
         assert lib.moe_status_string(code)
     assert b"unknown" in lib.moe_status_string(99)
+
+
+def _bind_backward(lib):
+    vp, i32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    lib.moe_backward_workspace_bytes.restype = sz
+    lib.moe_backward_workspace_bytes.argtypes = [i32] * 6
+    args = [vp] * 6 + [i32] * 7 + [vp] * 6 + [sz, vp, sz]
+    lib.moe_layer_backward.argtypes = args + [vp]
+    lib.moe_layer_backward_events.argtypes = args + [vp, i32, vp]
+    return lib
+
+
+def test_backward_workspace_sizes(lib):
+    L = _bind_backward(lib)
+    d, h = 4096, 14336
+    n = L.moe_backward_workspace_bytes(4096, d, h, 8, 2, BF16)
+    P = 2 * 4096
+    # dY (bf16), dH (fp32), [du dv] (bf16) and dX (fp32) at least
+    assert n >= P * d * 2 + P * h * 4 + P * 2 * h * 2 + P * d * 4
+    assert n % 1024 == 0
+    assert L.moe_backward_workspace_bytes(16, d, h, 8, 2, F32) == 0      # bf16 only
+    assert L.moe_backward_workspace_bytes(16, d, 14344, 8, 2, BF16) == 0  # h % 64
+    assert L.moe_backward_workspace_bytes(16, d, h, 8, 3, BF16) == 0      # k != 2
+
+
+def test_backward_validation(lib):
+    L = _bind_backward(lib)
+    p = FAKE
+    T, d, h, E = 8, 64, 128, 8
+    fw = lib.moe_workspace_bytes(T, d, h, E, 2, BF16)
+    bw = L.moe_backward_workspace_bytes(T, d, h, E, 2, BF16)
+
+    def call(*, x=p, dy=p, dW2=p, h_=h, dt=BF16, k=2, fws=fw, bws=bw, T_=T):
+        return L.moe_layer_backward(x, p, p, p, p, dy, T_, d, h_, E, k, dt, -1, p, p, p, p, dW2,
+                                    p, fws, p, bws, None)
+    assert call(fws=fw - 1) == WORKSPACE
+    assert call(bws=bw - 1) == WORKSPACE
+    assert call(dy=None) == INVALID
+    assert call(dW2=p + 4) == INVALID          # misaligned
+    assert call(h_=96) == UNSUPPORTED           # h % 64 != 0
+    assert call(dt=F32) == UNSUPPORTED
+    assert call(k=3) == UNSUPPORTED
+    assert call(T_=0, x=None, dy=None) == OK    # empty batch: nothing to do
+    # the events variant checks its event array too
+    assert L.moe_layer_backward_events(p, p, p, p, p, p, T, d, h, E, 2, BF16, -1, p, p, p, p,
+                                       p, p, fw, p, bw, None, 3, None) == INVALID
