@@ -44,7 +44,7 @@ constexpr int kRows = 128;                  // output rows per CTA (TMEM lanes)
 constexpr int kBK = 64;                     // K rows per stage
 constexpr int kN = 256;                     // output columns per tile
 constexpr int kStages = 6;
-constexpr int kBox = 64 * 128;              // one 64-column x 64-row bf16 box: 8 KiB
+constexpr int kBox = kMnBoxBytes;           // one 64-column x 64-row bf16 box: 8 KiB
 constexpr int kABytes = 2 * kBox;           // this CTA's 128 columns of A
 constexpr int kBBytes = 2 * kBox;           // this CTA's 128 columns of B
 constexpr int kStageBytes = kABytes + kBBytes;
@@ -58,19 +58,8 @@ constexpr int kSmemBytes = kStages * kStageBytes + 4 * kOutBufs * kStageOutBytes
 static_assert(kSmemBytes <= 232448, "shared memory");
 constexpr int kVoteBarrier = 2;
 constexpr uint16_t kBothCtas = 0x3;
-constexpr uint64_t kMnStep = (16 * 128) >> 4;  // descriptor step for K = 16 rows
-
-__device__ __forceinline__ uint64_t sw128_mn_desc(uint32_t saddr) {
-    uint64_t d = 0;
-    d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
-    d |= static_cast<uint64_t>(kBox >> 4) << 16;   // next 64-wide M/N group: one box on
-    d |= static_cast<uint64_t>(1024u >> 4) << 32;  // next 8 rows of K
-    d |= static_cast<uint64_t>(1u) << 46;
-    d |= static_cast<uint64_t>(2u) << 61;
-    return d;
-}
 // M = 256 (two CTAs), N = 256, both operands MN-major.
-constexpr uint32_t kIdesc = idesc_bf16_f32(2 * kRows, kN) | (1u << 15) | (1u << 16);
+constexpr uint32_t kIdesc = idesc_bf16_f32_major(2 * kRows, kN, true, true);
 
 struct Book {
     uint64_t landed[kStages];    // partial blocks: this CTA's loads are in shared memory
@@ -102,19 +91,6 @@ struct PArgs {
     int cap;
 };
 
-__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
-    const unsigned long long t0 = global_timer_ns();
-    while (!mbar_try_wait(bar, parity)) {
-        if (global_timer_ns() - t0 > kDrainTimeoutNs) break;
-    }
-}
-
-__device__ __forceinline__ void fence_proxy_async_smem() {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-__device__ __forceinline__ float bits_f32(uint32_t u) { return __uint_as_float(u); }
-
 // Bounded wait with cluster-scope acquire: pairs with the peer's cluster-scope release
 // arrive, so the peer's shared-memory writes before it are ordered before what follows.
 __device__ __forceinline__ bool wait_cluster_bounded(uint64_t* bar, uint32_t parity,
@@ -141,12 +117,6 @@ __device__ __forceinline__ bool wait_cluster_bounded(uint64_t* bar, uint32_t par
         }
     }
     return true;
-}
-
-__device__ __forceinline__ void short_pause_ns(unsigned long long ns) {
-    const unsigned long long t0 = global_timer_ns();
-    while (global_timer_ns() - t0 < ns) {
-    }
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -315,7 +285,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint64_t bd = sw128_mn_desc(smem_u32(sB + stage * kBBytes));
 #pragma unroll
                     for (int k = 0; k < kBK / 16; ++k)
-                        umma_bf16_pair(d_tmem, ad + kMnStep * k, bd + kMnStep * k, kIdesc,
+                        umma_bf16_pair(d_tmem, ad + kMnDescStep * k, bd + kMnDescStep * k, kIdesc,
                                        (kb | k) != 0);
                     umma_commit_pair(&bk.empty[stage], kBothCtas);
                     issued = true;

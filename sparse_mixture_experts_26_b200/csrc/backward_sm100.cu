@@ -75,32 +75,10 @@ constexpr int wgrad_smem_bytes() {
     return STAGES * kStageBytes + 4 * OUTBUFS * kStageOutBytes + 1024 /*align*/ + 1024 /*book*/;
 }
 constexpr int kVoteBarrier = 2;  // epilogue vote after a bounded wait
-constexpr int kBox = 64 * 128;             // one 64-column x 64-row box: 8 KiB
+constexpr int kBox = kMnBoxBytes;          // one 64-column x 64-row box: 8 KiB
 
 enum RowMode { kModeDH = 0, kModeDUV = 1, kModeDX = 2 };
 enum WMode { kModeW2 = 0, kModeW13 = 1 };
-
-// Shared-memory descriptor of an MN-major operand with 128-byte swizzle: each k is
-// one 128-byte row of 64 consecutive M/N elements; consecutive 64-element groups of
-// M/N are one box (kBox bytes) apart (leading byte offset), 8-row groups of k are
-// 1024 bytes apart (stride byte offset).  Version 1 (bit 46), swizzle mode 2.
-__device__ __forceinline__ uint64_t sw128_mn_desc(uint32_t saddr) {
-    uint64_t d = 0;
-    d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
-    d |= static_cast<uint64_t>(kBox >> 4) << 16;
-    d |= static_cast<uint64_t>(1024u >> 4) << 32;
-    d |= static_cast<uint64_t>(1u) << 46;
-    d |= static_cast<uint64_t>(2u) << 61;
-    return d;
-}
-// Descriptor step for K = 16: MN-major 16 rows of 128 bytes; K-major 32 bytes.
-constexpr uint64_t kMnStep = (16 * 128) >> 4;
-constexpr uint64_t kKStep = 32 >> 4;
-
-// bf16 x bf16 -> f32, M x N; transpose bits 15 (A) / 16 (B) select MN-major operands.
-__host__ __device__ constexpr uint32_t idesc_major(int M, int N, bool a_mn, bool b_mn) {
-    return idesc_bf16_f32(M, N) | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16);
-}
 
 struct Book {
     uint64_t full[kStages];
@@ -115,24 +93,6 @@ struct Book {
     int tile_start[kMaxExperts + 1];
 };
 static_assert(sizeof(Book) <= 1024, "bookkeeping reserve");
-
-__device__ __forceinline__ float bits_f32(uint32_t u) { return __uint_as_float(u); }
-
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<uint32_t*>(&v);
-}
-
-__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
-    const unsigned long long t0 = global_timer_ns();
-    while (!mbar_try_wait(bar, parity)) {
-        if (global_timer_ns() - t0 > kDrainTimeoutNs) break;
-    }
-}
-
-__device__ __forceinline__ void fence_proxy_async_smem() {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
 
 // Group offsets (clamped, monotone) and kept ends; thread 0 only.
 __device__ __forceinline__ void load_groups(Book& bk, const int32_t* offsets, int E, int rows,
@@ -192,7 +152,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bwd_rows_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                     const __grid_constant__ CUtensorMap tmB1, const RowArgs args) {
     constexpr bool kBmn = MODE != kModeDUV;
-    constexpr uint32_t kIdesc = idesc_major(kBM, kN, false, kBmn);
+    constexpr uint32_t kIdesc = idesc_bf16_f32_major(kBM, kN, false, kBmn);
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -309,7 +269,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint64_t bd = kBmn ? sw128_mn_desc(bs) : sw128_kmajor_desc(bs);
 #pragma unroll
                     for (int k = 0; k < kBK / 16; ++k)
-                        umma_bf16(d_tmem, ad + kKStep * k, bd + (kBmn ? kMnStep : kKStep) * k,
+                        umma_bf16(d_tmem, ad + kKDescStep * k, bd + (kBmn ? kMnDescStep : kKDescStep) * k,
                                   kIdesc, (kb | k) != 0);
                     umma_commit(&bk.empty[stage]);
                     issued = true;
@@ -468,7 +428,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bwd_wgrad_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmO0,
                      const __grid_constant__ CUtensorMap tmO1, const WArgs args) {
-    constexpr uint32_t kIdesc = idesc_major(kBM, kN, true, true);
+    constexpr uint32_t kIdesc = idesc_bf16_f32_major(kBM, kN, true, true);
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -592,7 +552,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint64_t bd = sw128_mn_desc(smem_u32(sB + stage * kBBytes));
 #pragma unroll
                     for (int k = 0; k < kBK / 16; ++k)
-                        umma_bf16(d_tmem, ad + kMnStep * k, bd + kMnStep * k, kIdesc,
+                        umma_bf16(d_tmem, ad + kMnDescStep * k, bd + kMnDescStep * k, kIdesc,
                                   (kb | k) != 0);
                     umma_commit(&bk.empty[stage]);
                 }

@@ -117,13 +117,6 @@ __device__ __forceinline__ Tile decode_tile(const DecodeBook<NACC>& bk, int E, i
     return t;
 }
 
-__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
-    const unsigned long long t0 = global_timer_ns();
-    while (!mbar_try_wait(bar, parity)) {
-        if (global_timer_ns() - t0 > kDrainTimeoutNs) break;
-    }
-}
-
 template <int NT>
 __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[NT]);
 
@@ -474,10 +467,6 @@ __device__ __forceinline__ FusedUnit fused_unit(const FusedBook<NACC>& bk, const
     const int left = bk.end[g] - f.row0;
     f.nvalid = left < NTc ? left : NTc;
     return f;
-}
-
-__device__ __forceinline__ void fence_proxy_async_global() {
-    asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
 template <int NT>

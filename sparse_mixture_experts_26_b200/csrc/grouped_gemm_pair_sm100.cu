@@ -69,7 +69,7 @@ enum Epilogue { kEpiSwiGLU = 0, kEpiStoreF32 = 1, kEpiBwdSwiGLU = 2 };
 // 64 x 64 boxes; backward dH = dY W2), optionally taken from W1 for k < h and from W3
 // for k >= h (backward dX = [du dv] [W1; W3]).
 enum BOperand { kBKMajor = 0, kBMn = 1, kBMnSplit = 2 };
-constexpr int kBoxMn = 64 * 128;  // one 64 x 64 bf16 box of an MN-major operand
+constexpr int kBoxMn = kMnBoxBytes;  // one 64 x 64 bf16 box of an MN-major operand
 
 struct PairArgs {
     const int32_t* offsets;
@@ -119,13 +119,6 @@ __device__ __forceinline__ PairTile decode_pair_tile(const PairBook& bk, int E, 
     return t;
 }
 
-__device__ __forceinline__ float bits_f32(uint32_t u) { return __uint_as_float(u); }
-
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<uint32_t*>(&v);
-}
-
 __device__ __forceinline__ float silu_mul(float a, float b) {
     return a / (1.0f + __expf(-a)) * b;
 }
@@ -135,29 +128,6 @@ __device__ __forceinline__ void bwd_swiglu(float a, float b, float g, float& du,
     const float s = 1.0f / (1.0f + __expf(-a));
     du = g * b * (s * (1.0f + a * (1.0f - s)));
     dv = g * (a * s);
-}
-
-__device__ __forceinline__ uint64_t sw128_mn_desc_pair(uint32_t saddr) {
-    uint64_t d = 0;
-    d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
-    d |= static_cast<uint64_t>(kBoxMn >> 4) << 16;  // next 64-wide group of N: one box on
-    d |= static_cast<uint64_t>(1024u >> 4) << 32;   // next 8 rows of K
-    d |= static_cast<uint64_t>(1u) << 46;
-    d |= static_cast<uint64_t>(2u) << 61;
-    return d;
-}
-
-__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
-    const unsigned long long t0 = global_timer_ns();
-    while (!mbar_try_wait(bar, parity)) {
-        if (global_timer_ns() - t0 > kDrainTimeoutNs) break;
-    }
-}
-
-__device__ __forceinline__ void short_pause_ns(unsigned long long ns) {
-    const unsigned long long t0 = global_timer_ns();
-    while (global_timer_ns() - t0 < ns) {
-    }
 }
 
 template <int EPI, int BOP = kBKMajor>
@@ -314,8 +284,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc_fence_after();
                     const uint64_t ad = sw128_kmajor_desc(smem_u32(sA + stage * kABytes));
                     const uint32_t bs = smem_u32(sB + stage * kBBytes);
-                    const uint64_t bd = BOP == kBKMajor ? sw128_kmajor_desc(bs) : sw128_mn_desc_pair(bs);
-                    constexpr uint64_t kBStep = BOP == kBKMajor ? 2 : (16 * 128) >> 4;
+                    const uint64_t bd = BOP == kBKMajor ? sw128_kmajor_desc(bs) : sw128_mn_desc(bs);
+                    constexpr uint64_t kBStep = BOP == kBKMajor ? kKDescStep : kMnDescStep;
 #pragma unroll
                     for (int k = 0; k < kBK / 16; ++k)
                         umma_bf16_pair(d_tmem, ad + 2 * k, bd + kBStep * k, idesc, (kb | k) != 0);

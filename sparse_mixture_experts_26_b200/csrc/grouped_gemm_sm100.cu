@@ -101,23 +101,8 @@ __device__ __forceinline__ TileCoord decode_tile(const Bookkeeping& bk, int E, i
     return c;
 }
 
-__device__ __forceinline__ float bits_f32(uint32_t u) { return __uint_as_float(u); }
-
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<uint32_t*>(&v);
-}
-
 __device__ __forceinline__ float silu_mul(float a, float b) {
     return a / (1.0f + __expf(-a)) * b;
-}
-
-// Bounded wait used only while tearing down after an abort.
-__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
-    const unsigned long long t0 = global_timer_ns();
-    while (!mbar_try_wait(bar, parity)) {
-        if (global_timer_ns() - t0 > kDrainTimeoutNs) break;
-    }
 }
 
 template <int EPI>

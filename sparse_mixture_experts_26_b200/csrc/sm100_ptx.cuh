@@ -6,6 +6,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cstdint>
 
 namespace moe {
@@ -79,6 +80,20 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
     }
 }
 
+// Bounded wait used only while tearing down after an abort (no flag, no status).
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
+    const unsigned long long t0 = global_timer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (global_timer_ns() - t0 > kDrainTimeoutNs) break;
+    }
+}
+
+__device__ __forceinline__ void short_pause_ns(unsigned long long ns) {
+    const unsigned long long t0 = global_timer_ns();
+    while (global_timer_ns() - t0 < ns) {
+    }
+}
+
 // True on every participating thread iff `v` is true on all `nthreads` threads
 // arriving at named barrier `id`.  Epilogue warps vote with it after a bounded wait,
 // so that all of them leave together when any one gave up (a later named barrier
@@ -118,6 +133,23 @@ __device__ __forceinline__ bool flag_wait_bounded(const uint32_t* counter, uint3
         }
     }
     return true;
+}
+
+// Order this thread's generic-proxy writes (shared / global memory) before later
+// async-proxy accesses (TMA, tcgen05.mma) that another thread starts after a barrier.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// ------------------------------------------------------------------ small numerics
+__device__ __forceinline__ float bits_f32(uint32_t u) { return __uint_as_float(u); }
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
 }
 
 // ------------------------------------------------------------------ TMA
@@ -222,6 +254,25 @@ __device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t saddr) {
     return d;
 }
 
+// Shared-memory descriptor of an MN-major operand with 128-byte swizzle: each k is one
+// 128-byte row of 64 consecutive M/N elements (a 64-column x 64-row TMA box holds 64
+// such rows); consecutive 64-element groups of M/N are one box (8 KiB) apart (leading
+// byte offset), 8-row groups of k are 1024 bytes apart (stride byte offset).
+constexpr uint32_t kMnBoxBytes = 64 * 128;
+__device__ __forceinline__ uint64_t sw128_mn_desc(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
+    d |= static_cast<uint64_t>(kMnBoxBytes >> 4) << 16;
+    d |= static_cast<uint64_t>(1024u >> 4) << 32;
+    d |= static_cast<uint64_t>(1u) << 46;
+    d |= static_cast<uint64_t>(2u) << 61;
+    return d;
+}
+// Descriptor steps for K = 16: an MN-major operand advances 16 rows of 128 bytes,
+// a K-major one 32 bytes.
+constexpr uint64_t kMnDescStep = (16 * 128) >> 4;
+constexpr uint64_t kKDescStep = 32 >> 4;
+
 // Instruction descriptor for kind::f16 with bf16 A and B, fp32 accumulator, both
 // operands K-major, shape M x N (PTX ISA, tcgen05 "instruction descriptor"):
 // D format in bits 4-5 (1 = f32), A format 7-9 and B format 10-12 (1 = bf16),
@@ -229,6 +280,10 @@ __device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t saddr) {
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
     return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
            (static_cast<uint32_t>(M >> 4) << 24);
+}
+// The same with either operand MN-major (transpose bits 15 for A, 16 for B).
+__host__ __device__ constexpr uint32_t idesc_bf16_f32_major(int M, int N, bool a_mn, bool b_mn) {
+    return idesc_bf16_f32(M, N) | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16);
 }
 
 // D[tmem] (+)= A[smem] * B[smem]^T for one K=16 slice; issued by one thread.
