@@ -25,8 +25,9 @@
  *   moe_device_status().
  * - dtype: MOE_BF16 (bfloat16 activations and weights, fp32 accumulation on tensor
  *   cores) or MOE_F32 (fp32 everywhere, CUDA cores, no TF32).
- * - Supported shapes: k == 2; 2 <= E <= 32; d and h multiples of 8; T >= 0
- *   (T == 0 is a no-op returning MOE_OK).  Inputs must be finite.
+ * - Supported shapes: k == 2; 2 <= E <= 32 (moe_expert_ffn, which routes nothing,
+ *   also takes E == 1); d and h multiples of 8; T >= 0 (T == 0 is a no-op returning
+ *   MOE_OK).  Inputs must be finite.
  * - Routing: experts are ranked by (logit descending, index ascending), so ties go
  *   to the lower index; logits are accumulated in fp64 from the exact products of
  *   the inputs.  Slot 0 holds the larger logit.  w1 = 1/(1+exp(l_i2-l_i1)) is
@@ -106,7 +107,10 @@ moe_status moe_permute(const int32_t *topk_idx, const void *x, int T, int d, int
  *   y_perm  [rows, d]   float out    Y_r = W2[e](silu(W1[e] x_r) * W3[e] x_r)
  *   ws, ws_bytes                      workspace (holds H [rows, h])
  * bf16 runs on tcgen05 tensor cores (fp32 accumulation in tensor memory; H is
- * rounded once to bf16); f32 runs on CUDA cores in fp32. */
+ * rounded once to bf16); f32 runs on CUDA cores in fp32.  rows must be even (pad with
+ * a row outside every group; output rows outside every group are unspecified);
+ * 1 <= E <= 32.  ws_bytes: at least moe_workspace_bytes(rows / 2, d, h, max(E, 2), 2,
+ * dt). */
 moe_status moe_expert_ffn(const void *x_perm, const int32_t *offsets, const void *W1,
                           const void *W3, const void *W2, int rows, int d, int h,
                           int E, moe_dtype dt, float *y_perm, void *ws,

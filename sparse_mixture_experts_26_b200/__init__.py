@@ -133,6 +133,12 @@ def moe_workspace_bytes(T: int, d: int, h: int, E: int = 8, k: int = 2,
     return int(_lib.moe_workspace_bytes(T, d, h, E, k, dt))
 
 
+def moe_expert_ffn_workspace_bytes(rows: int, d: int, h: int, E: int,
+                                   dtype: torch.dtype = torch.bfloat16) -> int:
+    """Workspace bytes moe_expert_ffn needs for `rows` (even) grouped rows of E experts."""
+    return moe_workspace_bytes(max(rows // 2, 1), d, h, max(E, 2), 2, dtype)
+
+
 def alloc_workspace(T: int, d: int, h: int, E: int = 8, k: int = 2,
                     dtype: torch.dtype = torch.bfloat16, device="cuda") -> torch.Tensor:
     """A zeroed workspace of ``moe_workspace_bytes`` bytes (the status word starts at 0)."""

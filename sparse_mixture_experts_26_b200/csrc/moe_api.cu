@@ -76,10 +76,12 @@ struct NvtxRange {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-moe_status check_shape(int T, int d, int h, int E, int k, moe_dtype dt, bool need_h) {
+// routed = false: the expert FFN alone, which also takes a single expert.
+moe_status check_shape(int T, int d, int h, int E, int k, moe_dtype dt, bool need_h,
+                       bool routed = true) {
     if (T < 0 || d <= 0 || (need_h && h <= 0) || E <= 0 || k <= 0) return MOE_ERR_INVALID_ARG;
     if (dt != MOE_F32 && dt != MOE_BF16) return MOE_ERR_INVALID_ARG;
-    if (k != 2 || E < 2 || E > kMaxExperts) return MOE_ERR_UNSUPPORTED;
+    if (k != 2 || E < (routed ? 2 : 1) || E > kMaxExperts) return MOE_ERR_UNSUPPORTED;
     if (d % 8 != 0 || (need_h && h % 8 != 0)) return MOE_ERR_UNSUPPORTED;
     // 32-bit row indices and element offsets inside one grouped buffer.
     const long long P = 2LL * T;
@@ -202,7 +204,7 @@ moe_status moe_expert_ffn(const void* x_perm, const int32_t* offsets, const void
                           cudaStream_t stream) {
     if (rows < 0 || rows % 2 != 0) return MOE_ERR_INVALID_ARG;
     const int T = rows / 2;
-    moe_status st = check_shape(T, d, h, E, 2, dt, true);
+    moe_status st = check_shape(T, d, h, E, 2, dt, true, /*routed=*/false);
     if (st != MOE_OK) return st;
     if (rows == 0) return MOE_OK;
     if (!ptrs_ok({x_perm, offsets, W1, W3, W2, y_perm, ws})) return MOE_ERR_INVALID_ARG;
