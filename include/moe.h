@@ -64,11 +64,12 @@ typedef enum {
 
 /* Bytes of workspace that moe_layer_forward needs for this shape (a 1 KiB-aligned
  * layout of routing results, permutation, gathered rows x_perm, the SwiGLU
- * activations H, the fp32 expert outputs and, for batches of at most 64 tokens, the
+ * activations H, the fp32 expert outputs and, for batches of at most 128 tokens, the
  * fp32 partial sums of the split-K down projection).  It also covers moe_permute and
- * moe_expert_ffn.  Zero the workspace once before its first use: it holds a status
- * word and dependency counters that every call leaves at zero.  Returns 0 for
- * unsupported arguments. */
+ * moe_expert_ffn.  The size never decreases with T: a workspace sized for T serves
+ * every batch of at most T tokens (same d, h, E, k, dt).  Zero the workspace once
+ * before its first use: it holds a status word and dependency counters that every
+ * call leaves at zero.  Returns 0 for unsupported arguments. */
 size_t moe_workspace_bytes(int T, int d, int h, int E, int k, moe_dtype dt);
 
 /* Router + top-2 + softmax of the two kept logits.

@@ -667,16 +667,21 @@ __device__ __forceinline__ bool pair_kept(const int32_t* idx, const int32_t* off
 }
 
 // One block per token: dY rows of its two pairs, dw, and the token's logit gradients.
-// Y is the sum of nsplit fp32 arrays split_stride floats apart (in order).
+// The forward left its expert outputs either in Y or as split-K partials in Ypart
+// (split_stride floats apart, summed in order); the byte at y_layout says which.
 __global__ void __launch_bounds__(kPrepThreads)
     bwd_prep_kernel(const __nv_bfloat16* __restrict__ dy, const int32_t* __restrict__ idx,
                     const float* __restrict__ w, const int32_t* __restrict__ inv,
                     const int32_t* __restrict__ offsets, int T, int d, int E, int cap,
-                    const float* __restrict__ Y, int nsplit, size_t split_stride,
+                    const float* __restrict__ Y1, const float* __restrict__ Ypart,
+                    const uint8_t* __restrict__ y_layout, size_t split_stride,
                     __nv_bfloat16* __restrict__ dY, float* __restrict__ dw,
                     float* __restrict__ dlogits) {
     __shared__ float red[2][kPrepThreads / 32];
     const int P = 2 * T;
+    int nsplit = *y_layout;
+    nsplit = nsplit < 1 ? 1 : (nsplit > kDecodeSplitK ? kDecodeSplitK : nsplit);
+    const float* __restrict__ Y = nsplit > 1 ? Ypart : Y1;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     for (int t = blockIdx.x; t < T; t += gridDim.x) {
         const bool keep0 = pair_kept(idx, offsets, inv, 2 * t, E, P, cap);
@@ -885,8 +890,8 @@ cudaError_t launch_layer_backward(const BwdArgs& a, cudaStream_t s) {
     // 1. dY, dw, dlogits
     err = launch_k(bwd_prep_kernel, grid_for(T, 8 * sms), kPrepThreads, 0, s,
                    static_cast<const __nv_bfloat16*>(a.dy), a.idx, a.w, a.inv, a.offsets, T, d, E,
-                   a.cap, a.Y, a.nsplit, a.split_stride, static_cast<__nv_bfloat16*>(a.dY), a.dw,
-                   a.dlogits);
+                   a.cap, a.Y, a.Ypart, a.y_layout, a.split_stride,
+                   static_cast<__nv_bfloat16*>(a.dY), a.dw, a.dlogits);
     if (err != cudaSuccess || (err = mark(1)) != cudaSuccess) return err;
 
     CUtensorMap m_dY128, m_W2, m_x, m_W1r, m_W3r, m_duv128, m_W1mn, m_W3mn;

@@ -48,9 +48,11 @@ __global__ void __launch_bounds__(kCombineThreads)
     combine_kernel(const float4* __restrict__ Y, int nsplit, size_t split_stride4,
                    const int32_t* __restrict__ inv, const float* __restrict__ w, int T, int d4,
                    Tout* __restrict__ y, const int32_t* __restrict__ idx,
-                   const int32_t* __restrict__ offsets, int E, int cap) {
+                   const int32_t* __restrict__ offsets, int E, int cap, uint8_t* layout_out) {
     pdl_wait();
     pdl_launch_dependents();
+    if (layout_out && blockIdx.x == 0 && threadIdx.x == 0)
+        *layout_out = static_cast<uint8_t>(nsplit);
     const size_t n = static_cast<size_t>(T) * d4;
     const unsigned P = 2u * static_cast<unsigned>(T);
     for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
@@ -116,17 +118,18 @@ cudaError_t launch_sum_splits(const float* parts, int nsplit, size_t n, float* Y
 cudaError_t launch_combine(const float* Y, int nsplit, size_t split_stride,
                            const int32_t* inv_perm, const float* w, int T, int d, moe_dtype dt,
                            void* y, cudaStream_t s, const int32_t* idx, const int32_t* offsets,
-                           int E, int cap) {
+                           int E, int cap, uint8_t* layout_out) {
     if (cap != INT_MAX && (!idx || !offsets)) return cudaErrorInvalidValue;
     const int d4 = d / 4;
     const unsigned blocks = grid_for(static_cast<size_t>(T) * d4);
     if (dt == MOE_BF16)
         return launch_k(combine_kernel<__nv_bfloat16>, blocks, kCombineThreads, 0, s,
                         reinterpret_cast<const float4*>(Y), nsplit, split_stride / 4, inv_perm,
-                        w, T, d4, static_cast<__nv_bfloat16*>(y), idx, offsets, E, cap);
+                        w, T, d4, static_cast<__nv_bfloat16*>(y), idx, offsets, E, cap,
+                        layout_out);
     return launch_k(combine_kernel<float>, blocks, kCombineThreads, 0, s,
                     reinterpret_cast<const float4*>(Y), nsplit, split_stride / 4, inv_perm, w, T,
-                    d4, static_cast<float*>(y), idx, offsets, E, cap);
+                    d4, static_cast<float*>(y), idx, offsets, E, cap, layout_out);
 }
 
 }  // namespace moe

@@ -43,7 +43,6 @@ constexpr int kBK = 64;          // one 128-byte swizzle span of bf16 along K
 constexpr int kM = 128;          // MMA rows = weight rows per tile
 constexpr int kThreads = 192;    // TMA warp, MMA warp, 4 epilogue warps
 constexpr int kEpiThreads = 128;
-constexpr uint32_t kTmemCols = 128;
 constexpr int kXferBarrier = 1;  // named barrier id for the epilogue exchange
 constexpr int kVoteBarrier = 2;  // epilogue vote after a bounded wait
 
@@ -70,13 +69,18 @@ struct DecodeCfg {
     static constexpr int kBStage = NT * 128;
     static constexpr int kStageTx = kAStage + kBStage;
     static constexpr int kStages = (200 * 1024) / (kAStage + kBStage);
+    // TMEM columns: 128 (8, 4 or 2 accumulators of 16, 32 or 64 token columns), or two
+    // accumulators of 128 token columns
+    static constexpr uint32_t kTmemCols = NT <= 64 ? 128 : 2 * NT;
     static constexpr int kAcc = kTmemCols / NT;  // accumulators in flight
-    static constexpr int kXferBytes = (MODE == kSwiGLU) ? kM * NT * 4 : 0;
+    // token columns the gate/up epilogue exchanges through shared memory at a time
+    static constexpr int kXferCols = NT <= 64 ? NT : 32;
+    static constexpr int kXferBytes = (MODE == kSwiGLU) ? kM * kXferCols * 4 : 0;
     static constexpr int kSmem =
         kStages * (kAStage + kBStage) + 1024 /*align*/ + 2048 /*bookkeeping*/ + kXferBytes;
     static constexpr uint32_t kIdesc = idesc_bf16_f32(kM, NT);
     static_assert(kBStage % 1024 == 0, "1 KiB-aligned stages");
-    static_assert(NT % 16 == 0 && NT >= 16 && NT <= 64, "N must be 16..64, multiple of 16");
+    static_assert(NT % 16 == 0 && NT >= 16 && NT <= 128, "N must be 16..128, multiple of 16");
     static_assert(kStages >= 4 && kStages <= 16, "stage count");
     static_assert(kSmem <= 232448, "shared memory");
 };
@@ -183,7 +187,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (MODE == kSwiGLU) tma_prefetch_desc(&tmW1);
         tma_prefetch_desc(&tmX);
     }
-    if (warp == 1) tmem_alloc(&bk.tmem_base, kTmemCols);
+    if (warp == 1) tmem_alloc(&bk.tmem_base, C::kTmemCols);
 
     pdl_wait();
     pdl_launch_dependents();
@@ -365,7 +369,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, kTmemCols);
+        tmem_dealloc(tmem_base, C::kTmemCols);
     }
 }
 
@@ -514,7 +518,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_prefetch_desc(&tmW2);
         tma_prefetch_desc(&tmH);
     }
-    if (warp == 1) tmem_alloc(&bk.tmem_base, kTmemCols);
+    if (warp == 1) tmem_alloc(&bk.tmem_base, C::kTmemCols);
 
     pdl_wait();
     pdl_launch_dependents();
@@ -664,47 +668,106 @@ __global__ void __launch_bounds__(kThreads, 1)
                          kVoteBarrier, kEpiThreads))
                 break;
             tc_fence_after();
-            uint32_t v[NT];
-            tmem_ld_cols<NT>(tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
-                                 static_cast<uint32_t>(acc * NT),
-                             v);
-            tmem_ld_wait();
-            tc_fence_before();
-            mbar_arrive(&bk.tmem_empty[acc]);
-            if (!f.down) {
+            const uint32_t tacc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                                  static_cast<uint32_t>(acc * NT);
+            if constexpr (NT <= 64) {
+                uint32_t v[NT];
+                tmem_ld_cols<NT>(tacc, v);
+                tmem_ld_wait();
+                tc_fence_before();
+                mbar_arrive(&bk.tmem_empty[acc]);
+                if (!f.down) {
 #pragma unroll
-                for (int c = 0; c < NT; ++c) xfer[c * kM + r] = __uint_as_float(v[c]);
-                asm volatile("bar.sync %0, %1;" ::"r"(kXferBarrier), "r"(kEpiThreads) : "memory");
-                if (r < J1) {
-                    const int col = f.blk * J1 + r;
-                    if (col < args.h) {
-                        __nv_bfloat16* out = static_cast<__nv_bfloat16*>(args.H);
+                    for (int c = 0; c < NT; ++c) xfer[c * kM + r] = __uint_as_float(v[c]);
+                    asm volatile("bar.sync %0, %1;" ::"r"(kXferBarrier), "r"(kEpiThreads) : "memory");
+                    if (r < J1) {
+                        const int col = f.blk * J1 + r;
+                        if (col < args.h) {
+                            __nv_bfloat16* out = static_cast<__nv_bfloat16*>(args.H);
 #pragma unroll
-                        for (int c = 0; c < NT; ++c) {
-                            if (c < f.nvalid) {
-                                const float a = xfer[c * kM + r];
-                                const float b = xfer[c * kM + J1 + r];
-                                out[static_cast<size_t>(f.row0 + c) * args.h + col] =
-                                    __float2bfloat16_rn(a / (1.0f + __expf(-a)) * b);
+                            for (int c = 0; c < NT; ++c) {
+                                if (c < f.nvalid) {
+                                    const float a = xfer[c * kM + r];
+                                    const float b = xfer[c * kM + J1 + r];
+                                    out[static_cast<size_t>(f.row0 + c) * args.h + col] =
+                                        __float2bfloat16_rn(a / (1.0f + __expf(-a)) * b);
+                                }
                             }
                         }
+                        __threadfence();  // H stores visible at device scope before the count
                     }
-                    __threadfence();  // H stores visible at device scope before the count
-                }
-                asm volatile("bar.sync %0, %1;" ::"r"(kXferBarrier), "r"(kEpiThreads) : "memory");
-                if (r == 0) {
-                    fence_proxy_async_global();
-                    atomicAdd(args.ready + f.e * args.ksplit + f.blk / kps, 1u);
+                    asm volatile("bar.sync %0, %1;" ::"r"(kXferBarrier), "r"(kEpiThreads) : "memory");
+                    if (r == 0) {
+                        fence_proxy_async_global();
+                        atomicAdd(args.ready + f.e * args.ksplit + f.blk / kps, 1u);
+                    }
+                } else {
+                    const int col = f.blk * kM + r;
+                    if (col < args.d) {
+                        float* out = args.Ypart + static_cast<size_t>(f.ks) * args.rows * args.d;
+#pragma unroll
+                        for (int c = 0; c < NT; ++c)
+                            if (c < f.nvalid)
+                                out[static_cast<size_t>(f.row0 + c) * args.d + col] =
+                                    __uint_as_float(v[c]);
+                    }
                 }
             } else {
-                const int col = f.blk * kM + r;
-                if (col < args.d) {
-                    float* out = args.Ypart + static_cast<size_t>(f.ks) * args.rows * args.d;
+                // 128 token columns: drain the accumulator 32 columns at a time (the
+                // exchange buffer holds 32 columns); chunks past the last row are skipped.
+                constexpr int kC = C::kXferCols;
+                if (!f.down) {
+                    for (int c0 = 0; c0 < NT && c0 < f.nvalid; c0 += kC) {
+                        uint32_t v[kC];
+                        tmem_ld_32cols(tacc + c0, v);
+                        tmem_ld_wait();
 #pragma unroll
-                    for (int c = 0; c < NT; ++c)
-                        if (c < f.nvalid)
-                            out[static_cast<size_t>(f.row0 + c) * args.d + col] =
-                                __uint_as_float(v[c]);
+                        for (int c = 0; c < kC; ++c) xfer[c * kM + r] = __uint_as_float(v[c]);
+                        asm volatile("bar.sync %0, %1;" ::"r"(kXferBarrier), "r"(kEpiThreads)
+                                     : "memory");
+                        if (r < J1) {
+                            const int col = f.blk * J1 + r;
+                            if (col < args.h) {
+                                __nv_bfloat16* out = static_cast<__nv_bfloat16*>(args.H);
+#pragma unroll
+                                for (int c = 0; c < kC; ++c) {
+                                    if (c0 + c < f.nvalid) {
+                                        const float a = xfer[c * kM + r];
+                                        const float b = xfer[c * kM + J1 + r];
+                                        out[static_cast<size_t>(f.row0 + c0 + c) * args.h + col] =
+                                            __float2bfloat16_rn(a / (1.0f + __expf(-a)) * b);
+                                    }
+                                }
+                            }
+                        }
+                        asm volatile("bar.sync %0, %1;" ::"r"(kXferBarrier), "r"(kEpiThreads)
+                                     : "memory");
+                    }
+                    tc_fence_before();
+                    mbar_arrive(&bk.tmem_empty[acc]);
+                    if (r < J1) __threadfence();  // H stores visible before the count
+                    asm volatile("bar.sync %0, %1;" ::"r"(kXferBarrier), "r"(kEpiThreads) : "memory");
+                    if (r == 0) {
+                        fence_proxy_async_global();
+                        atomicAdd(args.ready + f.e * args.ksplit + f.blk / kps, 1u);
+                    }
+                } else {
+                    const int col = f.blk * kM + r;
+                    float* out = args.Ypart + static_cast<size_t>(f.ks) * args.rows * args.d;
+                    for (int c0 = 0; c0 < NT && c0 < f.nvalid; c0 += kC) {
+                        uint32_t v[kC];
+                        tmem_ld_32cols(tacc + c0, v);
+                        tmem_ld_wait();
+                        if (col < args.d) {
+#pragma unroll
+                            for (int c = 0; c < kC; ++c)
+                                if (c0 + c < f.nvalid)
+                                    out[static_cast<size_t>(f.row0 + c0 + c) * args.d + col] =
+                                        __uint_as_float(v[c]);
+                        }
+                    }
+                    tc_fence_before();
+                    mbar_arrive(&bk.tmem_empty[acc]);
                 }
             }
             if (++acc == NACC) {
@@ -718,7 +781,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, kTmemCols);
+        tmem_dealloc(tmem_base, C::kTmemCols);
     }
 }
 
@@ -805,8 +868,11 @@ cudaError_t launch_ffn_bf16_decode_fused(const void* x_perm, const int32_t* offs
     if (T <= 32)
         return launch_ffn_fused_nt<32>(x_perm, offsets, W1, W3, W2, rows, d, h, E, H, Ypart,
                                        ksplit, counters, status, s, cap);
-    return launch_ffn_fused_nt<64>(x_perm, offsets, W1, W3, W2, rows, d, h, E, H, Ypart, ksplit,
-                                   counters, status, s, cap);
+    if (T <= 64)
+        return launch_ffn_fused_nt<64>(x_perm, offsets, W1, W3, W2, rows, d, h, E, H, Ypart,
+                                       ksplit, counters, status, s, cap);
+    return launch_ffn_fused_nt<128>(x_perm, offsets, W1, W3, W2, rows, d, h, E, H, Ypart, ksplit,
+                                    counters, status, s, cap);
 }
 
 cudaError_t launch_ffn_bf16_decode(const void* x_perm, const int32_t* offsets, const void* W1,

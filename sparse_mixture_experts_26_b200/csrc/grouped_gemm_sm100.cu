@@ -409,32 +409,40 @@ cudaError_t launch_ffn_bf16(const void* x_perm, const int32_t* offsets, const vo
                             void* H, float* Y, float* partials, int partial_cap, bool reduce,
                             FfnOut* out, uint32_t* status, cudaStream_t s,
                             cudaEvent_t between, uint32_t* counters, int cap) {
-    if (rows <= kDecodeMaxRows) {
+    // Small batches stream the weights: the fused cooperative launch up to
+    // kFusedMaxRows rows, the two-launch form (no co-residency needed) up to
+    // kDecodeMaxRows; above that, or where neither applies, the grouped GEMMs below.
+    const bool can_fuse = counters != nullptr && rows <= kFusedMaxRows;
+    if (rows <= kDecodeMaxRows || can_fuse) {
         int ksplit = partials ? decode_ksplit(h, partial_cap) : 1;
         float* dst = ksplit > 1 ? partials : Y;
         cudaError_t err;
         err = cudaErrorNotSupported;
-        if (counters) {
+        if (can_fuse) {
             err = launch_ffn_bf16_decode_fused(x_perm, offsets, W1, W3, W2, rows, d, h, E, H, dst,
                                                ksplit, counters, status, s, cap);
             if (err == cudaErrorCooperativeLaunchTooLarge || err == cudaErrorNotSupported)
-                cudaGetLastError();  // clear it: the two-launch path below needs no co-residency
+                cudaGetLastError();  // clear it: a path below needs no co-residency
             else if (err == cudaSuccess && between)
                 err = cudaEventRecord(between, s);
         }
-        if (err == cudaErrorCooperativeLaunchTooLarge || err == cudaErrorNotSupported) {
+        const bool fallback =
+            err == cudaErrorCooperativeLaunchTooLarge || err == cudaErrorNotSupported;
+        if (fallback && rows <= kDecodeMaxRows)
             err = launch_ffn_bf16_decode(x_perm, offsets, W1, W3, W2, rows, d, h, E, H, dst,
                                          ksplit, status, s, between, cap);
-        }
-        if (err != cudaSuccess) return err;
-        if (ksplit > 1 && reduce) {
-            err = launch_sum_splits(partials, ksplit, static_cast<size_t>(rows) * d, Y, s);
+        if (!fallback || rows <= kDecodeMaxRows) {
             if (err != cudaSuccess) return err;
-            ksplit = 1;
-            dst = Y;
+            if (ksplit > 1 && reduce) {
+                err = launch_sum_splits(partials, ksplit, static_cast<size_t>(rows) * d, Y, s);
+                if (err != cudaSuccess) return err;
+                ksplit = 1;
+                dst = Y;
+            }
+            if (out) *out = FfnOut{dst, ksplit};
+            return cudaSuccess;
         }
-        if (out) *out = FfnOut{dst, ksplit};
-        return cudaSuccess;
+        // 129..256 rows on a device that cannot co-schedule the fused launch: grouped GEMMs
     }
     if (out) *out = FfnOut{Y, 1};
     if (rows >= kPairMinRows && pair_gemm_enabled())

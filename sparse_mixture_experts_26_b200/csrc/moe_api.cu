@@ -150,7 +150,13 @@ extern "C" {
 
 size_t moe_workspace_bytes(int T, int d, int h, int E, int k, moe_dtype dt) {
     if (check_shape(T, d, h, E, k, dt, true) != MOE_OK) return 0;
-    return ws_layout(T, d, h, E, k, dt).total;
+    // Small batches keep split-K partial sums that larger ones do not, so the layout's
+    // size drops where the grouped GEMMs take over; report the largest size of any batch
+    // up to T, so that one workspace serves every smaller batch too.
+    const int t_small = T < kFusedMaxRows / 2 ? T : kFusedMaxRows / 2;
+    const size_t small = ws_layout(t_small, d, h, E, k, dt).total;
+    const size_t own = ws_layout(T, d, h, E, k, dt).total;
+    return own > small ? own : small;
 }
 
 const char* moe_status_string(moe_status st) {
@@ -306,7 +312,7 @@ moe_status layer_forward_impl(const void* x, const void* Wg, const void* W1, con
     {
         NvtxRange r("combine");
         err = launch_combine(fo.Y, fo.nsplit, static_cast<size_t>(P) * d, inv_perm, w, T, d, dt,
-                             y, stream, idx, offsets, E, cap);
+                             y, stream, idx, offsets, E, cap, at<uint8_t>(ws, L.y_layout));
     }
     if ((st = finish(err, stream, status)) != MOE_OK) return st;
     if (!mark(4)) return MOE_ERR_CUDA;
@@ -369,8 +375,6 @@ moe_status layer_backward_impl(const void* x, const void* Wg, const void* W1, co
     const BwdLayout B = bwd_layout(T, d, h, E);
     if (fwd_ws_bytes < L.total || bwd_ws_bytes < B.total) return MOE_ERR_WORKSPACE;
     const int P = 2 * T;
-    // Where the forward left the expert outputs: split-K partials for small batches.
-    const int nsplit = P <= kDecodeMaxRows ? decode_ksplit(h, kDecodeSplitK) : 1;
     void* fws = const_cast<void*>(fwd_ws);
     BwdArgs a{};
     a.T = T;
@@ -383,8 +387,10 @@ moe_status layer_backward_impl(const void* x, const void* Wg, const void* W1, co
     a.w = at<float>(fws, L.topk_w);
     a.inv = at<int32_t>(fws, L.inv_perm);
     a.offsets = at<int32_t>(fws, L.offsets);
-    a.Y = nsplit > 1 ? at<float>(fws, L.Ypart) : at<float>(fws, L.Y);
-    a.nsplit = nsplit;
+    // the forward's combine recorded whether Y or the split-K partials hold its outputs
+    a.Y = at<float>(fws, L.Y);
+    a.Ypart = at<float>(fws, L.Ypart);
+    a.y_layout = at<uint8_t>(fws, L.y_layout);
     a.split_stride = static_cast<size_t>(P) * d;
     a.x_perm = at<void>(fws, L.x_perm);
     a.H = at<void>(fws, L.H);

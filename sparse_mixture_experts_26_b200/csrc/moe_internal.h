@@ -17,9 +17,12 @@ constexpr int kMaxExperts = 32;
 // Tokens handled by one block of the permutation count / rank kernels.
 constexpr int kPermChunk = 256;
 
-// Grouped rows at or below which the weight-streaming (swap-AB) expert FFN is used,
-// and how many K ranges its down projection is split into at most.
+// Grouped rows at or below which the weight-streaming (swap-AB) expert FFN is used
+// (two launches, or one fused cooperative launch), the larger limit of the fused launch
+// alone (token tiles of up to 128 rows), and how many K ranges its down projection is
+// split into at most.
 constexpr int kDecodeMaxRows = 128;
+constexpr int kFusedMaxRows = 256;
 constexpr int kDecodeSplitK = 8;
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -28,8 +31,8 @@ inline size_t dtype_bytes(moe_dtype dt) { return dt == MOE_BF16 ? 2 : 4; }
 // Byte offsets of every workspace region (1 KiB aligned).  The status word sits at
 // offset 0 so that every entry point sharing a workspace reports into one place.
 struct WsLayout {
-    size_t status, sync, topk_idx, topk_w, offsets, blk_counts, blk_base, perm_token, inv_perm,
-        x_perm, H, Ypart, Y, total;
+    size_t status, y_layout, sync, topk_idx, topk_w, offsets, blk_counts, blk_base, perm_token,
+        inv_perm, x_perm, H, Ypart, Y, total;
     // Bytes needed by moe_permute (status + count/base scratch) and by moe_expert_ffn
     // (status + H); moe_layer_forward needs `total`.
     size_t permute_need, ffn_need;
@@ -48,6 +51,10 @@ inline WsLayout ws_layout(int T, int d, int h, int E, int k, moe_dtype dt) {
         return at;
     };
     L.status = take(256);
+    // one byte in the status region: how many split-K partials (in Ypart) hold the
+    // expert outputs of the last layer call, or 1 for the single array Y (written by
+    // the combine kernel, read by the backward pass)
+    L.y_layout = L.status + 64;
     // dependency counters of the fused small-batch FFN (zero between calls)
     L.sync = take(2 * kMaxExperts * kDecodeSplitK * 4);
     L.blk_counts = take(nb * E * 4);
@@ -55,7 +62,7 @@ inline WsLayout ws_layout(int T, int d, int h, int E, int k, moe_dtype dt) {
     L.permute_need = o;
     L.H = take(P * h * (dt == MOE_BF16 ? 2 : 4));
     // fp32 partial sums of the split-K down projection (small batches, bf16 only)
-    L.Ypart = take(dt == MOE_BF16 && P <= kDecodeMaxRows ? kDecodeSplitK * P * d * 4 : 0);
+    L.Ypart = take(dt == MOE_BF16 && P <= kFusedMaxRows ? kDecodeSplitK * P * d * 4 : 0);
     L.ffn_need = o;
     L.topk_idx = take(P * 4);
     L.topk_w = take(P * 4);
@@ -158,10 +165,13 @@ cudaError_t launch_ffn_bf16_decode(const void* x_perm, const int32_t* offsets, c
 // nsplit arrays Y + i * split_stride at row r.  With cap < INT_MAX (and idx,
 // offsets, E given) a pair whose row lies cap or more rows into its expert's group
 // was dropped and contributes nothing.
+// With `layout_out`, one thread also stores nsplit there (the layer records where
+// its expert outputs are, for the backward pass).
 cudaError_t launch_combine(const float* Y, int nsplit, size_t split_stride,
                            const int32_t* inv_perm, const float* w, int T, int d, moe_dtype dt,
                            void* y, cudaStream_t s, const int32_t* idx = nullptr,
-                           const int32_t* offsets = nullptr, int E = 0, int cap = INT_MAX);
+                           const int32_t* offsets = nullptr, int E = 0, int cap = INT_MAX,
+                           uint8_t* layout_out = nullptr);
 // K ranges of the small-batch down projection: the largest split (at most
 // partial_cap and kDecodeSplitK) that leaves no K range of 64-wide blocks empty.
 inline int decode_ksplit(int h, int partial_cap) {
@@ -179,9 +189,10 @@ struct BwdArgs {
     const float* w;            // [T, 2]
     const int32_t* inv;        // [T, 2]
     const int32_t* offsets;    // [E + 1]
-    const float* Y;            // expert outputs: sum of nsplit arrays [2T, d]
-    int nsplit;
-    size_t split_stride;       // floats between those arrays
+    const float* Y;            // expert outputs as one array [2T, d] ...
+    const float* Ypart;        // ... or as split-K partials, split_stride floats apart
+    const uint8_t* y_layout;   // device byte: number of partials, or 1 for Y
+    size_t split_stride;
     const void* x_perm;        // bf16 [2T, d]
     const void* H;             // bf16 [2T, h]
     const void *x, *Wg, *W1, *W3, *W2;

@@ -76,6 +76,14 @@ def test_workspace_sizes(lib):
     assert lib.moe_workspace_bytes(-1, d, h, 8, 2, BF16) == 0
 
 
+@pytest.mark.parametrize("d,h,dt", [(4096, 14336, BF16), (136, 192, BF16), (24, 40, 0)])
+def test_workspace_size_never_decreases_with_T(lib, d, h, dt):
+    """A workspace sized for T serves every smaller batch: small batches add split-K
+    partial sums that larger batches do not need, and the size must not drop there."""
+    sizes = [lib.moe_workspace_bytes(T, d, h, 8, 2, dt) for T in range(0, 400)]
+    assert all(a <= b for a, b in zip(sizes, sizes[1:]))
+
+
 FAKE = 1 << 20  # 16-byte aligned, never dereferenced: validation fails first
 
 

@@ -52,7 +52,8 @@ def gpu_grads(inp, dy, capacity=-1):
 
 SHAPES = [  # (T, d, h, kind): decode-path and grouped-path forwards, ragged tiles
     (1, 64, 128, "plain"), (16, 128, 256, "skew"), (37, 136, 192, "plain"),
-    (64, 256, 384, "plain"), (300, 136, 192, "plain"), (700, 256, 384, "skew"),
+    (64, 256, 384, "plain"), (100, 136, 192, "skew"), (128, 256, 384, "plain"),
+    (300, 136, 192, "plain"), (700, 256, 384, "skew"),
     (1100, 256, 384, "plain"), (2500, 128, 256, "long"),
 ]
 
@@ -75,7 +76,8 @@ def test_backward_small_shapes(T, d, h, kind):
         assert not g["dW1"][e].any() and not g["dW3"][e].any() and not g["dW2"][e].any()
 
 
-@pytest.mark.parametrize("T,d,h,cap", [(16, 128, 256, 3), (300, 136, 192, 40),
+@pytest.mark.parametrize("T,d,h,cap", [(16, 128, 256, 3), (100, 128, 256, 12),
+                                       (300, 136, 192, 40),
                                        (1500, 136, 192, 300)])
 def test_backward_with_capacity(T, d, h, cap):
     wl = small("bwc", T=T, d=d, h=h, seed=600 + T, kind="skew")
@@ -100,6 +102,26 @@ def test_backward_is_deterministic_and_rejects_unsupported():
         assert torch.equal(v, g1[k]), k
     assert moe.moe_backward_workspace_bytes(16, 128, 200, 8) == 0       # h % 64 != 0
     assert moe.moe_backward_workspace_bytes(16, 128, 256, 8, 2, torch.float32) == 0
+
+
+def test_backward_follows_the_last_forward_on_a_shared_workspace():
+    """Small batches leave their expert outputs as split-K partials, larger ones as one
+    array; the backward reads whichever the last forward on the workspace wrote."""
+    big = small("bwl", T=300, d=136, h=192, seed=8, kind="plain")
+    inp_big = make_inputs(big, "cuda")
+    inp_small = {k: (v[:100].contiguous() if k == "x" else v) for k, v in inp_big.items()}
+    ws = moe.alloc_workspace(300, 136, 192, big.E, 2, torch.bfloat16, "cuda")
+    for inp in (inp_small, inp_big, inp_small):
+        x = inp["x"]
+        T = x.shape[0]
+        dy = seeded_dy(T, 136, 13 + T)
+        ref, _ = gpu_grads(inp, dy)  # a fresh workspace of its own
+        y = torch.empty_like(x)
+        moe.moe_layer_forward(x, inp["Wg"], inp["W1"], inp["W3"], inp["W2"], y, ws)
+        out = moe.layer_backward(x, inp["Wg"], inp["W1"], inp["W3"], inp["W2"], dy, ws)
+        for k, v in zip(("dx", "dWg", "dW1", "dW3", "dW2"), out):
+            assert torch.equal(v, ref[k]), (T, k)
+    assert moe.moe_device_status(ws) == 0
 
 
 # ---------------------------------------------------------------- full size, sampled

@@ -46,6 +46,7 @@ def guarded_ws(T, d, h, E, dtype):
 
 @pytest.mark.parametrize("T,d,h,kind,dtype,cap", [
     (16, 256, 384, "skew", "bf16", -1),     # weight-streaming FFN
+    (100, 256, 384, "skew", "bf16", -1),    # weight-streaming FFN, 128-token tiles
     (300, 136, 200, "plain", "bf16", -1),   # single-SM grouped GEMM, ragged tiles
     (1100, 256, 384, "plain", "bf16", -1),  # CTA-pair grouped GEMM
     (1500, 136, 200, "skew", "bf16", 300),  # capacity on the pair path
@@ -86,7 +87,7 @@ def test_stepwise_writes_stay_in_bounds(T):
         assert g.intact(), name
 
 
-@pytest.mark.parametrize("T,cap", [(40, -1), (1100, -1), (1500, 300)])
+@pytest.mark.parametrize("T,cap", [(40, -1), (100, -1), (1100, -1), (1500, 300)])
 def test_backward_writes_stay_in_bounds(T, cap):
     wl = small("can3", T=T, d=136, h=192, seed=T + 2, kind="skew")
     inp = make_inputs(wl, "cuda")

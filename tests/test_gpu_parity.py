@@ -101,12 +101,13 @@ def check_routing_and_permutation(g, x_cpu, Wg_cpu, E):
 
 
 SMALL = [  # (T, d, h, kind): ragged row blocks, K tails, N tails, empty groups
-    # T <= 64 runs the weight-streaming kernels (token tiles of 16, 32 or 64)
+    # T <= 128 runs the weight-streaming kernels (token tiles of 16, 32, 64 or 128)
     (1, 64, 128, "plain"), (2, 64, 128, "plain"), (3, 128, 256, "plain"),
     (5, 136, 200, "plain"), (16, 256, 384, "skew"), (17, 128, 256, "plain"),
-    (33, 128, 256, "plain"), (64, 256, 512, "plain"),
-    # T > 64 runs the grouped GEMM (128-row blocks)
-    (65, 128, 256, "plain"), (129, 256, 512, "plain"), (300, 136, 200, "plain"),
+    (33, 128, 256, "plain"), (64, 256, 512, "plain"), (65, 128, 256, "plain"),
+    (100, 136, 200, "skew"), (128, 256, 512, "plain"),
+    # T > 128 runs the grouped GEMM (128-row blocks)
+    (129, 256, 512, "plain"), (300, 136, 200, "plain"),
     (1000, 512, 1024, "plain"), (700, 256, 384, "skew"), (513, 128, 256, "long"),
     # >= 2048 grouped rows run the CTA-pair grouped GEMM (256-row blocks; an expert's
     # last block of <= 128 rows runs in the pair's 128-row mode)
@@ -134,7 +135,8 @@ def test_layer_bf16_small_shapes(T, d, h, kind):
     assert torch.equal(layer_y(inp), g["y"])
 
 
-@pytest.mark.parametrize("T,kind", [(1, "plain"), (16, "skew"), (40, "plain"), (64, "skew")])
+@pytest.mark.parametrize("T,kind", [(1, "plain"), (16, "skew"), (40, "plain"), (64, "skew"),
+                                    (100, "plain"), (128, "skew")])
 def test_small_batch_layer_repeated_calls(T, kind):
     """The small-batch expert FFN is one cooperative launch whose dependency counters
     must be zero again after every call: repeated calls on one workspace, interleaved
@@ -286,6 +288,7 @@ def capped_y(inp, capacity):
 @pytest.mark.parametrize("T,d,h,kind,cap,dtype", [
     (16, 256, 384, "skew", 3, "bf16"),       # fused weight-streaming kernel
     (40, 128, 256, "skew", 5, "bf16"),
+    (100, 128, 256, "skew", 12, "bf16"),     # fused kernel, 128-token tiles
     (300, 136, 200, "skew", 40, "bf16"),     # single-SM grouped GEMM
     (1500, 136, 200, "skew", 300, "bf16"),   # CTA-pair grouped GEMM (half tiles too)
     (1100, 256, 384, "plain", 260, "bf16"),
