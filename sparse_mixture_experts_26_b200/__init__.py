@@ -41,9 +41,9 @@ EXPORTED_SYMBOLS = ("moe_workspace_bytes", "moe_route", "moe_permute", "moe_expe
                     "moe_layer_backward_events")
 def launches_per_layer(T: int) -> int:
     """Kernels one moe_layer_forward queues: router 1, permutation 1 (T <= 512) or 4
-    (count, scan, rank, gather), expert FFN 1 (T <= 64: gate/up and down fused) or 2,
+    (count, scan, rank, gather), expert FFN 1 (T <= 128: gate/up and down fused) or 2,
     combine 1."""
-    return 1 + (1 if T <= 512 else 4) + (1 if T <= 64 else 2) + 1
+    return 1 + (1 if T <= 512 else 4) + (1 if T <= 128 else 2) + 1
 
 
 class MoeError(RuntimeError):

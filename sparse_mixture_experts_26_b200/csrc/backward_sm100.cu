@@ -667,8 +667,11 @@ __device__ __forceinline__ bool pair_kept(const int32_t* idx, const int32_t* off
 }
 
 // One block per token: dY rows of its two pairs, dw, and the token's logit gradients.
-// The forward left its expert outputs either in Y or as split-K partials in Ypart
-// (split_stride floats apart, summed in order); the byte at y_layout says which.
+// Small batches (kSplit) may have left their expert outputs as split-K partials in
+// Ypart (split_stride floats apart, summed in order) and the byte at y_layout says
+// whether they did; larger batches always leave them in Y, and their form keeps its
+// register count low for streaming.
+template <bool kSplit>
 __global__ void __launch_bounds__(kPrepThreads)
     bwd_prep_kernel(const __nv_bfloat16* __restrict__ dy, const int32_t* __restrict__ idx,
                     const float* __restrict__ w, const int32_t* __restrict__ inv,
@@ -679,29 +682,69 @@ __global__ void __launch_bounds__(kPrepThreads)
                     float* __restrict__ dlogits) {
     __shared__ float red[2][kPrepThreads / 32];
     const int P = 2 * T;
-    int nsplit = *y_layout;
+    int nsplit = kSplit ? *y_layout : 1;
     nsplit = nsplit < 1 ? 1 : (nsplit > kDecodeSplitK ? kDecodeSplitK : nsplit);
     const float* __restrict__ Y = nsplit > 1 ? Ypart : Y1;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int d4 = d >> 2;  // d % 8 == 0: rows of Y, dy and dY hold whole 4-column groups
+    const size_t stride4 = split_stride >> 2;
+    const float4* __restrict__ Y4 = reinterpret_cast<const float4*>(Y);
+    // Expert output row r, columns 4c..4c+3: the partials summed in order.  Every
+    // partial is loaded before the first add, so the loads overlap instead of forming
+    // a chain of dependent misses.
+    auto y_row = [&](int r, int c) {
+        const size_t at = static_cast<size_t>(r) * d4 + c;
+        if constexpr (!kSplit) {
+            return Y4[at];
+        } else {
+            float4 p[kDecodeSplitK];
+#pragma unroll
+            for (int s = 0; s < kDecodeSplitK; ++s)
+                if (s < nsplit) p[s] = Y4[s * stride4 + at];
+            float4 y = p[0];
+#pragma unroll
+            for (int s = 1; s < kDecodeSplitK; ++s)
+                if (s < nsplit) {
+                    y.x += p[s].x;
+                    y.y += p[s].y;
+                    y.z += p[s].z;
+                    y.w += p[s].w;
+                }
+            return y;
+        }
+    };
+    auto store_dy = [&](int r, int c, float wt, const float (&g)[4]) {
+        uint2 v;
+        v.x = pack_bf16x2(wt * g[0], wt * g[1]);
+        v.y = pack_bf16x2(wt * g[2], wt * g[3]);
+        *reinterpret_cast<uint2*>(dY + static_cast<size_t>(r) * d + 4 * c) = v;
+    };
     for (int t = blockIdx.x; t < T; t += gridDim.x) {
         const bool keep0 = pair_kept(idx, offsets, inv, 2 * t, E, P, cap);
         const bool keep1 = pair_kept(idx, offsets, inv, 2 * t + 1, E, P, cap);
         const int r0 = inv[2 * t], r1 = inv[2 * t + 1];
         const float w0 = keep0 ? w[2 * t] : 0.f, w1 = keep1 ? w[2 * t + 1] : 0.f;
         float s0 = 0.f, s1 = 0.f;
-        for (int c = threadIdx.x; c < d; c += blockDim.x) {
-            const float g = __bfloat162float(dy[static_cast<size_t>(t) * d + c]);
+        for (int c = threadIdx.x; c < d4; c += blockDim.x) {
+            const uint2 graw =
+                *reinterpret_cast<const uint2*>(dy + static_cast<size_t>(t) * d + 4 * c);
+            const float g[4] = {bf16_lo(graw.x), bf16_hi(graw.x), bf16_lo(graw.y),
+                                bf16_hi(graw.y)};
             if (keep0) {
-                float y = Y[static_cast<size_t>(r0) * d + c];
-                for (int s = 1; s < nsplit; ++s) y += Y[s * split_stride + static_cast<size_t>(r0) * d + c];
-                s0 = fmaf(g, y, s0);
-                dY[static_cast<size_t>(r0) * d + c] = __float2bfloat16_rn(w0 * g);
+                const float4 y = y_row(r0, c);
+                s0 = fmaf(g[0], y.x, s0);
+                s0 = fmaf(g[1], y.y, s0);
+                s0 = fmaf(g[2], y.z, s0);
+                s0 = fmaf(g[3], y.w, s0);
+                store_dy(r0, c, w0, g);
             }
             if (keep1) {
-                float y = Y[static_cast<size_t>(r1) * d + c];
-                for (int s = 1; s < nsplit; ++s) y += Y[s * split_stride + static_cast<size_t>(r1) * d + c];
-                s1 = fmaf(g, y, s1);
-                dY[static_cast<size_t>(r1) * d + c] = __float2bfloat16_rn(w1 * g);
+                const float4 y = y_row(r1, c);
+                s1 = fmaf(g[0], y.x, s1);
+                s1 = fmaf(g[1], y.y, s1);
+                s1 = fmaf(g[2], y.z, s1);
+                s1 = fmaf(g[3], y.w, s1);
+                store_dy(r1, c, w1, g);
             }
         }
 #pragma unroll
@@ -743,53 +786,66 @@ __global__ void __launch_bounds__(kPrepThreads)
                   const __nv_bfloat16* __restrict__ Wg, __nv_bfloat16* __restrict__ dx) {
     const int P = 2 * T;
     const int d4 = d / 4;
-    const size_t n = static_cast<size_t>(T) * d4;
-    for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
-         i += static_cast<size_t>(gridDim.x) * blockDim.x) {
-        const int t = static_cast<int>(i / d4);
-        const int c = static_cast<int>(i - static_cast<size_t>(t) * d4) * 4;
-        float v[4] = {0.f, 0.f, 0.f, 0.f};
+    // One token per block iteration: its routing (which pairs were kept, their rows,
+    // its logit gradients) is read once, then the columns run with independent loads.
+    for (int t = blockIdx.x; t < T; t += gridDim.x) {
+        const bool keep0 = pair_kept(idx, offsets, inv, 2 * t, E, P, cap);
+        const bool keep1 = pair_kept(idx, offsets, inv, 2 * t + 1, E, P, cap);
+        const float4* __restrict__ row0 =
+            reinterpret_cast<const float4*>(dX + static_cast<size_t>(inv[2 * t]) * d);
+        const float4* __restrict__ row1 =
+            reinterpret_cast<const float4*>(dX + static_cast<size_t>(inv[2 * t + 1]) * d);
+        const float* dl = dlogits + static_cast<size_t>(t) * E;
+        float g8[8];
+        if (E == 8) {
 #pragma unroll
-        for (int j = 0; j < 2; ++j) {
-            if (pair_kept(idx, offsets, inv, 2 * t + j, E, P, cap)) {
-                const float4 a = *reinterpret_cast<const float4*>(
-                    dX + static_cast<size_t>(inv[2 * t + j]) * d + c);
+            for (int e = 0; e < 8; ++e) g8[e] = dl[e];
+        }
+#pragma unroll 2
+        for (int c4 = threadIdx.x; c4 < d4; c4 += blockDim.x) {
+            const int c = 4 * c4;
+            float v[4] = {0.f, 0.f, 0.f, 0.f};
+            if (keep0) {
+                const float4 a = row0[c4];
                 v[0] += a.x;
                 v[1] += a.y;
                 v[2] += a.z;
                 v[3] += a.w;
             }
-        }
-        const float* dl = dlogits + static_cast<size_t>(t) * E;
-        if (E == 8) {
-            // W_g rows of the four columns: one 16-byte load each
-            float g[8];
+            if (keep1) {
+                const float4 a = row1[c4];
+                v[0] += a.x;
+                v[1] += a.y;
+                v[2] += a.z;
+                v[3] += a.w;
+            }
+            if (E == 8) {
+                // W_g rows of the four columns: one 16-byte load each
 #pragma unroll
-            for (int e = 0; e < 8; ++e) g[e] = dl[e];
+                for (int u = 0; u < 4; ++u) {
+                    const uint4 q =
+                        *reinterpret_cast<const uint4*>(Wg + static_cast<size_t>(c + u) * 8);
+                    const uint32_t w4[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const uint4 q = *reinterpret_cast<const uint4*>(Wg + static_cast<size_t>(c + u) * 8);
-                const uint32_t w4[4] = {q.x, q.y, q.z, q.w};
+                    for (int p2 = 0; p2 < 4; ++p2) {
+                        v[u] = fmaf(g8[2 * p2], bf16_lo(w4[p2]), v[u]);
+                        v[u] = fmaf(g8[2 * p2 + 1], bf16_hi(w4[p2]), v[u]);
+                    }
+                }
+            } else {
+                for (int e = 0; e < E; ++e) {
+                    const float g = dl[e];
 #pragma unroll
-                for (int p2 = 0; p2 < 4; ++p2) {
-                    v[u] = fmaf(g[2 * p2], __uint_as_float(w4[p2] << 16), v[u]);
-                    v[u] = fmaf(g[2 * p2 + 1], __uint_as_float(w4[p2] & 0xffff0000u), v[u]);
+                    for (int u = 0; u < 4; ++u)
+                        v[u] = fmaf(g, __bfloat162float(Wg[static_cast<size_t>(c + u) * E + e]),
+                                    v[u]);
                 }
             }
-        } else {
-            for (int e = 0; e < E; ++e) {
-                const float g = dl[e];
-#pragma unroll
-                for (int u = 0; u < 4; ++u)
-                    v[u] = fmaf(g, __bfloat162float(Wg[static_cast<size_t>(c + u) * E + e]), v[u]);
-            }
+            uint2 o;
+            o.x = pack_bf16x2(v[0], v[1]);
+            o.y = pack_bf16x2(v[2], v[3]);
+            *reinterpret_cast<uint2*>(dx + static_cast<size_t>(t) * d + c) = o;
         }
-        __nv_bfloat162 lo = __floats2bfloat162_rn(v[0], v[1]);
-        __nv_bfloat162 hi = __floats2bfloat162_rn(v[2], v[3]);
-        uint2 o;
-        o.x = *reinterpret_cast<uint32_t*>(&lo);
-        o.y = *reinterpret_cast<uint32_t*>(&hi);
-        *reinterpret_cast<uint2*>(dx + static_cast<size_t>(t) * d + c) = o;
     }
 }
 
@@ -797,31 +853,49 @@ __global__ void __launch_bounds__(kPrepThreads)
 // partial [d, E], then the partials summed in chunk order.
 constexpr int kWgChunk = 64;
 
+// EMAX: the accumulator count (8 when E <= 8, else kMaxExperts); each thread owns two
+// adjacent columns and runs the chunk's tokens in order, so the sums do not depend on
+// the launch shape.
+template <int EMAX>
 __global__ void __launch_bounds__(kPrepThreads)
     bwd_dwg_partial_kernel(const __nv_bfloat16* __restrict__ x, const float* __restrict__ dlogits,
                            int T, int d, int E, float* __restrict__ part) {
-    __shared__ float dl[kWgChunk * kMaxExperts];
+    __shared__ __align__(16) float dl[kWgChunk * EMAX];
     const int chunk = blockIdx.y;
     const int t0 = chunk * kWgChunk;
     const int nt = min(kWgChunk, T - t0);
-    for (int i = threadIdx.x; i < nt * E; i += blockDim.x)
-        dl[i] = dlogits[static_cast<size_t>(t0) * E + i];
+    // the chunk's logit gradients, E per token, zero-padded to EMAX
+    for (int i = threadIdx.x; i < nt * EMAX; i += blockDim.x) {
+        const int t = i / EMAX, e = i - t * EMAX;
+        dl[i] = e < E ? dlogits[static_cast<size_t>(t0 + t) * E + e] : 0.f;
+    }
     __syncthreads();
-    const int c = blockIdx.x * blockDim.x + threadIdx.x;
+    const int c = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
     if (c >= d) return;
-    float acc[kMaxExperts];
+    float acc0[EMAX], acc1[EMAX];
 #pragma unroll
-    for (int e = 0; e < kMaxExperts; ++e) acc[e] = 0.f;
+    for (int e = 0; e < EMAX; ++e) acc0[e] = acc1[e] = 0.f;
+    const uint32_t* __restrict__ xc =
+        reinterpret_cast<const uint32_t*>(x + static_cast<size_t>(t0) * d + c);
+    const int d2 = d / 2;
+#pragma unroll 4
     for (int t = 0; t < nt; ++t) {
-        const float xv = __bfloat162float(x[static_cast<size_t>(t0 + t) * d + c]);
+        const uint32_t xv = xc[static_cast<size_t>(t) * d2];
+        const float x0 = bf16_lo(xv), x1 = bf16_hi(xv);
 #pragma unroll
-        for (int e = 0; e < kMaxExperts; ++e)
-            if (e < E) acc[e] = fmaf(xv, dl[t * E + e], acc[e]);
+        for (int e = 0; e < EMAX; ++e) {
+            const float g = dl[t * EMAX + e];
+            acc0[e] = fmaf(x0, g, acc0[e]);
+            acc1[e] = fmaf(x1, g, acc1[e]);
+        }
     }
     float* out = part + (static_cast<size_t>(chunk) * d + c) * E;
 #pragma unroll
-    for (int e = 0; e < kMaxExperts; ++e)
-        if (e < E) out[e] = acc[e];
+    for (int e = 0; e < EMAX; ++e)
+        if (e < E) {
+            out[e] = acc0[e];
+            out[E + e] = acc1[e];
+        }
 }
 
 __global__ void __launch_bounds__(kPrepThreads)
@@ -888,7 +962,8 @@ cudaError_t launch_layer_backward(const BwdArgs& a, cudaStream_t s) {
     };
     if ((err = mark(0)) != cudaSuccess) return err;
     // 1. dY, dw, dlogits
-    err = launch_k(bwd_prep_kernel, grid_for(T, 8 * sms), kPrepThreads, 0, s,
+    err = launch_k(P <= kFusedMaxRows ? bwd_prep_kernel<true> : bwd_prep_kernel<false>,
+                   grid_for(T, 8 * sms), kPrepThreads, 0, s,
                    static_cast<const __nv_bfloat16*>(a.dy), a.idx, a.w, a.inv, a.offsets, T, d, E,
                    a.cap, a.Y, a.Ypart, a.y_layout, a.split_stride,
                    static_cast<__nv_bfloat16*>(a.dY), a.dw, a.dlogits);
@@ -947,8 +1022,7 @@ cudaError_t launch_layer_backward(const BwdArgs& a, cudaStream_t s) {
     }
     // 5. dx
     {
-        const long long n = static_cast<long long>(T) * (d / 4);
-        err = launch_k(bwd_dx_kernel, grid_for((n + kPrepThreads - 1) / kPrepThreads, 8 * sms),
+        err = launch_k(bwd_dx_kernel, grid_for(T, 8 * sms),
                        kPrepThreads, 0, s, static_cast<const float*>(a.dX), a.idx, a.inv,
                        a.offsets, T, d, E, a.cap, static_cast<const float*>(a.dlogits),
                        static_cast<const __nv_bfloat16*>(a.Wg), static_cast<__nv_bfloat16*>(a.dx));
@@ -1002,8 +1076,9 @@ cudaError_t launch_layer_backward(const BwdArgs& a, cudaStream_t s) {
     // 7. dWg
     {
         const int nchunk = static_cast<int>(bwd_dwg_chunks(T));
-        err = launch_k(bwd_dwg_partial_kernel, dim3((d + kPrepThreads - 1) / kPrepThreads, nchunk),
-                       kPrepThreads, 0, s, static_cast<const __nv_bfloat16*>(a.x),
+        const dim3 grid((d / 2 + kPrepThreads - 1) / kPrepThreads, nchunk);
+        err = launch_k(E <= 8 ? bwd_dwg_partial_kernel<8> : bwd_dwg_partial_kernel<kMaxExperts>,
+                       grid, kPrepThreads, 0, s, static_cast<const __nv_bfloat16*>(a.x),
                        static_cast<const float*>(a.dlogits), T, d, E, a.dwg_part);
         if (err != cudaSuccess) return err;
         const long long n = static_cast<long long>(d) * E;

@@ -29,21 +29,33 @@ __device__ __forceinline__ void store4(__nv_bfloat16* y, size_t i, float4 v) {
     reinterpret_cast<uint2*>(y)[i] = u;
 }
 
-// Row r of the in-order sum of nsplit arrays split_stride4 float4s apart.
+// Row r of the in-order sum of nsplit arrays split_stride4 float4s apart.  The first
+// kDecodeSplitK partials are all loaded before the first add, so their loads overlap.
+__device__ __forceinline__ void add4(float4& a, const float4& b) {
+    a.x += b.x;
+    a.y += b.y;
+    a.z += b.z;
+    a.w += b.w;
+}
 __device__ __forceinline__ float4 split_sum(const float4* __restrict__ Y, int nsplit,
                                            size_t split_stride4, size_t at) {
-    float4 a = Y[at];
-    for (int i = 1; i < nsplit; ++i) {
-        const float4 b = Y[static_cast<size_t>(i) * split_stride4 + at];
-        a.x += b.x;
-        a.y += b.y;
-        a.z += b.z;
-        a.w += b.w;
-    }
+    float4 p[kDecodeSplitK];
+#pragma unroll
+    for (int i = 0; i < kDecodeSplitK; ++i)
+        if (i < nsplit) p[i] = Y[static_cast<size_t>(i) * split_stride4 + at];
+    float4 a = p[0];
+#pragma unroll
+    for (int i = 1; i < kDecodeSplitK; ++i)
+        if (i < nsplit) add4(a, p[i]);
+    for (int i = kDecodeSplitK; i < nsplit; ++i)
+        add4(a, Y[static_cast<size_t>(i) * split_stride4 + at]);
     return a;
 }
 
-template <typename Tout>
+// kSplit: the expert outputs arrive as split-K partials (small batches).  The
+// single-array form keeps its register count low, so that enough warps stay resident
+// to stream large batches at full bandwidth.
+template <typename Tout, bool kSplit>
 __global__ void __launch_bounds__(kCombineThreads)
     combine_kernel(const float4* __restrict__ Y, int nsplit, size_t split_stride4,
                    const int32_t* __restrict__ inv, const float* __restrict__ w, int T, int d4,
@@ -72,12 +84,17 @@ __global__ void __launch_bounds__(kCombineThreads)
         // inv_perm entries outside [0, 2T) would come from an invalid permutation;
         // they contribute nothing instead of reading out of bounds.
         // dropped pairs (w == 0) are not read: their rows were never written
-        const float4 a = (r0 < P && w0 != 0.f)
-                             ? split_sum(Y, nsplit, split_stride4, static_cast<size_t>(r0) * d4 + c)
-                             : make_float4(0, 0, 0, 0);
-        const float4 b = (r1 < P && w1 != 0.f)
-                             ? split_sum(Y, nsplit, split_stride4, static_cast<size_t>(r1) * d4 + c)
-                             : make_float4(0, 0, 0, 0);
+        const size_t at0 = static_cast<size_t>(r0) * d4 + c;
+        const size_t at1 = static_cast<size_t>(r1) * d4 + c;
+        const bool use0 = r0 < P && w0 != 0.f, use1 = r1 < P && w1 != 0.f;
+        float4 a = make_float4(0, 0, 0, 0), b = a;
+        if constexpr (kSplit) {
+            if (use0) a = split_sum(Y, nsplit, split_stride4, at0);
+            if (use1) b = split_sum(Y, nsplit, split_stride4, at1);
+        } else {
+            if (use0) a = Y[at0];
+            if (use1) b = Y[at1];
+        }
         float4 o;
         o.x = fmaf(w1, b.x, w0 * a.x);
         o.y = fmaf(w1, b.y, w0 * a.y);
@@ -122,14 +139,21 @@ cudaError_t launch_combine(const float* Y, int nsplit, size_t split_stride,
     if (cap != INT_MAX && (!idx || !offsets)) return cudaErrorInvalidValue;
     const int d4 = d / 4;
     const unsigned blocks = grid_for(static_cast<size_t>(T) * d4);
-    if (dt == MOE_BF16)
-        return launch_k(combine_kernel<__nv_bfloat16>, blocks, kCombineThreads, 0, s,
-                        reinterpret_cast<const float4*>(Y), nsplit, split_stride / 4, inv_perm,
-                        w, T, d4, static_cast<__nv_bfloat16*>(y), idx, offsets, E, cap,
+    const float4* Y4 = reinterpret_cast<const float4*>(Y);
+    if (dt == MOE_BF16) {
+        auto* yb = static_cast<__nv_bfloat16*>(y);
+        if (nsplit > 1)
+            return launch_k(combine_kernel<__nv_bfloat16, true>, blocks, kCombineThreads, 0, s, Y4,
+                            nsplit, split_stride / 4, inv_perm, w, T, d4, yb, idx, offsets, E,
+                            cap, layout_out);
+        return launch_k(combine_kernel<__nv_bfloat16, false>, blocks, kCombineThreads, 0, s, Y4,
+                        nsplit, split_stride / 4, inv_perm, w, T, d4, yb, idx, offsets, E, cap,
                         layout_out);
-    return launch_k(combine_kernel<float>, blocks, kCombineThreads, 0, s,
-                    reinterpret_cast<const float4*>(Y), nsplit, split_stride / 4, inv_perm, w, T,
-                    d4, static_cast<float*>(y), idx, offsets, E, cap, layout_out);
+    }
+    if (nsplit != 1) return cudaErrorInvalidValue;  // split-K partials are bf16-path only
+    return launch_k(combine_kernel<float, false>, blocks, kCombineThreads, 0, s, Y4, nsplit,
+                    split_stride / 4, inv_perm, w, T, d4, static_cast<float*>(y), idx, offsets, E,
+                    cap, layout_out);
 }
 
 }  // namespace moe

@@ -37,8 +37,9 @@ bool pdl_allowed() {
     }
     return v == 1;
 }
-// Small batches: every kernel is short, so overlapping launches pays off.
-bool small_batch(int T) { return T <= 64; }
+// Small batches (the weight-streaming FFN's range): every kernel but the FFN is short,
+// so overlapping launches pays off.
+bool small_batch(int T) { return T <= kFusedMaxRows / 2; }
 }  // namespace
 
 bool pdl_enabled() { return t_pdl_scope && pdl_allowed(); }

@@ -147,6 +147,10 @@ __device__ __forceinline__ void fence_proxy_async_global() {
 // ------------------------------------------------------------------ small numerics
 __device__ __forceinline__ float bits_f32(uint32_t u) { return __uint_as_float(u); }
 
+// The two bf16 halves of a 32-bit word as floats (bf16 is the upper half of an fp32).
+__device__ __forceinline__ float bf16_lo(uint32_t u) { return __uint_as_float(u << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t u) { return __uint_as_float(u & 0xffff0000u); }
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&v);
