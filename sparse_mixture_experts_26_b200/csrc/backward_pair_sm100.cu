@@ -452,14 +452,10 @@ cudaError_t launch_wgrad_pair(const CUtensorMap& A, const CUtensorMap& B, const 
                               const CUtensorMap& O1, const int32_t* offsets, int E, int rows,
                               int M, int N, int split, float* out0, float* out1, uint32_t* status,
                               int cap, cudaStream_t s) {
-    static int configured[64] = {0};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 64 && !configured[dev]) {
-        cudaFuncSetAttribute(bwd_wgrad_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kSmemBytes);
-        configured[dev] = 1;
-    }
+    static PerDeviceOnce smem_once;
+    if (const cudaError_t err = opt_in_smem(smem_once, bwd_wgrad_pair_kernel, kSmemBytes);
+        err != cudaSuccess)
+        return err;
     PArgs p{offsets, E, rows, M, N, (M + 2 * kRows - 1) / (2 * kRows), (N + kN - 1) / kN, split,
             out0, out1, status, cap};
     const long long tiles = static_cast<long long>(E) * p.m_pairs * p.n_tiles;

@@ -914,14 +914,9 @@ __global__ void __launch_bounds__(kPrepThreads)
 // the kernel: the instantiations share one function type, so it cannot be the key.
 enum KernelSlot { kSlotDH, kSlotDUV, kSlotDX, kSlotW2, kSlotW13, kSlotW2s, kSlotW13s, kSlots };
 template <typename Kern>
-void configure(Kern kern, KernelSlot slot, int smem_bytes) {
-    static int configured[kSlots][64] = {};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 64 && !configured[slot][dev]) {
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
-        configured[slot][dev] = 1;
-    }
+cudaError_t configure(Kern kern, KernelSlot slot, int smem_bytes) {
+    static PerDeviceOnce once[kSlots];
+    return opt_in_smem(once[slot], kern, smem_bytes);
 }
 
 // Grouped rows at or below which the weight-gradient GEMMs use the store-bound shape.
@@ -936,12 +931,16 @@ cudaError_t launch_wgrad(bool short_k, int grid, cudaStream_t s, const CUtensorM
     if (short_k) {
         constexpr int st = kWgradShort[0], ob = kWgradShort[1];
         auto kern = bwd_wgrad_kernel<MODE, st, ob>;
-        configure(kern, MODE == kModeW2 ? kSlotW2s : kSlotW13s, wgrad_smem_bytes<st, ob>());
+        const cudaError_t err =
+            configure(kern, MODE == kModeW2 ? kSlotW2s : kSlotW13s, wgrad_smem_bytes<st, ob>());
+        if (err != cudaSuccess) return err;
         return launch_k(kern, grid, kThreads, wgrad_smem_bytes<st, ob>(), s, A, B, O0, O1, w);
     }
     constexpr int st = kWgradLong[0], ob = kWgradLong[1];
     auto kern = bwd_wgrad_kernel<MODE, st, ob>;
-    configure(kern, MODE == kModeW2 ? kSlotW2 : kSlotW13, wgrad_smem_bytes<st, ob>());
+    const cudaError_t err =
+        configure(kern, MODE == kModeW2 ? kSlotW2 : kSlotW13, wgrad_smem_bytes<st, ob>());
+    if (err != cudaSuccess) return err;
     return launch_k(kern, grid, kThreads, wgrad_smem_bytes<st, ob>(), s, A, B, O0, O1, w);
 }
 
@@ -990,7 +989,8 @@ cudaError_t launch_layer_backward(const BwdArgs& a, cudaStream_t s) {
         if (err != cudaSuccess || (err = mark(2)) != cudaSuccess) return err;
     } else {
         RowArgs r{a.offsets, E, P, d, h, (h + kN - 1) / kN, h, d, a.dH, nullptr, a.status, a.cap};
-        configure(bwd_rows_kernel<kModeDH>, kSlotDH, kSmemBytes);
+        if ((err = configure(bwd_rows_kernel<kModeDH>, kSlotDH, kSmemBytes)) != cudaSuccess)
+            return err;
         err = launch_k(bwd_rows_kernel<kModeDH>, grid_for(row_blocks * r.n_tiles, sms), kThreads,
                        kSmemBytes, s, m_dY128, m_W2, m_W2, r);
         if (err != cudaSuccess || (err = mark(2)) != cudaSuccess) return err;
@@ -1002,7 +1002,8 @@ cudaError_t launch_layer_backward(const BwdArgs& a, cudaStream_t s) {
         if (err != cudaSuccess || (err = mark(3)) != cudaSuccess) return err;
     } else {
         RowArgs r{a.offsets, E, P, d, h, (h + 127) / 128, h, d, a.DUV, a.dH, a.status, a.cap};
-        configure(bwd_rows_kernel<kModeDUV>, kSlotDUV, kSmemBytes);
+        if ((err = configure(bwd_rows_kernel<kModeDUV>, kSlotDUV, kSmemBytes)) != cudaSuccess)
+            return err;
         err = launch_k(bwd_rows_kernel<kModeDUV>, grid_for(row_blocks * r.n_tiles, sms),
                        kThreads, kSmemBytes, s, m_x, m_W1r, m_W3r, r);
         if (err != cudaSuccess || (err = mark(3)) != cudaSuccess) return err;
@@ -1015,7 +1016,8 @@ cudaError_t launch_layer_backward(const BwdArgs& a, cudaStream_t s) {
     } else {
         RowArgs r{a.offsets, E, P, 2 * h, d, (d + kN - 1) / kN, h, d, a.dX, nullptr, a.status,
                   a.cap};
-        configure(bwd_rows_kernel<kModeDX>, kSlotDX, kSmemBytes);
+        if ((err = configure(bwd_rows_kernel<kModeDX>, kSlotDX, kSmemBytes)) != cudaSuccess)
+            return err;
         err = launch_k(bwd_rows_kernel<kModeDX>, grid_for(row_blocks * r.n_tiles, sms), kThreads,
                        kSmemBytes, s, m_duv128, m_W1mn, m_W3mn, r);
         if (err != cudaSuccess || (err = mark(4)) != cudaSuccess) return err;

@@ -378,13 +378,9 @@ cudaError_t launch_decode(const CUtensorMap& w0, const CUtensorMap& w1, const CU
                           const DecodeArgs& args, int grid, cudaStream_t s) {
     using C = DecodeCfg<MODE, NT>;
     auto kern = decode_gemm_kernel<MODE, NT>;
-    static int configured[64] = {0};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 64 && !configured[dev]) {
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
-        configured[dev] = 1;
-    }
+    static PerDeviceOnce smem_once;
+    if (const cudaError_t err = opt_in_smem(smem_once, kern, C::kSmem); err != cudaSuccess)
+        return err;
     return launch_k(kern, grid, kThreads, C::kSmem, s, w0, w1, x, args);
 }
 
@@ -799,13 +795,9 @@ cudaError_t launch_ffn_fused_nt(const void* x_perm, const int32_t* offsets, cons
         return cudaErrorInvalidValue;
     using C = DecodeCfg<kSwiGLU, NT>;
     auto kern = decode_ffn_fused_kernel<NT>;
-    static int configured[64] = {0};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 64 && !configured[dev]) {
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
-        configured[dev] = 1;
-    }
+    static PerDeviceOnce smem_once;
+    if (const cudaError_t err = opt_in_smem(smem_once, kern, C::kSmem); err != cudaSuccess)
+        return err;
     FusedArgs a{offsets, E, rows, d, h, (h + 63) / 64, (d + kM - 1) / kM, ksplit, H, Ypart,
                 counters, counters + E * ksplit, status, cap};
     const int sms = device_sm_count();

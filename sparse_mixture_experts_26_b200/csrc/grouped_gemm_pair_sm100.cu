@@ -535,13 +535,9 @@ template <int EPI, int BOP = kBKMajor>
 cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
                         const PairArgs& args, int npairs, cudaStream_t s) {
     auto kern = grouped_gemm_pair_kernel<EPI, BOP>;
-    static int configured[64] = {0};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 64 && !configured[dev]) {
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-        configured[dev] = 1;
-    }
+    static PerDeviceOnce smem_once;
+    if (const cudaError_t err = opt_in_smem(smem_once, kern, kSmemBytes); err != cudaSuccess)
+        return err;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * npairs);
     cfg.blockDim = dim3(kThreads);

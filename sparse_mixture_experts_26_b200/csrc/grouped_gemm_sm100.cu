@@ -339,13 +339,9 @@ template <int EPI>
 cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
                         const GemmArgs& args, int grid, cudaStream_t s) {
     auto kern = grouped_gemm_kernel<EPI>;
-    static int configured[64] = {0};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 64 && !configured[dev]) {
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-        configured[dev] = 1;
-    }
+    static PerDeviceOnce smem_once;
+    if (const cudaError_t err = opt_in_smem(smem_once, kern, kSmemBytes); err != cudaSuccess)
+        return err;
     return launch_k(kern, grid, kThreads, kSmemBytes, s, a, b0, b1, args);
 }
 

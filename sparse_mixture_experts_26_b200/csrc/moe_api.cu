@@ -16,26 +16,31 @@
 namespace moe {
 
 int device_sm_count() {
-    static int cache[64] = {0};
+    static std::atomic<int> cache[64] = {};  // 0 = not yet read
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return 148;
-    if (dev >= 0 && dev < 64 && cache[dev] > 0) return cache[dev];
+    const bool tracked = dev >= 0 && dev < 64;
+    if (tracked) {
+        const int n = cache[dev].load(std::memory_order_relaxed);
+        if (n > 0) return n;
+    }
     int n = 0;
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
         n = 148;
-    if (dev >= 0 && dev < 64) cache[dev] = n;
+    if (tracked) cache[dev].store(n, std::memory_order_relaxed);
     return n;
 }
 
 namespace {
 thread_local bool t_pdl_scope = false;
+// Environment switches, read once (thread-safe static initialisation).
+bool env_is(const char* name, char c) {
+    const char* e = std::getenv(name);
+    return e && e[0] == c;
+}
 bool pdl_allowed() {
-    static int v = -1;
-    if (v < 0) {
-        const char* e = std::getenv("MOE_NO_PDL");
-        v = (e && e[0] == '1') ? 0 : 1;
-    }
-    return v == 1;
+    static const bool v = !env_is("MOE_NO_PDL", '1');
+    return v;
 }
 // Small batches (the weight-streaming FFN's range): every kernel but the FFN is short,
 // so overlapping launches pays off.
@@ -45,23 +50,15 @@ bool small_batch(int T) { return T <= kFusedMaxRows / 2; }
 bool pdl_enabled() { return t_pdl_scope && pdl_allowed(); }
 
 bool pair_gemm_enabled() {
-    static int v = -1;
-    if (v < 0) {
-        const char* e = std::getenv("MOE_GEMM_PAIR");
-        v = (e && e[0] == '0') ? 0 : 1;
-    }
-    return v == 1;
+    static const bool v = !env_is("MOE_GEMM_PAIR", '0');
+    return v;
 }
 PdlScope::PdlScope(bool on) : prev(t_pdl_scope) { t_pdl_scope = on; }
 PdlScope::~PdlScope() { t_pdl_scope = prev; }
 
 bool debug_sync_enabled() {
-    static int v = -1;
-    if (v < 0) {
-        const char* e = std::getenv("MOE_DEBUG_SYNC");
-        v = (e && e[0] == '1') ? 1 : 0;
-    }
-    return v == 1;
+    static const bool v = env_is("MOE_DEBUG_SYNC", '1');
+    return v;
 }
 
 namespace {

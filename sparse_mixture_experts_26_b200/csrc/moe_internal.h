@@ -4,6 +4,7 @@
 
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <climits>
 #include <cstddef>
 #include <cstdint>
@@ -14,6 +15,36 @@
 namespace moe {
 
 constexpr int kMaxExperts = 32;
+
+// One-time host setup per device, such as a kernel's opt-in to more than 48 KiB of
+// dynamic shared memory.  Thread-safe: threads that race may each run `fn` (it must be
+// idempotent); a call skips it only once some call of it has succeeded on that device.
+class PerDeviceOnce {
+  public:
+    template <typename Fn>
+    cudaError_t operator()(Fn&& fn) {
+        int dev = 0;
+        cudaError_t err = cudaGetDevice(&dev);
+        if (err != cudaSuccess) return err;
+        const bool tracked = dev >= 0 && dev < kDevices;
+        if (tracked && done_[dev].load(std::memory_order_acquire)) return cudaSuccess;
+        err = fn();
+        if (err == cudaSuccess && tracked) done_[dev].store(1, std::memory_order_release);
+        return err;
+    }
+
+  private:
+    static constexpr int kDevices = 64;
+    std::atomic<int> done_[kDevices] = {};
+};
+
+// Opt `kern` into `bytes` of dynamic shared memory on the current device, once.
+template <typename Kern>
+cudaError_t opt_in_smem(PerDeviceOnce& once, Kern kern, int bytes) {
+    return once([&] {
+        return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    });
+}
 // Tokens handled by one block of the permutation count / rank kernels.
 constexpr int kPermChunk = 256;
 

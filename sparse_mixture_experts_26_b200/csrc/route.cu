@@ -294,13 +294,9 @@ cudaError_t launch_route_t(const void* x, const void* Wg, int T, int d, int E, i
     const size_t wgt_bytes = static_cast<size_t>(8) * d * 2;
     if (sizeof(Tin) == 2 && MAXE == 8 && T > 64 && d % 32 == 0 && wgt_bytes <= 96 * 1024) {
         auto kern = route_dmma_kernel;
-        static int configured[64] = {0};
-        int dev = 0;
-        cudaGetDevice(&dev);
-        if (dev < 64 && !configured[dev]) {
-            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 96 * 1024);
-            configured[dev] = 1;
-        }
+        static PerDeviceOnce smem_once;
+        if (const cudaError_t err = opt_in_smem(smem_once, kern, 96 * 1024); err != cudaSuccess)
+            return err;
         const int blocks_needed = ((T + 7) / 8 + kMmaGroupsPerBlock - 1) / kMmaGroupsPerBlock;
         const int cap = 3 * device_sm_count();
         return launch_k(kern, blocks_needed < cap ? blocks_needed : cap, kRouteThreads, wgt_bytes,
