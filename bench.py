@@ -47,7 +47,7 @@ DOMINANT = {
     "pair": ("grouped_gemm_pair_kernel<SwiGLU> (CTA-pair GEMM1 + silu*gate epilogue)",
              "grouped_gemm_pair_swiglu", os.path.join(CSRC, "grouped_gemm_pair_sm100.cu")),
 }
-DECODE_MAX_TOKENS = 64    # the library switches to the weight-streaming kernels here
+DECODE_MAX_TOKENS = 128   # up to here the library runs the weight-streaming kernels
 PAIR_MIN_TOKENS = 1024    # ... and to the CTA-pair kernels here (2048 grouped rows)
 
 

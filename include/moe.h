@@ -175,7 +175,7 @@ moe_status moe_layer_forward_capacity(const void *x, const void *Wg, const void 
  * between its stages, for timing them without a profiler:
  *   events[0] before the router, events[1] after the permutation (before the
  *   expert FFN), events[2] after the first FFN kernel (GEMM1 + SwiGLU; for batches
- *   of at most 64 tokens, where one fused kernel runs both GEMMs, after it),
+ *   of at most 128 tokens, where one fused kernel runs both GEMMs, after it),
  *   events[3] after the expert FFN, events[4] after the combine.
  * n_events may be 0..5; events beyond n_events, and null handles, are not recorded. */
 moe_status moe_layer_forward_events(const void *x, const void *Wg, const void *W1,
