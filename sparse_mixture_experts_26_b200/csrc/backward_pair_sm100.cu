@@ -73,6 +73,7 @@ struct Book {
     int abort_flag;
     int off[kMaxExperts + 1];
     int end[kMaxExperts];
+    int poff[kMaxExperts + 1];  // first row of each expert in a padded operand
 };
 static_assert(sizeof(Book) <= 1024, "bookkeeping reserve");
 
@@ -89,6 +90,10 @@ struct PArgs {
     float* out1;
     uint32_t* status;
     int cap;
+    // 1: the operand (A or B) is a padded copy whose expert e starts at row poff[e]
+    // and has zero rows up to the next multiple of 64.  With either set, every K
+    // block takes the plain pair path (no partial blocks to clear).
+    int pad_a, pad_b;
 };
 
 // Bounded wait with cluster-scope acquire: pairs with the peer's cluster-scope release
@@ -171,9 +176,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             bk.off[g] = v;
             prev = v;
         }
+        bk.poff[0] = 0;
         for (int g = 0; g < E; ++g) {
             const int n = bk.off[g + 1] - bk.off[g];
             bk.end[g] = bk.off[g] + (n < args.cap ? n : args.cap);
+            bk.poff[g + 1] = bk.poff[g] + (n + kBK - 1) / kBK * kBK;
         }
     }
     tc_fence_before();
@@ -182,6 +189,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
 
     const uint32_t tmem_base = bk.tmem_base;
+    const bool padded = (args.pad_a | args.pad_b) != 0;
     const int per_e = args.m_pairs * args.n_tiles;
     const int total = E * per_e;
 
@@ -207,6 +215,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int nkb = (n_rows + kBK - 1) / kBK;
                 const int mcol = mp * 2 * kRows + static_cast<int>(rank) * kRows;
                 const int ncol = nt * kN + static_cast<int>(rank) * (kN / 2);
+                const int ra0 = args.pad_a ? bk.poff[e] : r0;  // first K row of A, of B
+                const int rb0 = args.pad_b ? bk.poff[e] : r0;
                 for (int kb = 0; kb < nkb; ++kb) {
                     if (!mbar_wait_bounded(&bk.empty[stage], phase ^ 1u, abort_flag,
                                            args.status)) {
@@ -214,10 +224,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                         break;
                     }
                     const int r = r0 + kb * kBK;
+                    const int ra = ra0 + kb * kBK, rb = rb0 + kb * kBK;
                     uint8_t* a = sA + stage * kABytes;
                     uint8_t* b = sB + stage * kBBytes;
                     const uint32_t bit = 1u << stage;
-                    if (n_rows - kb * kBK < kBK) {
+                    if (!padded && n_rows - kb * kBK < kBK) {
                         // partial block: land locally, the fix-up warp takes over
                         mbar_arrive_expect_tx(&bk.landed[stage], kStageBytes);
                         tma_load_2d(&tmA, &bk.landed[stage], a, mcol, r);
@@ -230,10 +241,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     } else {
                         const uint32_t full_leader = map_to_cta(smem_u32(&bk.full[stage]), 0);
                         if (leader) mbar_arrive_expect_tx(&bk.full[stage], 2 * kStageBytes);
-                        tma_load_2d_pair(&tmA, full_leader, a, mcol, r);
-                        tma_load_2d_pair(&tmA, full_leader, a + kBox, mcol + 64, r);
-                        tma_load_2d_pair(&tmB, full_leader, b, ncol, r);
-                        tma_load_2d_pair(&tmB, full_leader, b + kBox, ncol + 64, r);
+                        tma_load_2d_pair(&tmA, full_leader, a, mcol, ra);
+                        tma_load_2d_pair(&tmA, full_leader, a + kBox, mcol + 64, ra);
+                        tma_load_2d_pair(&tmB, full_leader, b, ncol, rb);
+                        tma_load_2d_pair(&tmB, full_leader, b + kBox, ncol + 64, rb);
                         pend_full |= bit;
                         pend_full_ph = (pend_full_ph & ~bit) | (phase << stage);
                     }
@@ -317,7 +328,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int nkb = (n_rows + kBK - 1) / kBK;
             for (int kb = 0; kb < nkb; ++kb) {
                 const int kv = n_rows - kb * kBK;  // rows of this block inside the group
-                if (kv < kBK) {
+                if (!padded && kv < kBK) {
                     const uint32_t bit = 1u << stage;
                     int got = 1;
                     if (lane == 0)
@@ -451,13 +462,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 cudaError_t launch_wgrad_pair(const CUtensorMap& A, const CUtensorMap& B, const CUtensorMap& O0,
                               const CUtensorMap& O1, const int32_t* offsets, int E, int rows,
                               int M, int N, int split, float* out0, float* out1, uint32_t* status,
-                              int cap, cudaStream_t s) {
+                              int cap, cudaStream_t s, int pad_a, int pad_b) {
     static PerDeviceOnce smem_once;
     if (const cudaError_t err = opt_in_smem(smem_once, bwd_wgrad_pair_kernel, kSmemBytes);
         err != cudaSuccess)
         return err;
-    PArgs p{offsets, E, rows, M, N, (M + 2 * kRows - 1) / (2 * kRows), (N + kN - 1) / kN, split,
-            out0, out1, status, cap};
+    PArgs p{offsets, E, rows, M, N, (M + 2 * kRows - 1) / (2 * kRows),
+            (N + kN - 1) / kN, split, out0, out1, status, cap, pad_a, pad_b};
     const long long tiles = static_cast<long long>(E) * p.m_pairs * p.n_tiles;
     const int max_pairs = device_sm_count() / 2;
     const int npairs = static_cast<int>(tiles < max_pairs ? (tiles < 1 ? 1 : tiles) : max_pairs);

@@ -52,7 +52,7 @@ cudaError_t launch_bwd_rows_pair(int mode, const CUtensorMap& a, const CUtensorM
 cudaError_t launch_wgrad_pair(const CUtensorMap& A, const CUtensorMap& B, const CUtensorMap& O0,
                               const CUtensorMap& O1, const int32_t* offsets, int E, int rows,
                               int M, int N, int split, float* out0, float* out1, uint32_t* status,
-                              int cap, cudaStream_t s);
+                              int cap, cudaStream_t s, int pad_a = 0, int pad_b = 0);
 
 namespace {
 
@@ -849,6 +849,49 @@ __global__ void __launch_bounds__(kPrepThreads)
     }
 }
 
+// Padded copies of two grouped bf16 arrays [rows, d]: expert e's n_e rows move to
+// row poff[e] = sum over g < e of round_up(n_g, 64) and are followed by zero rows up to
+// the next multiple of 64.  A weight-gradient GEMM that reads one operand this way finds
+// zeros in the rows past each expert's end, so every 64-row K block is a whole one.
+constexpr int kPadRowAlign = 64;
+
+__global__ void __launch_bounds__(kPrepThreads)
+    bwd_pad_kernel(const int32_t* __restrict__ offsets, int E, int rows, int d8,
+                   const uint4* __restrict__ src0, const uint4* __restrict__ src1,
+                   uint4* __restrict__ dst0, uint4* __restrict__ dst1) {
+    __shared__ int off[kMaxExperts + 1], poff[kMaxExperts + 1];
+    if (threadIdx.x == 0) {
+        int prev = 0;
+        poff[0] = 0;
+        for (int g = 0; g <= E; ++g) {
+            int v = offsets[g];
+            v = v < prev ? prev : (v > rows ? rows : v);
+            off[g] = v;
+            if (g > 0) {
+                const int n = v - prev;
+                poff[g] = poff[g - 1] + (n + kPadRowAlign - 1) / kPadRowAlign * kPadRowAlign;
+            }
+            prev = v;
+        }
+    }
+    __syncthreads();
+    for (int pr = blockIdx.x; pr < poff[E]; pr += gridDim.x) {
+        int e = 0;
+        while (e + 1 < E && pr >= poff[e + 1]) ++e;
+        const int i = pr - poff[e];
+        const bool data = i < off[e + 1] - off[e];
+        const size_t src = static_cast<size_t>(off[e] + i) * d8;
+        const size_t dst = static_cast<size_t>(pr) * d8;
+        for (int c = threadIdx.x; c < d8; c += blockDim.x) {
+            const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
+            const uint4 v0 = data ? src0[src + c] : zero;
+            const uint4 v1 = data ? src1[src + c] : zero;
+            dst0[dst + c] = v0;
+            dst1[dst + c] = v1;
+        }
+    }
+}
+
 // dWg = x^T dlogits in two deterministic passes: per chunk of kWgChunk tokens a
 // partial [d, E], then the partials summed in chunk order.
 constexpr int kWgChunk = 64;
@@ -1053,9 +1096,30 @@ cudaError_t launch_layer_backward(const BwdArgs& a, cudaStream_t s) {
                                      s, m_duv64, m_x64, m_dW1, m_dW3, w13);
         if (err != cudaSuccess || (err = mark(7)) != cudaSuccess) return err;
     } else {
+        // CTA pairs.  Without a capacity, one operand of each GEMM is read from a copy
+        // whose experts are padded with zero rows (dY for dW2, x_perm for dW1/dW3), so
+        // every K block is whole; the other operand's rows past an expert's end are the
+        // next expert's (finite) rows or outside the array (zero-filled by TMA).  With a
+        // capacity the dropped rows were never written, so the kernel clears the rows
+        // of partial blocks in shared memory instead.
+        const bool padded = a.cap == INT_MAX;
+        CUtensorMap m_dYp64, m_xp64;
+        if (padded) {
+            const unsigned pad_rows = static_cast<unsigned>(bwd_pad_rows(T, E));
+            if (!encode_bf16_2d(&m_dYp64, a.dY_pad, pad_rows, d, 64) ||
+                !encode_bf16_2d(&m_xp64, a.x_pad, pad_rows, d, 64))
+                return cudaErrorInvalidValue;
+            err = launch_k(bwd_pad_kernel, grid_for(static_cast<long long>(pad_rows), 8 * sms),
+                           kPrepThreads, 0, s, a.offsets, E, P, d / 8,
+                           static_cast<const uint4*>(a.dY), static_cast<const uint4*>(a.x_perm),
+                           static_cast<uint4*>(a.dY_pad), static_cast<uint4*>(a.x_pad));
+            if (err != cudaSuccess) return err;
+        }
         // A device that cannot co-schedule a CTA pair takes the single-SM kernel.
-        err = launch_wgrad_pair(m_dY64, m_H64, m_dW2, m_dW2, a.offsets, E, P, d, h, d, a.dW2,
-                                a.dW2, a.status, a.cap, s);
+        err = padded ? launch_wgrad_pair(m_dYp64, m_H64, m_dW2, m_dW2, a.offsets, E, P, d, h, d,
+                                         a.dW2, a.dW2, a.status, a.cap, s, 1, 0)
+                     : launch_wgrad_pair(m_dY64, m_H64, m_dW2, m_dW2, a.offsets, E, P, d, h, d,
+                                         a.dW2, a.dW2, a.status, a.cap, s);
         if (err != cudaSuccess) {
             cudaGetLastError();
             WArgs w{a.offsets, E, P, d, h, (d + kBM - 1) / kBM, (h + kN - 1) / kN, d, a.dW2,
@@ -1064,8 +1128,10 @@ cudaError_t launch_layer_backward(const BwdArgs& a, cudaStream_t s) {
                                         s, m_dY64, m_H64, m_dW2, m_dW2, w);
         }
         if (err != cudaSuccess || (err = mark(6)) != cudaSuccess) return err;
-        err = launch_wgrad_pair(m_duv64, m_x64, m_dW1, m_dW3, a.offsets, E, P, 2 * h, d, h, a.dW1,
-                                a.dW3, a.status, a.cap, s);
+        err = padded ? launch_wgrad_pair(m_duv64, m_xp64, m_dW1, m_dW3, a.offsets, E, P, 2 * h,
+                                         d, h, a.dW1, a.dW3, a.status, a.cap, s, 0, 1)
+                     : launch_wgrad_pair(m_duv64, m_x64, m_dW1, m_dW3, a.offsets, E, P, 2 * h,
+                                         d, h, a.dW1, a.dW3, a.status, a.cap, s);
         if (err != cudaSuccess) {
             cudaGetLastError();
             WArgs w{a.offsets, E, P, 2 * h, d, (2 * h + kBM - 1) / kBM, (d + kN - 1) / kN, h,

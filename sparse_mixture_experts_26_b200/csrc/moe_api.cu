@@ -115,7 +115,7 @@ T* at(void* ws, size_t off) {
 
 // Backward workspace regions (1 KiB aligned); the status word at offset 0.
 struct BwdLayout {
-    size_t status, dY, dw, dlogits, dH, DUV, dX, dwg_part, total;
+    size_t status, dY, dw, dlogits, dH, DUV, dX, dwg_part, dY_pad, x_pad, total;
 };
 
 BwdLayout bwd_layout(int T, int d, int h, int E) {
@@ -135,6 +135,8 @@ BwdLayout bwd_layout(int T, int d, int h, int E) {
     B.DUV = take(P * 2 * h * 2);
     B.dX = take(P * d * 4);
     B.dwg_part = take(bwd_dwg_chunks(T) * d * E * 4);
+    B.dY_pad = take(bwd_pad_rows(T, E) * d * 2);
+    B.x_pad = take(bwd_pad_rows(T, E) * d * 2);
     B.total = o;
     return B;
 }
@@ -409,6 +411,8 @@ moe_status layer_backward_impl(const void* x, const void* Wg, const void* W1, co
     a.DUV = at<void>(bwd_ws, B.DUV);
     a.dX = at<float>(bwd_ws, B.dX);
     a.dwg_part = at<float>(bwd_ws, B.dwg_part);
+    a.dY_pad = at<void>(bwd_ws, B.dY_pad);
+    a.x_pad = at<void>(bwd_ws, B.x_pad);
     a.status = at<uint32_t>(bwd_ws, B.status);
     a.ev = ev;
     a.n_ev = n_ev;

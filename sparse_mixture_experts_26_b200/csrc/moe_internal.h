@@ -238,6 +238,10 @@ struct BwdArgs {
     void* DUV;                 // bf16 [2T, 2h]: du then dv
     float* dX;                 // [2T, d]
     float* dwg_part;           // [bwd_dwg_chunks(T), d, E]
+    // bf16 [bwd_pad_rows(T, E), d]: dY and x_perm with each expert's rows padded by
+    // zero rows to a multiple of 64 (the weight-gradient GEMMs on CTA pairs)
+    void* dY_pad;
+    void* x_pad;
     uint32_t* status;
     // optional events recorded before the first launch and after each stage:
     // prep, dH, du/dv, dX, dx, dW2, dW1/dW3, dWg (null handles skipped)
@@ -245,6 +249,8 @@ struct BwdArgs {
     int n_ev;
 };
 size_t bwd_dwg_chunks(int T);
+// Rows of a grouped [2T, d] array once every expert's rows are padded to a multiple of 64.
+inline size_t bwd_pad_rows(int T, int E) { return 2 * static_cast<size_t>(T) + 64 * E; }
 cudaError_t launch_layer_backward(const BwdArgs& a, cudaStream_t s);
 // Bounded-wait self-test (see moe_selftest_wait_timeout).
 cudaError_t launch_selftest_wait(uint32_t* status, uint32_t* scratch, unsigned long long limit_ns,
