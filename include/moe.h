@@ -17,7 +17,8 @@
  *   All entry points are stateless and may be called from several host threads.
  * - Pointers are DEVICE pointers (cudaMalloc or equivalent) unless stated
  *   otherwise, 16-byte aligned, tensors dense and row-major.  Outputs must not
- *   alias inputs.
+ *   alias inputs.  Every pointer must belong to the device current on the calling
+ *   thread, and `stream` to that device: the kernels launch on the current device.
  * - Execution: work is queued on `stream` and runs asynchronously.  Argument
  *   errors are returned before anything is queued.  A failed launch returns
  *   MOE_ERR_CUDA.  Errors found on the device (a pipeline wait that ran out of

@@ -109,12 +109,53 @@ def _dt(t: torch.Tensor) -> int:
     raise TypeError(f"unsupported dtype {t.dtype} (bf16 or fp32)")
 
 
-def _dev(*ts: torch.Tensor) -> None:
+def _dev(*ts: torch.Tensor) -> torch.device:
+    """Check that the tensors are contiguous CUDA tensors on one device; return it.
+    The library launches on the current device, so every call runs under it."""
     for t in ts:
         if not t.is_cuda:
             raise ValueError("all tensors must be CUDA tensors")
         if not t.is_contiguous():
             raise ValueError("all tensors must be contiguous")
+    dev = ts[0].device
+    for t in ts[1:]:
+        if t.device != dev:
+            raise ValueError(f"tensors on different devices: {dev} and {t.device}")
+    return dev
+
+
+def _expect(name: str, t: torch.Tensor, shape, dtype=None) -> None:
+    """The C ABI receives bare pointers: shapes and dtypes are checked here."""
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name}: dtype {t.dtype}, expected {dtype}")
+
+
+def _expect_numel(name: str, t: torch.Tensor, n: int, dtype) -> None:
+    if t.numel() != n:
+        raise ValueError(f"{name}: {t.numel()} elements, expected {n}")
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: dtype {t.dtype}, expected {dtype}")
+
+
+def _layer_dims(x, Wg, W1, W3, W2):
+    """T, d, h, E of a layer call, after checking every operand against them."""
+    if x.dim() != 2 or W1.dim() != 3:
+        raise ValueError("x must be [T, d] and W1 [E, h, d]")
+    T, d = x.shape
+    E, h, _ = W1.shape
+    _dt(x)
+    _expect("Wg", Wg, (d, E), x.dtype)
+    _expect("W1", W1, (E, h, d), x.dtype)
+    _expect("W3", W3, (E, h, d), x.dtype)
+    _expect("W2", W2, (E, d, h), x.dtype)
+    return T, d, h, E
+
+
+def _ws(name: str, ws: torch.Tensor) -> None:
+    if ws.dtype != torch.uint8 or ws.dim() != 1:
+        raise TypeError(f"{name}: expected a 1-D uint8 tensor")
 
 
 def _ptr(t: torch.Tensor | None) -> int | None:
@@ -149,79 +190,116 @@ def alloc_workspace(T: int, d: int, h: int, E: int = 8, k: int = 2,
 
 
 def moe_route(x, Wg, topk_idx, topk_w, k: int = 2, stream=None) -> None:
-    _dev(x, Wg, topk_idx, topk_w)
     T, d = x.shape
     E = Wg.shape[1]
-    _check("moe_route", _lib.moe_route(_ptr(x), _ptr(Wg), T, d, E, k, _dt(x), _ptr(topk_idx),
-                                       _ptr(topk_w), _stream(stream)))
+    _expect("Wg", Wg, (d, E), x.dtype)
+    _expect("topk_idx", topk_idx, (T, k), torch.int32)
+    _expect("topk_w", topk_w, (T, k), torch.float32)
+    dev = _dev(x, Wg, topk_idx, topk_w)
+    with torch.cuda.device(dev):
+        _check("moe_route", _lib.moe_route(_ptr(x), _ptr(Wg), T, d, E, k, _dt(x),
+                                           _ptr(topk_idx), _ptr(topk_w), _stream(stream)))
 
 
 def moe_permute(topk_idx, x, offsets, perm_token, inv_perm, x_perm, ws, E: int, k: int = 2,
                 stream=None) -> None:
-    _dev(topk_idx, x, offsets, perm_token, inv_perm, x_perm, ws)
     T, d = x.shape
-    _check("moe_permute", _lib.moe_permute(
-        _ptr(topk_idx), _ptr(x), T, d, E, k, _dt(x), _ptr(offsets), _ptr(perm_token),
-        _ptr(inv_perm), _ptr(x_perm), _ptr(ws), ws.numel() * ws.element_size(),
-        _stream(stream)))
+    _expect("topk_idx", topk_idx, (T, k), torch.int32)
+    _expect_numel("offsets", offsets, E + 1, torch.int32)
+    _expect_numel("perm_token", perm_token, T * k, torch.int32)
+    _expect_numel("inv_perm", inv_perm, T * k, torch.int32)
+    _expect("x_perm", x_perm, (T * k, d), x.dtype)
+    _ws("ws", ws)
+    dev = _dev(topk_idx, x, offsets, perm_token, inv_perm, x_perm, ws)
+    with torch.cuda.device(dev):
+        _check("moe_permute", _lib.moe_permute(
+            _ptr(topk_idx), _ptr(x), T, d, E, k, _dt(x), _ptr(offsets), _ptr(perm_token),
+            _ptr(inv_perm), _ptr(x_perm), _ptr(ws), ws.numel() * ws.element_size(),
+            _stream(stream)))
+
+
+def _ffn_dims(x_perm, offsets, W1, W3, W2, y_perm):
+    rows, d = x_perm.shape
+    E, h, _ = W1.shape
+    _dt(x_perm)
+    _expect_numel("offsets", offsets, E + 1, torch.int32)
+    _expect("W1", W1, (E, h, d), x_perm.dtype)
+    _expect("W3", W3, (E, h, d), x_perm.dtype)
+    _expect("W2", W2, (E, d, h), x_perm.dtype)
+    _expect("y_perm", y_perm, (rows, d), torch.float32)
+    return rows, d, h, E
 
 
 def moe_expert_ffn(x_perm, offsets, W1, W3, W2, y_perm, ws, stream=None) -> None:
-    _dev(x_perm, offsets, W1, W3, W2, y_perm, ws)
-    rows, d = x_perm.shape
-    E, h, _ = W1.shape
-    _check("moe_expert_ffn", _lib.moe_expert_ffn(
-        _ptr(x_perm), _ptr(offsets), _ptr(W1), _ptr(W3), _ptr(W2), rows, d, h, E, _dt(x_perm),
-        _ptr(y_perm), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
+    rows, d, h, E = _ffn_dims(x_perm, offsets, W1, W3, W2, y_perm)
+    _ws("ws", ws)
+    dev = _dev(x_perm, offsets, W1, W3, W2, y_perm, ws)
+    with torch.cuda.device(dev):
+        _check("moe_expert_ffn", _lib.moe_expert_ffn(
+            _ptr(x_perm), _ptr(offsets), _ptr(W1), _ptr(W3), _ptr(W2), rows, d, h, E,
+            _dt(x_perm), _ptr(y_perm), _ptr(ws), ws.numel() * ws.element_size(),
+            _stream(stream)))
 
 
 def moe_combine(y_perm, inv_perm, topk_w, y, k: int = 2, stream=None) -> None:
-    _dev(y_perm, inv_perm, topk_w, y)
     T, d = y.shape
-    _check("moe_combine", _lib.moe_combine(_ptr(y_perm), _ptr(inv_perm), _ptr(topk_w), T, d, k,
-                                           _dt(y), _ptr(y), _stream(stream)))
+    _expect("y_perm", y_perm, (T * k, d), torch.float32)
+    _expect_numel("inv_perm", inv_perm, T * k, torch.int32)
+    _expect_numel("topk_w", topk_w, T * k, torch.float32)
+    dev = _dev(y_perm, inv_perm, topk_w, y)
+    with torch.cuda.device(dev):
+        _check("moe_combine", _lib.moe_combine(_ptr(y_perm), _ptr(inv_perm), _ptr(topk_w), T, d,
+                                               k, _dt(y), _ptr(y), _stream(stream)))
 
 
 def moe_layer_forward(x, Wg, W1, W3, W2, y, ws, k: int = 2, stream=None) -> None:
-    _dev(x, Wg, W1, W3, W2, y, ws)
-    T, d = x.shape
-    E, h, _ = W1.shape
-    _check("moe_layer_forward", _lib.moe_layer_forward(
-        _ptr(x), _ptr(Wg), _ptr(W1), _ptr(W3), _ptr(W2), T, d, h, E, k, _dt(x), _ptr(y),
-        _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
+    T, d, h, E = _layer_dims(x, Wg, W1, W3, W2)
+    _expect("y", y, (T, d), x.dtype)
+    _ws("ws", ws)
+    dev = _dev(x, Wg, W1, W3, W2, y, ws)
+    with torch.cuda.device(dev):
+        _check("moe_layer_forward", _lib.moe_layer_forward(
+            _ptr(x), _ptr(Wg), _ptr(W1), _ptr(W3), _ptr(W2), T, d, h, E, k, _dt(x), _ptr(y),
+            _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
 
 
 def moe_layer_forward_capacity(x, Wg, W1, W3, W2, y, ws, capacity: int, k: int = 2,
                                stream=None) -> None:
     """The layer with each expert keeping at most ``capacity`` (token, slot) pairs, in
     token order; dropped pairs contribute nothing.  ``capacity < 0``: no limit."""
-    _dev(x, Wg, W1, W3, W2, y, ws)
-    T, d = x.shape
-    E, h, _ = W1.shape
-    _check("moe_layer_forward_capacity", _lib.moe_layer_forward_capacity(
-        _ptr(x), _ptr(Wg), _ptr(W1), _ptr(W3), _ptr(W2), T, d, h, E, k, _dt(x), int(capacity),
-        _ptr(y), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
+    T, d, h, E = _layer_dims(x, Wg, W1, W3, W2)
+    _expect("y", y, (T, d), x.dtype)
+    _ws("ws", ws)
+    dev = _dev(x, Wg, W1, W3, W2, y, ws)
+    with torch.cuda.device(dev):
+        _check("moe_layer_forward_capacity", _lib.moe_layer_forward_capacity(
+            _ptr(x), _ptr(Wg), _ptr(W1), _ptr(W3), _ptr(W2), T, d, h, E, k, _dt(x),
+            int(capacity), _ptr(y), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
 
 
 def moe_layer_forward_events(x, Wg, W1, W3, W2, y, ws, events, k: int = 2,
                              stream=None) -> None:
     """``moe_layer_forward`` recording ``events`` (up to 5 created handles, or None to skip
     one) between its stages."""
-    _dev(x, Wg, W1, W3, W2, y, ws)
-    T, d = x.shape
-    E, h, _ = W1.shape
+    T, d, h, E = _layer_dims(x, Wg, W1, W3, W2)
+    _expect("y", y, (T, d), x.dtype)
+    _ws("ws", ws)
+    dev = _dev(x, Wg, W1, W3, W2, y, ws)
     handles = (ctypes.c_void_p * max(1, len(events)))(*[int(e) if e else None for e in events])
-    _check("moe_layer_forward_events", _lib.moe_layer_forward_events(
-        _ptr(x), _ptr(Wg), _ptr(W1), _ptr(W3), _ptr(W2), T, d, h, E, k, _dt(x), _ptr(y),
-        _ptr(ws), ws.numel() * ws.element_size(), ctypes.addressof(handles), len(events),
-        _stream(stream)))
+    with torch.cuda.device(dev):
+        _check("moe_layer_forward_events", _lib.moe_layer_forward_events(
+            _ptr(x), _ptr(Wg), _ptr(W1), _ptr(W3), _ptr(W2), T, d, h, E, k, _dt(x), _ptr(y),
+            _ptr(ws), ws.numel() * ws.element_size(), ctypes.addressof(handles), len(events),
+            _stream(stream)))
 
 
 def moe_device_status(ws, stream=None) -> int:
     """Synchronise, return and clear the workspace's device status flags."""
+    dev = _dev(ws)
     flags = ctypes.c_uint32(0)
-    code = _lib.moe_device_status(_ptr(ws), ws.numel() * ws.element_size(),
-                                  ctypes.addressof(flags), _stream(stream))
+    with torch.cuda.device(dev):
+        code = _lib.moe_device_status(_ptr(ws), ws.numel() * ws.element_size(),
+                                      ctypes.addressof(flags), _stream(stream))
     if code not in (0, 5):
         _check("moe_device_status", code)
     return int(flags.value)
@@ -231,21 +309,23 @@ def moe_expert_ffn_static(x_perm, offsets, W1, W3, W2, y_perm, stream=None) -> N
     """``moe_expert_ffn`` without a workspace, for callers that cannot allocate device
     memory: the scratch is a fixed 8 MiB array inside the library (see include/moe.h
     for the size limit, the first-call set-up and why overlapping calls race)."""
-    _dev(x_perm, offsets, W1, W3, W2, y_perm)
-    rows, d = x_perm.shape
-    E, h, _ = W1.shape
-    _check("moe_expert_ffn_static", _lib.moe_expert_ffn_static(
-        _ptr(x_perm), _ptr(offsets), _ptr(W1), _ptr(W3), _ptr(W2), rows, d, h, E, _dt(x_perm),
-        _ptr(y_perm), _stream(stream)))
+    rows, d, h, E = _ffn_dims(x_perm, offsets, W1, W3, W2, y_perm)
+    dev = _dev(x_perm, offsets, W1, W3, W2, y_perm)
+    with torch.cuda.device(dev):
+        _check("moe_expert_ffn_static", _lib.moe_expert_ffn_static(
+            _ptr(x_perm), _ptr(offsets), _ptr(W1), _ptr(W3), _ptr(W2), rows, d, h, E,
+            _dt(x_perm), _ptr(y_perm), _stream(stream)))
 
 
 def moe_selftest_wait_timeout(ws, limit_seconds: float = 0.05, stream=None):
     """Run the bounded-wait self-test; returns (barrier outcome, counter outcome), each 2
     when the wait gave up as it must.  The timeout flag is left in the status word."""
+    dev = _dev(ws)
     out = (ctypes.c_uint32 * 2)()
-    _check("moe_selftest_wait_timeout", _lib.moe_selftest_wait_timeout(
-        _ptr(ws), ws.numel() * ws.element_size(), float(limit_seconds), ctypes.addressof(out),
-        _stream(stream)))
+    with torch.cuda.device(dev):
+        _check("moe_selftest_wait_timeout", _lib.moe_selftest_wait_timeout(
+            _ptr(ws), ws.numel() * ws.element_size(), float(limit_seconds),
+            ctypes.addressof(out), _stream(stream)))
     return int(out[0]), int(out[1])
 
 
@@ -275,34 +355,47 @@ def alloc_backward_workspace(T: int, d: int, h: int, E: int = 8, k: int = 2,
     return torch.zeros(n, dtype=torch.uint8, device=device)
 
 
+def _backward_dims(x, Wg, W1, W3, W2, dy, dx, dWg, dW1, dW3, dW2, fwd_ws, bwd_ws):
+    T, d, h, E = _layer_dims(x, Wg, W1, W3, W2)
+    _expect("dy", dy, (T, d), x.dtype)
+    _expect("dx", dx, (T, d), x.dtype)
+    _expect("dWg", dWg, (d, E), torch.float32)
+    _expect("dW1", dW1, (E, h, d), torch.float32)
+    _expect("dW3", dW3, (E, h, d), torch.float32)
+    _expect("dW2", dW2, (E, d, h), torch.float32)
+    _ws("fwd_ws", fwd_ws)
+    _ws("bwd_ws", bwd_ws)
+    return T, d, h, E
+
+
 def moe_layer_backward(x, Wg, W1, W3, W2, dy, dx, dWg, dW1, dW3, dW2, fwd_ws, bwd_ws,
                        capacity: int = -1, k: int = 2, stream=None) -> None:
     """Gradients of the layer for upstream gradient ``dy``; ``fwd_ws`` is the workspace
     of the forward call on the same inputs (``capacity`` as given to it, -1 for none)."""
-    _dev(x, Wg, W1, W3, W2, dy, dx, dWg, dW1, dW3, dW2, fwd_ws, bwd_ws)
-    T, d = x.shape
-    E, h, _ = W1.shape
-    _check("moe_layer_backward", _lib.moe_layer_backward(
-        _ptr(x), _ptr(Wg), _ptr(W1), _ptr(W3), _ptr(W2), _ptr(dy), T, d, h, E, k, _dt(x),
-        int(capacity), _ptr(dx), _ptr(dWg), _ptr(dW1), _ptr(dW3), _ptr(dW2), _ptr(fwd_ws),
-        fwd_ws.numel() * fwd_ws.element_size(), _ptr(bwd_ws),
-        bwd_ws.numel() * bwd_ws.element_size(), _stream(stream)))
+    T, d, h, E = _backward_dims(x, Wg, W1, W3, W2, dy, dx, dWg, dW1, dW3, dW2, fwd_ws, bwd_ws)
+    dev = _dev(x, Wg, W1, W3, W2, dy, dx, dWg, dW1, dW3, dW2, fwd_ws, bwd_ws)
+    with torch.cuda.device(dev):
+        _check("moe_layer_backward", _lib.moe_layer_backward(
+            _ptr(x), _ptr(Wg), _ptr(W1), _ptr(W3), _ptr(W2), _ptr(dy), T, d, h, E, k, _dt(x),
+            int(capacity), _ptr(dx), _ptr(dWg), _ptr(dW1), _ptr(dW3), _ptr(dW2), _ptr(fwd_ws),
+            fwd_ws.numel() * fwd_ws.element_size(), _ptr(bwd_ws),
+            bwd_ws.numel() * bwd_ws.element_size(), _stream(stream)))
 
 
 def moe_layer_backward_events(x, Wg, W1, W3, W2, dy, dx, dWg, dW1, dW3, dW2, fwd_ws, bwd_ws,
                               events, capacity: int = -1, k: int = 2, stream=None) -> None:
     """``moe_layer_backward`` recording ``events`` (up to 9 created handles, or None to
     skip one) before its first launch and after each stage."""
-    _dev(x, Wg, W1, W3, W2, dy, dx, dWg, dW1, dW3, dW2, fwd_ws, bwd_ws)
-    T, d = x.shape
-    E, h, _ = W1.shape
+    T, d, h, E = _backward_dims(x, Wg, W1, W3, W2, dy, dx, dWg, dW1, dW3, dW2, fwd_ws, bwd_ws)
+    dev = _dev(x, Wg, W1, W3, W2, dy, dx, dWg, dW1, dW3, dW2, fwd_ws, bwd_ws)
     handles = (ctypes.c_void_p * max(1, len(events)))(*[int(e) if e else None for e in events])
-    _check("moe_layer_backward_events", _lib.moe_layer_backward_events(
-        _ptr(x), _ptr(Wg), _ptr(W1), _ptr(W3), _ptr(W2), _ptr(dy), T, d, h, E, k, _dt(x),
-        int(capacity), _ptr(dx), _ptr(dWg), _ptr(dW1), _ptr(dW3), _ptr(dW2), _ptr(fwd_ws),
-        fwd_ws.numel() * fwd_ws.element_size(), _ptr(bwd_ws),
-        bwd_ws.numel() * bwd_ws.element_size(), ctypes.addressof(handles), len(events),
-        _stream(stream)))
+    with torch.cuda.device(dev):
+        _check("moe_layer_backward_events", _lib.moe_layer_backward_events(
+            _ptr(x), _ptr(Wg), _ptr(W1), _ptr(W3), _ptr(W2), _ptr(dy), T, d, h, E, k, _dt(x),
+            int(capacity), _ptr(dx), _ptr(dWg), _ptr(dW1), _ptr(dW3), _ptr(dW2), _ptr(fwd_ws),
+            fwd_ws.numel() * fwd_ws.element_size(), _ptr(bwd_ws),
+            bwd_ws.numel() * bwd_ws.element_size(), ctypes.addressof(handles), len(events),
+            _stream(stream)))
 
 
 def layer_backward(x, Wg, W1, W3, W2, dy, fwd_ws, capacity: int = -1, bwd_ws=None):
