@@ -48,7 +48,7 @@ DOMINANT = {
              "grouped_gemm_pair_swiglu", os.path.join(CSRC, "grouped_gemm_pair_sm100.cu")),
 }
 DECODE_MAX_TOKENS = 128   # up to here the library runs the weight-streaming kernels
-PAIR_MIN_TOKENS = 1024    # ... and to the CTA-pair kernels here (2048 grouped rows)
+PAIR_MIN_TOKENS = 512     # ... and to the CTA-pair kernels here (1024 grouped rows)
 
 
 # ------------------------------------------------------------------ ranks

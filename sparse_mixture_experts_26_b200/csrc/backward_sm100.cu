@@ -1023,7 +1023,7 @@ cudaError_t launch_layer_backward(const BwdArgs& a, cudaStream_t s) {
         return cudaErrorInvalidValue;
     const long long row_blocks = (static_cast<long long>(P) + 127LL * E) / kBM;
     // Many rows: the CTA-pair forms of the three row GEMMs (the forward's pair engine).
-    const bool pairs = P >= kPairMinRows && pair_gemm_enabled();
+    const bool pairs = P >= kBwdPairMinRows && pair_gemm_enabled();
 
     // 2. dH = dY W2_e
     if (pairs) {

@@ -12,7 +12,7 @@ pytestmark = pytest.mark.gpu
 
 def _kernel_names(fn):
     from torch.profiler import ProfilerActivity, profile
-    with profile(activities=[ProfilerActivity.CUDA]) as prof:
+    with profile(activities=[ProfilerActivity.CUDA], acc_events=True) as prof:
         fn()
         torch.cuda.synchronize()
     return [e.name for e in prof.events()
