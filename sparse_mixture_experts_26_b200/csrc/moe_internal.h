@@ -180,7 +180,7 @@ cudaError_t launch_ffn_bf16_pair(const void* x_perm, const int32_t* offsets, con
 // Grouped rows from which the CTA-pair kernels are used (MOE_GEMM_PAIR=0 disables them):
 // the forward's expert FFN, and the backward's row-grouped GEMMs.
 constexpr int kPairMinRows = 1024;
-constexpr int kBwdPairMinRows = 2048;
+constexpr int kBwdPairMinRows = 1024;
 bool pair_gemm_enabled();
 // Small-batch expert FFN as one cooperative launch (gate/up and split-K down units
 // with per-(expert, K range) dependency counters, 2*E*ksplit zeroed words).
