@@ -658,7 +658,7 @@ def run_ours_backward(args):
                                                "saved state)",
                                        "parallelism": f"replicas x{world}"}),
         "roofline": roofline, "layer": layer, "cpu_baseline": cpu_baseline, "e2e": e2e,
-        "gpu_launches": 9 * K, "clocks": clocks.summary(),
+        "gpu_launches": moe.launches_per_backward(T) * K, "clocks": clocks.summary(),
     }
 
 

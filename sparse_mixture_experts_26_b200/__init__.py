@@ -22,7 +22,7 @@ __all__ = [
     "LIB_PATH", "MoeError", "moe_workspace_bytes", "moe_route", "moe_permute",
     "moe_expert_ffn", "moe_combine", "moe_layer_forward", "moe_device_status",
     "moe_status_string", "moe_layer_forward_events", "alloc_workspace", "layer_forward",
-    "EXPORTED_SYMBOLS", "launches_per_layer", "moe_expert_ffn_static",
+    "EXPORTED_SYMBOLS", "launches_per_layer", "launches_per_backward", "moe_expert_ffn_static",
     "moe_layer_forward_capacity", "moe_selftest_wait_timeout", "moe_backward_workspace_bytes",
     "moe_layer_backward", "alloc_backward_workspace", "layer_backward",
     "moe_layer_backward_events",
@@ -42,8 +42,20 @@ EXPORTED_SYMBOLS = ("moe_workspace_bytes", "moe_route", "moe_permute", "moe_expe
 def launches_per_layer(T: int) -> int:
     """Kernels one moe_layer_forward queues: router 1, permutation 1 (T <= 512) or 4
     (count, scan, rank, gather), expert FFN 1 (T <= 128: gate/up and down fused) or 2,
-    combine 1."""
+    combine 1; none for T == 0."""
+    if T <= 0:
+        return 0
     return 1 + (1 if T <= 512 else 4) + (1 if T <= 128 else 2) + 1
+
+
+def launches_per_backward(T: int, capacity: int = -1) -> int:
+    """Kernels one moe_layer_backward queues: prep, dH, du/dv, dX, dx, the two
+    weight-gradient GEMMs, the dWg partials and their sum (9), plus the padded copies
+    of dY and x_perm when the weight gradients run on CTA pairs (more than 1024
+    grouped rows) without a capacity; none for T == 0."""
+    if T <= 0:
+        return 0
+    return 9 + (1 if 2 * T > 1024 and capacity < 0 else 0)
 
 
 class MoeError(RuntimeError):
