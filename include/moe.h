@@ -28,7 +28,8 @@
  *   cores) or MOE_F32 (fp32 everywhere, CUDA cores, no TF32).
  * - Supported shapes: k == 2; 2 <= E <= 32 (moe_expert_ffn, which routes nothing,
  *   also takes E == 1); d and h multiples of 8; T >= 0 (T == 0 is a no-op returning
- *   MOE_OK).  Inputs must be finite.
+ *   MOE_OK); T <= 2^29, and E*d, E*h below 2^31 (32-bit row coordinates).  Inputs
+ *   must be finite.
  * - Routing: experts are ranked by (logit descending, index ascending), so ties go
  *   to the lower index; logits are accumulated in fp64 from the exact products of
  *   the inputs.  Slot 0 holds the larger logit.  w1 = 1/(1+exp(l_i2-l_i1)) is

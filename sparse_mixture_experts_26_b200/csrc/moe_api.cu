@@ -81,9 +81,13 @@ moe_status check_shape(int T, int d, int h, int E, int k, moe_dtype dt, bool nee
     if (dt != MOE_F32 && dt != MOE_BF16) return MOE_ERR_INVALID_ARG;
     if (k != 2 || E < (routed ? 2 : 1) || E > kMaxExperts) return MOE_ERR_UNSUPPORTED;
     if (d % 8 != 0 || (need_h && h % 8 != 0)) return MOE_ERR_UNSUPPORTED;
-    // 32-bit row indices and element offsets inside one grouped buffer.
+    // 32-bit row indices inside one grouped buffer (element offsets are 64-bit), and
+    // 32-bit row coordinates in the flattened weight views [E*h, d] and [E*d, h].
     const long long P = 2LL * T;
     if (P * d >= (1LL << 40) || (need_h && P * h >= (1LL << 40)) || T > (1 << 29))
+        return MOE_ERR_UNSUPPORTED;
+    if (static_cast<long long>(E) * d >= (1LL << 31) ||
+        (need_h && static_cast<long long>(E) * h >= (1LL << 31)))
         return MOE_ERR_UNSUPPORTED;
     return MOE_OK;
 }

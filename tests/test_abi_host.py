@@ -74,6 +74,10 @@ def test_workspace_sizes(lib):
     assert lib.moe_workspace_bytes(16, 4095, h, 8, 2, BF16) == 0   # d % 8
     assert lib.moe_workspace_bytes(16, d, h, 33, 2, BF16) == 0     # E > 32
     assert lib.moe_workspace_bytes(-1, d, h, 8, 2, BF16) == 0
+    # the flattened weight views [E*h, d] / [E*d, h] need 32-bit row coordinates
+    assert lib.moe_workspace_bytes(1, 64, 1 << 26, 32, 2, BF16) == 0
+    assert lib.moe_workspace_bytes(1, 1 << 26, 64, 32, 2, BF16) == 0
+    assert lib.moe_workspace_bytes(1, 64, (1 << 26) - 8, 32, 2, BF16) > 0
 
 
 @pytest.mark.parametrize("d,h,dt", [(4096, 14336, BF16), (136, 192, BF16), (24, 40, 0)])
