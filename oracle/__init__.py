@@ -34,3 +34,29 @@ def loops_layer(x, Wg, W1, W3, W2):
     if rc != 0:
         raise ValueError("moe_oracle_loops rejected its arguments")
     return idx, w, y
+
+
+def loops_layer_backward(x, Wg, W1, W3, W2, dy):
+    """Run the plain-C loop backward (O3); returns ``(dx, dWg, dW1, dW3, dW2)`` in fp64."""
+    import ctypes
+
+    import numpy as np
+
+    from .build_oracle import build
+
+    lib = ctypes.CDLL(build())
+    f = lib.moe_oracle_loops_backward
+    dp = ctypes.POINTER(ctypes.c_double)
+    f.argtypes = [dp] * 6 + [ctypes.c_int] * 4 + [dp] * 5
+    f.restype = ctypes.c_int
+    arrs = [np.ascontiguousarray(a, dtype=np.float64) for a in (x, Wg, W1, W3, W2, dy)]
+    T, d = arrs[0].shape
+    E = arrs[1].shape[1]
+    h = arrs[2].shape[1]
+    outs = [np.zeros(s, dtype=np.float64) for s in ((T, d), (d, E), (E, h, d), (E, h, d),
+                                                     (E, d, h))]
+    rc = f(*[a.ctypes.data_as(dp) for a in arrs], T, d, h, E,
+           *[o.ctypes.data_as(dp) for o in outs])
+    if rc != 0:
+        raise ValueError("moe_oracle_loops_backward rejected its arguments")
+    return tuple(outs)

@@ -484,3 +484,39 @@ def test_backward_invariants():
     counts = np.bincount(g1["fwd"]["idx"].ravel(), minlength=8)
     for e in np.flatnonzero(counts == 0):
         assert not g1["dW1"][e].any() and not g1["dW2"][e].any()
+
+
+@pytest.mark.parametrize("T,d,h,E,kind", [(1, 8, 16, 8, "plain"), (37, 24, 40, 8, "skew"),
+                                          (64, 16, 24, 8, "long"), (29, 16, 8, 4, "plain")])
+def test_backward_routed_equals_loops(T, d, h, E, kind):
+    """O1 (grouped by expert, NumPy) against O3 (per token, plain C loops written from
+    the chain rule), which shares no code or data layout with it."""
+    inp = _inputs(small("bwl", T=T, d=d, h=h, E=E, seed=70 + T, kind=kind))
+    dy = np.random.default_rng(T + 1).normal(size=(T, d))
+    g = O.moe_layer_backward(**inp, dy=dy)
+    loops = dict(zip(("dx", "dWg", "dW1", "dW3", "dW2"), oracle.loops_layer_backward(**inp, dy=dy)))
+    for k, v in loops.items():
+        scale = max(np.abs(v).max(), 1e-300)
+        assert np.abs(g[k] - v).max() <= 1e-12 * scale, k
+
+
+def test_loops_backward_matches_finite_differences():
+    """The C loops on their own, against central differences of the C forward."""
+    inp, dy = _fd_case(seed=4)
+    names = ("x", "Wg", "W1", "W3", "W2")
+    got = dict(zip(("d" + n for n in names), oracle.loops_layer_backward(**inp, dy=dy)))
+    eps = 1e-6
+
+    def loss(args):
+        return float((oracle.loops_layer(*args)[2] * dy).sum())
+
+    for i, n in enumerate(names):
+        A = inp[n]
+        fd = np.zeros_like(A)
+        for ix in np.ndindex(A.shape):
+            plus = [inp[m].copy() for m in names]
+            minus = [inp[m].copy() for m in names]
+            plus[i][ix] += eps
+            minus[i][ix] -= eps
+            fd[ix] = (loss(plus) - loss(minus)) / (2 * eps)
+        np.testing.assert_allclose(got["d" + n], fd, rtol=0, atol=1e-7 * np.abs(fd).max())
