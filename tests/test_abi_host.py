@@ -177,3 +177,42 @@ def test_backward_validation(lib):
     # the events variant checks its event array too
     assert L.moe_layer_backward_events(p, p, p, p, p, p, T, d, h, E, 2, BF16, -1, p, p, p, p,
                                        p, p, fw, p, bw, None, 3, None) == INVALID
+
+
+C_PROGRAM = r"""
+#include <stdio.h>
+#include "moe.h"
+
+int main(void) {
+    size_t n = moe_workspace_bytes(16, 4096, 14336, 8, 2, MOE_BF16);
+    size_t bad = moe_workspace_bytes(16, 4096, 14336, 8, 3, MOE_BF16);
+    moe_status st = moe_route(NULL, NULL, 4, 64, 8, 2, MOE_BF16, NULL, NULL, 0);
+    printf("%zu %zu %d %s\n", n, bad, (int)st, moe_status_string(MOE_ERR_WORKSPACE));
+    return 0;
+}
+"""
+
+
+def test_header_compiles_as_c_and_links(lib, tmp_path):
+    """A plain C program (not C++; C11, which the CUDA runtime header itself needs for
+    its anonymous unions) includes the header, links against libmoe.so and calls the
+    host-only entry points."""
+    import shutil
+    import subprocess
+    cuda_inc = os.path.join(os.environ.get("CUDA_HOME", "/usr/local/cuda"), "include")
+    if shutil.which("gcc") is None or not os.path.exists(
+            os.path.join(cuda_inc, "cuda_runtime_api.h")):
+        pytest.skip("gcc or the CUDA headers are not available")
+    src = tmp_path / "abi.c"
+    src.write_text(C_PROGRAM)
+    exe = tmp_path / "abi"
+    libdir = os.path.join(ROOT, "sparse_mixture_experts_26_b200")
+    subprocess.run(["gcc", "-std=c11", "-Wall", "-Werror", "-pedantic",
+                    "-I", os.path.join(ROOT, "include"), "-I", cuda_inc, str(src),
+                    "-L", libdir, "-lmoe", f"-Wl,-rpath,{libdir}", "-o", str(exe)],
+                   check=True, capture_output=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split()
+    assert int(out[0]) == lib.moe_workspace_bytes(16, 4096, 14336, 8, 2, BF16) > 0
+    assert int(out[1]) == 0
+    assert int(out[2]) == INVALID
+    assert " ".join(out[3:]) == lib.moe_status_string(WORKSPACE).decode()
