@@ -2,11 +2,15 @@
 """Benchmark of the Mixtral top-2 sparse-MoE layer on B200 through libmoe's C ABI.
 
 One step = one moe_layer_forward over one batch of the workload (router, grouping,
-expert SwiGLU FFN on tensor cores, combine).  Default workload: the decode batch of
-the Mixtral-8x7B layer (T=16, d=4096, h=14336, E=8, k=2, bf16), which streams every
-touched expert's weights from HBM; ``--workload prefill`` etc. select the others.
+expert SwiGLU FFN on tensor cores, combine).  The default run's headline is the
+prefill batch of the Mixtral-8x7B layer (T=4096, d=4096, h=14336, E=8, k=2, bf16),
+whose GEMM1 (+SwiGLU) is reported against the bf16 tensor-core peak; the decode
+batch (T=16, weight streaming against HBM bandwidth), the skewed-routing and
+long-context (T=32768) layers and the prefill backward pass are then timed under
+the same rules and reported under ``workloads`` in the same line.
+``--workload NAME`` times one workload only.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--backward]
     python bench.py --impl reference ...     # the CPU oracle, timed on host cores
 
 Under torchrun (N > 1) every rank runs its own batch with replicated weights (tokens
@@ -266,31 +270,43 @@ def algorithmic_flops_gemm1(wl) -> int:
 
 
 # ------------------------------------------------------------------ our arm
-def run_ours(args):
-    import numpy as np
+def rank_inputs(wl, rank: int, world: int, device):
+    """The workload's tensors on ``device``; every rank past 0 draws its own batch x
+    (same recipe) while the weights stay the same on every rank."""
     import torch
 
-    import sparse_mixture_experts_26_b200 as moe
-    from workloads import WORKLOADS, make_inputs
-
-    rank, world, local = dist_env()
-    torch.cuda.set_device(local)
-    device = torch.device("cuda", local)
-    init_dist("nccl")
-    wl = WORKLOADS[args.workload]
-    # each rank draws its own batch; weights are the same on every rank
+    from workloads import make_inputs
     inp = make_inputs(wl, device)
     if world > 1 and rank > 0:
         g = torch.Generator(device=device)
         g.manual_seed(wl.seed * 1000 + rank)
         inp["x"] = torch.randn(inp["x"].shape, generator=g, device=device).to(inp["x"].dtype)
+    return inp
+
+
+def regime_of(T: int) -> str:
+    if T <= DECODE_MAX_TOKENS:
+        return "decode"
+    if T >= PAIR_MIN_TOKENS and os.environ.get("MOE_GEMM_PAIR", "1") != "0":
+        return "pair"
+    return "grouped"
+
+
+def measure_forward(wl, inp, K: int, W: int, world: int, local: int, device):
+    """Time K layer calls (after W warm-up calls) on the launching stream, with CUDA
+    events around the expert FFN inside the timed region, then the same K steps end to
+    end from pinned host buffers.  Returns the workload's result object (rank-local
+    timings already maxed over ranks)."""
+    import torch
+
+    import sparse_mixture_experts_26_b200 as moe
+
     x, Wg, W1, W3, W2 = (inp[k] for k in ("x", "Wg", "W1", "W3", "W2"))
     T, d, h, E = wl.T, wl.d, wl.h, wl.E
     ws = moe.alloc_workspace(T, d, h, E, wl.k, x.dtype, device)
     y = torch.empty_like(x)
     stream = torch.cuda.current_stream(device)
 
-    K, W = args.steps, args.warmup
     # Events around the expert FFN only (plus one between its two GEMMs for large
     # batches, where launches do not overlap anyway); the router, permutation and
     # combine run back to back, so small-batch launches keep overlapping their tails.
@@ -340,30 +356,33 @@ def run_ours(args):
     touched = int((counts > 0).sum())
 
     peaks, peak_src = load_peaks()
-    if wl.T <= DECODE_MAX_TOKENS:
-        regime = "decode"
-    elif wl.T >= PAIR_MIN_TOKENS and os.environ.get("MOE_GEMM_PAIR", "1") != "0":
-        regime = "pair"
-    else:
-        regime = "grouped"
+    regime = regime_of(wl.T)
     kname, tag, ksrc = DOMINANT[regime]
     if regime == "decode":  # weight streaming: HBM-bound, one fused FFN launch
         bound, unit = "hbm", "GB/s"
         ach = algorithmic_bytes_ffn_decode(wl, touched) / (t_ffn * 1e-3) / 1e9
         peak = float(peaks["hbm_gbs"])
+        per_launch = {"bytes": algorithmic_bytes_ffn_decode(wl, touched)}
     else:  # grouped GEMM1 (+SwiGLU): tensor-bound
         bound, unit = "tensor", "TFLOP/s"
         ach = algorithmic_flops_gemm1(wl) / (t_gemm1 * 1e-3) / 1e12
         peak = float(peaks["bf16_tflops"])
+        per_launch = {"flops": algorithmic_flops_gemm1(wl)}
     traffic = ncu_traffic(tag, wl.name, ksrc)
     roofline = {"bound": bound, "achieved": round(ach, 1), "peak": peak, "unit": unit,
                 "frac": round(ach / peak, 4), "traffic": traffic, "kernel": kname,
-                "peak_source": f"{peak_src} ({'burst' if bound == 'tensor' else 'copy'})"}
+                "peak_source": f"{peak_src} ({'burst' if bound == 'tensor' else 'copy'})",
+                "algorithmic_per_launch": per_launch,
+                "launch_ms": round(t_ffn if regime == "decode" else t_gemm1, 4)}
+    if bound == "tensor" and "bf16_tflops_sustained" in peaks:
+        roofline["frac_of_sustained"] = round(ach / float(peaks["bf16_tflops_sustained"]), 4)
     layer_bytes = touched * 3 * h * d * 2 + T * d * 2 * 2
     layer = {"ms": round(ms, 4), "tflops": round(wl.active_flops() / (ms * 1e-3) / 1e12, 1),
              "hbm_gbs": round(layer_bytes / (ms * 1e-3) / 1e9, 1),
-             "experts_touched": touched,
+             "experts_touched": touched, "rows_per_expert": [int(c) for c in counts],
              "stage_ms": {k: round(v, 4) for k, v in stages_ms.items()}}
+    if regime != "decode":
+        layer["frac_of_peak"] = round(wl.active_flops() / (ms * 1e-3) / 1e12 / peak, 4)
 
     # End to end through the public API with host buffers: every step copies its x
     # from pinned host memory, runs moe_layer_forward and reads y back to pinned host
@@ -412,34 +431,96 @@ def run_ours(args):
            "h2d_bytes_per_step": x.numel() * x.element_size(),
            "d2h_bytes_per_step": y.numel() * y.element_size(),
            "pipeline": "double-buffered: H2D and D2H copies on their own streams"}
+    return {"value": round(value, 1), "unit": UNIT, "steps": K, "warmup": W,
+            "ms_per_step": round(ms, 4), "config": workload_config(wl),
+            "roofline": roofline, "layer": layer, "e2e": e2e,
+            "gpu_launches": moe.launches_per_layer(T) * K, "clocks": clocks.summary()}
 
+
+def forward_cpu_baseline(inp, wl, args):
+    n = min(wl.T, args.cpu_sample_tokens)
+    tps, threads, reps, dt = oracle_tokens_per_s(cpu_copy(inp), n, args.cpu_budget_s)
+    return {"value": round(tps, 3), "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"fp64 numpy oracle on the first {n} tokens of the {wl.name} batch "
+                      f"(T={wl.T}), {reps} repeat(s) in {dt:.1f} s"}
+
+
+def free_device_memory():
+    import gc
+
+    import torch
+    gc.collect()
+    torch.cuda.empty_cache()
+
+
+# The default run: the prefill layer is the headline (its GEMM1 against the bf16
+# tensor-core peak); the decode, skewed and long-context layers and the prefill
+# backward are measured under the same timed-region rules and reported beside it.
+SUITE_HEADLINE = "prefill"
+SUITE_FORWARD = ("decode", "skew", "long")
+SUITE_BACKWARD = ("prefill",)
+DECODE_STEP_FACTOR = 10   # decode steps are ~0.4 ms: time 10x as many
+
+
+def run_ours(args):
+    import torch
+
+    from workloads import WORKLOADS
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    init_dist("nccl")
+    K, W = args.steps, args.warmup
+    suite = args.workload is None
+    name = SUITE_HEADLINE if suite else args.workload
+    wl = WORKLOADS[name]
+    inp = rank_inputs(wl, rank, world, device)
+    head = measure_forward(wl, inp, K, W, world, local, device)
     cpu_baseline = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        inp_cpu = cpu_copy(inp)
-        n = min(T, args.cpu_sample_tokens)
-        tps, threads, reps, dt = oracle_tokens_per_s(inp_cpu, n, args.cpu_budget_s)
-        cpu_baseline = {"value": round(tps, 3), "unit": UNIT, "cores": threads,
-                        "kind": "oracle",
-                        "sample": f"fp64 numpy oracle on the first {n} tokens of the batch, "
-                                  f"{reps} repeat(s) in {dt:.1f} s"}
+        cpu_baseline = forward_cpu_baseline(inp, wl, args)
+    del inp
+    free_device_memory()
+
+    sub = {}
+    if suite and not args.headline_only:
+        for other in SUITE_FORWARD:
+            owl = WORKLOADS[other]
+            oinp = rank_inputs(owl, rank, world, device)
+            k = K * DECODE_STEP_FACTOR if owl.T <= DECODE_MAX_TOKENS else K
+            sub[other] = measure_forward(owl, oinp, k, W, world, local, device)
+            del oinp
+            free_device_memory()
+        for other in SUITE_BACKWARD:
+            owl = WORKLOADS[other]
+            oinp = rank_inputs(owl, rank, world, device)
+            sub[f"backward_{other}"] = measure_backward(owl, oinp, K, W, world, local, device)
+            del oinp
+            free_device_memory()
 
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
     if rank != 0:
         return None
-    return {
-        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
-        "steps": K, "warmup": W, "ms_per_step": round(ms, 4), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype,
+    out = {
+        "metric": METRIC, "value": head["value"], "unit": UNIT, "n_gpus": world,
+        "steps": K, "warmup": W, "ms_per_step": head["ms_per_step"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype,
         "data": "synthetic (seeded normal draws of the Mixtral-8x7B layer shapes; "
                 "random-init weights)",
-        "config": workload_config(wl, {"parallelism": f"replicas x{world} (tokens sharded, "
-                                                      "weights replicated)"}),
-        "roofline": roofline, "layer": layer, "cpu_baseline": cpu_baseline, "e2e": e2e,
-        "gpu_launches": moe.launches_per_layer(T) * K,
-        "clocks": clocks.summary(),
+        "config": workload_config(wl, {"parallelism": parallelism(world)}),
+        "roofline": head["roofline"], "layer": head["layer"], "cpu_baseline": cpu_baseline,
+        "e2e": head["e2e"], "gpu_launches": head["gpu_launches"], "clocks": head["clocks"],
     }
+    if sub:
+        out["workloads"] = sub
+    return out
+
+
+def parallelism(world: int) -> str:
+    return f"replicas x{world} (tokens sharded, weights replicated)"
 
 
 # ------------------------------------------------------------------ our arm, backward
@@ -482,24 +563,18 @@ def wgrad_bytes(wl, stage: int) -> int:
     return 2 * wl.E * wl.h * wl.d * 4 + P * (2 * wl.h + wl.d) * 2
 
 
-def run_ours_backward(args):
+def measure_backward(wl, inp, K: int, W: int, world: int, local: int, device):
+    """Time K backward calls (after one forward that fills the saved state and W
+    warm-up calls), with events between the backward's stages inside the timed
+    region, then the same steps end to end (dy in, dx out through pinned host
+    buffers).  Returns the workload's result object."""
     import torch
 
     import sparse_mixture_experts_26_b200 as moe
-    from workloads import WORKLOADS, make_inputs
+    from workloads import WORKLOADS
 
-    rank, world, local = dist_env()
-    torch.cuda.set_device(local)
-    device = torch.device("cuda", local)
-    init_dist("nccl")
-    wl = WORKLOADS[args.workload]
     if wl.dtype != "bf16":
         raise SystemExit("the backward pass is built for bf16 layers")
-    inp = make_inputs(wl, device)
-    if world > 1 and rank > 0:
-        g = torch.Generator(device=device)
-        g.manual_seed(wl.seed * 1000 + rank)
-        inp["x"] = torch.randn(inp["x"].shape, generator=g, device=device).to(inp["x"].dtype)
     x, Wg, W1, W3, W2 = (inp[k] for k in ("x", "Wg", "W1", "W3", "W2"))
     T, d, h, E = wl.T, wl.d, wl.h, wl.E
     ws = moe.alloc_workspace(T, d, h, E, wl.k, x.dtype, device)
@@ -512,7 +587,6 @@ def run_ours_backward(args):
     dWg, dW1 = torch.empty(Wg.shape, **f32), torch.empty(W1.shape, **f32)
     dW3, dW2 = torch.empty(W3.shape, **f32), torch.empty(W2.shape, **f32)
     stream = torch.cuda.current_stream(device)
-    K, W = args.steps, args.warmup
     nst = len(BWD_STAGES) + 1
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nst)] for _ in range(K)]
     for row in evs:
@@ -557,10 +631,12 @@ def run_ours_backward(args):
         bound, unit, peak_kind = "hbm", "GB/s", "copy"
         ach = wgrad_bytes(wl, dom) / (st_ms[dom] * 1e-3) / 1e9
         peak = float(peaks["hbm_gbs"])
+        per_launch = {"bytes": wgrad_bytes(wl, dom)}
     else:
         bound, unit, peak_kind = "tensor", "TFLOP/s", "burst"
         ach = flops[dom] / (st_ms[dom] * 1e-3) / 1e12
         peak = float(peaks["bf16_tflops"])
+        per_launch = {"flops": flops[dom]}
     src = os.path.join(CSRC, "backward_pair_sm100.cu" if "pair" in kname else "backward_sm100.cu")
     if dom in (1, 2, 3) and "pair" in kname:
         src = os.path.join(CSRC, "grouped_gemm_pair_sm100.cu")
@@ -577,7 +653,8 @@ def run_ours_backward(args):
     roofline = {"bound": bound, "achieved": round(ach, 1), "peak": peak, "unit": unit,
                 "frac": round(ach / peak, 4), "traffic": traffic,
                 "kernel": f"{kname} (stage '{BWD_STAGES[dom]}')",
-                "peak_source": f"{peak_src} ({peak_kind})"}
+                "peak_source": f"{peak_src} ({peak_kind})",
+                "algorithmic_per_launch": per_launch, "launch_ms": round(st_ms[dom], 4)}
     if traffic_note:
         roofline["traffic_note"] = traffic_note
     total_flops = sum(flops.values())
@@ -632,10 +709,29 @@ def run_ours_backward(args):
            "d2h_bytes_per_step": dx.numel() * dx.element_size(),
            "pipeline": "double-buffered: dy in and dx out on their own streams; weight "
                        "gradients stay on the device"}
+    return {"metric": BWD_METRIC, "value": round(value, 1), "unit": UNIT, "steps": K,
+            "warmup": W, "ms_per_step": round(ms, 4),
+            "config": workload_config(wl, {"pass": "backward (after one forward that fills "
+                                                   "the saved state)"}),
+            "roofline": roofline, "layer": layer, "e2e": e2e,
+            "gpu_launches": moe.launches_per_backward(T) * K, "clocks": clocks.summary()}
 
+
+def run_ours_backward(args):
+    import torch
+
+    from workloads import WORKLOADS
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    init_dist("nccl")
+    wl = WORKLOADS[args.workload or SUITE_HEADLINE]
+    inp = rank_inputs(wl, rank, world, device)
+    r = measure_backward(wl, inp, args.steps, args.warmup, world, local, device)
     cpu_baseline = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        n = min(T, args.cpu_sample_tokens_bwd)
+        n = min(wl.T, args.cpu_sample_tokens_bwd)
         tps, threads, reps, dt = oracle_tokens_per_s(cpu_copy(inp), n, args.cpu_budget_s,
                                                      backward=True)
         cpu_baseline = {"value": round(tps, 3), "unit": UNIT, "cores": threads,
@@ -648,17 +744,16 @@ def run_ours_backward(args):
         dist.destroy_process_group()
     if rank != 0:
         return None
+    cfg = dict(r["config"], parallelism=parallelism(world))
     return {
-        "metric": BWD_METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
-        "steps": K, "warmup": W, "ms_per_step": round(ms, 4), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype,
+        "metric": BWD_METRIC, "value": r["value"], "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": r["ms_per_step"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype,
         "data": "synthetic (seeded normal draws of the Mixtral-8x7B layer shapes and of dy; "
                 "random-init weights)",
-        "config": workload_config(wl, {"pass": "backward (after one forward that fills the "
-                                               "saved state)",
-                                       "parallelism": f"replicas x{world}"}),
-        "roofline": roofline, "layer": layer, "cpu_baseline": cpu_baseline, "e2e": e2e,
-        "gpu_launches": moe.launches_per_backward(T) * K, "clocks": clocks.summary(),
+        "config": cfg, "roofline": r["roofline"], "layer": r["layer"],
+        "cpu_baseline": cpu_baseline, "e2e": r["e2e"], "gpu_launches": r["gpu_launches"],
+        "clocks": r["clocks"],
     }
 
 
@@ -672,7 +767,7 @@ def run_reference(args):
     rank, world, _ = dist_env()
     if rank != 0:
         return None
-    wl = WORKLOADS[args.workload]
+    wl = WORKLOADS[args.workload or SUITE_HEADLINE]
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     inp_cpu = cpu_copy(make_inputs(wl, dev))
     n = min(wl.T, args.cpu_sample_tokens)
@@ -710,7 +805,8 @@ def run_reference(args):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": workload_config(wl, {"pass": "backward"} if args.backward else None),
+        "config": workload_config(wl, dict({"pass": "backward"} if args.backward else {},
+                                           parallelism=parallelism(world))),
         "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": int(threads),
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0,
@@ -724,8 +820,12 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=None)
     ap.add_argument("--warmup", type=int, default=None)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="decode",
-                    choices=["decode", "prefill", "skew", "long", "tiny_f32", "prefill_half"])
+    ap.add_argument("--workload", default=None,
+                    choices=["decode", "prefill", "skew", "long", "tiny_f32", "prefill_half"],
+                    help="time one workload only (default: the prefill headline plus the "
+                         "decode, skew and long layers and the prefill backward)")
+    ap.add_argument("--headline-only", action="store_true",
+                    help="default run without the other workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-tokens", type=int, default=16)
     ap.add_argument("--cpu-budget-s", type=float, default=10.0)

@@ -71,7 +71,9 @@ typedef enum {
  * moe_expert_ffn.  The size never decreases with T: a workspace sized for T serves
  * every batch of at most T tokens (same d, h, E, k, dt).  Zero the workspace once
  * before its first use: it holds a status word and dependency counters that every
- * call leaves at zero.  Returns 0 for unsupported arguments. */
+ * completed call leaves at zero.  After a call that ended in MOE_ERR_TIMEOUT (or set
+ * MOE_DEV_FLAG_TIMEOUT), the counters may be left non-zero: zero the whole
+ * workspace again before reusing it.  Returns 0 for unsupported arguments. */
 size_t moe_workspace_bytes(int T, int d, int h, int E, int k, moe_dtype dt);
 
 /* Router + top-2 + softmax of the two kept logits.
@@ -141,7 +143,12 @@ moe_status moe_combine(const float *y_perm, const int32_t *inv_perm,
  *   of a bf16 Mixtral expert with h = 14336, i.e. up to 146 tokens).
  *   The first call on a device, with that device current, looks up the array's
  *   device address (cudaGetSymbolAddress) and caches it; make that first call
- *   before any stream capture on the device.
+ *   before any stream capture on the device.  The cached address belongs to the
+ *   device's primary context: after cudaDeviceReset it is stale, so do not call
+ *   this entry point on a device that the process has reset.
+ *   Device-side wait timeouts set a status word inside the library's array, which
+ *   no caller can read: they are reported (as MOE_ERR_TIMEOUT) only when the
+ *   MOE_DEBUG_SYNC=1 setting makes each call synchronise and check that word.
  *   All calls share the one array, which keeps the previous call's contents; each
  *   call clears the status word itself.  Calls whose work overlaps on the GPU
  *   (other streams, other threads) race on the array: serialise them.
@@ -188,7 +195,9 @@ moe_status moe_layer_forward_events(const void *x, const void *Wg, const void *W
 
 /* Synchronise `stream`, read the workspace status word into *flags (host
  * pointer; MOE_DEV_FLAG_* bits), then clear it.  Returns MOE_ERR_TIMEOUT if the
- * timeout flag was set, MOE_OK otherwise.  Diagnostic call: it synchronises. */
+ * timeout flag was set, MOE_OK otherwise.  Diagnostic call: it synchronises.  After
+ * a timeout, zero the whole workspace before its next use (the dependency counters
+ * of an interrupted call may be non-zero). */
 moe_status moe_device_status(void *ws, size_t ws_bytes, uint32_t *flags,
                              cudaStream_t stream);
 

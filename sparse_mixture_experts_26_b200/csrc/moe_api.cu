@@ -61,22 +61,11 @@ bool debug_sync_enabled() {
     return v;
 }
 
-namespace {
-
-// NVTX range around the host-side work of one stage (shows up in nsys / ncu timelines;
-// free when no tool is attached).
-struct NvtxRange {
-    explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
-    ~NvtxRange() { nvtxRangePop(); }
-    NvtxRange(const NvtxRange&) = delete;
-    NvtxRange& operator=(const NvtxRange&) = delete;
-};
-
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // routed = false: the expert FFN alone, which also takes a single expert.
 moe_status check_shape(int T, int d, int h, int E, int k, moe_dtype dt, bool need_h,
-                       bool routed = true) {
+                       bool routed) {
     if (T < 0 || d <= 0 || (need_h && h <= 0) || E <= 0 || k <= 0) return MOE_ERR_INVALID_ARG;
     if (dt != MOE_F32 && dt != MOE_BF16) return MOE_ERR_INVALID_ARG;
     if (k != 2 || E < (routed ? 2 : 1) || E > kMaxExperts) return MOE_ERR_UNSUPPORTED;
@@ -97,6 +86,17 @@ bool ptrs_ok(std::initializer_list<const void*> ps) {
         if (p == nullptr || !aligned16(p)) return false;
     return true;
 }
+
+namespace {
+
+// NVTX range around the host-side work of one stage (shows up in nsys / ncu timelines;
+// free when no tool is attached).
+struct NvtxRange {
+    explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange&) = delete;
+    NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 moe_status finish(cudaError_t err, cudaStream_t s, uint32_t* status) {
     if (err != cudaSuccess) return MOE_ERR_CUDA;

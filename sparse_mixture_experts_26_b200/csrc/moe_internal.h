@@ -2,6 +2,7 @@
 // the workspace layout and the launchers of each kernel family.
 #pragma once
 
+#include <initializer_list>
 #include <cuda_runtime.h>
 
 #include <atomic>
@@ -108,6 +109,13 @@ inline WsLayout ws_layout(int T, int d, int h, int E, int k, moe_dtype dt) {
 
 int device_sm_count();
 bool debug_sync_enabled();
+
+// Argument checks shared by every entry point.  routed = false: the expert FFN alone,
+// which also takes a single expert.
+moe_status check_shape(int T, int d, int h, int E, int k, moe_dtype dt, bool need_h,
+                       bool routed = true);
+bool aligned16(const void* p);
+bool ptrs_ok(std::initializer_list<const void*> ps);
 // Programmatic dependent launch: used for the launches made inside a PdlScope(true)
 // (the entry points open one for small batches, where launch gaps matter and every
 // kernel is short), never when MOE_NO_PDL=1.  Measured: on T=16 it saves ~2% of the

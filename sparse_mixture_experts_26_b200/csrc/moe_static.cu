@@ -11,7 +11,10 @@
 //
 // The array's name is only a host-side stand-in in host code, never a device
 // address, so the address is looked up with cudaGetSymbolAddress once per device
-// (on the first call made while that device is current) and cached.
+// (on the first call made while that device is current) and cached.  The cache
+// belongs to the device's primary context, the one the runtime API uses: after
+// cudaDeviceReset the module is loaded again and the cached address is stale, so a
+// process that resets a device must not call this entry point on it again.
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -55,17 +58,16 @@ extern "C" moe_status moe_expert_ffn_static(const void* x_perm, const int32_t* o
                                             const void* W1, const void* W3, const void* W2,
                                             int rows, int d, int h, int E, moe_dtype dt,
                                             float* y_perm, cudaStream_t stream) {
-    if (rows < 0 || rows % 2 != 0 || d <= 0 || h <= 0 || E <= 0) return MOE_ERR_INVALID_ARG;
-    if (dt != MOE_F32 && dt != MOE_BF16) return MOE_ERR_INVALID_ARG;
-    if (E < 2 || E > kMaxExperts || d % 8 != 0 || h % 8 != 0) return MOE_ERR_UNSUPPORTED;
+    // The same argument checks as moe_expert_ffn (which also takes a single expert),
+    // then the scratch limit in place of the workspace size.
+    if (rows < 0 || rows % 2 != 0) return MOE_ERR_INVALID_ARG;
+    moe_status st = check_shape(rows / 2, d, h, E, 2, dt, true, /*routed=*/false);
+    if (st != MOE_OK) return st;
     // H [rows, h] must fit behind the status word.
     const size_t h_bytes = static_cast<size_t>(rows) * h * dtype_bytes(dt);
     if (h_bytes > MOE_STATIC_SCRATCH_BYTES - kStatusBytes) return MOE_ERR_WORKSPACE;
     if (rows == 0) return MOE_OK;
-    for (const void* p : {x_perm, static_cast<const void*>(offsets), W1, W3, W2,
-                          static_cast<const void*>(y_perm)})
-        if (p == nullptr || (reinterpret_cast<uintptr_t>(p) & 15u) != 0)
-            return MOE_ERR_INVALID_ARG;
+    if (!ptrs_ok({x_perm, offsets, W1, W3, W2, y_perm})) return MOE_ERR_INVALID_ARG;
 
     void* base = nullptr;
     if (scratch_address(&base) != cudaSuccess) return MOE_ERR_CUDA;

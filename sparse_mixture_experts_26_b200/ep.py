@@ -35,7 +35,7 @@ import torch
 import torch.distributed as dist
 
 __all__ = ["TransferPlan", "plan_transfers", "exchange_counts", "run_transfers",
-           "ExpertParallelMoE"]
+           "LibmoeSteps", "ExpertParallelMoE"]
 
 
 @dataclass
@@ -125,16 +125,44 @@ def run_transfers(plan: TransferPlan, rank: int, src_rows: torch.Tensor,
             req.wait()
 
 
+class LibmoeSteps:
+    """The four layer steps an expert-parallel call runs, as libmoe's kernels."""
+
+    @staticmethod
+    def route(x, Wg, idx, w):
+        from . import moe_route
+        moe_route(x, Wg, idx, w)
+
+    @staticmethod
+    def permute(idx, x, offsets, perm_token, inv_perm, x_perm, ws, E):
+        from . import moe_permute
+        moe_permute(idx, x, offsets, perm_token, inv_perm, x_perm, ws, E)
+
+    @staticmethod
+    def expert_ffn(x_rows, offsets, W1, W3, W2, Y, ws):
+        from . import moe_expert_ffn
+        moe_expert_ffn(x_rows, offsets, W1, W3, W2, Y, ws)
+
+    @staticmethod
+    def combine(Y, inv_perm, w, y):
+        from . import moe_combine
+        moe_combine(Y, inv_perm, w, y)
+
+
 class ExpertParallelMoE:
     """One layer with its experts spread over the ranks of ``group``.
 
     Every rank passes the full router ``Wg [d, E]`` and the weights of its own experts
     (``W1_local, W3_local [El, h, d]``, ``W2_local [El, d, h]``; rank r holds experts
     r * El .. r * El + El - 1).  bf16 layers (the libmoe expert kernels); CUDA tensors.
+    ``steps`` replaces the four layer steps (route, permute, expert_ffn, combine;
+    default: libmoe's kernels) -- a test hook, so that the planning and transfer code
+    can be driven on CPU ranks with reference steps in place of the kernels.
     """
 
-    def __init__(self, Wg, W1_local, W3_local, W2_local, group=None):
+    def __init__(self, Wg, W1_local, W3_local, W2_local, group=None, steps=None):
         from . import alloc_workspace  # noqa: F401  (the package loads libmoe)
+        self.steps = LibmoeSteps if steps is None else steps
         self.group = group
         self.world = dist.get_world_size(group) if dist.is_initialized() else 1
         self.rank = dist.get_rank(group) if dist.is_initialized() else 0
@@ -154,8 +182,11 @@ class ExpertParallelMoE:
             self._ws["ws"] = ws
         return ws
 
-    def forward(self, x: torch.Tensor) -> torch.Tensor:
-        from . import moe_combine, moe_expert_ffn, moe_permute, moe_route
+    def forward(self, x: torch.Tensor, routing: dict | None = None) -> torch.Tensor:
+        """The layer on this rank's tokens ``x [T, d]``; returns ``y [T, d]``.  If a dict
+        is passed as ``routing``, it receives this rank's ``idx``, ``w``, ``offsets``,
+        ``perm_token`` and ``inv_perm``."""
+        st = self.steps
         T, d = x.shape
         dev = x.device
         E, El, N = self.E, self.El, self.world
@@ -167,8 +198,8 @@ class ExpertParallelMoE:
         x_perm = torch.empty(2 * T, d, dtype=x.dtype, device=dev)
         ws = self._workspace(max(T, 1), x)
         if T > 0:
-            moe_route(x, self.Wg, idx, w)
-        moe_permute(idx, x, offsets, perm_token, inv_perm, x_perm, ws, E)
+            st.route(x, self.Wg, idx, w)
+        st.permute(idx, x, offsets, perm_token, inv_perm, x_perm, ws, E)
         counts = (offsets[1:] - offsets[:-1]).to(torch.int64).cpu().view(N, El)
         recv_counts = exchange_counts(counts, self.group)
         plan = plan_transfers(counts.tolist(), recv_counts.tolist(), self.rank)
@@ -179,13 +210,16 @@ class ExpertParallelMoE:
         Y_recv = torch.empty(rows, d, dtype=torch.float32, device=dev)
         if plan.received > 0:
             local_off = torch.tensor(plan.local_offsets, dtype=torch.int32, device=dev)
-            moe_expert_ffn(x_recv, local_off, self.W1, self.W3, self.W2, Y_recv,
-                           self._ffn_workspace(rows, x))
+            st.expert_ffn(x_recv, local_off, self.W1, self.W3, self.W2, Y_recv,
+                          self._ffn_workspace(rows, x))
         Y_perm = torch.empty(2 * T, d, dtype=torch.float32, device=dev)
         run_transfers(plan, self.rank, Y_recv, Y_perm, reverse=True, group=self.group)
         y = torch.empty_like(x)
         if T > 0:
-            moe_combine(Y_perm, inv_perm, w, y)
+            st.combine(Y_perm, inv_perm, w, y)
+        if routing is not None:
+            routing.update(idx=idx, w=w, offsets=offsets, perm_token=perm_token,
+                           inv_perm=inv_perm)
         return y
 
     def _ffn_workspace(self, rows: int, x: torch.Tensor) -> torch.Tensor:

@@ -119,3 +119,106 @@ def test_two_ranks_reproduce_the_whole_layer(E):
     assert all(isinstance(e, float) for e in errs), errs
     assert all(p.exitcode == 0 for p in procs)
     assert max(errs) <= 1e-12, errs
+
+
+class OracleSteps:
+    """The four layer steps written with the fp64 oracle, on CPU tensors, standing in
+    for libmoe's kernels so that ExpertParallelMoE.forward's own planning and transfer
+    code runs on gloo ranks.  Outputs are stored in the tensors' dtypes (float32)."""
+
+    @staticmethod
+    def route(x, Wg, idx, w):
+        from oracle import moe_oracle as O
+        logits = O.router_logits(x.double().numpy(), Wg.double().numpy())
+        i = O.top2_select(logits)
+        idx.copy_(torch.from_numpy(i))
+        w.copy_(torch.from_numpy(O.gate_weights_f32(logits, i)))
+
+    @staticmethod
+    def permute(idx, x, offsets, perm_token, inv_perm, x_perm, ws, E):
+        from oracle import moe_oracle as O
+        off, pt, inv = O.permutation(idx.numpy(), E)
+        offsets.copy_(torch.from_numpy(off))
+        perm_token.copy_(torch.from_numpy(pt))
+        inv_perm.copy_(torch.from_numpy(inv))
+        x_perm.copy_(torch.from_numpy(O.gather_rows(x.numpy(), pt)))
+
+    @staticmethod
+    def expert_ffn(x_rows, offsets, W1, W3, W2, Y, ws):
+        from oracle import moe_oracle as O
+        off = offsets.numpy()
+        n = int(off[-1])  # a padding row past the last group belongs to no expert
+        Y[:n] = torch.from_numpy(O.expert_ffn_grouped(
+            x_rows[:n].double().numpy(), off, W1.double().numpy(), W3.double().numpy(),
+            W2.double().numpy())).to(Y.dtype)
+
+    @staticmethod
+    def combine(Y, inv_perm, w, y):
+        from oracle import moe_oracle as O
+        y.copy_(torch.from_numpy(O.combine(Y.double().numpy(), inv_perm.numpy(),
+                                           w.double().numpy())).to(y.dtype))
+
+
+def _forward_worker(rank, world, port, E, q):
+    import sys
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        from oracle import moe_oracle as O
+        from sparse_mixture_experts_26_b200.ep import ExpertParallelMoE
+        from tests.test_ep_cpu import OracleSteps
+        from workloads import make_inputs, small
+
+        T_all = 61
+        inp = make_inputs(small("epf", T=T_all, d=16, h=24, E=E, seed=19, dtype="f32",
+                                kind="skew" if E == 8 else "plain"), "cpu")
+        El = E // world
+        shard = np.array_split(np.arange(T_all), world)[rank]
+        layer = ExpertParallelMoE(inp["Wg"], inp["W1"][rank * El:(rank + 1) * El].contiguous(),
+                                  inp["W3"][rank * El:(rank + 1) * El].contiguous(),
+                                  inp["W2"][rank * El:(rank + 1) * El].contiguous(),
+                                  steps=OracleSteps)
+        routing = {}
+        y = layer.forward(inp["x"][shard].contiguous(), routing).double().numpy()
+        parts = [None] * world
+        dist.all_gather_object(parts, (y, routing["idx"].numpy()))
+        if rank == 0:
+            c = {k: v.double().numpy() for k, v in inp.items()}
+            ref = O.moe_layer(c["x"], c["Wg"], c["W1"], c["W3"], c["W2"])
+            y_all = np.concatenate([p[0] for p in parts])
+            idx_all = np.concatenate([p[1] for p in parts])
+            same_idx = bool((idx_all == ref["idx"]).all())
+            err = float(np.linalg.norm(y_all - ref["y"]) / np.linalg.norm(ref["y"]))
+            q.put((same_idx, err))
+        else:
+            q.put((True, 0.0))
+    except Exception as exc:  # report instead of leaving the parent waiting
+        q.put(repr(exc))
+        raise
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("E", [2, 8])
+def test_two_ranks_drive_expert_parallel_forward(E):
+    """ExpertParallelMoE.forward end to end on two gloo ranks (count exchange, plan,
+    dispatch, local experts, return, combine), with the oracle's steps injected in
+    place of the kernels: routing is bit-exact and y matches the whole-batch oracle
+    to float32 rounding (the steps store w, Y and y in float32)."""
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_forward_worker, args=(r, world, port, E, q))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    res = [q.get(timeout=180) for _ in range(world)]
+    for p in procs:
+        p.join(timeout=60)
+    assert all(isinstance(r, tuple) for r in res), res
+    assert all(p.exitcode == 0 for p in procs)
+    assert all(r[0] for r in res)
+    assert max(r[1] for r in res) <= 1e-6, res

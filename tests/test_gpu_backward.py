@@ -31,6 +31,13 @@ def rel_fro(a, b):
     return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300))
 
 
+def report(case, g, ref):
+    """Relative Frobenius error of every gradient, printed for the record."""
+    errs = {k: rel_fro(f64(g[k]), ref[k]) for k in ("dx", "dWg", "dW1", "dW3", "dW2")}
+    print("BWD_ERR " + case + " " + " ".join(f"{k}={v:.3e}" for k, v in errs.items()))
+    return errs
+
+
 def seeded_dy(T, d, seed):
     g = torch.Generator(device="cpu")
     g.manual_seed(seed)
@@ -66,10 +73,10 @@ def test_backward_small_shapes(T, d, h, kind):
     g, _ = gpu_grads(inp, dy)
     c = {k: f64(v) for k, v in inp.items()}
     ref = O.moe_layer_backward(c["x"], c["Wg"], c["W1"], c["W3"], c["W2"], f64(dy))
+    errs = report(f"T={T} d={d} h={h} {kind}", g, ref)
     for k in ("dx", "dW1", "dW3", "dW2"):
-        err = rel_fro(f64(g[k]), ref[k])
-        assert err <= BWD_TOL, (k, err)
-    assert rel_fro(f64(g["dWg"]), ref["dWg"]) <= ROUTER_TOL
+        assert errs[k] <= BWD_TOL, (k, errs[k])
+    assert errs["dWg"] <= ROUTER_TOL
     # experts that received no rows get exact zeros
     counts = np.bincount(ref["fwd"]["idx"].ravel(), minlength=wl.E)
     for e in np.flatnonzero(counts == 0):
@@ -87,9 +94,10 @@ def test_backward_with_capacity(T, d, h, cap):
     c = {k: f64(v) for k, v in inp.items()}
     ref = O.moe_layer_backward(c["x"], c["Wg"], c["W1"], c["W3"], c["W2"], f64(dy), capacity=cap)
     assert not ref["fwd"]["keep"].all()
+    errs = report(f"T={T} d={d} h={h} capacity={cap}", g, ref)
     for k in ("dx", "dW1", "dW3", "dW2"):
-        assert rel_fro(f64(g[k]), ref[k]) <= BWD_TOL, k
-    assert rel_fro(f64(g["dWg"]), ref["dWg"]) <= ROUTER_TOL
+        assert errs[k] <= BWD_TOL, k
+    assert errs["dWg"] <= ROUTER_TOL
 
 
 def test_backward_is_deterministic_and_rejects_unsupported():
@@ -209,6 +217,7 @@ def test_backward_other_expert_counts(T, E):
     g, _ = gpu_grads(inp, dy)
     c = {k: f64(v) for k, v in inp.items()}
     ref = O.moe_layer_backward(c["x"], c["Wg"], c["W1"], c["W3"], c["W2"], f64(dy))
+    errs = report(f"T={T} E={E}", g, ref)
     for k in ("dx", "dW1", "dW3", "dW2"):
-        assert rel_fro(f64(g[k]), ref[k]) <= BWD_TOL, k
-    assert rel_fro(f64(g["dWg"]), ref["dWg"]) <= ROUTER_TOL
+        assert errs[k] <= BWD_TOL, k
+    assert errs["dWg"] <= ROUTER_TOL

@@ -1,7 +1,8 @@
 """Expert parallelism on one GPU (world size 1: every expert is local) and the pieces
-it relies on: the layer through ExpertParallelMoE must equal moe_layer_forward bit for
-bit, and the expert FFN takes a single expert and a padding row outside every group.
-The exchange itself is covered on CPU by tests/test_ep_cpu.py (gloo, two ranks)."""
+it relies on: the layer through ExpertParallelMoE matches the fp64 oracle (routing
+bit-exact, y within the bf16 tolerance) and equals moe_layer_forward bit for bit, and
+the expert FFN takes a single expert and a padding row outside every group.  The
+exchange itself is covered on CPU by tests/test_ep_cpu.py (gloo, two ranks)."""
 import numpy as np
 import pytest
 import torch
@@ -19,7 +20,15 @@ def test_single_rank_expert_parallel_equals_the_layer(T, kind):
     wl = small("ep1", T=T, d=256, h=384, seed=40 + T, kind=kind)
     inp = make_inputs(wl, "cuda")
     layer = ExpertParallelMoE(inp["Wg"], inp["W1"], inp["W3"], inp["W2"])
-    y_ep = layer.forward(inp["x"])
+    routing = {}
+    y_ep = layer.forward(inp["x"], routing)
+    c = {k: v.double().cpu().numpy() for k, v in inp.items()}
+    ref = O.moe_layer(c["x"], c["Wg"], c["W1"], c["W3"], c["W2"])
+    np.testing.assert_array_equal(routing["idx"].cpu().numpy(), ref["idx"])
+    np.testing.assert_array_equal(routing["offsets"].cpu().numpy(), ref["offsets"])
+    np.testing.assert_array_equal(routing["perm_token"].cpu().numpy(), ref["perm_token"])
+    got = y_ep.double().cpu().numpy()
+    assert np.linalg.norm(got - ref["y"]) / np.linalg.norm(ref["y"]) <= 5e-3
     ws = moe.alloc_workspace(T, 256, 384, wl.E, 2, inp["x"].dtype)
     y = moe.layer_forward(inp["x"], inp["Wg"], inp["W1"], inp["W3"], inp["W2"], ws=ws)
     assert torch.equal(y_ep, y)

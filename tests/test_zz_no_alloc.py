@@ -5,8 +5,9 @@ its ops no allocator, or a serving loop that must not allocate after start-up --
 cannot give the library a workspace.  The static entry point keeps its scratch in
 a fixed array inside the library instead.  These tests call it through the C ABI
 (ctypes on libmoe.so) and check that two calls in a row give what the workspace
-entry point gives, within the tests' bf16 / fp32 tolerances, and that a shape whose
-scratch would not fit is refused with MOE_ERR_WORKSPACE before anything runs.
+entry point gives, and what the fp64 oracle gives, within the tests' bf16 / fp32
+tolerances, and that a shape whose scratch would not fit is refused with
+MOE_ERR_WORKSPACE before anything runs.
 
 The file name makes pytest collect it last; it must pass on its own in a fresh
 process as well as after the other GPU tests.
@@ -18,6 +19,7 @@ import pytest
 import torch
 
 import sparse_mixture_experts_26_b200 as moe
+from oracle import moe_oracle as O
 from workloads import make_inputs, small
 
 pytestmark = pytest.mark.gpu
@@ -61,8 +63,25 @@ def call_static(lib, xp, off, inp, wl, y):
 
 
 def rel_fro(a, b):
-    a, b = a.double().cpu().numpy(), b.double().cpu().numpy()
+    a = a.double().cpu().numpy() if torch.is_tensor(a) else a
+    b = b.double().cpu().numpy() if torch.is_tensor(b) else b
     return float(np.linalg.norm(a - b) / np.linalg.norm(b))
+
+
+class PerExpert:
+    """Hands the oracle one expert's weights at a time (exact values as float32)."""
+
+    def __init__(self, t):
+        self.t = t
+
+    def __getitem__(self, e):
+        return self.t[e].float().cpu().numpy()
+
+
+def oracle_Y(xp, off, inp):
+    return O.expert_ffn_grouped(xp.float().cpu().numpy(), off.cpu().numpy(),
+                                PerExpert(inp["W1"]), PerExpert(inp["W3"]),
+                                PerExpert(inp["W2"]))
 
 
 @pytest.mark.parametrize("wl,tol", [
@@ -75,12 +94,34 @@ def test_static_scratch_matches_workspace_entry_point(wl, tol):
     inp, xp, off, ws = grouped_inputs(wl)
     ref = torch.empty(xp.shape[0], wl.d, dtype=torch.float32, device="cuda")
     moe.moe_expert_ffn(xp, off, inp["W1"], inp["W3"], inp["W2"], ref, ws)
+    Y64 = oracle_Y(xp, off, inp)
     for _ in range(2):  # two calls in a row share (and reuse) the one scratch array
         y = torch.full_like(ref, float("nan"))
         assert call_static(lib, xp, off, inp, wl, y) == MOE_OK
         torch.cuda.synchronize()
         assert torch.isfinite(y).all()
-        assert rel_fro(y, ref) <= tol
+        assert rel_fro(y, ref) <= tol      # the workspace entry point
+        assert rel_fro(y, Y64) <= tol      # the fp64 oracle
+
+
+def test_static_scratch_single_expert():
+    """One expert (E = 1) with an odd group padded to an even row count, as the
+    workspace entry point takes it; the padding row's output is unspecified."""
+    lib = c_lib()
+    wl = small("static_e1", T=20, d=128, h=192, E=2, seed=24)
+    inp = make_inputs(wl, "cuda")
+    rows = 37
+    xp = torch.zeros(rows + 1, wl.d, dtype=torch.bfloat16, device="cuda")
+    xp[:rows] = inp["x"].repeat(2, 1)[:rows]
+    one = {k: inp[k][:1].contiguous() for k in ("W1", "W3", "W2")}
+    off = torch.tensor([0, rows], dtype=torch.int32, device="cuda")
+    e1 = small("static_e1", T=(rows + 1) // 2, d=128, h=192, E=1)
+    Y64 = oracle_Y(xp[:rows], off, one)
+    for _ in range(2):
+        y = torch.full((rows + 1, wl.d), float("nan"), device="cuda")
+        assert call_static(lib, xp, off, one, e1, y) == MOE_OK
+        torch.cuda.synchronize()
+        assert rel_fro(y[:rows], Y64) <= 5e-3
 
 
 def test_static_scratch_rejects_shapes_beyond_its_limit():
