@@ -13,15 +13,21 @@
 // instead of 48 KiB for the same math), which leaves room for 6 pipeline stages
 // and cuts the L2->SM traffic by a third.
 //
-// GEMM1 splits B as [128 rows of W1 | the same 128 rows of W3]: the leader stages
-// the W1 rows, the peer the W3 rows, so accumulator columns 0..127 hold a = x.W1 and
-// 128..255 hold b = x.W3 for the same outputs (as in the single-SM kernel).
+// GEMM1 covers 128 outputs n0 .. n0+127 per tile.  Each CTA stages 64 W1 rows and
+// the same 64 W3 rows (the leader outputs n0 .. n0+63, the peer n0+64 .. n0+127), so
+// accumulator columns [0,64) hold a = x.W1 and [64,128) b = x.W3 for the leader's
+// outputs and [128,192) / [192,256) the same for the peer's: every thread finds the a
+// and b of an output in its own TMEM lane, in both tile modes below.
 //
 // An expert's rows are covered by 256-row blocks; a last block with at most 128 rows
 // is issued with M = 128 (64 rows per CTA) so that no more rows are wasted than with
 // 128-row tiles.  In that mode the accumulator uses the "2x2" data-path layout:
 // columns 0..127 of the tile in TMEM lanes 0..63 and columns 128..255 in lanes
 // 64..127, both in the first 128 TMEM columns of the buffer.
+//
+// Without an exchange buffer in the epilogue, the forward GEMMs and the backward's
+// fp32-output GEMMs keep 7 pipeline stages (224 KiB); the backward SwiGLU step, whose
+// half-tile epilogue exchanges b through shared memory, keeps 6.
 //
 // Synchronisation: both CTAs' TMA loads count their bytes on the leader's "full"
 // barrier; the leader's MMA completions are multicast to both CTAs' "empty" and
@@ -45,7 +51,7 @@ constexpr int kRowsPerCta = 128;
 constexpr int kPairRows = 2 * kRowsPerCta;   // rows per full pair tile
 constexpr int kBK = 64;
 constexpr int kN = 256;                      // accumulator columns per tile
-constexpr int kStages = 6;
+constexpr int kMaxStages = 7;
 constexpr int kABytes = kRowsPerCta * kBK * 2;  // 16 KiB
 constexpr int kBBytes = 128 * kBK * 2;          // 16 KiB: this CTA's half of B
 constexpr int kStageBytes = kABytes + kBBytes;
@@ -55,8 +61,6 @@ constexpr uint32_t kTmemCols = 2 * kN;
 constexpr uint32_t kIdescFull = idesc_bf16_f32(2 * kRowsPerCta, kN);
 constexpr uint32_t kIdescHalf = idesc_bf16_f32(kRowsPerCta, kN);
 constexpr int kXferBytes = 32 * 64 * 4;  // one 32-column chunk of b for 64 rows
-constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 1024 /*bookkeeping*/ +
-                           kXferBytes;
 constexpr int kXferBarrier = 1;
 constexpr int kVoteBarrier = 2;  // epilogue vote after a bounded wait
 constexpr uint16_t kBothCtas = 0x3;
@@ -65,6 +69,16 @@ constexpr uint16_t kBothCtas = 0x3;
 // kEpiSwiGLU; with g = dH of the same outputs the epilogue writes du = g b silu'(a)
 // and dv = g silu(a) (bf16, row stride 2N: du in columns [0, N), dv in [N, 2N)).
 enum Epilogue { kEpiSwiGLU = 0, kEpiStoreF32 = 1, kEpiBwdSwiGLU = 2 };
+
+// Pipeline depth and shared memory of each epilogue kind (only the backward SwiGLU
+// step needs the exchange buffer).
+__host__ __device__ constexpr int stages_of(int epi) { return epi == kEpiBwdSwiGLU ? 6 : 7; }
+__host__ __device__ constexpr int smem_bytes_of(int epi) {
+    return stages_of(epi) * kStageBytes + 1024 /*align*/ + 1024 /*bookkeeping*/ +
+           (epi == kEpiBwdSwiGLU ? kXferBytes : 0);
+}
+static_assert(smem_bytes_of(kEpiSwiGLU) <= 227 * 1024, "shared memory per CTA");
+static_assert(smem_bytes_of(kEpiBwdSwiGLU) <= 227 * 1024, "shared memory per CTA");
 // B operand: K-major weight rows (the forward), or MN-major (weights [K, N] read as
 // 64 x 64 boxes; backward dH = dY W2), optionally taken from W1 for k < h and from W3
 // for k >= h (backward dX = [du dv] [W1; W3]).
@@ -87,8 +101,8 @@ struct PairArgs {
 };
 
 struct PairBook {
-    uint64_t full[kStages];
-    uint64_t empty[kStages];
+    uint64_t full[kMaxStages];
+    uint64_t empty[kMaxStages];
     uint64_t tmem_full[2];
     uint64_t tmem_empty[2];
     uint64_t drain;
@@ -135,12 +149,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                              const __grid_constant__ CUtensorMap tmB0,
                              const __grid_constant__ CUtensorMap tmB1, const PairArgs args) {
+    constexpr int kStages = stages_of(EPI);
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     uint8_t* sA = smem;
     uint8_t* sB = smem + kStages * kABytes;
     PairBook& bk = *reinterpret_cast<PairBook*>(smem + kStages * kStageBytes);
+    // exchange buffer of the backward SwiGLU half-tile epilogue (kEpiBwdSwiGLU only)
     float* xfer = reinterpret_cast<float*>(smem + kStages * kStageBytes + 1024);
     volatile int* abort_flag = &bk.abort_flag;
 
@@ -206,13 +222,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t phase = 0;
             uint32_t pending = 0, pending_phase = 0;
             bool ok = true, issued = false;
-            constexpr bool kStacked = EPI != kEpiStoreF32;  // B = [W1 rows | W3 rows]
+            // kEpiBwdSwiGLU: B = [128 W1 rows (leader) | the same 128 W3 rows (peer)]
+            constexpr bool kStacked = EPI == kEpiBwdSwiGLU;
             const CUtensorMap* tmB = (kStacked && !leader) ? &tmB1 : &tmB0;
             for (int tile = pair; ok && tile < total; tile += npairs) {
                 const PairTile t = decode_pair_tile(bk, E, tile);
                 const int a_row = t.row0 + static_cast<int>(rank) * (t.half ? 64 : kRowsPerCta);
-                const int b_row = t.e * args.b_rows + t.nt * (kStacked ? 128 : 256) +
-                                  (kStacked ? 0 : static_cast<int>(rank) * 128);
+                const int b_row =
+                    EPI == kEpiSwiGLU
+                        ? t.e * args.b_rows + t.nt * 128 + static_cast<int>(rank) * 64
+                        : t.e * args.b_rows + t.nt * (kStacked ? 128 : 256) +
+                              (kStacked ? 0 : static_cast<int>(rank) * 128);
                 const int b_col = t.nt * 256 + static_cast<int>(rank) * 128;  // MN-major B
                 for (int kb = 0; kb < num_kb; ++kb) {
                     if (!mbar_wait_bounded(&bk.empty[stage], phase ^ 1u, abort_flag,
@@ -224,7 +244,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (leader) mbar_arrive_expect_tx(&bk.full[stage], 2 * kStageBytes);
                     const int kc = kb * kBK;
                     tma_load_2d_pair(&tmA, full_leader, sA + stage * kABytes, kc, a_row);
-                    if (BOP == kBKMajor) {
+                    if (EPI == kEpiSwiGLU) {
+                        // 64 W1 rows, then the same 64 W3 rows (64-row boxes)
+                        tma_load_2d_pair(&tmB0, full_leader, sB + stage * kBBytes, kc, b_row);
+                        tma_load_2d_pair(&tmB1, full_leader, sB + stage * kBBytes + kBBytes / 2,
+                                         kc, b_row);
+                    } else if (BOP == kBKMajor) {
                         tma_load_2d_pair(tmB, full_leader, sB + stage * kBBytes, kc, b_row);
                     } else {
                         const CUtensorMap* mb = &tmB0;
@@ -329,11 +354,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                     __nv_bfloat16* out =
                         static_cast<__nv_bfloat16*>(args.out) + static_cast<size_t>(row) * args.N;
                     const int col0 = t.nt * 128;
+                    // chunk c: outputs col0 + 32c .. +31, a in accumulator column
+                    // (c / 2) * 128 + (c % 2) * 32, b 64 columns further
 #pragma unroll 1
                     for (int ch = 0; ch < 4; ++ch) {
+                        const uint32_t ca = static_cast<uint32_t>((ch >> 1) * 128 + (ch & 1) * 32);
                         uint32_t a[32], b[32];
-                        tmem_ld_32cols(tlane + ch * 32, a);
-                        tmem_ld_32cols(tlane + 128 + ch * 32, b);
+                        tmem_ld_32cols(tlane + ca, a);
+                        tmem_ld_32cols(tlane + ca + 64, b);
                         tmem_ld_wait();
                         uint32_t p[16];
 #pragma unroll
@@ -421,27 +449,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const bool valid = row < t.row_end;
                 const bool upper = q >= 2;  // holds tile columns 128..255
                 if (EPI == kEpiSwiGLU) {
+                    // lanes 0..63 hold the leader's 64 outputs (a in columns 0..63, b in
+                    // 64..127), lanes 64..127 the peer's: each thread writes 64 outputs
                     __nv_bfloat16* out =
                         static_cast<__nv_bfloat16*>(args.out) + static_cast<size_t>(row) * args.N;
-                    const int col0 = t.nt * 128;
+                    const int col0 = t.nt * 128 + (upper ? 64 : 0);
 #pragma unroll 1
-                    for (int ch = 0; ch < 4; ++ch) {
-                        uint32_t v[32];
-                        tmem_ld_32cols(tlane + ch * 32, v);
+                    for (int ch = 0; ch < 2; ++ch) {
+                        uint32_t a[32], b[32];
+                        tmem_ld_32cols(tlane + ch * 32, a);
+                        tmem_ld_32cols(tlane + 64 + ch * 32, b);
                         tmem_ld_wait();
-                        if (upper) {  // b for rows m, columns ch*32 .. ch*32+31
-#pragma unroll
-                            for (int j = 0; j < 32; ++j) xfer[j * 64 + m] = bits_f32(v[j]);
-                        }
-                        asm volatile("bar.sync %0, %1;" ::"r"(kXferBarrier), "r"(kEpiThreads)
-                                     : "memory");
-                        if (!upper && valid) {
+                        if (valid) {
                             uint32_t p[16];
 #pragma unroll
                             for (int i = 0; i < 16; ++i)
-                                p[i] = pack_bf16x2(silu_mul(bits_f32(v[2 * i]), xfer[(2 * i) * 64 + m]),
-                                                   silu_mul(bits_f32(v[2 * i + 1]),
-                                                            xfer[(2 * i + 1) * 64 + m]));
+                                p[i] = pack_bf16x2(silu_mul(bits_f32(a[2 * i]), bits_f32(b[2 * i])),
+                                                   silu_mul(bits_f32(a[2 * i + 1]),
+                                                            bits_f32(b[2 * i + 1])));
 #pragma unroll
                             for (int u = 0; u < 4; ++u) {
                                 const int col = col0 + ch * 32 + u * 8;
@@ -450,8 +475,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                                         make_uint4(p[4 * u], p[4 * u + 1], p[4 * u + 2], p[4 * u + 3]);
                             }
                         }
-                        asm volatile("bar.sync %0, %1;" ::"r"(kXferBarrier), "r"(kEpiThreads)
-                                     : "memory");
                     }
                 } else if (EPI == kEpiBwdSwiGLU) {
                     const int N = args.N;
@@ -535,6 +558,7 @@ template <int EPI, int BOP = kBKMajor>
 cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
                         const PairArgs& args, int npairs, cudaStream_t s) {
     auto kern = grouped_gemm_pair_kernel<EPI, BOP>;
+    constexpr int kSmemBytes = smem_bytes_of(EPI);
     static PerDeviceOnce smem_once;
     if (const cudaError_t err = opt_in_smem(smem_once, kern, kSmemBytes); err != cudaSuccess)
         return err;
@@ -563,8 +587,8 @@ cudaError_t launch_ffn_bf16_pair(const void* x_perm, const int32_t* offsets, con
                                  cudaEvent_t between, int cap) {
     CUtensorMap mx, mw1, mw3, mh, mw2;
     if (!encode_bf16_2d(&mx, x_perm, rows, d, kRowsPerCta) ||
-        !encode_bf16_2d(&mw1, W1, static_cast<uint64_t>(E) * h, d, 128) ||
-        !encode_bf16_2d(&mw3, W3, static_cast<uint64_t>(E) * h, d, 128) ||
+        !encode_bf16_2d(&mw1, W1, static_cast<uint64_t>(E) * h, d, 64) ||
+        !encode_bf16_2d(&mw3, W3, static_cast<uint64_t>(E) * h, d, 64) ||
         !encode_bf16_2d(&mh, H, rows, h, kRowsPerCta) ||
         !encode_bf16_2d(&mw2, W2, static_cast<uint64_t>(E) * d, h, 128))
         return cudaErrorInvalidValue;

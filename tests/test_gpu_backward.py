@@ -3,11 +3,16 @@
 The gradients pass through several bf16 roundings that the oracle does not make:
 the scaled upstream rows w*dy (one rounding each), H saved by the forward, and du,
 dv (one rounding each) feed tensor-core GEMMs with fp32 accumulation.  Each rounding
-is a relative error of at most 2^-9 per element, independent across elements, so
-over the three to four roundings on any path a relative Frobenius error of a few
-1e-3 is expected; the gate is 1e-2 (and 2e-2 for the router gradient, whose logit
-gap (dw1 - dw2) can cancel).  Full-size layers are checked on sampled tokens and
-sampled weight entries that the oracle computes one by one.
+is a relative error of at most 2^-9 per element (about 2^-9/sqrt(3) = 1.1e-3 RMS for
+uniformly distributed rounding errors), independent across elements, so two to three
+roundings on a path give a relative Frobenius error of about 2e-3 to 3e-3.  Measured
+over every case below (B200): dx 2.4e-3 .. 2.8e-3, dW1/dW3/dW2 1.8e-3 .. 2.5e-3,
+dWg 1.3e-3 .. 3.5e-3 (the router gradient also carries the cancellation in dw1 - dw2,
+largest on the smallest shape).  The gates are about twice the measured maxima: 6e-3,
+and 7e-3 for dWg.  Full-size layers are checked on sampled tokens (each token's dx
+row against the same 6e-3) and on sampled weight-gradient entries that the oracle
+computes one by one; a single entry is a sum whose rounding errors do not average
+out as a whole matrix's do, so entries are held to 1e-2 of their row's scale.
 """
 import numpy as np
 import pytest
@@ -19,8 +24,9 @@ from workloads import WORKLOADS, make_inputs, small
 
 pytestmark = pytest.mark.gpu
 
-BWD_TOL = 1e-2
-ROUTER_TOL = 2e-2
+BWD_TOL = 6e-3
+ROUTER_TOL = 7e-3
+ENTRY_TOL = 1e-2
 
 
 def f64(t):
@@ -206,7 +212,7 @@ def test_backward_full_size_sampled(workload):
         got = g[name][e, r_, c_].item()
         row = f64(g[name][e, r_])
         scale = np.linalg.norm(row) / np.sqrt(row.size) + 1e-30
-        assert abs(got - v) <= BWD_TOL * max(abs(v), scale), (key, got, v)
+        assert abs(got - v) <= ENTRY_TOL * max(abs(v), scale), (key, got, v)
 
 
 @pytest.mark.parametrize("T,E", [(40, 4), (300, 16), (1200, 2)])
