@@ -25,9 +25,15 @@
 // columns 0..127 of the tile in TMEM lanes 0..63 and columns 128..255 in lanes
 // 64..127, both in the first 128 TMEM columns of the buffer.
 //
-// Without an exchange buffer in the epilogue, the forward GEMMs and the backward's
-// fp32-output GEMMs keep 7 pipeline stages (224 KiB); the backward SwiGLU step, whose
-// half-tile epilogue exchanges b through shared memory, keeps 6.
+// Pipeline depth: GEMM1 keeps 7 stages (224 KiB).  The fp32-output GEMMs (GEMM2 and
+// the backward's dH and dX) keep 6 and use the rest for their store epilogue: each
+// epilogue warp stages 32 rows x 32 columns of its accumulator rows in shared memory
+// (128-byte swizzle) and one lane writes them with a TMA tensor store, so every row
+// segment leaves as whole 128-byte lines instead of 16-byte pieces from 32 rows at a
+// time.  A chunk whose 32 rows are not all inside the expert's group (the last block
+// of a group, whose further rows belong to the next expert) is stored row by row.
+// The backward SwiGLU step, whose half-tile epilogue exchanges b through shared
+// memory, keeps 6 stages.
 //
 // Synchronisation: both CTAs' TMA loads count their bytes on the leader's "full"
 // barrier; the leader's MMA completions are multicast to both CTAs' "empty" and
@@ -44,6 +50,8 @@ namespace moe {
 // Defined in grouped_gemm_sm100.cu.
 bool encode_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
                     uint32_t box_rows);
+bool encode_f32_3d(CUtensorMap* map, const void* base, uint64_t batches, uint64_t rows,
+                   uint64_t cols, uint32_t box_cols, uint32_t box_rows);
 
 namespace {
 
@@ -70,13 +78,18 @@ constexpr uint16_t kBothCtas = 0x3;
 // and dv = g silu(a) (bf16, row stride 2N: du in columns [0, N), dv in [N, 2N)).
 enum Epilogue { kEpiSwiGLU = 0, kEpiStoreF32 = 1, kEpiBwdSwiGLU = 2 };
 
-// Pipeline depth and shared memory of each epilogue kind (only the backward SwiGLU
-// step needs the exchange buffer).
-__host__ __device__ constexpr int stages_of(int epi) { return epi == kEpiBwdSwiGLU ? 6 : 7; }
+// fp32 store staging: per epilogue warp two 32 x 32 fp32 chunks (4 KiB each).
+constexpr int kOutChunkBytes = 32 * 32 * 4;
+constexpr int kOutBufs = 2;
+constexpr int kOutStageBytes = (kEpiThreads / 32) * kOutBufs * kOutChunkBytes;
+
+// Pipeline depth and shared memory of each epilogue kind.
+__host__ __device__ constexpr int stages_of(int epi) { return epi == kEpiSwiGLU ? 7 : 6; }
 __host__ __device__ constexpr int smem_bytes_of(int epi) {
     return stages_of(epi) * kStageBytes + 1024 /*align*/ + 1024 /*bookkeeping*/ +
-           (epi == kEpiBwdSwiGLU ? kXferBytes : 0);
+           (epi == kEpiBwdSwiGLU ? kXferBytes : epi == kEpiStoreF32 ? kOutStageBytes : 0);
 }
+static_assert(smem_bytes_of(kEpiStoreF32) <= 227 * 1024, "shared memory per CTA");
 static_assert(smem_bytes_of(kEpiSwiGLU) <= 227 * 1024, "shared memory per CTA");
 static_assert(smem_bytes_of(kEpiBwdSwiGLU) <= 227 * 1024, "shared memory per CTA");
 // B operand: K-major weight rows (the forward), or MN-major (weights [K, N] read as
@@ -148,7 +161,8 @@ template <int EPI, int BOP = kBKMajor>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                              const __grid_constant__ CUtensorMap tmB0,
-                             const __grid_constant__ CUtensorMap tmB1, const PairArgs args) {
+                             const __grid_constant__ CUtensorMap tmB1,
+                             const __grid_constant__ CUtensorMap tmOut, const PairArgs args) {
     constexpr int kStages = stages_of(EPI);
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -156,8 +170,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t* sA = smem;
     uint8_t* sB = smem + kStages * kABytes;
     PairBook& bk = *reinterpret_cast<PairBook*>(smem + kStages * kStageBytes);
-    // exchange buffer of the backward SwiGLU half-tile epilogue (kEpiBwdSwiGLU only)
+    // exchange buffer of the backward SwiGLU half-tile epilogue (kEpiBwdSwiGLU), or the
+    // fp32 store staging (kEpiStoreF32)
     float* xfer = reinterpret_cast<float*>(smem + kStages * kStageBytes + 1024);
+    uint8_t* out_stage = smem + kStages * kStageBytes + 1024;
     volatile int* abort_flag = &bk.abort_flag;
 
     const int warp = threadIdx.x >> 5;
@@ -185,6 +201,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB0);
         if (EPI != kEpiStoreF32 || BOP == kBMnSplit) tma_prefetch_desc(&tmB1);
+        if (EPI == kEpiStoreF32) tma_prefetch_desc(&tmOut);
     }
     if (warp == 1) tmem_alloc_pair(&bk.tmem_base, kTmemCols);
 
@@ -335,6 +352,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
         // ------------------------------------------------------------ epilogue (both CTAs)
         const int q = warp & 3;
+        uint8_t* wstage = out_stage + q * kOutBufs * kOutChunkBytes;  // this warp's staging
+        int obuf = 0;
         const uint32_t empty_leader0 = map_to_cta(smem_u32(&bk.tmem_empty[0]), 0);
         const uint32_t empty_leader1 = map_to_cta(smem_u32(&bk.tmem_empty[1]), 0);
         int acc = 0;
@@ -424,12 +443,32 @@ __global__ void __launch_bounds__(kThreads, 1)
                 } else {
                     float* out = static_cast<float*>(args.out) + static_cast<size_t>(row) * args.N;
                     const int col0 = t.nt * 256;
+                    const int wrow0 = t.row0 + static_cast<int>(rank) * kRowsPerCta + q * 32;
+                    const bool whole = wrow0 + 32 <= t.row_end;  // all 32 rows in the group
 #pragma unroll 1
                     for (int ch = 0; ch < 8; ++ch) {
                         uint32_t v[32];
                         tmem_ld_32cols(tlane + ch * 32, v);
                         tmem_ld_wait();
-                        if (valid) {
+                        if (col0 + ch * 32 >= args.N) continue;
+                        if (whole) {
+                            // TMA store of 32 rows x 32 columns (columns past N are outside
+                            // the tensor and not written)
+                            uint8_t* st = wstage + obuf * kOutChunkBytes;
+                            if (lane == 0) bulk_wait_group_read<kOutBufs - 1>();
+                            __syncwarp();
+#pragma unroll
+                            for (int j = 0; j < 8; ++j)
+                                *reinterpret_cast<uint4*>(st + lane * 128 + ((j ^ (lane & 7)) << 4)) =
+                                    make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+                            fence_proxy_async_smem();
+                            __syncwarp();
+                            if (lane == 0) {
+                                tma_store_3d(&tmOut, st, col0 + ch * 32, wrow0, 0);
+                                bulk_commit_group();
+                            }
+                            if (++obuf == kOutBufs) obuf = 0;
+                        } else if (valid) {
 #pragma unroll
                             for (int j = 0; j < 8; ++j) {
                                 const int col = col0 + ch * 32 + j * 4;
@@ -543,6 +582,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             acc ^= 1;
             if (acc == 0) acc_phase ^= 1u;
         }
+        if (EPI == kEpiStoreF32 && lane == 0)
+            bulk_wait_group<0>();  // every tensor store complete before the block exits
     }
 
     tc_fence_before();
@@ -556,7 +597,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <int EPI, int BOP = kBKMajor>
 cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
-                        const PairArgs& args, int npairs, cudaStream_t s) {
+                        const CUtensorMap& o, const PairArgs& args, int npairs, cudaStream_t s) {
     auto kern = grouped_gemm_pair_kernel<EPI, BOP>;
     constexpr int kSmemBytes = smem_bytes_of(EPI);
     static PerDeviceOnce smem_once;
@@ -574,7 +615,7 @@ cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b0, const CUten
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t err = cudaLaunchKernelEx(&cfg, kern, a, b0, b1, args);
+    cudaError_t err = cudaLaunchKernelEx(&cfg, kern, a, b0, b1, o, args);
     return err != cudaSuccess ? err : cudaGetLastError();
 }
 
@@ -585,8 +626,9 @@ cudaError_t launch_ffn_bf16_pair(const void* x_perm, const int32_t* offsets, con
                                  const void* W3, const void* W2, int rows, int d, int h, int E,
                                  void* H, float* Y, uint32_t* status, cudaStream_t s,
                                  cudaEvent_t between, int cap) {
-    CUtensorMap mx, mw1, mw3, mh, mw2;
-    if (!encode_bf16_2d(&mx, x_perm, rows, d, kRowsPerCta) ||
+    CUtensorMap mx, mw1, mw3, mh, mw2, my;
+    if (!encode_f32_3d(&my, Y, 1, rows, d, 32, 32) ||
+        !encode_bf16_2d(&mx, x_perm, rows, d, kRowsPerCta) ||
         !encode_bf16_2d(&mw1, W1, static_cast<uint64_t>(E) * h, d, 64) ||
         !encode_bf16_2d(&mw3, W3, static_cast<uint64_t>(E) * h, d, 64) ||
         !encode_bf16_2d(&mh, H, rows, h, kRowsPerCta) ||
@@ -597,13 +639,13 @@ cudaError_t launch_ffn_bf16_pair(const void* x_perm, const int32_t* offsets, con
     PairArgs g1{offsets, E, rows, d, h, h, (h + 127) / 128, H, status, cap};
     long long t1 = blocks * g1.n_tiles;
     cudaError_t err = launch_pair<kEpiSwiGLU>(
-        mx, mw1, mw3, g1, static_cast<int>(t1 < max_pairs ? (t1 < 1 ? 1 : t1) : max_pairs), s);
+        mx, mw1, mw3, mx, g1, static_cast<int>(t1 < max_pairs ? (t1 < 1 ? 1 : t1) : max_pairs), s);
     if (err != cudaSuccess) return err;
     if (between && (err = cudaEventRecord(between, s)) != cudaSuccess) return err;
     PairArgs g2{offsets, E, rows, h, d, d, (d + 255) / 256, Y, status, cap};
     long long t2 = blocks * g2.n_tiles;
     return launch_pair<kEpiStoreF32>(
-        mh, mw2, mw2, g2, static_cast<int>(t2 < max_pairs ? (t2 < 1 ? 1 : t2) : max_pairs), s);
+        mh, mw2, mw2, my, g2, static_cast<int>(t2 < max_pairs ? (t2 < 1 ? 1 : t2) : max_pairs), s);
 }
 
 // Backward row-grouped GEMMs on CTA pairs (the backward pass is described in
@@ -621,15 +663,19 @@ cudaError_t launch_bwd_rows_pair(int mode, const CUtensorMap& a, const CUtensorM
         return static_cast<int>(tiles < max_pairs ? (tiles < 1 ? 1 : tiles) : max_pairs);
     };
     if (mode == 0) {
+        CUtensorMap mo;  // dH [rows, h] fp32
+        if (!encode_f32_3d(&mo, out, 1, rows, h, 32, 32)) return cudaErrorInvalidValue;
         PairArgs g{offsets, E, rows, d, h, d, (h + 255) / 256, out, status, cap, h, nullptr};
-        return launch_pair<kEpiStoreF32, kBMn>(a, b0, b0, g, grid(blocks * g.n_tiles), s);
+        return launch_pair<kEpiStoreF32, kBMn>(a, b0, b0, mo, g, grid(blocks * g.n_tiles), s);
     }
     if (mode == 1) {
         PairArgs g{offsets, E, rows, d, h, h, (h + 127) / 128, out, status, cap, h, dH};
-        return launch_pair<kEpiBwdSwiGLU, kBKMajor>(a, b0, b1, g, grid(blocks * g.n_tiles), s);
+        return launch_pair<kEpiBwdSwiGLU, kBKMajor>(a, b0, b1, a, g, grid(blocks * g.n_tiles), s);
     }
+    CUtensorMap mo;  // dX [rows, d] fp32
+    if (!encode_f32_3d(&mo, out, 1, rows, d, 32, 32)) return cudaErrorInvalidValue;
     PairArgs g{offsets, E, rows, 2 * h, d, h, (d + 255) / 256, out, status, cap, h, nullptr};
-    return launch_pair<kEpiStoreF32, kBMnSplit>(a, b0, b1, g, grid(blocks * g.n_tiles), s);
+    return launch_pair<kEpiStoreF32, kBMnSplit>(a, b0, b1, mo, g, grid(blocks * g.n_tiles), s);
 }
 
 }  // namespace moe
