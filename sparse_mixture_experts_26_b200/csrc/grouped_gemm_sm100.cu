@@ -14,16 +14,22 @@
 //   A = grouped activations [rows, K], B = the expert's weight rows [N, K].
 //
 // Design (one CTA per SM, persistent, 6 warps):
-//   warp 0      TMA producer: 128x64 A tile + 256x64 B tile per stage (48 KiB),
-//               kStages-deep ring of shared-memory stages guarded by mbarriers.
+//   warp 0      TMA producer: 128x64 A tile + (2 NO)x64 or 256x64 B tile per stage,
+//               a ring of shared-memory stages guarded by mbarriers.
 //   warp 1      allocates 512 TMEM columns; one thread issues tcgen05.mma
-//               (M=128, N=256, K=16; four per 64-wide K block) into one of two
-//               128x256 fp32 accumulators, and commits stage/accumulator barriers.
+//               (M=128, N=2 NO or 256, K=16; four per 64-wide K block) into one of
+//               two fp32 accumulators 256 columns apart, and commits stage/accumulator
+//               barriers.
 //   warps 2-5   epilogue: tcgen05.ld the accumulator (one row per thread), apply
 //               silu(a)*b (GEMM1) or nothing (GEMM2), store to global, release
 //               the accumulator.  The other accumulator is being filled meanwhile.
-// For GEMM1 the B tile stacks 128 rows of W1 over the same 128 rows of W3, so
-// accumulator columns [0,128) hold a and [128,256) hold b for the same outputs.
+// For GEMM1 the B tile stacks NO rows of W1 over the same NO rows of W3, so
+// accumulator columns [0,NO) hold a and [NO,2 NO) hold b for the same outputs.  NO is
+// 128, or 112 when h is a multiple of 112: a batch of 129..511 tokens has one or two
+// 128-row blocks per expert, and with Mixtral's h = 14336 the 112 columns give
+// 8 x 128 = 1024 tiles (6.9 rounds of 148 SMs, the last one full) instead of
+// 8 x 112 = 896 (6.05 rounds, the 7th nearly empty); the smaller stage (44 KiB) also
+// lets 5 stages fit instead of 4.
 //
 // Tiles never mix experts' weights: a tile is (expert, 128-row block of that
 // expert's rows, output-column block).  A row block may run past the expert's last
@@ -44,18 +50,30 @@ namespace {
 
 constexpr int kBM = 128;        // rows per tile (TMEM lanes)
 constexpr int kBK = 64;         // K per stage: one 128-byte swizzle atom of bf16
-constexpr int kMmaN = 256;      // accumulator columns per tile
-constexpr int kStages = 4;
+constexpr int kMmaN = 256;      // accumulator stride (columns) in TMEM
+constexpr int kMaxStages = 5;
 constexpr int kABytes = kBM * kBK * 2;      // 16 KiB
-constexpr int kBBytes = kMmaN * kBK * 2;    // 32 KiB
-constexpr int kStageBytes = kABytes + kBBytes;
 constexpr int kThreads = 192;
 constexpr int kEpiThreads = 128;
 constexpr uint32_t kTmemCols = 2 * kMmaN;   // two accumulators: all 512 columns
-constexpr uint32_t kIdesc = idesc_bf16_f32(kBM, kMmaN);
-constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 1024 /*bookkeeping*/;
 
 enum Epilogue { kEpiSwiGLU = 0, kEpiStoreF32 = 1 };
+
+// Shape of one instantiation: GEMM1 tiles cover NO outputs (B = NO W1 rows + NO W3
+// rows), GEMM2 tiles 256 output columns.  Stages fill the shared memory.
+template <int EPI, int NO>
+struct GemmShape {
+    static constexpr int kBRows = EPI == kEpiSwiGLU ? 2 * NO : 256;
+    static constexpr int kBBytes = kBRows * kBK * 2;
+    static constexpr int kStageBytes = kABytes + kBBytes;
+    static constexpr int kStages = (227 * 1024 - 2048) / kStageBytes < kMaxStages
+                                       ? (227 * 1024 - 2048) / kStageBytes
+                                       : kMaxStages;
+    static constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 1024 /*book*/;
+    static constexpr uint32_t kIdesc = idesc_bf16_f32(kBM, kBRows);
+    static_assert(kBRows % 16 == 0 && kBRows <= 256, "MMA N");
+    static_assert((NO * kBK * 2) % 1024 == 0, "W3 half of B must start on a swizzle atom");
+};
 
 struct GemmArgs {
     const int32_t* offsets;  // [E+1] group row offsets (device)
@@ -71,8 +89,8 @@ struct GemmArgs {
 };
 
 struct Bookkeeping {
-    uint64_t full[kStages];
-    uint64_t empty[kStages];
+    uint64_t full[kMaxStages];
+    uint64_t empty[kMaxStages];
     uint64_t tmem_full[2];
     uint64_t tmem_empty[2];
     uint64_t drain;
@@ -105,11 +123,15 @@ __device__ __forceinline__ float silu_mul(float a, float b) {
     return a / (1.0f + __expf(-a)) * b;
 }
 
-template <int EPI>
+template <int EPI, int NO>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB0,
                         const __grid_constant__ CUtensorMap tmB1, const GemmArgs args) {
+    using S = GemmShape<EPI, NO>;
+    constexpr int kStages = S::kStages;
+    constexpr int kBBytes = S::kBBytes;
+    constexpr int kStageBytes = S::kStageBytes;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -180,7 +202,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             bool ok = true;
             for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
                 const TileCoord c = decode_tile(bk, E, tile);
-                const int brow = c.e * args.b_rows + c.nt * (EPI == kEpiSwiGLU ? 128 : 256);
+                const int brow = c.e * args.b_rows + c.nt * (EPI == kEpiSwiGLU ? NO : 256);
                 for (int kb = 0; kb < num_kb; ++kb) {
                     if (!mbar_wait_bounded(&bk.empty[stage], phase ^ 1u, abort_flag,
                                            args.status)) {
@@ -192,7 +214,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     uint8_t* a_dst = sA + stage * kABytes;
                     uint8_t* b_dst = sB + stage * kBBytes;
                     tma_load_2d(&tmA, &bk.full[stage], a_dst, kc, c.row0);
-                    if (EPI == kEpiSwiGLU) {
+                    if (EPI == kEpiSwiGLU) {  // NO-row boxes: W1 rows, then W3 rows
                         tma_load_2d(&tmB0, &bk.full[stage], b_dst, kc, brow);
                         tma_load_2d(&tmB1, &bk.full[stage], b_dst + kBBytes / 2, kc, brow);
                     } else {
@@ -240,7 +262,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint64_t bd = sw128_kmajor_desc(smem_u32(sB + stage * kBBytes));
 #pragma unroll
                     for (int k = 0; k < kBK / 16; ++k)
-                        umma_bf16(d_tmem, ad + 2 * k, bd + 2 * k, kIdesc, (kb | k) != 0);
+                        umma_bf16(d_tmem, ad + 2 * k, bd + 2 * k, S::kIdesc, (kb | k) != 0);
                     umma_commit(&bk.empty[stage]);
                     issued = true;
                     if (++stage == kStages) {
@@ -275,15 +297,41 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * kMmaN);
             const int row = c.row0 + row_in_tile;
             const bool valid = row < c.row_end;
-            if (EPI == kEpiSwiGLU) {
+            if (EPI == kEpiSwiGLU && NO % 32 != 0) {
+                // a in columns [0, NO), b in [NO, 2 NO): 16-column chunks
                 __nv_bfloat16* out =
                     static_cast<__nv_bfloat16*>(args.out) + static_cast<size_t>(row) * args.N;
-                const int col0 = c.nt * 128;
+                const int col0 = c.nt * NO;
 #pragma unroll 1
-                for (int ch = 0; ch < 4; ++ch) {
+                for (int ch = 0; ch < NO / 16; ++ch) {
+                    uint32_t a[16], b[16];
+                    tmem_ld_16cols(tbase + ch * 16, a);
+                    tmem_ld_16cols(tbase + NO + ch * 16, b);
+                    tmem_ld_wait();
+                    uint32_t p[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        p[i] = pack_bf16x2(silu_mul(bits_f32(a[2 * i]), bits_f32(b[2 * i])),
+                                           silu_mul(bits_f32(a[2 * i + 1]), bits_f32(b[2 * i + 1])));
+                    if (valid) {
+#pragma unroll
+                        for (int v = 0; v < 2; ++v) {
+                            const int col = col0 + ch * 16 + v * 8;
+                            if (col < args.N)
+                                *reinterpret_cast<uint4*>(out + col) =
+                                    make_uint4(p[4 * v], p[4 * v + 1], p[4 * v + 2], p[4 * v + 3]);
+                        }
+                    }
+                }
+            } else if (EPI == kEpiSwiGLU) {
+                __nv_bfloat16* out =
+                    static_cast<__nv_bfloat16*>(args.out) + static_cast<size_t>(row) * args.N;
+                const int col0 = c.nt * NO;
+#pragma unroll 1
+                for (int ch = 0; ch < NO / 32; ++ch) {
                     uint32_t a[32], b[32];
                     tmem_ld_32cols(tbase + ch * 32, a);
-                    tmem_ld_32cols(tbase + 128 + ch * 32, b);
+                    tmem_ld_32cols(tbase + NO + ch * 32, b);
                     tmem_ld_wait();
                     uint32_t p[16];
 #pragma unroll
@@ -335,10 +383,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-template <int EPI>
+template <int EPI, int NO = 128>
 cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
                         const GemmArgs& args, int grid, cudaStream_t s) {
-    auto kern = grouped_gemm_kernel<EPI>;
+    auto kern = grouped_gemm_kernel<EPI, NO>;
+    constexpr int kSmemBytes = GemmShape<EPI, NO>::kSmemBytes;
     static PerDeviceOnce smem_once;
     if (const cudaError_t err = opt_in_smem(smem_once, kern, kSmemBytes); err != cudaSuccess)
         return err;
@@ -444,10 +493,12 @@ cudaError_t launch_ffn_bf16(const void* x_perm, const int32_t* offsets, const vo
     if (rows >= kPairMinRows && pair_gemm_enabled())
         return launch_ffn_bf16_pair(x_perm, offsets, W1, W3, W2, rows, d, h, E, H, Y, status, s,
                                     between, cap);
+    // GEMM1 tile width: 112 outputs where h is a multiple of 112 (see the file comment)
+    const int no = h % 112 == 0 ? 112 : 128;
     CUtensorMap mx, mw1, mw3, mh, mw2;
     if (!encode_bf16_2d(&mx, x_perm, rows, d, kBM) ||
-        !encode_bf16_2d(&mw1, W1, static_cast<uint64_t>(E) * h, d, 128) ||
-        !encode_bf16_2d(&mw3, W3, static_cast<uint64_t>(E) * h, d, 128) ||
+        !encode_bf16_2d(&mw1, W1, static_cast<uint64_t>(E) * h, d, no) ||
+        !encode_bf16_2d(&mw3, W3, static_cast<uint64_t>(E) * h, d, no) ||
         !encode_bf16_2d(&mh, H, rows, h, kBM) ||
         !encode_bf16_2d(&mw2, W2, static_cast<uint64_t>(E) * d, h, 128))
         return cudaErrorInvalidValue;
@@ -456,10 +507,11 @@ cudaError_t launch_ffn_bf16(const void* x_perm, const int32_t* offsets, const vo
     // Upper bound on row blocks: sum_e ceil(n_e / 128) <= (rows + 127 E) / 128.
     const long long row_blocks = (static_cast<long long>(rows) + 127LL * E) / kBM;
 
-    GemmArgs g1{offsets, E, rows, d, h, h, (h + 127) / 128, H, status, cap};
+    GemmArgs g1{offsets, E, rows, d, h, h, (h + no - 1) / no, H, status, cap};
     long long tiles1 = row_blocks * g1.n_tiles;
     int grid1 = static_cast<int>(tiles1 < sms ? (tiles1 < 1 ? 1 : tiles1) : sms);
-    cudaError_t err = launch_gemm<kEpiSwiGLU>(mx, mw1, mw3, g1, grid1, s);
+    cudaError_t err = no == 112 ? launch_gemm<kEpiSwiGLU, 112>(mx, mw1, mw3, g1, grid1, s)
+                                : launch_gemm<kEpiSwiGLU, 128>(mx, mw1, mw3, g1, grid1, s);
     if (err != cudaSuccess) return err;
     if (between && (err = cudaEventRecord(between, s)) != cudaSuccess) return err;
 

@@ -66,7 +66,7 @@ def gpu_grads(inp, dy, capacity=-1):
 SHAPES = [  # (T, d, h, kind): decode-path and grouped-path forwards, ragged tiles
     (1, 64, 128, "plain"), (16, 128, 256, "skew"), (37, 136, 192, "plain"),
     (64, 256, 384, "plain"), (100, 136, 192, "skew"), (128, 256, 384, "plain"),
-    (300, 136, 192, "plain"), (700, 256, 384, "skew"),
+    (300, 136, 192, "plain"), (200, 128, 448, "skew"), (700, 256, 384, "skew"),
     (1100, 256, 384, "plain"), (2500, 128, 256, "long"),
 ]
 

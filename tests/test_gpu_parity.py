@@ -106,8 +106,10 @@ SMALL = [  # (T, d, h, kind): ragged row blocks, K tails, N tails, empty groups
     (5, 136, 200, "plain"), (16, 256, 384, "skew"), (17, 128, 256, "plain"),
     (33, 128, 256, "plain"), (64, 256, 512, "plain"), (65, 128, 256, "plain"),
     (100, 136, 200, "skew"), (128, 256, 512, "plain"),
-    # 128 < T < 512 runs the single-SM grouped GEMM (128-row blocks)
+    # 128 < T < 512 runs the single-SM grouped GEMM (128-row blocks); h a multiple of
+    # 112 selects its 112-output GEMM1 tiles
     (129, 256, 512, "plain"), (300, 136, 200, "plain"), (511, 128, 256, "skew"),
+    (200, 128, 224, "plain"), (300, 256, 448, "skew"), (450, 136, 336, "long"),
     # >= 1024 grouped rows run the CTA-pair grouped GEMM (256-row blocks; an expert's
     # last block of <= 128 rows runs in the pair's 128-row mode)
     (512, 128, 256, "plain"), (513, 128, 256, "long"), (700, 256, 384, "skew"),
