@@ -317,18 +317,18 @@ def measure_forward(wl, inp, K: int, W: int, world: int, local: int, device):
             e.record(stream)
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
 
+    layer_call, events_call = moe.moe_layer_forward, moe.moe_layer_forward_events
     with ClockSampler(local) as clocks:
         for _ in range(W):
-            moe.moe_layer_forward(x, Wg, W1, W3, W2, y, ws)
+            layer_call(x, Wg, W1, W3, W2, y, ws)
         torch.cuda.synchronize()
         barrier(world, device)
         torch.cuda.synchronize()
         start.record(stream)
         for i in range(K):
-            moe.moe_layer_forward_events(x, Wg, W1, W3, W2, y, ws,
-                                         [None, evs[i][0].cuda_event,
-                                          None if fused else evs[i][1].cuda_event,
-                                          evs[i][2].cuda_event])
+            events_call(x, Wg, W1, W3, W2, y, ws,
+                        [None, evs[i][0].cuda_event, None if fused else evs[i][1].cuda_event,
+                         evs[i][2].cuda_event])
         end.record(stream)
         torch.cuda.synchronize()
         barrier(world, device)
@@ -409,7 +409,7 @@ def measure_forward(wl, inp, K: int, W: int, world: int, local: int, device):
                 ev_in[b].record(s_in)
             stream.wait_event(ev_in[b])
             stream.wait_event(ev_out[b])              # y_dev[b] already copied out
-            moe.moe_layer_forward(x_dev[b], Wg, W1, W3, W2, y_dev[b], ws)
+            layer_call(x_dev[b], Wg, W1, W3, W2, y_dev[b], ws)
             ev_layer[b].record(stream)
             with torch.cuda.stream(s_out):
                 s_out.wait_event(ev_layer[b])
@@ -431,10 +431,11 @@ def measure_forward(wl, inp, K: int, W: int, world: int, local: int, device):
            "h2d_bytes_per_step": x.numel() * x.element_size(),
            "d2h_bytes_per_step": y.numel() * y.element_size(),
            "pipeline": "double-buffered: H2D and D2H copies on their own streams"}
+    launches = moe.launches_per_layer(T, d, E, wl.dtype == "bf16")
     return {"value": round(value, 1), "unit": UNIT, "steps": K, "warmup": W,
             "ms_per_step": round(ms, 4), "config": workload_config(wl),
             "roofline": roofline, "layer": layer, "e2e": e2e,
-            "gpu_launches": moe.launches_per_layer(T) * K, "clocks": clocks.summary()}
+            "gpu_launches": launches * K, "clocks": clocks.summary()}
 
 
 def forward_cpu_baseline(inp, wl, args):

@@ -39,13 +39,16 @@ EXPORTED_SYMBOLS = ("moe_workspace_bytes", "moe_route", "moe_permute", "moe_expe
                     "moe_layer_forward_capacity", "moe_selftest_wait_timeout",
                     "moe_backward_workspace_bytes", "moe_layer_backward",
                     "moe_layer_backward_events")
-def launches_per_layer(T: int) -> int:
+def launches_per_layer(T: int, d: int = 4096, E: int = 8, bf16: bool = True) -> int:
     """Kernels one moe_layer_forward queues: router 1, permutation 1 (T <= 512) or 4
-    (count, scan, rank, gather), expert FFN 1 (T <= 128: gate/up and down fused) or 2,
-    combine 1; none for T == 0."""
+    (count, scan, rank, gather; 3 where the bf16 fp64-tensor-core router counts the
+    grouping itself: E <= 8, d a multiple of 32 and at most 6144), expert FFN 1
+    (T <= 128: gate/up and down fused) or 2, combine 1; none for T == 0."""
     if T <= 0:
         return 0
-    return 1 + (1 if T <= 512 else 4) + (1 if T <= 128 else 2) + 1
+    router_counts = bf16 and E <= 8 and d % 32 == 0 and d <= 6144
+    perm = 1 if T <= 512 else (3 if router_counts else 4)
+    return 1 + perm + (1 if T <= 128 else 2) + 1
 
 
 def launches_per_backward(T: int, capacity: int = -1) -> int:

@@ -638,8 +638,8 @@ cudaError_t launch_ffn_bf16_pair(const void* x_perm, const int32_t* offsets, con
     const long long blocks = (static_cast<long long>(rows) + (kPairRows - 1LL) * E) / kPairRows;
     PairArgs g1{offsets, E, rows, d, h, h, (h + 127) / 128, H, status, cap};
     long long t1 = blocks * g1.n_tiles;
-    cudaError_t err = launch_pair<kEpiSwiGLU>(
-        mx, mw1, mw3, mx, g1, static_cast<int>(t1 < max_pairs ? (t1 < 1 ? 1 : t1) : max_pairs), s);
+    const int grid1 = static_cast<int>(t1 < max_pairs ? (t1 < 1 ? 1 : t1) : max_pairs);
+    cudaError_t err = launch_pair<kEpiSwiGLU>(mx, mw1, mw3, mx, g1, grid1, s);
     if (err != cudaSuccess) return err;
     if (between && (err = cudaEventRecord(between, s)) != cudaSuccess) return err;
     PairArgs g2{offsets, E, rows, h, d, d, (d + 255) / 256, Y, status, cap};

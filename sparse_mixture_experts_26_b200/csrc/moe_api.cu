@@ -253,7 +253,9 @@ moe_status moe_combine(const float* y_perm, const int32_t* inv_perm, const float
 namespace moe {
 namespace {
 
-// The layer, with optional events recorded between its stages (profiling).
+// The layer, with optional events recorded between its stages (profiling).  Above 512
+// tokens (the four-launch grouping) the fp64 tensor-core router also counts the pairs
+// of every chunk per expert, so the grouping skips its count pass.
 moe_status layer_forward_impl(const void* x, const void* Wg, const void* W1, const void* W3,
                               const void* W2, int T, int d, int h, int E, int k, moe_dtype dt,
                               void* y, void* ws, size_t ws_bytes, cudaEvent_t* ev, int n_ev,
@@ -279,19 +281,21 @@ moe_status layer_forward_impl(const void* x, const void* Wg, const void* W1, con
         return i >= n_ev || ev[i] == nullptr || cudaEventRecord(ev[i], stream) == cudaSuccess;
     };
 
+    const bool counts_in_router = T > kPermSmallTokens && dmma_route_applies(T, d, E, dt);
     NvtxRange layer_range("moe_layer_forward");
     if (!mark(0)) return MOE_ERR_CUDA;
     cudaError_t err;
     {
         NvtxRange r("route");
-        err = launch_route(x, Wg, T, d, E, dt, idx, w, stream);
+        err = launch_route(x, Wg, T, d, E, dt, idx, w, stream,
+                           counts_in_router ? at<int32_t>(ws, L.blk_counts) : nullptr);
     }
     if ((st = finish(err, stream, status)) != MOE_OK) return st;
     {
         NvtxRange r("permute");
         err = launch_permute(idx, x, T, d, E, dt, offsets, perm_token, inv_perm, x_perm,
                              at<int32_t>(ws, L.blk_counts), at<int32_t>(ws, L.blk_base), status,
-                             stream);
+                             stream, counts_in_router);
     }
     if ((st = finish(err, stream, status)) != MOE_OK) return st;
     if (!mark(1)) return MOE_ERR_CUDA;

@@ -148,12 +148,21 @@ cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
 }
 
 // ---- launchers (each returns cudaGetLastError() of its launch) ----
+// With `blk_counts` (zero on entry) the router also counts the pairs of every
+// kPermChunk-token chunk per expert (only where dmma_route_applies(); otherwise
+// cudaErrorInvalidValue).
 cudaError_t launch_route(const void* x, const void* Wg, int T, int d, int E, moe_dtype dt,
-                         int32_t* idx, float* w, cudaStream_t s);
+                         int32_t* idx, float* w, cudaStream_t s, int32_t* blk_counts = nullptr);
+bool dmma_route_applies(int T, int d, int E, moe_dtype dt);
+// Batches of up to kPermSmallTokens tokens are grouped in one launch; larger ones in
+// four (count, scan, rank, gather).  counts_ready: blk_counts already hold the
+// router's per-chunk counts, so the count pass is skipped (larger batches only).  The
+// scan leaves blk_counts at zero.
+constexpr int kPermSmallTokens = 512;
 cudaError_t launch_permute(const int32_t* idx, const void* x, int T, int d, int E, moe_dtype dt,
                            int32_t* offsets, int32_t* perm_token, int32_t* inv_perm,
                            void* x_perm, int32_t* blk_counts, int32_t* blk_base,
-                           uint32_t* status, cudaStream_t s);
+                           uint32_t* status, cudaStream_t s, bool counts_ready = false);
 // `cap` (all FFN launchers): rows kept per expert group -- the first `cap` rows of
 // each group are computed, the rest are neither computed nor written.
 cudaError_t launch_ffn_f32(const float* x_perm, const int32_t* offsets, const float* W1,

@@ -7,7 +7,8 @@
 //
 // The grouping is a deterministic, stable counting sort over the flattened index
 // f = t*k + j, done in four launches with no atomics that decide an order:
-//   1. count:  per block of kPermChunk tokens, how many pairs go to each expert;
+//   1. count:  per block of kPermChunk tokens, how many pairs go to each expert (in
+//              the layer, the fp64 tensor-core router counts them instead);
 //   2. scan:   one block turns the per-block counts into group offsets and the base
 //              row of every (block, expert);
 //   3. rank:   each block walks its pairs in order, 256 at a time, ranking equal
@@ -29,7 +30,7 @@ namespace {
 constexpr int kPermThreads = 256;
 constexpr int kPermWarps = kPermThreads / 32;
 constexpr uint32_t kFlagBadIndex = 0x2u;
-constexpr int kPermSmallT = 512;
+constexpr int kPermSmallT = kPermSmallTokens;
 
 // Stable ranks of the pairs [f_begin, f_end) in order, 256 at a time: pair f of
 // expert e gets row running[e] + (number of earlier pairs of e in this range);
@@ -91,8 +92,10 @@ __global__ void __launch_bounds__(kPermThreads)
 }
 
 // One block of 32 threads: thread e sums expert e's counts over blocks, thread 0
-// scans over experts, then thread e writes the base row of each (block, e).
-__global__ void perm_scan_kernel(const int32_t* __restrict__ blk_counts, int nblk, int E,
+// scans over experts, then thread e writes the base row of each (block, e) and
+// clears the counts it read, so that they are zero for a router that accumulates
+// them in the next call.
+__global__ void perm_scan_kernel(int32_t* __restrict__ blk_counts, int nblk, int E,
                                  int32_t* __restrict__ offsets, int32_t* __restrict__ blk_base) {
     pdl_wait();
     pdl_launch_dependents();
@@ -120,6 +123,7 @@ __global__ void perm_scan_kernel(const int32_t* __restrict__ blk_counts, int nbl
         for (int b = 0; b < nblk; ++b) {
             blk_base[b * E + e] = s;
             s += blk_counts[b * E + e];
+            blk_counts[b * E + e] = 0;
         }
     }
 }
@@ -222,21 +226,23 @@ __global__ void __launch_bounds__(kPermThreads)
 cudaError_t launch_permute(const int32_t* idx, const void* x, int T, int d, int E, moe_dtype dt,
                            int32_t* offsets, int32_t* perm_token, int32_t* inv_perm,
                            void* x_perm, int32_t* blk_counts, int32_t* blk_base,
-                           uint32_t* status, cudaStream_t s) {
+                           uint32_t* status, cudaStream_t s, bool counts_ready) {
     const int k = 2;
     const int vec_per_row = static_cast<int>(d * dtype_bytes(dt) / 16);
     if (T <= kPermSmallT) {
+        if (counts_ready) return cudaErrorInvalidValue;  // the one-launch form counts itself
         const int grid = T < 2 * device_sm_count() ? T : 2 * device_sm_count();
         return launch_k(perm_small_kernel, grid, kPermThreads, 0, s, idx,
                         static_cast<const uint4*>(x), T, k, E, vec_per_row, offsets, perm_token,
                         inv_perm, static_cast<uint4*>(x_perm), status);
     }
     const int nblk = perm_blocks(T);
-    cudaError_t err = launch_k(perm_count_kernel, nblk, kPermThreads, 0, s, idx, T, k, E,
-                               blk_counts, status);
+    cudaError_t err = cudaSuccess;
+    if (!counts_ready)  // otherwise the router has counted
+        err = launch_k(perm_count_kernel, nblk, kPermThreads, 0, s, idx, T, k, E, blk_counts,
+                       status);
     if (err == cudaSuccess)
-        err = launch_k(perm_scan_kernel, 1, 32, 0, s, static_cast<const int32_t*>(blk_counts),
-                       nblk, E, offsets, blk_base);
+        err = launch_k(perm_scan_kernel, 1, 32, 0, s, blk_counts, nblk, E, offsets, blk_base);
     if (err == cudaSuccess)
         err = launch_k(perm_rank_kernel, nblk, kPermThreads, 0, s, idx, T, k, E,
                        static_cast<const int32_t*>(blk_base), perm_token, inv_perm);

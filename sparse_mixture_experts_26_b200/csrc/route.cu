@@ -192,9 +192,14 @@ __device__ __forceinline__ void dmma_8x8x4(double& d0, double& d1, double a, dou
 __device__ __forceinline__ double bf16_lo(uint32_t u) { return __uint_as_float(u << 16); }
 __device__ __forceinline__ double bf16_hi(uint32_t u) { return __uint_as_float(u & 0xffff0000u); }
 
+// With `blk_counts` (zero on entry) the kernel also counts, for every kPermChunk-token
+// chunk, the pairs sent to each expert -- the first step of the grouping, so that the
+// permutation can skip its own count pass.  Integer atomics: the counts do not depend
+// on the order in which they are added.
 __global__ void __launch_bounds__(kRouteThreads)
     route_dmma_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ Wg,
-                      int T, int d, int E, int32_t* __restrict__ idx, float* __restrict__ w) {
+                      int T, int d, int E, int32_t* __restrict__ idx, float* __restrict__ w,
+                      int32_t* __restrict__ blk_counts) {
     extern __shared__ __align__(16) unsigned char route_smem[];
     __nv_bfloat16* wgT = reinterpret_cast<__nv_bfloat16*>(route_smem);  // [8][d]
     __shared__ double part[kRouteWarps][32][2];
@@ -279,6 +284,11 @@ __global__ void __launch_bounds__(kRouteThreads)
                 idx[2 * t + 1] = i2;
                 w[2 * t] = w1;
                 w[2 * t + 1] = 1.0f - w1;
+                if (blk_counts) {
+                    int32_t* c = blk_counts + static_cast<size_t>(t / kPermChunk) * E;
+                    atomicAdd(c + i1, 1);
+                    atomicAdd(c + i2, 1);
+                }
             }
         }
         __syncthreads();
@@ -290,7 +300,7 @@ __global__ void __launch_bounds__(kRouteThreads)
 // above.  Otherwise: one token per block.
 template <typename Tin, int MAXE>
 cudaError_t launch_route_t(const void* x, const void* Wg, int T, int d, int E, int32_t* idx,
-                           float* w, cudaStream_t s) {
+                           float* w, cudaStream_t s, int32_t* blk_counts) {
     const size_t wgt_bytes = static_cast<size_t>(8) * d * 2;
     if (sizeof(Tin) == 2 && MAXE == 8 && T > 64 && d % 32 == 0 && wgt_bytes <= 96 * 1024) {
         auto kern = route_dmma_kernel;
@@ -301,21 +311,28 @@ cudaError_t launch_route_t(const void* x, const void* Wg, int T, int d, int E, i
         const int cap = 3 * device_sm_count();
         return launch_k(kern, blocks_needed < cap ? blocks_needed : cap, kRouteThreads, wgt_bytes,
                         s, static_cast<const __nv_bfloat16*>(x),
-                        static_cast<const __nv_bfloat16*>(Wg), T, d, E, idx, w);
+                        static_cast<const __nv_bfloat16*>(Wg), T, d, E, idx, w, blk_counts);
     }
+    if (blk_counts) return cudaErrorInvalidValue;  // the histogram needs the kernel above
     return launch_route_tb<Tin, MAXE, 1>(x, Wg, T, d, E, idx, w, s);
 }
 
 }  // namespace
 
+bool dmma_route_applies(int T, int d, int E, moe_dtype dt) {
+    return dt == MOE_BF16 && E <= 8 && T > 64 && d % 32 == 0 &&
+           static_cast<size_t>(8) * d * 2 <= 96 * 1024;
+}
+
 cudaError_t launch_route(const void* x, const void* Wg, int T, int d, int E, moe_dtype dt,
-                         int32_t* idx, float* w, cudaStream_t s) {
+                         int32_t* idx, float* w, cudaStream_t s, int32_t* blk_counts) {
     if (dt == MOE_BF16) {
-        return E <= 8 ? launch_route_t<__nv_bfloat16, 8>(x, Wg, T, d, E, idx, w, s)
-                      : launch_route_t<__nv_bfloat16, kMaxExperts>(x, Wg, T, d, E, idx, w, s);
+        return E <= 8 ? launch_route_t<__nv_bfloat16, 8>(x, Wg, T, d, E, idx, w, s, blk_counts)
+                      : launch_route_t<__nv_bfloat16, kMaxExperts>(x, Wg, T, d, E, idx, w, s,
+                                                                   blk_counts);
     }
-    return E <= 8 ? launch_route_t<float, 8>(x, Wg, T, d, E, idx, w, s)
-                  : launch_route_t<float, kMaxExperts>(x, Wg, T, d, E, idx, w, s);
+    return E <= 8 ? launch_route_t<float, 8>(x, Wg, T, d, E, idx, w, s, blk_counts)
+                  : launch_route_t<float, kMaxExperts>(x, Wg, T, d, E, idx, w, s, blk_counts);
 }
 
 }  // namespace moe

@@ -19,12 +19,15 @@ def _kernel_names(fn):
             if e.device_type == torch.autograd.DeviceType.CUDA]
 
 
-@pytest.mark.parametrize("T", [16, 100, 300, 700, 1100])
-def test_layer_launch_count(T):
-    wl = small("lc", T=T, d=256, h=384, seed=T)
+@pytest.mark.parametrize("T,d,E", [(16, 256, 8), (100, 256, 8), (300, 256, 8), (700, 256, 8),
+                                   (1100, 256, 8), (1100, 136, 8), (700, 256, 16)])
+def test_layer_launch_count(T, d, E):
+    """Above 512 tokens the router counts the grouping (no count pass) where the fp64
+    tensor-core router applies (E <= 8, d a multiple of 32)."""
+    wl = small("lc", T=T, d=d, h=384, E=E, seed=T)
     inp = make_inputs(wl, "cuda")
     x = inp["x"]
-    ws = moe.alloc_workspace(T, 256, 384, wl.E, 2, x.dtype, x.device)
+    ws = moe.alloc_workspace(T, d, 384, wl.E, 2, x.dtype, x.device)
     y = torch.empty_like(x)
 
     def call():
@@ -37,7 +40,7 @@ def test_layer_launch_count(T):
         pytest.skip("the CUDA profiler records no kernels on this system")
     names = _kernel_names(call)
     ours = [n for n in names if "moe::" in n]
-    assert len(ours) == moe.launches_per_layer(T), ours
+    assert len(ours) == moe.launches_per_layer(T, d, E), ours
     assert len(ours) == len(names), names  # nothing but libmoe kernels
 
 
