@@ -111,6 +111,7 @@ struct PairArgs {
     int cap;      // rows kept per group (capacity; INT_MAX = no limit)
     int h;             // kBMnSplit: the K index where W3 takes over from W1
     const float* dH;   // kEpiBwdSwiGLU: dH fp32 [rows, N]
+    int group;         // row blocks whose A rows stay in L2 together (tile order)
 };
 
 struct PairBook {
@@ -132,15 +133,35 @@ struct PairTile {
     bool half;
 };
 
-__device__ __forceinline__ PairTile decode_pair_tile(const PairBook& bk, int E, int tile) {
+// Tile order inside an expert: row blocks in groups of `group` (the last group may be
+// smaller); a group's tiles run column tile by column tile with its row blocks
+// innermost.  Concurrent pairs then share each weight tile (read from DRAM once) and
+// a group's A rows (sized on the host to fit L2 with room to spare) are read from DRAM
+// once for all column tiles; an expert with at most `group` row blocks runs in plain
+// column-major order.
+__device__ __forceinline__ PairTile decode_pair_tile(const PairBook& bk, int E, int tile,
+                                                    int n_tiles, int group) {
     int g = 0;
     while (g + 1 < E && tile >= bk.tile_start[g + 1]) ++g;
     const int local = tile - bk.tile_start[g];
     const int blocks = (bk.end[g] - bk.off[g] + kPairRows - 1) / kPairRows;
+    const int full = blocks / group;                // complete row-block groups
+    const int per_full = group * n_tiles;
+    int rb, nt;
+    if (local < full * per_full) {
+        const int r = local % per_full;
+        rb = (local / per_full) * group + r % group;
+        nt = r / group;
+    } else {
+        const int rem = blocks - full * group;      // > 0 here
+        const int r = local - full * per_full;
+        rb = full * group + r % rem;
+        nt = r / rem;
+    }
     PairTile t;
     t.e = g;
-    t.row0 = bk.off[g] + (local % blocks) * kPairRows;
-    t.nt = local / blocks;
+    t.row0 = bk.off[g] + rb * kPairRows;
+    t.nt = nt;
     t.row_end = bk.end[g];
     t.half = t.row_end - t.row0 <= kRowsPerCta;
     return t;
@@ -243,7 +264,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             constexpr bool kStacked = EPI == kEpiBwdSwiGLU;
             const CUtensorMap* tmB = (kStacked && !leader) ? &tmB1 : &tmB0;
             for (int tile = pair; ok && tile < total; tile += npairs) {
-                const PairTile t = decode_pair_tile(bk, E, tile);
+                const PairTile t = decode_pair_tile(bk, E, tile, args.n_tiles, args.group);
                 const int a_row = t.row0 + static_cast<int>(rank) * (t.half ? 64 : kRowsPerCta);
                 const int b_row =
                     EPI == kEpiSwiGLU
@@ -308,7 +329,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t phase = 0, acc_phase = 0;
             bool ok = true, issued = false;
             for (int tile = pair; ok && tile < total; tile += npairs) {
-                const PairTile t = decode_pair_tile(bk, E, tile);
+                const PairTile t = decode_pair_tile(bk, E, tile, args.n_tiles, args.group);
                 constexpr uint32_t kBT = BOP == kBKMajor ? 0u : (1u << 16);  // B MN-major
                 const uint32_t idesc = (t.half ? kIdescHalf : kIdescFull) | kBT;
                 if (!mbar_wait_bounded(&bk.tmem_empty[acc], acc_phase ^ 1u, abort_flag,
@@ -359,7 +380,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int tile = pair; tile < total; tile += npairs) {
-            const PairTile t = decode_pair_tile(bk, E, tile);
+            const PairTile t = decode_pair_tile(bk, E, tile, args.n_tiles, args.group);
             if (!bar_all(mbar_wait_bounded(&bk.tmem_full[acc], acc_phase, abort_flag, args.status),
                          kVoteBarrier, kEpiThreads))
                 break;
@@ -600,6 +621,11 @@ cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b0, const CUten
                         const CUtensorMap& o, const PairArgs& args, int npairs, cudaStream_t s) {
     auto kern = grouped_gemm_pair_kernel<EPI, BOP>;
     constexpr int kSmemBytes = smem_bytes_of(EPI);
+    // Row blocks per tile-order group: A rows of at most ~64 MB (a half of L2) per group.
+    PairArgs a2 = args;
+    const long long a_block_bytes = static_cast<long long>(kPairRows) * args.K * 2;
+    const long long g = (64LL << 20) / (a_block_bytes > 0 ? a_block_bytes : 1);
+    a2.group = static_cast<int>(g < 1 ? 1 : (g > 1024 ? 1024 : g));
     static PerDeviceOnce smem_once;
     if (const cudaError_t err = opt_in_smem(smem_once, kern, kSmemBytes); err != cudaSuccess)
         return err;
@@ -615,7 +641,7 @@ cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b0, const CUten
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t err = cudaLaunchKernelEx(&cfg, kern, a, b0, b1, o, args);
+    cudaError_t err = cudaLaunchKernelEx(&cfg, kern, a, b0, b1, o, a2);
     return err != cudaSuccess ? err : cudaGetLastError();
 }
 
