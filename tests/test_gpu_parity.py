@@ -294,7 +294,9 @@ def test_out_of_range_expert_ids_are_flagged(T):
 
 
 @pytest.mark.parametrize("E", [2, 4, 16, 32])
-@pytest.mark.parametrize("T", [40, 300])  # weight-streaming and grouped kernels
+@pytest.mark.parametrize("T", [40, 300, 700])  # weight-streaming, grouped and pair kernels;
+                                                # above 512 tokens the router counts the
+                                                # grouping for E <= 8
 def test_other_expert_counts(E, T):
     """The layer for E other than 8 (the ABI allows 2..32): routing and permutation
     bit-exact, output within the bf16 tolerance."""
