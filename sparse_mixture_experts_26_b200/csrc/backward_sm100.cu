@@ -336,7 +336,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             for (int u = 0; u < 2; ++u) {
                                 const float av = bits_f32(a[2 * i + u]);
                                 const float bv = bits_f32(b[2 * i + u]);
-                                const float s = 1.0f / (1.0f + __expf(-av));
+                                const float s = __frcp_rn(1.0f + __expf(-av));
                                 ru[u] = gv[2 * i + u] * bv * (s * (1.0f + av * (1.0f - s)));
                                 rv[u] = gv[2 * i + u] * (av * s);
                             }

@@ -340,7 +340,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 const float a = xfer[c * kM + r];
                                 const float b = xfer[c * kM + J + r];
                                 out[static_cast<size_t>(t.row0 + c) * args.N + col] =
-                                    __float2bfloat16_rn(a / (1.0f + __expf(-a)) * b);
+                                    __float2bfloat16_rn(a * b * __frcp_rn(1.0f + __expf(-a)));
                             }
                         }
                     }
@@ -686,7 +686,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                     const float a = xfer[c * kM + r];
                                     const float b = xfer[c * kM + J1 + r];
                                     out[static_cast<size_t>(f.row0 + c) * args.h + col] =
-                                        __float2bfloat16_rn(a / (1.0f + __expf(-a)) * b);
+                                        __float2bfloat16_rn(a * b * __frcp_rn(1.0f + __expf(-a)));
                                 }
                             }
                         }
@@ -731,7 +731,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                         const float a = xfer[c * kM + r];
                                         const float b = xfer[c * kM + J1 + r];
                                         out[static_cast<size_t>(f.row0 + c0 + c) * args.h + col] =
-                                            __float2bfloat16_rn(a / (1.0f + __expf(-a)) * b);
+                                            __float2bfloat16_rn(a * b * __frcp_rn(1.0f + __expf(-a)));
                                     }
                                 }
                             }

@@ -167,13 +167,16 @@ __device__ __forceinline__ PairTile decode_pair_tile(const PairBook& bk, int E, 
     return t;
 }
 
+// silu(a) * b = a b / (1 + e^-a), with a correctly rounded reciprocal instead of a
+// division: the division's slow path (one warp per scheduler, no latency hiding) made
+// the epilogue, not the tensor cores, set GEMM1's pace at full clock.
 __device__ __forceinline__ float silu_mul(float a, float b) {
-    return a / (1.0f + __expf(-a)) * b;
+    return a * b * __frcp_rn(1.0f + __expf(-a));
 }
 
 // du = g b silu'(a), dv = g silu(a) for one output of the backward SwiGLU step.
 __device__ __forceinline__ void bwd_swiglu(float a, float b, float g, float& du, float& dv) {
-    const float s = 1.0f / (1.0f + __expf(-a));
+    const float s = __frcp_rn(1.0f + __expf(-a));
     du = g * b * (s * (1.0f + a * (1.0f - s)));
     dv = g * (a * s);
 }

@@ -119,8 +119,10 @@ __device__ __forceinline__ TileCoord decode_tile(const Bookkeeping& bk, int E, i
     return c;
 }
 
+// silu(a) * b = a b / (1 + e^-a), with a correctly rounded reciprocal (cheaper than a
+// division in the epilogue).
 __device__ __forceinline__ float silu_mul(float a, float b) {
-    return a / (1.0f + __expf(-a)) * b;
+    return a * b * __frcp_rn(1.0f + __expf(-a));
 }
 
 template <int EPI, int NO>

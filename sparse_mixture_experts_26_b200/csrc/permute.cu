@@ -117,7 +117,8 @@ __global__ void perm_scan_kernel(int32_t* __restrict__ blk_counts, int nblk, int
         off[E] = s;
     }
     __syncthreads();
-    if (e <= E) offsets[e] = off[e];
+    if (e < E) offsets[e] = off[e];
+    if (e == 0) offsets[E] = off[E];  // E may be 32: no thread E in a block of 32
     if (e < E) {
         int s = off[e];
         for (int b = 0; b < nblk; ++b) {
