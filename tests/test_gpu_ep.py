@@ -34,7 +34,7 @@ def test_single_rank_expert_parallel_equals_the_layer(T, kind):
     assert torch.equal(y_ep, y)
 
 
-@pytest.mark.parametrize("rows", [7, 40, 301])
+@pytest.mark.parametrize("rows", [7, 40, 301, 1501])  # small-batch, single-SM, pair paths
 def test_expert_ffn_single_expert_with_padding_row(rows):
     """One expert, an odd number of grouped rows padded to an even count (the padding
     row belongs to no group; its output row is unspecified)."""
