@@ -10,7 +10,7 @@
 // and one thread of the leader issues tcgen05.mma.cta_group::2 (M = 256 from the two
 // A halves, N = 256 from the two B halves); each CTA's TMEM receives its 128 rows.
 // Per SM a stage is 32 KiB instead of 48 KiB for the same math, which leaves room for
-// 6 stages next to the output staging buffers.
+// 7 stages.
 //
 // A reduction starts and ends at arbitrary rows, so the rows of an expert's last,
 // partial K block that belong to the next expert must be zero before the MMA reads
@@ -22,9 +22,15 @@
 // the leader's, once both are done, arrives on "full".  (A handshake on every block
 // instead measured 2-4x slower: a cluster-scope arrive per block serialises the
 // pipeline.)  The leader's MMA completions are multicast to both CTAs' "empty" and
-// "tmem_full" barriers; both epilogues arrive on the leader's "tmem_empty".  The
-// epilogue writes with per-warp TMA tensor stores, as the single-SM kernel does.
-// Every wait is bounded.
+// "tmem_full" barriers; both epilogues arrive on the leader's "tmem_empty".
+//
+// The epilogue stores straight from registers: each warp reads its TMEM lanes in the
+// 16x256b shape, where four consecutive threads hold eight consecutive columns of a
+// row, so every store instruction writes whole 32-byte sectors.  (Staging 32 x 32
+// chunks in shared memory for TMA tensor stores, as the single-SM kernel does, was
+// slower here -- the stores queued behind the operand loads on the TMA path: dW1+dW3
+// 1.66 -> 1.62 ms with real data, 1.43 -> 1.25 ms at full clock -- and its 32 KiB of
+// staging now holds a 7th input stage.)  Every wait is bounded.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -33,17 +39,12 @@
 
 namespace moe {
 
-bool encode_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
-                    uint32_t box_rows);
-bool encode_f32_3d(CUtensorMap* map, const void* base, uint64_t batches, uint64_t rows,
-                   uint64_t cols, uint32_t box_cols, uint32_t box_rows);
-
 namespace {
 
 constexpr int kRows = 128;                  // output rows per CTA (TMEM lanes)
 constexpr int kBK = 64;                     // K rows per stage
 constexpr int kN = 256;                     // output columns per tile
-constexpr int kStages = 6;
+constexpr int kStages = 7;
 constexpr int kBox = kMnBoxBytes;           // one 64-column x 64-row bf16 box: 8 KiB
 constexpr int kABytes = 2 * kBox;           // this CTA's 128 columns of A
 constexpr int kBBytes = 2 * kBox;           // this CTA's 128 columns of B
@@ -51,10 +52,7 @@ constexpr int kStageBytes = kABytes + kBBytes;
 constexpr int kThreads = 224;  // TMA, MMA, 4 epilogue warps, fix-up warp
 constexpr int kEpiThreads = 128;
 constexpr uint32_t kTmemCols = 2 * kN;
-constexpr int kOutBufs = 2;                 // staging buffers per epilogue warp
-constexpr int kStageOutBytes = 32 * 32 * 4; // one 32 x 32 fp32 chunk
-constexpr int kSmemBytes = kStages * kStageBytes + 4 * kOutBufs * kStageOutBytes +
-                           1024 /*align*/ + 1024 /*book*/;
+constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 1024 /*book*/;
 static_assert(kSmemBytes <= 232448, "shared memory");
 constexpr int kVoteBarrier = 2;
 constexpr uint16_t kBothCtas = 0x3;
@@ -85,7 +83,7 @@ struct PArgs {
     int N;
     int m_pairs;     // ceil(M / 256)
     int n_tiles;     // ceil(N / 256)
-    int split;       // output rows m < split go to out0 (tmO0), the rest to out1 (tmO1)
+    int split;       // output rows m < split go to out0, the rest to out1
     float* out0;
     float* out1;
     uint32_t* status;
@@ -126,16 +124,13 @@ __device__ __forceinline__ bool wait_cluster_bounded(uint64_t* bar, uint32_t par
 
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_wgrad_pair_kernel(const __grid_constant__ CUtensorMap tmA,
-                          const __grid_constant__ CUtensorMap tmB,
-                          const __grid_constant__ CUtensorMap tmO0,
-                          const __grid_constant__ CUtensorMap tmO1, const PArgs args) {
+                          const __grid_constant__ CUtensorMap tmB, const PArgs args) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     uint8_t* sA = smem;
     uint8_t* sB = smem + kStages * kABytes;
-    uint8_t* sOut = smem + kStages * kStageBytes;
-    Book& bk = *reinterpret_cast<Book*>(sOut + 4 * kOutBufs * kStageOutBytes);
+    Book& bk = *reinterpret_cast<Book*>(smem + kStages * kStageBytes);
     volatile int* abort_flag = &bk.abort_flag;
 
     const int warp = threadIdx.x >> 5;
@@ -164,8 +159,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
-        tma_prefetch_desc(&tmO0);
-        tma_prefetch_desc(&tmO1);
     }
     if (warp == 1) tmem_alloc_pair(&bk.tmem_base, kTmemCols);
     if (threadIdx.x == 0) {
@@ -373,24 +366,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int q = warp & 3;  // warps 2..5: TMEM lane quarters 2, 3, 0, 1
         const uint32_t empty_leader0 = map_to_cta(smem_u32(&bk.tmem_empty[0]), 0);
         const uint32_t empty_leader1 = map_to_cta(smem_u32(&bk.tmem_empty[1]), 0);
-        uint8_t* wstage = sOut + q * kOutBufs * kStageOutBytes;
-        int acc = 0, buf = 0;
+        const int c2 = 2 * (lane & 3), r4 = lane >> 2;  // this thread's columns / rows
+        int acc = 0;
         uint32_t acc_phase = 0;
+        // output row m of the tile: dW2 rows, or dW1 rows (m < split) then dW3 rows
+        auto out_row = [&](int e, int m) -> float* {
+            return m < args.split
+                       ? args.out0 + (static_cast<size_t>(e) * args.split + m) * args.N
+                       : args.out1 + (static_cast<size_t>(e) * (args.M - args.split) +
+                                      (m - args.split)) * args.N;
+        };
         for (int tile = pair; tile < total; tile += npairs) {
             int e, mp, nt, r0, n_rows;
             tile_of(tile, e, mp, nt, r0, n_rows);
             const int m0 = mp * 2 * kRows + static_cast<int>(rank) * kRows;  // this CTA's rows
-            const int m = m0 + q * 32 + lane;
-            const bool mvalid = m < args.M;
-            float* out = m < args.split
-                             ? args.out0 + (static_cast<size_t>(e) * args.split + m) * args.N
-                             : args.out1 + (static_cast<size_t>(e) * (args.M - args.split) +
-                                            (m - args.split)) * args.N;
             const int col0 = nt * kN;
             if (n_rows == 0) {
-                if (mvalid)
+                const int m = m0 + q * 32 + lane;
+                if (m < args.M) {
+                    float* out = out_row(e, m);
                     for (int col = col0; col < col0 + kN && col < args.N; col += 4)
                         *reinterpret_cast<float4*>(out + col) = make_float4(0.f, 0.f, 0.f, 0.f);
+                }
                 continue;
             }
             if (!bar_all(mbar_wait_bounded(&bk.tmem_full[acc], acc_phase, abort_flag,
@@ -400,41 +397,29 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
             const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                                    static_cast<uint32_t>(acc * kN);
-            // A slice that starts at or past M (the peer's half of a last, partial pair
-            // tile) stores nothing: for dW2 the second output map is the first one again.
-            const bool slice_valid = m0 < args.M;
-            const bool second = m0 >= args.split;
-            const bool straddle = m0 < args.split && m0 + kRows > args.split;
+            // rows past M (the peer's half of a last, partial pair tile) store nothing
+            if (m0 + q * 32 < args.M) {
 #pragma unroll 1
-            for (int ch = 0; ch < 8; ++ch) {
-                uint32_t v[32];
-                tmem_ld_32cols(tbase + ch * 32, v);
-                tmem_ld_wait();
-                if (!slice_valid) continue;
-                if (!straddle) {
-                    uint8_t* st = wstage + buf * kStageOutBytes;
-                    if (lane == 0) bulk_wait_group_read<kOutBufs - 1>();
-                    __syncwarp();
+                for (int hf = 0; hf < 2; ++hf) {  // lanes 0..15 and 16..31 of this quarter
+#pragma unroll 1
+                    for (int cb = 0; cb < kN / 64; ++cb) {
+                        uint32_t v[32];
+                        tmem_ld_16x256b_x8(tbase + (static_cast<uint32_t>(hf * 16) << 16) + cb * 64, v);
+                        tmem_ld_wait();
 #pragma unroll
-                    for (int j = 0; j < 8; ++j)
-                        *reinterpret_cast<uint4*>(st + lane * 128 + ((j ^ (lane & 7)) << 4)) =
-                            make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) {
-                        tma_store_3d(second ? &tmO1 : &tmO0, st, col0 + ch * 32,
-                                     (second ? m0 - args.split : m0) + q * 32, e);
-                        bulk_commit_group();
-                    }
-                    if (++buf == kOutBufs) buf = 0;
-                } else if (mvalid) {
+                        for (int w = 0; w < 2; ++w) {
+                            const int m = m0 + q * 32 + hf * 16 + r4 + 8 * w;
+                            if (m >= args.M) continue;
+                            float* out = out_row(e, m);
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        const int col = col0 + ch * 32 + j * 4;
-                        if (col < args.N)
-                            *reinterpret_cast<float4*>(out + col) =
-                                make_float4(bits_f32(v[4 * j]), bits_f32(v[4 * j + 1]),
-                                            bits_f32(v[4 * j + 2]), bits_f32(v[4 * j + 3]));
+                            for (int rep = 0; rep < 8; ++rep) {
+                                const int col = col0 + cb * 64 + rep * 8 + c2;
+                                if (col < args.N)  // N is a multiple of 8: col + 1 < N too
+                                    *reinterpret_cast<float2*>(out + col) =
+                                        make_float2(bits_f32(v[4 * rep + 2 * w]),
+                                                    bits_f32(v[4 * rep + 2 * w + 1]));
+                            }
+                        }
                     }
                 }
             }
@@ -443,7 +428,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             acc ^= 1;
             if (acc == 0) acc_phase ^= 1u;
         }
-        if (lane == 0) bulk_wait_group<0>();  // every store complete before the block exits
     }
 
     tc_fence_before();
@@ -458,9 +442,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 }  // namespace
 
 // Weight gradients on CTA pairs: A [rows, M] and B [rows, N] grouped bf16 operands
-// (tensor maps with 64 x 64 boxes), outputs through 3-D fp32 maps with 32 x 32 boxes.
-cudaError_t launch_wgrad_pair(const CUtensorMap& A, const CUtensorMap& B, const CUtensorMap& O0,
-                              const CUtensorMap& O1, const int32_t* offsets, int E, int rows,
+// (tensor maps with 64 x 64 boxes); fp32 outputs out0 [E, split, N] and out1
+// [E, M - split, N].
+cudaError_t launch_wgrad_pair(const CUtensorMap& A, const CUtensorMap& B, const int32_t* offsets,
+                              int E, int rows,
                               int M, int N, int split, float* out0, float* out1, uint32_t* status,
                               int cap, cudaStream_t s, int pad_a, int pad_b) {
     static PerDeviceOnce smem_once;
@@ -484,7 +469,7 @@ cudaError_t launch_wgrad_pair(const CUtensorMap& A, const CUtensorMap& B, const 
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t err = cudaLaunchKernelEx(&cfg, bwd_wgrad_pair_kernel, A, B, O0, O1, p);
+    cudaError_t err = cudaLaunchKernelEx(&cfg, bwd_wgrad_pair_kernel, A, B, p);
     return err != cudaSuccess ? err : cudaGetLastError();
 }
 

@@ -49,8 +49,8 @@ cudaError_t launch_bwd_rows_pair(int mode, const CUtensorMap& a, const CUtensorM
                                  int d, int h, void* out, const float* dH, uint32_t* status,
                                  int cap, cudaStream_t s);
 // Defined in backward_pair_sm100.cu.
-cudaError_t launch_wgrad_pair(const CUtensorMap& A, const CUtensorMap& B, const CUtensorMap& O0,
-                              const CUtensorMap& O1, const int32_t* offsets, int E, int rows,
+cudaError_t launch_wgrad_pair(const CUtensorMap& A, const CUtensorMap& B, const int32_t* offsets,
+                              int E, int rows,
                               int M, int N, int split, float* out0, float* out1, uint32_t* status,
                               int cap, cudaStream_t s, int pad_a = 0, int pad_b = 0);
 
@@ -1116,10 +1116,10 @@ cudaError_t launch_layer_backward(const BwdArgs& a, cudaStream_t s) {
             if (err != cudaSuccess) return err;
         }
         // A device that cannot co-schedule a CTA pair takes the single-SM kernel.
-        err = padded ? launch_wgrad_pair(m_dYp64, m_H64, m_dW2, m_dW2, a.offsets, E, P, d, h, d,
-                                         a.dW2, a.dW2, a.status, a.cap, s, 1, 0)
-                     : launch_wgrad_pair(m_dY64, m_H64, m_dW2, m_dW2, a.offsets, E, P, d, h, d,
-                                         a.dW2, a.dW2, a.status, a.cap, s);
+        err = padded ? launch_wgrad_pair(m_dYp64, m_H64, a.offsets, E, P, d, h, d, a.dW2, a.dW2,
+                                         a.status, a.cap, s, 1, 0)
+                     : launch_wgrad_pair(m_dY64, m_H64, a.offsets, E, P, d, h, d, a.dW2, a.dW2,
+                                         a.status, a.cap, s);
         if (err != cudaSuccess) {
             cudaGetLastError();
             WArgs w{a.offsets, E, P, d, h, (d + kBM - 1) / kBM, (h + kN - 1) / kN, d, a.dW2,
@@ -1128,10 +1128,10 @@ cudaError_t launch_layer_backward(const BwdArgs& a, cudaStream_t s) {
                                         s, m_dY64, m_H64, m_dW2, m_dW2, w);
         }
         if (err != cudaSuccess || (err = mark(6)) != cudaSuccess) return err;
-        err = padded ? launch_wgrad_pair(m_duv64, m_xp64, m_dW1, m_dW3, a.offsets, E, P, 2 * h,
-                                         d, h, a.dW1, a.dW3, a.status, a.cap, s, 0, 1)
-                     : launch_wgrad_pair(m_duv64, m_x64, m_dW1, m_dW3, a.offsets, E, P, 2 * h,
-                                         d, h, a.dW1, a.dW3, a.status, a.cap, s);
+        err = padded ? launch_wgrad_pair(m_duv64, m_xp64, a.offsets, E, P, 2 * h, d, h, a.dW1,
+                                         a.dW3, a.status, a.cap, s, 0, 1)
+                     : launch_wgrad_pair(m_duv64, m_x64, a.offsets, E, P, 2 * h, d, h, a.dW1,
+                                         a.dW3, a.status, a.cap, s);
         if (err != cudaSuccess) {
             cudaGetLastError();
             WArgs w{a.offsets, E, P, 2 * h, d, (2 * h + kBM - 1) / kBM, (d + kN - 1) / kN, h,
