@@ -110,6 +110,9 @@ SMALL = [  # (T, d, h, kind): ragged row blocks, K tails, N tails, empty groups
     # 112 selects its 112-output GEMM1 tiles
     (129, 256, 512, "plain"), (300, 136, 200, "plain"), (511, 128, 256, "skew"),
     (200, 128, 224, "plain"), (300, 256, 448, "skew"), (450, 136, 336, "long"),
+    # ... with stream-K work split (>= one (tile, K block) unit per SM): tiles cut
+    # between CTAs and finished from fp32 partials; ragged K (1000 = 15 x 64 + 40)
+    (300, 1000, 1792, "plain"), (400, 1024, 2048, "skew"), (160, 512, 3584, "long"),
     # >= 1024 grouped rows run the CTA-pair grouped GEMM (256-row blocks; an expert's
     # last block of <= 128 rows runs in the pair's 128-row mode)
     (512, 128, 256, "plain"), (513, 128, 256, "long"), (700, 256, 384, "skew"),
@@ -236,13 +239,17 @@ def test_exact_invariants_on_gpu(T):
     assert torch.equal(layer_y(s), y)
 
 
-@pytest.mark.parametrize("name", ["decode", "prefill", "skew", "long"])
-def test_full_size_workloads(name):
+@pytest.mark.parametrize("name,T", [("decode", None), ("prefill", None), ("skew", None),
+                                    ("long", None),
+                                    # batches between the two: stream-K grouped GEMMs
+                                    ("prefill", 192), ("prefill", 511), ("skew", 256),
+                                    ("skew", 384)])
+def test_full_size_workloads(name, T):
     """The Mixtral-8x7B-shaped workloads at full size: routing and permutation over all
     tokens, gathered rows byte-exact, and y against the fp64 oracle over every token
     (relative Frobenius error of the whole output, and every token's own error).  A
     sample of tokens is checked first, so a gross error fails in seconds."""
-    wl = WORKLOADS[name]
+    wl = WORKLOADS[name] if T is None else WORKLOADS[name].with_tokens(T)
     inp = make_inputs(wl, "cuda")
     g = run_steps(inp, wl.E)
     x_cpu = inp["x"].float().cpu().numpy()
