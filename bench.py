@@ -271,16 +271,16 @@ def algorithmic_flops_gemm1(wl) -> int:
 
 # ------------------------------------------------------------------ our arm
 def rank_inputs(wl, rank: int, world: int, device):
-    """The workload's tensors on ``device``; every rank past 0 draws its own batch x
-    (same recipe) while the weights stay the same on every rank."""
-    import torch
+    """The workload's tensors on ``device``; every rank past 0 draws its own batch x by
+    the same recipe (skewed or long-context rows included) from its own seed, while the
+    weights stay the same on every rank."""
+    from dataclasses import replace
 
     from workloads import make_inputs
     inp = make_inputs(wl, device)
     if world > 1 and rank > 0:
-        g = torch.Generator(device=device)
-        g.manual_seed(wl.seed * 1000 + rank)
-        inp["x"] = torch.randn(inp["x"].shape, generator=g, device=device).to(inp["x"].dtype)
+        own = replace(wl, seed=wl.seed * 1000 + rank)
+        inp["x"] = make_inputs(own, device, weights=False)["x"]
     return inp
 
 
@@ -438,6 +438,54 @@ def measure_forward(wl, inp, K: int, W: int, world: int, local: int, device):
             "gpu_launches": launches * K, "clocks": clocks.summary()}
 
 
+# Batches between the two measured serving regimes (the grouped-GEMM range, 129..511
+# tokens), with plain and skewed routing: the layer alone, no events inside the timed
+# region, against the copy bandwidth (the layer reads each touched expert's weights once).
+SWEEP_TOKENS = (192, 256, 384)
+SWEEP_ROUTINGS = ("prefill", "skew")
+
+
+def measure_layer_only(wl, inp, K: int, W: int, world: int, local: int, device):
+    import torch
+
+    import sparse_mixture_experts_26_b200 as moe
+
+    x, Wg, W1, W3, W2 = (inp[k] for k in ("x", "Wg", "W1", "W3", "W2"))
+    T, d, h, E = wl.T, wl.d, wl.h, wl.E
+    ws = moe.alloc_workspace(T, d, h, E, wl.k, x.dtype, device)
+    y = torch.empty_like(x)
+    stream = torch.cuda.current_stream(device)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clocks:
+        for _ in range(W):
+            moe.moe_layer_forward(x, Wg, W1, W3, W2, y, ws)
+        torch.cuda.synchronize()
+        barrier(world, device)
+        start.record(stream)
+        for _ in range(K):
+            moe.moe_layer_forward(x, Wg, W1, W3, W2, y, ws)
+        end.record(stream)
+        torch.cuda.synchronize()
+        barrier(world, device)
+    if moe.moe_device_status(ws):
+        raise RuntimeError("device status flags set after the timed region")
+    ms = max_over_ranks(start.elapsed_time(end) / K, world, device)
+    idx = torch.empty(T, 2, dtype=torch.int32, device=device)
+    wts = torch.empty(T, 2, dtype=torch.float32, device=device)
+    moe.moe_route(x, Wg, idx, wts)
+    counts = torch.bincount(idx.flatten().long(), minlength=E).cpu().numpy()
+    touched = int((counts > 0).sum())
+    layer_bytes = touched * 3 * h * d * 2 + T * d * 2 * 2
+    peaks, peak_src = load_peaks()
+    gbs = layer_bytes / (ms * 1e-3) / 1e9
+    return {"T": T, "routing": "skewed" if wl.kind == "skew" else "plain",
+            "ms": round(ms, 4), "tokens_per_s": round(world * T / (ms * 1e-3), 1),
+            "experts_touched": touched, "rows_per_expert": [int(c) for c in counts],
+            "layer_bytes": int(layer_bytes), "hbm_gbs": round(gbs, 1),
+            "frac_of_copy": round(gbs / float(peaks["hbm_gbs"]), 4),
+            "peak_source": f"{peak_src} (copy)", "clocks": clocks.summary()}
+
+
 def forward_cpu_baseline(inp, wl, args):
     n = min(wl.T, args.cpu_sample_tokens)
     tps, threads, reps, dt = oracle_tokens_per_s(cpu_copy(inp), n, args.cpu_budget_s)
@@ -493,6 +541,19 @@ def run_ours(args):
             sub[other] = measure_forward(owl, oinp, k, W, world, local, device)
             del oinp
             free_device_memory()
+        sweep = []
+        for T in SWEEP_TOKENS:
+            for routing in SWEEP_ROUTINGS:
+                owl = WORKLOADS[routing].with_tokens(T)
+                oinp = rank_inputs(owl, rank, world, device)
+                sweep.append(measure_layer_only(owl, oinp, K, W, world, local, device))
+                del oinp
+                free_device_memory()
+        sub["batch_sweep"] = {
+            "what": "layer time at batches between the small-batch and CTA-pair kernels "
+                    "(grouped GEMMs), no events inside the timed region; bytes = touched "
+                    "experts' weights + x + y",
+            "steps": K, "warmup": W, "points": sweep}
         for other in SUITE_BACKWARD:
             owl = WORKLOADS[other]
             oinp = rank_inputs(owl, rank, world, device)
