@@ -425,6 +425,8 @@ struct FusedBook {
     int end[kMaxExperts];         // end of the rows kept in group g (capacity)
     int start1[kMaxExperts + 1];  // gate/up tiles before expert g
     int start2[kMaxExperts + 1];  // down units before expert g
+    int ntr;                      // token rows per tile in this launch (<= NT)
+    int stages;                   // stages the ring holds at that tile size
 };
 
 struct FusedUnit {
@@ -444,8 +446,11 @@ __device__ __forceinline__ FusedUnit fused_unit(const FusedBook<NACC>& bk, const
         local = u - bk.start1[g];
         f.down = false;
         f.ks = 0;
-        const int chunk = local / a.n_hb;
-        f.blk = local - chunk * a.n_hb;
+        f.chunks = (bk.end[g] - bk.off[g] + NTc - 1) / NTc;
+        // token chunks innermost: the chunks of one weight block run on neighbouring
+        // CTAs at the same time, so the weights cross HBM once
+        f.blk = local / f.chunks;
+        const int chunk = local - f.blk * f.chunks;
         f.row0 = bk.off[g] + chunk * NTc;
         f.kb0 = 0;
         f.kb1 = num_kb1;
@@ -454,38 +459,55 @@ __device__ __forceinline__ FusedUnit fused_unit(const FusedBook<NACC>& bk, const
         while (g + 1 < a.E && v >= bk.start2[g + 1]) ++g;
         local = v - bk.start2[g];
         f.down = true;
+        f.chunks = (bk.end[g] - bk.off[g] + NTc - 1) / NTc;
+        const int chunk = local % f.chunks;
+        local /= f.chunks;
         f.ks = local % a.ksplit;
-        local /= a.ksplit;
-        const int chunk = local / a.n_db;
-        f.blk = local - chunk * a.n_db;
+        f.blk = local / a.ksplit;
         f.row0 = bk.off[g] + chunk * NTc;
         f.kb0 = f.ks * kps;
         f.kb1 = min(num_kb2, f.kb0 + kps);
     }
     f.e = g;
-    f.chunks = (bk.end[g] - bk.off[g] + NTc - 1) / NTc;
     const int left = bk.end[g] - f.row0;
     f.nvalid = left < NTc ? left : NTc;
     return f;
+}
+
+// Token operands of the fused launch, each as tensor maps whose boxes hold 16, 32, 64
+// and 128 rows (at most NT).  The launch reads the group sizes first and takes the
+// smallest token tile that holds its largest group (every group is then one chunk);
+// the stage ring is cut into as many stages as fit at that tile size (128 rows: 6,
+// 64: 8, 32: 10, 16: 12 of the same ~200 KiB), so a batch whose groups are small keeps
+// more weight bytes in flight per SM, which is what sets the streaming rate here.
+struct TokMaps {
+    CUtensorMap m[4];
+};
+constexpr int kTokBoxes = 4;
+__host__ __device__ constexpr int tok_box_rows(int i, int NT) {
+    return (16 << i) < NT ? (16 << i) : NT;
+}
+__device__ __forceinline__ int tok_box_index(int n) {
+    return n <= 16 ? 0 : n <= 32 ? 1 : n <= 64 ? 2 : 3;
 }
 
 template <int NT>
 __global__ void __launch_bounds__(kThreads, 1)
     decode_ffn_fused_kernel(const __grid_constant__ CUtensorMap tmW1,
                             const __grid_constant__ CUtensorMap tmW3,
-                            const __grid_constant__ CUtensorMap tmX,
+                            const __grid_constant__ TokMaps tmX,
                             const __grid_constant__ CUtensorMap tmW2,
-                            const __grid_constant__ CUtensorMap tmH, const FusedArgs args) {
-    using C = DecodeCfg<kSwiGLU, NT>;  // same stage layout for both GEMMs
+                            const __grid_constant__ TokMaps tmH, const FusedArgs args) {
+    using C = DecodeCfg<kSwiGLU, NT>;  // the ring's size and the accumulators
     constexpr int NACC = C::kAcc;
     constexpr int J1 = kM / 2;         // 64 output columns of H per gate/up tile
+    constexpr int kRingBytes = C::kStages * (C::kAStage + C::kBStage);
     using Book = FusedBook<NACC>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     uint8_t* sA = smem;
-    uint8_t* sB = smem + C::kStages * C::kAStage;
-    Book& bk = *reinterpret_cast<Book*>(sB + C::kStages * C::kBStage);
+    Book& bk = *reinterpret_cast<Book*>(smem + kRingBytes);
     float* xfer = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(&bk) + 2048);
     static_assert(sizeof(Book) <= 2048, "bookkeeping reserve");
     volatile int* abort_flag = &bk.abort_flag;
@@ -495,7 +517,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int E = args.E;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < C::kStages; ++s) {
+        for (int s = 0; s < 16; ++s) {  // every stage the ring can be cut into
             mbar_init(&bk.full[s], 1);
             mbar_init(&bk.empty[s], 1);
         }
@@ -510,9 +532,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&tmW1);
         tma_prefetch_desc(&tmW3);
-        tma_prefetch_desc(&tmX);
         tma_prefetch_desc(&tmW2);
-        tma_prefetch_desc(&tmH);
+        for (int i = 0; i < kTokBoxes; ++i) {
+            tma_prefetch_desc(&tmX.m[i]);
+            tma_prefetch_desc(&tmH.m[i]);
+        }
     }
     if (warp == 1) tmem_alloc(&bk.tmem_base, C::kTmemCols);
 
@@ -526,12 +550,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             bk.off[g] = v;
             prev = v;
         }
-        bk.start1[0] = 0;
-        bk.start2[0] = 0;
+        int max_n = 1;
         for (int g = 0; g < E; ++g) {
             const int n = bk.off[g + 1] - bk.off[g];
             bk.end[g] = bk.off[g] + (n < args.cap ? n : args.cap);
-            const int chunks = (bk.end[g] - bk.off[g] + NT - 1) / NT;
+            max_n = bk.end[g] - bk.off[g] > max_n ? bk.end[g] - bk.off[g] : max_n;
+        }
+        const int ntr = tok_box_rows(tok_box_index(max_n), NT);
+        const int st = kRingBytes / (C::kAStage + ntr * 128);
+        bk.ntr = ntr;
+        bk.stages = st < 16 ? st : 16;
+        bk.start1[0] = 0;
+        bk.start2[0] = 0;
+        for (int g = 0; g < E; ++g) {
+            const int chunks = (bk.end[g] - bk.off[g] + ntr - 1) / ntr;
             bk.start1[g + 1] = bk.start1[g] + chunks * args.n_hb;
             bk.start2[g + 1] = bk.start2[g] + chunks * args.n_db * args.ksplit;
         }
@@ -540,6 +572,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
 
+    // the ring at this launch's tile size: A slots, then B slots of ntr rows
+    const int ntr = bk.ntr, n_stages = bk.stages;
+    const int b_slot = ntr * 128;
+    uint8_t* sB = smem + n_stages * C::kAStage;
+    const int tok_map = tok_box_index(ntr);
     const uint32_t tmem_base = bk.tmem_base;
     const int total = bk.start1[E] + bk.start2[E];
     const int num_kb1 = (args.d + kBK - 1) / kBK;
@@ -554,7 +591,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t phase = 0, pending = 0, pending_phase = 0;
             bool ok = true;
             for (int u = blockIdx.x; ok && u < total; u += gridDim.x) {
-                const FusedUnit f = fused_unit(bk, args, NT, num_kb1, kps, num_kb2, u);
+                const FusedUnit f = fused_unit(bk, args, ntr, num_kb1, kps, num_kb2, u);
                 if (f.down) {
                     // wait until every gate/up tile of this K range has published its H
                     const uint32_t need = static_cast<uint32_t>(f.chunks * (f.kb1 - f.kb0));
@@ -578,29 +615,29 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ok = false;
                         break;
                     }
-                    mbar_arrive_expect_tx(&bk.full[stage], C::kStageTx);
+                    mbar_arrive_expect_tx(&bk.full[stage], C::kAStage + b_slot);
                     const int kc = kb * kBK;
                     uint8_t* a = sA + stage * C::kAStage;
-                    uint8_t* b = sB + stage * C::kBStage;
+                    uint8_t* b = sB + stage * b_slot;
                     if (f.down) {
                         tma_load_2d_hint(&tmW2, &bk.full[stage], a, kc, wrow, evict_first);
-                        tma_load_2d(&tmH, &bk.full[stage], b, kc, f.row0);
+                        tma_load_2d(&tmH.m[tok_map], &bk.full[stage], b, kc, f.row0);
                     } else {
                         tma_load_2d_hint(&tmW1, &bk.full[stage], a, kc, wrow, evict_first);
                         tma_load_2d_hint(&tmW3, &bk.full[stage], a + J1 * 128, kc, wrow,
                                          evict_first);
-                        tma_load_2d(&tmX, &bk.full[stage], b, kc, f.row0);
+                        tma_load_2d(&tmX.m[tok_map], &bk.full[stage], b, kc, f.row0);
                     }
                     pending |= 1u << stage;
                     pending_phase = (pending_phase & ~(1u << stage)) | (phase << stage);
-                    if (++stage == C::kStages) {
+                    if (++stage == n_stages) {
                         stage = 0;
                         phase ^= 1u;
                     }
                 }
             }
             if (!ok) {
-                for (int s2 = 0; s2 < C::kStages; ++s2)
+                for (int s2 = 0; s2 < n_stages; ++s2)
                     if (pending & (1u << s2)) drain_wait(&bk.full[s2], (pending_phase >> s2) & 1u);
             }
         }
@@ -612,7 +649,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t phase = 0, acc_phase = 0;
             bool ok = true, issued = false;
             for (int u = blockIdx.x; ok && u < total; u += gridDim.x) {
-                const FusedUnit f = fused_unit(bk, args, NT, num_kb1, kps, num_kb2, u);
+                const FusedUnit f = fused_unit(bk, args, ntr, num_kb1, kps, num_kb2, u);
                 if (!mbar_wait_bounded(&bk.tmem_empty[acc], acc_phase ^ 1u, abort_flag,
                                        args.status)) {
                     ok = false;
@@ -620,6 +657,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * NT);
+                const uint32_t idesc = idesc_bf16_f32(kM, ntr);
                 for (int kb = f.kb0; kb < f.kb1; ++kb) {
                     if (!mbar_wait_bounded(&bk.full[stage], phase, abort_flag, args.status)) {
                         ok = false;
@@ -627,14 +665,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     tc_fence_after();
                     const uint64_t ad = sw128_kmajor_desc(smem_u32(sA + stage * C::kAStage));
-                    const uint64_t bd = sw128_kmajor_desc(smem_u32(sB + stage * C::kBStage));
+                    const uint64_t bd = sw128_kmajor_desc(smem_u32(sB + stage * b_slot));
 #pragma unroll
                     for (int k = 0; k < kBK / 16; ++k)
-                        umma_bf16(d_tmem, ad + 2 * k, bd + 2 * k, C::kIdesc,
+                        umma_bf16(d_tmem, ad + 2 * k, bd + 2 * k, idesc,
                                   (kb > f.kb0 || k > 0) ? 1u : 0u);
                     umma_commit(&bk.empty[stage]);
                     issued = true;
-                    if (++stage == C::kStages) {
+                    if (++stage == n_stages) {
                         stage = 0;
                         phase ^= 1u;
                     }
@@ -659,7 +697,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int u = blockIdx.x; u < total; u += gridDim.x) {
-            const FusedUnit f = fused_unit(bk, args, NT, num_kb1, kps, num_kb2, u);
+            const FusedUnit f = fused_unit(bk, args, ntr, num_kb1, kps, num_kb2, u);
             if (!bar_all(mbar_wait_bounded(&bk.tmem_full[acc], acc_phase, abort_flag, args.status),
                          kVoteBarrier, kEpiThreads))
                 break;
@@ -786,13 +824,16 @@ cudaError_t launch_ffn_fused_nt(const void* x_perm, const int32_t* offsets, cons
                                 const void* W3, const void* W2, int rows, int d, int h, int E,
                                 void* H, float* Ypart, int ksplit, uint32_t* counters,
                                 uint32_t* status, cudaStream_t s, int cap) {
-    CUtensorMap mw1, mw3, mx, mw2, mh;
+    CUtensorMap mw1, mw3, mw2;
+    TokMaps mx, mh;
     if (!encode_bf16_2d(&mw1, W1, static_cast<uint64_t>(E) * h, d, kM / 2) ||
         !encode_bf16_2d(&mw3, W3, static_cast<uint64_t>(E) * h, d, kM / 2) ||
-        !encode_bf16_2d(&mx, x_perm, rows, d, NT) ||
-        !encode_bf16_2d(&mw2, W2, static_cast<uint64_t>(E) * d, h, kM) ||
-        !encode_bf16_2d(&mh, H, rows, h, NT))
+        !encode_bf16_2d(&mw2, W2, static_cast<uint64_t>(E) * d, h, kM))
         return cudaErrorInvalidValue;
+    for (int i = 0; i < kTokBoxes; ++i)
+        if (!encode_bf16_2d(&mx.m[i], x_perm, rows, d, tok_box_rows(i, NT)) ||
+            !encode_bf16_2d(&mh.m[i], H, rows, h, tok_box_rows(i, NT)))
+            return cudaErrorInvalidValue;
     using C = DecodeCfg<kSwiGLU, NT>;
     auto kern = decode_ffn_fused_kernel<NT>;
     static PerDeviceOnce smem_once;
