@@ -523,7 +523,7 @@ def run_ours(args):
     K, W = args.steps, args.warmup
     suite = args.workload is None
     name = SUITE_HEADLINE if suite else args.workload
-    wl = WORKLOADS[name]
+    wl = with_tokens(WORKLOADS[name], args)
     inp = rank_inputs(wl, rank, world, device)
     head = measure_forward(wl, inp, K, W, world, local, device)
     cpu_baseline = None
@@ -579,6 +579,15 @@ def run_ours(args):
     if sub:
         out["workloads"] = sub
     return out
+
+
+def with_tokens(wl, args):
+    """The workload at --tokens tokens (same recipe and seed), if given."""
+    if getattr(args, "tokens", None):
+        if args.workload is None:
+            raise SystemExit("--tokens needs --workload")
+        return wl.with_tokens(args.tokens)
+    return wl
 
 
 def parallelism(world: int) -> str:
@@ -788,7 +797,7 @@ def run_ours_backward(args):
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
     init_dist("nccl")
-    wl = WORKLOADS[args.workload or SUITE_HEADLINE]
+    wl = with_tokens(WORKLOADS[args.workload or SUITE_HEADLINE], args)
     inp = rank_inputs(wl, rank, world, device)
     r = measure_backward(wl, inp, args.steps, args.warmup, world, local, device)
     cpu_baseline = None
@@ -829,7 +838,7 @@ def run_reference(args):
     rank, world, _ = dist_env()
     if rank != 0:
         return None
-    wl = WORKLOADS[args.workload or SUITE_HEADLINE]
+    wl = with_tokens(WORKLOADS[args.workload or SUITE_HEADLINE], args)
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     inp_cpu = cpu_copy(make_inputs(wl, dev))
     n = min(wl.T, args.cpu_sample_tokens)
@@ -886,6 +895,8 @@ def main(argv=None):
                     choices=["decode", "prefill", "skew", "long", "tiny_f32", "prefill_half"],
                     help="time one workload only (default: the prefill headline plus the "
                          "decode, skew and long layers and the prefill backward)")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="with --workload: the same recipe at this many tokens")
     ap.add_argument("--headline-only", action="store_true",
                     help="default run without the other workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
