@@ -284,6 +284,17 @@ def rank_inputs(wl, rank: int, world: int, device):
     return inp
 
 
+ZERO_WEIGHTS_NOTE = ("all-zero expert weights: a diagnostic that keeps the data path and the "
+                     "math but draws little power, so the SM clock stays near its maximum")
+
+
+def zero_expert_weights(inp, args):
+    """--zero-weights: W1, W3 and W2 set to zero (x and W_g, hence the routing, unchanged)."""
+    if getattr(args, "zero_weights", False):
+        for k in ("W1", "W3", "W2"):
+            inp[k].zero_()
+
+
 def regime_of(T: int) -> str:
     if T <= DECODE_MAX_TOKENS:
         return "decode"
@@ -525,6 +536,7 @@ def run_ours(args):
     name = SUITE_HEADLINE if suite else args.workload
     wl = with_tokens(WORKLOADS[name], args)
     inp = rank_inputs(wl, rank, world, device)
+    zero_expert_weights(inp, args)
     head = measure_forward(wl, inp, K, W, world, local, device)
     cpu_baseline = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -572,7 +584,8 @@ def run_ours(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype,
         "data": "synthetic (seeded normal draws of the Mixtral-8x7B layer shapes; "
                 "random-init weights)",
-        "config": workload_config(wl, {"parallelism": parallelism(world)}),
+        "config": workload_config(wl, {"parallelism": parallelism(world)}
+                                  | ({"weights": ZERO_WEIGHTS_NOTE} if args.zero_weights else {})),
         "roofline": head["roofline"], "layer": head["layer"], "cpu_baseline": cpu_baseline,
         "e2e": head["e2e"], "gpu_launches": head["gpu_launches"], "clocks": head["clocks"],
     }
@@ -799,6 +812,7 @@ def run_ours_backward(args):
     init_dist("nccl")
     wl = with_tokens(WORKLOADS[args.workload or SUITE_HEADLINE], args)
     inp = rank_inputs(wl, rank, world, device)
+    zero_expert_weights(inp, args)
     r = measure_backward(wl, inp, args.steps, args.warmup, world, local, device)
     cpu_baseline = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -816,6 +830,8 @@ def run_ours_backward(args):
     if rank != 0:
         return None
     cfg = dict(r["config"], parallelism=parallelism(world))
+    if args.zero_weights:
+        cfg["weights"] = ZERO_WEIGHTS_NOTE
     return {
         "metric": BWD_METRIC, "value": r["value"], "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": r["ms_per_step"],
@@ -897,6 +913,8 @@ def main(argv=None):
                          "decode, skew and long layers and the prefill backward)")
     ap.add_argument("--tokens", type=int, default=None,
                     help="with --workload: the same recipe at this many tokens")
+    ap.add_argument("--zero-weights", action="store_true",
+                    help="with --workload: all-zero expert weights (power diagnostic)")
     ap.add_argument("--headline-only", action="store_true",
                     help="default run without the other workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -913,6 +931,8 @@ def main(argv=None):
         args.warmup = 1 if ref else 10
     if not ref and args.warmup < 3:
         args.warmup = 3
+    if args.zero_weights and (args.workload is None or ref):
+        raise SystemExit("--zero-weights needs --workload (our arm)")
     if ref:
         out = run_reference(args)
     else:

@@ -10,7 +10,7 @@
 // shared memory) and N = 256 columns whose B operand is split between the CTAs
 // (128 rows of B each); each CTA's tensor memory receives its 128 rows x 256
 // columns.  Per SM this halves the B bytes staged per K block (32 KiB per stage
-// instead of 48 KiB for the same math), which leaves room for 6 pipeline stages
+// instead of 48 KiB for the same math), which leaves room for 6 or 7 pipeline stages
 // and cuts the L2->SM traffic by a third.
 //
 // GEMM1 covers 128 outputs n0 .. n0+127 per tile.  Each CTA stages 64 W1 rows and
