@@ -546,13 +546,19 @@ def run_ours(args):
 
     sub = {}
     if suite and not args.headline_only:
-        for other in SUITE_FORWARD:
+        def forward_workload(other):
             owl = WORKLOADS[other]
             oinp = rank_inputs(owl, rank, world, device)
             k = K * DECODE_STEP_FACTOR if owl.T <= DECODE_MAX_TOKENS else K
             sub[other] = measure_forward(owl, oinp, k, W, world, local, device)
             del oinp
             free_device_memory()
+
+        # the long-context layer runs for seconds at the power limit, so the
+        # bandwidth-bound sweep goes before it
+        for other in SUITE_FORWARD:
+            if other != "long":
+                forward_workload(other)
         sweep = []
         for T in SWEEP_TOKENS:
             for routing in SWEEP_ROUTINGS:
@@ -566,6 +572,8 @@ def run_ours(args):
                     "(grouped GEMMs), no events inside the timed region; bytes = touched "
                     "experts' weights + x + y",
             "steps": K, "warmup": W, "points": sweep}
+        if "long" in SUITE_FORWARD:
+            forward_workload("long")
         for other in SUITE_BACKWARD:
             owl = WORKLOADS[other]
             oinp = rank_inputs(owl, rank, world, device)

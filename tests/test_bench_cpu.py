@@ -7,6 +7,9 @@ import os
 import subprocess
 import sys
 
+import pytest
+import torch
+
 import bench
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -39,3 +42,25 @@ def test_default_run_headline_is_prefill():
     assert p.returncode == 0
     for opt in ("--gpus", "--steps", "--warmup", "--impl", "--workload", "--backward"):
         assert opt in p.stdout, opt
+
+
+def test_batch_size_and_diagnostic_options():
+    """--tokens runs a workload's recipe at another batch size (same seed); the
+    zero-weight power diagnostic is refused for the default line and the reference arm,
+    and leaves the routing inputs unchanged."""
+    from workloads import WORKLOADS, make_inputs
+    ns = argparse.Namespace(workload="prefill", tokens=96)
+    wl = bench.with_tokens(WORKLOADS["prefill"], ns)
+    assert wl.T == 96 and wl.seed == WORKLOADS["prefill"].seed and wl.kind == "plain"
+    with pytest.raises(SystemExit):
+        bench.with_tokens(WORKLOADS["prefill"], argparse.Namespace(workload=None, tokens=96))
+    for argv in (["--zero-weights"], ["--impl", "reference", "--workload", "tiny_f32",
+                                      "--zero-weights"]):
+        with pytest.raises(SystemExit):
+            bench.main(argv)
+    inp = make_inputs(WORKLOADS["tiny_f32"], "cpu")
+    x, wg = inp["x"].clone(), inp["Wg"].clone()
+    bench.zero_expert_weights(inp, argparse.Namespace(zero_weights=True))
+    assert all(float(inp[k].abs().max()) == 0.0 for k in ("W1", "W3", "W2"))
+    assert torch.equal(inp["x"], x) and torch.equal(inp["Wg"], wg)
+    assert bench.SWEEP_TOKENS == (192, 256, 384) and set(bench.SWEEP_ROUTINGS) == {"prefill", "skew"}
