@@ -617,7 +617,7 @@ def parallelism(world: int) -> str:
 
 # ------------------------------------------------------------------ our arm, backward
 BWD_METRIC = "MoE-layer backward tokens/s (dx, dW1, dW3, dW2, dWg) and % of bf16 TC peak"
-BWD_STAGES = ["prep (dY, dw, dlogits)", "dH = dY W2", "du, dv (recompute a, b)",
+BWD_STAGES = ["prep (dY, dw, dlogits)", "dH = dY W2", "du, dv",
               "dX = [du dv][W1; W3]", "dx combine", "dW2", "dW1 + dW3", "dWg"]
 BWD_KERNELS = (1, 2, 3, 5, 6)  # the tensor-core stages
 BWD_PAIR_MIN_ROWS = 2048      # row GEMMs on CTA pairs from here (grouped rows)
@@ -639,10 +639,20 @@ def backward_kernel(wl, stage: int):
     return names[stage][0 if pair else 1], {1: "bwd_dh", 2: "bwd_duv", 3: "bwd_dx"}[stage]
 
 
+def keeps_pre_activations(wl) -> bool:
+    """From 1024 grouped rows on, the training forward keeps a and b, and the
+    backward's du/dv step is element-wise instead of a second GEMM1."""
+    return wl.T * wl.k >= 1024
+
+
 def backward_stage_flops(wl):
-    """Tensor-core flops of each GEMM stage (2*P*d*h units; P = 2T grouped rows)."""
+    """Tensor-core flops of each GEMM stage (2*P*d*h units; P = 2T grouped rows); the
+    du/dv step counts only where it recomputes a and b."""
     u = 2 * (wl.T * wl.k) * wl.d * wl.h
-    return {1: u, 2: 2 * u, 3: 2 * u, 5: u, 6: 2 * u}
+    f = {1: u, 2: 2 * u, 3: 2 * u, 5: u, 6: 2 * u}
+    if keeps_pre_activations(wl):
+        del f[2]
+    return f
 
 
 def wgrad_bytes(wl, stage: int) -> int:
@@ -656,10 +666,12 @@ def wgrad_bytes(wl, stage: int) -> int:
 
 
 def measure_backward(wl, inp, K: int, W: int, world: int, local: int, device):
-    """Time K backward calls (after one forward that fills the saved state and W
-    warm-up calls), with events between the backward's stages inside the timed
-    region, then the same steps end to end (dy in, dx out through pinned host
-    buffers).  Returns the workload's result object."""
+    """Time K backward calls (after one training forward that fills the saved state --
+    from 512 tokens on it keeps the pre-activations a, b, so the backward computes du,
+    dv element by element -- and W warm-up calls), with events between the backward's
+    stages inside the timed region, then K training and K plain forward calls (the
+    training forward's cost), then the same backward steps end to end (dy in, dx out
+    through pinned host buffers).  Returns the workload's result object."""
     import torch
 
     import sparse_mixture_experts_26_b200 as moe
@@ -672,7 +684,7 @@ def measure_backward(wl, inp, K: int, W: int, world: int, local: int, device):
     ws = moe.alloc_workspace(T, d, h, E, wl.k, x.dtype, device)
     bws = moe.alloc_backward_workspace(T, d, h, E, wl.k, x.dtype, device)
     y = torch.empty_like(x)
-    moe.moe_layer_forward(x, Wg, W1, W3, W2, y, ws)  # the saved state the backward reads
+    moe.moe_layer_forward_train(x, Wg, W1, W3, W2, y, ws, bws)  # the state the backward reads
     dy = backward_dy(T, d).to(device)
     dx = torch.empty_like(x)
     f32 = dict(dtype=torch.float32, device=device)
@@ -714,7 +726,7 @@ def measure_backward(wl, inp, K: int, W: int, world: int, local: int, device):
     st_ms = [sum(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(K)) / K
              for j in range(nst - 1)]
     flops = backward_stage_flops(wl)
-    dom = max(BWD_KERNELS, key=lambda j: st_ms[j])
+    dom = max((j for j in BWD_KERNELS if j in flops), key=lambda j: st_ms[j])
     kname, tag = backward_kernel(wl, dom)
     peaks, peak_src = load_peaks()
     if T <= DECODE_MAX_TOKENS and dom in (5, 6):
@@ -754,6 +766,29 @@ def measure_backward(wl, inp, K: int, W: int, world: int, local: int, device):
              "stage_ms": {n: round(v, 4) for n, v in zip(BWD_STAGES, st_ms)},
              "stage_tflops": {BWD_STAGES[j]: round(flops[j] / (st_ms[j] * 1e-3) / 1e12, 1)
                               for j in flops}}
+
+    # The forward a training step pays: moe_layer_forward (nothing kept) and
+    # moe_layer_forward_train (a and b kept), K calls each, the training one last so
+    # that the end-to-end backward steps below read the state it keeps.
+    def time_forward(call):
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        call()
+        torch.cuda.synchronize()
+        barrier(world, device)
+        f0.record(stream)
+        for _ in range(K):
+            call()
+        f1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world, device)
+        return max_over_ranks(f0.elapsed_time(f1) / K, world, device)
+    fwd_ms = time_forward(lambda: moe.moe_layer_forward(x, Wg, W1, W3, W2, y, ws))
+    fwd_train_ms = time_forward(lambda: moe.moe_layer_forward_train(x, Wg, W1, W3, W2, y, ws,
+                                                                    bws))
+    layer["forward_ms"] = round(fwd_ms, 4)
+    layer["forward_train_ms"] = round(fwd_train_ms, 4)
+    layer["train_step_ms"] = round(fwd_train_ms + ms, 4)
+    layer["pre_activations_kept"] = keeps_pre_activations(wl)
 
     # End to end through the public API with host buffers: dy in from pinned host memory,
     # dx back to pinned host memory, both on their own streams, double-buffered; the

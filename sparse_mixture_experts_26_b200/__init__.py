@@ -25,7 +25,7 @@ __all__ = [
     "EXPORTED_SYMBOLS", "launches_per_layer", "launches_per_backward", "moe_expert_ffn_static",
     "moe_layer_forward_capacity", "moe_selftest_wait_timeout", "moe_backward_workspace_bytes",
     "moe_layer_backward", "alloc_backward_workspace", "layer_backward",
-    "moe_layer_backward_events",
+    "moe_layer_backward_events", "moe_layer_forward_train",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe.so")
@@ -38,7 +38,7 @@ EXPORTED_SYMBOLS = ("moe_workspace_bytes", "moe_route", "moe_permute", "moe_expe
                     "moe_device_status", "moe_status_string", "moe_expert_ffn_static",
                     "moe_layer_forward_capacity", "moe_selftest_wait_timeout",
                     "moe_backward_workspace_bytes", "moe_layer_backward",
-                    "moe_layer_backward_events")
+                    "moe_layer_backward_events", "moe_layer_forward_train")
 def launches_per_layer(T: int, d: int = 4096, E: int = 8, bf16: bool = True) -> int:
     """Kernels one moe_layer_forward queues: router 1, permutation 1 (T <= 512) or 4
     (count, scan, rank, gather; 3 where the bf16 fp64-tensor-core router counts the
@@ -53,12 +53,14 @@ def launches_per_layer(T: int, d: int = 4096, E: int = 8, bf16: bool = True) -> 
 
 def launches_per_backward(T: int, capacity: int = -1) -> int:
     """Kernels one moe_layer_backward queues: prep, dH, du/dv, dX, dx, the two
-    weight-gradient GEMMs, the dWg partials and their sum (9), plus the padded copies
-    of dY and x_perm when the weight gradients run on CTA pairs (more than 1024
-    grouped rows) without a capacity; none for T == 0."""
+    weight-gradient GEMMs, the dWg partials and their sum (9), plus, without a
+    capacity, the element-wise du/dv kernel beside the recomputing one from 1024
+    grouped rows on (one of the two returns at once, by what the forward kept) and the
+    padded copies of dY and x_perm above 1024 grouped rows; none for T == 0."""
     if T <= 0:
         return 0
-    return 9 + (1 if 2 * T > 1024 and capacity < 0 else 0)
+    free = capacity < 0
+    return 9 + (1 if 2 * T >= 1024 and free else 0) + (1 if 2 * T > 1024 and free else 0)
 
 
 class MoeError(RuntimeError):
@@ -93,6 +95,8 @@ def _load() -> ctypes.CDLL:
         "moe_backward_workspace_bytes": (sz, [i32, i32, i32, i32, i32, i32]),
         "moe_layer_backward": (i32, [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32,
                                      vp, vp, vp, vp, vp, vp, sz, vp, sz, vp]),
+        "moe_layer_forward_train": (i32, [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp,
+                                          vp, sz, vp, sz, vp]),
         "moe_layer_backward_events": (i32, [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
                                             i32, vp, vp, vp, vp, vp, vp, sz, vp, sz, vp, i32,
                                             vp]),
@@ -276,6 +280,21 @@ def moe_layer_forward(x, Wg, W1, W3, W2, y, ws, k: int = 2, stream=None) -> None
         _check("moe_layer_forward", _lib.moe_layer_forward(
             _ptr(x), _ptr(Wg), _ptr(W1), _ptr(W3), _ptr(W2), T, d, h, E, k, _dt(x), _ptr(y),
             _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def moe_layer_forward_train(x, Wg, W1, W3, W2, y, ws, bwd_ws, k: int = 2, stream=None) -> None:
+    """``moe_layer_forward`` that also keeps the pre-activations a, b (fp32) in
+    ``bwd_ws`` from 512 tokens on, for the ``moe_layer_backward`` call that follows."""
+    T, d, h, E = _layer_dims(x, Wg, W1, W3, W2)
+    _expect("y", y, (T, d), x.dtype)
+    _ws("ws", ws)
+    _ws("bwd_ws", bwd_ws)
+    dev = _dev(x, Wg, W1, W3, W2, y, ws, bwd_ws)
+    with torch.cuda.device(dev):
+        _check("moe_layer_forward_train", _lib.moe_layer_forward_train(
+            _ptr(x), _ptr(Wg), _ptr(W1), _ptr(W3), _ptr(W2), T, d, h, E, k, _dt(x), _ptr(y),
+            _ptr(ws), ws.numel() * ws.element_size(), _ptr(bwd_ws),
+            bwd_ws.numel() * bwd_ws.element_size(), _stream(stream)))
 
 
 def moe_layer_forward_capacity(x, Wg, W1, W3, W2, y, ws, capacity: int, k: int = 2,

@@ -47,7 +47,7 @@ bool encode_f32_3d(CUtensorMap* map, const void* base, uint64_t batches, uint64_
 cudaError_t launch_bwd_rows_pair(int mode, const CUtensorMap& a, const CUtensorMap& b0,
                                  const CUtensorMap& b1, const int32_t* offsets, int E, int rows,
                                  int d, int h, void* out, const float* dH, uint32_t* status,
-                                 int cap, cudaStream_t s);
+                                 int cap, cudaStream_t s, const uint8_t* skip_flag = nullptr);
 // Defined in backward_pair_sm100.cu.
 cudaError_t launch_wgrad_pair(const CUtensorMap& A, const CUtensorMap& B, const int32_t* offsets,
                               int E, int rows,
@@ -657,6 +657,43 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ================================================================ CUDA-core kernels
 constexpr int kPrepThreads = 256;
 
+// du, dv from dH and the pre-activations a, b that moe_layer_forward_train kept, element
+// by element, with the formula of the recomputing GEMM's epilogue: the same a and b
+// (the forward's GEMM1 accumulators) give the same du and dv.  Does nothing unless the
+// forward's layout byte says that a and b were kept (then the recomputing GEMM does
+// nothing instead).  du in columns [0, h) of each DUV row, dv in [h, 2h).
+__global__ void __launch_bounds__(kPrepThreads)
+    bwd_duv_saved_kernel(const uint8_t* __restrict__ y_layout, const float* __restrict__ dH,
+                         const float* __restrict__ a_pre, const float* __restrict__ b_pre,
+                         int P, int h, __nv_bfloat16* __restrict__ duv) {
+    if ((*y_layout & kLayoutSavedAB) == 0) return;
+    const int h4 = h / 4;
+    const size_t n = static_cast<size_t>(P) * h4;
+    for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
+         i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+        const size_t r = i / h4;
+        const size_t c = (i - r * h4) * 4;
+        const float4 g = *reinterpret_cast<const float4*>(dH + r * h + c);
+        const float4 a = *reinterpret_cast<const float4*>(a_pre + r * h + c);
+        const float4 b = *reinterpret_cast<const float4*>(b_pre + r * h + c);
+        const float gv[4] = {g.x, g.y, g.z, g.w}, av4[4] = {a.x, a.y, a.z, a.w},
+                    bv4[4] = {b.x, b.y, b.z, b.w};
+        float ru[4], rv[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const float av = av4[u];
+            const float bv = bv4[u];
+            const float s = __frcp_rn(1.0f + __expf(-av));
+            ru[u] = gv[u] * bv * (s * (1.0f + av * (1.0f - s)));
+            rv[u] = gv[u] * (av * s);
+        }
+        __nv_bfloat16* row = duv + r * 2 * h;
+        *reinterpret_cast<uint2*>(row + c) = make_uint2(pack_bf16x2(ru[0], ru[1]), pack_bf16x2(ru[2], ru[3]));
+        *reinterpret_cast<uint2*>(row + h + c) =
+            make_uint2(pack_bf16x2(rv[0], rv[1]), pack_bf16x2(rv[2], rv[3]));
+    }
+}
+
 // Is pair (t, j) kept?  (expert id valid, grouped row in range, within capacity)
 __device__ __forceinline__ bool pair_kept(const int32_t* idx, const int32_t* offsets,
                                           const int32_t* inv, int f, int E, int P, int cap) {
@@ -682,7 +719,7 @@ __global__ void __launch_bounds__(kPrepThreads)
                     float* __restrict__ dlogits) {
     __shared__ float red[2][kPrepThreads / 32];
     const int P = 2 * T;
-    int nsplit = kSplit ? *y_layout : 1;
+    int nsplit = kSplit ? (*y_layout & kLayoutSplitMask) : 1;
     nsplit = nsplit < 1 ? 1 : (nsplit > kDecodeSplitK ? kDecodeSplitK : nsplit);
     const float* __restrict__ Y = nsplit > 1 ? Ypart : Y1;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -1038,10 +1075,20 @@ cudaError_t launch_layer_backward(const BwdArgs& a, cudaStream_t s) {
                        kSmemBytes, s, m_dY128, m_W2, m_W2, r);
         if (err != cudaSuccess || (err = mark(2)) != cudaSuccess) return err;
     }
-    // 3. du, dv (recomputes a and b)
+    // 3. du, dv: from the pre-activations the forward kept (moe_layer_forward_train), or
+    // recomputing a and b; the forward's layout byte selects which of the two launches
+    // does the work (the other returns at once), so the host never waits for it
     if (pairs) {
+        if (a.a_pre != nullptr) {
+            const long long n4 = static_cast<long long>(P) * (h / 4);
+            err = launch_k(bwd_duv_saved_kernel,
+                           grid_for((n4 + kPrepThreads - 1) / kPrepThreads, 8 * sms), kPrepThreads,
+                           0, s, a.y_layout, static_cast<const float*>(a.dH), a.a_pre, a.b_pre, P,
+                           h, static_cast<__nv_bfloat16*>(a.DUV));
+            if (err != cudaSuccess) return err;
+        }
         err = launch_bwd_rows_pair(1, m_x, m_W1r, m_W3r, a.offsets, E, P, d, h, a.DUV, a.dH,
-                                   a.status, a.cap, s);
+                                   a.status, a.cap, s, a.a_pre != nullptr ? a.y_layout : nullptr);
         if (err != cudaSuccess || (err = mark(3)) != cudaSuccess) return err;
     } else {
         RowArgs r{a.offsets, E, P, d, h, (h + 127) / 128, h, d, a.DUV, a.dH, a.status, a.cap};

@@ -60,11 +60,12 @@ __global__ void __launch_bounds__(kCombineThreads)
     combine_kernel(const float4* __restrict__ Y, int nsplit, size_t split_stride4,
                    const int32_t* __restrict__ inv, const float* __restrict__ w, int T, int d4,
                    Tout* __restrict__ y, const int32_t* __restrict__ idx,
-                   const int32_t* __restrict__ offsets, int E, int cap, uint8_t* layout_out) {
+                   const int32_t* __restrict__ offsets, int E, int cap, uint8_t* layout_out,
+                   int layout_value) {
     pdl_wait();
     pdl_launch_dependents();
     if (layout_out && blockIdx.x == 0 && threadIdx.x == 0)
-        *layout_out = static_cast<uint8_t>(nsplit);
+        *layout_out = static_cast<uint8_t>(layout_value);
     const size_t n = static_cast<size_t>(T) * d4;
     const unsigned P = 2u * static_cast<unsigned>(T);
     for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
@@ -135,8 +136,10 @@ cudaError_t launch_sum_splits(const float* parts, int nsplit, size_t n, float* Y
 cudaError_t launch_combine(const float* Y, int nsplit, size_t split_stride,
                            const int32_t* inv_perm, const float* w, int T, int d, moe_dtype dt,
                            void* y, cudaStream_t s, const int32_t* idx, const int32_t* offsets,
-                           int E, int cap, uint8_t* layout_out) {
+                           int E, int cap, uint8_t* layout_out, uint8_t layout_flags) {
     if (cap != INT_MAX && (!idx || !offsets)) return cudaErrorInvalidValue;
+    if (nsplit < 1 || nsplit > kLayoutSplitMask) return cudaErrorInvalidValue;
+    const int lv = nsplit | layout_flags;
     const int d4 = d / 4;
     const unsigned blocks = grid_for(static_cast<size_t>(T) * d4);
     const float4* Y4 = reinterpret_cast<const float4*>(Y);
@@ -145,15 +148,15 @@ cudaError_t launch_combine(const float* Y, int nsplit, size_t split_stride,
         if (nsplit > 1)
             return launch_k(combine_kernel<__nv_bfloat16, true>, blocks, kCombineThreads, 0, s, Y4,
                             nsplit, split_stride / 4, inv_perm, w, T, d4, yb, idx, offsets, E,
-                            cap, layout_out);
+                            cap, layout_out, lv);
         return launch_k(combine_kernel<__nv_bfloat16, false>, blocks, kCombineThreads, 0, s, Y4,
                         nsplit, split_stride / 4, inv_perm, w, T, d4, yb, idx, offsets, E, cap,
-                        layout_out);
+                        layout_out, lv);
     }
     if (nsplit != 1) return cudaErrorInvalidValue;  // split-K partials are bf16-path only
     return launch_k(combine_kernel<float, false>, blocks, kCombineThreads, 0, s, Y4, nsplit,
                     split_stride / 4, inv_perm, w, T, d4, static_cast<float*>(y), idx, offsets, E,
-                    cap, layout_out);
+                    cap, layout_out, lv);
 }
 
 }  // namespace moe

@@ -112,6 +112,13 @@ struct PairArgs {
     int h;             // kBMnSplit: the K index where W3 takes over from W1
     const float* dH;   // kEpiBwdSwiGLU: dH fp32 [rows, N]
     int group;         // row blocks whose A rows stay in L2 together (tile order)
+    // kEpiSwiGLU, optional: the pre-activations a = x W1^T and b = x W3^T, fp32
+    // [rows, N] each, kept for the backward pass (nullptr: not written)
+    float* a_out;
+    float* b_out;
+    // optional: the launch does nothing when bit 7 of this device byte is set (the
+    // backward's recompute of a and b, when the forward kept them)
+    const uint8_t* skip_flag;
 };
 
 struct PairBook {
@@ -181,6 +188,25 @@ __device__ __forceinline__ void bwd_swiglu(float a, float b, float g, float& du,
     dv = g * (a * s);
 }
 
+// The 32 pre-activations a and b of one row that a GEMM1 epilogue chunk holds, kept in
+// fp32 for the backward pass (columns past N are not written).
+__device__ __forceinline__ void store_pre_activations(const PairArgs& args, int row, int col0,
+                                                      const uint32_t (&a)[32],
+                                                      const uint32_t (&b)[32]) {
+    float* ar = args.a_out + static_cast<size_t>(row) * args.N;
+    float* br = args.b_out + static_cast<size_t>(row) * args.N;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const int col = col0 + 4 * j;
+        if (col < args.N) {
+            *reinterpret_cast<float4*>(ar + col) = make_float4(
+                bits_f32(a[4 * j]), bits_f32(a[4 * j + 1]), bits_f32(a[4 * j + 2]), bits_f32(a[4 * j + 3]));
+            *reinterpret_cast<float4*>(br + col) = make_float4(
+                bits_f32(b[4 * j]), bits_f32(b[4 * j + 1]), bits_f32(b[4 * j + 2]), bits_f32(b[4 * j + 3]));
+        }
+    }
+}
+
 template <int EPI, int BOP = kBKMajor>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
@@ -207,6 +233,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool leader = rank == 0;
     const int pair = blockIdx.x >> 1;
     const int npairs = gridDim.x >> 1;
+    // Both CTAs of every pair read the same byte, so a skipped launch leaves together
+    // before any barrier, cluster synchronisation or tensor-memory allocation.
+    if (args.skip_flag != nullptr && (*args.skip_flag & 0x80u) != 0) return;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
@@ -419,6 +448,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                     *reinterpret_cast<uint4*>(out + col) =
                                         make_uint4(p[4 * v], p[4 * v + 1], p[4 * v + 2], p[4 * v + 3]);
                             }
+                            if (args.a_out != nullptr)
+                                store_pre_activations(args, row, col0 + ch * 32, a, b);
                         }
                     }
                 } else if (EPI == kEpiBwdSwiGLU) {
@@ -537,6 +568,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                     *reinterpret_cast<uint4*>(out + col) =
                                         make_uint4(p[4 * u], p[4 * u + 1], p[4 * u + 2], p[4 * u + 3]);
                             }
+                            if (args.a_out != nullptr)
+                                store_pre_activations(args, row, col0 + ch * 32, a, b);
                         }
                     }
                 } else if (EPI == kEpiBwdSwiGLU) {
@@ -654,7 +687,7 @@ cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b0, const CUten
 cudaError_t launch_ffn_bf16_pair(const void* x_perm, const int32_t* offsets, const void* W1,
                                  const void* W3, const void* W2, int rows, int d, int h, int E,
                                  void* H, float* Y, uint32_t* status, cudaStream_t s,
-                                 cudaEvent_t between, int cap) {
+                                 cudaEvent_t between, int cap, float* a_out, float* b_out) {
     CUtensorMap mx, mw1, mw3, mh, mw2, my;
     if (!encode_f32_3d(&my, Y, 1, rows, d, 32, 32) ||
         !encode_bf16_2d(&mx, x_perm, rows, d, kRowsPerCta) ||
@@ -666,6 +699,8 @@ cudaError_t launch_ffn_bf16_pair(const void* x_perm, const int32_t* offsets, con
     const int max_pairs = device_sm_count() / 2;
     const long long blocks = (static_cast<long long>(rows) + (kPairRows - 1LL) * E) / kPairRows;
     PairArgs g1{offsets, E, rows, d, h, h, (h + 127) / 128, H, status, cap};
+    g1.a_out = a_out;
+    g1.b_out = b_out;
     long long t1 = blocks * g1.n_tiles;
     const int grid1 = static_cast<int>(t1 < max_pairs ? (t1 < 1 ? 1 : t1) : max_pairs);
     cudaError_t err = launch_pair<kEpiSwiGLU>(mx, mw1, mw3, mx, g1, grid1, s);
@@ -685,7 +720,7 @@ cudaError_t launch_ffn_bf16_pair(const void* x_perm, const int32_t* offsets, con
 cudaError_t launch_bwd_rows_pair(int mode, const CUtensorMap& a, const CUtensorMap& b0,
                                  const CUtensorMap& b1, const int32_t* offsets, int E, int rows,
                                  int d, int h, void* out, const float* dH, uint32_t* status,
-                                 int cap, cudaStream_t s) {
+                                 int cap, cudaStream_t s, const uint8_t* skip_flag) {
     const int max_pairs = device_sm_count() / 2;
     const long long blocks = (static_cast<long long>(rows) + (kPairRows - 1LL) * E) / kPairRows;
     auto grid = [&](long long tiles) {
@@ -699,6 +734,7 @@ cudaError_t launch_bwd_rows_pair(int mode, const CUtensorMap& a, const CUtensorM
     }
     if (mode == 1) {
         PairArgs g{offsets, E, rows, d, h, h, (h + 127) / 128, out, status, cap, h, dH};
+        g.skip_flag = skip_flag;
         return launch_pair<kEpiBwdSwiGLU, kBKMajor>(a, b0, b1, a, g, grid(blocks * g.n_tiles), s);
     }
     CUtensorMap mo;  // dX [rows, d] fp32

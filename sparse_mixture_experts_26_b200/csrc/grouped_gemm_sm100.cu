@@ -455,7 +455,8 @@ cudaError_t launch_ffn_bf16(const void* x_perm, const int32_t* offsets, const vo
                             const void* W3, const void* W2, int rows, int d, int h, int E,
                             void* H, float* Y, float* partials, int partial_cap, bool reduce,
                             FfnOut* out, uint32_t* status, cudaStream_t s,
-                            cudaEvent_t between, uint32_t* counters, int cap) {
+                            cudaEvent_t between, uint32_t* counters, int cap, float* a_save,
+                            float* b_save) {
     // Small batches stream the weights: the fused cooperative launch up to
     // kFusedMaxRows rows, the two-launch form (no co-residency needed) up to
     // kDecodeMaxRows; above that, or where neither applies, the grouped GEMMs below.
@@ -492,9 +493,12 @@ cudaError_t launch_ffn_bf16(const void* x_perm, const int32_t* offsets, const vo
         // 129..256 rows on a device that cannot co-schedule the fused launch: grouped GEMMs
     }
     if (out) *out = FfnOut{Y, 1};
-    if (rows >= kPairMinRows && pair_gemm_enabled())
+    if (rows >= kPairMinRows && pair_gemm_enabled()) {
+        // the CTA-pair GEMM1 can also keep the pre-activations for the backward pass
+        if (out) out->saved_ab = a_save != nullptr && b_save != nullptr;
         return launch_ffn_bf16_pair(x_perm, offsets, W1, W3, W2, rows, d, h, E, H, Y, status, s,
-                                    between, cap);
+                                    between, cap, a_save, b_save);
+    }
     // GEMM1 tile width: 112 outputs where h is a multiple of 112 (see the file comment)
     const int no = h % 112 == 0 ? 112 : 128;
     CUtensorMap mx, mw1, mw3, mh, mw2;

@@ -119,8 +119,12 @@ T* at(void* ws, size_t off) {
 
 // Backward workspace regions (1 KiB aligned); the status word at offset 0.
 struct BwdLayout {
-    size_t status, dY, dw, dlogits, dH, DUV, dX, dwg_part, dY_pad, x_pad, total;
+    size_t status, dY, dw, dlogits, dH, DUV, dX, dwg_part, dY_pad, x_pad, a_pre, b_pre, total;
 };
+
+// Batches whose forward can keep the pre-activations for the backward pass (the
+// CTA-pair range of the expert FFN).
+bool keeps_pre_activations(int T) { return 2 * T >= kPairMinRows; }
 
 BwdLayout bwd_layout(int T, int d, int h, int E) {
     BwdLayout B{};
@@ -141,6 +145,11 @@ BwdLayout bwd_layout(int T, int d, int h, int E) {
     B.dwg_part = take(bwd_dwg_chunks(T) * d * E * 4);
     B.dY_pad = take(bwd_pad_rows(T, E) * d * 2);
     B.x_pad = take(bwd_pad_rows(T, E) * d * 2);
+    // a = x W1^T and b = x W3^T of every grouped row, fp32, as moe_layer_forward_train
+    // keeps them
+    const bool keep = keeps_pre_activations(T);
+    B.a_pre = take(keep ? P * h * 4 : 0);
+    B.b_pre = take(keep ? P * h * 4 : 0);
     B.total = o;
     return B;
 }
@@ -259,7 +268,8 @@ namespace {
 moe_status layer_forward_impl(const void* x, const void* Wg, const void* W1, const void* W3,
                               const void* W2, int T, int d, int h, int E, int k, moe_dtype dt,
                               void* y, void* ws, size_t ws_bytes, cudaEvent_t* ev, int n_ev,
-                              cudaStream_t stream, int cap) {
+                              cudaStream_t stream, int cap, float* a_save = nullptr,
+                              float* b_save = nullptr) {
     moe_status st = check_shape(T, d, h, E, k, dt, true);
     if (st != MOE_OK) return st;
     if (n_ev < 0 || (n_ev > 0 && ev == nullptr)) return MOE_ERR_INVALID_ARG;
@@ -306,7 +316,7 @@ moe_status layer_forward_impl(const void* x, const void* Wg, const void* W1, con
             err = launch_ffn_bf16(x_perm, offsets, W1, W3, W2, P, d, h, E, at<void>(ws, L.H), Y,
                                   at<float>(ws, L.Ypart), kDecodeSplitK, /*reduce=*/false, &fo,
                                   status, stream, n_ev > 2 ? ev[2] : nullptr,
-                                  at<uint32_t>(ws, L.sync), cap);
+                                  at<uint32_t>(ws, L.sync), cap, a_save, b_save);
             if (err == cudaErrorInvalidValue) return MOE_ERR_INVALID_ARG;
         } else {
             err = launch_ffn_f32(static_cast<const float*>(x_perm), offsets,
@@ -320,7 +330,8 @@ moe_status layer_forward_impl(const void* x, const void* Wg, const void* W1, con
     {
         NvtxRange r("combine");
         err = launch_combine(fo.Y, fo.nsplit, static_cast<size_t>(P) * d, inv_perm, w, T, d, dt,
-                             y, stream, idx, offsets, E, cap, at<uint8_t>(ws, L.y_layout));
+                             y, stream, idx, offsets, E, cap, at<uint8_t>(ws, L.y_layout),
+                             fo.saved_ab ? kLayoutSavedAB : 0);
     }
     if ((st = finish(err, stream, status)) != MOE_OK) return st;
     if (!mark(4)) return MOE_ERR_CUDA;
@@ -353,6 +364,22 @@ moe_status moe_layer_forward_events(const void* x, const void* Wg, const void* W
                                     cudaEvent_t* events, int n_events, cudaStream_t stream) {
     return layer_forward_impl(x, Wg, W1, W3, W2, T, d, h, E, k, dt, y, ws, ws_bytes, events,
                               n_events, stream, INT_MAX);
+}
+
+moe_status moe_layer_forward_train(const void* x, const void* Wg, const void* W1, const void* W3,
+                                   const void* W2, int T, int d, int h, int E, int k,
+                                   moe_dtype dt, void* y, void* ws, size_t ws_bytes,
+                                   void* bwd_ws, size_t bwd_ws_bytes, cudaStream_t stream) {
+    moe_status st = check_shape(T, d, h, E, k, dt, true);
+    if (st != MOE_OK) return st;
+    if (dt != MOE_BF16 || h % 64 != 0) return MOE_ERR_UNSUPPORTED;
+    if (T > 0 && !ptrs_ok({bwd_ws})) return MOE_ERR_INVALID_ARG;
+    const BwdLayout B = bwd_layout(T, d, h, E);
+    if (bwd_ws_bytes < B.total) return MOE_ERR_WORKSPACE;
+    const bool keep = keeps_pre_activations(T);
+    return layer_forward_impl(x, Wg, W1, W3, W2, T, d, h, E, k, dt, y, ws, ws_bytes, nullptr, 0,
+                              stream, INT_MAX, keep ? at<float>(bwd_ws, B.a_pre) : nullptr,
+                              keep ? at<float>(bwd_ws, B.b_pre) : nullptr);
 }
 
 size_t moe_backward_workspace_bytes(int T, int d, int h, int E, int k, moe_dtype dt) {
@@ -421,6 +448,11 @@ moe_status layer_backward_impl(const void* x, const void* Wg, const void* W1, co
     a.dwg_part = at<float>(bwd_ws, B.dwg_part);
     a.dY_pad = at<void>(bwd_ws, B.dY_pad);
     a.x_pad = at<void>(bwd_ws, B.x_pad);
+    // where moe_layer_forward_train may have kept a and b (the forward's layout byte
+    // says whether it did); a capacity layer always recomputes them
+    const bool keep = keeps_pre_activations(T) && a.cap == INT_MAX;
+    a.a_pre = keep ? at<float>(bwd_ws, B.a_pre) : nullptr;
+    a.b_pre = keep ? at<float>(bwd_ws, B.b_pre) : nullptr;
     a.status = at<uint32_t>(bwd_ws, B.status);
     a.ev = ev;
     a.n_ev = n_ev;

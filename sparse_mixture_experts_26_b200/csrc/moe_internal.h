@@ -180,20 +180,22 @@ cudaError_t launch_ffn_f32(const float* x_perm, const int32_t* offsets, const fl
 struct FfnOut {
     const float* Y;
     int nsplit;
+    bool saved_ab = false;  // the pre-activations a and b were written (a_save / b_save)
 };
 cudaError_t launch_ffn_bf16(const void* x_perm, const int32_t* offsets, const void* W1,
                             const void* W3, const void* W2, int rows, int d, int h, int E,
                             void* H, float* Y, float* partials, int partial_cap, bool reduce,
                             FfnOut* out, uint32_t* status, cudaStream_t s,
                             cudaEvent_t between = nullptr, uint32_t* counters = nullptr,
-                            int cap = INT_MAX);
+                            int cap = INT_MAX, float* a_save = nullptr, float* b_save = nullptr);
 // With `counters` (2 * kMaxExperts * kDecodeSplitK zeroed words, left zeroed) small
 // batches run the fused single-launch FFN; `between` is then recorded after it.
 // Large-batch expert FFN on CTA pairs (tcgen05 cta_group::2).
 cudaError_t launch_ffn_bf16_pair(const void* x_perm, const int32_t* offsets, const void* W1,
                                  const void* W3, const void* W2, int rows, int d, int h, int E,
                                  void* H, float* Y, uint32_t* status, cudaStream_t s,
-                                 cudaEvent_t between, int cap);
+                                 cudaEvent_t between, int cap, float* a_out = nullptr,
+                                 float* b_out = nullptr);
 // Grouped rows from which the CTA-pair kernels are used (MOE_GEMM_PAIR=0 disables them):
 // the forward's expert FFN, and the backward's row-grouped GEMMs.
 constexpr int kPairMinRows = 1024;
@@ -221,7 +223,12 @@ cudaError_t launch_combine(const float* Y, int nsplit, size_t split_stride,
                            const int32_t* inv_perm, const float* w, int T, int d, moe_dtype dt,
                            void* y, cudaStream_t s, const int32_t* idx = nullptr,
                            const int32_t* offsets = nullptr, int E = 0, int cap = INT_MAX,
-                           uint8_t* layout_out = nullptr);
+                           uint8_t* layout_out = nullptr, uint8_t layout_flags = 0);
+// The layout byte the combine records for the backward pass: the number of split-K
+// partials holding the expert outputs (1: the single array Y) in bits 0..6, and bit 7
+// set when the forward kept the pre-activations a and b (moe_layer_forward_train).
+constexpr uint8_t kLayoutSavedAB = 0x80;
+constexpr uint8_t kLayoutSplitMask = 0x7F;
 // K ranges of the small-batch down projection: the largest split (at most
 // partial_cap and kDecodeSplitK) that leaves no K range of 64-wide blocks empty.
 inline int decode_ksplit(int h, int partial_cap) {
@@ -241,7 +248,7 @@ struct BwdArgs {
     const int32_t* offsets;    // [E + 1]
     const float* Y;            // expert outputs as one array [2T, d] ...
     const float* Ypart;        // ... or as split-K partials, split_stride floats apart
-    const uint8_t* y_layout;   // device byte: number of partials, or 1 for Y
+    const uint8_t* y_layout;   // device byte: number of partials (or 1 for Y), bit 7: a, b kept
     size_t split_stride;
     const void* x_perm;        // bf16 [2T, d]
     const void* H;             // bf16 [2T, h]
@@ -261,6 +268,10 @@ struct BwdArgs {
     // zero rows to a multiple of 64 (the weight-gradient GEMMs on CTA pairs)
     void* dY_pad;
     void* x_pad;
+    // fp32 [2T, h] each: the pre-activations a and b moe_layer_forward_train kept (the
+    // CTA-pair range); nullptr below that range
+    const float* a_pre;
+    const float* b_pre;
     uint32_t* status;
     // optional events recorded before the first launch and after each stage:
     // prep, dH, du/dv, dX, dx, dW2, dW1/dW3, dWg (null handles skipped)

@@ -227,3 +227,59 @@ def test_backward_other_expert_counts(T, E):
     for k in ("dx", "dW1", "dW3", "dW2"):
         assert errs[k] <= BWD_TOL, k
     assert errs["dWg"] <= ROUTER_TOL
+
+
+# ------------------------------------------------ pre-activations kept by the forward
+
+def _train_grads(inp, dy, ws, bws):
+    x = inp["x"]
+    y = torch.empty_like(x)
+    moe.moe_layer_forward_train(x, inp["Wg"], inp["W1"], inp["W3"], inp["W2"], y, ws, bws)
+    out = moe.layer_backward(x, inp["Wg"], inp["W1"], inp["W3"], inp["W2"], dy, ws, -1, bws)
+    return y, dict(zip(("dx", "dWg", "dW1", "dW3", "dW2"), out))
+
+
+@pytest.mark.parametrize("T,d,h,kind", [(512, 128, 256, "plain"), (700, 256, 384, "skew"),
+                                        (1100, 256, 384, "plain"), (2500, 128, 256, "long")])
+def test_forward_train_gives_the_same_layer_and_gradients(T, d, h, kind):
+    """moe_layer_forward_train keeps a = x W1^T and b = x W3^T (CTA-pair range, T >= 512)
+    and the backward then computes du, dv from them element by element instead of a
+    second GEMM1: the forward output and every gradient are bit-identical to the
+    recomputing path (the same accumulators, the same formula)."""
+    wl = small("ftr", T=T, d=d, h=h, seed=900 + T, kind=kind)
+    inp = make_inputs(wl, "cuda")
+    dy = seeded_dy(T, d, 77 + T)
+    ref, ws_ref = gpu_grads(inp, dy)
+    y_ref = torch.empty_like(inp["x"])
+    moe.moe_layer_forward(inp["x"], inp["Wg"], inp["W1"], inp["W3"], inp["W2"], y_ref, ws_ref)
+    ws = moe.alloc_workspace(T, d, h, wl.E, 2, torch.bfloat16, "cuda")
+    bws = moe.alloc_backward_workspace(T, d, h, wl.E, 2, torch.bfloat16, "cuda")
+    y, g = _train_grads(inp, dy, ws, bws)
+    assert torch.equal(y, y_ref)
+    for k in ref:
+        assert torch.equal(g[k], ref[k]), k
+    assert moe.moe_device_status(ws) == 0 and moe.moe_device_status(bws) == 0
+
+
+def test_plain_forward_after_a_training_forward_recomputes():
+    """A moe_layer_forward on the workspace after moe_layer_forward_train records that
+    nothing was kept, so the backward (same bwd_ws, whose a and b are now stale)
+    recomputes a and b; a later training forward keeps them again."""
+    wl = small("ftr2", T=600, d=128, h=256, seed=31)
+    inp1 = make_inputs(wl, "cuda")
+    inp2 = dict(inp1, x=make_inputs(small("ftr3", T=600, d=128, h=256, seed=32), "cuda")["x"])
+    dy = seeded_dy(600, 128, 5)
+    ref2, _ = gpu_grads(inp2, dy)
+    ref1, _ = gpu_grads(inp1, dy)
+    ws = moe.alloc_workspace(600, 128, 256, wl.E, 2, torch.bfloat16, "cuda")
+    bws = moe.alloc_backward_workspace(600, 128, 256, wl.E, 2, torch.bfloat16, "cuda")
+    _train_grads(inp1, dy, ws, bws)                 # keeps inp1's a, b in bws
+    y = torch.empty_like(inp2["x"])
+    moe.moe_layer_forward(inp2["x"], inp2["Wg"], inp2["W1"], inp2["W3"], inp2["W2"], y, ws)
+    out = moe.layer_backward(inp2["x"], inp2["Wg"], inp2["W1"], inp2["W3"], inp2["W2"], dy, ws,
+                             -1, bws)
+    for k, v in zip(("dx", "dWg", "dW1", "dW3", "dW2"), out):
+        assert torch.equal(v, ref2[k]), k
+    _, g = _train_grads(inp1, dy, ws, bws)
+    for k in ref1:
+        assert torch.equal(g[k], ref1[k]), k
