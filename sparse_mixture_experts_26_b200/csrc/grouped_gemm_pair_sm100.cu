@@ -112,8 +112,8 @@ struct PairArgs {
     int h;             // kBMnSplit: the K index where W3 takes over from W1
     const float* dH;   // kEpiBwdSwiGLU: dH fp32 [rows, N]
     int group;         // row blocks whose A rows stay in L2 together (tile order)
-    // kEpiSwiGLU, optional: the pre-activations a = x W1^T and b = x W3^T, fp32
-    // [rows, N] each, kept for the backward pass (nullptr: not written)
+    // kEpiSwiGLU with KEEP: the pre-activations a = x W1^T and b = x W3^T, fp32
+    // [rows, N] each, kept for the backward pass
     float* a_out;
     float* b_out;
     // optional: the launch does nothing when bit 7 of this device byte is set (the
@@ -207,7 +207,9 @@ __device__ __forceinline__ void store_pre_activations(const PairArgs& args, int 
     }
 }
 
-template <int EPI, int BOP = kBKMajor>
+// KEEP (kEpiSwiGLU only): also write the pre-activations a, b (moe_layer_forward_train);
+// a separate instance, so that the plain GEMM1 carries none of that code.
+template <int EPI, int BOP = kBKMajor, bool KEEP = false>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                              const __grid_constant__ CUtensorMap tmB0,
@@ -448,7 +450,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                     *reinterpret_cast<uint4*>(out + col) =
                                         make_uint4(p[4 * v], p[4 * v + 1], p[4 * v + 2], p[4 * v + 3]);
                             }
-                            if (args.a_out != nullptr)
+                            if (KEEP)
                                 store_pre_activations(args, row, col0 + ch * 32, a, b);
                         }
                     }
@@ -568,7 +570,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                     *reinterpret_cast<uint4*>(out + col) =
                                         make_uint4(p[4 * u], p[4 * u + 1], p[4 * u + 2], p[4 * u + 3]);
                             }
-                            if (args.a_out != nullptr)
+                            if (KEEP)
                                 store_pre_activations(args, row, col0 + ch * 32, a, b);
                         }
                     }
@@ -652,10 +654,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-template <int EPI, int BOP = kBKMajor>
+template <int EPI, int BOP = kBKMajor, bool KEEP = false>
 cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
                         const CUtensorMap& o, const PairArgs& args, int npairs, cudaStream_t s) {
-    auto kern = grouped_gemm_pair_kernel<EPI, BOP>;
+    auto kern = grouped_gemm_pair_kernel<EPI, BOP, KEEP>;
     constexpr int kSmemBytes = smem_bytes_of(EPI);
     // Row blocks per tile-order group: A rows of at most ~64 MB (a half of L2) per group.
     PairArgs a2 = args;
@@ -703,7 +705,9 @@ cudaError_t launch_ffn_bf16_pair(const void* x_perm, const int32_t* offsets, con
     g1.b_out = b_out;
     long long t1 = blocks * g1.n_tiles;
     const int grid1 = static_cast<int>(t1 < max_pairs ? (t1 < 1 ? 1 : t1) : max_pairs);
-    cudaError_t err = launch_pair<kEpiSwiGLU>(mx, mw1, mw3, mx, g1, grid1, s);
+    cudaError_t err = a_out != nullptr
+                          ? launch_pair<kEpiSwiGLU, kBKMajor, true>(mx, mw1, mw3, mx, g1, grid1, s)
+                          : launch_pair<kEpiSwiGLU>(mx, mw1, mw3, mx, g1, grid1, s);
     if (err != cudaSuccess) return err;
     if (between && (err = cudaEventRecord(between, s)) != cudaSuccess) return err;
     PairArgs g2{offsets, E, rows, h, d, d, (d + 255) / 256, Y, status, cap};
