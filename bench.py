@@ -640,9 +640,9 @@ def backward_kernel(wl, stage: int):
 
 
 def keeps_pre_activations(wl) -> bool:
-    """From 1024 grouped rows on, the training forward keeps a and b, and the
-    backward's du/dv step is element-wise instead of a second GEMM1."""
-    return wl.T * wl.k >= 1024
+    """The training forward keeps a and b at every batch size, and the backward's du/dv
+    step is element-wise instead of a second GEMM1."""
+    return wl.T > 0
 
 
 def backward_stage_flops(wl):
@@ -667,8 +667,8 @@ def wgrad_bytes(wl, stage: int) -> int:
 
 def measure_backward(wl, inp, K: int, W: int, world: int, local: int, device):
     """Time K backward calls (after one training forward that fills the saved state --
-    from 512 tokens on it keeps the pre-activations a, b, so the backward computes du,
-    dv element by element -- and W warm-up calls), with events between the backward's
+    it keeps the pre-activations a, b, so the backward computes du, dv element by
+    element -- and W warm-up calls), with events between the backward's
     stages inside the timed region, then K training and K plain forward calls (the
     training forward's cost), then the same backward steps end to end (dy in, dx out
     through pinned host buffers).  Returns the workload's result object."""

@@ -216,19 +216,27 @@ moe_status moe_selftest_wait_timeout(void *ws, size_t ws_bytes, double limit_sec
 
 /* Bytes of backward workspace moe_layer_backward needs for these sizes (0 for an
  * unsupported shape: the backward pass is built for bf16 layers with h % 64 == 0).
- * From T = 512 on (the CTA-pair range) it includes 2 * (2T) * h fp32 values for the
- * pre-activations moe_layer_forward_train keeps. */
+ * It includes 2 * (2T) * h fp32 values for the pre-activations moe_layer_forward_train
+ * keeps. */
 size_t moe_backward_workspace_bytes(int T, int d, int h, int E, int k, moe_dtype dt);
 
 /* moe_layer_forward for training: the same layer, the same y and forward workspace,
- * and in addition, from T = 512 on, the pre-activations a = x W1_e^T and b = x W3_e^T
- * of every grouped row kept in fp32 in bwd_ws (a GEMM1 epilogue writes them next to
- * H).  A moe_layer_backward call with the same fwd_ws and bwd_ws (and capacity < 0)
- * then computes du and dv from them element by element instead of recomputing a and b
- * with a second GEMM1 (same gradients: the same accumulators).  Any later forward call
- * on fwd_ws (moe_layer_forward, or this one below T = 512) records that nothing was
- * kept, and the backward recomputes.  Costs 4 * (2T) * h * 2 bytes of extra writes in
- * the forward.  dt must be MOE_BF16 and h % 64 == 0 (MOE_ERR_UNSUPPORTED otherwise);
+ * and in addition the pre-activations a = x W1_e^T and b = x W3_e^T of every grouped
+ * row kept in fp32 in bwd_ws (the GEMM1 epilogue writes them next to H).  A
+ * moe_layer_backward call with the same fwd_ws and bwd_ws (and capacity < 0) then
+ * computes du and dv from them element by element instead of recomputing a and b with
+ * a second GEMM1.  From T = 512 on the backward's recompute runs the same GEMM as the
+ * forward, so the gradients are bit-identical to the recomputing path by construction;
+ * below, a and b come from the forward's own kernels (weight streaming up to 128
+ * tokens, single-SM tiles above), which sum over d in the same 16-wide tensor-core
+ * steps and the same order as the backward's recompute (bit-identical gradients in
+ * every case measured on B200), though the two are separate kernels and only rounding
+ * (fp32 accumulation, then a bf16 store of du and dv) could tell them apart.  Any later
+ * forward call on fwd_ws
+ * (moe_layer_forward), and the two-launch small-batch form this call falls back to on
+ * a device that cannot co-schedule the fused launch, record that nothing was kept, and
+ * the backward recomputes.  Costs 4 * (2T) * h * 2 bytes of extra writes in the
+ * forward.  dt must be MOE_BF16 and h % 64 == 0 (MOE_ERR_UNSUPPORTED otherwise);
  * bwd_ws_bytes >= moe_backward_workspace_bytes (MOE_ERR_WORKSPACE otherwise). */
 moe_status moe_layer_forward_train(const void *x, const void *Wg, const void *W1,
                                    const void *W3, const void *W2, int T, int d, int h, int E,

@@ -54,13 +54,13 @@ def launches_per_layer(T: int, d: int = 4096, E: int = 8, bf16: bool = True) -> 
 def launches_per_backward(T: int, capacity: int = -1) -> int:
     """Kernels one moe_layer_backward queues: prep, dH, du/dv, dX, dx, the two
     weight-gradient GEMMs, the dWg partials and their sum (9), plus, without a
-    capacity, the element-wise du/dv kernel beside the recomputing one from 1024
-    grouped rows on (one of the two returns at once, by what the forward kept) and the
-    padded copies of dY and x_perm above 1024 grouped rows; none for T == 0."""
+    capacity, the element-wise du/dv kernel beside the recomputing one (one of the two
+    returns at once, by what the forward kept) and the padded copies of dY and x_perm
+    above 1024 grouped rows; none for T == 0."""
     if T <= 0:
         return 0
     free = capacity < 0
-    return 9 + (1 if 2 * T >= 1024 and free else 0) + (1 if 2 * T > 1024 and free else 0)
+    return 9 + (1 if free else 0) + (1 if 2 * T > 1024 and free else 0)
 
 
 class MoeError(RuntimeError):
@@ -284,7 +284,7 @@ def moe_layer_forward(x, Wg, W1, W3, W2, y, ws, k: int = 2, stream=None) -> None
 
 def moe_layer_forward_train(x, Wg, W1, W3, W2, y, ws, bwd_ws, k: int = 2, stream=None) -> None:
     """``moe_layer_forward`` that also keeps the pre-activations a, b (fp32) in
-    ``bwd_ws`` from 512 tokens on, for the ``moe_layer_backward`` call that follows."""
+    ``bwd_ws``, for the ``moe_layer_backward`` call that follows."""
     T, d, h, E = _layer_dims(x, Wg, W1, W3, W2)
     _expect("y", y, (T, d), x.dtype)
     _ws("ws", ws)

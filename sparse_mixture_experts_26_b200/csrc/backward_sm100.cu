@@ -145,6 +145,9 @@ struct RowArgs {
     const float* dH;   // kModeDUV: dH fp32 [rows, h]
     uint32_t* status;
     int cap;
+    // optional: the launch does nothing when bit 7 of this device byte is set (kModeDUV
+    // after a forward that kept the pre-activations)
+    const uint8_t* skip_flag;
 };
 
 template <int MODE>
@@ -162,6 +165,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     volatile int* abort_flag = &bk.abort_flag;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int E = args.E;
+    if (args.skip_flag != nullptr && (*args.skip_flag & kLayoutSavedAB) != 0) return;  // uniform
 
     if (threadIdx.x == 0) init_barriers(bk);
     if (warp == 0 && lane == 0) {
@@ -1078,20 +1082,22 @@ cudaError_t launch_layer_backward(const BwdArgs& a, cudaStream_t s) {
     // 3. du, dv: from the pre-activations the forward kept (moe_layer_forward_train), or
     // recomputing a and b; the forward's layout byte selects which of the two launches
     // does the work (the other returns at once), so the host never waits for it
+    if (a.a_pre != nullptr) {
+        const long long n4 = static_cast<long long>(P) * (h / 4);
+        err = launch_k(bwd_duv_saved_kernel,
+                       grid_for((n4 + kPrepThreads - 1) / kPrepThreads, 8 * sms), kPrepThreads, 0,
+                       s, a.y_layout, static_cast<const float*>(a.dH), a.a_pre, a.b_pre, P, h,
+                       static_cast<__nv_bfloat16*>(a.DUV));
+        if (err != cudaSuccess) return err;
+    }
+    const uint8_t* duv_skip = a.a_pre != nullptr ? a.y_layout : nullptr;
     if (pairs) {
-        if (a.a_pre != nullptr) {
-            const long long n4 = static_cast<long long>(P) * (h / 4);
-            err = launch_k(bwd_duv_saved_kernel,
-                           grid_for((n4 + kPrepThreads - 1) / kPrepThreads, 8 * sms), kPrepThreads,
-                           0, s, a.y_layout, static_cast<const float*>(a.dH), a.a_pre, a.b_pre, P,
-                           h, static_cast<__nv_bfloat16*>(a.DUV));
-            if (err != cudaSuccess) return err;
-        }
         err = launch_bwd_rows_pair(1, m_x, m_W1r, m_W3r, a.offsets, E, P, d, h, a.DUV, a.dH,
-                                   a.status, a.cap, s, a.a_pre != nullptr ? a.y_layout : nullptr);
+                                   a.status, a.cap, s, duv_skip);
         if (err != cudaSuccess || (err = mark(3)) != cudaSuccess) return err;
     } else {
-        RowArgs r{a.offsets, E, P, d, h, (h + 127) / 128, h, d, a.DUV, a.dH, a.status, a.cap};
+        RowArgs r{a.offsets, E, P, d, h, (h + 127) / 128, h, d, a.DUV, a.dH, a.status, a.cap,
+                  duv_skip};
         if ((err = configure(bwd_rows_kernel<kModeDUV>, kSlotDUV, kSmemBytes)) != cudaSuccess)
             return err;
         err = launch_k(bwd_rows_kernel<kModeDUV>, grid_for(row_blocks * r.n_tiles, sms),

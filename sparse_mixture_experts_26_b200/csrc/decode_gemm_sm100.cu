@@ -410,6 +410,10 @@ struct FusedArgs {
     uint32_t* readers;  // [E][ksplit]
     uint32_t* status;
     int cap;            // rows kept per group (capacity; INT_MAX = no limit)
+    // optional: the pre-activations a = x W1^T and b = x W3^T, fp32 [rows, h] each,
+    // kept for the backward pass (moe_layer_forward_train); nullptr: not written
+    float* a_out;
+    float* b_out;
 };
 
 template <int NACC>
@@ -723,8 +727,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 if (c < f.nvalid) {
                                     const float a = xfer[c * kM + r];
                                     const float b = xfer[c * kM + J1 + r];
-                                    out[static_cast<size_t>(f.row0 + c) * args.h + col] =
-                                        __float2bfloat16_rn(a * b * __frcp_rn(1.0f + __expf(-a)));
+                                    const size_t at = static_cast<size_t>(f.row0 + c) * args.h + col;
+                                    out[at] = __float2bfloat16_rn(a * b * __frcp_rn(1.0f + __expf(-a)));
+                                    if (args.a_out != nullptr) {
+                                        args.a_out[at] = a;
+                                        args.b_out[at] = b;
+                                    }
                                 }
                             }
                         }
@@ -768,8 +776,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                                     if (c0 + c < f.nvalid) {
                                         const float a = xfer[c * kM + r];
                                         const float b = xfer[c * kM + J1 + r];
-                                        out[static_cast<size_t>(f.row0 + c0 + c) * args.h + col] =
-                                            __float2bfloat16_rn(a * b * __frcp_rn(1.0f + __expf(-a)));
+                                        const size_t at =
+                                            static_cast<size_t>(f.row0 + c0 + c) * args.h + col;
+                                        out[at] = __float2bfloat16_rn(a * b * __frcp_rn(1.0f + __expf(-a)));
+                                        if (args.a_out != nullptr) {
+                                            args.a_out[at] = a;
+                                            args.b_out[at] = b;
+                                        }
                                     }
                                 }
                             }
@@ -823,7 +836,8 @@ template <int NT>
 cudaError_t launch_ffn_fused_nt(const void* x_perm, const int32_t* offsets, const void* W1,
                                 const void* W3, const void* W2, int rows, int d, int h, int E,
                                 void* H, float* Ypart, int ksplit, uint32_t* counters,
-                                uint32_t* status, cudaStream_t s, int cap) {
+                                uint32_t* status, cudaStream_t s, int cap, float* a_out,
+                                float* b_out) {
     CUtensorMap mw1, mw3, mw2;
     TokMaps mx, mh;
     if (!encode_bf16_2d(&mw1, W1, static_cast<uint64_t>(E) * h, d, kM / 2) ||
@@ -840,7 +854,7 @@ cudaError_t launch_ffn_fused_nt(const void* x_perm, const int32_t* offsets, cons
     if (const cudaError_t err = opt_in_smem(smem_once, kern, C::kSmem); err != cudaSuccess)
         return err;
     FusedArgs a{offsets, E, rows, d, h, (h + 63) / 64, (d + kM - 1) / kM, ksplit, H, Ypart,
-                counters, counters + E * ksplit, status, cap};
+                counters, counters + E * ksplit, status, cap, a_out, b_out};
     const int sms = device_sm_count();
     const long long chunks = static_cast<long long>(rows) / NT + E;
     const long long units = chunks * (a.n_hb + static_cast<long long>(a.n_db) * ksplit);
@@ -893,19 +907,19 @@ cudaError_t launch_ffn_bf16_decode_fused(const void* x_perm, const int32_t* offs
                                          const void* W1, const void* W3, const void* W2, int rows,
                                          int d, int h, int E, void* H, float* Ypart, int ksplit,
                                          uint32_t* counters, uint32_t* status, cudaStream_t s,
-                                         int cap) {
+                                         int cap, float* a_out, float* b_out) {
     const int T = rows / 2;
     if (T <= 16)
         return launch_ffn_fused_nt<16>(x_perm, offsets, W1, W3, W2, rows, d, h, E, H, Ypart,
-                                       ksplit, counters, status, s, cap);
+                                       ksplit, counters, status, s, cap, a_out, b_out);
     if (T <= 32)
         return launch_ffn_fused_nt<32>(x_perm, offsets, W1, W3, W2, rows, d, h, E, H, Ypart,
-                                       ksplit, counters, status, s, cap);
+                                       ksplit, counters, status, s, cap, a_out, b_out);
     if (T <= 64)
         return launch_ffn_fused_nt<64>(x_perm, offsets, W1, W3, W2, rows, d, h, E, H, Ypart,
-                                       ksplit, counters, status, s, cap);
+                                       ksplit, counters, status, s, cap, a_out, b_out);
     return launch_ffn_fused_nt<128>(x_perm, offsets, W1, W3, W2, rows, d, h, E, H, Ypart, ksplit,
-                                    counters, status, s, cap);
+                                    counters, status, s, cap, a_out, b_out);
 }
 
 cudaError_t launch_ffn_bf16_decode(const void* x_perm, const int32_t* offsets, const void* W1,

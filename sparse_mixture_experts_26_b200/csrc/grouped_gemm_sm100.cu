@@ -86,6 +86,8 @@ struct GemmArgs {
     void* out;          // H (bf16) or Y (fp32), row-major [rows, N]
     uint32_t* status;   // workspace status word
     int cap;            // rows kept per group (capacity; INT_MAX = no limit)
+    float* a_out;       // KEEP: a = x W1^T, fp32 [rows, N]
+    float* b_out;       // KEEP: b = x W3^T, fp32 [rows, N]
 };
 
 struct Bookkeeping {
@@ -119,13 +121,35 @@ __device__ __forceinline__ TileCoord decode_tile(const Bookkeeping& bk, int E, i
     return c;
 }
 
+// C pre-activations a and b of one row (fp32 bits), kept for the backward pass
+// (columns past N are not written; N is a multiple of 8 and C of 16).
+template <int C>
+__device__ __forceinline__ void keep_pre_activations(const GemmArgs& args, int row, int col0,
+                                                     const uint32_t (&a)[C],
+                                                     const uint32_t (&b)[C]) {
+    float* ar = args.a_out + static_cast<size_t>(row) * args.N;
+    float* br = args.b_out + static_cast<size_t>(row) * args.N;
+#pragma unroll
+    for (int j = 0; j < C / 4; ++j) {
+        const int col = col0 + 4 * j;
+        if (col < args.N) {
+            *reinterpret_cast<float4*>(ar + col) = make_float4(
+                bits_f32(a[4 * j]), bits_f32(a[4 * j + 1]), bits_f32(a[4 * j + 2]), bits_f32(a[4 * j + 3]));
+            *reinterpret_cast<float4*>(br + col) = make_float4(
+                bits_f32(b[4 * j]), bits_f32(b[4 * j + 1]), bits_f32(b[4 * j + 2]), bits_f32(b[4 * j + 3]));
+        }
+    }
+}
+
 // silu(a) * b = a b / (1 + e^-a), with a correctly rounded reciprocal (cheaper than a
 // division in the epilogue).
 __device__ __forceinline__ float silu_mul(float a, float b) {
     return a * b * __frcp_rn(1.0f + __expf(-a));
 }
 
-template <int EPI, int NO>
+// KEEP (kEpiSwiGLU only): also write the pre-activations a, b in fp32 (the training
+// forward); a separate instance, so that the plain GEMM1 carries none of that code.
+template <int EPI, int NO, bool KEEP = false>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB0,
@@ -315,6 +339,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int i = 0; i < 8; ++i)
                         p[i] = pack_bf16x2(silu_mul(bits_f32(a[2 * i]), bits_f32(b[2 * i])),
                                            silu_mul(bits_f32(a[2 * i + 1]), bits_f32(b[2 * i + 1])));
+                    if (KEEP && valid) keep_pre_activations<16>(args, row, col0 + ch * 16, a, b);
                     if (valid) {
 #pragma unroll
                         for (int v = 0; v < 2; ++v) {
@@ -340,6 +365,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int i = 0; i < 16; ++i)
                         p[i] = pack_bf16x2(silu_mul(bits_f32(a[2 * i]), bits_f32(b[2 * i])),
                                            silu_mul(bits_f32(a[2 * i + 1]), bits_f32(b[2 * i + 1])));
+                    if (KEEP && valid) keep_pre_activations<32>(args, row, col0 + ch * 32, a, b);
                     if (valid) {
 #pragma unroll
                         for (int v = 0; v < 4; ++v) {
@@ -385,10 +411,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-template <int EPI, int NO = 128>
+template <int EPI, int NO = 128, bool KEEP = false>
 cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
                         const GemmArgs& args, int grid, cudaStream_t s) {
-    auto kern = grouped_gemm_kernel<EPI, NO>;
+    auto kern = grouped_gemm_kernel<EPI, NO, KEEP>;
     constexpr int kSmemBytes = GemmShape<EPI, NO>::kSmemBytes;
     static PerDeviceOnce smem_once;
     if (const cudaError_t err = opt_in_smem(smem_once, kern, kSmemBytes); err != cudaSuccess)
@@ -468,7 +494,7 @@ cudaError_t launch_ffn_bf16(const void* x_perm, const int32_t* offsets, const vo
         err = cudaErrorNotSupported;
         if (can_fuse) {
             err = launch_ffn_bf16_decode_fused(x_perm, offsets, W1, W3, W2, rows, d, h, E, H, dst,
-                                               ksplit, counters, status, s, cap);
+                                               ksplit, counters, status, s, cap, a_save, b_save);
             if (err == cudaErrorCooperativeLaunchTooLarge || err == cudaErrorNotSupported)
                 cudaGetLastError();  // clear it: a path below needs no co-residency
             else if (err == cudaSuccess && between)
@@ -487,7 +513,11 @@ cudaError_t launch_ffn_bf16(const void* x_perm, const int32_t* offsets, const vo
                 ksplit = 1;
                 dst = Y;
             }
-            if (out) *out = FfnOut{dst, ksplit};
+            if (out) {
+                *out = FfnOut{dst, ksplit};
+                // only the fused launch keeps the pre-activations
+                out->saved_ab = can_fuse && !fallback && a_save != nullptr && b_save != nullptr;
+            }
             return cudaSuccess;
         }
         // 129..256 rows on a device that cannot co-schedule the fused launch: grouped GEMMs
@@ -516,8 +546,15 @@ cudaError_t launch_ffn_bf16(const void* x_perm, const int32_t* offsets, const vo
     GemmArgs g1{offsets, E, rows, d, h, h, (h + no - 1) / no, H, status, cap};
     long long tiles1 = row_blocks * g1.n_tiles;
     int grid1 = static_cast<int>(tiles1 < sms ? (tiles1 < 1 ? 1 : tiles1) : sms);
-    cudaError_t err = no == 112 ? launch_gemm<kEpiSwiGLU, 112>(mx, mw1, mw3, g1, grid1, s)
-                                : launch_gemm<kEpiSwiGLU, 128>(mx, mw1, mw3, g1, grid1, s);
+    const bool keep = a_save != nullptr && b_save != nullptr;
+    g1.a_out = a_save;
+    g1.b_out = b_save;
+    if (out) out->saved_ab = keep;
+    cudaError_t err =
+        keep ? (no == 112 ? launch_gemm<kEpiSwiGLU, 112, true>(mx, mw1, mw3, g1, grid1, s)
+                          : launch_gemm<kEpiSwiGLU, 128, true>(mx, mw1, mw3, g1, grid1, s))
+             : (no == 112 ? launch_gemm<kEpiSwiGLU, 112>(mx, mw1, mw3, g1, grid1, s)
+                          : launch_gemm<kEpiSwiGLU, 128>(mx, mw1, mw3, g1, grid1, s));
     if (err != cudaSuccess) return err;
     if (between && (err = cudaEventRecord(between, s)) != cudaSuccess) return err;
 

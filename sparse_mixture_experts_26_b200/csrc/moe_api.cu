@@ -122,9 +122,11 @@ struct BwdLayout {
     size_t status, dY, dw, dlogits, dH, DUV, dX, dwg_part, dY_pad, x_pad, a_pre, b_pre, total;
 };
 
-// Batches whose forward can keep the pre-activations for the backward pass (the
-// CTA-pair range of the expert FFN).
-bool keeps_pre_activations(int T) { return 2 * T >= kPairMinRows; }
+// Batches whose training forward can keep the pre-activations for the backward pass:
+// every size (the fused small-batch FFN, the grouped GEMM1 and the CTA-pair GEMM1 all
+// write them; the two-launch small-batch form, used only where the fused launch cannot
+// be co-scheduled, does not, and the backward then recomputes).
+bool keeps_pre_activations(int T) { return T > 0; }
 
 BwdLayout bwd_layout(int T, int d, int h, int E) {
     BwdLayout B{};

@@ -207,7 +207,7 @@ cudaError_t launch_ffn_bf16_decode_fused(const void* x_perm, const int32_t* offs
                                          const void* W1, const void* W3, const void* W2, int rows,
                                          int d, int h, int E, void* H, float* Ypart, int ksplit,
                                          uint32_t* counters, uint32_t* status, cudaStream_t s,
-                                         int cap);
+                                         int cap, float* a_out = nullptr, float* b_out = nullptr);
 // Small-batch expert FFN; the down projection writes `ksplit` partial arrays.
 cudaError_t launch_ffn_bf16_decode(const void* x_perm, const int32_t* offsets, const void* W1,
                                    const void* W3, const void* W2, int rows, int d, int h, int E,
