@@ -396,12 +396,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 // are grouped activations, row-major with m / n contiguous (MN-major).  Tiles are
 // (expert, 256-column block, 128-row block), row blocks inner so that consecutive
 // tiles share B.  An expert with no rows gets a zero tile.
-// The output is written by TMA, each epilogue warp on its own: a 32-column chunk of
-// the warp's 32 accumulator rows goes to one of its staging buffers in the
-// 128-byte-swizzled layout (row r at r * 128 bytes, 16-byte chunk j at position
-// j ^ (r % 8), so the warp's stores hit distinct banks), and lane 0 stores it with a
-// 3-D tensor store ([E, rows, cols]: rows past an expert's last are outside the
-// tensor and not written).  A buffer is reused once its previous store has read it;
+// The output is written by TMA (with an L2 evict-first hint), each epilogue warp on
+// its own: a 32-column chunk of the warp's 32 accumulator rows goes to one of its
+// staging buffers in the 128-byte-swizzled layout (row r at r * 128 bytes, 16-byte
+// chunk j at position j ^ (r % 8), so the warp's stores hit distinct banks), and lane
+// 0 stores it with a 3-D tensor store ([E, rows, cols]: rows past an expert's last
+// are outside the tensor and not written).  A buffer is reused once its previous store has read it;
 // no block-wide barrier is involved.  A tile that straddles the dW1 / dW3 boundary
 // (h not a multiple of 128) is stored row by row instead.
 // STAGES input stages and the staging buffers share the shared memory: a short
@@ -582,6 +582,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int q = warp & 3;
         const int r = q * 32 + lane;          // accumulator row of this thread
         uint8_t* wstage = sOut + q * OUTBUFS * kStageOutBytes;  // this warp's buffers
+        // The gradients are written once and not read again here: first out of L2, so
+        // that the stream of them does not evict the operand rows the next tiles reuse.
+        const uint64_t out_policy = l2_policy_evict_first();
         int acc = 0, buf = 0;
         uint32_t acc_phase = 0;
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
@@ -626,8 +629,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     fence_proxy_async_smem();
                     __syncwarp();
                     if (lane == 0) {
-                        tma_store_3d(second ? &tmO1 : &tmO0, st, col0 + ch * 32,
-                                     (second ? m0 - args.split : m0) + q * 32, e);
+                        tma_store_3d_hint(second ? &tmO1 : &tmO0, st, col0 + ch * 32,
+                                          (second ? m0 - args.split : m0) + q * 32, e,
+                                          out_policy);
                         bulk_commit_group();
                     }
                     if (++buf == OUTBUFS) buf = 0;
