@@ -237,7 +237,8 @@ size_t moe_backward_workspace_bytes(int T, int d, int h, int E, int k, moe_dtype
  * a device that cannot co-schedule the fused launch, record that nothing was kept, and
  * the backward recomputes.  Costs 4 * (2T) * h * 2 bytes of extra writes in the
  * forward.  dt must be MOE_BF16 and h % 64 == 0 (MOE_ERR_UNSUPPORTED otherwise);
- * bwd_ws_bytes >= moe_backward_workspace_bytes (MOE_ERR_WORKSPACE otherwise). */
+ * bwd_ws_bytes >= moe_backward_workspace_bytes (MOE_ERR_WORKSPACE otherwise).  T == 0
+ * queues nothing and returns MOE_OK. */
 moe_status moe_layer_forward_train(const void *x, const void *Wg, const void *W1,
                                    const void *W3, const void *W2, int T, int d, int h, int E,
                                    int k, moe_dtype dt, void *y, void *ws, size_t ws_bytes,

@@ -375,7 +375,8 @@ moe_status moe_layer_forward_train(const void* x, const void* Wg, const void* W1
     moe_status st = check_shape(T, d, h, E, k, dt, true);
     if (st != MOE_OK) return st;
     if (dt != MOE_BF16 || h % 64 != 0) return MOE_ERR_UNSUPPORTED;
-    if (T > 0 && !ptrs_ok({bwd_ws})) return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;  // empty batch: nothing to queue, as moe_layer_forward
+    if (!ptrs_ok({bwd_ws})) return MOE_ERR_INVALID_ARG;
     const BwdLayout B = bwd_layout(T, d, h, E);
     if (bwd_ws_bytes < B.total) return MOE_ERR_WORKSPACE;
     const bool keep = keeps_pre_activations(T);

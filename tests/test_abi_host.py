@@ -179,6 +179,31 @@ def test_backward_validation(lib):
                                        p, p, fw, p, bw, None, 3, None) == INVALID
 
 
+def test_forward_train_validation(lib):
+    """moe_layer_forward_train: the forward's checks, plus bf16 only, h % 64 == 0 and a
+    backward workspace large enough for the kept pre-activations (2 * 2T * h fp32)."""
+    L = _bind_backward(lib)
+    vp, i32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    L.moe_layer_forward_train.restype = i32
+    L.moe_layer_forward_train.argtypes = [vp] * 5 + [i32] * 6 + [vp, vp, sz, vp, sz, vp]
+    p = FAKE
+    T, d, h, E = 8, 64, 128, 8
+    fw = lib.moe_workspace_bytes(T, d, h, E, 2, BF16)
+    bw = L.moe_backward_workspace_bytes(T, d, h, E, 2, BF16)
+    assert bw >= 2 * (2 * T) * h * 4  # the kept a and b
+
+    def call(*, W2=p, h_=h, dt=BF16, fws=fw, bws=bw, bptr=p, T_=T, x=p):
+        return L.moe_layer_forward_train(x, p, p, p, W2, T_, d, h_, E, 2, dt, p, p, fws, bptr,
+                                         bws, None)
+    assert call(bws=bw - 1) == WORKSPACE
+    assert call(fws=fw - 1) == WORKSPACE
+    assert call(bptr=None) == INVALID
+    assert call(W2=None) == INVALID
+    assert call(h_=96) == UNSUPPORTED           # h % 64 != 0
+    assert call(dt=F32) == UNSUPPORTED
+    assert call(T_=0, x=None, bptr=None, bws=0, fws=0) == OK  # empty batch: nothing queued
+
+
 C_PROGRAM = r"""
 #include <stdio.h>
 #include "moe.h"
