@@ -768,23 +768,36 @@ def measure_backward(wl, inp, K: int, W: int, world: int, local: int, device):
                               for j in flops}}
 
     # The forward a training step pays: moe_layer_forward (nothing kept) and
-    # moe_layer_forward_train (a and b kept), K calls each, the training one last so
-    # that the end-to-end backward steps below read the state it keeps.
-    def time_forward(call):
+    # moe_layer_forward_train (a and b kept), K calls each, in four alternating blocks
+    # (the power limit slows whichever runs later), the training one last so that the
+    # end-to-end backward steps below read the state it keeps.
+    def time_block(call, n):
         f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        call()
         torch.cuda.synchronize()
         barrier(world, device)
         f0.record(stream)
-        for _ in range(K):
+        for _ in range(n):
             call()
         f1.record(stream)
         torch.cuda.synchronize()
         barrier(world, device)
-        return max_over_ranks(f0.elapsed_time(f1) / K, world, device)
-    fwd_ms = time_forward(lambda: moe.moe_layer_forward(x, Wg, W1, W3, W2, y, ws))
-    fwd_train_ms = time_forward(lambda: moe.moe_layer_forward_train(x, Wg, W1, W3, W2, y, ws,
-                                                                    bws))
+        return f0.elapsed_time(f1)
+    plain = lambda: moe.moe_layer_forward(x, Wg, W1, W3, W2, y, ws)  # noqa: E731
+    train = lambda: moe.moe_layer_forward_train(x, Wg, W1, W3, W2, y, ws, bws)  # noqa: E731
+    plain()
+    train()
+    blocks = [K // 4 + (1 if j < K % 4 else 0) for j in range(4)]
+    tot = {"plain": 0.0, "train": 0.0}
+    for j, n in enumerate(blocks):
+        if n == 0:
+            continue
+        order = (("plain", plain), ("train", train)) if j % 2 == 0 else \
+            (("train", train), ("plain", plain))
+        for name, call in order:
+            tot[name] += time_block(call, n)
+    train()
+    fwd_ms = max_over_ranks(tot["plain"] / K, world, device)
+    fwd_train_ms = max_over_ranks(tot["train"] / K, world, device)
     layer["forward_ms"] = round(fwd_ms, 4)
     layer["forward_train_ms"] = round(fwd_train_ms, 4)
     layer["train_step_ms"] = round(fwd_train_ms + ms, 4)
