@@ -761,6 +761,9 @@ def measure_backward(wl, inp, K: int, W: int, world: int, local: int, device):
                 "algorithmic_per_launch": per_launch, "launch_ms": round(st_ms[dom], 4)}
     if traffic_note:
         roofline["traffic_note"] = traffic_note
+    if bound == "tensor" and "bf16_tflops_sustained" in peaks:
+        # the backward runs for seconds under the power limit: the sustained figure
+        roofline["frac_of_sustained"] = round(ach / float(peaks["bf16_tflops_sustained"]), 4)
     total_flops = sum(flops.values())
     layer = {"ms": round(ms, 4), "tflops": round(total_flops / (ms * 1e-3) / 1e12, 1),
              "stage_ms": {n: round(v, 4) for n, v in zip(BWD_STAGES, st_ms)},
