@@ -204,6 +204,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             int stage = 0;
             uint32_t phase = 0, pending = 0, pending_phase = 0;
             bool ok = true;
+            const uint64_t w_policy = l2_policy_evict_first();
             for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
                 int e, row0, row_end, nt;
                 tile_of(tile, e, row0, row_end, nt);
@@ -232,9 +233,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                             map = second ? &tmB1 : &tmB0;
                             krow = e * args.h + (second ? kc - args.h : kc);
                         }
+                        // dH streams W2 once: first out of L2 (4-5% faster); dX keeps the
+                        // default policy (slower with the hint)
 #pragma unroll
-                        for (int i = 0; i < kN / 64; ++i)
-                            tma_load_2d(map, &bk.full[stage], b + i * kBox, nt * kN + 64 * i, krow);
+                        for (int i = 0; i < kN / 64; ++i) {
+                            if (MODE == kModeDH)
+                                tma_load_2d_hint(map, &bk.full[stage], b + i * kBox,
+                                                 nt * kN + 64 * i, krow, w_policy);
+                            else
+                                tma_load_2d(map, &bk.full[stage], b + i * kBox, nt * kN + 64 * i,
+                                            krow);
+                        }
                     }
                     pending |= 1u << stage;
                     pending_phase = (pending_phase & ~(1u << stage)) | (phase << stage);

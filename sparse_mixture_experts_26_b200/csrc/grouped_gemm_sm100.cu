@@ -226,6 +226,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t phase = 0;
             uint32_t pending = 0, pending_phase = 0;
             bool ok = true;
+            const uint64_t w_policy = l2_policy_evict_first();
             for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
                 const TileCoord c = decode_tile(bk, E, tile);
                 const int brow = c.e * args.b_rows + c.nt * (EPI == kEpiSwiGLU ? NO : 256);
@@ -241,8 +242,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     uint8_t* b_dst = sB + stage * kBBytes;
                     tma_load_2d(&tmA, &bk.full[stage], a_dst, kc, c.row0);
                     if (EPI == kEpiSwiGLU) {  // NO-row boxes: W1 rows, then W3 rows
-                        tma_load_2d(&tmB0, &bk.full[stage], b_dst, kc, brow);
-                        tma_load_2d(&tmB1, &bk.full[stage], b_dst + kBBytes / 2, kc, brow);
+                        // weights first out of L2 (the gathered rows are the reused
+                        // operand): GEMM1 1.5-2% faster at 192-256 tokens, GEMM2 not
+                        tma_load_2d_hint(&tmB0, &bk.full[stage], b_dst, kc, brow, w_policy);
+                        tma_load_2d_hint(&tmB1, &bk.full[stage], b_dst + kBBytes / 2, kc, brow,
+                                         w_policy);
                     } else {
                         tma_load_2d(&tmB0, &bk.full[stage], b_dst, kc, brow);
                         tma_load_2d(&tmB0, &bk.full[stage], b_dst + kBBytes / 2, kc, brow + 128);
