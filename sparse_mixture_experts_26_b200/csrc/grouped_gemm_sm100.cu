@@ -101,6 +101,8 @@ struct Bookkeeping {
     int off[kMaxExperts + 1];        // sanitised group offsets
     int end[kMaxExperts];            // end of the rows kept in group g (capacity)
     int tile_start[kMaxExperts + 1]; // prefix sum of tiles per group
+    int tile_n;                      // output columns per tile (GEMM2: chosen per launch)
+    int n_tiles;                     // column tiles per row block
 };
 static_assert(sizeof(Bookkeeping) <= 1024, "bookkeeping must fit its reserve");
 
@@ -147,13 +149,41 @@ __device__ __forceinline__ float silu_mul(float a, float b) {
     return a * b * __frcp_rn(1.0f + __expf(-a));
 }
 
+// GEMM2's weight rows past the first 128 of a tile narrower than 256 columns: tensor
+// maps with 32-, 64- and 96-row boxes (unused by GEMM1).
+struct W2Tails {
+    CUtensorMap box[3];
+};
+
+// GEMM2 tile width for `row_blocks` row blocks on `grid` CTAs: each CTA streams its
+// tiles' A rows and weight rows from L2, so the time goes as the rounds of tiles a CTA
+// runs times the rows one tile streams (128 + width); the narrowest tiles refill the
+// rounds that 256-column tiles would leave half empty (e.g. 13 row blocks: 208 tiles
+// of 256 columns, two rounds of 148 with 60 CTAs in the second, against 286 tiles of
+// 192 columns in two full rounds).
+__host__ __device__ inline int gemm2_tile_width(int row_blocks, int N, int grid) {
+    int best = 256, best_cost = 0x7fffffff;
+#pragma unroll
+    for (int i = 0; i < 5; ++i) {
+        const int w = 256 - 32 * i;  // constant after unrolling: no runtime division by w
+        const int tiles = row_blocks * ((N + w - 1) / w);
+        const int cost = (tiles + grid - 1) / grid * (128 + w);
+        if (cost < best_cost) {
+            best_cost = cost;
+            best = w;
+        }
+    }
+    return best;
+}
+
 // KEEP (kEpiSwiGLU only): also write the pre-activations a, b in fp32 (the training
 // forward); a separate instance, so that the plain GEMM1 carries none of that code.
 template <int EPI, int NO, bool KEEP = false>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB0,
-                        const __grid_constant__ CUtensorMap tmB1, const GemmArgs args) {
+                        const __grid_constant__ CUtensorMap tmB1,
+                        const __grid_constant__ W2Tails tails, const GemmArgs args) {
     using S = GemmShape<EPI, NO>;
     constexpr int kStages = S::kStages;
     constexpr int kBBytes = S::kBBytes;
@@ -203,13 +233,24 @@ __global__ void __launch_bounds__(kThreads, 1)
             bk.off[g] = v;
             prev = v;
         }
-        bk.tile_start[0] = 0;
+        int row_blocks = 0;
         for (int g = 0; g < E; ++g) {
             const int n = bk.off[g + 1] - bk.off[g];
             bk.end[g] = bk.off[g] + (n < args.cap ? n : args.cap);
-            bk.tile_start[g + 1] =
-                bk.tile_start[g] + (bk.end[g] - bk.off[g] + kBM - 1) / kBM * args.n_tiles;
+            row_blocks += (bk.end[g] - bk.off[g] + kBM - 1) / kBM;
         }
+        if (EPI == kEpiSwiGLU) {
+            bk.tile_n = NO;
+            bk.n_tiles = args.n_tiles;
+        } else {
+            const int w = gemm2_tile_width(row_blocks, args.N, static_cast<int>(gridDim.x));
+            bk.tile_n = w;
+            bk.n_tiles = (args.N + w - 1) / w;
+        }
+        bk.tile_start[0] = 0;
+        for (int g = 0; g < E; ++g)
+            bk.tile_start[g + 1] =
+                bk.tile_start[g] + (bk.end[g] - bk.off[g] + kBM - 1) / kBM * bk.n_tiles;
     }
     tc_fence_before();
     __syncthreads();
@@ -217,6 +258,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const uint32_t tmem_base = bk.tmem_base;
     const int total_tiles = bk.tile_start[E];
+    const int tile_n = bk.tile_n;
     const int num_kb = (args.K + kBK - 1) / kBK;
 
     if (warp == 0) {
@@ -229,14 +271,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t w_policy = l2_policy_evict_first();
             for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
                 const TileCoord c = decode_tile(bk, E, tile);
-                const int brow = c.e * args.b_rows + c.nt * (EPI == kEpiSwiGLU ? NO : 256);
+                const int brow = c.e * args.b_rows + c.nt * tile_n;
+                // GEMM2: 128 weight rows from the 128-row map, the rest of a narrower
+                // tile from the map whose box is that many rows
+                const CUtensorMap* tail = tile_n == 256 ? &tmB0
+                                          : tile_n > 128 ? &tails.box[(tile_n - 128) / 32 - 1]
+                                                         : nullptr;
+                const uint32_t tx_bytes =
+                    EPI == kEpiSwiGLU ? kStageBytes : kABytes + tile_n * kBK * 2;
                 for (int kb = 0; kb < num_kb; ++kb) {
                     if (!mbar_wait_bounded(&bk.empty[stage], phase ^ 1u, abort_flag,
                                            args.status)) {
                         ok = false;
                         break;
                     }
-                    mbar_arrive_expect_tx(&bk.full[stage], kStageBytes);
+                    mbar_arrive_expect_tx(&bk.full[stage], tx_bytes);
                     const int kc = kb * kBK;
                     uint8_t* a_dst = sA + stage * kABytes;
                     uint8_t* b_dst = sB + stage * kBBytes;
@@ -249,7 +298,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                          w_policy);
                     } else {
                         tma_load_2d(&tmB0, &bk.full[stage], b_dst, kc, brow);
-                        tma_load_2d(&tmB0, &bk.full[stage], b_dst + kBBytes / 2, kc, brow + 128);
+                        if (tail != nullptr)
+                            tma_load_2d(tail, &bk.full[stage], b_dst + kBBytes / 2, kc, brow + 128);
                     }
                     pending |= 1u << stage;
                     pending_phase = (pending_phase & ~(1u << stage)) | (phase << stage);
@@ -274,6 +324,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             int acc = 0;
             uint32_t acc_phase = 0;
             bool ok = true, issued = false;
+            const uint32_t idesc = EPI == kEpiSwiGLU ? S::kIdesc : idesc_bf16_f32(kBM, tile_n);
             for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
                 if (!mbar_wait_bounded(&bk.tmem_empty[acc], acc_phase ^ 1u, abort_flag,
                                        args.status)) {
@@ -292,7 +343,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint64_t bd = sw128_kmajor_desc(smem_u32(sB + stage * kBBytes));
 #pragma unroll
                     for (int k = 0; k < kBK / 16; ++k)
-                        umma_bf16(d_tmem, ad + 2 * k, bd + 2 * k, S::kIdesc, (kb | k) != 0);
+                        umma_bf16(d_tmem, ad + 2 * k, bd + 2 * k, idesc, (kb | k) != 0);
                     umma_commit(&bk.empty[stage]);
                     issued = true;
                     if (++stage == kStages) {
@@ -382,9 +433,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             } else {
                 float* out = static_cast<float*>(args.out) + static_cast<size_t>(row) * args.N;
-                const int col0 = c.nt * 256;
+                const int col0 = c.nt * tile_n;
 #pragma unroll 1
-                for (int ch = 0; ch < 8; ++ch) {
+                for (int ch = 0; ch < tile_n / 32; ++ch) {
                     uint32_t v[32];
                     tmem_ld_32cols(tbase + ch * 32, v);
                     tmem_ld_wait();
@@ -417,13 +468,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <int EPI, int NO = 128, bool KEEP = false>
 cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
-                        const GemmArgs& args, int grid, cudaStream_t s) {
+                        const W2Tails& tails, const GemmArgs& args, int grid, cudaStream_t s) {
     auto kern = grouped_gemm_kernel<EPI, NO, KEEP>;
     constexpr int kSmemBytes = GemmShape<EPI, NO>::kSmemBytes;
     static PerDeviceOnce smem_once;
     if (const cudaError_t err = opt_in_smem(smem_once, kern, kSmemBytes); err != cudaSuccess)
         return err;
-    return launch_k(kern, grid, kThreads, kSmemBytes, s, a, b0, b1, args);
+    return launch_k(kern, grid, kThreads, kSmemBytes, s, a, b0, b1, tails, args);
 }
 
 }  // namespace
@@ -542,6 +593,10 @@ cudaError_t launch_ffn_bf16(const void* x_perm, const int32_t* offsets, const vo
         !encode_bf16_2d(&mh, H, rows, h, kBM) ||
         !encode_bf16_2d(&mw2, W2, static_cast<uint64_t>(E) * d, h, 128))
         return cudaErrorInvalidValue;
+    W2Tails tails;
+    for (int i = 0; i < 3; ++i)
+        if (!encode_bf16_2d(&tails.box[i], W2, static_cast<uint64_t>(E) * d, h, 32 * (i + 1)))
+            return cudaErrorInvalidValue;
 
     const int sms = device_sm_count();
     // Upper bound on row blocks: sum_e ceil(n_e / 128) <= (rows + 127 E) / 128.
@@ -555,17 +610,19 @@ cudaError_t launch_ffn_bf16(const void* x_perm, const int32_t* offsets, const vo
     g1.b_out = b_save;
     if (out) out->saved_ab = keep;
     cudaError_t err =
-        keep ? (no == 112 ? launch_gemm<kEpiSwiGLU, 112, true>(mx, mw1, mw3, g1, grid1, s)
-                          : launch_gemm<kEpiSwiGLU, 128, true>(mx, mw1, mw3, g1, grid1, s))
-             : (no == 112 ? launch_gemm<kEpiSwiGLU, 112>(mx, mw1, mw3, g1, grid1, s)
-                          : launch_gemm<kEpiSwiGLU, 128>(mx, mw1, mw3, g1, grid1, s));
+        keep ? (no == 112 ? launch_gemm<kEpiSwiGLU, 112, true>(mx, mw1, mw3, tails, g1, grid1, s)
+                          : launch_gemm<kEpiSwiGLU, 128, true>(mx, mw1, mw3, tails, g1, grid1, s))
+             : (no == 112 ? launch_gemm<kEpiSwiGLU, 112>(mx, mw1, mw3, tails, g1, grid1, s)
+                          : launch_gemm<kEpiSwiGLU, 128>(mx, mw1, mw3, tails, g1, grid1, s));
     if (err != cudaSuccess) return err;
     if (between && (err = cudaEventRecord(between, s)) != cudaSuccess) return err;
 
-    GemmArgs g2{offsets, E, rows, h, d, d, (d + 255) / 256, Y, status, cap};
+    // GEMM2's tile width is chosen on the device from the row blocks (up to 32 tiles of
+    // 128 columns per row block), so the grid covers the narrowest tiling
+    GemmArgs g2{offsets, E, rows, h, d, d, (d + 127) / 128, Y, status, cap};
     long long tiles2 = row_blocks * g2.n_tiles;
     int grid2 = static_cast<int>(tiles2 < sms ? (tiles2 < 1 ? 1 : tiles2) : sms);
-    return launch_gemm<kEpiStoreF32>(mh, mw2, mw2, g2, grid2, s);
+    return launch_gemm<kEpiStoreF32>(mh, mw2, mw2, tails, g2, grid2, s);
 }
 
 }  // namespace moe
