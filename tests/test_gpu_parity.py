@@ -110,8 +110,7 @@ SMALL = [  # (T, d, h, kind): ragged row blocks, K tails, N tails, empty groups
     # 112 selects its 112-output GEMM1 tiles
     (129, 256, 512, "plain"), (300, 136, 200, "plain"), (511, 128, 256, "skew"),
     (200, 128, 224, "plain"), (300, 256, 448, "skew"), (450, 136, 336, "long"),
-    # ... with stream-K work split (>= one (tile, K block) unit per SM): tiles cut
-    # between CTAs and finished from fp32 partials; ragged K (1000 = 15 x 64 + 40)
+    # ... at larger d and h: many K blocks per tile, ragged K (1000 = 15 x 64 + 40)
     (300, 1000, 1792, "plain"), (400, 1024, 2048, "skew"), (160, 512, 3584, "long"),
     # >= 1024 grouped rows run the CTA-pair grouped GEMM (256-row blocks; an expert's
     # last block of <= 128 rows runs in the pair's 128-row mode)
@@ -140,6 +139,52 @@ def test_layer_bf16_small_shapes(T, d, h, kind):
     # the fused entry point runs the same kernels (above 512 tokens the router also
     # counts the grouping, so the count pass is skipped): identical bits
     assert torch.equal(layer_y(inp), g["y"])
+
+
+def gemm2_width(row_blocks, d, grid=148):
+    """The single-SM GEMM2 tile width the kernel picks: the width w of 256, 224, 192, 160
+    or 128 columns that minimises rounds(row_blocks * ceil(d / w) tiles) * (128 + w)."""
+    best, best_cost = 256, None
+    for w in (256, 224, 192, 160, 128):
+        cost = -(-row_blocks * -(-d // w) // grid) * (128 + w)
+        if best_cost is None or cost < best_cost:
+            best, best_cost = w, cost
+    return best
+
+
+@pytest.mark.parametrize("sizes,width", [
+    ([100] * 8, 256),                                   # 8 row blocks: one round
+    ([200, 200, 60, 60, 60, 60, 60, 60], 160),          # 10 row blocks
+    ([200, 200, 200, 200, 50, 50, 50, 50], 192),        # 12
+    ([129] * 6 + [100, 100], 224),                      # 14, single-row second blocks
+    ([300, 0, 0, 250, 130, 100, 100, 100], 160),        # empty groups, 10 row blocks
+])
+def test_grouped_ffn_every_gemm2_tile_width(sizes, width):
+    """The grouped expert FFN (257..1023 rows) on crafted group sizes whose row-block
+    counts make the kernel's GEMM2 take each of its tile widths (ragged last column
+    tile: d = 4096 is no multiple of 160, 192 or 224), against the fp64 oracle."""
+    d, h, E = 4096, 256, 8
+    blocks = sum(-(-n // 128) for n in sizes)
+    assert gemm2_width(blocks, d) == width
+    wl = small("g2w", T=16, d=d, h=h, seed=70 + blocks)
+    inp = make_inputs(wl, "cuda")
+    P = sum(sizes)
+    g = torch.Generator(device="cpu")
+    g.manual_seed(1000 + blocks)
+    xp = torch.randn(P, d, generator=g).to(torch.bfloat16).cuda()
+    off = torch.tensor(np.concatenate([[0], np.cumsum(sizes)]), dtype=torch.int32,
+                       device="cuda")
+    ws = moe.alloc_workspace(P // 2, d, h, E, 2, torch.bfloat16, "cuda")
+    Y = torch.full((P, d), float("nan"), dtype=torch.float32, device="cuda")
+    moe.moe_expert_ffn(xp, off, inp["W1"], inp["W3"], inp["W2"], Y, ws)
+    assert moe.moe_device_status(ws) == 0
+    ref = O.expert_ffn_grouped(xp.float().cpu().numpy(), off.cpu().numpy(),
+                               PerExpert(inp["W1"]), PerExpert(inp["W3"]), PerExpert(inp["W2"]))
+    got = Y.double().cpu().numpy()
+    assert np.isfinite(got).all()
+    err = float(np.linalg.norm(got - ref) / np.linalg.norm(ref))
+    print(f"GEMM2_WIDTH {width} blocks={blocks} rel_fro={err:.3e}")
+    assert err <= 5e-3
 
 
 def test_router_counts_are_cleared_between_calls():
@@ -241,7 +286,8 @@ def test_exact_invariants_on_gpu(T):
 
 @pytest.mark.parametrize("name,T", [("decode", None), ("prefill", None), ("skew", None),
                                     ("long", None),
-                                    # batches between the two: stream-K grouped GEMMs
+                                    # batches between the two: single-SM grouped GEMMs
+                                    # (511 tokens: 13 row blocks, 192-column GEMM2 tiles)
                                     ("prefill", 192), ("prefill", 511), ("skew", 256),
                                     ("skew", 384)])
 def test_full_size_workloads(name, T):
