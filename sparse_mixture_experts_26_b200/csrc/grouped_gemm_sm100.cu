@@ -14,10 +14,10 @@
 //   A = grouped activations [rows, K], B = the expert's weight rows [N, K].
 //
 // Design (one CTA per SM, persistent, 6 warps):
-//   warp 0      TMA producer: 128x64 A tile + (2 NO)x64 or 256x64 B tile per stage,
-//               a ring of shared-memory stages guarded by mbarriers.
+//   warp 0      TMA producer: 128x64 A tile + (2 NO)x64 or (GEMM2) Wx64 B tile per
+//               stage, a ring of shared-memory stages guarded by mbarriers.
 //   warp 1      allocates 512 TMEM columns; one thread issues tcgen05.mma
-//               (M=128, N=2 NO or 256, K=16; four per 64-wide K block) into one of
+//               (M=128, N=2 NO or W, K=16; four per 64-wide K block) into one of
 //               two fp32 accumulators 256 columns apart, and commits stage/accumulator
 //               barriers.
 //   warps 2-5   epilogue: tcgen05.ld the accumulator (one row per thread), apply
@@ -29,7 +29,9 @@
 // 128-row blocks per expert, and with Mixtral's h = 14336 the 112 columns give
 // 8 x 128 = 1024 tiles (6.9 rounds of 148 SMs, the last one full) instead of
 // 8 x 112 = 896 (6.05 rounds, the 7th nearly empty); the smaller stage (44 KiB) also
-// lets 5 stages fit instead of 4.
+// lets 5 stages fit instead of 4.  GEMM2's tile width W (256 down to 128 columns) is
+// chosen on the device from the number of row blocks, so that the tiles fill whole
+// rounds of the grid (gemm2_tile_width below).
 //
 // Tiles never mix experts' weights: a tile is (expert, 128-row block of that
 // expert's rows, output-column block).  A row block may run past the expert's last
@@ -60,7 +62,8 @@ constexpr uint32_t kTmemCols = 2 * kMmaN;   // two accumulators: all 512 columns
 enum Epilogue { kEpiSwiGLU = 0, kEpiStoreF32 = 1 };
 
 // Shape of one instantiation: GEMM1 tiles cover NO outputs (B = NO W1 rows + NO W3
-// rows), GEMM2 tiles 256 output columns.  Stages fill the shared memory.
+// rows), GEMM2 tiles up to 256 output columns (the stage holds 256 weight rows).
+// Stages fill the shared memory.
 template <int EPI, int NO>
 struct GemmShape {
     static constexpr int kBRows = EPI == kEpiSwiGLU ? 2 * NO : 256;
