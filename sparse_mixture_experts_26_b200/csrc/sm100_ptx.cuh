@@ -221,12 +221,6 @@ __device__ __forceinline__ uint64_t l2_policy_evict_first() {
     return p;
 }
 
-__device__ __forceinline__ uint64_t l2_policy_evict_last() {
-    uint64_t p;
-    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
-    return p;
-}
-
 // ------------------------------------------------------------------ TMEM / tcgen05
 // Allocate `ncols` tensor-memory columns (power of two >= 32); the base address is
 // written to shared memory at `slot`.  Executed by one whole warp.
