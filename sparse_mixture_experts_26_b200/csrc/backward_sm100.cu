@@ -410,8 +410,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 // staging buffers in the 128-byte-swizzled layout (row r at r * 128 bytes, 16-byte
 // chunk j at position j ^ (r % 8), so the warp's stores hit distinct banks), and lane
 // 0 stores it with a 3-D tensor store ([E, rows, cols]: rows past an expert's last
-// are outside the tensor and not written).  A buffer is reused once its previous store has read it;
-// no block-wide barrier is involved.  A tile that straddles the dW1 / dW3 boundary
+// are outside the tensor and not written).  A buffer is reused once its previous
+// store has read it; no block-wide barrier is involved.  A tile that straddles the dW1 / dW3 boundary
 // (h not a multiple of 128) is stored row by row instead.
 // STAGES input stages and the staging buffers share the shared memory: a short
 // reduction (few rows per expert) leaves the kernel bound by its output stores (more
